@@ -1,0 +1,273 @@
+"""CPU oracle for the CSA / HCA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never calls it and
+shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, single-threaded, double
+accumulation); this module compiles it with gcc on first use and marshals
+numpy arrays through ctypes, looping over the batch dimension.  Sources are
+cited in ``oracle.c``:
+
+  [HA] "DeepSeek-V4 混合注意力：从压缩记忆到百万上下文": §4.1 compressor, §4.2 indexer,
+       §5 HCA compressor and dense attention, §6 SWA and attention sink,
+       §7 call chain.
+  [P1] "揭秘DeepSeek-V4-Pro-MXFP4稀疏注意力：哈希索引与DSA如何撑起1M超长上下文？"
+  [P2] "解密DeepSeek-V4-Flash-NVFP4的混合注意力机制：压缩稀疏注意力如何提升长文本处理能力"
+
+Parity status: every function here is pinned by a ``-m "not gpu"`` test
+(tests/test_oracle_pins.py) except the FP8 *recall* statistic, which the pages
+do not fix ("parity unpinned" for recall only; the e4m3 codec and the FP8
+score definition are pinned).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+_vp = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+    lib.oracle_compress_csa.argtypes = [_f32p, _f32p, _f32p, _f32p, _vp, _vp, i64, i32, i32, _f64p, _f64p]
+    lib.oracle_compress_hca.argtypes = [_f32p, _f32p, i64, i32, i32, _f64p, _f64p]
+    lib.oracle_n_visible.argtypes = [i64, i32, i64]
+    lib.oracle_n_visible.restype = i64
+    lib.oracle_index_scores.argtypes = [_f32p, _f32p, _f32p, _i32p, i32, i64, i32, i32, _f64p, _f64p]
+    lib.oracle_index_scores_e4m3.argtypes = [_u8p, _f32p, _f32p, _u8p, _f32p, _i32p, i32, i64, i32, i32,
+                                             _f64p, _f64p]
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = dbl
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_quantize_rows_e4m3.argtypes = [_f32p, i64, i32, _u8p, _f32p]
+    lib.oracle_topk.argtypes = [_f32p, _i32p, i32, i64, i32, _i32p]
+    lib.oracle_sparse_attn.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _f32p, _i32p, i32, dbl, i32,
+                                       i32, i32, i32, i64, _f64p, _f64p]
+    lib.oracle_hca_attn.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _f32p, i32, dbl, i32,
+                                    i32, i32, i32, i64, _f64p, _f64p]
+    for name in ("oracle_compress_csa", "oracle_compress_hca", "oracle_index_scores",
+                 "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_topk",
+                 "oracle_sparse_attn", "oracle_hca_attn"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _f32(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle: {what} rejected its arguments")
+
+
+# --------------------------------------------------------------------------- compressor
+def compress_csa(Ca, Cb, Za, Zb, prev_Cb=None, prev_Zb=None, m: int = 4, with_mag: bool = False):
+    """[HA] §4.1 overlapped 2m-position softmax pooling.  Inputs [B, L, c] (or [L, c]);
+    optional carry prev_* [B, m, c].  Returns [B, L//m, c] float64 (and the magnitude)."""
+    lib = _load()
+    Ca, Cb, Za, Zb = (_f32(x) for x in (Ca, Cb, Za, Zb))
+    squeeze = Ca.ndim == 2
+    if squeeze:
+        Ca, Cb, Za, Zb = (x[None] for x in (Ca, Cb, Za, Zb))
+        prev_Cb = None if prev_Cb is None else _f32(prev_Cb)[None]
+        prev_Zb = None if prev_Zb is None else _f32(prev_Zb)[None]
+    B, L, c = Ca.shape
+    out = np.empty((B, L // m, c), np.float64)
+    mag = np.empty_like(out)
+    for b in range(B):
+        pc = None if prev_Cb is None else np.ascontiguousarray(_f32(prev_Cb)[b])
+        pz = None if prev_Zb is None else np.ascontiguousarray(_f32(prev_Zb)[b])
+        ob, mb = np.empty((L // m, c), np.float64), np.empty((L // m, c), np.float64)
+        rc = lib.oracle_compress_csa(np.ascontiguousarray(Ca[b]), np.ascontiguousarray(Cb[b]),
+                                     np.ascontiguousarray(Za[b]), np.ascontiguousarray(Zb[b]),
+                                     None if pc is None else pc.ctypes.data,
+                                     None if pz is None else pz.ctypes.data,
+                                     L, c, m, ob, mb)
+        _check(rc, "compress_csa")
+        out[b], mag[b] = ob, mb
+    if squeeze:
+        out, mag = out[0], mag[0]
+    return (out, mag) if with_mag else out
+
+
+def compress_hca(C, Z, m: int = 128, with_mag: bool = False):
+    """[HA] §5 non-overlapped m-position softmax pooling.  [B, L, c] -> [B, L//m, c]."""
+    lib = _load()
+    C, Z = _f32(C), _f32(Z)
+    squeeze = C.ndim == 2
+    if squeeze:
+        C, Z = C[None], Z[None]
+    B, L, c = C.shape
+    out = np.empty((B, L // m, c), np.float64)
+    mag = np.empty_like(out)
+    for b in range(B):
+        ob, mb = np.empty((L // m, c), np.float64), np.empty((L // m, c), np.float64)
+        _check(lib.oracle_compress_hca(np.ascontiguousarray(C[b]), np.ascontiguousarray(Z[b]),
+                                       L, c, m, ob, mb), "compress_hca")
+        out[b], mag[b] = ob, mb
+    if squeeze:
+        out, mag = out[0], mag[0]
+    return (out, mag) if with_mag else out
+
+
+def n_visible(q_pos, m: int, N: int):
+    """Number of complete compressed entries visible at each absolute position."""
+    lib = _load()
+    q = np.asarray(q_pos, np.int64)
+    flat = [lib.oracle_n_visible(int(t), m, N) for t in q.reshape(-1)]
+    return np.asarray(flat, np.int32).reshape(q.shape)
+
+
+# --------------------------------------------------------------------------- indexer
+def index_scores(qI, w, kI, n_valid, with_mag: bool = False):
+    """[HA] §4.2.  qI [B,T,Hi,d], w [B,T,Hi], kI [B,N,d], n_valid [B,T] -> [B,T,N] float64."""
+    lib = _load()
+    qI, w, kI = _f32(qI), _f32(w), _f32(kI)
+    nv = np.ascontiguousarray(np.asarray(n_valid, np.int32))
+    B, T, Hi, d = qI.shape
+    N = kI.shape[1]
+    out = np.empty((B, T, N), np.float64)
+    mag = np.empty_like(out)
+    for b in range(B):
+        ob, mb = np.empty((T, N), np.float64), np.empty((T, N), np.float64)
+        _check(lib.oracle_index_scores(np.ascontiguousarray(qI[b]), np.ascontiguousarray(w[b]),
+                                       np.ascontiguousarray(kI[b]), np.ascontiguousarray(nv[b]),
+                                       T, N, Hi, d, ob, mb), "index_scores")
+        out[b], mag[b] = ob, mb
+    return (out, mag) if with_mag else out
+
+
+def index_scores_e4m3(q8, q_scale, w, k8, k_scale, n_valid, with_mag: bool = False):
+    """[HA] §4.2 on dequantised e4m3 codes.  q8 [B,T,Hi,d] u8, q_scale [B,T,Hi],
+    k8 [B,N,d] u8, k_scale [B,N] -> [B,T,N] float64."""
+    lib = _load()
+    q8 = np.ascontiguousarray(np.asarray(q8, np.uint8))
+    k8 = np.ascontiguousarray(np.asarray(k8, np.uint8))
+    q_scale, w, k_scale = _f32(q_scale), _f32(w), _f32(k_scale)
+    nv = np.ascontiguousarray(np.asarray(n_valid, np.int32))
+    B, T, Hi, d = q8.shape
+    N = k8.shape[1]
+    out = np.empty((B, T, N), np.float64)
+    mag = np.empty_like(out)
+    for b in range(B):
+        ob, mb = np.empty((T, N), np.float64), np.empty((T, N), np.float64)
+        _check(lib.oracle_index_scores_e4m3(np.ascontiguousarray(q8[b]), np.ascontiguousarray(q_scale[b]),
+                                            np.ascontiguousarray(w[b]), np.ascontiguousarray(k8[b]),
+                                            np.ascontiguousarray(k_scale[b]), np.ascontiguousarray(nv[b]),
+                                            T, N, Hi, d, ob, mb), "index_scores_e4m3")
+        out[b], mag[b] = ob, mb
+    return (out, mag) if with_mag else out
+
+
+def e4m3_decode(codes):
+    lib = _load()
+    c = np.asarray(codes, np.uint8)
+    return np.asarray([lib.oracle_e4m3_decode(int(b)) for b in c.reshape(-1)], np.float64).reshape(c.shape)
+
+
+def e4m3_encode(x):
+    lib = _load()
+    a = np.asarray(x, np.float32)
+    return np.asarray([lib.oracle_e4m3_encode(float(v)) for v in a.reshape(-1)], np.uint8).reshape(a.shape)
+
+
+def quantize_rows_e4m3(x):
+    """Per-row e4m3 quantisation (scale = amax/448 in fp32).  x [..., cols] -> (codes u8, scale f32)."""
+    lib = _load()
+    x = _f32(x)
+    cols = x.shape[-1]
+    rows = x.size // cols
+    codes = np.empty(x.shape, np.uint8)
+    scale = np.empty(x.shape[:-1], np.float32)
+    _check(lib.oracle_quantize_rows_e4m3(x, rows, cols, codes, scale), "quantize_rows_e4m3")
+    return codes, scale
+
+
+# --------------------------------------------------------------------------- top-k
+def topk(scores, n_valid, k: int):
+    """Full-sort top-k.  scores [B,T,N] float32, n_valid [B,T] -> idx [B,T,k] int32."""
+    lib = _load()
+    s = _f32(scores)
+    nv = np.ascontiguousarray(np.asarray(n_valid, np.int32))
+    B, T, N = s.shape
+    out = np.empty((B, T, k), np.int32)
+    for b in range(B):
+        ob = np.empty((T, k), np.int32)
+        _check(lib.oracle_topk(np.ascontiguousarray(s[b]), np.ascontiguousarray(nv[b]), T, N, k, ob), "topk")
+        out[b] = ob
+    return out
+
+
+# --------------------------------------------------------------------------- attention
+def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale, window: int = 128, with_mag: bool = False):
+    """[HA] §6-§7 / [P2] sparse_attn.  q [B,T,H,D], kv [B,N,D], swa_kv [B,W,D], swa_pos0 [B],
+    q_pos [B,T], sink [H], idx [B,T,k] -> out [B,T,H,D] float64."""
+    lib = _load()
+    q, kv, swa_kv, sink = _f32(q), _f32(kv), _f32(swa_kv), _f32(sink)
+    idx = np.ascontiguousarray(np.asarray(idx, np.int32))
+    q_pos = np.ascontiguousarray(np.asarray(q_pos, np.int64))
+    swa_pos0 = np.asarray(swa_pos0, np.int64).reshape(-1)
+    B, T, H, D = q.shape
+    N, W, k = kv.shape[1], swa_kv.shape[1], idx.shape[2]
+    out = np.empty((B, T, H, D), np.float64)
+    mag = np.empty_like(out)
+    for b in range(B):
+        ob, mb = np.empty((T, H, D), np.float64), np.empty((T, H, D), np.float64)
+        _check(lib.oracle_sparse_attn(np.ascontiguousarray(q[b]), np.ascontiguousarray(kv[b]),
+                                      np.ascontiguousarray(swa_kv[b]), int(swa_pos0[b]), W,
+                                      np.ascontiguousarray(q_pos[b]), sink, np.ascontiguousarray(idx[b]),
+                                      k, float(scale), window, T, H, D, N, ob, mb), "sparse_attn")
+        out[b], mag[b] = ob, mb
+    return (out, mag) if with_mag else out
+
+
+def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale, ratio: int = 128, window: int = 128,
+             with_mag: bool = False):
+    """[HA] §5 dense MQA over every complete summary plus the SWA rows."""
+    lib = _load()
+    q, kv, swa_kv, sink = _f32(q), _f32(kv), _f32(swa_kv), _f32(sink)
+    q_pos = np.ascontiguousarray(np.asarray(q_pos, np.int64))
+    swa_pos0 = np.asarray(swa_pos0, np.int64).reshape(-1)
+    B, T, H, D = q.shape
+    N, W = kv.shape[1], swa_kv.shape[1]
+    out = np.empty((B, T, H, D), np.float64)
+    mag = np.empty_like(out)
+    for b in range(B):
+        ob, mb = np.empty((T, H, D), np.float64), np.empty((T, H, D), np.float64)
+        _check(lib.oracle_hca_attn(np.ascontiguousarray(q[b]), np.ascontiguousarray(kv[b]),
+                                   np.ascontiguousarray(swa_kv[b]), int(swa_pos0[b]), W,
+                                   np.ascontiguousarray(q_pos[b]), sink, ratio, float(scale), window,
+                                   T, H, D, N, ob, mb), "hca_attn")
+        out[b], mag[b] = ob, mb
+    return (out, mag) if with_mag else out

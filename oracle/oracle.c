@@ -1,0 +1,422 @@
+/*
+ * oracle.c -- plain, single-threaded CPU oracle for the CSA / HCA hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or constant with the
+ * CUDA library.
+ *
+ * Every stage is the literal definition, accumulated in double precision.
+ * Inputs arrive as float (fp32, and bf16 / e4m3 values widened exactly), or
+ * as raw e4m3 codes; outputs are double.  Sources:
+ *
+ *   [HA] "DeepSeek-V4 混合注意力：从压缩记忆到百万上下文" (brenchcc.github.io notes):
+ *        §4.1 two-branch overlapped compression (alpha and C^comp equations),
+ *        §4.2 Lightning Indexer score s_{t,i}, §5 HCA (beta and C^hca equations),
+ *        §6 SWA window and attention-sink probability p_i, §7 call chain
+ *        (compress -> index -> top-k -> gather -> concat with SWA -> one MQA).
+ *   [P1] "揭秘DeepSeek-V4-Pro-MXFP4稀疏注意力：哈希索引与DSA如何撑起1M超长上下文？":
+ *        window_size 128, index_topk, attn_sink, sparse_attn_kernel gather.
+ *   [P2] "解密DeepSeek-V4-Flash-NVFP4的混合注意力机制：压缩稀疏注意力如何提升长文本处理能力":
+ *        sparse_attn(q, kv, attn_sink, topk_idxs, softmax_scale) call shape.
+ *
+ * Readings of points the pages leave open (each is listed in the design notes):
+ *   - Compressor rows are 0-based: entry i takes b-rows (i-1)m..im-1 and
+ *     a-rows im..(i+1)m-1; softmax position 0..m-1 are the b rows.
+ *   - Entry 0 with no previous block has no b positions (logit -inf).
+ *   - A trailing partial block yields no entry.
+ *   - Index keys are shared by the 64 index heads; no 1/sqrt(d) in the score.
+ *   - FP8 (e4m3) inputs are dequantised as code * scale and the score is the
+ *     plain definition on the dequantised values.
+ *   - Top-k: k largest over i < n_valid, ties to the lower index, output
+ *     ascending, padded with -1; -0.0 and +0.0 compare equal.
+ *   - Attention: z_j = scale * <q, row_j>; the sink logit is used unscaled;
+ *     rows are the gathered entries (idx outside [0, N) contributes nothing)
+ *     and the SWA positions max(0, t-127)..t that lie inside the SWA buffer;
+ *     no de-duplication between the two sets.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_BAD 1
+
+/* ------------------------------------------------------------------------ */
+/* [HA] §4.1: C^comp_{i,j} = sum_r alpha_{i,r,j} C^b_{(i-1)m+r,j}
+ *                         + sum_r alpha_{i,m+r,j} C^a_{im+r,j},
+ * alpha_{i,:,j} = softmax([Z^b_{(i-1)m:im,j} ; Z^a_{im:(i+1)m,j}]) over 2m.
+ * One sequence.  Inputs are [L, c] row-major; prev_Cb / prev_Zb hold the
+ * b-branch rows of the block before row 0 ([m, c]) or are NULL.
+ * out and mag are [L/m, c]; mag = sum_r alpha |C| (forward-error scale). */
+int oracle_compress_csa(const float *Ca, const float *Cb, const float *Za, const float *Zb,
+                        const float *prev_Cb, const float *prev_Zb, int64_t L, int c, int m,
+                        double *out, double *mag)
+{
+    if (m <= 0 || c <= 0 || L < 0) return ORC_BAD;
+    int64_t n_entries = L / m;
+    double *logit = (double *)malloc(sizeof(double) * 2 * m);
+    double *value = (double *)malloc(sizeof(double) * 2 * m);
+    int *present = (int *)malloc(sizeof(int) * 2 * m);
+    if (!logit || !value || !present) { free(logit); free(value); free(present); return ORC_BAD; }
+    for (int64_t i = 0; i < n_entries; ++i) {
+        for (int j = 0; j < c; ++j) {
+            /* the 2m positions: r = 0..m-1 from the previous block's b branch,
+             * r = m..2m-1 from this block's a branch */
+            for (int r = 0; r < m; ++r) {
+                if (i > 0) {
+                    int64_t row = (i - 1) * m + r;
+                    logit[r] = Zb[row * c + j];
+                    value[r] = Cb[row * c + j];
+                    present[r] = 1;
+                } else if (prev_Zb && prev_Cb) {
+                    logit[r] = prev_Zb[(int64_t)r * c + j];
+                    value[r] = prev_Cb[(int64_t)r * c + j];
+                    present[r] = 1;
+                } else {
+                    present[r] = 0;
+                }
+                int64_t arow = i * m + r;
+                logit[m + r] = Za[arow * c + j];
+                value[m + r] = Ca[arow * c + j];
+                present[m + r] = 1;
+            }
+            double mx = -INFINITY;
+            for (int r = 0; r < 2 * m; ++r)
+                if (present[r] && logit[r] > mx) mx = logit[r];
+            double den = 0.0;
+            for (int r = 0; r < 2 * m; ++r)
+                if (present[r]) den += exp(logit[r] - mx);
+            double acc = 0.0, amag = 0.0;
+            for (int r = 0; r < 2 * m; ++r) {
+                if (!present[r]) continue;
+                double alpha = exp(logit[r] - mx) / den;
+                acc += alpha * value[r];
+                amag += alpha * fabs(value[r]);
+            }
+            out[i * c + j] = acc;
+            if (mag) mag[i * c + j] = amag;
+        }
+    }
+    free(logit); free(value); free(present);
+    return ORC_OK;
+}
+
+/* [HA] §5: beta_{i,:,j} = softmax(Z_{im':(i+1)m', j}),
+ *          C^hca_{i,j} = sum_r beta_{i,r,j} C_{im'+r, j}.   One sequence. */
+int oracle_compress_hca(const float *C, const float *Z, int64_t L, int c, int m,
+                        double *out, double *mag)
+{
+    if (m <= 0 || c <= 0 || L < 0) return ORC_BAD;
+    int64_t n_entries = L / m;
+    for (int64_t i = 0; i < n_entries; ++i) {
+        for (int j = 0; j < c; ++j) {
+            double mx = -INFINITY;
+            for (int r = 0; r < m; ++r) {
+                double z = Z[(i * m + r) * c + j];
+                if (z > mx) mx = z;
+            }
+            double den = 0.0;
+            for (int r = 0; r < m; ++r) den += exp((double)Z[(i * m + r) * c + j] - mx);
+            double acc = 0.0, amag = 0.0;
+            for (int r = 0; r < m; ++r) {
+                double beta = exp((double)Z[(i * m + r) * c + j] - mx) / den;
+                double v = C[(i * m + r) * c + j];
+                acc += beta * v;
+                amag += beta * fabs(v);
+            }
+            out[i * c + j] = acc;
+            if (mag) mag[i * c + j] = amag;
+        }
+    }
+    return ORC_OK;
+}
+
+/* Causal visibility of compressed entries: entry i (covering raw tokens
+ * im..(i+1)m-1) is complete, hence visible to the query at absolute position
+ * t, iff (i+1)m <= t+1 ([HA] §6: the SWA branch holds tokens of the block
+ * that is not yet full).  Number of visible entries, capped at N. */
+int64_t oracle_n_visible(int64_t t, int m, int64_t N)
+{
+    if (t < 0 || m <= 0) return 0;
+    int64_t nv = (t + 1) / m;
+    return nv < N ? nv : N;
+}
+
+/* [HA] §4.2: s_{t,i} = sum_h w_{t,h} ReLU(<q^I_{t,h}, k^I_i>), i < n_valid(t);
+ * s = -inf for n_valid(t) <= i < N.  qI [T, Hi, d], w [T, Hi], kI [N, d],
+ * scores and mag [T, N]; mag = sum_h |w| sum_d |q k| (forward-error scale). */
+int oracle_index_scores(const float *qI, const float *w, const float *kI, const int32_t *n_valid,
+                        int T, int64_t N, int Hi, int d, double *scores, double *mag)
+{
+    if (T < 0 || N < 0 || Hi <= 0 || d <= 0) return ORC_BAD;
+    for (int t = 0; t < T; ++t) {
+        int64_t nv = n_valid[t];
+        if (nv < 0 || nv > N) return ORC_BAD;
+        for (int64_t i = 0; i < N; ++i) {
+            if (i >= nv) {
+                scores[(int64_t)t * N + i] = -INFINITY;
+                if (mag) mag[(int64_t)t * N + i] = 0.0;
+                continue;
+            }
+            double s = 0.0, smag = 0.0;
+            for (int h = 0; h < Hi; ++h) {
+                const float *q = qI + ((int64_t)t * Hi + h) * d;
+                const float *k = kI + i * d;
+                double dot = 0.0, dmag = 0.0;
+                for (int e = 0; e < d; ++e) {
+                    double p = (double)q[e] * (double)k[e];
+                    dot += p;
+                    dmag += fabs(p);
+                }
+                double wh = w[(int64_t)t * Hi + h];
+                s += wh * (dot > 0.0 ? dot : 0.0);
+                smag += fabs(wh) * dmag;
+            }
+            scores[(int64_t)t * N + i] = s;
+            if (mag) mag[(int64_t)t * N + i] = smag;
+        }
+    }
+    return ORC_OK;
+}
+
+/* ---- OCP 8-bit floating point, E4M3 variant (bias 7, no infinities,
+ * S.1111.111 is NaN, largest finite 448 = 1.75 * 2^8, subnormals 2^-9 * m). */
+double oracle_e4m3_decode(uint8_t b)
+{
+    int s = b >> 7, e = (b >> 3) & 15, mt = b & 7;
+    double v;
+    if (e == 15 && mt == 7) return NAN;
+    if (e == 0) v = ldexp((double)mt, -9);
+    else v = ldexp(1.0 + mt / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Round to the nearest finite e4m3 value, ties to the code with an even
+ * mantissa, magnitudes beyond 448 saturate to 448 ("satfinite").  Plain
+ * search over the 127 non-negative finite codes, which are increasing. */
+uint8_t oracle_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    int lo = 0, hi = 0x7E;               /* decode(lo) <= a < decode(hi) */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (oracle_e4m3_decode((uint8_t)mid) <= a) lo = mid; else hi = mid;
+    }
+    double dlo = a - oracle_e4m3_decode((uint8_t)lo);
+    double dhi = oracle_e4m3_decode((uint8_t)hi) - a;
+    int code;
+    if (dlo < dhi) code = lo;
+    else if (dhi < dlo) code = hi;
+    else code = (lo & 1) ? hi : lo;      /* tie: even mantissa */
+    return sign | (uint8_t)code;
+}
+
+/* Per-row symmetric e4m3 quantisation: scale = amax / 448 (fp32),
+ * code = e4m3(x / scale) with the division in fp32; an all-zero row gets
+ * scale 1.  x [rows, cols] -> codes [rows, cols], scale [rows]. */
+int oracle_quantize_rows_e4m3(const float *x, int64_t rows, int cols, uint8_t *codes, float *scale)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int j = 0; j < cols; ++j) {
+            float a = fabsf(x[r * cols + j]);
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax / 448.0f;
+        if (amax == 0.0f) s = 1.0f;
+        scale[r] = s;
+        for (int j = 0; j < cols; ++j) {
+            volatile float y = x[r * cols + j] / s;
+            codes[r * cols + j] = oracle_e4m3_encode(y);
+        }
+    }
+    return ORC_OK;
+}
+
+/* [HA] §4.2 on dequantised e4m3 inputs: q = code * q_scale[t,h],
+ * k = code * k_scale[i]; the score is the plain definition on those values. */
+int oracle_index_scores_e4m3(const uint8_t *q8, const float *q_scale, const float *w,
+                             const uint8_t *k8, const float *k_scale, const int32_t *n_valid,
+                             int T, int64_t N, int Hi, int d, double *scores, double *mag)
+{
+    double table[256];
+    for (int b = 0; b < 256; ++b) table[b] = oracle_e4m3_decode((uint8_t)b);
+    double *qd = (double *)malloc(sizeof(double) * (size_t)Hi * d);
+    if (!qd) return ORC_BAD;
+    for (int t = 0; t < T; ++t) {
+        int64_t nv = n_valid[t];
+        if (nv < 0 || nv > N) { free(qd); return ORC_BAD; }
+        for (int h = 0; h < Hi; ++h)
+            for (int e = 0; e < d; ++e)
+                qd[h * d + e] = table[q8[((int64_t)t * Hi + h) * d + e]] * (double)q_scale[(int64_t)t * Hi + h];
+        for (int64_t i = 0; i < N; ++i) {
+            if (i >= nv) {
+                scores[(int64_t)t * N + i] = -INFINITY;
+                if (mag) mag[(int64_t)t * N + i] = 0.0;
+                continue;
+            }
+            double ks = k_scale[i];
+            double s = 0.0, smag = 0.0;
+            for (int h = 0; h < Hi; ++h) {
+                double dot = 0.0, dmag = 0.0;
+                for (int e = 0; e < d; ++e) {
+                    double p = qd[h * d + e] * (table[k8[i * d + e]] * ks);
+                    dot += p;
+                    dmag += fabs(p);
+                }
+                double wh = w[(int64_t)t * Hi + h];
+                s += wh * (dot > 0.0 ? dot : 0.0);
+                smag += fabs(wh) * dmag;
+            }
+            scores[(int64_t)t * N + i] = s;
+            if (mag) mag[(int64_t)t * N + i] = smag;
+        }
+    }
+    free(qd);
+    return ORC_OK;
+}
+
+/* ---- top-k: full sort by (score descending, index ascending) ------------ */
+typedef struct { double s; int64_t i; } orc_pair;
+
+static int orc_cmp_desc(const void *a, const void *b)
+{
+    const orc_pair *x = (const orc_pair *)a, *y = (const orc_pair *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->i < y->i) ? -1 : (x->i > y->i);
+}
+
+static int orc_cmp_i32(const void *a, const void *b)
+{
+    int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/* [HA] §4.2 / §7 topk(scores, k): the k largest s_{t,i} over i < n_valid(t),
+ * lower index first among equal scores, returned in ascending index order,
+ * padded with -1 when n_valid(t) < k.  scores [T, N] -> idx [T, k]. */
+int oracle_topk(const float *scores, const int32_t *n_valid, int T, int64_t N, int k, int32_t *idx)
+{
+    if (k <= 0 || N < 0) return ORC_BAD;
+    orc_pair *buf = (orc_pair *)malloc(sizeof(orc_pair) * (N > 0 ? N : 1));
+    if (!buf) return ORC_BAD;
+    for (int t = 0; t < T; ++t) {
+        int64_t nv = n_valid[t];
+        if (nv < 0 || nv > N) { free(buf); return ORC_BAD; }
+        for (int64_t i = 0; i < nv; ++i) {
+            buf[i].s = (double)scores[(int64_t)t * N + i];   /* -0.0 == +0.0 here */
+            buf[i].i = i;
+        }
+        qsort(buf, (size_t)nv, sizeof(orc_pair), orc_cmp_desc);
+        int64_t take = nv < k ? nv : k;
+        int32_t *row = idx + (int64_t)t * k;
+        for (int64_t j = 0; j < take; ++j) row[j] = (int32_t)buf[j].i;
+        qsort(row, (size_t)take, sizeof(int32_t), orc_cmp_i32);
+        for (int64_t j = take; j < k; ++j) row[j] = -1;
+    }
+    free(buf);
+    return ORC_OK;
+}
+
+/* ---- attention ------------------------------------------------------------
+ * [HA] §6: p_j = exp(z_j) / (exp(z_s) + sum_l exp(z_l)), o = sum_j p_j v_j with
+ * the shared latent as both key and value ([HA] §4.2 Shared-KV MQA), over
+ * memory = concat(SWA rows, selected rows) ([HA] §7).  Two passes: maximum
+ * first, then the normalised sum.  One sequence; rows[] lists the memory. */
+static void orc_attend(const float *q, int H, int D, double scale, const float *sink,
+                       const float **rows, int64_t n_rows, double *out, double *mag, double *z)
+{
+    for (int h = 0; h < H; ++h) {
+        const float *qh = q + (int64_t)h * D;
+        double mx = (double)sink[h];
+        for (int64_t j = 0; j < n_rows; ++j) {
+            double dot = 0.0;
+            for (int e = 0; e < D; ++e) dot += (double)qh[e] * (double)rows[j][e];
+            z[j] = scale * dot;
+            if (z[j] > mx) mx = z[j];
+        }
+        double den = exp((double)sink[h] - mx);
+        for (int64_t j = 0; j < n_rows; ++j) den += exp(z[j] - mx);
+        double *oh = out + (int64_t)h * D;
+        double *mh = mag ? mag + (int64_t)h * D : NULL;
+        for (int e = 0; e < D; ++e) { oh[e] = 0.0; if (mh) mh[e] = 0.0; }
+        for (int64_t j = 0; j < n_rows; ++j) {
+            double p = exp(z[j] - mx) / den;
+            for (int e = 0; e < D; ++e) {
+                oh[e] += p * (double)rows[j][e];
+                if (mh) mh[e] += p * fabs((double)rows[j][e]);
+            }
+        }
+    }
+}
+
+/* SWA rows visible to the query at absolute position t: positions
+ * max(0, t-window+1)..t ([P1] window_size 128; [HA] §6), taken from the raw
+ * buffer swa[W, D] whose row 0 is absolute position swa_pos0. */
+static int64_t orc_swa_rows(const float *swa, int64_t swa_pos0, int W, int D, int64_t t, int window,
+                            const float **rows)
+{
+    int64_t n = 0;
+    int64_t p0 = t - window + 1;
+    if (p0 < 0) p0 = 0;
+    for (int64_t p = p0; p <= t; ++p) {
+        int64_t r = p - swa_pos0;
+        if (r < 0 || r >= W) continue;
+        rows[n++] = swa + r * D;
+    }
+    return n;
+}
+
+/* sparse_attn for one sequence ([P2] sparse_attn(q, kv, attn_sink, topk_idxs,
+ * softmax_scale); [HA] §7 gather + concat + shared_kv_mqa).
+ * q [T, H, D], kv [N, D], swa [W, D], q_pos [T], sink [H], idx [T, k]
+ * -> out, mag [T, H, D]. */
+int oracle_sparse_attn(const float *q, const float *kv, const float *swa, int64_t swa_pos0, int W,
+                       const int64_t *q_pos, const float *sink, const int32_t *idx, int k,
+                       double scale, int window, int T, int H, int D, int64_t N,
+                       double *out, double *mag)
+{
+    int64_t cap = (int64_t)k + window;
+    const float **rows = (const float **)malloc(sizeof(float *) * (cap > 0 ? cap : 1));
+    double *z = (double *)malloc(sizeof(double) * (cap > 0 ? cap : 1));
+    if (!rows || !z) { free(rows); free(z); return ORC_BAD; }
+    for (int t = 0; t < T; ++t) {
+        int64_t n = orc_swa_rows(swa, swa_pos0, W, D, q_pos[t], window, rows);
+        for (int j = 0; j < k; ++j) {
+            int64_t i = idx[(int64_t)t * k + j];
+            if (i < 0 || i >= N) continue;
+            rows[n++] = kv + i * D;
+        }
+        orc_attend(q + (int64_t)t * H * D, H, D, scale, sink, rows, n,
+                   out + (int64_t)t * H * D, mag ? mag + (int64_t)t * H * D : NULL, z);
+    }
+    free(rows); free(z);
+    return ORC_OK;
+}
+
+/* hca_attn for one sequence ([HA] §5: dense MQA over every complete summary,
+ * concatenated with the SWA rows): entries 0..n_visible(t)-1 of kv. */
+int oracle_hca_attn(const float *q, const float *kv, const float *swa, int64_t swa_pos0, int W,
+                    const int64_t *q_pos, const float *sink, int ratio, double scale, int window,
+                    int T, int H, int D, int64_t N, double *out, double *mag)
+{
+    int64_t cap = N + window;
+    const float **rows = (const float **)malloc(sizeof(float *) * (cap > 0 ? cap : 1));
+    double *z = (double *)malloc(sizeof(double) * (cap > 0 ? cap : 1));
+    if (!rows || !z) { free(rows); free(z); return ORC_BAD; }
+    for (int t = 0; t < T; ++t) {
+        int64_t n = orc_swa_rows(swa, swa_pos0, W, D, q_pos[t], window, rows);
+        int64_t nv = oracle_n_visible(q_pos[t], ratio, N);
+        for (int64_t i = 0; i < nv; ++i) rows[n++] = kv + i * D;
+        orc_attend(q + (int64_t)t * H * D, H, D, scale, sink, rows, n,
+                   out + (int64_t)t * H * D, mag ? mag + (int64_t)t * H * D : NULL, z);
+    }
+    free(rows); free(z);
+    return ORC_OK;
+}

@@ -1,0 +1,471 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU).
+
+Each test fixes the oracle to something other than itself: the worked example
+and entry counts printed in "DeepSeek-V4 混合注意力：从压缩记忆到百万上下文" (§3, §4.1),
+closed forms, invariants, library routines for special cases (numpy stable
+sort, torch scaled_dot_product_attention in float64, numpy matmul), and brute
+force over all subsets on tiny inputs.  Each is chosen so that a plausible slip
+in the oracle (a dropped branch, an off-by-one row, a transposed operand, a
+wrong sign) fails at least one of them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_compressed_b200 import synth
+
+RNG = np.random.default_rng(1234)
+
+
+def rnd(*shape, scale=1.0):
+    return (RNG.standard_normal(shape) * scale).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------- compressor
+def test_worked_example_alpha(golden):
+    """§4.1: logits log([1,2,1,2,4,2,1,3]) give alpha = [1,2,1,2,4,2,1,3]/16.
+
+    Entry i=1 of a two-block sequence: positions 0..3 are the b-branch rows 0..3
+    (block 0), positions 4..7 the a-branch rows 4..7 (block 1).  Channel j holds
+    one-hot contents selecting position j, so out[1, j] = alpha_j."""
+    g = golden("worked_example_alpha.json")
+    w = np.array(g["weights"], np.float64)
+    m, L, c = 4, 8, 8
+    Zb = np.zeros((L, c), np.float32)
+    Za = np.zeros((L, c), np.float32)
+    Cb = np.zeros((L, c), np.float32)
+    Ca = np.zeros((L, c), np.float32)
+    for r in range(m):
+        Zb[r, :] = np.log(w[r])
+        Za[m + r, :] = np.log(w[m + r])
+        Cb[r, r] = 1.0
+        Ca[m + r, m + r] = 1.0
+    out = oracle.compress_csa(Ca, Cb, Za, Zb, m=m)
+    expect = np.array(g["alpha_times_16"], np.float64) / g["denominator"]
+    # log() of the weights is rounded to fp32 on input: allow that rounding only.
+    np.testing.assert_allclose(out[1], expect, rtol=0, atol=1e-7)
+    assert abs(out[1].sum() - 1.0) < 1e-12
+
+
+def test_compress_row_mapping_one_hot():
+    """A dominant logit at one of the 2m rows selects exactly that row's content:
+    pins which raw rows (b: (i-1)m..im-1, a: im..(i+1)m-1) feed entry i."""
+    m, L, c = 4, 24, 3
+    Ca, Cb = rnd(L, c), rnd(L, c)
+    for i in range(1, L // m):
+        for branch in ("a", "b"):
+            for r in range(m):
+                Za = np.zeros((L, c), np.float32)
+                Zb = np.zeros((L, c), np.float32)
+                row = i * m + r if branch == "a" else (i - 1) * m + r
+                (Za if branch == "a" else Zb)[row, :] = 80.0
+                out = oracle.compress_csa(Ca, Cb, Za, Zb, m=m)
+                src = Ca if branch == "a" else Cb
+                np.testing.assert_allclose(out[i], src[row], rtol=0, atol=1e-20 + 1e-30)
+
+
+def test_compress_channels_independent():
+    """Each channel has its own softmax: channel j one-hot at a different position."""
+    m, L, c = 4, 8, 8
+    Ca, Cb = rnd(L, c), rnd(L, c)
+    Za = np.zeros((L, c), np.float32)
+    Zb = np.zeros((L, c), np.float32)
+    for j in range(c):
+        if j < m:
+            Zb[j, j] = 90.0
+        else:
+            Za[j, j] = 90.0
+    out = oracle.compress_csa(Ca, Cb, Za, Zb, m=m)
+    for j in range(c):
+        src = Cb if j < m else Ca
+        assert out[1, j] == pytest.approx(float(src[j, j]), abs=1e-30)
+
+
+def test_compress_invariants():
+    m, L, c = 4, 64, 16
+    Za, Zb = rnd(L, c, scale=3.0), rnd(L, c, scale=3.0)
+    # constant content along each channel -> that constant (sum alpha = 1)
+    const = rnd(1, c)
+    out = oracle.compress_csa(np.repeat(const, L, 0), np.repeat(const, L, 0), Za, Zb, m=m)
+    np.testing.assert_allclose(out, np.repeat(const.astype(np.float64), L // m, 0), rtol=1e-6)
+    # constant logits -> plain mean of the 2m rows (entry 0: of its m a-rows)
+    Ca, Cb = rnd(L, c), rnd(L, c)
+    zero = np.zeros((L, c), np.float32)
+    out = oracle.compress_csa(Ca, Cb, zero, zero, m=m)
+    for i in range(L // m):
+        rows = [Ca[i * m:(i + 1) * m]] + ([Cb[(i - 1) * m:i * m]] if i > 0 else [])
+        expect = np.concatenate(rows).astype(np.float64).mean(0)
+        np.testing.assert_allclose(out[i], expect, rtol=1e-12, atol=1e-12)
+    # convexity: output lies within [min, max] of the 2m contributing rows
+    out = oracle.compress_csa(Ca, Cb, Za, Zb, m=m)
+    for i in range(1, L // m):
+        rows = np.concatenate([Cb[(i - 1) * m:i * m], Ca[i * m:(i + 1) * m]])
+        assert np.all(out[i] <= rows.max(0) + 1e-12) and np.all(out[i] >= rows.min(0) - 1e-12)
+
+
+def test_compress_first_entry_is_a_branch_softmax():
+    """Entry 0 without a carry reduces to softmax over its m a-rows (torch.softmax in float64)."""
+    m, L, c = 4, 16, 8
+    Ca, Cb, Za, Zb = rnd(L, c), rnd(L, c), rnd(L, c), rnd(L, c)
+    out = oracle.compress_csa(Ca, Cb, Za, Zb, m=m)
+    a = torch.softmax(torch.from_numpy(Za[:m].astype(np.float64)), dim=0)
+    expect = (a * torch.from_numpy(Ca[:m].astype(np.float64))).sum(0).numpy()
+    np.testing.assert_allclose(out[0], expect, rtol=1e-12, atol=1e-14)
+
+
+def test_compress_carry_chunked_equals_whole():
+    """compress(0..L) == compress(0..L1) ++ compress(L1..L, carry = b rows of block L1/m - 1), bit-exact."""
+    m, L, c = 4, 64, 8
+    Ca, Cb, Za, Zb = rnd(L, c), rnd(L, c), rnd(L, c), rnd(L, c)
+    whole = oracle.compress_csa(Ca, Cb, Za, Zb, m=m)
+    L1 = 24
+    first = oracle.compress_csa(Ca[:L1], Cb[:L1], Za[:L1], Zb[:L1], m=m)
+    second = oracle.compress_csa(Ca[L1:], Cb[L1:], Za[L1:], Zb[L1:],
+                                 prev_Cb=Cb[L1 - m:L1], prev_Zb=Zb[L1 - m:L1], m=m)
+    assert np.array_equal(np.concatenate([first, second]), whole)
+
+
+def test_compress_partial_block_dropped():
+    m, c = 4, 4
+    Ca, Cb, Za, Zb = rnd(10, c), rnd(10, c), rnd(10, c), rnd(10, c)
+    assert oracle.compress_csa(Ca, Cb, Za, Zb, m=m).shape == (2, c)
+
+
+def test_hca_compress_pins():
+    m, L, c = 128, 384, 8
+    C = rnd(L, c)
+    zero = np.zeros((L, c), np.float32)
+    out = oracle.compress_hca(C, zero, m=m)
+    np.testing.assert_allclose(out, C.astype(np.float64).reshape(3, m, c).mean(1), rtol=1e-12, atol=1e-13)
+    # a dominant logit selects its row; blocks do not overlap
+    Z = rnd(L, c)
+    Z[128 + 37, 2] = 200.0
+    out = oracle.compress_hca(C, Z, m=m)
+    assert out[1, 2] == pytest.approx(float(C[128 + 37, 2]), abs=1e-30)
+    Z2 = Z.copy()
+    Z2[:128] += rnd(128, c)   # perturb block 0 only
+    C2 = C.copy()
+    C2[256:] += 1.0           # and block 2's contents
+    out2 = oracle.compress_hca(C2, Z2, m=m)
+    assert np.array_equal(out2[1], out[1])
+    # softmax over a block equals torch.softmax (library routine) weighted sum
+    b = torch.softmax(torch.from_numpy(Z[256:384].astype(np.float64)), 0)
+    np.testing.assert_allclose(out[2], (b * torch.from_numpy(C[256:384].astype(np.float64))).sum(0).numpy(),
+                               rtol=1e-12, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- counts / causality
+def test_entry_counts(golden):
+    g = golden("entry_counts.json")
+    n = g["n"]
+    assert oracle.n_visible([n - 1], 4, 1 << 40)[0] == g["csa_entries"]
+    assert oracle.n_visible([n - 1], 128, 1 << 40)[0] == g["hca_entries"]
+    assert g["topk"]["flash"] + g["swa_window"] == g["working_set_rows"]["flash_csa"]
+    assert g["topk"]["pro"] + g["swa_window"] == g["working_set_rows"]["pro_csa"]
+    assert g["hca_entries"] + g["swa_window"] == g["working_set_rows"]["hca"]
+    wl = synth.WORKLOADS["pro1m"]
+    assert wl.N == g["csa_entries"] and wl.topk == g["topk"]["pro"]
+    assert synth.WORKLOADS["pro_hca"].N == g["hca_entries"]
+
+
+def test_tiny_n_valid(golden):
+    g = golden("tiny_n_valid.json")
+    assert oracle.n_visible(g["q_pos"], g["ratio"], 1024).tolist() == g["n_valid"]
+    # the boundary itself: entry i becomes visible exactly at t = (i+1)m - 1
+    for i in range(5):
+        t = (i + 1) * 4 - 1
+        assert oracle.n_visible([t - 1, t], 4, 100).tolist() == [i, i + 1]
+
+
+# ----------------------------------------------------------------------------- indexer
+def _index_inputs(T=3, N=50, Hi=64, d=128):
+    return rnd(1, T, Hi, d), rnd(1, T, Hi), rnd(1, N, d)
+
+
+def test_index_relu_split_reduces_to_matmul():
+    """ReLU(x) - ReLU(-x) = x, so s(q) - s(-q) = sum_h w_h <q_h, k_i> = numpy matmul."""
+    qI, w, kI = _index_inputs()
+    nv = np.array([[50, 50, 50]], np.int32)
+    s_pos = oracle.index_scores(qI, w, kI, nv)
+    s_neg = oracle.index_scores(-qI, w, kI, nv)
+    lin = np.einsum("th,thd->td", w[0].astype(np.float64), qI[0].astype(np.float64)) @ kI[0].astype(np.float64).T
+    np.testing.assert_allclose(s_pos[0] - s_neg[0], lin, rtol=1e-10, atol=1e-9)
+    # and s(q) + s(-q) = sum_h w_h |<q_h, k_i>|
+    dots = np.einsum("thd,nd->thn", qI[0].astype(np.float64), kI[0].astype(np.float64))
+    np.testing.assert_allclose(s_pos[0] + s_neg[0], np.einsum("th,thn->tn", w[0], np.abs(dots)),
+                               rtol=1e-10, atol=1e-9)
+
+
+def test_index_unit_vectors_closed_form():
+    """q_{t,h} = e_{a_h}, k_i = e_{b_i}: s_{t,i} = sum_h w_h [a_h == b_i]; also a negative dot contributes 0."""
+    Hi, d, N = 64, 128, 20
+    a = RNG.integers(0, d, Hi)
+    b = RNG.integers(0, d, N)
+    q = np.zeros((1, 1, Hi, d), np.float32)
+    q[0, 0, np.arange(Hi), a] = 1.0
+    k = np.zeros((1, N, d), np.float32)
+    k[0, np.arange(N), b] = -1.0
+    w = rnd(1, 1, Hi)
+    s = oracle.index_scores(q, w, k, np.array([[N]], np.int32))
+    assert np.all(s == 0.0)
+    s = oracle.index_scores(q, w, -k, np.array([[N]], np.int32))
+    expect = np.array([w[0, 0][a == b[i]].astype(np.float64).sum() for i in range(N)])
+    np.testing.assert_allclose(s[0, 0], expect, rtol=1e-15, atol=1e-15)
+
+
+def test_index_rotation_invariance_and_causal_tail():
+    """A shared orthogonal rotation of q and k leaves scores unchanged; i >= n_valid is -inf."""
+    qI, w, kI = _index_inputs(T=2, N=40)
+    Q, _ = np.linalg.qr(RNG.standard_normal((128, 128)))
+    nv = np.array([[40, 17]], np.int32)
+    s0 = oracle.index_scores(qI.astype(np.float64), w, kI.astype(np.float64), nv)
+    s1 = oracle.index_scores((qI.astype(np.float64) @ Q), w, (kI.astype(np.float64) @ Q), nv)
+    # rotated inputs are rounded to fp32 on the way in; compare at that precision
+    mag = oracle.index_scores(np.abs(qI), np.abs(w), np.abs(kI), np.array([[40, 40]], np.int32))
+    assert np.all(np.abs(s0[0, 0] - s1[0, 0]) <= 1e-5 * mag[0, 0] + 1e-6)
+    assert np.all(np.isneginf(s0[0, 1, 17:])) and np.all(np.isfinite(s0[0, 1, :17]))
+
+
+# ----------------------------------------------------------------------------- e4m3
+def test_e4m3_codec_points(golden):
+    g = golden("e4m3_points.json")
+    for code, val in g["decode"]:
+        got = oracle.e4m3_decode([code])[0]
+        assert got == val and math.copysign(1, got) == math.copysign(1, val)
+    for x, code in g["encode_ties_to_even"]:
+        assert oracle.e4m3_encode([x])[0] == code, x
+    for code in g["nan_codes"]:
+        assert np.isnan(oracle.e4m3_decode([code])[0])
+
+
+def test_e4m3_roundtrip_and_monotone():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    back = oracle.e4m3_encode(vals.astype(np.float32))
+    assert np.array_equal(back, codes)
+    pos = oracle.e4m3_decode(np.arange(0, 127, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)
+    # nearest: a random value's code is at least as close as both neighbours
+    x = (RNG.standard_normal(2000) * 50).astype(np.float32)
+    enc = oracle.e4m3_decode(oracle.e4m3_encode(x))
+    sorted_vals = np.sort(vals[np.isfinite(vals)])
+    for xv, ev in zip(x.astype(np.float64), enc):
+        if abs(xv) >= 448:
+            assert abs(ev) == 448
+            continue
+        best = np.min(np.abs(sorted_vals - xv))
+        assert abs(ev - xv) == best
+
+
+def test_quantize_rows():
+    x = rnd(6, 128, scale=3.0)
+    x[3] = 0.0
+    codes, scale = oracle.quantize_rows_e4m3(x)
+    assert scale[3] == 1.0 and np.all(codes[3] == 0)
+    for r in (0, 1, 2, 4, 5):
+        amax = np.float32(np.abs(x[r]).max())
+        assert scale[r] == np.float32(amax / np.float32(448.0))
+        j = int(np.abs(x[r]).argmax())
+        assert codes[r, j] & 0x7F == 0x7E
+    deq = oracle.e4m3_decode(codes) * scale[:, None]
+    # relative error bound of e4m3 rounding (3 mantissa bits): half an ulp, 2^-4 relative for normals
+    big = np.abs(x) >= scale[:, None] * 2 ** -6
+    assert np.all(np.abs(deq - x)[big] <= 2 ** -4 * np.abs(x)[big] * (1 + 1e-6))
+
+
+def test_index_e4m3_matches_dequantised_f32():
+    """With power-of-two scales the dequantised values are exact in fp32, so the e4m3
+    definition must equal the (pinned) fp32 definition on those values."""
+    T, N, Hi, d = 2, 30, 64, 128
+    q8 = RNG.integers(0, 256, (1, T, Hi, d)).astype(np.uint8)
+    k8 = RNG.integers(0, 256, (1, N, d)).astype(np.uint8)
+    q8[(q8 & 0x7F) == 0x7F] = 0
+    k8[(k8 & 0x7F) == 0x7F] = 0
+    qs = (2.0 ** RNG.integers(-8, -2, (1, T, Hi))).astype(np.float32)
+    ks = (2.0 ** RNG.integers(-8, -2, (1, N))).astype(np.float32)
+    w = rnd(1, T, Hi)
+    nv = np.array([[N, 11]], np.int32)
+    s8 = oracle.index_scores_e4m3(q8, qs, w, k8, ks, nv)
+    qf = (oracle.e4m3_decode(q8) * qs[..., None]).astype(np.float32)
+    kf = (oracle.e4m3_decode(k8) * ks[..., None]).astype(np.float32)
+    sf = oracle.index_scores(qf, w, kf, nv)
+    np.testing.assert_array_equal(np.isneginf(s8), np.isneginf(sf))
+    fin = np.isfinite(sf)
+    np.testing.assert_allclose(s8[fin], sf[fin], rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- top-k
+def _brute_topk(s, nv, k):
+    """The unique k-subset S where every member beats every non-member
+    (greater score, or equal score and lower index)."""
+    cand = range(nv)
+    take = min(k, nv)
+    for S in itertools.combinations(cand, take):
+        Sset = set(S)
+        if all((s[i] > s[j]) or (s[i] == s[j] and i < j) for i in Sset for j in cand if j not in Sset):
+            return sorted(S) + [-1] * (k - take)
+    raise AssertionError("no valid subset")
+
+
+def test_topk_brute_force_tiny():
+    for trial in range(60):
+        N = int(RNG.integers(1, 11))
+        k = int(RNG.integers(1, 6))
+        nv = int(RNG.integers(0, N + 1))
+        s = RNG.integers(-3, 4, N).astype(np.float32)       # many exact ties
+        if trial % 3 == 0:
+            s[s == 0] = -0.0                                  # -0.0 ties +0.0
+        got = oracle.topk(s[None, None], [[nv]], k)[0, 0].tolist()
+        assert got == _brute_topk(s.astype(np.float64), nv, k), (s, nv, k)
+
+
+def test_topk_matches_stable_sort_on_tiny_rows():
+    """All tiny-workload-sized rows: numpy stable argsort (library routine) of -s, first k, ascending."""
+    s = synth.draw_scores(0, "pin/topk", 1, 8, 1024, ties=6).numpy()
+    nv = oracle.n_visible(list(range(4088, 4096)), 4, 1024)[None]
+    got = oracle.topk(s, nv, 64)
+    for t in range(8):
+        row = s[0, t, :nv[0, t]].astype(np.float64) + 0.0    # +0.0 folds -0.0
+        order = np.argsort(-row, kind="stable")[:64]
+        assert got[0, t].tolist() == sorted(order.tolist())
+
+
+# ----------------------------------------------------------------------------- attention
+def _sdpa_with_sink(q, rows, sink, scale):
+    """torch scaled_dot_product_attention in float64 over [sink slot; rows]: the sink
+    is a key with logit z_s (an additive mask on a zero key) and a zero value."""
+    H, D = q.shape
+    qt = torch.from_numpy(q.astype(np.float64))[:, None, :]                         # [H, 1, D]
+    keys = torch.cat([torch.zeros(1, D, dtype=torch.float64), torch.from_numpy(rows.astype(np.float64))])
+    kt = keys[None].expand(H, -1, -1)
+    mask = torch.zeros(H, 1, keys.shape[0], dtype=torch.float64)
+    mask[:, 0, 0] = torch.from_numpy(sink.astype(np.float64))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, kt, attn_mask=mask, scale=scale)
+    return o[:, 0, :].numpy()
+
+
+def test_sparse_attn_matches_sdpa_with_sink():
+    H, D, N, k = 4, 32, 40, 12
+    T = 3
+    q = rnd(1, T, H, D)
+    kv = rnd(1, N, D)
+    q_pos = np.array([[300, 301, 302]])
+    swa_pos0 = 300 - 127
+    swa = rnd(1, 130, D)
+    sink = rnd(H)
+    idx = np.stack([np.sort(RNG.choice(N, k, replace=False)) for _ in range(T)]).astype(np.int32)[None]
+    idx[0, 1, -3:] = -1                                   # padding contributes nothing
+    scale = 1 / math.sqrt(D)
+    out = oracle.sparse_attn(q, kv, swa, [swa_pos0], q_pos, sink, idx, scale)
+    for t in range(T):
+        p = q_pos[0, t]
+        swa_rows = swa[0, (p - 127 - swa_pos0):(p - swa_pos0 + 1)]
+        sel = kv[0, [i for i in idx[0, t] if i >= 0]]
+        ref = _sdpa_with_sink(q[0, t], np.concatenate([swa_rows, sel]), sink, scale)
+        np.testing.assert_allclose(out[0, t], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_sink_closed_form():
+    """Equal logits z on L rows: p = e^z / (e^{z_s} + L e^z); with all rows v, o = L p v."""
+    H, D, N = 3, 16, 20
+    v = rnd(D)
+    kv = np.repeat(v[None], N, 0)[None]
+    swa = np.repeat(v[None], 128, 0)[None]
+    q = np.zeros((1, 1, H, D), np.float32)                # z = 0 for every row
+    sink = np.array([-1.0, 0.5, 2.0], np.float32)
+    k = 7
+    idx = np.arange(k, dtype=np.int32)[None, None]
+    out = oracle.sparse_attn(q, kv, swa, [1000 - 127], [[1000]], sink, idx, 0.1)
+    L = k + 128
+    for h in range(H):
+        p = 1.0 / (math.exp(float(sink[h])) + L)
+        np.testing.assert_allclose(out[0, 0, h], L * p * v.astype(np.float64), rtol=1e-13)
+
+
+def test_sparse_attn_causal_window_and_poison():
+    """SWA rows outside t-127..t and unselected entries are never read: NaN there changes nothing."""
+    H, D, N, k = 2, 16, 30, 5
+    q = rnd(1, 2, H, D)
+    kv = rnd(1, N, D)
+    swa = rnd(1, 300, D)
+    sink = rnd(H)
+    q_pos = np.array([[500, 520]])
+    swa_pos0 = 400
+    idx = np.array([[[1, 4, 9, 20, 29], [0, 2, 3, -1, -1]]], np.int32)
+    ref = oracle.sparse_attn(q, kv, swa, [swa_pos0], q_pos, sink, idx, 0.25)
+    kv2, swa2 = kv.copy(), swa.copy()
+    used = {1, 4, 9, 20, 29, 0, 2, 3}
+    for i in range(N):
+        if i not in used:
+            kv2[0, i] = np.nan
+    for r in range(300):
+        p = swa_pos0 + r
+        if not (500 - 127 <= p <= 520):
+            swa2[0, r] = np.nan
+    got = oracle.sparse_attn(q, kv2, swa2, [swa_pos0], q_pos, sink, idx, 0.25)
+    assert np.array_equal(got, ref)
+    # the window is exactly 128 rows: query 500 must not see position 500-128
+    swa3 = swa.copy()
+    swa3[0, 500 - 128 - swa_pos0] = np.nan
+    assert np.all(np.isfinite(oracle.sparse_attn(q[:, :1], kv, swa3, [swa_pos0], q_pos[:, :1], sink,
+                                                 idx[:, :1], 0.25)))
+
+
+def test_hca_equals_sparse_with_all_entries_and_sdpa():
+    H, D, N = 4, 32, 10
+    q = rnd(2, 1, H, D)
+    kv = rnd(2, N, D)
+    swa = rnd(2, 128, D)
+    sink = rnd(H)
+    t = 128 * 7 + 5                                       # 7 complete blocks
+    q_pos = np.array([[t], [t]])
+    swa_pos0 = [t - 127, t - 127]
+    hca = oracle.hca_attn(q, kv, swa, swa_pos0, q_pos, sink, 0.2, ratio=128)
+    idx = np.full((2, 1, N), -1, np.int32)
+    idx[:, 0, :7] = np.arange(7)
+    sp = oracle.sparse_attn(q, kv, swa, swa_pos0, q_pos, sink, idx, 0.2)
+    np.testing.assert_allclose(hca, sp, rtol=1e-14, atol=1e-15)
+    kv_poison = kv.copy()
+    kv_poison[:, 7:] = np.nan                             # incomplete / future summaries
+    assert np.array_equal(oracle.hca_attn(q, kv_poison, swa, swa_pos0, q_pos, sink, 0.2, ratio=128), hca)
+    ref = _sdpa_with_sink(q[0, 0], np.concatenate([swa[0], kv[0, :7]]), sink, 0.2)
+    np.testing.assert_allclose(hca[0, 0], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_sink_minus_infinity_is_textbook_softmax():
+    H, D = 2, 8
+    q = rnd(1, 1, H, D)
+    kv = rnd(1, 6, D)
+    swa = rnd(1, 128, D)
+    sink = np.full(H, -1e30, np.float32)
+    idx = np.arange(6, dtype=np.int32)[None, None]
+    out = oracle.sparse_attn(q, kv, swa, [0], [[127]], sink, idx, 0.3)
+    rows = torch.from_numpy(np.concatenate([swa[0], kv[0]]).astype(np.float64))
+    qt = torch.from_numpy(q[0, 0].astype(np.float64))
+    ref = torch.softmax(0.3 * qt @ rows.T, dim=-1) @ rows
+    np.testing.assert_allclose(out[0, 0], ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- generator
+def test_generator_splitmix_reference(golden):
+    g = golden("splitmix64_seed0.json")
+    got = [format(v & ((1 << 64) - 1), "016x") for v in synth.raw_u64(g["state"], 0, 3).tolist()]
+    assert got == g["outputs_hex"]
+    key = synth.stream_key(0, "abc")
+    ints = [synth._mix_int(key + (i + 1) * synth._GOLDEN) for i in range(1000, 1010)]
+    assert [v & ((1 << 64) - 1) for v in synth.raw_u64(key, 1000, 10).tolist()] == ints
+
+
+def test_generator_moments_and_independence():
+    x = synth.normal(0, "moments", (200000,)).double()
+    assert abs(x.mean().item()) < 0.01 and abs(x.std().item() - 1) < 0.01
+    y = synth.normal(0, "moments2", (200000,)).double()
+    assert abs(torch.corrcoef(torch.stack([x, y]))[0, 1].item()) < 0.01
+    u = synth.uniform(0, "u", (200000,)).double()
+    assert 0 <= u.min().item() and u.max().item() < 1 and abs(u.mean().item() - 0.5) < 0.01
+    # order-independence: drawing a prefix gives the same values
+    assert torch.equal(synth.normal(3, "p", (10,)), synth.normal(3, "p", (1000,))[:10])
