@@ -1,0 +1,171 @@
+/*
+ * csa.h -- C ABI of libcsa.so: the CSA / HCA hybrid-attention hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, then section):
+ *   [HA] "DeepSeek-V4 混合注意力：从压缩记忆到百万上下文"
+ *   [P1] "揭秘DeepSeek-V4-Pro-MXFP4稀疏注意力：哈希索引与DSA如何撑起1M超长上下文？"
+ *   [P2] "解密DeepSeek-V4-Flash-NVFP4的混合注意力机制：压缩稀疏注意力如何提升长文本处理能力"
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major ("C order"), in device memory, with the
+ *     shapes stated below.  Pointers to bf16 / fp32 / e4m3 data must be
+ *     16-byte aligned; the innermost dimension must be a multiple of 8.
+ *   - The caller owns every buffer, including workspaces.  The library never
+ *     allocates, frees or synchronises; every call only enqueues kernels on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream) and returns.
+ *   - Arguments are validated on the host before anything is launched.  On
+ *     CSA_ERR_INVALID or CSA_ERR_UNSUPPORTED nothing is launched and no output
+ *     is touched.  CSA_ERR_CUDA reports a launch failure (cudaGetLastError).
+ *   - Kernels never wait without bound: a wait that runs out records
+ *     CSA_ERR_TIMEOUT in a device status word that csa_poll_status() returns.
+ *   - dtype codes: CSA_F32 (fp32), CSA_BF16 (bfloat16), CSA_E4M3 (OCP FP8 e4m3,
+ *     one byte per element).
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID = 1,     /* bad pointer, size, alignment or dtype code */
+  CSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. D not 128/256/512) */
+  CSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  CSA_ERR_TIMEOUT = 4      /* a kernel gave up a bounded wait (see csa_poll_status) */
+};
+
+enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2 };
+
+#define CSA_INDEX_HEADS 64   /* index heads per query ([HA] §2 table, §4.2) */
+#define CSA_INDEX_DIM 128    /* dims per index head */
+#define CSA_SWA_WINDOW 128   /* SWA tokens per query ([HA] §6; [P1] window_size 128) */
+#define CSA_MAX_TOPK 2048
+
+/* Human-readable name of a status code (static string). */
+const char *csa_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int csa_version(void);
+
+/*
+ * csa_compress -- token-level Compressor ([HA] §4.1 for ratio 4, §5 for 128).
+ *
+ * ratio 4 (CSA, overlapped two-branch pooling):
+ *   out[b,i,j] = sum_{r<2m} alpha_r * V_r,  alpha = softmax_r(Zcat_r) per channel j,
+ *   with positions r = 0..3 the b-branch rows (i-1)*4+r of C_b / Z_b and
+ *   r = 4..7 the a-branch rows i*4+(r-4) of C_a / Z_a.  For entry 0 the
+ *   b-branch rows are prev_Cb / prev_Zb (the b branch of the 4 raw rows just
+ *   before this chunk), or absent when those are NULL.
+ * ratio 128 (HCA, non-overlapped): out[b,i,j] = sum_{r<128} beta_r * C[b,128i+r,j],
+ *   beta = softmax_r(Z[b,128i+r,j]); C_b, Z_b, prev_* must be NULL.
+ *
+ *   C_a, Z_a (C, Z for ratio 128), C_b, Z_b : [B, L, c], dtype in_dtype (F32|BF16)
+ *   prev_Cb, prev_Zb : [B, 4, c] in_dtype, or both NULL
+ *   out   : [B, L/ratio, c], dtype out_dtype (F32|BF16); a partial trailing block
+ *           (L % ratio rows) produces no entry
+ *   c     : multiple of 8 (ratio 4) or of 128 (ratio 128)
+ * Softmax and sums in fp32.  Streaming, HBM-bound.
+ */
+int csa_compress(const void *C_a, const void *C_b, const void *Z_a, const void *Z_b, const void *prev_Cb,
+                 const void *prev_Zb, int B, int64_t L, int c, int ratio, int in_dtype, int out_dtype, void *out,
+                 void *stream);
+
+/*
+ * csa_quantize_e4m3 -- per-row symmetric e4m3 quantisation for the
+ * low-precision index QK path ([HA] §4.2 and §9: the index QK runs in low
+ * precision; this library's variant is e4m3 with a per-row scale).
+ *   x      : [rows, cols] F32 or BF16 (x_dtype)
+ *   codes  : [rows, cols] uint8 e4m3, code = RN-even(x / scale), saturating to +-448
+ *   scale  : [rows] fp32, scale = amax(|x_row|) / 448 (IEEE fp32 division); 1 for an all-zero row
+ * Use it for index keys ([B*N, 128] -> k_scale [B, N]) and index queries
+ * ([B*T*64, 128] -> q_scale [B, T, 64]).
+ */
+int csa_quantize_e4m3(const void *x, int x_dtype, int64_t rows, int cols, uint8_t *codes, float *scale,
+                      void *stream);
+
+/*
+ * csa_index_scores -- Lightning Indexer ([HA] §4.2):
+ *   scores[b,t,i] = sum_{h<64} w[b,t,h] * ReLU(<qI[b,t,h,:], kI[b,i,:]>)   for i < n_valid[b,t]
+ *   scores[b,t,i] = -inf                                                   for n_valid[b,t] <= i < N
+ * with dequantised values (code * scale) when dtype = CSA_E4M3.
+ *   qI      : [B, T, 64, 128] dtype
+ *   q_scale : [B, T, 64] fp32 (E4M3 only, else NULL)
+ *   w       : [B, T, 64] fp32
+ *   kI      : [B, N, 128] dtype   (keys shared by the 64 heads)
+ *   k_scale : [B, N] fp32 (E4M3 only, else NULL)
+ *   n_valid : [B, T] int32, 0 <= n_valid <= N (visible complete entries, (t+1)/4)
+ *   scores  : [B, T, N] fp32
+ * BF16 / E4M3 run on tcgen05 tensor cores (fp32 accumulation); F32 runs on
+ * the fp32 FMA pipes.
+ */
+int csa_index_scores(const void *qI, const float *q_scale, const float *w, const void *kI, const float *k_scale,
+                     int dtype, const int32_t *n_valid, int B, int T, int64_t N, float *scores, void *stream);
+
+/*
+ * csa_topk -- top-k of each score row ([HA] §4.2 / §7 topk(scores, k);
+ * k = 512 Flash, 1024 Pro):
+ *   idx[b,t,:] = the k indices i < n_valid[b,t] with the largest scores[b,t,i],
+ *   ties toward the lower index, in ascending index order; when
+ *   n_valid[b,t] < k the row holds 0..n_valid-1 followed by -1.
+ *   -0.0 equals +0.0; NaN scores are not supported.
+ *   scores  : [B, T, N] fp32;  n_valid : [B, T] int32;  idx : [B, T, k] int32
+ *   1 <= k <= CSA_MAX_TOPK;  N <= 2^20
+ *   workspace : csa_topk_workspace_size(B, T, N, k) bytes of device memory,
+ *               16-byte aligned, ZERO-FILLED by the caller before its first use;
+ *               every call leaves it zero-filled again.  Calls that share a
+ *               workspace must be ordered on one stream.
+ */
+size_t csa_topk_workspace_size(int B, int T, int64_t N, int k);
+int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t N, int k, int32_t *idx,
+             void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * sparse_attn -- CSA core attention ([P2] sparse_attn(q, kv, attn_sink,
+ * topk_idxs, softmax_scale); [HA] §4.2 Shared-KV MQA, §6 SWA + sink, §7 call chain):
+ *   for query (b,t) at absolute position pos = q_pos[b,t] and head h:
+ *     memory = [swa_kv rows of positions max(0,pos-127)..pos held in the buffer
+ *               (buffer row = position - swa_pos0[b])] ++ [kv[b, idx[b,t,e]] for e < k]
+ *     z_j = scale * <q[b,t,h,:], memory_j>,
+ *     out[b,t,h,:] = sum_j exp(z_j) memory_j / (exp(sink[h]) + sum_l exp(z_l))
+ *   The latent row is both key and value.  idx entries outside [0, N) (e.g.
+ *   the -1 padding of csa_topk) contribute nothing.
+ *   q      : [B, T, H, D] dtype;  kv : [B, N, D] dtype;  swa_kv : [B, W, D] dtype
+ *   swa_pos0 : [B] int64;  q_pos : [B, T] int64;  sink : [H] fp32 (unscaled logit)
+ *   idx    : [B, T, k] int32;  out : [B, T, H, D] dtype
+ *   dtype CSA_BF16 (tcgen05, fp32 softmax and accumulation; H <= 128,
+ *   D in {128, 256, 512}) or CSA_F32 (fp32 FMA; D multiple of 32, <= 512).
+ *   workspace : csa_attn_workspace_size(...) bytes (split-KV partials; may be
+ *               0 bytes / NULL when that size is 0).
+ */
+size_t csa_attn_workspace_size(int B, int T, int H, int D, int64_t rows_per_query, int dtype);
+int sparse_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
+                const int64_t *q_pos, const float *sink, const int32_t *idx, int k, float scale, int B, int T,
+                int H, int D, int64_t N, int dtype, void *out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * hca_attn -- HCA core attention ([HA] §5: dense MQA over every compressed
+ * summary plus the SWA rows, no indexer): as sparse_attn with the memory rows
+ * kv[b, 0 .. min(N, (pos+1)/ratio) - 1] (complete blocks only).
+ */
+int hca_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
+             const int64_t *q_pos, const float *sink, int ratio, float scale, int B, int T, int H, int D, int64_t N,
+             int dtype, void *out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * csa_poll_status -- synchronise `stream`, then return and clear the device
+ * status word (CSA_OK, or CSA_ERR_TIMEOUT if a kernel abandoned a bounded
+ * wait since the last poll).  CSA_ERR_CUDA if synchronisation fails.
+ */
+int csa_poll_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,203 @@
+"""ctypes binding of libcsa.so (the C ABI in include/csa.h), same entry-point names.
+
+Argument marshalling only: shapes and dtype codes are read off torch tensors,
+device pointers and the current CUDA stream are passed through, and a non-zero
+status raises ``CsaError``.  Every step of the computation runs in the CUDA
+kernels of libcsa.so; there is no other implementation behind these names.
+Importing this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_context_compressed_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+CSA_OK, CSA_ERR_INVALID, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA, CSA_ERR_TIMEOUT = range(5)
+CSA_F32, CSA_BF16, CSA_E4M3 = 0, 1, 2
+INDEX_HEADS, INDEX_DIM, SWA_WINDOW, MAX_TOPK = 64, 128, 128, 2048
+
+_vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+
+_SIGS = {
+    "csa_status_string": ([_i32], ctypes.c_char_p),
+    "csa_version": ([], _i32),
+    "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
+    "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
+    "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp], _i32),
+    "csa_topk_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
+    "csa_topk": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
+    "csa_attn_workspace_size": ([_i32, _i32, _i32, _i32, _i64, _i32], _sz),
+    "sparse_attn": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
+                     _vp, _vp, _sz, _vp], _i32),
+    "hca_attn": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
+                  _vp, _vp, _sz, _vp], _i32),
+    "csa_poll_status": ([_vp], _i32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {_lib.csa_status_string(status).decode()}")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != CSA_OK:
+        raise CsaError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return CSA_F32
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    if t.dtype == torch.uint8:
+        return CSA_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def csa_status_string(status: int) -> str:
+    return _lib.csa_status_string(status).decode()
+
+
+def csa_version() -> int:
+    return _lib.csa_version()
+
+
+def csa_compress(C_a, C_b=None, Z_a=None, Z_b=None, prev_Cb=None, prev_Zb=None, *, ratio=4, out=None,
+                 out_dtype=None, stream=None):
+    """Compressor.  ratio 4: C_a, C_b, Z_a, Z_b [B, L, c] (+ carry [B, 4, c]); ratio 128: C_a = C,
+    Z_a = Z, C_b = Z_b = None.  Returns out [B, L // ratio, c]."""
+    B, L, c = C_a.shape
+    if out is None:
+        out = torch.empty((B, L // ratio, c), dtype=out_dtype or C_a.dtype, device=C_a.device)
+    _check(_lib.csa_compress(_ptr(C_a), _ptr(C_b), _ptr(Z_a), _ptr(Z_b), _ptr(prev_Cb), _ptr(prev_Zb), B, L, c,
+                             ratio, _dtype_code(C_a), _dtype_code(out), _ptr(out), _stream(stream)), "csa_compress")
+    return out
+
+
+def csa_quantize_e4m3(x, codes=None, scale=None, stream=None):
+    """Per-row e4m3 quantisation of x [..., cols] -> (codes uint8 [..., cols], scale fp32 [...])."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(_lib.csa_quantize_e4m3(_ptr(x), _dtype_code(x), rows, cols, _ptr(codes), _ptr(scale),
+                                  _stream(stream)), "csa_quantize_e4m3")
+    return codes, scale
+
+
+def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=None, stream=None):
+    """Indexer scores.  qI [B, T, 64, 128] (fp32 | bf16 | uint8 e4m3 codes), w [B, T, 64] fp32,
+    kI [B, N, 128] same dtype, n_valid [B, T] int32 -> scores [B, T, N] fp32."""
+    B, T = qI.shape[0], qI.shape[1]
+    N = kI.shape[1]
+    if scores is None:
+        scores = torch.empty((B, T, N), dtype=torch.float32, device=qI.device)
+    _check(_lib.csa_index_scores(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), _dtype_code(qI),
+                                 _ptr(n_valid), B, T, N, _ptr(scores), _stream(stream)), "csa_index_scores")
+    return scores
+
+
+def csa_topk_workspace_size(B: int, T: int, N: int, k: int) -> int:
+    return int(_lib.csa_topk_workspace_size(B, T, N, k))
+
+
+def topk_workspace(B: int, T: int, N: int, k: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size csa_topk needs (the library keeps it zeroed)."""
+    n = max(16, csa_topk_workspace_size(B, T, N, k))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def csa_topk(scores, n_valid, k: int, *, idx=None, workspace=None, stream=None):
+    """Top-k indices per row of scores [B, T, N] -> idx [B, T, k] int32 (ascending, -1 padded)."""
+    B, T, N = scores.shape
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
+    if workspace is None:
+        workspace = topk_workspace(B, T, N, k, scores.device)
+    _check(_lib.csa_topk(_ptr(scores), _ptr(n_valid), B, T, N, k, _ptr(idx), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream)), "csa_topk")
+    return idx
+
+
+def csa_attn_workspace_size(B: int, T: int, H: int, D: int, rows_per_query: int, dtype: int = CSA_BF16) -> int:
+    return int(_lib.csa_attn_workspace_size(B, T, H, D, rows_per_query, dtype))
+
+
+def attn_workspace(B, T, H, D, rows_per_query, dtype=CSA_BF16, device="cuda"):
+    n = max(16, csa_attn_workspace_size(B, T, H, D, rows_per_query, dtype))
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale: float, *, out=None, workspace=None,
+                stream=None):
+    """CSA core attention.  q [B,T,H,D], kv [B,N,D], swa_kv [B,W,D], swa_pos0 [B] int64, q_pos [B,T] int64,
+    sink [H] fp32, idx [B,T,k] int32 -> out [B,T,H,D]."""
+    B, T, H, D = q.shape
+    N, W, k = kv.shape[1], swa_kv.shape[1], idx.shape[2]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = attn_workspace(B, T, H, D, min(W, SWA_WINDOW) + k, dt, q.device)
+    _check(_lib.sparse_attn(_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), _ptr(idx),
+                            k, float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream)), "sparse_attn")
+    return out
+
+
+def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int = 128, out=None, workspace=None,
+             stream=None):
+    """HCA core attention: dense over kv[b, :min(N, (pos+1)//ratio)] plus the SWA rows."""
+    B, T, H, D = q.shape
+    N, W = kv.shape[1], swa_kv.shape[1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = attn_workspace(B, T, H, D, min(W, SWA_WINDOW) + N, dt, q.device)
+    _check(_lib.hca_attn(_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), ratio,
+                         float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream)), "hca_attn")
+    return out
+
+
+def csa_poll_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(_lib.csa_poll_status(_stream(stream)))
+
+
+def n_valid_for(q_pos: torch.Tensor, ratio: int, N: int) -> torch.Tensor:
+    """Visible complete entries per query, min(N, (pos + 1) // ratio), as int32 (host-side helper)."""
+    return torch.clamp((q_pos.to(torch.int64) + 1) // ratio, max=N).to(torch.int32)

@@ -1,0 +1,497 @@
+// attn.cuh -- shared-KV multi-query attention with an attention sink over the
+// memory [SWA rows ; compressed rows]:
+//   z_j = scale * <q_h, row_j>,  p_j = exp(z_j) / (exp(sink_h) + sum_l exp(z_l)),
+//   o_h = sum_j p_j row_j            (the latent row is both key and value)
+// "DeepSeek-V4 混合注意力：从压缩记忆到百万上下文" §4.2 (Shared-KV MQA over the
+// selected entries), §6 (128-token SWA branch, sink probability), §7 (memory =
+// concat(local_kv, selected_kv), one softmax); "解密DeepSeek-V4-Flash-NVFP4的混合
+// 注意力机制…" (sparse_attn(q, kv, attn_sink, topk_idxs, softmax_scale), gather by
+// index + online softmax).
+//
+// Row list of query (b, t) at absolute position pos:
+//   SWA rows   : positions max(0, pos-127)..pos that lie inside the SWA buffer
+//                (buffer row = position - swa_pos0), in position order;
+//   memory rows: sparse_attn -> kv[idx[b,t,e]] for e < k (an index outside
+//                [0, N) contributes nothing); hca_attn -> kv[e] for
+//                e < min(N, (pos+1)/ratio) (complete blocks only).
+//
+// attn_tc_kernel (bf16): one CTA per (split, D-slice, query).  The query block
+// (H heads padded to the M = 128 operand, all D dims) stays in shared memory;
+// KV rows are gathered with 16-byte cp.async into 128-byte-swizzled K-major
+// tiles of R rows; S = Q K^T (tcgen05, fp32 in TMEM, double buffered); four
+// softmax warps (one head per thread) run the online softmax in the log2
+// domain, writing P (bf16) to shared memory; O += P V (tcgen05; the same KV
+// tile read as an MN-major operand, restricted to this CTA's D-slice of width
+// DH <= 256) accumulates in TMEM.  O is rescaled only when a tile's maximum
+// exceeds the running reference by more than 2^8, so exponentials stay <= 256.
+// With several splits the CTA writes (O, m, l) partials that attn_combine_kernel
+// merges together with the sink.
+//
+// attn_f32_kernel: fp32 SIMT (one warp per head), exact online softmax.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace csa {
+
+constexpr int kSwaWindow = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct AttnParams {
+  const void* q;          // [B, T, H, D]
+  const void* kv;         // [B, N, D]
+  const void* swa;        // [B, W, D]
+  const int64_t* swa_pos0;  // [B]
+  const int64_t* q_pos;   // [B, T]
+  const float* sink;      // [H]
+  const int32_t* idx;     // [B, T, k] (sparse) or null (hca)
+  void* out;              // [B, T, H, D]
+  float* ws_o;            // [nsplit, B*T, H, D] partial O (nsplit > 1)
+  float* ws_ml;           // [nsplit, B*T, H, 2] partial (m, l), log2 domain
+  float scale;
+  int B, T, H, D, W, k, ratio, nsplit;
+  int sparse;             // 1: memory rows from idx (sparse_attn); 0: dense prefix (hca_attn)
+  int64_t N;
+};
+
+struct RowList {
+  int64_t swa_row0;   // first SWA buffer row
+  int n_swa;          // SWA rows
+  int n_mem;          // memory rows (k for sparse, visible entries for hca)
+};
+
+__device__ __forceinline__ RowList make_row_list(const AttnParams& p, int b, int t) {
+  RowList rl;
+  const int64_t pos = p.q_pos[(int64_t)b * p.T + t];
+  const int64_t s0 = p.swa_pos0[b];
+  int64_t lo = pos - (kSwaWindow - 1);
+  if (lo < 0) lo = 0;
+  if (lo < s0) lo = s0;
+  int64_t hi = pos;
+  if (hi > s0 + p.W - 1) hi = s0 + p.W - 1;
+  rl.n_swa = hi >= lo ? (int)(hi - lo + 1) : 0;
+  rl.swa_row0 = lo - s0;
+  if (p.sparse) {
+    rl.n_mem = p.k;
+  } else {
+    int64_t nv = pos >= 0 ? (pos + 1) / p.ratio : 0;
+    if (nv > p.N) nv = p.N;
+    rl.n_mem = (int)nv;
+  }
+  return rl;
+}
+
+// Row r of the list -> element offset of its first value, or -1 if it contributes nothing.
+__device__ __forceinline__ int64_t row_offset(const AttnParams& p, const RowList& rl, int b, int t, int r,
+                                              bool* is_swa) {
+  if (r < rl.n_swa) {
+    *is_swa = true;
+    return ((int64_t)b * p.W + rl.swa_row0 + r) * p.D;
+  }
+  *is_swa = false;
+  const int e = r - rl.n_swa;
+  int64_t i;
+  if (p.sparse) {
+    i = p.idx[((int64_t)b * p.T + t) * p.k + e];
+    if (i < 0 || i >= p.N) return -1;
+  } else {
+    i = e;
+  }
+  return ((int64_t)b * p.N + i) * p.D;
+}
+
+// ------------------------------------------------------------------ fp32 SIMT
+// One warp per (b, t, h); lane holds D/32 dims of q and o.  The sink enters as a
+// row with logit sink_h and value 0 (initial state m = sink, l = 1, o = 0).
+template <int DPL>  // dims per lane
+__global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
+  const int h = blockIdx.x * 4 + warp_id();
+  const int t = blockIdx.y, b = blockIdx.z;
+  if (h >= p.H) return;
+  const float* q = static_cast<const float*>(p.q) + (((int64_t)b * p.T + t) * p.H + h) * p.D;
+  const float* kv = static_cast<const float*>(p.kv);
+  const float* swa = static_cast<const float*>(p.swa);
+  float qv[DPL], o[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) {
+    qv[j] = q[lane_id() + 32 * j];
+    o[j] = 0.f;
+  }
+  float m = p.sink[h], l = 1.f;
+  const RowList rl = make_row_list(p, b, t);
+  const int n = rl.n_swa + rl.n_mem;
+  for (int r = 0; r < n; ++r) {
+    bool sw;
+    const int64_t off = row_offset(p, rl, b, t, r, &sw);
+    if (off < 0) continue;
+    const float* row = (sw ? swa : kv) + off;
+    float rv[DPL];
+    float dot = 0.f;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      rv[j] = row[lane_id() + 32 * j];
+      dot = fmaf(qv[j], rv[j], dot);
+    }
+#pragma unroll
+    for (int off2 = 16; off2 > 0; off2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off2);
+    const float z = dot * p.scale;
+    const float mn = fmaxf(m, z);
+    const float c = expf(m - mn), e = expf(z - mn);
+    l = l * c + e;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) o[j] = fmaf(o[j], c, e * rv[j]);
+    m = mn;
+  }
+  float* out = static_cast<float*>(p.out) + (((int64_t)b * p.T + t) * p.H + h) * p.D;
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) out[lane_id() + 32 * j] = o[j] * inv;
+}
+
+// ------------------------------------------------------------------ tcgen05 bf16
+template <int D>
+struct AttnCfg {
+  static constexpr int R = (D >= 512) ? 32 : 64;           // rows per KV tile
+  static constexpr int DH = (D > 256) ? 256 : D;           // D-slice per CTA
+  static constexpr int NDH = D / DH;
+  static constexpr int kAtoms = D / 64;                    // 128-byte atoms per row
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = R * D * 2;
+  static constexpr int kPRowBytes = R * 2;                 // 64 (SW64) or 128 (SW128)
+  static constexpr int kPBytes = 128 * kPRowBytes;
+  static constexpr uint32_t kPLayout = (kPRowBytes == 128) ? kLayoutSW128 : kLayoutSW64;
+  static constexpr int kPSBO = 8 * kPRowBytes;
+  static constexpr int kTmemCols = (DH + 2 * R) <= 256 ? 256 : 512;  // O slice + two S buffers
+  static constexpr int kSCol0 = DH;                        // S buffers after O
+  static constexpr int kThreads = 288;                     // 4 softmax + 4 loader + 1 MMA warps
+  static constexpr int kSmem = kQBytes + 2 * kKVBytes + 2 * kPBytes + 1024 + 256;
+};
+
+// Byte offset of 16-byte chunk c of row r in a K-major tile with 128-byte
+// swizzle, whose 64-element atoms are `rows` rows tall.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
+  return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const AttnParams p) {
+  using Cfg = AttnCfg<D>;
+  constexpr int R = Cfg::R, DH = Cfg::DH;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem;
+  uint8_t* kv_s = q_s + Cfg::kQBytes;                       // [2][kKVBytes]
+  uint8_t* p_s = kv_s + 2 * Cfg::kKVBytes;                  // [2][kPBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Cfg::kPBytes);
+  uint64_t* full = bars;        // [2] KV stage loaded (128 cp.async arrivals + 1 mask arrival)
+  uint64_t* empty = bars + 2;   // [2] KV stage consumed by PV
+  uint64_t* sfull = bars + 4;   // [2] S ready
+  uint64_t* sfree = bars + 6;   // [2] S read by softmax
+  uint64_t* pfull = bars + 8;   // [2] P written
+  uint64_t* pdone = bars + 10;  // [2] PV done (P buffer free, O consistent)
+  uint64_t* qfull = bars + 12;
+  uint64_t* odone = bars + 13;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* mask_s = bars + 16;  // [2] validity of the tile's rows
+
+  const int qi = blockIdx.z;                 // b * T + t
+  const int b = qi / p.T, t = qi % p.T;
+  const int dh = blockIdx.y;
+  const int split = blockIdx.x;
+  const RowList rl = make_row_list(p, b, t);
+  const int n_rows = rl.n_swa + rl.n_mem;
+  const int n_tiles_all = (n_rows + R - 1) / R;
+  const int tps = (n_tiles_all + p.nsplit - 1) / p.nsplit;
+  const int j0 = split * tps;
+  const int j1 = min(n_tiles_all, j0 + tps);
+  const int nt = j1 > j0 ? j1 - j0 : 0;      // tiles of this CTA
+  const int warp = warp_id();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 128 + 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sfree[i], 4);
+      mbar_init(&pfull[i], 4);
+      mbar_init(&pdone[i], 1);
+    }
+    mbar_init(qfull, 128);
+    mbar_init(odone, 1);
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_holder, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ loaders (128 threads)
+    const int lt = threadIdx.x - 128;
+    if (nt > 0) {
+      const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q) + (int64_t)qi * p.H * D;
+      for (int c = lt; c < 128 * (D / 8); c += 128) {
+        const int r = c / (D / 8), ch = c % (D / 8);
+        uint8_t* dst = q_s + sw128_off(r, ch, 128);
+        if (r < p.H) cp_async_16(dst, qg + (int64_t)r * D + ch * 8);
+        else st_shared_zero16(dst);
+      }
+      fence_proxy_async_smem();
+      cp_async_arrive_noinc(qfull);
+      const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(p.kv);
+      const __nv_bfloat16* swa = static_cast<const __nv_bfloat16*>(p.swa);
+      constexpr int CPR = D / 8;                 // 16-byte chunks per row
+      for (int jj = 0; jj < nt; ++jj) {
+        const int j = j0 + jj;
+        const int s = jj & 1;
+        if (!mbar_wait(&empty[s], ((jj >> 1) & 1) ^ 1)) break;
+        uint8_t* tile = kv_s + s * Cfg::kKVBytes;
+        for (int c = lt; c < R * CPR; c += 128) {
+          const int r = c / CPR, ch = c % CPR;
+          const int rg = j * R + r;
+          bool sw = false;
+          const int64_t off = rg < n_rows ? row_offset(p, rl, b, t, rg, &sw) : -1;
+          uint8_t* dst = tile + sw128_off(r, ch, R);
+          if (off >= 0) cp_async_16(dst, (sw ? swa : kv) + off + ch * 8);
+          else st_shared_zero16(dst);                 // finite filler for rows that do not contribute
+        }
+        fence_proxy_async_smem();
+        cp_async_arrive_noinc(&full[s]);
+        if (lt == 0) {
+          // which rows of the tile contribute (read by the softmax warps after full[s])
+          uint64_t valid = 0;
+          for (int r = 0; r < R; ++r) {
+            const int rg = j * R + r;
+            bool sw;
+            if (rg < n_rows && row_offset(p, rl, b, t, rg, &sw) >= 0) valid |= 1ull << r;
+          }
+          mask_s[s] = valid;
+          mbar_arrive(&full[s]);
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one() && nt > 0) {
+      const uint32_t idesc_s = make_idesc(128, R, 1, 0, 0);
+      const uint32_t idesc_o = make_idesc(128, DH, 1, 0, 1);
+      const uint32_t qb = smem_u32(q_s);
+      bool ok = mbar_wait(qfull, 0);
+      fence_proxy_async_smem();
+      tc_fence_after();
+      auto issue_s = [&](int jj) -> bool {
+        const int s = jj & 1;
+        const uint32_t ph = (jj >> 1) & 1;
+        if (!mbar_wait(&full[s], ph)) return false;
+        if (!mbar_wait(&sfree[s], ph ^ 1)) return false;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t kb = smem_u32(kv_s + s * Cfg::kKVBytes);
+        const uint32_t d = tmem + Cfg::kSCol0 + s * R;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int atom = kk >> 2, inner = (kk & 3) * 32;
+          const uint64_t ad = smem_desc(qb + atom * 128 * 128 + inner, 16, 1024, kLayoutSW128);
+          const uint64_t bd = smem_desc(kb + atom * R * 128 + inner, 16, 1024, kLayoutSW128);
+          mma_bf16(d, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sfull[s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int jj = 0; ok && jj < nt; ++jj) {
+        if (jj + 1 < nt && !issue_s(jj + 1)) { ok = false; break; }
+        const int s = jj & 1;
+        if (!mbar_wait(&pfull[s], (jj >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t pb = smem_u32(p_s + s * Cfg::kPBytes);
+        const uint32_t vb = smem_u32(kv_s + s * Cfg::kKVBytes) + dh * (DH / 64) * R * 128;
+#pragma unroll
+        for (int kk = 0; kk < R / 16; ++kk) {
+          const uint64_t ad = smem_desc(pb + kk * 32, 16, Cfg::kPSBO, Cfg::kPLayout);
+          const uint64_t bd = smem_desc(vb + kk * 2048, R * 128, 1024, kLayoutSW128);
+          mma_bf16(tmem, ad, bd, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&pdone[s]);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(odone);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue (warps 0..3)
+    const int h = threadIdx.x;                 // TMEM lane = head row
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sinkL = (h < p.H) ? p.sink[h] * kLog2e : 0.f;
+    const float zs = p.scale * kLog2e;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < nt; ++jj) {
+      const int s = jj & 1;
+      const uint32_t ph = (jj >> 1) & 1;
+      if (!mbar_wait(&full[s], ph) || !mbar_wait(&sfull[s], ph)) { ok = false; break; }
+      tc_fence_after();
+      const uint64_t valid = mask_s[s];
+      float z[R];
+      tmem_ld32(tmem + lane_base + Cfg::kSCol0 + s * R, z);
+      if constexpr (R == 64) tmem_ld32(tmem + lane_base + Cfg::kSCol0 + s * R + 32, z + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&sfree[s]);
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < R; ++c) {
+        z[c] = ((valid >> c) & 1) ? z[c] * zs : -INFINITY;
+        mt = fmaxf(mt, z[c]);
+      }
+      // P buffer s is free once PV of tile jj-2 completed
+      if (!mbar_wait(&pdone[s], ph ^ 1)) { ok = false; break; }
+      if (mt > m_used + 8.f) {
+        const float m_new = mt;
+        if (m_used != -INFINITY && jj > 0) {
+          // O must be consistent: PV of tile jj-1 completed
+          const int ps = (jj - 1) & 1;
+          if (!mbar_wait(&pdone[ps], ((jj - 1) >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const float f = exp2f(m_used - m_new);
+          for (int c0 = 0; c0 < DH; c0 += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= f;
+            tmem_st32(tmem + lane_base + c0, o);
+          }
+          tmem_wait_st();
+          l *= f;
+        }
+        m_used = m_new;
+      }
+      float psum = 0.f;
+      uint32_t packed[R / 2];
+#pragma unroll
+      for (int c = 0; c < R; c += 2) {
+        const float p0 = (m_used == -INFINITY) ? 0.f : exp2f(z[c] - m_used);
+        const float p1 = (m_used == -INFINITY) ? 0.f : exp2f(z[c + 1] - m_used);
+        psum += p0 + p1;
+        __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
+        packed[c / 2] = *reinterpret_cast<uint32_t*>(&v);
+      }
+      l += psum;
+      uint8_t* prow = p_s + s * Cfg::kPBytes + h * Cfg::kPRowBytes;
+#pragma unroll
+      for (int c = 0; c < R / 8; ++c) {
+        const int phys = (R == 64) ? (c ^ (h & 7)) : (c ^ ((h >> 1) & 3));
+        *reinterpret_cast<uint4*>(prow + phys * 16) =
+            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&pfull[s]);
+    }
+    // ---- epilogue
+    const bool have_o = ok && nt > 0 && mbar_wait(odone, 0);
+    tc_fence_after();
+    const int64_t orow = ((int64_t)qi * p.H + h) * D + dh * DH;
+    if (p.nsplit == 1) {
+      const float M = fmaxf(m_used, sinkL);
+      const float fo = (m_used == -INFINITY) ? 0.f : exp2f(m_used - M);
+      const float den = l * fo + exp2f(sinkL - M);
+      const float g = fo / den;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float o[32];
+        if (have_o) {
+          tmem_ld32(tmem + lane_base + c0, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        }
+        if (h < p.H) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 u;
+            __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hv[e] = __floats2bfloat162_rn(o[c + 2 * e] * g, o[c + 2 * e + 1] * g);
+            *reinterpret_cast<uint4*>(out + orow + c0 + c) = u;
+          }
+        }
+      }
+    } else {
+      float* wo = p.ws_o + (int64_t)split * p.B * p.T * p.H * D;
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float o[32];
+        if (have_o) {
+          tmem_ld32(tmem + lane_base + c0, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        }
+        if (h < p.H) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(wo + orow + c0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        }
+      }
+      if (h < p.H && dh == 0) {
+        float* ml = p.ws_ml + (((int64_t)split * p.B * p.T + qi) * p.H + h) * 2;
+        ml[0] = have_o ? m_used : -INFINITY;
+        ml[1] = have_o ? l : 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// Merge split partials with the sink: M = max(sink, m_s); den = e^(sink-M) +
+// sum_s l_s e^(m_s-M); o = sum_s O_s e^(m_s-M) / den  (log2 domain).  One
+// thread per (query, head, 8 dims).
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
+  const int64_t groups = (int64_t)p.B * p.T * p.H * (p.D / 8);
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= groups) return;
+  const int d0 = (int)(g % (p.D / 8)) * 8;
+  const int64_t qh = g / (p.D / 8);         // (b*T + t) * H + h
+  const int h = (int)(qh % p.H);
+  const float sinkL = p.sink[h] * kLog2e;
+  const int64_t stride_ml = (int64_t)p.B * p.T * p.H * 2;
+  const int64_t stride_o = (int64_t)p.B * p.T * p.H * p.D;
+  float M = sinkL;
+  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.ws_ml[s * stride_ml + qh * 2]);
+  float den = exp2f(sinkL - M);
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int s = 0; s < p.nsplit; ++s) {
+    const float ms = p.ws_ml[s * stride_ml + qh * 2];
+    if (ms == -INFINITY) continue;
+    const float f = exp2f(ms - M);
+    den = fmaf(p.ws_ml[s * stride_ml + qh * 2 + 1], f, den);
+    const float4* src = reinterpret_cast<const float4*>(p.ws_o + s * stride_o + qh * p.D + d0);
+    const float4 a = src[0], c = src[1];
+    acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
+    acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
+    acc[4] = fmaf(c.x, f, acc[4]); acc[5] = fmaf(c.y, f, acc[5]);
+    acc[6] = fmaf(c.z, f, acc[6]); acc[7] = fmaf(c.w, f, acc[7]);
+  }
+  const float inv = 1.f / den;
+  uint4 u;
+  __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) hv[e] = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + qh * p.D + d0) = u;
+}
+
+}  // namespace csa

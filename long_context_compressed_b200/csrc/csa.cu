@@ -1,0 +1,392 @@
+// csa.cu -- host side of the C ABI declared in include/csa.h: argument
+// validation, TMA tensor-map encoding, launch configuration.  All kernels
+// live in the *.cuh files of this directory and are compiled into this one
+// translation unit (one copy of the device status word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/csa.h"
+#include "attn.cuh"
+#include "compress.cuh"
+#include "index.cuh"
+#include "quantize.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using csa::AttnCfg;
+using csa::AttnParams;
+using csa::IndexParams;
+
+constexpr int kMaxDev = 64;
+constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per CTA on sm_100
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int sm_count() {
+  static int cache[kMaxDev] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over [dim2][dim1][inner] with a 128-byte-swizzled box {box0, box1, 1}.
+bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t dim1,
+              uint64_t dim2, uint32_t box0, uint32_t box1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, dim1, dim2};
+  cuuint64_t strides[2] = {inner * esize, inner * dim1 * esize};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ attention split policy
+template <int D>
+int attn_rows_per_tile() { return AttnCfg<D>::R; }
+
+int attn_ndh(int D) { return D > 256 ? D / 256 : 1; }
+
+int attn_nsplit(int B, int T, int D, int64_t max_rows) {
+  const int64_t items = (int64_t)B * T * attn_ndh(D);
+  const int sms = sm_count();
+  if (items <= 0 || items >= 2 * sms) return 1;
+  const int R = D >= 512 ? 32 : 64;
+  const int64_t tiles = (max_rows + R - 1) / R;
+  const int64_t want = (2 * sms + items - 1) / items;
+  const int64_t cap = std::max<int64_t>(1, tiles / 4);
+  return (int)std::max<int64_t>(1, std::min(want, cap));
+}
+
+size_t attn_ws_bytes(int B, int T, int H, int D, int64_t max_rows, int dtype) {
+  if (dtype != CSA_BF16) return 0;
+  const int ns = attn_nsplit(B, T, D, max_rows);
+  if (ns <= 1) return 0;
+  const size_t per = (size_t)B * T * H;
+  return (size_t)ns * per * ((size_t)D + 2) * sizeof(float) + 256;
+}
+
+int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_rows, cudaStream_t st) {
+  if (p.B == 0 || p.T == 0) return CSA_OK;
+  if (dtype == CSA_F32) {
+    dim3 grid((p.H + 3) / 4, p.T, p.B);
+    switch (p.D) {
+      case 32: csa::attn_f32_kernel<1><<<grid, 128, 0, st>>>(p); break;
+      case 64: csa::attn_f32_kernel<2><<<grid, 128, 0, st>>>(p); break;
+      case 128: csa::attn_f32_kernel<4><<<grid, 128, 0, st>>>(p); break;
+      case 256: csa::attn_f32_kernel<8><<<grid, 128, 0, st>>>(p); break;
+      case 512: csa::attn_f32_kernel<16><<<grid, 128, 0, st>>>(p); break;
+      default: return CSA_ERR_UNSUPPORTED;
+    }
+    return launch_status();
+  }
+  p.nsplit = attn_nsplit(p.B, p.T, p.D, max_rows);
+  const size_t need = attn_ws_bytes(p.B, p.T, p.H, p.D, max_rows, dtype);
+  if (need > 0) {
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return CSA_ERR_INVALID;
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_ml = p.ws_o + (size_t)p.nsplit * p.B * p.T * p.H * p.D;
+  }
+  dim3 grid(p.nsplit, attn_ndh(p.D), p.B * p.T);
+  switch (p.D) {
+    case 128:
+      if (!set_smem(csa::attn_tc_kernel<128>, AttnCfg<128>::kSmem)) return CSA_ERR_CUDA;
+      csa::attn_tc_kernel<128><<<grid, AttnCfg<128>::kThreads, AttnCfg<128>::kSmem, st>>>(p);
+      break;
+    case 256:
+      if (!set_smem(csa::attn_tc_kernel<256>, AttnCfg<256>::kSmem)) return CSA_ERR_CUDA;
+      csa::attn_tc_kernel<256><<<grid, AttnCfg<256>::kThreads, AttnCfg<256>::kSmem, st>>>(p);
+      break;
+    case 512:
+      if (!set_smem(csa::attn_tc_kernel<512>, AttnCfg<512>::kSmem)) return CSA_ERR_CUDA;
+      csa::attn_tc_kernel<512><<<grid, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, st>>>(p);
+      break;
+    default: return CSA_ERR_UNSUPPORTED;
+  }
+  int rc = launch_status();
+  if (rc != CSA_OK || p.nsplit == 1) return rc;
+  const int64_t groups = (int64_t)p.B * p.T * p.H * (p.D / 8);
+  csa::attn_combine_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, st>>>(p);
+  return launch_status();
+}
+
+int check_attn_common(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                      const int64_t* q_pos, const float* sink, float scale, int B, int T, int H, int D, int64_t N,
+                      int dtype, const void* out) {
+  if (B < 0 || T < 0 || H <= 0 || D <= 0 || N < 0 || W < 0) return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (!(scale == scale)) return CSA_ERR_INVALID;
+  if (B == 0 || T == 0) return CSA_OK;
+  if (!q || !out || !swa_pos0 || !q_pos || !sink) return CSA_ERR_INVALID;
+  if (N > 0 && !kv) return CSA_ERR_INVALID;
+  if (W > 0 && !swa_kv) return CSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(out) || (kv && !aligned16(kv)) || (swa_kv && !aligned16(swa_kv)))
+    return CSA_ERR_INVALID;
+  if (dtype == CSA_BF16) {
+    if (D != 128 && D != 256 && D != 512) return CSA_ERR_UNSUPPORTED;
+    if (H > 128) return CSA_ERR_UNSUPPORTED;
+  } else {
+    if (D % 32 != 0 || D > 512) return CSA_ERR_UNSUPPORTED;
+  }
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* csa_status_string(int status) {
+  switch (status) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID: return "CSA_ERR_INVALID: invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED: unsupported shape or dtype";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA: CUDA runtime or launch failure";
+    case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT: a kernel abandoned a bounded wait";
+    default: return "unknown csa status";
+  }
+}
+
+int csa_version(void) { return 100; }
+
+int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* Z_b, const void* prev_Cb,
+                 const void* prev_Zb, int B, int64_t L, int c, int ratio, int in_dtype, int out_dtype, void* out,
+                 void* stream) {
+  if (B < 0 || L < 0 || c <= 0) return CSA_ERR_INVALID;
+  if (ratio != 4 && ratio != 128) return CSA_ERR_INVALID;
+  if ((in_dtype != CSA_F32 && in_dtype != CSA_BF16) || (out_dtype != CSA_F32 && out_dtype != CSA_BF16))
+    return CSA_ERR_INVALID;
+  if ((prev_Cb == nullptr) != (prev_Zb == nullptr)) return CSA_ERR_INVALID;
+  if (ratio == 4 && c % 8 != 0) return CSA_ERR_INVALID;
+  if (ratio == 128 && (c % 128 != 0 || C_b || Z_b || prev_Cb || prev_Zb)) return CSA_ERR_INVALID;
+  const int64_t n_entries = L / ratio;
+  if (B == 0 || n_entries == 0) return CSA_OK;
+  if (!C_a || !Z_a || !out || (ratio == 4 && (!C_b || !Z_b))) return CSA_ERR_INVALID;
+  const void* ptrs[] = {C_a, C_b, Z_a, Z_b, prev_Cb, prev_Zb, out};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CSA_ERR_INVALID;
+  cudaStream_t st = as_stream(stream);
+  const bool bf_in = in_dtype == CSA_BF16, bf_out = out_dtype == CSA_BF16;
+  if (ratio == 4) {
+    const int64_t total = (int64_t)B * n_entries * (c / 8);
+    const int64_t blocks64 = (total + 255) / 256;
+    const unsigned blocks = (unsigned)std::min<int64_t>(blocks64, (int64_t)sm_count() * 16);
+#define CSA_LAUNCH_CSA(TI, TO)                                                                              \
+  csa::compress_csa_kernel<TI, TO, 4><<<blocks, 256, 0, st>>>(                                              \
+      (const TI*)C_a, (const TI*)C_b, (const TI*)Z_a, (const TI*)Z_b, (const TI*)prev_Cb, (const TI*)prev_Zb, \
+      B, L, c, (TO*)out)
+    if (bf_in && bf_out) CSA_LAUNCH_CSA(__nv_bfloat16, __nv_bfloat16);
+    else if (bf_in) CSA_LAUNCH_CSA(__nv_bfloat16, float);
+    else if (bf_out) CSA_LAUNCH_CSA(float, __nv_bfloat16);
+    else CSA_LAUNCH_CSA(float, float);
+#undef CSA_LAUNCH_CSA
+  } else {
+    if (n_entries > 65535 || B > 65535) return CSA_ERR_UNSUPPORTED;
+    const int G = std::min(c / 8, 64);
+    dim3 grid((unsigned)(c / 8 / G), (unsigned)n_entries, (unsigned)B);
+#define CSA_LAUNCH_HCA(TI, TO) \
+  csa::compress_hca_kernel<TI, TO><<<grid, 256, 0, st>>>((const TI*)C_a, (const TI*)Z_a, B, L, c, (TO*)out)
+    if (bf_in && bf_out) CSA_LAUNCH_HCA(__nv_bfloat16, __nv_bfloat16);
+    else if (bf_in) CSA_LAUNCH_HCA(__nv_bfloat16, float);
+    else if (bf_out) CSA_LAUNCH_HCA(float, __nv_bfloat16);
+    else CSA_LAUNCH_HCA(float, float);
+#undef CSA_LAUNCH_HCA
+  }
+  return launch_status();
+}
+
+int csa_quantize_e4m3(const void* x, int x_dtype, int64_t rows, int cols, uint8_t* codes, float* scale,
+                      void* stream) {
+  if (rows < 0 || cols <= 0) return CSA_ERR_INVALID;
+  if (x_dtype != CSA_F32 && x_dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (rows == 0) return CSA_OK;
+  if (!x || !codes || !scale) return CSA_ERR_INVALID;
+  const int64_t blocks64 = (rows + 7) / 8;
+  const unsigned blocks = (unsigned)std::min<int64_t>(blocks64, (int64_t)sm_count() * 32);
+  cudaStream_t st = as_stream(stream);
+  if (x_dtype == CSA_BF16)
+    csa::quantize_e4m3_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)x, rows, cols, codes, scale);
+  else
+    csa::quantize_e4m3_kernel<float><<<blocks, 256, 0, st>>>((const float*)x, rows, cols, codes, scale);
+  return launch_status();
+}
+
+int csa_index_scores(const void* qI, const float* q_scale, const float* w, const void* kI, const float* k_scale,
+                     int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* stream) {
+  if (B < 0 || T < 0 || N < 0) return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3) return CSA_ERR_INVALID;
+  if (B == 0 || T == 0 || N == 0) return CSA_OK;
+  if (!qI || !w || !kI || !n_valid || !scores) return CSA_ERR_INVALID;
+  if (dtype == CSA_E4M3 && (!q_scale || !k_scale)) return CSA_ERR_INVALID;
+  if (!aligned16(qI) || !aligned16(kI)) return CSA_ERR_INVALID;
+  if (N >= (int64_t(1) << 31) || (int64_t)T * csa::kIdxHeads >= (int64_t(1) << 31) || B > 65535)
+    return CSA_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  if (dtype == CSA_F32) {
+    if (T > 65535) return CSA_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)((N + 63) / 64), (unsigned)T, (unsigned)B);
+    if (!set_smem(csa::index_f32_kernel, csa::kIdxF32Smem)) return CSA_ERR_CUDA;
+    csa::index_f32_kernel<<<grid, 256, csa::kIdxF32Smem, st>>>((const float*)qI, w, (const float*)kI, n_valid, T,
+                                                               N, scores);
+    return launch_status();
+  }
+  const bool fp8 = dtype == CSA_E4M3;
+  IndexParams p;
+  p.w = w;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.n_valid = n_valid;
+  p.scores = scores;
+  p.B = B;
+  p.T = T;
+  p.N = N;
+  p.TQ = T >= 4 ? 4 : (T >= 2 ? 2 : 1);
+  const int key_bytes = fp8 ? csa::IndexCfg<true>::kKeyBytes : csa::IndexCfg<false>::kKeyBytes;
+  const int qrow = fp8 ? 128 : 256;
+  const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
+  const int fixed = 1024 + q_bytes + 1024 * p.TQ + 8 * 8;
+  p.stages = std::min(12, (kSmemLimit - fixed) / (key_bytes + 16));
+  if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
+  const int smem = fixed + p.stages * (key_bytes + 16);
+  CUtensorMap kmap, qmap;
+  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int es = fp8 ? 1 : 2;
+  const uint32_t box0 = fp8 ? 128 : 64;
+  if (!make_map(&kmap, kI, dt, es, csa::kIdxDim, (uint64_t)N, (uint64_t)B, box0, csa::kIdxTileKeys) ||
+      !make_map(&qmap, qI, dt, es, csa::kIdxDim, (uint64_t)T * csa::kIdxHeads, (uint64_t)B, box0,
+                (uint32_t)(p.TQ * csa::kIdxHeads)))
+    return CSA_ERR_CUDA;
+  const int QG = (T + p.TQ - 1) / p.TQ;
+  const int64_t items = (int64_t)B * QG * ((N + csa::kIdxTileKeys - 1) / csa::kIdxTileKeys);
+  const unsigned grid = (unsigned)std::min<int64_t>(items, sm_count());
+  if (fp8) {
+    if (!set_smem(csa::index_tc_kernel<true>, smem)) return CSA_ERR_CUDA;
+    csa::index_tc_kernel<true><<<grid, 192, smem, st>>>(kmap, qmap, p);
+  } else {
+    if (!set_smem(csa::index_tc_kernel<false>, smem)) return CSA_ERR_CUDA;
+    csa::index_tc_kernel<false><<<grid, 192, smem, st>>>(kmap, qmap, p);
+  }
+  return launch_status();
+}
+
+static bool topk_long_path(int B, int T, int64_t N) {
+  const int64_t rows = (int64_t)B * T;
+  return N > csa::kRowSmemMax || (rows < 74 && N >= 4 * csa::kChunk);
+}
+
+size_t csa_topk_workspace_size(int B, int T, int64_t N, int k) {
+  (void)k;
+  if (B <= 0 || T <= 0 || N <= 0) return 0;
+  if (!topk_long_path(B, T, N)) return 0;
+  return (size_t)B * T * (size_t)csa::TopkWs::row_bytes(N);
+}
+
+int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t N, int k, int32_t* idx,
+             void* workspace, size_t ws_bytes, void* stream) {
+  if (B < 0 || T < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (N > (int64_t(1) << 20)) return CSA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return CSA_OK;
+  if (!idx || !n_valid || (N > 0 && !scores)) return CSA_ERR_INVALID;
+  const int64_t rows = (int64_t)B * T;
+  if (rows > 65535 && topk_long_path(B, T, N)) return CSA_ERR_UNSUPPORTED;
+  if (rows > (int64_t(1) << 31) - 1) return CSA_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  if (!topk_long_path(B, T, N)) {
+    const int smem = (int)std::max<int64_t>(4, std::min<int64_t>(N, csa::kRowSmemMax) * 4);
+    if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
+    csa::topk_row_kernel<<<(unsigned)rows, 1024, smem, st>>>(scores, n_valid, N, k, idx);
+    return launch_status();
+  }
+  const size_t need = csa_topk_workspace_size(B, T, N, k);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSA_ERR_INVALID;
+  dim3 grid((unsigned)((N + csa::kChunk - 1) / csa::kChunk), (unsigned)rows);
+  csa::topk_hist_kernel<<<grid, 512, 0, st>>>(scores, n_valid, N, k, static_cast<uint8_t*>(workspace));
+  int rc = launch_status();
+  if (rc != CSA_OK) return rc;
+  csa::topk_gather_select_kernel<<<grid, 1024, 0, st>>>(scores, n_valid, N, k, idx,
+                                                        static_cast<uint8_t*>(workspace));
+  return launch_status();
+}
+
+size_t csa_attn_workspace_size(int B, int T, int H, int D, int64_t rows_per_query, int dtype) {
+  if (B <= 0 || T <= 0 || H <= 0 || D <= 0 || rows_per_query < 0) return 0;
+  return attn_ws_bytes(B, T, H, D, rows_per_query, dtype);
+}
+
+int sparse_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                const int64_t* q_pos, const float* sink, const int32_t* idx, int k, float scale, int B, int T,
+                int H, int D, int64_t N, int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_attn_common(q, kv, swa_kv, swa_pos0, W, q_pos, sink, scale, B, T, H, D, N, dtype, out);
+  if (rc != CSA_OK || B == 0 || T == 0) return rc;
+  if (k < 0 || (k > 0 && !idx)) return CSA_ERR_INVALID;
+  AttnParams p{};
+  p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
+  p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale;
+  p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = k; p.ratio = 1; p.N = N; p.nsplit = 1;
+  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k;
+  return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
+}
+
+int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+             const int64_t* q_pos, const float* sink, int ratio, float scale, int B, int T, int H, int D, int64_t N,
+             int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_attn_common(q, kv, swa_kv, swa_pos0, W, q_pos, sink, scale, B, T, H, D, N, dtype, out);
+  if (rc != CSA_OK || B == 0 || T == 0) return rc;
+  if (ratio < 1) return CSA_ERR_INVALID;
+  AttnParams p{};
+  p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
+  p.idx = nullptr; p.sparse = 0; p.out = out; p.scale = scale;
+  p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = 0; p.ratio = ratio; p.N = N; p.nsplit = 1;
+  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + N;
+  return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
+}
+
+int csa_poll_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, csa::g_status, sizeof(int)) != cudaSuccess) return CSA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(csa::g_status, &zero, sizeof(int)) != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

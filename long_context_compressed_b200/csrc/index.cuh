@@ -1,0 +1,328 @@
+// index.cuh -- Lightning Indexer scores
+//   s[b,t,i] = sum_h w[b,t,h] * ReLU(<qI[b,t,h,:], kI[b,i,:]>)   for i < n_valid[b,t]
+//   s[b,t,i] = -inf                                                  for n_valid[b,t] <= i < N
+// ("DeepSeek-V4 混合注意力：从压缩记忆到百万上下文" §4.2; 64 index heads of
+// 128 dims, keys shared by the heads, no 1/sqrt(d) factor).
+//
+// index_tc_kernel: a genuine dense contraction on the 5th-generation tensor
+// cores.  Keys are the M = 128 operand (one tile = 128 keys x 128 dims), the
+// TQ queries x 64 heads of a query group are the N = 64*TQ operand, K = 128.
+// Both are staged by TMA (128-byte swizzle, K-major) into shared memory;
+// one elected thread issues tcgen05.mma into a double-buffered fp32 TMEM
+// accumulator; four epilogue warps read their 32 TMEM lanes (one key per
+// thread), apply ReLU and the head weights, reduce over the 64 heads and store
+// one fp32 score per (query, key).  Persistent: one CTA per SM walks a
+// contiguous range of (sequence, query group, key tile) work items so that
+// the key stream of each SM is sequential.
+//   bf16 : kind::f16, fp32 accumulate.
+//   e4m3 : kind::f8f6f4 with a per-key scale ks[b,i] and a per-(query, head)
+//          scale qs[b,t,h]; both are positive so they commute with ReLU:
+//          s = ks * sum_h (w * qs)_h * ReLU(<q8, k8>).
+//
+// index_f32_kernel: fp32 SIMT path (FMA), used for fp32 inputs.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace csa {
+
+constexpr int kIdxHeads = 64;
+constexpr int kIdxDim = 128;
+constexpr int kIdxTileKeys = 128;
+
+struct IndexParams {
+  const float* w;        // [B, T, 64]
+  const float* q_scale;  // [B, T, 64] or null (bf16)
+  const float* k_scale;  // [B, N] or null (bf16)
+  const int32_t* n_valid;  // [B, T]
+  float* scores;         // [B, T, N]
+  int B, T;
+  int64_t N;
+  int TQ;                // queries per group (1, 2 or 4)
+  int stages;            // key pipeline depth
+};
+
+template <bool FP8>
+struct IndexCfg {
+  static constexpr int kKeyBytes = kIdxTileKeys * kIdxDim * (FP8 ? 1 : 2);  // one key tile
+  static constexpr int kQRowBytes = kIdxDim * (FP8 ? 1 : 2);               // one (t, h) row
+  static constexpr int kAtoms = FP8 ? 1 : 2;                                // 128-byte K atoms per row
+  static constexpr int kKInstr = FP8 ? 32 : 16;                             // K per MMA instruction
+  static constexpr int kKSteps = kIdxDim / kKInstr;
+};
+
+// Work item w -> (b, query group, key tile), ordered with the key tile fastest.
+struct IndexItem {
+  int b, qg;
+  int64_t kt;
+};
+__device__ __forceinline__ IndexItem index_item(int64_t w, int QG, int64_t KT) {
+  IndexItem it;
+  it.kt = w % KT;
+  const int64_t r = w / KT;
+  it.qg = (int)(r % QG);
+  it.b = (int)(r / QG);
+  return it;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                          const __grid_constant__ CUtensorMap qmap,
+                                                          const IndexParams p) {
+  using Cfg = IndexCfg<FP8>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int TQ = p.TQ;
+  const int NQ = TQ * kIdxHeads;                    // MMA N
+  const int q_bytes = NQ * Cfg::kQRowBytes;
+  uint8_t* q_smem = smem;
+  uint8_t* k_smem = smem + q_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(k_smem + (size_t)p.stages * Cfg::kKeyBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + p.stages;
+  uint64_t* qfull = bars + 2 * p.stages;
+  uint64_t* qempty = qfull + 1;
+  uint64_t* tfull = qfull + 2;                      // [2]
+  uint64_t* tempty = qfull + 4;                     // [2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 6);
+  float* w_all = reinterpret_cast<float*>(qfull + 8);  // [4 epilogue warps][TQ][64]
+
+  const int QG = (p.T + TQ - 1) / TQ;
+  const int64_t KT = (p.N + kIdxTileKeys - 1) / kIdxTileKeys;
+  const int64_t items = (int64_t)p.B * QG * KT;
+  const int64_t w0 = items * blockIdx.x / gridDim.x;
+  const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
+  const uint32_t tmem_cols = (uint32_t)(2 * NQ) < 32 ? 32u : (uint32_t)(2 * NQ);
+
+  const int warp = warp_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);                     // one arrive per epilogue warp
+    }
+    fence_mbar_init();
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (elect_one()) {
+      int prev_b = -1, prev_qg = -1;
+      uint32_t qe_phase = 0;
+      int64_t cnt = 0;
+      for (int64_t w = w0; w < w1; ++w, ++cnt) {
+        const IndexItem it = index_item(w, QG, KT);
+        if (it.b != prev_b || it.qg != prev_qg) {
+          if (prev_b >= 0) {
+            if (!mbar_wait(qempty, qe_phase)) break;
+            qe_phase ^= 1;
+          }
+          mbar_arrive_expect_tx(qfull, (uint32_t)q_bytes);
+          for (int a = 0; a < Cfg::kAtoms; ++a)
+            tma_load_3d(q_smem + (size_t)a * NQ * 128, &qmap, qfull, a * 64, it.qg * NQ, it.b);
+          prev_b = it.b;
+          prev_qg = it.qg;
+        }
+        const int s = (int)(cnt % p.stages);
+        const uint32_t ph = (uint32_t)((cnt / p.stages) & 1);
+        if (!mbar_wait(&empty[s], ph ^ 1)) break;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKeyBytes);
+        uint8_t* dst = k_smem + (size_t)s * Cfg::kKeyBytes;
+        for (int a = 0; a < Cfg::kAtoms; ++a)
+          tma_load_3d(dst + (size_t)a * kIdxTileKeys * 128, &kmap, &full[s], a * 64, (int)(it.kt * kIdxTileKeys),
+                      it.b);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc = make_idesc(128, NQ, FP8 ? 0u : 1u, 0, 0);
+      int prev_b = -1, prev_qg = -1;
+      uint32_t qf_phase = 0;
+      int64_t cnt = 0;
+      for (int64_t w = w0; w < w1; ++w, ++cnt) {
+        const IndexItem it = index_item(w, QG, KT);
+        if (it.b != prev_b || it.qg != prev_qg) {
+          if (prev_b >= 0) mma_commit(qempty);      // old Q free once its MMAs finish
+          if (!mbar_wait(qfull, qf_phase)) break;
+          qf_phase ^= 1;
+          prev_b = it.b;
+          prev_qg = it.qg;
+        }
+        const int s = (int)(cnt % p.stages);
+        const uint32_t ph = (uint32_t)((cnt / p.stages) & 1);
+        const int acc = (int)(cnt & 1);
+        const uint32_t aph = (uint32_t)((cnt >> 1) & 1);
+        if (!mbar_wait(&tempty[acc], aph ^ 1)) break;
+        if (!mbar_wait(&full[s], ph)) break;
+        tc_fence_after();
+        const uint32_t kbase = smem_u32(k_smem + (size_t)s * Cfg::kKeyBytes);
+        const uint32_t qbase = smem_u32(q_smem);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NQ);
+#pragma unroll
+        for (int kk = 0; kk < Cfg::kKSteps; ++kk) {
+          const int byte_k = kk * Cfg::kKInstr * (FP8 ? 1 : 2);   // byte offset along K
+          const int atom = byte_k / 128;
+          const int inner = byte_k % 128;
+          const uint64_t adesc =
+              smem_desc(kbase + atom * kIdxTileKeys * 128 + inner, 16, 1024, kLayoutSW128);
+          const uint64_t bdesc = smem_desc(qbase + atom * NQ * 128 + inner, 16, 1024, kLayoutSW128);
+          if (FP8)
+            mma_f8(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          else
+            mma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int quarter = warp & 3;                   // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + (int)lane_id();  // key within the tile
+    float* w_s = w_all + (warp - 2) * TQ * kIdxHeads;
+    int prev_b = -1, prev_qg = -1;
+    int64_t cnt = 0;
+    for (int64_t w = w0; w < w1; ++w, ++cnt) {
+      const IndexItem it = index_item(w, QG, KT);
+      if (it.b != prev_b || it.qg != prev_qg) {
+        // each epilogue warp keeps a private copy of the group's head weights
+        __syncwarp();
+        for (int j = (int)lane_id(); j < TQ * kIdxHeads; j += 32) {
+          const int t = it.qg * TQ + j / kIdxHeads;
+          float v = 0.f;
+          if (t < p.T) {
+            const int64_t o = ((int64_t)it.b * p.T + t) * kIdxHeads + (j % kIdxHeads);
+            v = p.w[o];
+            if (FP8) v *= p.q_scale[o];
+          }
+          w_s[j] = v;
+        }
+        __syncwarp();
+        prev_b = it.b;
+        prev_qg = it.qg;
+      }
+      const int acc = (int)(cnt & 1);
+      const uint32_t aph = (uint32_t)((cnt >> 1) & 1);
+      if (!mbar_wait(&tfull[acc], aph)) break;
+      tc_fence_after();
+      const int64_t i = it.kt * kIdxTileKeys + row;
+      const float ks = (FP8 && i < p.N) ? p.k_scale[(int64_t)it.b * p.N + i] : 1.f;
+      for (int q = 0; q < TQ; ++q) {
+        const int t = it.qg * TQ + q;
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NQ + q * 64);
+        float v0[32], v1[32];
+        tmem_ld32(taddr, v0);
+        tmem_ld32(taddr + 32, v1);
+        tmem_wait_ld();
+        if (t >= p.T) continue;
+        const float* wq = w_s + q * kIdxHeads;
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s = fmaf(wq[h], fmaxf(v0[h], 0.f), s);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s = fmaf(wq[32 + h], fmaxf(v1[h], 0.f), s);
+        if (i < p.N) {
+          const int64_t nv = p.n_valid[(int64_t)it.b * p.T + t];
+          p.scores[((int64_t)it.b * p.T + t) * p.N + i] = (i < nv) ? s * ks : -INFINITY;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+constexpr int kIdxF32Smem = (kIdxHeads + 64) * (kIdxDim + 4) * 4;
+
+// fp32 SIMT path: CTA = (tile of 64 keys, query t, sequence b); 256 threads as a
+// 16 x 16 grid, each computing 4 keys x 4 heads over the 128 dims from shared
+// memory, then ReLU, head weights, and a reduction over the 16 head groups.
+__global__ void __launch_bounds__(256) index_f32_kernel(const float* __restrict__ qI, const float* __restrict__ w,
+                                                        const float* __restrict__ kI,
+                                                        const int32_t* __restrict__ n_valid, int T, int64_t N,
+                                                        float* __restrict__ scores) {
+  constexpr int KT = 64, PAD = 4;
+  extern __shared__ __align__(16) float f32_smem[];
+  float(*qs)[kIdxDim + PAD] = reinterpret_cast<float(*)[kIdxDim + PAD]>(f32_smem);
+  float(*ks)[kIdxDim + PAD] = reinterpret_cast<float(*)[kIdxDim + PAD]>(f32_smem + kIdxHeads * (kIdxDim + PAD));
+  __shared__ float red[16][KT];
+  __shared__ float ws[kIdxHeads];
+  const int b = blockIdx.z, t = blockIdx.y;
+  const int64_t k0 = (int64_t)blockIdx.x * KT;
+  const float* qrow = qI + ((int64_t)b * T + t) * kIdxHeads * kIdxDim;
+  for (int j = threadIdx.x; j < kIdxHeads * kIdxDim / 4; j += 256) {
+    const int h = j / (kIdxDim / 4), d = (j % (kIdxDim / 4)) * 4;
+    *reinterpret_cast<float4*>(&qs[h][d]) = *reinterpret_cast<const float4*>(qrow + h * kIdxDim + d);
+  }
+  for (int j = threadIdx.x; j < KT * kIdxDim / 4; j += 256) {
+    const int r = j / (kIdxDim / 4), d = (j % (kIdxDim / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (k0 + r < N) v = *reinterpret_cast<const float4*>(kI + ((int64_t)b * N + k0 + r) * kIdxDim + d);
+    *reinterpret_cast<float4*>(&ks[r][d]) = v;
+  }
+  if (threadIdx.x < kIdxHeads) ws[threadIdx.x] = w[((int64_t)b * T + t) * kIdxHeads + threadIdx.x];
+  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+  for (int d = 0; d < kIdxDim; d += 4) {
+    float4 kv[4], qv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kv[u] = *reinterpret_cast<const float4*>(&ks[tx + 16 * u][d]);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) qv[v] = *reinterpret_cast<const float4*>(&qs[ty + 16 * v][d]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        acc[u][v] = fmaf(kv[u].x, qv[v].x, acc[u][v]);
+        acc[u][v] = fmaf(kv[u].y, qv[v].y, acc[u][v]);
+        acc[u][v] = fmaf(kv[u].z, qv[v].z, acc[u][v]);
+        acc[u][v] = fmaf(kv[u].w, qv[v].w, acc[u][v]);
+      }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float s = 0.f;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) s = fmaf(ws[ty + 16 * v], fmaxf(acc[u][v], 0.f), s);
+    red[ty][tx + 16 * u] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x < KT) {
+    const int64_t i = k0 + threadIdx.x;
+    float s = 0.f;
+    for (int g = 0; g < 16; ++g) s += red[g][threadIdx.x];
+    if (i < N) {
+      const int64_t nv = n_valid[(int64_t)b * T + t];
+      scores[((int64_t)b * T + t) * N + i] = (i < nv) ? s : -INFINITY;
+    }
+  }
+}
+
+}  // namespace csa

@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI without a GPU: the library loads, exports every
+function include/csa.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_compressed_b200 import build
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "csa.h"), encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_header_declares_the_five_calls():
+    names = declared_functions()
+    for n in ("csa_compress", "csa_index_scores", "csa_topk", "sparse_attn", "hca_attn"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_names_match_header():
+    from long_context_compressed_b200 import csa
+    assert sorted(csa.EXPORTED) == declared_functions()
+
+
+def test_status_strings(lib):
+    lib.csa_status_string.restype = ctypes.c_char_p
+    assert lib.csa_status_string(0) == b"CSA_OK"
+    assert b"INVALID" in lib.csa_status_string(1)
+    assert lib.csa_version() == 100
+
+
+def _vp(x=16):
+    return ctypes.c_void_p(x)
+
+
+def test_compress_rejects_bad_arguments(lib):
+    f = lib.csa_compress
+    f.restype = ctypes.c_int
+    i64 = ctypes.c_int64
+    p = _vp()
+    # ratio must be 4 or 128
+    assert f(p, p, p, p, None, None, 1, i64(64), 8, 5, 1, 1, p, None) == 1
+    # carry given for one branch only
+    assert f(p, p, p, p, p, None, 1, i64(64), 8, 4, 1, 1, p, None) == 1
+    # channels not a multiple of 8
+    assert f(p, p, p, p, None, None, 1, i64(64), 12, 4, 1, 1, p, None) == 1
+    # misaligned pointer
+    assert f(_vp(18), p, p, p, None, None, 1, i64(64), 8, 4, 1, 1, p, None) == 1
+    # HCA with a b branch
+    assert f(p, p, p, None, None, None, 1, i64(256), 128, 128, 1, 1, p, None) == 1
+    # bad dtype code
+    assert f(p, p, p, p, None, None, 1, i64(64), 8, 4, 7, 1, p, None) == 1
+    # nothing to do is OK and launches nothing
+    assert f(p, p, p, p, None, None, 0, i64(64), 8, 4, 1, 1, p, None) == 0
+    assert f(p, p, p, p, None, None, 1, i64(3), 8, 4, 1, 1, p, None) == 0
+
+
+def test_topk_rejects_bad_arguments(lib):
+    f = lib.csa_topk
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    p = 16
+    assert f(p, p, 1, 1, 100, 0, p, None, 0, None) == 1           # k < 1
+    assert f(p, p, 1, 1, 100, 4096, p, None, 0, None) == 1        # k > max
+    assert f(p, p, 1, 1, (1 << 20) + 1, 8, p, None, 0, None) == 2  # N too large
+    # long rows need a workspace of csa_topk_workspace_size bytes
+    lib.csa_topk_workspace_size.restype = ctypes.c_size_t
+    lib.csa_topk_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int]
+    need = lib.csa_topk_workspace_size(1, 1, 262144, 1024)
+    assert need > 262144 * 8
+    assert f(p, p, 1, 1, 262144, 1024, p, None, 0, None) == 1
+    assert f(p, p, 1, 1, 262144, 1024, p, 16, need - 1, None) == 1
+    assert lib.csa_topk_workspace_size(4096, 1, 32768, 512) == 0   # row-resident path needs none
+
+
+def test_index_and_attention_reject_bad_arguments(lib):
+    f = lib.csa_index_scores
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    p = 16
+    assert f(p, None, p, p, None, 2, p, 1, 1, 100, p, None) == 1   # e4m3 without scales
+    assert f(p, None, p, p, None, 9, p, 1, 1, 100, p, None) == 1   # bad dtype
+    assert f(p, None, None, p, None, 1, p, 1, 1, 100, p, None) == 1  # no head weights
+    g = lib.sparse_attn
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    # bf16 supports D in {128, 256, 512} and H <= 128
+    assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 16, 96, 100, 1, p, None, 0, None) == 2
+    assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 256, 512, 100, 1, p, None, 0, None) == 2
+    # NaN scale, negative k
+    assert g(p, p, p, p, 128, p, p, p, 8, float("nan"), 1, 1, 16, 128, 100, 1, p, None, 0, None) == 1
+    assert g(p, p, p, p, 128, p, p, p, -1, 0.1, 1, 1, 16, 128, 100, 1, p, None, 0, None) == 1

@@ -1,0 +1,132 @@
+"""Indexer parity: fp32 SIMT, bf16 and e4m3 tcgen05 paths vs the CPU oracle; e4m3
+quantiser bit-exactness; FP8 top-k recall against the exact (unquantised) ranking."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_compressed_b200 import synth
+from tolerances import check_f32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csa():
+    from long_context_compressed_b200 import csa
+    return csa
+
+
+def _inputs(wl, seed=0, N=None):
+    ix = synth.draw_indexer(wl, seed=seed, N=N)
+    q_pos = np.array([wl.q_pos] * wl.B, np.int64)
+    nv = oracle.n_visible(q_pos, wl.ratio, ix["kI"].shape[1])
+    return ix, q_pos, nv
+
+
+def _check_scores(gpu, ref, mag, what):
+    fin = np.isfinite(ref)
+    assert np.all(np.isneginf(gpu[~fin])), f"{what}: invalid tail not -inf"
+    check_f32(gpu[fin], ref[fin], mag[fin], what=what)
+
+
+def test_f32_tiny_full(csa):
+    wl = synth.WORKLOADS["tiny"]
+    ix, _, nv = _inputs(wl)
+    s = csa.csa_index_scores(ix["qI"].cuda(), ix["w"].cuda(), ix["kI"].cuda(), torch.from_numpy(nv).cuda())
+    ref, mag = oracle.index_scores(ix["qI"].numpy(), ix["w"].numpy(), ix["kI"].numpy(), nv, with_mag=True)
+    _check_scores(s.cpu().numpy().astype(np.float64), ref, mag, "tiny fp32")
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 9])
+@pytest.mark.parametrize("N", [128, 1000, 3 * 128 + 1])
+def test_bf16_ragged(csa, T, N):
+    """Several query groups (T not a multiple of the group size), a ragged last key tile,
+    and per-query n_valid below N."""
+    wl = synth.Workload("idx_ragged", "bf16", B=2, ctx=4 * N, T=T, q_pos0=4 * N - 3 * T - 2, ratio=4, N=N,
+                        H=16, D=128, index_dtype="bf16")
+    ix, _, nv = _inputs(wl, seed=T * 1000 + N)
+    nv[1, 0] = min(N, 5)                                 # a short row
+    s = csa.csa_index_scores(ix["qI"].cuda(), ix["w"].cuda(), ix["kI"].cuda(), torch.from_numpy(nv).cuda())
+    ref, mag = oracle.index_scores(ix["qI"].float().numpy(), ix["w"].numpy(), ix["kI"].float().numpy(), nv,
+                                   with_mag=True)
+    _check_scores(s.cpu().numpy().astype(np.float64), ref, mag, f"bf16 T={T} N={N}")
+
+
+def test_quantizer_bit_exact(csa):
+    x = synth.store(synth.normal(0, "quant/x", (3000, 128), std=2.0), "bf16")
+    x[7] = 0                                             # all-zero row -> scale 1
+    x[8, 5] = 1e-30                                      # tiny values
+    codes, scale = csa.csa_quantize_e4m3(x.cuda())
+    rc, rs = oracle.quantize_rows_e4m3(x.float().numpy())
+    assert np.array_equal(scale.cpu().numpy(), rs)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    xf = synth.normal(0, "quant/xf", (257, 128), std=30.0)
+    codes, scale = csa.csa_quantize_e4m3(xf.cuda())
+    rc, rs = oracle.quantize_rows_e4m3(xf.numpy())
+    assert np.array_equal(scale.cpu().numpy(), rs) and np.array_equal(codes.cpu().numpy(), rc)
+
+
+@pytest.mark.parametrize("T,N", [(1, 1000), (3, 517), (4, 256), (6, 130)])
+def test_e4m3_ragged(csa, T, N):
+    wl = synth.Workload("idx8", "bf16", B=2, ctx=4 * N, T=T, q_pos0=4 * N - T - 9, ratio=4, N=N, H=16, D=128,
+                        index_dtype="e4m3")
+    ix, _, nv = _inputs(wl, seed=17 + T)
+    q8, qs = oracle.quantize_rows_e4m3(ix["qI"].float().numpy())
+    k8, ks = oracle.quantize_rows_e4m3(ix["kI"].float().numpy())
+    s = csa.csa_index_scores(torch.from_numpy(q8).cuda(), ix["w"].cuda(), torch.from_numpy(k8).cuda(),
+                             torch.from_numpy(nv).cuda(), q_scale=torch.from_numpy(qs).cuda(),
+                             k_scale=torch.from_numpy(ks).cuda())
+    ref, mag = oracle.index_scores_e4m3(q8, qs, ix["w"].numpy(), k8, ks, nv, with_mag=True)
+    _check_scores(s.cpu().numpy().astype(np.float64), ref, mag, f"e4m3 T={T} N={N}")
+
+
+@pytest.mark.parametrize("name", ["flash64k", "pro1m"])
+def test_full_decode_workloads(csa, name):
+    """Full-size decode indexers: bf16 and the e4m3 variant, every score checked."""
+    wl = synth.WORKLOADS[name]
+    ix, _, nv = _inputs(wl)
+    g_nv = torch.from_numpy(nv).cuda()
+    if name == "flash64k":
+        s = csa.csa_index_scores(ix["qI"].cuda(), ix["w"].cuda(), ix["kI"].cuda(), g_nv)
+        ref, mag = oracle.index_scores(ix["qI"].float().numpy(), ix["w"].numpy(), ix["kI"].float().numpy(), nv,
+                                       with_mag=True)
+        _check_scores(s.cpu().numpy().astype(np.float64), ref, mag, name + " bf16")
+    q8, qs = oracle.quantize_rows_e4m3(ix["qI"].float().numpy())
+    k8, ks = oracle.quantize_rows_e4m3(ix["kI"].float().numpy())
+    s8 = csa.csa_index_scores(torch.from_numpy(q8).cuda(), ix["w"].cuda(), torch.from_numpy(k8).cuda(), g_nv,
+                              q_scale=torch.from_numpy(qs).cuda(), k_scale=torch.from_numpy(ks).cuda())
+    ref8, mag8 = oracle.index_scores_e4m3(q8, qs, ix["w"].numpy(), k8, ks, nv, with_mag=True)
+    _check_scores(s8.cpu().numpy().astype(np.float64), ref8, mag8, name + " e4m3")
+
+
+def test_prefill_sampled_rows(csa):
+    """Full prefill launch (4096 queries x 32768 keys); the oracle checks sampled query rows."""
+    wl = synth.WORKLOADS["flash_prefill"]
+    ix, _, nv = _inputs(wl)
+    s = csa.csa_index_scores(ix["qI"].cuda(), ix["w"].cuda(), ix["kI"].cuda(), torch.from_numpy(nv).cuda())
+    rows = [0, 1, 2, 3, 4, 1023, 2048, 3071, 4092, 4093, 4094, 4095]
+    ref, mag = oracle.index_scores(ix["qI"][:, rows].float().numpy(), ix["w"][:, rows].numpy(),
+                                   ix["kI"].float().numpy(), nv[:, rows], with_mag=True)
+    _check_scores(s[:, rows].cpu().numpy().astype(np.float64), ref, mag, "prefill sampled")
+    # every row: the invalid tail is -inf exactly and the valid part is finite
+    s_all = s.cpu()
+    for t in range(0, wl.T, 97):
+        assert torch.isneginf(s_all[0, t, nv[0, t]:]).all() and torch.isfinite(s_all[0, t, :nv[0, t]]).all()
+
+
+def test_e4m3_recall_pro1m(csa):
+    """FP8 indexer (GPU quantiser + GPU e4m3 scores + GPU top-k) against the exact top-1024
+    of the unquantised bf16 inputs (oracle scores + oracle top-k): recall >= 0.99."""
+    wl = synth.WORKLOADS["pro1m"]
+    ix, _, nv = _inputs(wl)
+    g_nv = torch.from_numpy(nv).cuda()
+    q8, qs = csa.csa_quantize_e4m3(ix["qI"].cuda())
+    k8, ks = csa.csa_quantize_e4m3(ix["kI"].cuda())
+    s8 = csa.csa_index_scores(q8, ix["w"].cuda(), k8, g_nv, q_scale=qs, k_scale=ks)
+    idx8 = csa.csa_topk(s8, g_nv, wl.topk).cpu().numpy()
+    ref = oracle.index_scores(ix["qI"].float().numpy(), ix["w"].numpy(), ix["kI"].float().numpy(), nv)
+    idx_ref = oracle.topk(ref.astype(np.float32), nv, wl.topk)
+    recall = len(np.intersect1d(idx8[0, 0], idx_ref[0, 0])) / wl.topk
+    print(f"pro1m e4m3 top-{wl.topk} recall = {recall:.4f}")
+    assert recall >= 0.99
