@@ -126,6 +126,23 @@ int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t 
              void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * csa_index_rerank -- exact rescoring of a candidate list, then top-k among it
+ * ([HA] §9: the indexer forms its candidates at twice top-k; this is the
+ * second stage that makes a low-precision first pass exact on its candidates).
+ *   cand[b,t,:] (kc ascending indices, -1 padded; typically csa_topk of the e4m3
+ *   scores with 2k) is rescored with the plain definition of csa_index_scores on
+ *   the full-precision qI / kI (dtype F32 or BF16, fp32 accumulation), then
+ *   idx[b,t,:] = the k best candidates (ties toward the lower index), ascending,
+ *   -1 padded -- equal to csa_topk of the full-precision scores whenever the true
+ *   top-k lies inside the candidate list.
+ *   qI [B,T,64,128], w [B,T,64] fp32, kI [B,N,128], cand [B,T,kc] int32,
+ *   cand_scores [B,T,kc] fp32 (caller scratch), idx [B,T,k] int32;
+ *   k <= kc <= 32768.
+ */
+int csa_index_rerank(const void *qI, const float *w, const void *kI, int dtype, const int32_t *cand, int kc, int B,
+                     int T, int64_t N, int k, float *cand_scores, int32_t *idx, void *stream);
+
+/*
  * sparse_attn -- CSA core attention ([P2] sparse_attn(q, kv, attn_sink,
  * topk_idxs, softmax_scale); [HA] §4.2 Shared-KV MQA, §6 SWA + sink, §7 call chain):
  *   for query (b,t) at absolute position pos = q_pos[b,t] and head h:

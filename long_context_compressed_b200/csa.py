@@ -33,6 +33,7 @@ _SIGS = {
     "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp], _i32),
+    "csa_index_rerank": ([_vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_topk_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "csa_topk": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "csa_attn_workspace_size": ([_i32, _i32, _i32, _i32, _i64, _i32], _sz),
@@ -127,6 +128,20 @@ def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=N
     _check(_lib.csa_index_scores(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), _dtype_code(qI),
                                  _ptr(n_valid), B, T, N, _ptr(scores), _stream(stream)), "csa_index_scores")
     return scores
+
+
+def csa_index_rerank(qI, w, kI, cand, k: int, *, cand_scores=None, idx=None, stream=None):
+    """Exact rescoring of candidates cand [B, T, kc] (ascending, -1 padded) with full-precision
+    qI / kI (fp32 or bf16), then the k best -> idx [B, T, k] int32 (ascending, -1 padded)."""
+    B, T, kc = cand.shape
+    N = kI.shape[1]
+    if cand_scores is None:
+        cand_scores = torch.empty((B, T, kc), dtype=torch.float32, device=qI.device)
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=qI.device)
+    _check(_lib.csa_index_rerank(_ptr(qI), _ptr(w), _ptr(kI), _dtype_code(qI), _ptr(cand), kc, B, T, N, k,
+                                 _ptr(cand_scores), _ptr(idx), _stream(stream)), "csa_index_rerank")
+    return idx
 
 
 def csa_topk_workspace_size(B: int, T: int, N: int, k: int) -> int:

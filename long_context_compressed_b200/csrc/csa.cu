@@ -262,9 +262,9 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
   if (dtype == CSA_F32) {
     if (T > 65535) return CSA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)((N + 63) / 64), (unsigned)T, (unsigned)B);
-    if (!set_smem(csa::index_f32_kernel, csa::kIdxF32Smem)) return CSA_ERR_CUDA;
-    csa::index_f32_kernel<<<grid, 256, csa::kIdxF32Smem, st>>>((const float*)qI, w, (const float*)kI, n_valid, T,
-                                                               N, scores);
+    if (!set_smem(csa::index_simt_kernel<float, false>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
+    csa::index_simt_kernel<float, false><<<grid, 256, csa::kIdxSimtSmem, st>>>(
+        (const float*)qI, w, (const float*)kI, n_valid, nullptr, 0, T, N, scores);
     return launch_status();
   }
   const bool fp8 = dtype == CSA_E4M3;
@@ -306,6 +306,34 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
   return launch_status();
 }
 
+int csa_index_rerank(const void* qI, const float* w, const void* kI, int dtype, const int32_t* cand, int kc, int B,
+                     int T, int64_t N, int k, float* cand_scores, int32_t* idx, void* stream) {
+  if (B < 0 || T < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK || kc < k || kc > csa::kRowSmemMax)
+    return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (B == 0 || T == 0) return CSA_OK;
+  if (!qI || !w || !kI || !cand || !cand_scores || !idx) return CSA_ERR_INVALID;
+  if (!aligned16(qI) || !aligned16(kI)) return CSA_ERR_INVALID;
+  if (T > 65535 || B > 65535) return CSA_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  dim3 grid((unsigned)((kc + 63) / 64), (unsigned)T, (unsigned)B);
+  if (dtype == CSA_BF16) {
+    if (!set_smem(csa::index_simt_kernel<__nv_bfloat16, true>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
+    csa::index_simt_kernel<__nv_bfloat16, true><<<grid, 256, csa::kIdxSimtSmem, st>>>(
+        (const __nv_bfloat16*)qI, w, (const __nv_bfloat16*)kI, nullptr, cand, kc, T, N, cand_scores);
+  } else {
+    if (!set_smem(csa::index_simt_kernel<float, true>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
+    csa::index_simt_kernel<float, true><<<grid, 256, csa::kIdxSimtSmem, st>>>(
+        (const float*)qI, w, (const float*)kI, nullptr, cand, kc, T, N, cand_scores);
+  }
+  int rc = launch_status();
+  if (rc != CSA_OK) return rc;
+  const int smem = kc * 4;
+  if (!set_smem(csa::topk_row_kernel, std::max(smem, 4))) return CSA_ERR_CUDA;
+  csa::topk_row_kernel<<<(unsigned)((int64_t)B * T), 1024, smem, st>>>(cand_scores, nullptr, kc, k, idx, cand);
+  return launch_status();
+}
+
 static bool topk_long_path(int B, int T, int64_t N) {
   const int64_t rows = (int64_t)B * T;
   return N > csa::kRowSmemMax || (rows < 74 && N >= 4 * csa::kChunk);
@@ -331,7 +359,7 @@ int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t 
   if (!topk_long_path(B, T, N)) {
     const int smem = (int)std::max<int64_t>(4, std::min<int64_t>(N, csa::kRowSmemMax) * 4);
     if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
-    csa::topk_row_kernel<<<(unsigned)rows, 1024, smem, st>>>(scores, n_valid, N, k, idx);
+    csa::topk_row_kernel<<<(unsigned)rows, 1024, smem, st>>>(scores, n_valid, N, k, idx, nullptr);
     return launch_status();
   }
   const size_t need = csa_topk_workspace_size(B, T, N, k);

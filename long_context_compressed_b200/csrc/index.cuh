@@ -19,7 +19,8 @@
 //          scale qs[b,t,h]; both are positive so they commute with ReLU:
 //          s = ks * sum_h (w * qs)_h * ReLU(<q8, k8>).
 //
-// index_f32_kernel: fp32 SIMT path (FMA), used for fp32 inputs.
+// index_simt_kernel: fp32 SIMT path (FMA), used for fp32 inputs and for the
+// exact rescoring of a candidate list.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -254,35 +255,63 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
   if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
 }
 
-constexpr int kIdxF32Smem = (kIdxHeads + 64) * (kIdxDim + 4) * 4;
+constexpr int kIdxSimtSmem = (kIdxHeads + 64) * (kIdxDim + 4) * 4;
 
-// fp32 SIMT path: CTA = (tile of 64 keys, query t, sequence b); 256 threads as a
-// 16 x 16 grid, each computing 4 keys x 4 heads over the 128 dims from shared
-// memory, then ReLU, head weights, and a reduction over the 16 head groups.
-__global__ void __launch_bounds__(256) index_f32_kernel(const float* __restrict__ qI, const float* __restrict__ w,
-                                                        const float* __restrict__ kI,
-                                                        const int32_t* __restrict__ n_valid, int T, int64_t N,
-                                                        float* __restrict__ scores) {
+__device__ __forceinline__ float4 load4f(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4f(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// SIMT path (fp32 FMA): CTA = (tile of 64 keys, query t, sequence b); 256 threads
+// as a 16 x 16 grid, each computing 4 keys x 4 heads over the 128 dims from
+// shared memory, then ReLU, head weights, and a reduction over the 16 head
+// groups.  Inputs fp32 or bf16 (widened exactly to fp32).
+//   GATHER = false: keys 0..N-1, scores[b,t,i] (-inf for i >= n_valid[b,t]).
+//   GATHER = true : keys cand[b,t,j] for j < kc (the exact rescoring of a
+//                   candidate list); out[b,t,j], -inf where cand is outside [0, N).
+template <typename Tin, bool GATHER>
+__global__ void __launch_bounds__(256) index_simt_kernel(const Tin* __restrict__ qI, const float* __restrict__ w,
+                                                         const Tin* __restrict__ kI,
+                                                         const int32_t* __restrict__ n_valid,
+                                                         const int32_t* __restrict__ cand, int kc, int T, int64_t N,
+                                                         float* __restrict__ out) {
   constexpr int KT = 64, PAD = 4;
   extern __shared__ __align__(16) float f32_smem[];
   float(*qs)[kIdxDim + PAD] = reinterpret_cast<float(*)[kIdxDim + PAD]>(f32_smem);
   float(*ks)[kIdxDim + PAD] = reinterpret_cast<float(*)[kIdxDim + PAD]>(f32_smem + kIdxHeads * (kIdxDim + PAD));
   __shared__ float red[16][KT];
   __shared__ float ws[kIdxHeads];
+  __shared__ int64_t krow[KT];
   const int b = blockIdx.z, t = blockIdx.y;
+  const int64_t bt = (int64_t)b * T + t;
   const int64_t k0 = (int64_t)blockIdx.x * KT;
-  const float* qrow = qI + ((int64_t)b * T + t) * kIdxHeads * kIdxDim;
+  const int64_t width = GATHER ? (int64_t)kc : N;     // entries of the output row
+  if (threadIdx.x < KT) {
+    const int64_t j = k0 + threadIdx.x;
+    int64_t r = -1;
+    if (j < width) {
+      r = GATHER ? (int64_t)cand[bt * kc + j] : j;
+      if (r < 0 || r >= N) r = -1;
+    }
+    krow[threadIdx.x] = r;
+  }
+  const Tin* qrow = qI + bt * kIdxHeads * kIdxDim;
   for (int j = threadIdx.x; j < kIdxHeads * kIdxDim / 4; j += 256) {
     const int h = j / (kIdxDim / 4), d = (j % (kIdxDim / 4)) * 4;
-    *reinterpret_cast<float4*>(&qs[h][d]) = *reinterpret_cast<const float4*>(qrow + h * kIdxDim + d);
+    *reinterpret_cast<float4*>(&qs[h][d]) = load4f(qrow + h * kIdxDim + d);
   }
+  if (threadIdx.x < kIdxHeads) ws[threadIdx.x] = w[bt * kIdxHeads + threadIdx.x];
+  __syncthreads();
   for (int j = threadIdx.x; j < KT * kIdxDim / 4; j += 256) {
     const int r = j / (kIdxDim / 4), d = (j % (kIdxDim / 4)) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (k0 + r < N) v = *reinterpret_cast<const float4*>(kI + ((int64_t)b * N + k0 + r) * kIdxDim + d);
+    const int64_t row = krow[r];
+    if (row >= 0) v = load4f(kI + ((int64_t)b * N + row) * kIdxDim + d);
     *reinterpret_cast<float4*>(&ks[r][d]) = v;
   }
-  if (threadIdx.x < kIdxHeads) ws[threadIdx.x] = w[((int64_t)b * T + t) * kIdxHeads + threadIdx.x];
   __syncthreads();
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4];
@@ -315,12 +344,13 @@ __global__ void __launch_bounds__(256) index_f32_kernel(const float* __restrict_
   }
   __syncthreads();
   if (threadIdx.x < KT) {
-    const int64_t i = k0 + threadIdx.x;
+    const int64_t j = k0 + threadIdx.x;
     float s = 0.f;
     for (int g = 0; g < 16; ++g) s += red[g][threadIdx.x];
-    if (i < N) {
-      const int64_t nv = n_valid[(int64_t)b * T + t];
-      scores[((int64_t)b * T + t) * N + i] = (i < nv) ? s : -INFINITY;
+    if (j < width) {
+      bool ok = krow[threadIdx.x] >= 0;
+      if (!GATHER) ok = ok && j < n_valid[bt];
+      out[bt * width + j] = ok ? s : -INFINITY;
     }
   }
 }

@@ -13,9 +13,17 @@ namespace csa {
 __device__ int g_status;
 
 constexpr int kStatusTimeout = 4;
-// try_wait polls before a wait is declared lost (each poll may also suspend
-// for a hardware-chosen interval); about a second on B200.
-constexpr uint32_t kSpinLimit = 1u << 25;
+// A wait on a barrier that has not completed after this many nanoseconds of
+// %globaltimer is abandoned.  Every wait in this library is on work of the
+// same CTA that takes microseconds, so the bound is never reached in normal
+// operation.
+constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -60,12 +68,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// records a timeout) if it does not complete within kSpinLimit polls.
+// records a timeout) if it does not complete within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-  record_status(kStatusTimeout);
-  return false;
+    if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      record_status(kStatusTimeout);
+      return false;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ async copies

@@ -136,19 +136,25 @@ __device__ __forceinline__ void write_all_valid(int32_t* out, int nv, int k) {
 }
 
 // ---------------------------------------------------------------- row kernel
+// n_valid may be null (every row has N valid entries); map may be null, else the
+// output holds map[row, position] instead of the position (used to return the
+// original indices of a rescored candidate list; map rows must be ascending so
+// that the output stays ascending).
 __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict__ scores,
                                                         const int32_t* __restrict__ n_valid, int64_t N, int k,
-                                                        int32_t* __restrict__ idx) {
+                                                        int32_t* __restrict__ idx,
+                                                        const int32_t* __restrict__ map) {
   extern __shared__ __align__(16) uint32_t keys[];  // [min(N, kRowSmemMax)]
   __shared__ int hist[256];
   __shared__ int scratch[33];
   __shared__ int res[2];
   const int64_t row = blockIdx.x;
-  int nv = n_valid[row];
+  int nv = n_valid ? n_valid[row] : (int)N;
   nv = nv < 0 ? 0 : (nv > (int)N ? (int)N : nv);
   int32_t* out = idx + row * k;
+  const int32_t* mrow = map ? map + row * N : nullptr;
   if (nv <= k) {
-    write_all_valid(out, nv, k);
+    for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < nv ? (mrow ? mrow[j] : j) : -1;
     return;
   }
   const float* s = scores + row * N;
@@ -177,6 +183,10 @@ __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict_
   const int64_t lo = (int64_t)threadIdx.x * per;
   const int64_t hi = lo + per < nv ? lo + per : nv;
   write_selection(lo < nv ? lo : nv, hi, [&](int64_t i) { return keys[i]; }, prefix, remaining, out, scratch);
+  if (mrow) {
+    __syncthreads();
+    for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = mrow[out[j]];
+  }
 }
 
 // ---------------------------------------------------------------- long rows
@@ -344,6 +354,10 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
     bm_eq[wv] = 0;
   }
   for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
+  for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+    ckey[i] = 0;
+    cidx[i] = 0;
+  }
   if (threadIdx.x == 0) {
     *cand_count = 0;
     *done = 0;

@@ -52,3 +52,22 @@ def check_attn_bf16(gpu, ref, what=""):
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside abs 2e-2 + rel 1e-2; first at {tuple(i)}: "
                              f"gpu={gpu[tuple(i)]!r} ref={ref[tuple(i)]!r}; max err {err.max():.3g}")
+
+
+def check_topk_sets(gpu_idx, ref_scores, k, err_bound, what=""):
+    """Index sets from scores that carry rounding error: the GPU set may differ from the
+    exact top-k only at entries whose exact score is within the error window of the
+    k-th largest exact score (|s_i - s_k| <= max(1e-6 |s_k|, 2 E), E = measured max
+    score error).  gpu_idx [k] (ascending, -1 padded), ref_scores [n] exact scores."""
+    s = np.asarray(ref_scores, np.float64)
+    order = np.lexsort((np.arange(s.size), -s))
+    ref = np.sort(order[:k])
+    sk = s[order[min(k, s.size) - 1]]
+    win = max(1e-6 * abs(sk), 2.0 * err_bound)
+    g = np.asarray([i for i in gpu_idx if i >= 0])
+    assert len(set(g.tolist())) == len(g), f"{what}: duplicate indices"
+    assert np.all(np.diff(g) > 0), f"{what}: not ascending"
+    diff = np.setxor1d(g, ref)
+    bad = [int(i) for i in diff if abs(s[i] - sk) > win]
+    assert not bad, f"{what}: {len(bad)} indices differ beyond the tie window (e.g. {bad[:5]}, window {win:.3g})"
+    return len(np.intersect1d(g, ref)) / max(1, min(k, s.size))
