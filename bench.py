@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA / HCA decode hot path on B200 (one JSON line on rank 0).
+
+Step (default workload "flash64k"): one decode token for each of B = 8 sequences
+at 65,536 tokens of context, through one CSA layer and one HCA layer, as the
+Flash configuration alternates them ("DeepSeek-V4 混合注意力：从压缩记忆到百万上下文"
+§2 configuration table, §4-§7):
+  CSA: compress the newest 4-token block (latent c=512 and index keys c=128, with
+       the carry of the previous block) -> quantise the index queries (e4m3) ->
+       e4m3 index scores over 16,384 keys -> top-1024 candidates -> exact rerank
+       (bf16) to top-512 -> sparse_attn (64 heads, D=512, 512 + 128 SWA rows).
+  HCA: compress the newest 128-token block (c=512) -> hca_attn over 512 summaries
+       + 128 SWA rows.
+Metric: decode tokens/s = B x (GPUs) / step time.  "pro1m" (the 1M-context Pro CSA
+layer, B=1) is measured in the same run and reported under "pro1m".
+
+Every step is a CUDA graph replay of the library's C-ABI calls; S input sets (caches
+and per-step inputs) rotate so that the data the steps touch exceeds 2x the L2.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import platform
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """Maximum of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", f"-lms={period_ms}"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------- the step
+class DecodeSet:
+    """One input set of a decode workload: resident caches, per-step inputs, outputs and
+    workspaces on the device, plus pinned host copies of the per-step inputs/outputs."""
+
+    def __init__(self, wl, seed: int, index: str, with_hca: bool, device):
+        import torch
+
+        from long_context_compressed_b200 import csa, synth
+        self.wl, self.index, self.with_hca = wl, index, with_hca
+        B, T, N, H, D, k = wl.B, wl.T, wl.N, wl.H, wl.D, wl.topk
+        dev = device
+        g = lambda nm, shape: synth.store(synth.normal(seed, f"bench/{wl.name}/{nm}", shape, device=dev), "bf16")
+        f32 = lambda nm, shape: synth.normal(seed, f"bench/{wl.name}/{nm}", shape, device=dev)
+        # resident state (caches)
+        self.kv = g("kv", (B, N, D))
+        self.swa = g("swa", (B, wl.W, D))
+        self.kI = g("kI", (B, N, 128))
+        if index == "e4m3":
+            self.k8, self.ks = csa.csa_quantize_e4m3(self.kI)
+        self.sink = f32("sink", (H,))
+        self.q_pos = torch.full((B, T), wl.q_pos0, dtype=torch.int64, device=dev)
+        self.swa_pos0 = torch.full((B,), wl.swa_pos0, dtype=torch.int64, device=dev)
+        self.n_valid = csa.n_valid_for(self.q_pos, 4, N)
+        # per-step inputs
+        cL, cc = wl.comp_L, wl.comp_c
+        self.inputs = {
+            "q": g("q", (B, T, H, D)), "qI": g("qI", (B, T, 64, 128)), "w": f32("w", (B, T, 64)),
+            "C_a": g("C_a", (B, cL, cc)), "C_b": g("C_b", (B, cL, cc)), "Z_a": g("Z_a", (B, cL, cc)),
+            "Z_b": g("Z_b", (B, cL, cc)), "prev_Cb": g("prev_Cb", (B, 4, cc)), "prev_Zb": g("prev_Zb", (B, 4, cc)),
+        }
+        if wl.comp_ci:
+            ci = wl.comp_ci
+            self.inputs.update({"iC_a": g("iC_a", (B, cL, ci)), "iC_b": g("iC_b", (B, cL, ci)),
+                                "iZ_a": g("iZ_a", (B, cL, ci)), "iZ_b": g("iZ_b", (B, cL, ci)),
+                                "iprev_Cb": g("iprev_Cb", (B, 4, ci)), "iprev_Zb": g("iprev_Zb", (B, 4, ci))})
+        # outputs and scratch
+        self.comp_kv = torch.empty((B, cL // 4, cc), dtype=torch.bfloat16, device=dev)
+        self.comp_ki = torch.empty((B, cL // 4, wl.comp_ci or 8), dtype=torch.bfloat16, device=dev)
+        self.scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
+        self.q8 = torch.empty((B, T, 64, 128), dtype=torch.uint8, device=dev)
+        self.qs = torch.empty((B, T, 64), dtype=torch.float32, device=dev)
+        kc = 2 * k if index == "e4m3" else k
+        self.cand = torch.empty((B, T, kc), dtype=torch.int32, device=dev)
+        self.cand_scores = torch.empty((B, T, kc), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
+        self.topk_ws = csa.topk_workspace(B, T, N, kc, dev)
+        self.attn_ws = csa.attn_workspace(B, T, H, D, 128 + k, device=dev)
+        self.out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+        if with_hca:
+            Nh = wl.ctx // 128
+            self.hkv = g("hkv", (B, Nh, D))
+            self.hswa = g("hswa", (B, wl.W, D))
+            self.hsink = f32("hsink", (H,))
+            self.inputs.update({"hq": g("hq", (B, T, H, D)), "hC": g("hC", (B, 128, D)), "hZ": g("hZ", (B, 128, D))})
+            self.hcomp = torch.empty((B, 1, D), dtype=torch.bfloat16, device=dev)
+            self.hattn_ws = csa.attn_workspace(B, T, H, D, 128 + Nh, device=dev)
+            self.hout = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+        self.outputs = [self.out] + ([self.hout] if with_hca else [])
+        self.host_in = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in self.inputs.items()}
+        for n, t in self.inputs.items():
+            self.host_in[n].copy_(t)
+        self.host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in self.outputs]
+        self.ev = None
+
+    # -- byte accounting (algorithmic: inputs read once, outputs written once, intermediates excluded)
+    def index_bytes(self):
+        wl = self.wl
+        B, T, N = wl.B, wl.T, wl.N
+        if self.index == "e4m3":
+            keys = B * N * (128 + 4)
+            q = B * T * 64 * (128 + 4 + 4)
+        else:
+            keys = B * N * 256
+            q = B * T * 64 * (256 + 4)
+        return keys + q + B * T * N * 4
+
+    def step_bytes(self):
+        wl = self.wl
+        B, T, N, H, D, k = wl.B, wl.T, wl.N, wl.H, wl.D, wl.topk
+        nb = lambda t: t.numel() * t.element_size()
+        total = sum(nb(t) for t in self.inputs.values())                       # per-step inputs
+        total += nb(self.comp_kv) + (nb(self.comp_ki) if wl.comp_ci else 0)   # compressor outputs
+        total += B * N * (132 if self.index == "e4m3" else 256)               # index keys (+ scales)
+        if self.index == "e4m3":
+            total += B * T * 2 * k * 256                                      # rerank: bf16 keys of candidates
+        total += B * T * (k + min(wl.W, 128)) * D * 2                          # gathered latent + SWA rows
+        total += nb(self.out)
+        if self.with_hca:
+            total += B * (wl.ctx // 128) * D * 2 + B * min(wl.W, 128) * D * 2 + nb(self.hcomp) + nb(self.hout)
+        return total
+
+    def per_step_io(self):
+        nb = lambda t: t.numel() * t.element_size()
+        return sum(nb(t) for t in self.inputs.values()), sum(nb(o) for o in self.outputs)
+
+    # -- the step
+    def run(self, side_stream, timing_events: bool = False, copies: bool = False):
+        import torch
+
+        from long_context_compressed_b200 import csa
+        wl = self.wl
+        x = self.inputs
+        main = torch.cuda.current_stream()
+        if copies:
+            for n, t in x.items():
+                t.copy_(self.host_in[n], non_blocking=True)
+        side_stream.wait_stream(main)
+        # compressors and the HCA layer run on the side stream (independent of the indexer chain)
+        with torch.cuda.stream(side_stream):
+            csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"], ratio=4,
+                             out=self.comp_kv)
+            if wl.comp_ci:
+                csa.csa_compress(x["iC_a"], x["iC_b"], x["iZ_a"], x["iZ_b"], x["iprev_Cb"], x["iprev_Zb"], ratio=4,
+                                 out=self.comp_ki)
+            if self.with_hca:
+                csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=self.hcomp)
+                csa.hca_attn(x["hq"], self.hkv, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
+                             1.0 / math.sqrt(wl.D), out=self.hout, workspace=self.hattn_ws)
+        if timing_events:
+            self.ev = (torch.cuda.Event(enable_timing=True, external=True),
+                       torch.cuda.Event(enable_timing=True, external=True))
+        if self.index == "e4m3":
+            csa.csa_quantize_e4m3(x["qI"], codes=self.q8, scale=self.qs)
+            if timing_events:
+                self.ev[0].record()
+            csa.csa_index_scores(self.q8, x["w"], self.k8, self.n_valid, q_scale=self.qs, k_scale=self.ks,
+                                 scores=self.scores)
+            if timing_events:
+                self.ev[1].record()
+            csa.csa_topk(self.scores, self.n_valid, 2 * wl.topk, idx=self.cand, workspace=self.topk_ws)
+            csa.csa_index_rerank(x["qI"], x["w"], self.kI, self.cand, wl.topk, cand_scores=self.cand_scores,
+                                 idx=self.idx)
+        else:
+            if timing_events:
+                self.ev[0].record()
+            csa.csa_index_scores(x["qI"], x["w"], self.kI, self.n_valid, scores=self.scores)
+            if timing_events:
+                self.ev[1].record()
+            csa.csa_topk(self.scores, self.n_valid, wl.topk, idx=self.idx, workspace=self.topk_ws)
+        csa.sparse_attn(x["q"], self.kv, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
+                        1.0 / math.sqrt(wl.D), out=self.out, workspace=self.attn_ws)
+        main.wait_stream(side_stream)
+        if copies:
+            for h, o in zip(self.host_out, self.outputs):
+                h.copy_(o, non_blocking=True)
+
+
+def capture(sets, side, **kw):
+    import torch
+
+    from long_context_compressed_b200 import csa
+    graphs, launches = [], None
+    for s in sets:
+        s.run(side, **{k: v for k, v in kw.items() if k != "timing_events"})      # eager warm-up
+    torch.cuda.synchronize()
+    for s in sets:
+        g = torch.cuda.CUDAGraph()
+        c0 = csa.csa_launch_count()
+        with torch.cuda.graph(g):
+            s.run(side, **kw)
+        if launches is None:
+            launches = csa.csa_launch_count() - c0
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs, launches
+
+
+def timed_replays(graphs, steps: int, warmup: int, world: int):
+    import torch
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / 1e3          # seconds
+
+
+def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=None):
+    import torch
+
+    from long_context_compressed_b200 import csa, synth
+    wl = synth.WORKLOADS[name]
+    probe = DecodeSet(wl, 0, index, with_hca, device)
+    touched = probe.step_bytes()
+    n_sets = n_sets or max(2, math.ceil(2 * L2_BYTES / touched) + 1)
+    sets = [probe] + [DecodeSet(wl, s, index, with_hca, device) for s in range(1, n_sets)]
+    side = torch.cuda.Stream(device=device)
+    graphs, launches = capture(sets, side, timing_events=True)
+    t = timed_replays(graphs, steps, warmup, world)
+    t = max_over_ranks(t, world, device)
+    try:
+        idx_ms = [s.ev[0].elapsed_time(s.ev[1]) for s in sets]
+    except RuntimeError:
+        idx_ms = [float("nan")]
+    # end to end: the same step with its inputs copied in from pinned host memory and its
+    # outputs read back, inside every timed step
+    e2e_graphs, _ = capture(sets, side, copies=True)
+    t_e2e = max_over_ranks(timed_replays(e2e_graphs, steps, warmup, world), world, device)
+    assert csa.csa_poll_status() == csa.CSA_OK
+    h2d, d2h = probe.per_step_io()
+    res = {"wl": wl, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
+           "index_ms": statistics.mean(idx_ms), "index_bytes": probe.index_bytes(), "step_bytes": touched,
+           "e2e_seconds": t_e2e, "h2d": h2d, "d2h": d2h, "tokens_per_step": wl.B * wl.T}
+    del graphs, e2e_graphs, sets
+    torch.cuda.empty_cache()
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) leg
+def oracle_decode_token(wl, seed, index, with_hca):
+    """One sequence's decode step through the CPU oracle (fp64), on the same recipe."""
+    import numpy as np
+
+    import oracle
+    from long_context_compressed_b200 import synth
+    one = synth.Workload(**{**wl.__dict__, "B": 1, "extra": {}})
+    g = lambda nm, shape: synth.store(synth.normal(seed, f"bench/{wl.name}/{nm}", shape), "bf16").float().numpy()
+    f32 = lambda nm, shape: synth.normal(seed, f"bench/{wl.name}/{nm}", shape).numpy()
+    N, H, D, k, cL, cc = one.N, one.H, one.D, one.topk, one.comp_L, one.comp_c
+    kv, swa, kI = g("kv", (1, N, D)), g("swa", (1, one.W, D)), g("kI", (1, N, 128))
+    q, qI, w = g("q", (1, 1, H, D)), g("qI", (1, 1, 64, 128)), f32("w", (1, 1, 64))
+    sink = f32("sink", (H,))
+    comp = {nm: g(nm, (1, cL, cc)) for nm in ("C_a", "C_b", "Z_a", "Z_b")}
+    prev = {nm: g(nm, (1, 4, cc)) for nm in ("prev_Cb", "prev_Zb")}
+    k8, ks = oracle.quantize_rows_e4m3(kI) if index == "e4m3" else (None, None)
+    q_pos = np.array([[one.q_pos0]], np.int64)
+    nv = oracle.n_visible(q_pos, 4, N)
+    t0 = time.perf_counter()
+    oracle.compress_csa(comp["C_a"], comp["C_b"], comp["Z_a"], comp["Z_b"], prev["prev_Cb"], prev["prev_Zb"])
+    if index == "e4m3":
+        q8, qs = oracle.quantize_rows_e4m3(qI)
+        s8 = oracle.index_scores_e4m3(q8, qs, w, k8, ks, nv)
+        cand = oracle.topk(s8.astype(np.float32), nv, 2 * k)[0, 0]
+        cand = cand[cand >= 0]
+        sc = oracle.index_scores(qI, w, kI[:, cand], np.array([[len(cand)]], np.int32))
+        pos = oracle.topk(sc.astype(np.float32), np.array([[len(cand)]], np.int32), k)[0, 0]
+        idx = np.where(pos >= 0, cand[np.maximum(pos, 0)], -1).astype(np.int32)[None, None]
+    else:
+        s = oracle.index_scores(qI, w, kI, nv)
+        idx = oracle.topk(s.astype(np.float32), nv, k)
+    oracle.sparse_attn(q, kv, swa, [one.swa_pos0], q_pos, sink, idx, 1 / math.sqrt(D))
+    if with_hca:
+        Nh = one.ctx // 128
+        oracle.compress_hca(g("hC", (1, 128, D)), g("hZ", (1, 128, D)))
+        oracle.hca_attn(g("hq", (1, 1, H, D)), g("hkv", (1, Nh, D)), g("hswa", (1, one.W, D)), [one.swa_pos0],
+                        q_pos, f32("hsink", (H,)), 1 / math.sqrt(D))
+    return time.perf_counter() - t0
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def oracle_baseline(wl, index, with_hca, budget_s=12.0, max_tokens=24):
+    """Oracle tokens/s on a bounded sample: whole single-sequence decode steps (one token
+    each, seeds 1000+) until about budget_s of oracle time.  Single-threaded C."""
+    times = []
+    while sum(times) < budget_s and len(times) < max_tokens:
+        times.append(oracle_decode_token(wl, 1000 + len(times), index, with_hca))
+    return {"value": len(times) / sum(times), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(times)} single-sequence decode tokens of the {wl.name} step (one sequence of the "
+                      f"B={wl.B} batch each), {sum(times):.1f} s of single-threaded fp64 C oracle on "
+                      f"{cpu_model()}"}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="flash64k", choices=["flash64k", "pro1m"])
+    ap.add_argument("--index", default="e4m3", choices=["e4m3", "bf16"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the pro1m measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_env()
+    with_hca = args.workload == "flash64k"
+
+    if args.impl == "reference":
+        # the reference arm is the CPU oracle, on rank 0 only
+        if rank != 0:
+            return
+        from long_context_compressed_b200 import synth
+        wl = synth.WORKLOADS[args.workload]
+        budget = 150.0
+        per = oracle_decode_token(wl, 999, args.index, with_hca)     # calibration, untimed
+        steps = max(1, min(args.steps, int(budget / max(per, 1e-3))))
+        for i in range(min(args.warmup, 3)):
+            oracle_decode_token(wl, 900 + i, args.index, with_hca)
+        times = [oracle_decode_token(wl, 1000 + i, args.index, with_hca) for i in range(steps)]
+        v = steps / sum(times)
+        line = {"impl": "reference", "metric": "CSA decode tokens/s (64K Flash CSA+HCA layer pair)",
+                "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * sum(times) / steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"{wl.name}: B={wl.B} decode, ctx {wl.ctx}, N={wl.N}, top-{wl.topk}, "
+                                       f"H={wl.H}, D={wl.D}, index {args.index}" + (" + HCA layer" if with_hca else ""),
+                           "sample": "one sequence per step"},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                 "sample": f"{steps} steps of one single-sequence decode token each "
+                                           f"(capped from {args.steps} to stay within minutes) on {cpu_model()}"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    init_dist(world, "nccl")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import __graft_entry__
+    __graft_entry__.build()
+    from long_context_compressed_b200 import csa  # noqa: F401  (fails loudly if libcsa.so is missing)
+
+    peak, peak_kind = measured_peaks()
+    sampler = ClockSampler(local)
+    main_res = bench_workload(args.workload, args.index, with_hca, args.steps, args.warmup, world, device)
+    clocks = sampler.stop()
+    extra = None
+    if not args.no_extra and args.workload != "pro1m":
+        extra = bench_workload("pro1m", args.index, False, args.steps, args.warmup, world, device)
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(main_res["wl"], args.index, with_hca)
+    if rank != 0:
+        return
+
+    def summarise(r):
+        wl = r["wl"]
+        tok = r["tokens_per_step"] * world
+        steps = args.steps
+        idx_gbs = r["index_bytes"] / (r["index_ms"] * 1e-3) / 1e9
+        step_gbs = r["step_bytes"] / (r["step_ms"] * 1e-3) / 1e9
+        return {
+            "value": tok * steps / r["seconds"], "ms_per_step": r["step_ms"],
+            "e2e": {"value": tok * steps / r["e2e_seconds"], "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "roofline": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if args.index == "e4m3"
+                         else "index_tc_kernel (csa_index_scores, bf16)",
+                         "achieved": idx_gbs, "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak,
+                         "peak_source": peak_kind, "traffic": None, "bytes_per_launch": r["index_bytes"],
+                         "avg_launch_us": r["index_ms"] * 1e3},
+            "step_roofline": {"bytes_per_step": r["step_bytes"], "achieved_gbs": step_gbs, "frac": step_gbs / peak,
+                              "floor_us": r["step_bytes"] / (peak * 1e9) * 1e6},
+            "indexer_keys_per_s": wl.B * wl.T * wl.N * world * steps / r["seconds"],
+            "gpu_launches": r["launches"] * steps, "launches_per_step": r["launches"], "input_sets": r["sets"],
+        }
+
+    m = summarise(main_res)
+    wl = main_res["wl"]
+    line = {
+        "metric": "CSA decode tokens/s (64K Flash CSA+HCA layer pair)" if with_hca else
+                  "CSA decode tokens/s (1M Pro CSA layer)",
+        "value": m["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16+e4m3" if args.index == "e4m3" else "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={wl.B} decode tokens/GPU at ctx {wl.ctx}; CSA layer (compress 4:1 "
+                               f"c=512+128, {args.index} index over N={wl.N}, top-{wl.topk}"
+                               + (" via 2k rerank" if args.index == "e4m3" else "") +
+                               f", sparse_attn H={wl.H} D={wl.D})" + (" + HCA layer (compress 128:1, hca_attn over "
+                               f"{wl.ctx // 128}+128 rows)" if with_hca else ""),
+                   "l2": f"{m['input_sets']} rotating input sets, > 2x L2 touched between reuses",
+                   "parallelism": f"replicas x{world}"},
+        "e2e": m["e2e"], "roofline": m["roofline"], "step_roofline": m["step_roofline"],
+        "indexer_keys_per_s": m["indexer_keys_per_s"], "gpu_launches": m["gpu_launches"],
+        "launches_per_step": m["launches_per_step"], "clocks": clocks,
+    }
+    if extra is not None:
+        e = summarise(extra)
+        line["pro1m"] = {"value": e["value"], "unit": "tokens/s", "ms_per_step": e["ms_per_step"],
+                         "step_roofline": e["step_roofline"], "roofline": e["roofline"], "e2e": e["e2e"],
+                         "indexer_keys_per_s": e["indexer_keys_per_s"], "launches_per_step": e["launches_per_step"]}
+        line["gpu_launches"] += e["gpu_launches"]
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

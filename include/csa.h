@@ -175,6 +175,12 @@ int hca_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *s
              int dtype, void *out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * csa_launch_count -- number of kernels this library has enqueued in this
+ * process so far (all devices, all streams; captured launches included).
+ */
+unsigned long long csa_launch_count(void);
+
+/*
  * csa_poll_status -- synchronise `stream`, then return and clear the device
  * status word (CSA_OK, or CSA_ERR_TIMEOUT if a kernel abandoned a bounded
  * wait since the last poll).  CSA_ERR_CUDA if synchronisation fails.

@@ -41,6 +41,7 @@ _SIGS = {
                      _vp, _vp, _sz, _vp], _i32),
     "hca_attn": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                   _vp, _vp, _sz, _vp], _i32),
+    "csa_launch_count": ([], ctypes.c_ulonglong),
     "csa_poll_status": ([_vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -206,6 +207,11 @@ def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int =
                          float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream)), "hca_attn")
     return out
+
+
+def csa_launch_count() -> int:
+    """Kernels enqueued by libcsa.so in this process so far."""
+    return int(_lib.csa_launch_count())
 
 
 def csa_poll_status(stream=None) -> int:

@@ -7,9 +7,11 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/csa.h"
 #include "attn.cuh"
@@ -42,14 +44,42 @@ int sm_count() {
   return cache[dev];
 }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+std::atomic<unsigned long long> g_launches{0};
 
-// Raise a kernel's dynamic shared-memory limit once per device.
+// Status of the kernel launches just enqueued (n of them), counted into the
+// library-wide launch counter.
+int launch_status(int n = 1) {
+  if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA;
+  g_launches += (unsigned long long)n;
+  return CSA_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit; the attribute is set once per
+// (kernel, device) and only raised afterwards, so a call made during stream
+// capture after a first eager call issues no runtime call.
 template <typename K>
 bool set_smem(K kernel, int bytes) {
+  struct Grant {
+    const void* fn;
+    int dev, bytes;
+  };
   static std::mutex mu;
+  static std::vector<Grant> granted;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const void* fn = reinterpret_cast<const void*>(kernel);
   std::lock_guard<std::mutex> lock(mu);
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+  for (Grant& g : granted)
+    if (g.fn == fn && g.dev == dev) {
+      if (g.bytes >= bytes) return true;
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+      g.bytes = bytes;
+      return true;
+    }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  granted.push_back({fn, dev, bytes});
+  return true;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -405,6 +435,8 @@ int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* s
   const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + N;
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
+
+unsigned long long csa_launch_count(void) { return g_launches.load(); }
 
 int csa_poll_status(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CSA_ERR_CUDA;
