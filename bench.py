@@ -170,11 +170,8 @@ class DecodeSet:
         self.scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         self.q8 = torch.empty((B, T, 64, 128), dtype=torch.uint8, device=dev)
         self.qs = torch.empty((B, T, 64), dtype=torch.float32, device=dev)
-        kc = 2 * k if index == "e4m3" else k
-        self.cand = torch.empty((B, T, kc), dtype=torch.int32, device=dev)
-        self.cand_scores = torch.empty((B, T, kc), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
-        self.topk_ws = csa.topk_workspace(B, T, N, kc, dev)
+        self.select_ws = csa.select_workspace(B, N, dev)
         self.attn_ws = csa.attn_workspace(B, T, H, D, 128 + k, device=dev)
         self.out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
         if with_hca:
@@ -235,42 +232,59 @@ class DecodeSet:
         if copies:
             for n, t in x.items():
                 t.copy_(self.host_in[n], non_blocking=True)
-        side_stream.wait_stream(main)
-        # compressors and the HCA layer run on the side stream (independent of the indexer chain)
-        with torch.cuda.stream(side_stream):
-            csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"], ratio=4,
-                             out=self.comp_kv)
-            if wl.comp_ci:
-                csa.csa_compress(x["iC_a"], x["iC_b"], x["iZ_a"], x["iZ_b"], x["iprev_Cb"], x["iprev_Zb"], ratio=4,
-                                 out=self.comp_ki)
-            if self.with_hca:
-                csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=self.hcomp)
-                csa.hca_attn(x["hq"], self.hkv, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
-                             1.0 / math.sqrt(wl.D), out=self.hout, workspace=self.hattn_ws)
-        if timing_events:
-            self.ev = (torch.cuda.Event(enable_timing=True, external=True),
-                       torch.cuda.Event(enable_timing=True, external=True))
+        def side_branch():
+            # compressors and the HCA layer: independent of the indexer chain, so they run
+            # on a side stream, started once the bandwidth-bound indexer is done and
+            # overlapping the latency-bound top-k / rerank / attention kernels
+            side_stream.wait_stream(main)
+            with torch.cuda.stream(side_stream):
+                csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"], ratio=4,
+                                 out=self.comp_kv)
+                if wl.comp_ci:
+                    csa.csa_compress(x["iC_a"], x["iC_b"], x["iZ_a"], x["iZ_b"], x["iprev_Cb"], x["iprev_Zb"],
+                                     ratio=4, out=self.comp_ki)
+                if self.with_hca:
+                    csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=self.hcomp)
+                    csa.hca_attn(x["hq"], self.hkv, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
+                                 1.0 / math.sqrt(wl.D), out=self.hout, workspace=self.hattn_ws)
+        # stage boundaries on the main stream (event record nodes inside the graph)
+        # timing_events: False, "index" (only around the indexer: the timed graphs) or "all"
+        # (every stage: a diagnostic graph; the event nodes cost programmatic-launch overlap)
+        marks = []
+
+        def mark(name):
+            if timing_events == "all" or (timing_events == "index" and name in ("quantize_q", "start", "index")):
+                ev = torch.cuda.Event(enable_timing=True, external=True)
+                ev.record()
+                marks.append((name, ev))
+        mark("start")
         if self.index == "e4m3":
             csa.csa_quantize_e4m3(x["qI"], codes=self.q8, scale=self.qs)
-            if timing_events:
-                self.ev[0].record()
+            mark("quantize_q")
             csa.csa_index_scores(self.q8, x["w"], self.k8, self.n_valid, q_scale=self.qs, k_scale=self.ks,
-                                 scores=self.scores)
-            if timing_events:
-                self.ev[1].record()
-            csa.csa_topk(self.scores, self.n_valid, 2 * wl.topk, idx=self.cand, workspace=self.topk_ws)
-            csa.csa_index_rerank(x["qI"], x["w"], self.kI, self.cand, wl.topk, cand_scores=self.cand_scores,
-                                 idx=self.idx)
+                                 scores=self.scores, select_ws=self.select_ws)
+            mark("index")
+            side_branch()
+            # top-2k bin of the e4m3 scores, exact bf16 rescoring, best k -- one launch
+            csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, kc=2 * wl.topk, qI=x["qI"],
+                                w=x["w"], kI=self.kI, idx=self.idx)
+            mark("select")
         else:
-            if timing_events:
-                self.ev[0].record()
-            csa.csa_index_scores(x["qI"], x["w"], self.kI, self.n_valid, scores=self.scores)
-            if timing_events:
-                self.ev[1].record()
-            csa.csa_topk(self.scores, self.n_valid, wl.topk, idx=self.idx, workspace=self.topk_ws)
+            csa.csa_index_scores(x["qI"], x["w"], self.kI, self.n_valid, scores=self.scores,
+                                 select_ws=self.select_ws)
+            mark("index")
+            side_branch()
+            csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, idx=self.idx)
+            mark("select")
         csa.sparse_attn(x["q"], self.kv, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
                         1.0 / math.sqrt(wl.D), out=self.out, workspace=self.attn_ws)
+        mark("sparse_attn")
         main.wait_stream(side_stream)
+        mark("join")
+        if timing_events:
+            self.marks = marks
+            names = [n for n, _ in marks]
+            self.ev = (marks[names.index("index") - 1][1], marks[names.index("index")][1])
         if copies:
             for h, o in zip(self.host_out, self.outputs):
                 h.copy_(o, non_blocking=True)
@@ -324,13 +338,25 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     n_sets = n_sets or max(2, math.ceil(2 * L2_BYTES / touched) + 1)
     sets = [probe] + [DecodeSet(wl, s, index, with_hca, device) for s in range(1, n_sets)]
     side = torch.cuda.Stream(device=device)
-    graphs, launches = capture(sets, side, timing_events=True)
+    graphs, launches = capture(sets, side, timing_events="index")
     t = timed_replays(graphs, steps, warmup, world)
     t = max_over_ranks(t, world, device)
     try:
         idx_ms = [s.ev[0].elapsed_time(s.ev[1]) for s in sets]
     except RuntimeError:
         idx_ms = [float("nan")]
+    # per-stage breakdown from a separate diagnostic graph with events between all stages
+    diag, _ = capture(sets, side, timing_events="all")
+    timed_replays(diag, min(steps, 200), 5, world)
+    breakdown = {}
+    try:
+        for s in sets:
+            for (n0, e0), (n1, e1) in zip(s.marks[:-1], s.marks[1:]):
+                breakdown.setdefault(n1, []).append(1e3 * e0.elapsed_time(e1))
+        breakdown = {k: round(statistics.mean(v), 2) for k, v in breakdown.items()}
+    except RuntimeError:
+        breakdown = {}
+    del diag
     # end to end: the same step with its inputs copied in from pinned host memory and its
     # outputs read back, inside every timed step
     e2e_graphs, _ = capture(sets, side, copies=True)
@@ -339,10 +365,62 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     h2d, d2h = probe.per_step_io()
     res = {"wl": wl, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
            "index_ms": statistics.mean(idx_ms), "index_bytes": probe.index_bytes(), "step_bytes": touched,
-           "e2e_seconds": t_e2e, "h2d": h2d, "d2h": d2h, "tokens_per_step": wl.B * wl.T}
+           "e2e_seconds": t_e2e, "h2d": h2d, "d2h": d2h, "tokens_per_step": wl.B * wl.T,
+           "breakdown": breakdown}
     del graphs, e2e_graphs, sets
     torch.cuda.empty_cache()
     return res
+
+
+STAGES = ("compress", "quantize", "index", "select", "attn", "hcompress", "hca")
+
+
+def run_stage(name, stage, index, steps, warmup, device):
+    """One stage of the step (one ABI call), eagerly, for profiling a single kernel.
+    Prints the mean device time per call measured with CUDA events."""
+    import torch
+
+    from long_context_compressed_b200 import csa, synth
+    wl = synth.WORKLOADS[name]
+    st = DecodeSet(wl, 0, index, name == "flash64k", device)
+    x = st.inputs
+    calls = {
+        "compress": lambda: csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"],
+                                             ratio=4, out=st.comp_kv),
+        "quantize": lambda: csa.csa_quantize_e4m3(x["qI"], codes=st.q8, scale=st.qs),
+        "index": (lambda: csa.csa_index_scores(st.q8, x["w"], st.k8, st.n_valid, q_scale=st.qs, k_scale=st.ks,
+                                               scores=st.scores)) if index == "e4m3" else
+                 (lambda: csa.csa_index_scores(x["qI"], x["w"], st.kI, st.n_valid, scores=st.scores)),
+        "select": (lambda: (csa.csa_score_histogram(st.scores, st.n_valid, st.select_ws),
+                            csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws, kc=2 * wl.topk,
+                                                qI=x["qI"], w=x["w"], kI=st.kI, idx=st.idx)))
+                  if index == "e4m3" else
+                  (lambda: (csa.csa_score_histogram(st.scores, st.n_valid, st.select_ws),
+                            csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws, idx=st.idx))),
+        "attn": lambda: csa.sparse_attn(x["q"], st.kv, st.swa, st.swa_pos0, st.q_pos, st.sink, st.idx,
+                                        1.0 / math.sqrt(wl.D), out=st.out, workspace=st.attn_ws),
+        "hcompress": lambda: csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=st.hcomp),
+        "hca": lambda: csa.hca_attn(x["hq"], st.hkv, st.hswa, st.swa_pos0, st.q_pos, st.hsink,
+                                    1.0 / math.sqrt(wl.D), out=st.hout, workspace=st.hattn_ws),
+    }
+    # inputs of the later stages come from the earlier ones
+    order = ["quantize", "index", "select"] if index == "e4m3" else ["index", "select"]
+    if stage in ("select", "attn"):
+        for pre in order[:order.index(stage)] if stage in order else order:
+            calls[pre]()
+    fn = calls[stage]
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    assert csa.csa_poll_status() == csa.CSA_OK
+    print(json.dumps({"stage": stage, "workload": name, "index": index, "steps": steps,
+                      "us_per_call": 1e3 * a.elapsed_time(b) / steps}), flush=True)
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) leg
@@ -419,6 +497,7 @@ def main():
     ap.add_argument("--index", default="e4m3", choices=["e4m3", "bf16"])
     ap.add_argument("--no-extra", action="store_true", help="skip the pro1m measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=STAGES, help="time one stage alone (eager calls), e.g. under ncu")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_env()
@@ -461,6 +540,9 @@ def main():
     __graft_entry__.build()
     from long_context_compressed_b200 import csa  # noqa: F401  (fails loudly if libcsa.so is missing)
 
+    if args.stage:
+        run_stage(args.workload, args.stage, args.index, args.steps, args.warmup, device)
+        return
     peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
     main_res = bench_workload(args.workload, args.index, with_hca, args.steps, args.warmup, world, device)
@@ -493,6 +575,7 @@ def main():
                               "floor_us": r["step_bytes"] / (peak * 1e9) * 1e6},
             "indexer_keys_per_s": wl.B * wl.T * wl.N * world * steps / r["seconds"],
             "gpu_launches": r["launches"] * steps, "launches_per_step": r["launches"], "input_sets": r["sets"],
+            "breakdown_us": r["breakdown"],
         }
 
     m = summarise(main_res)
@@ -513,12 +596,14 @@ def main():
         "e2e": m["e2e"], "roofline": m["roofline"], "step_roofline": m["step_roofline"],
         "indexer_keys_per_s": m["indexer_keys_per_s"], "gpu_launches": m["gpu_launches"],
         "launches_per_step": m["launches_per_step"], "clocks": clocks,
+        "breakdown_us_diagnostic": m["breakdown_us"],
     }
     if extra is not None:
         e = summarise(extra)
         line["pro1m"] = {"value": e["value"], "unit": "tokens/s", "ms_per_step": e["ms_per_step"],
                          "step_roofline": e["step_roofline"], "roofline": e["roofline"], "e2e": e["e2e"],
-                         "indexer_keys_per_s": e["indexer_keys_per_s"], "launches_per_step": e["launches_per_step"]}
+                         "indexer_keys_per_s": e["indexer_keys_per_s"], "launches_per_step": e["launches_per_step"],
+                         "breakdown_us": e["breakdown_us"]}
         line["gpu_launches"] += e["gpu_launches"]
     if cpu is not None:
         line["cpu_baseline"] = cpu

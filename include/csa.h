@@ -101,11 +101,15 @@ int csa_quantize_e4m3(const void *x, int x_dtype, int64_t rows, int cols, uint8_
  *   k_scale : [B, N] fp32 (E4M3 only, else NULL)
  *   n_valid : [B, T] int32, 0 <= n_valid <= N (visible complete entries, (t+1)/4)
  *   scores  : [B, T, N] fp32
+ *   select_ws : NULL, or (T == 1 only) a csa_topk_select workspace: the call then
+ *               also accumulates each row's 4096-bin histogram of its valid scores
+ *               there, to be consumed by the next csa_topk_select on that workspace.
  * BF16 / E4M3 run on tcgen05 tensor cores (fp32 accumulation); F32 runs on
  * the fp32 FMA pipes.
  */
 int csa_index_scores(const void *qI, const float *q_scale, const float *w, const void *kI, const float *k_scale,
-                     int dtype, const int32_t *n_valid, int B, int T, int64_t N, float *scores, void *stream);
+                     int dtype, const int32_t *n_valid, int B, int T, int64_t N, float *scores, void *select_ws,
+                     void *stream);
 
 /*
  * csa_topk -- top-k of each score row ([HA] §4.2 / §7 topk(scores, k);
@@ -141,6 +145,34 @@ int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t 
  */
 int csa_index_rerank(const void *qI, const float *w, const void *kI, int dtype, const int32_t *cand, int kc, int B,
                      int T, int64_t N, int k, float *cand_scores, int32_t *idx, void *stream);
+
+/*
+ * csa_topk_select -- decode top-k in one launch, fed by the histogram that
+ * csa_index_scores(..., select_ws) accumulated ([HA] §4.2 / §7 topk; §9: the
+ * indexer forms its candidates at twice top-k).  One query per sequence (T == 1):
+ * scores [B, N] fp32, n_valid [B] int32, idx [B, k] int32.
+ *   qI == NULL : idx = the exact top-k of each row (as csa_topk).
+ *   qI != NULL : candidates = every index whose score lies in the histogram bin of
+ *                the kc-th largest score or above (a superset of the kc largest);
+ *                each is rescored with the plain indexer definition on the
+ *                full-precision qI [B, 64, 128] / kI [B, N, 128] (dtype F32 or BF16)
+ *                and w [B, 64], and idx = the k best rescored candidates.
+ *   Ties go to the lower index; rows are ascending and -1 padded (n_valid < k).
+ *   k <= CSA_MAX_TOPK, k <= kc, N <= 2^19.
+ *   workspace : csa_select_workspace_size(B, N) bytes, 16-byte aligned, ZERO-FILLED
+ *               before first use; csa_index_scores(..., workspace) fills the
+ *               histograms and this call consumes them and leaves the workspace
+ *               ready (zeroed histograms) for the next pair of calls.
+ */
+size_t csa_select_workspace_size(int B, int64_t N);
+/* csa_score_histogram -- accumulate the per-row histogram of scores [B, N] (entries
+ * i < n_valid[b]) into a csa_topk_select workspace, for scores that did not come
+ * from csa_index_scores(..., select_ws). */
+int csa_score_histogram(const float *scores, const int32_t *n_valid, int B, int64_t N, void *workspace,
+                        size_t ws_bytes, void *stream);
+int csa_topk_select(const float *scores, const int32_t *n_valid, int B, int64_t N, int k, int kc, const void *qI,
+                    const float *w, const void *kI, int dtype, int32_t *idx, void *workspace, size_t ws_bytes,
+                    void *stream);
 
 /*
  * sparse_attn -- CSA core attention ([P2] sparse_attn(q, kv, attn_sink,

@@ -32,7 +32,10 @@ _SIGS = {
     "csa_version": ([], _i32),
     "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
-    "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp], _i32),
+    "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
+    "csa_select_workspace_size": ([_i32, _i64], _sz),
+    "csa_score_histogram": ([_vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
+    "csa_topk_select": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp], _i32),
     "csa_index_rerank": ([_vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_topk_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "csa_topk": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
@@ -119,16 +122,52 @@ def csa_quantize_e4m3(x, codes=None, scale=None, stream=None):
     return codes, scale
 
 
-def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=None, stream=None):
+def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=None, select_ws=None,
+                     stream=None):
     """Indexer scores.  qI [B, T, 64, 128] (fp32 | bf16 | uint8 e4m3 codes), w [B, T, 64] fp32,
-    kI [B, N, 128] same dtype, n_valid [B, T] int32 -> scores [B, T, N] fp32."""
+    kI [B, N, 128] same dtype, n_valid [B, T] int32 -> scores [B, T, N] fp32.  With select_ws
+    (T == 1) the per-row score histogram for csa_topk_select is accumulated there."""
     B, T = qI.shape[0], qI.shape[1]
     N = kI.shape[1]
     if scores is None:
         scores = torch.empty((B, T, N), dtype=torch.float32, device=qI.device)
     _check(_lib.csa_index_scores(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), _dtype_code(qI),
-                                 _ptr(n_valid), B, T, N, _ptr(scores), _stream(stream)), "csa_index_scores")
+                                 _ptr(n_valid), B, T, N, _ptr(scores), _ptr(select_ws), _stream(stream)),
+           "csa_index_scores")
     return scores
+
+
+def csa_select_workspace_size(B: int, N: int) -> int:
+    return int(_lib.csa_select_workspace_size(B, N))
+
+
+def select_workspace(B: int, N: int, device="cuda") -> torch.Tensor:
+    """A zero-filled csa_topk_select workspace (the library keeps it ready between call pairs)."""
+    return torch.zeros(max(16, csa_select_workspace_size(B, N)), dtype=torch.uint8, device=device)
+
+
+def csa_score_histogram(scores, n_valid, workspace, stream=None):
+    """Accumulate the per-row score histogram of scores [B, (1,) N] into a select workspace."""
+    B, N = scores.shape[0], scores.shape[-1]
+    _check(_lib.csa_score_histogram(_ptr(scores), _ptr(n_valid), B, N, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "csa_score_histogram")
+
+
+def csa_topk_select(scores, n_valid, k: int, workspace, *, kc=None, qI=None, w=None, kI=None, idx=None,
+                    stream=None):
+    """Decode top-k from the histogram csa_index_scores(select_ws=workspace) accumulated.
+    scores [B, 1, N] (or [B, N]), n_valid [B, 1] -> idx [B, 1, k].  With qI/w/kI (full precision)
+    the candidates of the kc-th score's bin are rescored exactly and the best k kept."""
+    B, N = scores.shape[0], scores.shape[-1]
+    if idx is None:
+        idx = torch.empty((B, 1, k), dtype=torch.int32, device=scores.device)
+    kc = k if kc is None else kc
+    dt = _dtype_code(qI) if qI is not None else CSA_F32
+    _check(_lib.csa_topk_select(_ptr(scores), _ptr(n_valid), B, N, k, kc, _ptr(qI), _ptr(w), _ptr(kI), dt, _ptr(idx),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "csa_topk_select")
+    return idx
 
 
 def csa_index_rerank(qI, w, kI, cand, k: int, *, cand_scores=None, idx=None, stream=None):

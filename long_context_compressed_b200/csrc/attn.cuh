@@ -105,6 +105,7 @@ __device__ __forceinline__ int64_t row_offset(const AttnParams& p, const RowList
 // row with logit sink_h and value 0 (initial state m = sink, l = 1, o = 0).
 template <int DPL>  // dims per lane
 __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
+  griddep_sync();
   const int h = blockIdx.x * 4 + warp_id();
   const int t = blockIdx.y, b = blockIdx.z;
   if (h >= p.H) return;
@@ -155,7 +156,6 @@ struct AttnCfg {
   static constexpr int DH = (D > 256) ? 256 : D;           // D-slice per CTA
   static constexpr int NDH = D / DH;
   static constexpr int kAtoms = D / 64;                    // 128-byte atoms per row
-  static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = R * D * 2;
   static constexpr int kPRowBytes = R * 2;                 // 64 (SW64) or 128 (SW128)
   static constexpr int kPBytes = 128 * kPRowBytes;
@@ -164,7 +164,20 @@ struct AttnCfg {
   static constexpr int kTmemCols = (DH + 2 * R) <= 256 ? 256 : 512;  // O slice + two S buffers
   static constexpr int kSCol0 = DH;                        // S buffers after O
   static constexpr int kThreads = 288;                     // 4 softmax + 4 loader + 1 MMA warps
-  static constexpr int kSmem = kQBytes + 2 * kKVBytes + 2 * kPBytes + 1024 + 256;
+  static constexpr int kMaxStages = 4;
+  static constexpr int kMaxCtaRows = 2048;                 // index values staged per CTA (larger lists stream)
+  static constexpr int kBarBytes = 256 + 4 * kMaxCtaRows;
+  // Q rows held per 64-dim atom: 64 when H <= 64 (compact), else 128
+  static __host__ __device__ int q_rows(int H) { return H <= 64 ? 64 : 128; }
+  static __host__ __device__ int q_bytes(int H) { return q_rows(H) * D * 2; }
+  static __host__ __device__ int stages(int H) {
+    const int avail = 232448 - 1024 - kBarBytes - q_bytes(H) - 2 * kPBytes;
+    const int n = avail / kKVBytes;
+    return n >= kMaxStages ? kMaxStages : n;
+  }
+  static __host__ __device__ int smem(int H) {
+    return 1024 + q_bytes(H) + stages(H) * kKVBytes + 2 * kPBytes + kBarBytes;
+  }
 };
 
 // Byte offset of 16-byte chunk c of row r in a K-major tile with 128-byte
@@ -173,50 +186,54 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
   return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// Q [B*T, H, D] is loaded by TMA as D/64 boxes of {64 dims, QR rows}.  With
+// QR = 64 (H <= 64) the M = 128 MMA operand of atom a also spans the first 64
+// rows of atom a+1 (or, for the last atom, the next 8 KB of shared memory):
+// finite values whose result rows (>= H) are never used.
 template <int D>
-__global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                           const AttnParams p) {
   using Cfg = AttnCfg<D>;
   constexpr int R = Cfg::R, DH = Cfg::DH;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int QR = Cfg::q_rows(p.H);
+  const int NS = Cfg::stages(p.H);
   uint8_t* q_s = smem;
-  uint8_t* kv_s = q_s + Cfg::kQBytes;                       // [2][kKVBytes]
-  uint8_t* p_s = kv_s + 2 * Cfg::kKVBytes;                  // [2][kPBytes]
+  uint8_t* kv_s = q_s + Cfg::q_bytes(p.H);                  // [NS][kKVBytes]
+  uint8_t* p_s = kv_s + NS * Cfg::kKVBytes;                 // [2][kPBytes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Cfg::kPBytes);
-  uint64_t* full = bars;        // [2] KV stage loaded (128 cp.async arrivals + 1 mask arrival)
-  uint64_t* empty = bars + 2;   // [2] KV stage consumed by PV
-  uint64_t* sfull = bars + 4;   // [2] S ready
-  uint64_t* sfree = bars + 6;   // [2] S read by softmax
-  uint64_t* pfull = bars + 8;   // [2] P written
-  uint64_t* pdone = bars + 10;  // [2] PV done (P buffer free, O consistent)
-  uint64_t* qfull = bars + 12;
-  uint64_t* odone = bars + 13;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
-  uint64_t* mask_s = bars + 16;  // [2] validity of the tile's rows
+  uint64_t* full = bars;        // [4] KV stage loaded (128 cp.async arrivals)
+  uint64_t* empty = bars + 4;   // [4] KV stage consumed by PV
+  uint64_t* sfull = bars + 8;   // [2] S ready
+  uint64_t* sfree = bars + 10;  // [2] S read by softmax
+  uint64_t* pfull = bars + 12;  // [2] P written
+  uint64_t* pdone = bars + 14;  // [2] PV done (P buffer free, O consistent)
+  uint64_t* qfull = bars + 16;
+  uint64_t* odone = bars + 17;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 20);      // [4 stages][4 loader warps]
+  int32_t* idx_s = reinterpret_cast<int32_t*>(bars + 32);         // [kMaxCtaRows] raw index values
 
   const int qi = blockIdx.z;                 // b * T + t
   const int b = qi / p.T, t = qi % p.T;
   const int dh = blockIdx.y;
   const int split = blockIdx.x;
-  const RowList rl = make_row_list(p, b, t);
-  const int n_rows = rl.n_swa + rl.n_mem;
-  const int n_tiles_all = (n_rows + R - 1) / R;
-  const int tps = (n_tiles_all + p.nsplit - 1) / p.nsplit;
-  const int j0 = split * tps;
-  const int j1 = min(n_tiles_all, j0 + tps);
-  const int nt = j1 > j0 ? j1 - j0 : 0;      // tiles of this CTA
   const int warp = warp_id();
+  const int32_t* idx_row = p.sparse ? p.idx + ((int64_t)b * p.T + t) * p.k : nullptr;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&full[i], 128 + 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&full[i], 128 + 4);          // cp.async of 128 threads + a mask word per loader warp
       mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&sfree[i], 4);
       mbar_init(&pfull[i], 4);
       mbar_init(&pdone[i], 1);
     }
-    mbar_init(qfull, 128);
+    mbar_init(qfull, 1);
     mbar_init(odone, 1);
     fence_mbar_init();
   }
@@ -228,87 +245,125 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  griddep_sync();
+  const RowList rl = make_row_list(p, b, t);
+  const int n_rows = rl.n_swa + rl.n_mem;
+  const int n_tiles_all = (n_rows + R - 1) / R;
+  const int tps = (n_tiles_all + p.nsplit - 1) / p.nsplit;
+  const int j0 = split * tps;
+  const int j1 = min(n_tiles_all, j0 + tps);
+  const int nt = j1 > j0 ? j1 - j0 : 0;      // tiles of this CTA
+  // the index value behind list row rg (only memory rows of sparse_attn read memory)
+  auto fetch_raw = [&](int rg) -> int32_t {
+    if (!p.sparse || rg < rl.n_swa || rg >= n_rows) return 0;
+    return __ldg(idx_row + (rg - rl.n_swa));
+  };
+  // element offset of list row rg given its raw index; -1 if it contributes nothing;
+  // SWA rows are encoded as -2 - offset
+  auto row_src = [&](int rg, int32_t raw) -> int64_t {
+    if (rg >= n_rows) return -1;
+    if (rg < rl.n_swa) return -2 - ((int64_t)b * p.W + rl.swa_row0 + rg) * D;
+    const int64_t i = p.sparse ? (int64_t)raw : (int64_t)(rg - rl.n_swa);
+    if (i < 0 || i >= p.N) return -1;
+    return ((int64_t)b * p.N + i) * D;
+  };
+
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ loaders (128 threads)
     const int lt = threadIdx.x - 128;
     if (nt > 0) {
-      const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q) + (int64_t)qi * p.H * D;
-      for (int c = lt; c < 128 * (D / 8); c += 128) {
-        const int r = c / (D / 8), ch = c % (D / 8);
-        uint8_t* dst = q_s + sw128_off(r, ch, 128);
-        if (r < p.H) cp_async_16(dst, qg + (int64_t)r * D + ch * 8);
-        else st_shared_zero16(dst);
-      }
-      fence_proxy_async_smem();
-      cp_async_arrive_noinc(qfull);
       const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(p.kv);
       const __nv_bfloat16* swa = static_cast<const __nv_bfloat16*>(p.swa);
       constexpr int CPR = D / 8;                 // 16-byte chunks per row
+      constexpr int TPR = 128 / R;               // loader threads per row
+      constexpr int CPT = CPR / TPR;             // chunks per thread and tile
+      const int my_r = lt / TPR, my_c = lt % TPR;
+      // stage this CTA's index values in shared memory once (coalesced), so no
+      // global load sits between the tiles
+      const int row0 = j0 * R, nrow = nt * R;
+      const bool staged = p.sparse && nrow <= Cfg::kMaxCtaRows;
+      if (staged) {
+        for (int r = lt; r < nrow; r += 128) {
+          const int rg = row0 + r;
+          idx_s[r] = (rg >= rl.n_swa && rg < n_rows) ? __ldg(idx_row + (rg - rl.n_swa)) : 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+      int ks = 0;
+      uint32_t kph = 0;
       for (int jj = 0; jj < nt; ++jj) {
-        const int j = j0 + jj;
-        const int s = jj & 1;
-        if (!mbar_wait(&empty[s], ((jj >> 1) & 1) ^ 1)) break;
+        const int rg = (j0 + jj) * R + my_r;
+        const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
+        const int s = ks;
+        const uint32_t ph = kph;
+        if (++ks == NS) { ks = 0; kph ^= 1; }
+        if (!mbar_wait(&empty[s], ph ^ 1)) break;
+        const int64_t src_off = row_src(rg, raw);
+        const __nv_bfloat16* src = src_off >= 0 ? kv + src_off : (src_off <= -2 ? swa + (-2 - src_off) : nullptr);
         uint8_t* tile = kv_s + s * Cfg::kKVBytes;
-        for (int c = lt; c < R * CPR; c += 128) {
-          const int r = c / CPR, ch = c % CPR;
-          const int rg = j * R + r;
-          bool sw = false;
-          const int64_t off = rg < n_rows ? row_offset(p, rl, b, t, rg, &sw) : -1;
-          uint8_t* dst = tile + sw128_off(r, ch, R);
-          if (off >= 0) cp_async_16(dst, (sw ? swa : kv) + off + ch * 8);
+#pragma unroll 4
+        for (int i = 0; i < CPT; ++i) {
+          const int ch = my_c + TPR * i;
+          uint8_t* dst = tile + sw128_off(my_r, ch, R);
+          if (src) cp_async_16(dst, src + ch * 8);
           else st_shared_zero16(dst);                 // finite filler for rows that do not contribute
         }
         fence_proxy_async_smem();
         cp_async_arrive_noinc(&full[s]);
-        if (lt == 0) {
-          // which rows of the tile contribute (read by the softmax warps after full[s])
-          uint64_t valid = 0;
-          for (int r = 0; r < R; ++r) {
-            const int rg = j * R + r;
-            bool sw;
-            if (rg < n_rows && row_offset(p, rl, b, t, rg, &sw) >= 0) valid |= 1ull << r;
-          }
-          mask_s[s] = valid;
+        // validity of this warp's rows (TPR threads per row): one word per loader warp
+        const uint32_t bal = __ballot_sync(0xffffffffu, src != nullptr);
+        if (lane_id() == 0) {
+          uint32_t rows = 0;                          // bit j: row (warp's first row + j)
+          for (int j = 0; j < 32 / TPR; ++j) rows |= ((bal >> (j * TPR)) & 1u) << j;
+          mask_s[s * 4 + (lt >> 5)] = rows;
           mbar_arrive(&full[s]);
         }
       }
     }
   } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Q by TMA, then the MMA issuer
     if (elect_one() && nt > 0) {
+      prefetch_tmap(&qmap);
+      mbar_arrive_expect_tx(qfull, (uint32_t)Cfg::q_bytes(p.H));
+      for (int a = 0; a < Cfg::kAtoms; ++a) tma_load_3d(q_s + a * QR * 128, &qmap, qfull, a * 64, 0, qi);
       const uint32_t idesc_s = make_idesc(128, R, 1, 0, 0);
       const uint32_t idesc_o = make_idesc(128, DH, 1, 0, 1);
       const uint32_t qb = smem_u32(q_s);
       bool ok = mbar_wait(qfull, 0);
-      fence_proxy_async_smem();
       tc_fence_after();
+      int ks = 0;
+      uint32_t kph = 0;
       auto issue_s = [&](int jj) -> bool {
-        const int s = jj & 1;
-        const uint32_t ph = (jj >> 1) & 1;
+        const int sb = jj & 1;
+        const uint32_t sph = (jj >> 1) & 1;
+        const int s = ks;
+        const uint32_t ph = kph;
         if (!mbar_wait(&full[s], ph)) return false;
-        if (!mbar_wait(&sfree[s], ph ^ 1)) return false;
-        fence_proxy_async_smem();
+        if (!mbar_wait(&sfree[sb], sph ^ 1)) return false;
+        fence_proxy_async_smem();                   // cp.async data -> tensor core reads
         tc_fence_after();
         const uint32_t kb = smem_u32(kv_s + s * Cfg::kKVBytes);
-        const uint32_t d = tmem + Cfg::kSCol0 + s * R;
+        const uint32_t d = tmem + Cfg::kSCol0 + sb * R;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int atom = kk >> 2, inner = (kk & 3) * 32;
-          const uint64_t ad = smem_desc(qb + atom * 128 * 128 + inner, 16, 1024, kLayoutSW128);
+          const uint64_t ad = smem_desc(qb + atom * QR * 128 + inner, 16, 1024, kLayoutSW128);
           const uint64_t bd = smem_desc(kb + atom * R * 128 + inner, 16, 1024, kLayoutSW128);
           mma_bf16(d, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sfull[s]);
+        mma_commit(&sfull[sb]);
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int jj = 0; ok && jj < nt; ++jj) {
+        const int s = ks;                           // KV stage of tile jj
+        if (++ks == NS) { ks = 0; kph ^= 1; }
         if (jj + 1 < nt && !issue_s(jj + 1)) { ok = false; break; }
-        const int s = jj & 1;
-        if (!mbar_wait(&pfull[s], (jj >> 1) & 1)) { ok = false; break; }
+        const int sb = jj & 1;
+        if (!mbar_wait(&pfull[sb], (jj >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t pb = smem_u32(p_s + s * Cfg::kPBytes);
+        const uint32_t pb = smem_u32(p_s + sb * Cfg::kPBytes);
         const uint32_t vb = smem_u32(kv_s + s * Cfg::kKVBytes) + dh * (DH / 64) * R * 128;
 #pragma unroll
         for (int kk = 0; kk < R / 16; ++kk) {
@@ -316,7 +371,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
           const uint64_t bd = smem_desc(vb + kk * 2048, R * 128, 1024, kLayoutSW128);
           mma_bf16(tmem, ad, bd, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&pdone[s]);
+        mma_commit(&pdone[sb]);
         mma_commit(&empty[s]);
       }
       mma_commit(odone);
@@ -329,35 +384,46 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     const float zs = p.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    // validity of the tile's rows: lane r (and r + 32) checks row r of the tile; the
+    // index value is fetched one tile ahead and a warp ballot gives every thread the mask
+    int ks = 0;
+    uint32_t kph = 0;
+    constexpr int RPW = R / 4;                 // tile rows covered by one loader warp
     for (int jj = 0; jj < nt; ++jj) {
-      const int s = jj & 1;
+      const int sb = jj & 1;
       const uint32_t ph = (jj >> 1) & 1;
-      if (!mbar_wait(&full[s], ph) || !mbar_wait(&sfull[s], ph)) { ok = false; break; }
+      const int s = ks;
+      const uint32_t kp = kph;
+      if (++ks == NS) { ks = 0; kph ^= 1; }
+      // the loaders' row-validity words for this tile (published with full[s])
+      if (!mbar_wait(&full[s], kp)) { ok = false; break; }
+      uint64_t valid = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) valid |= (uint64_t)(mask_s[s * 4 + w] & ((1ull << RPW) - 1)) << (w * RPW);
+      if (!mbar_wait(&sfull[sb], ph)) { ok = false; break; }
       tc_fence_after();
-      const uint64_t valid = mask_s[s];
       float z[R];
-      tmem_ld32(tmem + lane_base + Cfg::kSCol0 + s * R, z);
-      if constexpr (R == 64) tmem_ld32(tmem + lane_base + Cfg::kSCol0 + s * R + 32, z + 32);
+      tmem_ld32(tmem + lane_base + Cfg::kSCol0 + sb * R, z);
+      if constexpr (R == 64) tmem_ld32(tmem + lane_base + Cfg::kSCol0 + sb * R + 32, z + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane_id() == 0) mbar_arrive(&sfree[s]);
+      if (lane_id() == 0) mbar_arrive(&sfree[sb]);
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < R; ++c) {
         z[c] = ((valid >> c) & 1) ? z[c] * zs : -INFINITY;
         mt = fmaxf(mt, z[c]);
       }
-      // P buffer s is free once PV of tile jj-2 completed
-      if (!mbar_wait(&pdone[s], ph ^ 1)) { ok = false; break; }
+      // P buffer sb is free once PV of tile jj-2 completed
+      if (!mbar_wait(&pdone[sb], ph ^ 1)) { ok = false; break; }
       if (mt > m_used + 8.f) {
         const float m_new = mt;
         if (m_used != -INFINITY && jj > 0) {
           // O must be consistent: PV of tile jj-1 completed
-          const int ps = (jj - 1) & 1;
-          if (!mbar_wait(&pdone[ps], ((jj - 1) >> 1) & 1)) { ok = false; break; }
+          if (!mbar_wait(&pdone[(jj - 1) & 1], ((jj - 1) >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
-          const float f = exp2f(m_used - m_new);
+          const float f = ex2_approx(m_used - m_new);
           for (int c0 = 0; c0 < DH; c0 += 32) {
             float o[32];
             tmem_ld32(tmem + lane_base + c0, o);
@@ -371,18 +437,21 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         }
         m_used = m_new;
       }
-      float psum = 0.f;
+      // p = 2^(z - m); rows with no valid column so far keep m = -inf and p = 0
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      float ps0 = 0.f, ps1 = 0.f;
       uint32_t packed[R / 2];
 #pragma unroll
       for (int c = 0; c < R; c += 2) {
-        const float p0 = (m_used == -INFINITY) ? 0.f : exp2f(z[c] - m_used);
-        const float p1 = (m_used == -INFINITY) ? 0.f : exp2f(z[c + 1] - m_used);
-        psum += p0 + p1;
+        const float p0 = ex2_approx(z[c] - mref);        // z = -inf (masked) -> 0
+        const float p1 = ex2_approx(z[c + 1] - mref);
+        ps0 += p0;
+        ps1 += p1;
         __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
         packed[c / 2] = *reinterpret_cast<uint32_t*>(&v);
       }
-      l += psum;
-      uint8_t* prow = p_s + s * Cfg::kPBytes + h * Cfg::kPRowBytes;
+      l += ps0 + ps1;
+      uint8_t* prow = p_s + sb * Cfg::kPBytes + h * Cfg::kPRowBytes;
 #pragma unroll
       for (int c = 0; c < R / 8; ++c) {
         const int phys = (R == 64) ? (c ^ (h & 7)) : (c ^ ((h >> 1) & 3));
@@ -392,60 +461,62 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane_id() == 0) mbar_arrive(&pfull[s]);
+      if (lane_id() == 0) mbar_arrive(&pfull[sb]);
     }
     // ---- epilogue
     const bool have_o = ok && nt > 0 && mbar_wait(odone, 0);
     tc_fence_after();
-    const int64_t orow = ((int64_t)qi * p.H + h) * D + dh * DH;
+    // O rows leave TMEM as 32-column chunks; each warp transposes its 32 x 32 chunk
+    // through shared memory (the KV stages are idle now) so that each store
+    // instruction writes four full 128-byte row segments.
+    float* stage = reinterpret_cast<float*>(kv_s) + warp * 32 * 36;
+    const int hw0 = warp * 32;                 // first head row of this warp
+    float g = 1.f;
     if (p.nsplit == 1) {
       const float M = fmaxf(m_used, sinkL);
       const float fo = (m_used == -INFINITY) ? 0.f : exp2f(m_used - M);
       const float den = l * fo + exp2f(sinkL - M);
-      const float g = fo / den;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_base + c0, o);
-          tmem_wait_ld();
-        } else {
+      g = fo / den;
+    }
+    const int sub = (int)lane_id() >> 3, q4 = ((int)lane_id() & 7) * 4;   // row within a group of 4, column
+    __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + hw0) * D + dh * DH;
+    float* wbase = p.ws_o + (((int64_t)split * p.B * p.T + qi) * p.H + hw0) * D + dh * DH;
+    for (int c0 = 0; c0 < DH; c0 += 32) {
+      float o[32];
+      if (have_o) {
+        tmem_ld32(tmem + lane_base + c0, o);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0.f;
-        }
-        if (h < p.H) {
+        for (int c = 0; c < 32; ++c) o[c] = 0.f;
+      }
+      __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint4 u;
-            __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+      for (int c = 0; c < 32; c += 4)
+        *reinterpret_cast<float4*>(stage + lane_id() * 36 + c) =
+            make_float4(o[c] * g, o[c + 1] * g, o[c + 2] * g, o[c + 3] * g);
+      __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) hv[e] = __floats2bfloat162_rn(o[c + 2 * e] * g, o[c + 2 * e + 1] * g);
-            *reinterpret_cast<uint4*>(out + orow + c0 + c) = u;
+      for (int r4 = 0; r4 < 32; r4 += 4) {
+        const int r = r4 + sub;
+        if (hw0 + r < p.H) {
+          const float4 v = *reinterpret_cast<const float4*>(stage + r * 36 + q4);
+          if (p.nsplit == 1) {
+            __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), bb = __floats2bfloat162_rn(v.z, v.w);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&a);
+            u.y = *reinterpret_cast<uint32_t*>(&bb);
+            *reinterpret_cast<uint2*>(obase + (int64_t)r * D + c0 + q4) = u;
+          } else {
+            *reinterpret_cast<float4*>(wbase + (int64_t)r * D + c0 + q4) = v;
           }
         }
       }
-    } else {
-      float* wo = p.ws_o + (int64_t)split * p.B * p.T * p.H * D;
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_base + c0, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0.f;
-        }
-        if (h < p.H) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(wo + orow + c0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-        }
-      }
-      if (h < p.H && dh == 0) {
-        float* ml = p.ws_ml + (((int64_t)split * p.B * p.T + qi) * p.H + h) * 2;
-        ml[0] = have_o ? m_used : -INFINITY;
-        ml[1] = have_o ? l : 0.f;
-      }
+    }
+    if (p.nsplit > 1 && h < p.H && dh == 0) {
+      float* ml = p.ws_ml + (((int64_t)split * p.B * p.T + qi) * p.H + h) * 2;
+      ml[0] = have_o ? m_used : -INFINITY;
+      ml[1] = have_o ? l : 0.f;
     }
   }
 
@@ -459,12 +530,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
 // sum_s l_s e^(m_s-M); o = sum_s O_s e^(m_s-M) / den  (log2 domain).  One
 // thread per (query, head, 8 dims).
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
-  const int64_t groups = (int64_t)p.B * p.T * p.H * (p.D / 8);
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  griddep_sync();
+  const uint32_t gpr = (uint32_t)(p.D / 8);  // 32-bit index math: B*T*H*D/8 < 2^31 (host-checked)
+  const uint32_t groups = (uint32_t)(p.B * p.T * p.H) * gpr;
+  const uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= groups) return;
-  const int d0 = (int)(g % (p.D / 8)) * 8;
-  const int64_t qh = g / (p.D / 8);         // (b*T + t) * H + h
-  const int h = (int)(qh % p.H);
+  const int d0 = (int)(g % gpr) * 8;
+  const uint32_t qh = g / gpr;               // (b*T + t) * H + h
+  const int h = (int)(qh % (uint32_t)p.H);
   const float sinkL = p.sink[h] * kLog2e;
   const int64_t stride_ml = (int64_t)p.B * p.T * p.H * 2;
   const int64_t stride_o = (int64_t)p.B * p.T * p.H * p.D;

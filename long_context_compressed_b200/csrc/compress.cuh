@@ -58,13 +58,14 @@ __global__ void __launch_bounds__(256) compress_csa_kernel(const Tin* __restrict
                                                            const Tin* __restrict__ pCb,
                                                            const Tin* __restrict__ pZb, int B, int64_t L, int c,
                                                            Tout* __restrict__ out) {
-  const int groups = c >> 3;
-  const int64_t n_entries = L / M;
-  const int64_t total = (int64_t)B * n_entries * groups;
-  for (int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
-       gid += (int64_t)gridDim.x * blockDim.x) {
+  griddep_sync();
+  // 32-bit index arithmetic (the host guarantees B * L/M * c/8 < 2^31)
+  const uint32_t groups = (uint32_t)c >> 3;
+  const uint32_t n_entries = (uint32_t)(L / M);
+  const uint32_t total = (uint32_t)B * n_entries * groups;
+  for (uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x; gid < total; gid += gridDim.x * blockDim.x) {
     const int g = (int)(gid % groups);
-    const int64_t rest = gid / groups;
+    const uint32_t rest = gid / groups;
     const int64_t i = rest % n_entries;
     const int b = (int)(rest / n_entries);
     const int ch = g * 8;
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(256) compress_csa_kernel(const Tin* __restrict
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) compress_hca_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z,
                                                            int B, int64_t L, int c, Tout* __restrict__ out) {
+  griddep_sync();
   constexpr int M = 128;
   constexpr int CH = 8;
   const int groups = c >> 3;

@@ -9,7 +9,9 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
+#include <utility>
 #include <mutex>
 #include <vector>
 
@@ -109,6 +111,33 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Kernel launch with programmatic stream serialization (PDL): the kernel may begin
+// launching while its predecessor in the stream finishes; every kernel of this
+// library waits for the predecessor (griddepcontrol.wait) before touching global
+// memory.  Set CSA_NO_PDL=1 in the environment to launch without the attribute.
+bool use_pdl() {
+  static const bool on = [] {
+    const char* e = getenv("CSA_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------------ attention split policy
 template <int D>
 int attn_rows_per_tile() { return AttnCfg<D>::R; }
@@ -139,11 +168,11 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
   if (dtype == CSA_F32) {
     dim3 grid((p.H + 3) / 4, p.T, p.B);
     switch (p.D) {
-      case 32: csa::attn_f32_kernel<1><<<grid, 128, 0, st>>>(p); break;
-      case 64: csa::attn_f32_kernel<2><<<grid, 128, 0, st>>>(p); break;
-      case 128: csa::attn_f32_kernel<4><<<grid, 128, 0, st>>>(p); break;
-      case 256: csa::attn_f32_kernel<8><<<grid, 128, 0, st>>>(p); break;
-      case 512: csa::attn_f32_kernel<16><<<grid, 128, 0, st>>>(p); break;
+      case 32: launch_k(csa::attn_f32_kernel<1>, grid, 128, 0, st, p); break;
+      case 64: launch_k(csa::attn_f32_kernel<2>, grid, 128, 0, st, p); break;
+      case 128: launch_k(csa::attn_f32_kernel<4>, grid, 128, 0, st, p); break;
+      case 256: launch_k(csa::attn_f32_kernel<8>, grid, 128, 0, st, p); break;
+      case 512: launch_k(csa::attn_f32_kernel<16>, grid, 128, 0, st, p); break;
       default: return CSA_ERR_UNSUPPORTED;
     }
     return launch_status();
@@ -156,25 +185,31 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     p.ws_ml = p.ws_o + (size_t)p.nsplit * p.B * p.T * p.H * p.D;
   }
   dim3 grid(p.nsplit, attn_ndh(p.D), p.B * p.T);
+  // Q [B*T, H, D] by TMA: boxes of {64 dims, 64 or 128 rows}, rows past H zero-filled
+  CUtensorMap qmap;
+  const uint32_t qrows = p.H <= 64 ? 64 : 128;
+  if (!make_map(&qmap, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D, (uint64_t)p.H,
+                (uint64_t)p.B * p.T, 64, qrows))
+    return CSA_ERR_CUDA;
   switch (p.D) {
-    case 128:
-      if (!set_smem(csa::attn_tc_kernel<128>, AttnCfg<128>::kSmem)) return CSA_ERR_CUDA;
-      csa::attn_tc_kernel<128><<<grid, AttnCfg<128>::kThreads, AttnCfg<128>::kSmem, st>>>(p);
-      break;
-    case 256:
-      if (!set_smem(csa::attn_tc_kernel<256>, AttnCfg<256>::kSmem)) return CSA_ERR_CUDA;
-      csa::attn_tc_kernel<256><<<grid, AttnCfg<256>::kThreads, AttnCfg<256>::kSmem, st>>>(p);
-      break;
-    case 512:
-      if (!set_smem(csa::attn_tc_kernel<512>, AttnCfg<512>::kSmem)) return CSA_ERR_CUDA;
-      csa::attn_tc_kernel<512><<<grid, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, st>>>(p);
-      break;
+#define CSA_LAUNCH_ATTN(DD)                                                                       \
+  case DD: {                                                                                      \
+    const int sm = AttnCfg<DD>::smem(p.H);                                                        \
+    if (!set_smem(csa::attn_tc_kernel<DD>, std::max(AttnCfg<DD>::smem(1), AttnCfg<DD>::smem(128))))   \
+      return CSA_ERR_CUDA;                                                                        \
+    launch_k(csa::attn_tc_kernel<DD>, grid, AttnCfg<DD>::kThreads, sm, st, qmap, p);                    \
+    break;                                                                                        \
+  }
+    CSA_LAUNCH_ATTN(128)
+    CSA_LAUNCH_ATTN(256)
+    CSA_LAUNCH_ATTN(512)
+#undef CSA_LAUNCH_ATTN
     default: return CSA_ERR_UNSUPPORTED;
   }
   int rc = launch_status();
   if (rc != CSA_OK || p.nsplit == 1) return rc;
   const int64_t groups = (int64_t)p.B * p.T * p.H * (p.D / 8);
-  csa::attn_combine_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, st>>>(p);
+  launch_k(csa::attn_combine_kernel, (unsigned)((groups + 255) / 256), 256, 0, st, p);
   return launch_status();
 }
 
@@ -182,6 +217,8 @@ int check_attn_common(const void* q, const void* kv, const void* swa_kv, const i
                       const int64_t* q_pos, const float* sink, float scale, int B, int T, int H, int D, int64_t N,
                       int dtype, const void* out) {
   if (B < 0 || T < 0 || H <= 0 || D <= 0 || N < 0 || W < 0) return CSA_ERR_INVALID;
+  if ((int64_t)B * T * H * (D / 8) >= (int64_t(1) << 31) || (int64_t)B * T > 65535 * 1024)
+    return CSA_ERR_UNSUPPORTED;
   if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_ERR_INVALID;
   if (!(scale == scale)) return CSA_ERR_INVALID;
   if (B == 0 || T == 0) return CSA_OK;
@@ -236,10 +273,11 @@ int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* 
   const bool bf_in = in_dtype == CSA_BF16, bf_out = out_dtype == CSA_BF16;
   if (ratio == 4) {
     const int64_t total = (int64_t)B * n_entries * (c / 8);
+    if (total >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
     const int64_t blocks64 = (total + 255) / 256;
     const unsigned blocks = (unsigned)std::min<int64_t>(blocks64, (int64_t)sm_count() * 16);
 #define CSA_LAUNCH_CSA(TI, TO)                                                                              \
-  csa::compress_csa_kernel<TI, TO, 4><<<blocks, 256, 0, st>>>(                                              \
+  launch_k(csa::compress_csa_kernel<TI, TO, 4>, blocks, 256, 0, st,                                               \
       (const TI*)C_a, (const TI*)C_b, (const TI*)Z_a, (const TI*)Z_b, (const TI*)prev_Cb, (const TI*)prev_Zb, \
       B, L, c, (TO*)out)
     if (bf_in && bf_out) CSA_LAUNCH_CSA(__nv_bfloat16, __nv_bfloat16);
@@ -252,7 +290,7 @@ int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* 
     const int G = std::min(c / 8, 64);
     dim3 grid((unsigned)(c / 8 / G), (unsigned)n_entries, (unsigned)B);
 #define CSA_LAUNCH_HCA(TI, TO) \
-  csa::compress_hca_kernel<TI, TO><<<grid, 256, 0, st>>>((const TI*)C_a, (const TI*)Z_a, B, L, c, (TO*)out)
+  launch_k(csa::compress_hca_kernel<TI, TO>, grid, 256, 0, st, (const TI*)C_a, (const TI*)Z_a, B, L, c, (TO*)out)
     if (bf_in && bf_out) CSA_LAUNCH_HCA(__nv_bfloat16, __nv_bfloat16);
     else if (bf_in) CSA_LAUNCH_HCA(__nv_bfloat16, float);
     else if (bf_out) CSA_LAUNCH_HCA(float, __nv_bfloat16);
@@ -272,14 +310,15 @@ int csa_quantize_e4m3(const void* x, int x_dtype, int64_t rows, int cols, uint8_
   const unsigned blocks = (unsigned)std::min<int64_t>(blocks64, (int64_t)sm_count() * 32);
   cudaStream_t st = as_stream(stream);
   if (x_dtype == CSA_BF16)
-    csa::quantize_e4m3_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)x, rows, cols, codes, scale);
+    launch_k(csa::quantize_e4m3_kernel<__nv_bfloat16>, blocks, 256, 0, st, (const __nv_bfloat16*)x, rows, cols, codes, scale);
   else
-    csa::quantize_e4m3_kernel<float><<<blocks, 256, 0, st>>>((const float*)x, rows, cols, codes, scale);
+    launch_k(csa::quantize_e4m3_kernel<float>, blocks, 256, 0, st, (const float*)x, rows, cols, codes, scale);
   return launch_status();
 }
 
 int csa_index_scores(const void* qI, const float* q_scale, const float* w, const void* kI, const float* k_scale,
-                     int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* stream) {
+                     int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* select_ws,
+                     void* stream) {
   if (B < 0 || T < 0 || N < 0) return CSA_ERR_INVALID;
   if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3) return CSA_ERR_INVALID;
   if (B == 0 || T == 0 || N == 0) return CSA_OK;
@@ -293,7 +332,7 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
     if (T > 65535) return CSA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)((N + 63) / 64), (unsigned)T, (unsigned)B);
     if (!set_smem(csa::index_simt_kernel<float, false>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
-    csa::index_simt_kernel<float, false><<<grid, 256, csa::kIdxSimtSmem, st>>>(
+    launch_k(csa::index_simt_kernel<float, false>, grid, 256, csa::kIdxSimtSmem, st, 
         (const float*)qI, w, (const float*)kI, n_valid, nullptr, 0, T, N, scores);
     return launch_status();
   }
@@ -308,10 +347,18 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
   p.T = T;
   p.N = N;
   p.TQ = T >= 4 ? 4 : (T >= 2 ? 2 : 1);
+  p.hist = nullptr;
+  p.hist_stride = 0;
+  if (select_ws != nullptr) {
+    if (T != 1 || !aligned16(select_ws)) return CSA_ERR_INVALID;
+    p.hist = reinterpret_cast<int*>(select_ws);
+    p.hist_stride = csa::SelectWs::row_bytes(N) / 4;
+  }
   const int key_bytes = fp8 ? csa::IndexCfg<true>::kKeyBytes : csa::IndexCfg<false>::kKeyBytes;
   const int qrow = fp8 ? 128 : 256;
   const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
-  const int fixed = 1024 + q_bytes + 1024 * p.TQ + 8 * 8;
+  const int fixed = 1024 + q_bytes + 2048 * p.TQ + 8 * (4 + 2 * csa::kMaxAcc) +
+                    (select_ws ? 2 * csa::kHistBinsIdx * 4 : 0);
   p.stages = std::min(12, (kSmemLimit - fixed) / (key_bytes + 16));
   if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
   const int smem = fixed + p.stages * (key_bytes + 16);
@@ -328,10 +375,10 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
   const unsigned grid = (unsigned)std::min<int64_t>(items, sm_count());
   if (fp8) {
     if (!set_smem(csa::index_tc_kernel<true>, smem)) return CSA_ERR_CUDA;
-    csa::index_tc_kernel<true><<<grid, 192, smem, st>>>(kmap, qmap, p);
+    launch_k(csa::index_tc_kernel<true>, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
   } else {
     if (!set_smem(csa::index_tc_kernel<false>, smem)) return CSA_ERR_CUDA;
-    csa::index_tc_kernel<false><<<grid, 192, smem, st>>>(kmap, qmap, p);
+    launch_k(csa::index_tc_kernel<false>, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
   }
   return launch_status();
 }
@@ -349,18 +396,18 @@ int csa_index_rerank(const void* qI, const float* w, const void* kI, int dtype, 
   dim3 grid((unsigned)((kc + 63) / 64), (unsigned)T, (unsigned)B);
   if (dtype == CSA_BF16) {
     if (!set_smem(csa::index_simt_kernel<__nv_bfloat16, true>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
-    csa::index_simt_kernel<__nv_bfloat16, true><<<grid, 256, csa::kIdxSimtSmem, st>>>(
+    launch_k(csa::index_simt_kernel<__nv_bfloat16, true>, grid, 256, csa::kIdxSimtSmem, st, 
         (const __nv_bfloat16*)qI, w, (const __nv_bfloat16*)kI, nullptr, cand, kc, T, N, cand_scores);
   } else {
     if (!set_smem(csa::index_simt_kernel<float, true>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
-    csa::index_simt_kernel<float, true><<<grid, 256, csa::kIdxSimtSmem, st>>>(
+    launch_k(csa::index_simt_kernel<float, true>, grid, 256, csa::kIdxSimtSmem, st, 
         (const float*)qI, w, (const float*)kI, nullptr, cand, kc, T, N, cand_scores);
   }
   int rc = launch_status();
   if (rc != CSA_OK) return rc;
   const int smem = kc * 4;
   if (!set_smem(csa::topk_row_kernel, std::max(smem, 4))) return CSA_ERR_CUDA;
-  csa::topk_row_kernel<<<(unsigned)((int64_t)B * T), 1024, smem, st>>>(cand_scores, nullptr, kc, k, idx, cand);
+  launch_k(csa::topk_row_kernel, (unsigned)((int64_t)B * T), 1024, smem, st, cand_scores, nullptr, kc, k, idx, cand);
   return launch_status();
 }
 
@@ -389,17 +436,84 @@ int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t 
   if (!topk_long_path(B, T, N)) {
     const int smem = (int)std::max<int64_t>(4, std::min<int64_t>(N, csa::kRowSmemMax) * 4);
     if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
-    csa::topk_row_kernel<<<(unsigned)rows, 1024, smem, st>>>(scores, n_valid, N, k, idx, nullptr);
+    launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, smem, st, scores, n_valid, N, k, idx, nullptr);
     return launch_status();
   }
   const size_t need = csa_topk_workspace_size(B, T, N, k);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSA_ERR_INVALID;
   dim3 grid((unsigned)((N + csa::kChunk - 1) / csa::kChunk), (unsigned)rows);
-  csa::topk_hist_kernel<<<grid, 512, 0, st>>>(scores, n_valid, N, k, static_cast<uint8_t*>(workspace));
+  launch_k(csa::topk_hist_kernel, grid, 512, 0, st, scores, n_valid, N, k, static_cast<uint8_t*>(workspace),
+           (int64_t)csa::TopkWs::row_bytes(N));
   int rc = launch_status();
   if (rc != CSA_OK) return rc;
-  csa::topk_gather_select_kernel<<<grid, 1024, 0, st>>>(scores, n_valid, N, k, idx,
-                                                        static_cast<uint8_t*>(workspace));
+  const int gsmem = 2 * csa::kCandSmem * 4;
+  if (!set_smem(csa::topk_gather_select_kernel, gsmem)) return CSA_ERR_CUDA;
+  launch_k(csa::topk_gather_select_kernel, grid, 1024, gsmem, st, scores, n_valid, N, k, idx,
+                                                            static_cast<uint8_t*>(workspace));
+  return launch_status();
+}
+
+size_t csa_select_workspace_size(int B, int64_t N) {
+  if (B <= 0 || N <= 0) return 0;
+  return (size_t)B * (size_t)csa::SelectWs::row_bytes(N);
+}
+
+int csa_score_histogram(const float* scores, const int32_t* n_valid, int B, int64_t N, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  if (B < 0 || N < 0) return CSA_ERR_INVALID;
+  if (N > csa::kSelMaxN || B > 65535) return CSA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return CSA_OK;
+  if (!scores || !n_valid || !workspace || ws_bytes < csa_select_workspace_size(B, N) || !aligned16(workspace))
+    return CSA_ERR_INVALID;
+  dim3 grid((unsigned)((N + csa::kChunk - 1) / csa::kChunk), (unsigned)B);
+  // k = 0: every row with a valid entry is histogrammed
+  launch_k(csa::topk_hist_kernel, grid, 512, 0, as_stream(stream), scores, n_valid, N, 0,
+           static_cast<uint8_t*>(workspace), (int64_t)csa::SelectWs::row_bytes(N));
+  return launch_status();
+}
+
+int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t N, int k, int kc, const void* qI,
+                    const float* w, const void* kI, int dtype, int32_t* idx, void* workspace, size_t ws_bytes,
+                    void* stream) {
+  if (B < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (N > csa::kSelMaxN || B > 65535) return CSA_ERR_UNSUPPORTED;
+  const bool rescore = qI != nullptr;
+  if (rescore && (kc < k || !w || !kI || (dtype != CSA_F32 && dtype != CSA_BF16))) return CSA_ERR_INVALID;
+  if (rescore && (!aligned16(qI) || !aligned16(kI))) return CSA_ERR_INVALID;
+  if (B == 0) return CSA_OK;
+  if (!idx || !n_valid || (N > 0 && !scores)) return CSA_ERR_INVALID;
+  const size_t need = csa_select_workspace_size(B, N);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSA_ERR_INVALID;
+  if (N == 0) {
+    launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr);
+    return launch_status();
+  }
+  // chunks: about two CTAs per SM in total, at least 256 entries each
+  const int sms = sm_count();
+  int64_t nchunks = std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (2 * sms + B - 1) / B));
+  int chunk = (int)(((N + nchunks - 1) / nchunks + 255) / 256 * 256);
+  nchunks = (N + chunk - 1) / chunk;
+  const int64_t words = (N + 31) / 32;
+  const int phase3 = csa::kSelTileBytes + csa::kSelQBytes + chunk * 8 +
+                     (64 + 64 * 129 + csa::kSelKeyBatch * 128) * 4;
+  const int phase4 = (int)(2 * csa::kSelCandSmem * 4 + 2 * words * 4);
+  const int smem = 1024 + std::max(phase3, phase4);
+  cudaStream_t st = as_stream(stream);
+  dim3 grid((unsigned)nchunks, (unsigned)B);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (!rescore) {
+    if (!set_smem(csa::topk_select_kernel<false, float>, smem)) return CSA_ERR_CUDA;
+    launch_k(csa::topk_select_kernel<false, float>, grid, csa::kSelThreads, smem, st, scores, n_valid, N, k, k,
+             chunk, (const float*)nullptr, w, (const float*)nullptr, idx, ws);
+  } else if (dtype == CSA_BF16) {
+    if (!set_smem(csa::topk_select_kernel<true, __nv_bfloat16>, smem)) return CSA_ERR_CUDA;
+    launch_k(csa::topk_select_kernel<true, __nv_bfloat16>, grid, csa::kSelThreads, smem, st, scores, n_valid, N,
+             k, kc, chunk, (const __nv_bfloat16*)qI, w, (const __nv_bfloat16*)kI, idx, ws);
+  } else {
+    if (!set_smem(csa::topk_select_kernel<true, float>, smem)) return CSA_ERR_CUDA;
+    launch_k(csa::topk_select_kernel<true, float>, grid, csa::kSelThreads, smem, st, scores, n_valid, N, k, kc,
+             chunk, (const float*)qI, w, (const float*)kI, idx, ws);
+  }
   return launch_status();
 }
 

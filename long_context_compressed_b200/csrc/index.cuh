@@ -9,7 +9,8 @@
 // TQ queries x 64 heads of a query group are the N = 64*TQ operand, K = 128.
 // Both are staged by TMA (128-byte swizzle, K-major) into shared memory;
 // one elected thread issues tcgen05.mma into a double-buffered fp32 TMEM
-// accumulator; four epilogue warps read their 32 TMEM lanes (one key per
+// accumulator; eight epilogue warps (two sets taking alternate tiles) read
+// their 32 TMEM lanes (one key per
 // thread), apply ReLU and the head weights, reduce over the 64 heads and store
 // one fp32 score per (query, key).  Persistent: one CTA per SM walks a
 // contiguous range of (sequence, query group, key tile) work items so that
@@ -30,6 +31,18 @@ namespace csa {
 constexpr int kIdxHeads = 64;
 constexpr int kIdxDim = 128;
 constexpr int kIdxTileKeys = 128;
+constexpr int kMaxAcc = 4;
+constexpr int kIdxThreads = 320;                // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kHistBinsIdx = 4096;              // 12-bit histogram of order-preserving score keys
+
+// Top 12 bits of the order-preserving uint32 key of a score (-0.0 folded to +0.0):
+// bin order equals score order.
+__device__ __forceinline__ uint32_t score_bin(float x) {
+  uint32_t u = __float_as_uint(x);
+  if ((u << 1) == 0) u = 0;
+  const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return key >> 20;
+}
 
 struct IndexParams {
   const float* w;        // [B, T, 64]
@@ -37,6 +50,8 @@ struct IndexParams {
   const float* k_scale;  // [B, N] or null (bf16)
   const int32_t* n_valid;  // [B, T]
   float* scores;         // [B, T, N]
+  int* hist;             // per-row 4096-bin histogram of the score keys (T == 1), row stride hist_stride, or null
+  int64_t hist_stride;   // ints between consecutive rows' histograms
   int B, T;
   int64_t N;
   int TQ;                // queries per group (1, 2 or 4)
@@ -65,9 +80,20 @@ __device__ __forceinline__ IndexItem index_item(int64_t w, int QG, int64_t KT) {
   it.b = (int)(r / QG);
   return it;
 }
+// Advance to the next work item without division (the loops below are latency
+// critical: a 64-bit division per item costs several hundred cycles).
+__device__ __forceinline__ void index_next(IndexItem& it, int QG, int64_t KT) {
+  if (++it.kt == KT) {
+    it.kt = 0;
+    if (++it.qg == QG) {
+      it.qg = 0;
+      ++it.b;
+    }
+  }
+}
 
 template <bool FP8>
-__global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap qmap,
                                                           const IndexParams p) {
   using Cfg = IndexCfg<FP8>;
@@ -83,17 +109,20 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
   uint64_t* empty = bars + p.stages;
   uint64_t* qfull = bars + 2 * p.stages;
   uint64_t* qempty = qfull + 1;
-  uint64_t* tfull = qfull + 2;                      // [2]
-  uint64_t* tempty = qfull + 4;                     // [2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 6);
-  float* w_all = reinterpret_cast<float*>(qfull + 8);  // [4 epilogue warps][TQ][64]
+  uint64_t* tfull = qfull + 2;                      // [kMaxAcc]
+  uint64_t* tempty = qfull + 2 + kMaxAcc;           // [kMaxAcc]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 2 + 2 * kMaxAcc);
+  float* w_all = reinterpret_cast<float*>(qfull + 4 + 2 * kMaxAcc);  // [8 epilogue warps][TQ][64]
+  // score histograms of the first two rows this CTA touches (when p.hist is set)
+  int* hist_s = reinterpret_cast<int*>(w_all + 8 * TQ * kIdxHeads);   // [2][kHistBinsIdx]
 
   const int QG = (p.T + TQ - 1) / TQ;
   const int64_t KT = (p.N + kIdxTileKeys - 1) / kIdxTileKeys;
   const int64_t items = (int64_t)p.B * QG * KT;
   const int64_t w0 = items * blockIdx.x / gridDim.x;
   const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
-  const uint32_t tmem_cols = (uint32_t)(2 * NQ) < 32 ? 32u : (uint32_t)(2 * NQ);
+  const int NACC = (512 / NQ) < kMaxAcc ? (512 / NQ) : kMaxAcc;   // TMEM accumulators in flight
+  const uint32_t tmem_cols = (uint32_t)(NACC * NQ) < 32 ? 32u : (uint32_t)(NACC * NQ);
 
   const int warp = warp_id();
   if (threadIdx.x == 0) {
@@ -103,7 +132,7 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kMaxAcc; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 4);                     // one arrive per epilogue warp
     }
@@ -115,10 +144,14 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
     tmem_alloc(tmem_holder, tmem_cols);
     tmem_relinquish();
   }
+  if (p.hist)
+    for (int j = threadIdx.x; j < 2 * kHistBinsIdx; j += blockDim.x) hist_s[j] = 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  griddep_sync();
+  const int hist_row0 = index_item(w0, QG, KT).b;   // T == 1 whenever p.hist is set: row = sequence
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -126,8 +159,10 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
       int prev_b = -1, prev_qg = -1;
       uint32_t qe_phase = 0;
       int64_t cnt = 0;
-      for (int64_t w = w0; w < w1; ++w, ++cnt) {
-        const IndexItem it = index_item(w, QG, KT);
+      int st_i = 0;
+      uint32_t st_ph = 0;
+      IndexItem it = index_item(w0, QG, KT);
+      for (int64_t w = w0; w < w1; ++w, ++cnt, index_next(it, QG, KT)) {
         if (it.b != prev_b || it.qg != prev_qg) {
           if (prev_b >= 0) {
             if (!mbar_wait(qempty, qe_phase)) break;
@@ -139,8 +174,9 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
           prev_b = it.b;
           prev_qg = it.qg;
         }
-        const int s = (int)(cnt % p.stages);
-        const uint32_t ph = (uint32_t)((cnt / p.stages) & 1);
+        const int s = st_i;
+        const uint32_t ph = st_ph;
+        if (++st_i == p.stages) { st_i = 0; st_ph ^= 1; }
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
         mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKeyBytes);
         uint8_t* dst = k_smem + (size_t)s * Cfg::kKeyBytes;
@@ -156,8 +192,10 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
       int prev_b = -1, prev_qg = -1;
       uint32_t qf_phase = 0;
       int64_t cnt = 0;
-      for (int64_t w = w0; w < w1; ++w, ++cnt) {
-        const IndexItem it = index_item(w, QG, KT);
+      int st_i = 0, ac_i = 0;
+      uint32_t st_ph = 0, ac_ph = 0;
+      IndexItem it = index_item(w0, QG, KT);
+      for (int64_t w = w0; w < w1; ++w, ++cnt, index_next(it, QG, KT)) {
         if (it.b != prev_b || it.qg != prev_qg) {
           if (prev_b >= 0) mma_commit(qempty);      // old Q free once its MMAs finish
           if (!mbar_wait(qfull, qf_phase)) break;
@@ -165,10 +203,12 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
           prev_b = it.b;
           prev_qg = it.qg;
         }
-        const int s = (int)(cnt % p.stages);
-        const uint32_t ph = (uint32_t)((cnt / p.stages) & 1);
-        const int acc = (int)(cnt & 1);
-        const uint32_t aph = (uint32_t)((cnt >> 1) & 1);
+        const int s = st_i;
+        const uint32_t ph = st_ph;
+        if (++st_i == p.stages) { st_i = 0; st_ph ^= 1; }
+        const int acc = ac_i;
+        const uint32_t aph = ac_ph;
+        if (++ac_i == NACC) { ac_i = 0; ac_ph ^= 1; }
         if (!mbar_wait(&tempty[acc], aph ^ 1)) break;
         if (!mbar_wait(&full[s], ph)) break;
         tc_fence_after();
@@ -193,14 +233,37 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
       }
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    // ---------------------------------------------------------------- epilogue (warps 2..9)
+    // Two sets of four warps take alternate tiles; within a set, warp w owns TMEM
+    // lanes 32*(w%4) .. +31, i.e. one key per thread.
     const int quarter = warp & 3;                   // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + (int)lane_id();  // key within the tile
+    const int es = (warp - 2) >> 2;                 // epilogue set: 0 or 1
+    const int acc_shift = NACC == 4 ? 2 : (NACC == 2 ? 1 : 0);
     float* w_s = w_all + (warp - 2) * TQ * kIdxHeads;
+    int64_t nv_q[4] = {0, 0, 0, 0};
+    // key scales are fetched two of this set's items ahead along a second iterator
+    IndexItem ahead = index_item(w0, QG, KT);
+    int64_t w_ahead = w0;
+    if (es) { index_next(ahead, QG, KT); ++w_ahead; }
+    auto ks_next = [&]() -> float {
+      float v = 1.f;
+      if (FP8 && w_ahead < w1) {
+        const int64_t ii = ahead.kt * kIdxTileKeys + row;
+        if (ii < p.N) v = __ldg(p.k_scale + (int64_t)ahead.b * p.N + ii);
+      }
+      w_ahead += 2;
+      index_next(ahead, QG, KT);
+      index_next(ahead, QG, KT);
+      return v;
+    };
+    float ks0 = ks_next(), ks1 = ks_next();
     int prev_b = -1, prev_qg = -1;
-    int64_t cnt = 0;
-    for (int64_t w = w0; w < w1; ++w, ++cnt) {
-      const IndexItem it = index_item(w, QG, KT);
+    IndexItem it = index_item(w0, QG, KT);
+    int64_t w = w0;
+    int cnt = 0;
+    if (es) { index_next(it, QG, KT); ++w; ++cnt; }
+    for (; w < w1; w += 2, cnt += 2, index_next(it, QG, KT), index_next(it, QG, KT)) {
       if (it.b != prev_b || it.qg != prev_qg) {
         // each epilogue warp keeps a private copy of the group's head weights
         __syncwarp();
@@ -215,16 +278,25 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
           w_s[j] = v;
         }
         __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = it.qg * TQ + q;
+          nv_q[q] = (q < TQ && t < p.T) ? (int64_t)p.n_valid[(int64_t)it.b * p.T + t] : 0;
+        }
         prev_b = it.b;
         prev_qg = it.qg;
       }
-      const int acc = (int)(cnt & 1);
-      const uint32_t aph = (uint32_t)((cnt >> 1) & 1);
+      const int acc = cnt & (NACC - 1);
+      const uint32_t aph = (uint32_t)(cnt >> acc_shift) & 1u;
+      const float ks = ks0;
+      ks0 = ks1;
+      ks1 = ks_next();
       if (!mbar_wait(&tfull[acc], aph)) break;
       tc_fence_after();
       const int64_t i = it.kt * kIdxTileKeys + row;
-      const float ks = (FP8 && i < p.N) ? p.k_scale[(int64_t)it.b * p.N + i] : 1.f;
-      for (int q = 0; q < TQ; ++q) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q >= TQ) break;
         const int t = it.qg * TQ + q;
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NQ + q * 64);
         float v0[32], v1[32];
@@ -233,14 +305,32 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
         tmem_wait_ld();
         if (t >= p.T) continue;
         const float* wq = w_s + q * kIdxHeads;
-        float s = 0.f;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;   // independent chains
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s = fmaf(wq[h], fmaxf(v0[h], 0.f), s);
+        for (int h = 0; h < 32; h += 4) {
+          s0 = fmaf(wq[h], fmaxf(v0[h], 0.f), s0);
+          s1 = fmaf(wq[h + 1], fmaxf(v0[h + 1], 0.f), s1);
+          s2 = fmaf(wq[h + 2], fmaxf(v0[h + 2], 0.f), s2);
+          s3 = fmaf(wq[h + 3], fmaxf(v0[h + 3], 0.f), s3);
+        }
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s = fmaf(wq[32 + h], fmaxf(v1[h], 0.f), s);
+        for (int h = 0; h < 32; h += 4) {
+          s0 = fmaf(wq[32 + h], fmaxf(v1[h], 0.f), s0);
+          s1 = fmaf(wq[33 + h], fmaxf(v1[h + 1], 0.f), s1);
+          s2 = fmaf(wq[34 + h], fmaxf(v1[h + 2], 0.f), s2);
+          s3 = fmaf(wq[35 + h], fmaxf(v1[h + 3], 0.f), s3);
+        }
+        const float sc = (s0 + s1) + (s2 + s3);
         if (i < p.N) {
-          const int64_t nv = p.n_valid[(int64_t)it.b * p.T + t];
-          p.scores[((int64_t)it.b * p.T + t) * p.N + i] = (i < nv) ? s * ks : -INFINITY;
+          const bool valid = i < nv_q[q];
+          const float val = valid ? sc * ks : -INFINITY;
+          p.scores[((int64_t)it.b * p.T + t) * p.N + i] = val;
+          if (p.hist && valid) {
+            const uint32_t bin = score_bin(val);
+            const int slot = it.b - hist_row0;
+            if (slot < 2) atomicAdd(&hist_s[slot * kHistBinsIdx + bin], 1);
+            else atomicAdd(&p.hist[(int64_t)it.b * p.hist_stride + bin], 1);
+          }
         }
       }
       tc_fence_before();
@@ -253,6 +343,13 @@ __global__ void __launch_bounds__(192, 1) index_tc_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+  if (p.hist) {
+    for (int j = threadIdx.x; j < 2 * kHistBinsIdx; j += blockDim.x) {
+      const int c = hist_s[j];
+      const int row = hist_row0 + j / kHistBinsIdx;
+      if (c != 0 && row < p.B) atomicAdd(&p.hist[(int64_t)row * p.hist_stride + (j % kHistBinsIdx)], c);
+    }
+  }
 }
 
 constexpr int kIdxSimtSmem = (kIdxHeads + 64) * (kIdxDim + 4) * 4;
@@ -278,6 +375,7 @@ __global__ void __launch_bounds__(256) index_simt_kernel(const Tin* __restrict__
                                                          const int32_t* __restrict__ n_valid,
                                                          const int32_t* __restrict__ cand, int kc, int T, int64_t N,
                                                          float* __restrict__ out) {
+  griddep_sync();
   constexpr int KT = 64, PAD = 4;
   extern __shared__ __align__(16) float f32_smem[];
   float(*qs)[kIdxDim + PAD] = reinterpret_cast<float(*)[kIdxDim + PAD]>(f32_smem);

@@ -229,6 +229,23 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t ab_form
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// 2^x with the SFU instruction (approximate, ~2 ulp; flushes subnormal results
+// to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Programmatic dependent launch: wait until the preceding kernel in the stream has
+// completed (a no-op when this kernel was not launched as a dependent), then let
+// the following kernel begin launching.  Every kernel calls this pair before its
+// first global-memory access and after allocating tensor memory.
+__device__ __forceinline__ void griddep_sync() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 

@@ -19,6 +19,7 @@ __device__ __forceinline__ float load_as_float(const __nv_bfloat16* p, int64_t i
 template <typename Tin>
 __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const Tin* __restrict__ x, int64_t rows, int cols,
                                                             uint8_t* __restrict__ codes, float* __restrict__ scale) {
+  griddep_sync();
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const Tin* xr = x + r * cols;

@@ -22,6 +22,7 @@
 //                     the row through index bitmaps.  It leaves its workspace
 //                     zeroed for the next call (no inter-CTA waiting).
 #pragma once
+#include <cuda_bf16.h>
 #include "ptx.cuh"
 
 namespace csa {
@@ -30,6 +31,7 @@ constexpr int kRowSmemMax = 32768;
 constexpr int kHistBits = 12;
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kChunk = 4096;
+constexpr int kCandSmem = 8192;                 // candidates the last CTA stages in shared memory
 
 __device__ __forceinline__ uint32_t order_key(float x) {
   uint32_t u = __float_as_uint(x);
@@ -105,6 +107,35 @@ __device__ __forceinline__ void find_digit(const int* hist, int nbins, int remai
   }
 }
 
+// Block-wide version of find_digit for nbins == BPT * blockDim.x: thread i owns
+// the BPT bins nbins-BPT*i-1 .. nbins-BPT*(i+1) (top first); a block scan of the
+// owned counts locates the bin.  All threads must call it.
+template <int BPT = 4>
+__device__ __forceinline__ void find_digit_block(const int* hist, int nbins, int remaining, int* res,
+                                                 int* scratch) {
+  const int hi = nbins - 1 - BPT * (int)threadIdx.x;
+  int c[BPT], local = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    c[j] = hist[hi - j];
+    local += c[j];
+  }
+  int total;
+  const int exc = block_excl_scan(local, scratch, &total);
+  if (exc < remaining && remaining <= exc + local) {
+    int above = exc;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (above + c[j] >= remaining) {
+        res[0] = hi - j;
+        res[1] = above;
+        break;
+      }
+      above += c[j];
+    }
+  }
+}
+
 // Write the selection of a segment in index order.  Every thread owns the
 // contiguous index range [lo, hi) and calls get(i) -> key.
 template <typename GetKey>
@@ -144,6 +175,7 @@ __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict_
                                                         const int32_t* __restrict__ n_valid, int64_t N, int k,
                                                         int32_t* __restrict__ idx,
                                                         const int32_t* __restrict__ map) {
+  griddep_sync();
   extern __shared__ __align__(16) uint32_t keys[];  // [min(N, kRowSmemMax)]
   __shared__ int hist[256];
   __shared__ int scratch[33];
@@ -201,7 +233,8 @@ struct TopkWs {
 
 __global__ void __launch_bounds__(512) topk_hist_kernel(const float* __restrict__ scores,
                                                         const int32_t* __restrict__ n_valid, int64_t N, int k,
-                                                        uint8_t* __restrict__ ws) {
+                                                        uint8_t* __restrict__ ws, int64_t ws_row_bytes) {
+  griddep_sync();
   __shared__ int hist[kHistBins];
   const int64_t row = blockIdx.y;
   int nv = n_valid[row];
@@ -219,7 +252,7 @@ __global__ void __launch_bounds__(512) topk_hist_kernel(const float* __restrict_
     warp_hist_add(hist, key >> (32 - kHistBits), act);
   }
   __syncthreads();
-  int* ghist = reinterpret_cast<int*>(ws + row * TopkWs::row_bytes(N));
+  int* ghist = reinterpret_cast<int*>(ws + row * ws_row_bytes);
   for (int j = threadIdx.x; j < kHistBins; j += blockDim.x)
     if (hist[j]) atomicAdd(&ghist[j], hist[j]);
 }
@@ -228,11 +261,13 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
                                                                   const int32_t* __restrict__ n_valid, int64_t N,
                                                                   int k, int32_t* __restrict__ idx,
                                                                   uint8_t* __restrict__ ws) {
+  griddep_sync();
   __shared__ int hist[256];
   __shared__ int scratch[33];
   __shared__ int res[2];
   __shared__ int is_last;
   __shared__ int hist4k[kHistBins];
+  extern __shared__ __align__(16) uint32_t cand_smem[];   // [kCandSmem] keys + [kCandSmem] indices
   const int64_t row = blockIdx.y;
   int nv = n_valid[row];
   nv = nv < 0 ? 0 : (nv > (int)N ? (int)N : nv);
@@ -256,7 +291,7 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
   // threshold bin b*: count(bins > b*) < k <= count(bins >= b*), 128 bins per lane of warp 0
   for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) hist4k[j] = __ldcg(ghist + j);
   __syncthreads();
-  find_digit(hist4k, kHistBins, k, res);
+  find_digit_block<4>(hist4k, kHistBins, k, res, scratch);
   __syncthreads();
   const uint32_t bstar = (uint32_t)res[0];
   // append every key whose top bits are >= b* (warp-aggregated slot reservation)
@@ -290,8 +325,20 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
   if (!is_last) return;
   __threadfence();
 
-  // ---- last CTA: exact select among the candidates
+  // ---- last CTA: exact select among the candidates (staged in shared memory when they fit)
   const int nc = *((volatile int*)cand_count);
+  uint32_t* skey = cand_smem;
+  int32_t* sidx = reinterpret_cast<int32_t*>(cand_smem + kCandSmem);
+  const bool in_smem = nc <= kCandSmem;
+  if (in_smem) {
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      skey[i] = __ldcg(ckey + i);
+      sidx[i] = __ldcg(cidx + i);
+    }
+    __syncthreads();
+  }
+  auto cand_key = [&](int i) -> uint32_t { return in_smem ? skey[i] : __ldcg(ckey + i); };
+  auto cand_idx = [&](int i) -> int32_t { return in_smem ? sidx[i] : __ldcg(cidx + i); };
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
   for (int pass = 0; pass < 4; ++pass) {
@@ -300,7 +347,7 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
     __syncthreads();
     for (int i0 = 0; i0 < nc; i0 += blockDim.x) {
       const int i = i0 + threadIdx.x;
-      const uint32_t key = i < nc ? __ldcg(ckey + i) : 0u;
+      const uint32_t key = i < nc ? cand_key(i) : 0u;
       const bool act = i < nc && (key & pmask) == prefix;
       warp_hist_add(hist, (key >> shift) & 255u, act);
     }
@@ -314,8 +361,8 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
   }
   // mark candidates > K* and == K* in two index bitmaps
   for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-    const uint32_t key = __ldcg(ckey + i);
-    const int32_t j = __ldcg(cidx + i);
+    const uint32_t key = cand_key(i);
+    const int32_t j = cand_idx(i);
     if (key > prefix) atomicOr(&bm_gt[j >> 5], 1u << (j & 31));
     else if (key == prefix) atomicOr(&bm_eq[j >> 5], 1u << (j & 31));
   }
@@ -358,6 +405,476 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
     ckey[i] = 0;
     cidx[i] = 0;
   }
+  if (threadIdx.x == 0) {
+    *cand_count = 0;
+    *done = 0;
+  }
+}
+
+// ---------------------------------------------------------------- fused select (decode)
+// Per-row workspace of topk_select_kernel: [4096-bin histogram][candidate count]
+// [finished CTAs][pad] then candidate keys [N] and indices [N].  The histogram is
+// accumulated by the indexer (csa_index_scores with this workspace); the last CTA
+// of each row leaves the row's header zeroed for the next call.
+struct SelectWs {
+  static constexpr int64_t kHeaderInts = kHistBins + 64;
+  static __host__ __device__ int64_t row_bytes(int64_t N) {
+    return ((kHeaderInts + 2 * N) * 4 + 15) / 16 * 16;
+  }
+};
+constexpr int kSelThreads = 256;
+constexpr int kSelPerThread = 4;     // scores each thread loads per pass of the chunk scan
+constexpr int kSelTcRows = 128;      // candidates rescored per tensor-core batch (bf16)
+constexpr int kSelKeyBatch = 64;     // candidate key rows per SIMT batch (fp32)
+constexpr int kSelCandSmem = 4096;   // candidates the last CTA stages in shared memory
+constexpr int64_t kSelMaxN = int64_t(1) << 19;
+constexpr int kSelTileBytes = 2 * kSelTcRows * 128;    // candidate key tile, 2 x 128-byte K atoms (bf16)
+constexpr int kSelQBytes = 2 * 64 * 128;               // q tile: 64 heads x 128 dims bf16
+
+template <typename T>
+__device__ __forceinline__ void unpack_vec(uint4 v, float* f);
+template <>
+__device__ __forceinline__ void unpack_vec<__nv_bfloat16>(uint4 v, float* f) {   // 8 bf16
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+template <>
+__device__ __forceinline__ void unpack_vec<float>(uint4 v, float* f) {  // 4 fp32
+  f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+}
+
+// Skewed shared-memory histogram index: bin h lives at h + h/32, so threads that
+// own consecutive groups of 8 or 16 bins read them without bank conflicts.
+__device__ __forceinline__ int skew(int h) { return h + (h >> 5); }
+
+// find_digit_block over a skewed histogram (nbins == BPT * blockDim.x).
+template <int BPT>
+__device__ __forceinline__ void find_digit_skewed(const int* hist, int nbins, int remaining, int* res,
+                                                  int* scratch) {
+  const int hi = nbins - 1 - BPT * (int)threadIdx.x;
+  int c[BPT], local = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    c[j] = hist[skew(hi - j)];
+    local += c[j];
+  }
+  int total;
+  const int exc = block_excl_scan(local, scratch, &total);
+  if (exc < remaining && remaining <= exc + local) {
+    int above = exc;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (above + c[j] >= remaining) {
+        res[0] = hi - j;
+        res[1] = above;
+        break;
+      }
+      above += c[j];
+    }
+  }
+}
+
+// Write, in ascending index order, every index set in bm_gt and the first r_eq
+// (lowest) indices set in bm_eq, for words [0, used_words).  Warp w walks a
+// contiguous segment of words 32 at a time (lane l reads word base + l: no bank
+// conflicts); per-warp totals are scanned to give each warp its output offset.
+__device__ __forceinline__ void emit_ordered(const uint32_t* bm_gt, const uint32_t* bm_eq, int64_t used_words,
+                                             int r_eq, int32_t* out, int* scratch) {
+  const int nwarps = blockDim.x >> 5, warp = warp_id(), lane = lane_id();
+  const int64_t per = ((used_words + nwarps - 1) / nwarps + 31) / 32 * 32;
+  const int64_t s0 = (int64_t)warp * per < used_words ? (int64_t)warp * per : used_words;
+  const int64_t s1 = s0 + per < used_words ? s0 + per : used_words;
+  int gt = 0, eq = 0;
+  for (int64_t w = s0 + lane; w < s1; w += 32) {
+    gt += __popc(bm_gt[w]);
+    eq += __popc(bm_eq[w]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+  __syncthreads();
+  if (lane == 0) {
+    scratch[warp] = gt;
+    scratch[16 + warp] = eq;
+  }
+  __syncthreads();
+  int sel_before = 0, eq_before = 0;
+  for (int v = 0; v < warp; ++v) {
+    const int eb = eq_before;
+    int te = r_eq - eb;
+    te = te < 0 ? 0 : (te > scratch[16 + v] ? scratch[16 + v] : te);
+    sel_before += scratch[v] + te;
+    eq_before += scratch[16 + v];
+  }
+  int run_sel = sel_before, run_eq = eq_before;
+  for (int64_t base = s0; base < s1; base += 32) {
+    const int64_t w = base + lane;
+    const uint32_t g = w < s1 ? bm_gt[w] : 0u;
+    const uint32_t e = w < s1 ? bm_eq[w] : 0u;
+    const int ce = __popc(e);
+    int ie = ce;                                      // inclusive scan of eq counts over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, ie, o);
+      if (lane >= o) ie += n;
+    }
+    int te = r_eq - (run_eq + ie - ce);
+    te = te < 0 ? 0 : (te > ce ? ce : te);
+    uint32_t etake = 0, x = e;
+    for (int t = 0; t < te; ++t) {
+      const uint32_t bbit = x & (0u - x);
+      etake |= bbit;
+      x ^= bbit;
+    }
+    uint32_t sel = g | etake;
+    const int cs = __popc(sel);
+    int is = cs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, is, o);
+      if (lane >= o) is += n;
+    }
+    int pos = run_sel + is - cs;
+    while (sel) {
+      const int bit = __ffs(sel) - 1;
+      out[pos++] = (int32_t)(w * 32 + bit);
+      sel &= sel - 1;
+    }
+    run_sel += __shfl_sync(0xffffffffu, is, 31);
+    run_eq += __shfl_sync(0xffffffffu, ie, 31);
+  }
+}
+
+// Row r (one query per sequence: T == 1) of scores [rows, N].  Candidates are the
+// indices whose score lies in the histogram bin of the kk-th largest score or above
+// (kk = kc when RESCORE, else k) -- a superset of the kk largest.  With RESCORE each
+// candidate is rescored with the plain indexer definition on full-precision qI / kI
+// (fp32 accumulation; bf16 inputs on tcgen05, fp32 inputs on the FMA pipes); the
+// exact top-k of the (re)scored candidates, lower index first among equal scores, is
+// written in ascending index order by the last CTA of the row.
+template <bool RESCORE, typename Tin>
+__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* __restrict__ scores,
+                                                                  const int32_t* __restrict__ n_valid, int64_t N,
+                                                                  int k, int kc, int chunk,
+                                                                  const Tin* __restrict__ qI,
+                                                                  const float* __restrict__ w,
+                                                                  const Tin* __restrict__ kI, int32_t* __restrict__ idx,
+                                                                  uint8_t* __restrict__ ws) {
+  constexpr bool TC = RESCORE && sizeof(Tin) == 2;
+  extern __shared__ __align__(1024) uint8_t sel_raw[];
+  uint8_t* sel_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sel_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(16) int histk[kHistBins + kHistBins / 32];   // skewed
+  __shared__ int scratch[33];
+  __shared__ int res[2];
+  __shared__ int lcount, gslot, is_last;
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_holder;
+  if (TC) {
+    if (threadIdx.x == 0) {
+      mbar_init(&mma_bar, 1);
+      fence_mbar_init();
+    }
+    if (warp_id() == 0) {
+      tmem_alloc(&tmem_holder, 64);
+      tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  griddep_sync();
+  const int64_t row = blockIdx.y;
+  int nv = n_valid[row];
+  nv = nv < 0 ? 0 : (nv > (int)N ? (int)N : nv);
+  uint8_t* rws = ws + row * SelectWs::row_bytes(N);
+  int* ghist = reinterpret_cast<int*>(rws);
+  int* cand_count = ghist + kHistBins;
+  int* done = cand_count + 1;
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(rws + SelectWs::kHeaderInts * 4);
+  int32_t* cidx = reinterpret_cast<int32_t*>(ckey + N);
+  int32_t* out = idx + row * k;
+  const bool all_valid = nv <= k;
+  const bool active = !all_valid && (int64_t)blockIdx.x * chunk < nv;
+  if (all_valid && blockIdx.x == 0) {
+    write_all_valid(out, nv, k);
+    for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
+  }
+  int nloc = 0;
+  // shared-memory map: [key tile 32 KB][q tile 16 KB] (tensor-core rescoring) then
+  // lidx / lkey [chunk] and the fp32 rescoring scratch; the last CTA reuses all of it
+  uint8_t* tile_s = sel_smem;
+  uint8_t* qt_s = tile_s + kSelTileBytes;
+  int32_t* lidx = reinterpret_cast<int32_t*>(qt_s + kSelQBytes);
+  uint32_t* lkey = reinterpret_cast<uint32_t*>(lidx + chunk);
+  float* wsm = reinterpret_cast<float*>(lkey + chunk);               // [64]
+  if (active) {
+    const int kk = RESCORE ? (kc < nv ? kc : nv) : k;
+    // ---- threshold bin b*: count(bins > b*) < kk <= count(bins >= b*)
+    {
+      const int4* g4 = reinterpret_cast<const int4*>(ghist);
+      int4 v[kHistBins / 4 / kSelThreads];
+#pragma unroll
+      for (int u = 0; u < kHistBins / 4 / kSelThreads; ++u) v[u] = __ldcg(g4 + threadIdx.x + u * kSelThreads);
+#pragma unroll
+      for (int u = 0; u < kHistBins / 4 / kSelThreads; ++u) {
+        const int h = 4 * (threadIdx.x + u * kSelThreads);
+        histk[skew(h)] = v[u].x;
+        histk[skew(h + 1)] = v[u].y;
+        histk[skew(h + 2)] = v[u].z;
+        histk[skew(h + 3)] = v[u].w;
+      }
+    }
+    if (threadIdx.x == 0) lcount = 0;
+    __syncthreads();
+    find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, kk, res, scratch);
+    __syncthreads();
+    const uint32_t bstar = (uint32_t)res[0];
+    // ---- this chunk's candidates (each thread loads its scores before using them)
+    const float* srow = scores + row * N;
+    const int64_t c0 = (int64_t)blockIdx.x * chunk;
+    const int64_t c1 = c0 + chunk < nv ? c0 + chunk : nv;
+    for (int64_t base0 = c0; base0 < c1; base0 += (int64_t)kSelPerThread * blockDim.x) {
+      float v[kSelPerThread];
+#pragma unroll
+      for (int u = 0; u < kSelPerThread; ++u) {
+        const int64_t i = base0 + (int64_t)u * blockDim.x + threadIdx.x;
+        v[u] = i < c1 ? __ldg(srow + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kSelPerThread; ++u) {
+        const int64_t i = base0 + (int64_t)u * blockDim.x + threadIdx.x;
+        const uint32_t key = order_key(v[u]);
+        const bool take = i < c1 && (key >> (32 - kHistBits)) >= bstar;
+        const uint32_t m = __ballot_sync(0xffffffffu, take);
+        if (m) {
+          int base = 0;
+          if (lane_id() == 0) base = atomicAdd(&lcount, __popc(m));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (take) {
+            const int slot = base + __popc(m & ((1u << lane_id()) - 1));
+            lidx[slot] = (int32_t)i;
+            lkey[slot] = key;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    nloc = lcount;
+  }
+  if (TC && active && nloc > 0) {
+    // ---- exact rescoring on tcgen05: candidates (M = 128 per batch) x 64 heads, K = 128
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qI) + row * 64 * 128;
+    const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(kI) + row * N * 128;
+    {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(qrow) + threadIdx.x + u * kSelThreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = threadIdx.x + u * kSelThreads, r = j >> 4, c = j & 15;
+        *reinterpret_cast<uint4*>(qt_s + (c >> 3) * 64 * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v[u];
+      }
+    }
+    if (threadIdx.x < 64) wsm[threadIdx.x] = w[row * 64 + threadIdx.x];
+    const uint32_t idesc = make_idesc(128, 64, 1, 0, 0);
+    uint32_t mph = 0;
+    for (int cb = 0; cb < nloc; cb += kSelTcRows) {
+      const int nb = nloc - cb < kSelTcRows ? nloc - cb : kSelTcRows;
+      // gather the batch's key rows (16-byte pieces, all issued before use)
+      uint4 v[kSelTcRows * 16 / kSelThreads];
+#pragma unroll
+      for (int u = 0; u < kSelTcRows * 16 / kSelThreads; ++u) {
+        const int j = threadIdx.x + u * kSelThreads, r = j >> 4, c = j & 15;
+        v[u] = r < nb ? __ldg(reinterpret_cast<const uint4*>(kbase + (int64_t)lidx[cb + r] * 128) + c)
+                      : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kSelTcRows * 16 / kSelThreads; ++u) {
+        const int j = threadIdx.x + u * kSelThreads, r = j >> 4, c = j & 15;
+        *reinterpret_cast<uint4*>(tile_s + (c >> 3) * kSelTcRows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v[u];
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (threadIdx.x == 0) {
+        const uint32_t ab = smem_u32(tile_s), bb = smem_u32(qt_s);
+#pragma unroll
+        for (int kq = 0; kq < 8; ++kq) {
+          const int atom = kq >> 2, inner = (kq & 3) * 32;
+          mma_bf16(tmem_holder, smem_desc(ab + atom * kSelTcRows * 128 + inner, 16, 1024, kLayoutSW128),
+                   smem_desc(bb + atom * 64 * 128 + inner, 16, 1024, kLayoutSW128), idesc, kq > 0 ? 1u : 0u);
+        }
+        mma_commit(&mma_bar);
+      }
+      mbar_wait(&mma_bar, mph);
+      mph ^= 1;
+      tc_fence_after();
+      if (warp_id() < 4) {
+        const int r = warp_id() * 32 + lane_id();           // TMEM lane = candidate row
+        const uint32_t ta = tmem_holder + ((uint32_t)(warp_id() * 32) << 16);
+        float a0[32], a1[32];
+        tmem_ld32(ta, a0);
+        tmem_ld32(ta + 32, a1);
+        tmem_wait_ld();
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+          s0 = fmaf(wsm[h], fmaxf(a0[h], 0.f), s0);
+          s1 = fmaf(wsm[32 + h], fmaxf(a1[h], 0.f), s1);
+        }
+        if (r < nb) lkey[cb + r] = order_key(s0 + s1);
+      }
+      tc_fence_before();
+      __syncthreads();
+    }
+  } else if (RESCORE && !TC && active && nloc > 0) {
+    // ---- exact rescoring on the FMA pipes (fp32 inputs)
+    float* qs = wsm + 64;                                            // [64][129]
+    float* kb = qs + 64 * 129;                                       // [kSelKeyBatch][128]
+    const float* qrow = reinterpret_cast<const float*>(qI) + row * 64 * 128;
+    const float* kbase = reinterpret_cast<const float*>(kI) + row * N * 128;
+    {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(qrow) + threadIdx.x + u * kSelThreads);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e0 = (threadIdx.x + u * kSelThreads) * 4;
+        float f[4];
+        unpack_vec<float>(v[u], f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qs[((e0 + e) >> 7) * 129 + ((e0 + e) & 127)] = f[e];
+      }
+    }
+    if (threadIdx.x < 64) wsm[threadIdx.x] = w[row * 64 + threadIdx.x];
+    const int l = lane_id();
+    for (int cb = 0; cb < nloc; cb += kSelKeyBatch) {
+      const int nb = nloc - cb < kSelKeyBatch ? nloc - cb : kSelKeyBatch;
+      __syncthreads();
+      uint4 v[kSelKeyBatch * 32 / kSelThreads];
+#pragma unroll
+      for (int u = 0; u < kSelKeyBatch * 32 / kSelThreads; ++u) {
+        const int j = threadIdx.x + u * kSelThreads, c = j >> 5, part = j & 31;
+        v[u] = c < nb ? __ldg(reinterpret_cast<const uint4*>(kbase + (int64_t)lidx[cb + c] * 128) + part)
+                      : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kSelKeyBatch * 32 / kSelThreads; ++u) {
+        const int j = threadIdx.x + u * kSelThreads, c = j >> 5, part = j & 31;
+        *reinterpret_cast<uint4*>(kb + c * 128 + part * 4) = v[u];
+      }
+      __syncthreads();
+      for (int c = warp_id(); c < nb; c += kSelThreads / 32) {
+        const float* kr = kb + c * 128;
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < 128; d += 2) {
+          d0 = fmaf(qs[l * 129 + d], kr[d], d0);
+          d1 = fmaf(qs[(l + 32) * 129 + d], kr[d], d1);
+          d2 = fmaf(qs[l * 129 + d + 1], kr[d + 1], d2);
+          d3 = fmaf(qs[(l + 32) * 129 + d + 1], kr[d + 1], d3);
+        }
+        float v2 = wsm[l] * fmaxf(d0 + d2, 0.f) + wsm[l + 32] * fmaxf(d1 + d3, 0.f);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v2 += __shfl_xor_sync(0xffffffffu, v2, o);
+        if (l == 0) lkey[cb + c] = order_key(v2);
+      }
+    }
+    __syncthreads();
+  }
+  if (TC) {
+    __syncthreads();
+    if (warp_id() == 0) tmem_dealloc(tmem_holder, 64);
+  }
+  if (!active) return;
+  // ---- append to the row's candidate list
+  if (threadIdx.x == 0) gslot = nloc > 0 ? atomicAdd(cand_count, nloc) : 0;
+  __syncthreads();
+  for (int c = threadIdx.x; c < nloc; c += blockDim.x) {
+    ckey[gslot + c] = lkey[c];
+    cidx[gslot + c] = lidx[c];
+  }
+  __threadfence();
+  __syncthreads();
+  const int nchunks = (int)((nv + chunk - 1) / chunk);
+  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1) == nchunks - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  // ---- last CTA of the row: exact top-k among the candidates
+  const int nc = *((volatile int*)cand_count);
+  uint32_t* skey = reinterpret_cast<uint32_t*>(sel_smem);
+  int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSelCandSmem);
+  const int64_t words = (N + 31) / 32;
+  uint32_t* bm_gt = reinterpret_cast<uint32_t*>(sidx + kSelCandSmem);
+  uint32_t* bm_eq = bm_gt + words;
+  const bool in_smem = nc <= kSelCandSmem;
+  if (in_smem)
+    for (int i0 = 0; i0 < nc; i0 += 4 * kSelThreads) {
+      uint32_t a[4];
+      int32_t bi[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kSelThreads + threadIdx.x;
+        a[u] = i < nc ? __ldcg(ckey + i) : 0u;
+        bi[u] = i < nc ? __ldcg(cidx + i) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kSelThreads + threadIdx.x;
+        if (i < nc) {
+          skey[i] = a[u];
+          sidx[i] = bi[u];
+        }
+      }
+    }
+  const int64_t used_words = ((int64_t)nv + 31) / 32;
+  for (int64_t j = threadIdx.x; j < used_words; j += blockDim.x) {
+    bm_gt[j] = 0;
+    bm_eq[j] = 0;
+  }
+  __syncthreads();
+  auto cand_key = [&](int i) -> uint32_t { return in_smem ? skey[i] : __ldcg(ckey + i); };
+  auto cand_idx = [&](int i) -> int32_t { return in_smem ? sidx[i] : __ldcg(cidx + i); };
+  // radix select on the 32-bit keys: digits of 11, 11 and 10 bits (skewed 2048-bin histogram)
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = k;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+    for (int j = threadIdx.x; j < 2048 + 64; j += blockDim.x) histk[j] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      const uint32_t key = cand_key(i);
+      if ((key & pmask) == prefix) atomicAdd(&histk[skew((int)((key >> shift) & dmask))], 1);
+    }
+    __syncthreads();
+    find_digit_skewed<2048 / kSelThreads>(histk, 2048, remaining, res, scratch);
+    __syncthreads();
+    prefix |= (uint32_t)res[0] << shift;
+    pmask |= dmask << shift;
+    remaining -= res[1];
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+    const uint32_t key = cand_key(i);
+    const int32_t j = cand_idx(i);
+    if (key > prefix) atomicOr(&bm_gt[j >> 5], 1u << (j & 31));
+    else if (key == prefix) atomicOr(&bm_eq[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  emit_ordered(bm_gt, bm_eq, used_words, remaining, out, scratch);
+  // leave the row's header zeroed for the next call
+  for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
   if (threadIdx.x == 0) {
     *cand_count = 0;
     *done = 0;

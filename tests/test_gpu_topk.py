@@ -6,6 +6,7 @@ import torch
 
 import oracle
 from long_context_compressed_b200 import synth
+from tolerances import check_topk_sets
 
 pytestmark = pytest.mark.gpu
 
@@ -87,3 +88,89 @@ def test_topk_workspace_stays_zero(csa):
         assert np.array_equal(g, oracle.topk(s.numpy(), nv, k))
         torch.cuda.synchronize()
         assert int(ws.count_nonzero()) == 0
+
+
+# ----------------------------------------------------------------------------- fused decode select
+def _order_key(x):
+    u = np.asarray(x, np.float32).view(np.uint32).copy()
+    u[(u << 1) == 0] = 0                                  # -0.0 -> +0.0
+    return np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+
+
+@pytest.mark.parametrize("B,N,k", [(8, 16384, 512), (1, 262144, 1024), (3, 5000, 700), (1, 1 << 19, 2048)])
+def test_select_plain_matches_oracle(csa, B, N, k):
+    """csa_score_histogram + csa_topk_select (no rescoring) == full-sort top-k, bit-exact,
+    twice in a row on the same workspace (which must come back zeroed)."""
+    s = synth.draw_scores(5, f"select/{B}/{N}", B, 1, N, ties=6)
+    nv = np.full((B, 1), N, np.int32)
+    if B >= 3:
+        nv[1, 0] = N // 3
+        nv[2, 0] = k - 5                                  # fewer valid than k
+    ws = csa.select_workspace(B, N)
+    g_s, g_nv = s.cuda(), torch.from_numpy(nv).cuda()
+    ref = oracle.topk(s.numpy(), nv, k)
+    for _ in range(2):
+        csa.csa_score_histogram(g_s, g_nv, ws)
+        got = csa.csa_topk_select(g_s, g_nv, k, ws).cpu().numpy()
+        assert np.array_equal(got, ref)
+    torch.cuda.synchronize()
+    hdr = ws.view(torch.int32)
+    stride = csa.csa_select_workspace_size(1, N) // 4
+    for b in range(B):
+        assert int(hdr[b * stride: b * stride + 4096 + 2].count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_select_rescore_semantics(csa, dtype):
+    """Rescoring mode: candidates are the indices whose (low-precision) score falls in the
+    bin of the kc-th largest score or above; the result is the exact top-k of the plain
+    indexer scores of those candidates (oracle), up to the rescoring error window."""
+    B, N, k, kc = 2, 3000, 100, 200
+    wl = synth.Workload("sel_rescore", dtype, B=B, ctx=4 * N, T=1, q_pos0=4 * N - 1, ratio=4, N=N, H=16, D=128,
+                        index_dtype=dtype)
+    ix = synth.draw_indexer(wl, seed=31)
+    s = synth.draw_scores(31, "select/rescore", B, 1, N)
+    nv = np.array([[N], [N - 777]], np.int32)
+    ws = csa.select_workspace(B, N)
+    g_s, g_nv = s.cuda(), torch.from_numpy(nv).cuda()
+    csa.csa_score_histogram(g_s, g_nv, ws)
+    got = csa.csa_topk_select(g_s, g_nv, k, ws, kc=kc, qI=ix["qI"].cuda(), w=ix["w"].cuda(),
+                              kI=ix["kI"].cuda()).cpu().numpy()
+    for b in range(B):
+        v = s[b, 0, :nv[b, 0]].numpy()
+        order = np.lexsort((np.arange(v.size), -v.astype(np.float64)))
+        bstar = _order_key(v[order[kc - 1]]) >> 20
+        cand = np.nonzero((_order_key(v) >> 20) >= bstar)[0]
+        ex, mag = oracle.index_scores(ix["qI"][b:b + 1].float().numpy(), ix["w"][b:b + 1].numpy(),
+                                      ix["kI"][b:b + 1, cand].float().numpy(), np.array([[len(cand)]], np.int32),
+                                      with_mag=True)
+        pos = [int(np.searchsorted(cand, i)) for i in got[b, 0] if i >= 0]
+        assert np.all(np.isin(got[b, 0], cand))
+        check_topk_sets(pos, ex[0, 0], k, 1e-5 * mag.max(), what=f"select rescore b={b}")
+
+
+def test_select_fed_by_indexer_histogram(csa):
+    """The histogram the indexer epilogue accumulates equals the one the histogram kernel
+    builds from the same scores: both selections are identical (e4m3 decode workload)."""
+    wl = synth.WORKLOADS["flash64k"]
+    ix = synth.draw_indexer(wl)
+    q_pos = np.array([wl.q_pos] * wl.B, np.int64)
+    nv = oracle.n_visible(q_pos, 4, wl.N)
+    g_nv = torch.from_numpy(nv).cuda()
+    qI, kI, w = ix["qI"].cuda(), ix["kI"].cuda(), ix["w"].cuda()
+    q8, qs = csa.csa_quantize_e4m3(qI)
+    k8, ks = csa.csa_quantize_e4m3(kI)
+    ws1, ws2 = csa.select_workspace(wl.B, wl.N), csa.select_workspace(wl.B, wl.N)
+    s_fused = csa.csa_index_scores(q8, w, k8, g_nv, q_scale=qs, k_scale=ks, select_ws=ws1)
+    s_plain = csa.csa_index_scores(q8, w, k8, g_nv, q_scale=qs, k_scale=ks)
+    assert torch.equal(s_fused, s_plain)
+    csa.csa_score_histogram(s_plain, g_nv, ws2)
+    a = csa.csa_topk_select(s_fused, g_nv, wl.topk, ws1, kc=2 * wl.topk, qI=qI, w=w, kI=kI)
+    b = csa.csa_topk_select(s_plain, g_nv, wl.topk, ws2, kc=2 * wl.topk, qI=qI, w=w, kI=kI)
+    assert torch.equal(a, b)
+    ref = oracle.index_scores(ix["qI"].float().numpy(), ix["w"].numpy(), ix["kI"].float().numpy(), nv)
+    idx_ref = oracle.topk(ref.astype(np.float32), nv, wl.topk)
+    got = a.cpu().numpy()
+    recall = min(len(np.intersect1d(got[i, 0], idx_ref[i, 0])) / wl.topk for i in range(wl.B))
+    print(f"flash64k fused e4m3 select recall {recall:.4f}")
+    assert recall >= 0.99
