@@ -130,6 +130,30 @@ int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t 
              void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * csa_topk_noalloc -- csa_topk without a caller-provided workspace.  The pages
+ * have no counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- code that runs while a CUDA stream is being captured (an
+ * allocation there breaks or is refused by the capture), embedded or real-time
+ * hosts that fix their device memory at start-up, and C callers with no device
+ * allocator of their own.
+ *   Same arguments and results as csa_topk, minus the workspace.  Rows that need
+ *   scratch (see csa_topk_workspace_size) use a library-owned device array of
+ *   CSA_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads the library
+ *   holds until the process exits; a call whose csa_topk_workspace_size exceeds
+ *   it returns CSA_ERR_UNSUPPORTED and launches nothing.  No cudaMalloc / cudaFree
+ *   is ever made: the array is cleared with cudaMemsetAsync on `stream` at the
+ *   start of each call.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  All calls share the one array: calls that may
+ *   overlap on the GPU (different streams, or graphs replayed concurrently)
+ *   race and give wrong results -- order them on one stream.
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int csa_topk_noalloc(const float *scores, const int32_t *n_valid, int B, int T, int64_t N, int k, int32_t *idx,
+                     void *stream);
+
+/*
  * csa_index_rerank -- exact rescoring of a candidate list, then top-k among it
  * ([HA] §9: the indexer forms its candidates at twice top-k; this is the
  * second stage that makes a low-precision first pass exact on its candidates).

@@ -36,6 +36,7 @@ _SIGS = {
     "csa_select_workspace_size": ([_i32, _i64], _sz),
     "csa_score_histogram": ([_vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
     "csa_topk_select": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp], _i32),
+    "csa_topk_noalloc": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp], _i32),
     "csa_index_rerank": ([_vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_topk_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "csa_topk": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
@@ -203,6 +204,25 @@ def csa_topk(scores, n_valid, k: int, *, idx=None, workspace=None, stream=None):
         workspace = topk_workspace(B, T, N, k, scores.device)
     _check(_lib.csa_topk(_ptr(scores), _ptr(n_valid), B, T, N, k, _ptr(idx), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream)), "csa_topk")
+    return idx
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def csa_topk_noalloc(scores, n_valid, k: int, *, idx=None, stream=None):
+    """csa_topk for callers that cannot allocate device memory: the scratch is the library's own
+    16 MiB device array (no workspace argument, no allocation inside the call).  Calls that could
+    overlap on the GPU race on that array.  Raises CsaError (CSA_ERR_UNSUPPORTED) when the rows
+    need more scratch than the array holds."""
+    B, T, N = scores.shape
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
+    rc = _lib.csa_topk_noalloc(_ptr(scores), _ptr(n_valid), B, T, N, k, _ptr(idx), _stream(stream))
+    if rc == CSA_ERR_UNSUPPORTED and csa_topk_workspace_size(B, T, N, k) > NOALLOC_SCRATCH_BYTES:
+        raise CsaError(rc, f"csa_topk_noalloc: {csa_topk_workspace_size(B, T, N, k)} bytes of scratch needed, "
+                           f"the static array holds {NOALLOC_SCRATCH_BYTES}")
+    _check(rc, "csa_topk_noalloc")
     return idx
 
 

@@ -552,6 +552,49 @@ int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* s
 
 unsigned long long csa_launch_count(void) { return g_launches.load(); }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free top-k
+// Scratch for csa_topk_noalloc: a file-scope device array, so callers that cannot
+// allocate device memory still get the chunked top-k.  Every GPU that loads this
+// library holds it until the process exits.
+static __device__ __align__(256) uint8_t g_topk_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once per
+// device with that device current (cudaGetSymbolAddress) and cached.
+void* noalloc_scratch_ptr() {
+  static std::mutex mu;
+  static void* ptrs[kMaxDev] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_topk_noalloc_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+}  // namespace
+
+extern "C" {
+
+int csa_topk_noalloc(const float* scores, const int32_t* n_valid, int B, int T, int64_t N, int k, int32_t* idx,
+                     void* stream) {
+  if (B < 0 || T < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (N > (int64_t(1) << 20)) return CSA_ERR_UNSUPPORTED;
+  const size_t need = csa_topk_workspace_size(B, T, N, k);
+  if (need == 0) return csa_topk(scores, n_valid, B, T, N, k, idx, nullptr, 0, stream);   // needs no scratch
+  if (need > (size_t)CSA_NOALLOC_SCRATCH_BYTES) return CSA_ERR_UNSUPPORTED;                 // beyond the array
+  void* scratch = noalloc_scratch_ptr();
+  if (scratch == nullptr) return CSA_ERR_CUDA;
+  // the array keeps the previous call's contents: clear the part this call relies on being zero
+  if (cudaMemsetAsync(scratch, 0, need, as_stream(stream)) != cudaSuccess) return CSA_ERR_CUDA;
+  return csa_topk(scores, n_valid, B, T, N, k, idx, scratch, need, stream);
+}
+
 int csa_poll_status(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CSA_ERR_CUDA;
   int v = 0;
