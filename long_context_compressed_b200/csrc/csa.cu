@@ -488,15 +488,15 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
     launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr);
     return launch_status();
   }
-  // chunks: about two CTAs per SM in total, at least 256 entries each
+  // chunks: one wave (at most one CTA per SM over all rows), at least 512 entries each
   const int sms = sm_count();
-  int64_t nchunks = std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (2 * sms + B - 1) / B));
+  int64_t nchunks = std::max<int64_t>(1, std::min<int64_t>((N + 511) / 512, std::max(1, sms / std::max(B, 1))));
   int chunk = (int)(((N + nchunks - 1) / nchunks + 255) / 256 * 256);
   nchunks = (N + chunk - 1) / chunk;
-  const int64_t words = (N + 31) / 32;
-  const int phase3 = csa::kSelTileBytes + csa::kSelQBytes + chunk * 8 +
-                     (64 + 64 * 129 + csa::kSelKeyBatch * 128) * 4;
-  const int phase4 = (int)(2 * csa::kSelCandSmem * 4 + 2 * words * 4);
+  const bool tc = rescore && dtype == CSA_BF16;
+  const int phase3 = csa::kSelTileBytes + csa::kSelQBytes + chunk * 8 + 64 * 4 +
+                     (rescore && !tc ? (64 * 129 + csa::kSelKeyBatch * 128) * 4 : 0);
+  const int phase4 = (int)(2 * csa::kSelCandSmem * 4 + 2 * CSA_MAX_TOPK * 4 + (nchunks + 1) * 4);
   const int smem = 1024 + std::max(phase3, phase4);
   cudaStream_t st = as_stream(stream);
   dim3 grid((unsigned)nchunks, (unsigned)B);

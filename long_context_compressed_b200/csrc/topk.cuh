@@ -426,7 +426,7 @@ constexpr int kSelThreads = 256;
 constexpr int kSelPerThread = 4;     // scores each thread loads per pass of the chunk scan
 constexpr int kSelTcRows = 128;      // candidates rescored per tensor-core batch (bf16)
 constexpr int kSelKeyBatch = 64;     // candidate key rows per SIMT batch (fp32)
-constexpr int kSelCandSmem = 4096;   // candidates the last CTA stages in shared memory
+constexpr int kSelCandSmem = 8192;   // candidates the last CTA stages in shared memory
 constexpr int64_t kSelMaxN = int64_t(1) << 19;
 constexpr int kSelTileBytes = 2 * kSelTcRows * 128;    // candidate key tile, 2 x 128-byte K atoms (bf16)
 constexpr int kSelQBytes = 2 * 64 * 128;               // q tile: 64 heads x 128 dims bf16
@@ -480,86 +480,14 @@ __device__ __forceinline__ void find_digit_skewed(const int* hist, int nbins, in
   }
 }
 
-// Write, in ascending index order, every index set in bm_gt and the first r_eq
-// (lowest) indices set in bm_eq, for words [0, used_words).  Warp w walks a
-// contiguous segment of words 32 at a time (lane l reads word base + l: no bank
-// conflicts); per-warp totals are scanned to give each warp its output offset.
-__device__ __forceinline__ void emit_ordered(const uint32_t* bm_gt, const uint32_t* bm_eq, int64_t used_words,
-                                             int r_eq, int32_t* out, int* scratch) {
-  const int nwarps = blockDim.x >> 5, warp = warp_id(), lane = lane_id();
-  const int64_t per = ((used_words + nwarps - 1) / nwarps + 31) / 32 * 32;
-  const int64_t s0 = (int64_t)warp * per < used_words ? (int64_t)warp * per : used_words;
-  const int64_t s1 = s0 + per < used_words ? s0 + per : used_words;
-  int gt = 0, eq = 0;
-  for (int64_t w = s0 + lane; w < s1; w += 32) {
-    gt += __popc(bm_gt[w]);
-    eq += __popc(bm_eq[w]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    gt += __shfl_xor_sync(0xffffffffu, gt, o);
-    eq += __shfl_xor_sync(0xffffffffu, eq, o);
-  }
-  __syncthreads();
-  if (lane == 0) {
-    scratch[warp] = gt;
-    scratch[16 + warp] = eq;
-  }
-  __syncthreads();
-  int sel_before = 0, eq_before = 0;
-  for (int v = 0; v < warp; ++v) {
-    const int eb = eq_before;
-    int te = r_eq - eb;
-    te = te < 0 ? 0 : (te > scratch[16 + v] ? scratch[16 + v] : te);
-    sel_before += scratch[v] + te;
-    eq_before += scratch[16 + v];
-  }
-  int run_sel = sel_before, run_eq = eq_before;
-  for (int64_t base = s0; base < s1; base += 32) {
-    const int64_t w = base + lane;
-    const uint32_t g = w < s1 ? bm_gt[w] : 0u;
-    const uint32_t e = w < s1 ? bm_eq[w] : 0u;
-    const int ce = __popc(e);
-    int ie = ce;                                      // inclusive scan of eq counts over lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, ie, o);
-      if (lane >= o) ie += n;
-    }
-    int te = r_eq - (run_eq + ie - ce);
-    te = te < 0 ? 0 : (te > ce ? ce : te);
-    uint32_t etake = 0, x = e;
-    for (int t = 0; t < te; ++t) {
-      const uint32_t bbit = x & (0u - x);
-      etake |= bbit;
-      x ^= bbit;
-    }
-    uint32_t sel = g | etake;
-    const int cs = __popc(sel);
-    int is = cs;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, is, o);
-      if (lane >= o) is += n;
-    }
-    int pos = run_sel + is - cs;
-    while (sel) {
-      const int bit = __ffs(sel) - 1;
-      out[pos++] = (int32_t)(w * 32 + bit);
-      sel &= sel - 1;
-    }
-    run_sel += __shfl_sync(0xffffffffu, is, 31);
-    run_eq += __shfl_sync(0xffffffffu, ie, 31);
-  }
-}
-
 // Row r (one query per sequence: T == 1) of scores [rows, N].  Candidates are the
 // indices whose score lies in the histogram bin of the kk-th largest score or above
 // (kk = kc when RESCORE, else k) -- a superset of the kk largest.  With RESCORE each
 // candidate is rescored with the plain indexer definition on full-precision qI / kI
 // (fp32 accumulation; bf16 inputs on tcgen05, fp32 inputs on the FMA pipes); the
 // exact top-k of the (re)scored candidates, lower index first among equal scores, is
-// written in ascending index order by the last CTA of the row.
+// written in ascending index order by the last CTA of the row (chunks are contiguous
+// index ranges: the k indices are bucketed by chunk and ranked inside their bucket).
 template <bool RESCORE, typename Tin>
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* __restrict__ scores,
                                                                   const int32_t* __restrict__ n_valid, int64_t N,
@@ -814,9 +742,9 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   const int nc = *((volatile int*)cand_count);
   uint32_t* skey = reinterpret_cast<uint32_t*>(sel_smem);
   int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSelCandSmem);
-  const int64_t words = (N + 31) / 32;
-  uint32_t* bm_gt = reinterpret_cast<uint32_t*>(sidx + kSelCandSmem);
-  uint32_t* bm_eq = bm_gt + words;
+  int32_t* sel = sidx + kSelCandSmem;                    // [k] selected indices, then bucketed
+  int32_t* bucket = sel + CSA_MAX_TOPK;                  // [k] indices grouped by chunk
+  int* ccount = bucket + CSA_MAX_TOPK;                   // [nchunks + 1] per-chunk counts -> offsets
   const bool in_smem = nc <= kSelCandSmem;
   if (in_smem)
     for (int i0 = 0; i0 < nc; i0 += 4 * kSelThreads) {
@@ -837,11 +765,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         }
       }
     }
-  const int64_t used_words = ((int64_t)nv + 31) / 32;
-  for (int64_t j = threadIdx.x; j < used_words; j += blockDim.x) {
-    bm_gt[j] = 0;
-    bm_eq[j] = 0;
-  }
+  for (int j = threadIdx.x; j <= nchunks; j += blockDim.x) ccount[j] = 0;
   __syncthreads();
   auto cand_key = [&](int i) -> uint32_t { return in_smem ? skey[i] : __ldcg(ckey + i); };
   auto cand_idx = [&](int i) -> int32_t { return in_smem ? sidx[i] : __ldcg(cidx + i); };
@@ -865,14 +789,107 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     remaining -= res[1];
     __syncthreads();
   }
-  for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-    const uint32_t key = cand_key(i);
-    const int32_t j = cand_idx(i);
-    if (key > prefix) atomicOr(&bm_gt[j >> 5], 1u << (j & 31));
-    else if (key == prefix) atomicOr(&bm_eq[j >> 5], 1u << (j & 31));
+  // selected = keys above K*, plus the `remaining` lowest indices among keys equal to K*.
+  // Slots come from warp-aggregated atomics (one per warp, or per distinct chunk within a
+  // warp) -- contended shared-memory atomics serialise lane by lane.
+  int32_t* eqlist = bucket;                              // keys equal to K* (scratch, before bucketing)
+  if (threadIdx.x == 0) {
+    lcount = 0;
+    gslot = 0;
   }
   __syncthreads();
-  emit_ordered(bm_gt, bm_eq, used_words, remaining, out, scratch);
+  for (int i0 = 0; i0 < nc; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const uint32_t key = i < nc ? cand_key(i) : 0u;
+    const bool gt = i < nc && key > prefix;
+    const bool eq = i < nc && key == prefix;
+    const uint32_t mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
+    int bg = 0, be = 0;
+    if (lane_id() == 0) {
+      if (mg) bg = atomicAdd(&lcount, __popc(mg));
+      if (me) be = atomicAdd(&gslot, __popc(me));
+    }
+    bg = __shfl_sync(0xffffffffu, bg, 0);
+    be = __shfl_sync(0xffffffffu, be, 0);
+    const uint32_t below = (1u << lane_id()) - 1;
+    if (gt) sel[bg + __popc(mg & below)] = cand_idx(i);
+    if (eq && be + __popc(me & below) < CSA_MAX_TOPK) eqlist[be + __popc(me & below)] = cand_idx(i);
+  }
+  __syncthreads();
+  const int ngt = lcount, neq = gslot;
+  // the `remaining` lowest indices among the equal keys (rank = equal keys with a lower index)
+  if (neq <= CSA_MAX_TOPK) {
+    for (int e = threadIdx.x; e < neq; e += blockDim.x) {
+      const int32_t j = eqlist[e];
+      int rank = 0;
+      for (int q = 0; q < neq; ++q) rank += eqlist[q] < j;
+      if (rank < remaining) sel[ngt + rank] = j;
+    }
+  } else {
+    // more ties than the list holds (degenerate rows, e.g. constant scores): rank against
+    // the whole candidate list
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      if (cand_key(i) != prefix) continue;
+      const int32_t j = cand_idx(i);
+      int rank = 0;
+      for (int q = 0; q < nc && rank < remaining; ++q) rank += (cand_key(q) == prefix && cand_idx(q) < j);
+      if (rank < remaining) sel[ngt + rank] = j;
+    }
+  }
+  __syncthreads();
+  const int nsel = ngt + (remaining < neq ? remaining : neq);   // == k (nv > k)
+  // ascending order: chunks are contiguous index ranges, so order = (chunk, rank in chunk)
+  for (int i0 = 0; i0 < nsel; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const bool act = i < nsel;
+    const int c = act ? sel[i] / chunk : -1;
+    const uint32_t m = __ballot_sync(0xffffffffu, act);
+    if (act) {
+      const uint32_t peers = __match_any_sync(m, c);
+      if ((int)lane_id() == __ffs(peers) - 1) atomicAdd(&ccount[c], __popc(peers));
+    }
+  }
+  __syncthreads();
+  {
+    int total;
+    const int per = (nchunks + blockDim.x - 1) / blockDim.x;
+    int loc = 0;
+    for (int c = threadIdx.x * per; c < (int)(threadIdx.x + 1) * per && c < nchunks; ++c) loc += ccount[c];
+    int off = block_excl_scan(loc, scratch, &total);
+    __syncthreads();
+    for (int c = threadIdx.x * per; c < (int)(threadIdx.x + 1) * per && c < nchunks; ++c) {
+      const int n = ccount[c];
+      ccount[c] = off;                                   // start of chunk c's bucket
+      off += n;
+    }
+  }
+  __syncthreads();
+  for (int i0 = 0; i0 < nsel; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const bool act = i < nsel;
+    const int32_t j = act ? sel[i] : 0;
+    const int c = act ? j / chunk : -1;
+    const uint32_t m = __ballot_sync(0xffffffffu, act);
+    if (act) {
+      const uint32_t peers = __match_any_sync(m, c);
+      const int leader = __ffs(peers) - 1;
+      int base = 0;
+      if ((int)lane_id() == leader) base = atomicAdd(&ccount[c], __popc(peers));
+      base = __shfl_sync(peers, base, leader);
+      bucket[base + __popc(peers & ((1u << lane_id()) - 1))] = j;   // ccount ends at the bucket's end
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
+    const int32_t j = bucket[i];
+    const int c = j / chunk;
+    const int b_end = ccount[c];                         // end of this chunk's bucket
+    const int b_start = c > 0 ? ccount[c - 1] : 0;       // = end of the previous bucket
+    int rank = 0;
+    for (int q = b_start; q < b_end; ++q) rank += bucket[q] < j;
+    out[b_start + rank] = j;
+  }
+  __syncthreads();
   // leave the row's header zeroed for the next call
   for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
   if (threadIdx.x == 0) {

@@ -174,3 +174,24 @@ def test_select_fed_by_indexer_histogram(csa):
     recall = min(len(np.intersect1d(got[i, 0], idx_ref[i, 0])) / wl.topk for i in range(wl.B))
     print(f"flash64k fused e4m3 select recall {recall:.4f}")
     assert recall >= 0.99
+
+
+@pytest.mark.parametrize("N", [3000, 50000])
+def test_select_degenerate_ties(csa, N):
+    """Fused select on rows dominated by ties: a constant row (every candidate ties with
+    the k-th score, more ties than the tie list holds), a +-0.0 row, and a row with k-1
+    values above a tied block -- the k lowest tied indices must win, as in the full sort."""
+    B, k = 3, 512
+    s = torch.zeros(B, 1, N)
+    s[0, 0] = 3.25
+    s[1, 0] = torch.where(torch.arange(N) % 3 == 0, torch.tensor(-0.0), torch.tensor(0.0))
+    s[2, 0] = 1.0
+    pos = torch.unique((synth.uniform(7, f"select/eqpos/{N}", (4 * k,)) * N).long())[: k - 1]
+    s[2, 0, pos] = 2.0
+    nv = np.full((B, 1), N, np.int32)
+    ws = csa.select_workspace(B, N)
+    g_s, g_nv = s.cuda(), torch.from_numpy(nv).cuda()
+    csa.csa_score_histogram(g_s, g_nv, ws)
+    got = csa.csa_topk_select(g_s, g_nv, k, ws).cpu().numpy()
+    assert np.array_equal(got, oracle.topk(s.numpy(), nv, k))
+    assert got[0, 0].tolist() == list(range(k))
