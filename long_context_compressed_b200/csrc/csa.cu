@@ -488,15 +488,20 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
     launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr);
     return launch_status();
   }
-  // chunks: one wave (at most one CTA per SM over all rows), at least 512 entries each
+  // chunks: one wave (at most one CTA per SM over all rows), at least 512 entries each,
+  // at most kSelMaxChunkLen (the chunk's candidate list lives in shared memory)
   const int sms = sm_count();
   int64_t nchunks = std::max<int64_t>(1, std::min<int64_t>((N + 511) / 512, std::max(1, sms / std::max(B, 1))));
+  nchunks = std::max<int64_t>(nchunks, (N + csa::kSelMaxChunkLen - 1) / csa::kSelMaxChunkLen);
+  nchunks = std::min<int64_t>(nchunks, csa::kSelMaxChunks);
   int chunk = (int)(((N + nchunks - 1) / nchunks + 255) / 256 * 256);
   nchunks = (N + chunk - 1) / chunk;
   const bool tc = rescore && dtype == CSA_BF16;
   const int phase3 = csa::kSelTileBytes + csa::kSelQBytes + chunk * 8 + 64 * 4 +
                      (rescore && !tc ? (64 * 129 + csa::kSelKeyBatch * 128) * 4 : 0);
-  const int phase4 = (int)(2 * csa::kSelCandSmem * 4 + 2 * CSA_MAX_TOPK * 4 + (nchunks + 1) * 4);
+  // last CTA: staged candidates + chunk table, or (overflow) the bucketed selection
+  const int phase4 = (int)std::max<int64_t>(2 * csa::kSelCandSmem * 4 + 2 * csa::kSelMaxChunks * 4,
+                                            2 * CSA_MAX_TOPK * 4 + (nchunks + 1) * 4);
   const int smem = 1024 + std::max(phase3, phase4);
   cudaStream_t st = as_stream(stream);
   dim3 grid((unsigned)nchunks, (unsigned)B);

@@ -246,6 +246,14 @@ __device__ __forceinline__ void griddep_sync() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Device-scope fetch-and-add with acquire-release order: a CTA's writes before the
+// preceding barrier are visible to whichever CTA later reads the counter this way.
+__device__ __forceinline__ unsigned long long atom_add_acq_rel(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 

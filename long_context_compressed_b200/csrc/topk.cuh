@@ -412,12 +412,15 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
 }
 
 // ---------------------------------------------------------------- fused select (decode)
-// Per-row workspace of topk_select_kernel: [4096-bin histogram][candidate count]
-// [finished CTAs][pad] then candidate keys [N] and indices [N].  The histogram is
+// Per-row workspace of topk_select_kernel: [4096-bin histogram][64-bit counter:
+// candidates appended (low word) | CTAs finished (high word)][slot counter][pad]
+// [per-chunk (first slot, count) table] then candidate keys [N] and indices [N].  The histogram is
 // accumulated by the indexer (csa_index_scores with this workspace); the last CTA
 // of each row leaves the row's header zeroed for the next call.
+constexpr int kSelMaxChunks = 1024;   // chunks per row (table in the row header)
 struct SelectWs {
-  static constexpr int64_t kHeaderInts = kHistBins + 64;
+  static constexpr int64_t kTableInt = kHistBins + 64;            // [chunk] -> (first slot, count)
+  static constexpr int64_t kHeaderInts = kTableInt + 2 * kSelMaxChunks;
   static __host__ __device__ int64_t row_bytes(int64_t N) {
     return ((kHeaderInts + 2 * N) * 4 + 15) / 16 * 16;
   }
@@ -427,6 +430,9 @@ constexpr int kSelPerThread = 4;     // scores each thread loads per pass of the
 constexpr int kSelTcRows = 128;      // candidates rescored per tensor-core batch (bf16)
 constexpr int kSelKeyBatch = 64;     // candidate key rows per SIMT batch (fp32)
 constexpr int kSelCandSmem = 8192;   // candidates the last CTA stages in shared memory
+constexpr int kSelMaxChunkLen = 16384;  // entries per chunk (shared-memory candidate list)
+static_assert(kSelPerThread * (kSelThreads / 32) == 32, "one scan lane per (pass, warp)");
+static_assert(kSelMaxChunks % kSelThreads == 0, "chunk table split evenly over the threads");
 constexpr int64_t kSelMaxN = int64_t(1) << 19;
 constexpr int kSelTileBytes = 2 * kSelTcRows * 128;    // candidate key tile, 2 x 128-byte K atoms (bf16)
 constexpr int kSelQBytes = 2 * 64 * 128;               // q tile: 64 heads x 128 dims bf16
@@ -503,6 +509,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   __shared__ int scratch[33];
   __shared__ int res[2];
   __shared__ int lcount, gslot, is_last;
+  __shared__ int wcnt[32], wexc[33];
+  __shared__ uint32_t kext[2];
   __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_holder;
   if (TC) {
@@ -524,8 +532,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   nv = nv < 0 ? 0 : (nv > (int)N ? (int)N : nv);
   uint8_t* rws = ws + row * SelectWs::row_bytes(N);
   int* ghist = reinterpret_cast<int*>(rws);
-  int* cand_count = ghist + kHistBins;
-  int* done = cand_count + 1;
+  // header: [candidates appended | CTAs finished] as one 64-bit counter, then the slot counter
+  unsigned long long* fin = reinterpret_cast<unsigned long long*>(ghist + kHistBins);
+  int* slots = ghist + kHistBins + 2;
+  int* ctab = reinterpret_cast<int*>(rws) + SelectWs::kTableInt;
   uint32_t* ckey = reinterpret_cast<uint32_t*>(rws + SelectWs::kHeaderInts * 4);
   int32_t* cidx = reinterpret_cast<int32_t*>(ckey + N);
   int32_t* out = idx + row * k;
@@ -565,10 +575,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, kk, res, scratch);
     __syncthreads();
     const uint32_t bstar = (uint32_t)res[0];
-    // ---- this chunk's candidates (each thread loads its scores before using them)
+    // ---- this chunk's candidates, compacted in index order (each thread loads its
+    // scores before using them; one warp scans the 32 (pass, warp) counts)
     const float* srow = scores + row * N;
     const int64_t c0 = (int64_t)blockIdx.x * chunk;
     const int64_t c1 = c0 + chunk < nv ? c0 + chunk : nv;
+    int lbase = 0;
     for (int64_t base0 = c0; base0 < c1; base0 += (int64_t)kSelPerThread * blockDim.x) {
       float v[kSelPerThread];
 #pragma unroll
@@ -576,26 +588,34 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         const int64_t i = base0 + (int64_t)u * blockDim.x + threadIdx.x;
         v[u] = i < c1 ? __ldg(srow + i) : 0.f;
       }
+      uint32_t key[kSelPerThread], m[kSelPerThread];
 #pragma unroll
       for (int u = 0; u < kSelPerThread; ++u) {
         const int64_t i = base0 + (int64_t)u * blockDim.x + threadIdx.x;
-        const uint32_t key = order_key(v[u]);
-        const bool take = i < c1 && (key >> (32 - kHistBits)) >= bstar;
-        const uint32_t m = __ballot_sync(0xffffffffu, take);
-        if (m) {
-          int base = 0;
-          if (lane_id() == 0) base = atomicAdd(&lcount, __popc(m));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (take) {
-            const int slot = base + __popc(m & ((1u << lane_id()) - 1));
-            lidx[slot] = (int32_t)i;
-            lkey[slot] = key;
-          }
-        }
+        key[u] = order_key(v[u]);
+        m[u] = __ballot_sync(0xffffffffu, i < c1 && (key[u] >> (32 - kHistBits)) >= bstar);
+        if (lane_id() == 0) wcnt[u * (kSelThreads / 32) + warp_id()] = __popc(m[u]);
       }
+      __syncthreads();
+      if (warp_id() == 0) {
+        const int x = wcnt[lane_id()];
+        const int xi = warp_incl_scan(x);
+        wexc[lane_id()] = xi - x;
+        if (lane_id() == 31) wexc[32] = xi;
+      }
+      __syncthreads();
+      const uint32_t below = (1u << lane_id()) - 1;
+#pragma unroll
+      for (int u = 0; u < kSelPerThread; ++u)
+        if (m[u] >> lane_id() & 1u) {
+          const int slot = lbase + wexc[u * (kSelThreads / 32) + warp_id()] + __popc(m[u] & below);
+          lidx[slot] = (int32_t)(base0 + (int64_t)u * blockDim.x + threadIdx.x);
+          lkey[slot] = key[u];
+        }
+      lbase += wexc[32];
     }
     __syncthreads();
-    nloc = lcount;
+    nloc = lbase;
   }
   if (TC && active && nloc > 0) {
     // ---- exact rescoring on tcgen05: candidates (M = 128 per batch) x 64 heads, K = 128
@@ -725,176 +745,295 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   }
   if (!active) return;
   // ---- append to the row's candidate list
-  if (threadIdx.x == 0) gslot = nloc > 0 ? atomicAdd(cand_count, nloc) : 0;
+  if (threadIdx.x == 0) {
+    const int g = nloc > 0 ? atomicAdd(slots, nloc) : 0;
+    gslot = g;
+    reinterpret_cast<int2*>(ctab)[blockIdx.x] = make_int2(g, nloc);
+  }
   __syncthreads();
   for (int c = threadIdx.x; c < nloc; c += blockDim.x) {
     ckey[gslot + c] = lkey[c];
     cidx[gslot + c] = lidx[c];
   }
-  __threadfence();
   __syncthreads();
   const int nchunks = (int)((nv + chunk - 1) / chunk);
-  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1) == nchunks - 1);
+  if (threadIdx.x == 0) {
+    // one counter tells the last CTA both that it is last and how many candidates there are
+    const unsigned long long old = atom_add_acq_rel(fin, (1ull << 32) | (unsigned)nloc);
+    is_last = (int)(old >> 32) == nchunks - 1;
+    lcount = (int)(uint32_t)old + nloc;
+  }
   __syncthreads();
   if (!is_last) return;
-  __threadfence();
   // ---- last CTA of the row: exact top-k among the candidates
-  const int nc = *((volatile int*)cand_count);
-  uint32_t* skey = reinterpret_cast<uint32_t*>(sel_smem);
-  int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSelCandSmem);
-  int32_t* sel = sidx + kSelCandSmem;                    // [k] selected indices, then bucketed
-  int32_t* bucket = sel + CSA_MAX_TOPK;                  // [k] indices grouped by chunk
-  int* ccount = bucket + CSA_MAX_TOPK;                   // [nchunks + 1] per-chunk counts -> offsets
-  const bool in_smem = nc <= kSelCandSmem;
-  if (in_smem)
-    for (int i0 = 0; i0 < nc; i0 += 4 * kSelThreads) {
-      uint32_t a[4];
-      int32_t bi[4];
+  const int nc = lcount;
+  if (nc <= kSelCandSmem) {
+    // Stage the candidates in index order: chunk c's list (index-ordered by the scan)
+    // goes to offset pre[c] = the earlier chunks' counts.  Loads of the chunk table
+    // and of the first candidates are issued together.
+    uint32_t* okey = reinterpret_cast<uint32_t*>(sel_smem);
+    int32_t* oidx = reinterpret_cast<int32_t*>(okey + kSelCandSmem);
+    int* tslot = oidx + kSelCandSmem;                    // [chunk] first slot of its list
+    int* tpre = tslot + kSelMaxChunks;                   // [chunk] offset of its list in index order
+    constexpr int CPT = kSelMaxChunks / kSelThreads;
+    constexpr int U = 16;                                // candidates per thread per batch
+    int2 ct[CPT];                                        // (first slot, count) of this thread's chunks
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * kSelThreads + threadIdx.x;
-        a[u] = i < nc ? __ldcg(ckey + i) : 0u;
-        bi[u] = i < nc ? __ldcg(cidx + i) : 0;
+    for (int u = 0; u < CPT; ++u) {
+      const int c = threadIdx.x * CPT + u;
+      ct[u] = c < nchunks ? __ldcg(reinterpret_cast<const int2*>(ctab) + c) : make_int2(0, 0);
+    }
+    uint32_t ck[U];
+    int32_t ci[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = u * kSelThreads + threadIdx.x;
+      ck[u] = i < nc ? __ldcg(ckey + i) : 0u;
+      ci[u] = i < nc ? __ldcg(cidx + i) : 0;
+    }
+    if (threadIdx.x == 0) {
+      kext[0] = 0xffffffffu;
+      kext[1] = 0u;
+    }
+    {
+      int local = 0;
+#pragma unroll
+      for (int u = 0; u < CPT; ++u) local += ct[u].y;
+      int total;
+      int off = block_excl_scan(local, scratch, &total);
+#pragma unroll
+      for (int u = 0; u < CPT; ++u) {
+        const int c = threadIdx.x * CPT + u;
+        if (c < nchunks) {
+          tslot[c] = ct[u].x;
+          tpre[c] = off;
+        }
+        off += ct[u].y;
       }
+    }
+    __syncthreads();
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    const float inv_chunk = 1.f / (float)chunk;
+    for (int i0 = 0;;) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int i = i0 + u * kSelThreads + threadIdx.x;
         if (i < nc) {
-          skey[i] = a[u];
-          sidx[i] = bi[u];
+          int c = (int)((float)ci[u] * inv_chunk);        // ci / chunk, corrected below
+          c -= c * chunk > ci[u];
+          c += (c + 1) * chunk <= ci[u];
+          const int pos = tpre[c] + (i - tslot[c]);
+          okey[pos] = ck[u];
+          oidx[pos] = ci[u];
+          kmin = min(kmin, ck[u]);
+          kmax = max(kmax, ck[u]);
         }
       }
+      i0 += U * kSelThreads;
+      if (i0 >= nc) break;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * kSelThreads + threadIdx.x;
+        ck[u] = i < nc ? __ldcg(ckey + i) : 0u;
+        ci[u] = i < nc ? __ldcg(cidx + i) : 0;
+      }
     }
-  for (int j = threadIdx.x; j <= nchunks; j += blockDim.x) ccount[j] = 0;
-  __syncthreads();
-  auto cand_key = [&](int i) -> uint32_t { return in_smem ? skey[i] : __ldcg(ckey + i); };
-  auto cand_idx = [&](int i) -> int32_t { return in_smem ? sidx[i] : __ldcg(cidx + i); };
-  // radix select on the 32-bit keys: digits of 11, 11 and 10 bits (skewed 2048-bin histogram)
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = k;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const uint32_t dmask = pass == 2 ? 1023u : 2047u;
-    for (int j = threadIdx.x; j < 2048 + 64; j += blockDim.x) histk[j] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-      const uint32_t key = cand_key(i);
-      if ((key & pmask) == prefix) atomicAdd(&histk[skew((int)((key >> shift) & dmask))], 1);
-    }
-    __syncthreads();
-    find_digit_skewed<2048 / kSelThreads>(histk, 2048, remaining, res, scratch);
-    __syncthreads();
-    prefix |= (uint32_t)res[0] << shift;
-    pmask |= dmask << shift;
-    remaining -= res[1];
-    __syncthreads();
-  }
-  // selected = keys above K*, plus the `remaining` lowest indices among keys equal to K*.
-  // Slots come from warp-aggregated atomics (one per warp, or per distinct chunk within a
-  // warp) -- contended shared-memory atomics serialise lane by lane.
-  int32_t* eqlist = bucket;                              // keys equal to K* (scratch, before bucketing)
-  if (threadIdx.x == 0) {
-    lcount = 0;
-    gslot = 0;
-  }
-  __syncthreads();
-  for (int i0 = 0; i0 < nc; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const uint32_t key = i < nc ? cand_key(i) : 0u;
-    const bool gt = i < nc && key > prefix;
-    const bool eq = i < nc && key == prefix;
-    const uint32_t mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
-    int bg = 0, be = 0;
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
     if (lane_id() == 0) {
-      if (mg) bg = atomicAdd(&lcount, __popc(mg));
-      if (me) be = atomicAdd(&gslot, __popc(me));
+      atomicMin(&kext[0], kmin);
+      atomicMax(&kext[1], kmax);
     }
-    bg = __shfl_sync(0xffffffffu, bg, 0);
-    be = __shfl_sync(0xffffffffu, be, 0);
-    const uint32_t below = (1u << lane_id()) - 1;
-    if (gt) sel[bg + __popc(mg & below)] = cand_idx(i);
-    if (eq && be + __popc(me & below) < CSA_MAX_TOPK) eqlist[be + __popc(me & below)] = cand_idx(i);
-  }
-  __syncthreads();
-  const int ngt = lcount, neq = gslot;
-  // the `remaining` lowest indices among the equal keys (rank = equal keys with a lower index)
-  if (neq <= CSA_MAX_TOPK) {
-    for (int e = threadIdx.x; e < neq; e += blockDim.x) {
-      const int32_t j = eqlist[e];
-      int rank = 0;
-      for (int q = 0; q < neq; ++q) rank += eqlist[q] < j;
-      if (rank < remaining) sel[ngt + rank] = j;
-    }
-  } else {
-    // more ties than the list holds (degenerate rows, e.g. constant scores): rank against
-    // the whole candidate list
-    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-      if (cand_key(i) != prefix) continue;
-      const int32_t j = cand_idx(i);
-      int rank = 0;
-      for (int q = 0; q < nc && rank < remaining; ++q) rank += (cand_key(q) == prefix && cand_idx(q) < j);
-      if (rank < remaining) sel[ngt + rank] = j;
-    }
-  }
-  __syncthreads();
-  const int nsel = ngt + (remaining < neq ? remaining : neq);   // == k (nv > k)
-  // ascending order: chunks are contiguous index ranges, so order = (chunk, rank in chunk)
-  for (int i0 = 0; i0 < nsel; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const bool act = i < nsel;
-    const int c = act ? sel[i] / chunk : -1;
-    const uint32_t m = __ballot_sync(0xffffffffu, act);
-    if (act) {
-      const uint32_t peers = __match_any_sync(m, c);
-      if ((int)lane_id() == __ffs(peers) - 1) atomicAdd(&ccount[c], __popc(peers));
-    }
-  }
-  __syncthreads();
-  {
-    int total;
-    const int per = (nchunks + blockDim.x - 1) / blockDim.x;
-    int loc = 0;
-    for (int c = threadIdx.x * per; c < (int)(threadIdx.x + 1) * per && c < nchunks; ++c) loc += ccount[c];
-    int off = block_excl_scan(loc, scratch, &total);
     __syncthreads();
-    for (int c = threadIdx.x * per; c < (int)(threadIdx.x + 1) * per && c < nchunks; ++c) {
-      const int n = ccount[c];
-      ccount[c] = off;                                   // start of chunk c's bucket
-      off += n;
+    kmin = kext[0];
+    const uint32_t span = kext[1] - kmin;
+    // radix select on u = key - kmin, 12-bit digits from the highest bit of the span down
+    // (the candidates share their leading key bits, so the digits spread over the bins)
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+    for (int hi = span ? 32 - __clz(span) : 0; hi > 0;) {
+      const int lo = hi > kHistBits ? hi - kHistBits : 0;
+      const uint32_t dmask = (1u << (hi - lo)) - 1;
+      for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) histk[j] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+        const uint32_t u = okey[i] - kmin;
+        if ((u & pmask) == prefix) atomicAdd(&histk[skew((int)((u >> lo) & dmask))], 1);
+      }
+      __syncthreads();
+      find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, remaining, res, scratch);
+      __syncthreads();
+      prefix |= (uint32_t)res[0] << lo;
+      pmask |= dmask << lo;
+      remaining -= res[1];
+      hi = lo;
     }
-  }
-  __syncthreads();
-  for (int i0 = 0; i0 < nsel; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const bool act = i < nsel;
-    const int32_t j = act ? sel[i] : 0;
-    const int c = act ? j / chunk : -1;
-    const uint32_t m = __ballot_sync(0xffffffffu, act);
-    if (act) {
-      const uint32_t peers = __match_any_sync(m, c);
-      const int leader = __ffs(peers) - 1;
-      int base = 0;
-      if ((int)lane_id() == leader) base = atomicAdd(&ccount[c], __popc(peers));
-      base = __shfl_sync(peers, base, leader);
-      bucket[base + __popc(peers & ((1u << lane_id()) - 1))] = j;   // ccount ends at the bucket's end
+    // ordered emit: every key above K*, and the first `remaining` keys equal to K* (the
+    // staged order is index order); each thread walks a contiguous run of odd length
+    // (conflict-free banks) after one block scan of its (above, equal) counts
+    const int per = ((nc + kSelThreads - 1) / kSelThreads) | 1;
+    const int p0 = (int)threadIdx.x * per;
+    const int p1 = p0 + per < nc ? p0 + per : nc;
+    int cg = 0, ce = 0;
+    for (int i = p0; i < p1; ++i) {
+      const uint32_t u = okey[i] - kmin;
+      cg += u > prefix;
+      ce += u == prefix;
     }
+    int total;
+    const int ex = block_excl_scan((cg << 16) | ce, scratch, &total);
+    int g = ex >> 16, e = ex & 0xffff;
+    for (int i = p0; i < p1; ++i) {
+      const uint32_t u = okey[i] - kmin;
+      if (u > prefix) {
+        const int o = g + (e < remaining ? e : remaining);
+        if (o < k) out[o] = oidx[i];                     // (bound holds unless the histogram is stale)
+        ++g;
+      } else if (u == prefix) {
+        if (e < remaining && g + e < k) out[g + e] = oidx[i];
+        ++e;
+      }
+    }
+    __syncthreads();
+  } else {
+    // more candidates than shared memory holds (rows dominated by ties): select on the
+    // candidate list in global memory
+    int32_t* sel = reinterpret_cast<int32_t*>(sel_smem);   // [k] selected indices, then bucketed
+    int32_t* bucket = sel + CSA_MAX_TOPK;                  // [k] indices grouped by chunk
+    int* ccount = bucket + CSA_MAX_TOPK;                   // [nchunks + 1] per-chunk counts -> offsets
+    for (int j = threadIdx.x; j <= nchunks; j += blockDim.x) ccount[j] = 0;
+    for (int j = threadIdx.x; j < k; j += blockDim.x) sel[j] = 0;   // in range even if a slot stays unset
+    __syncthreads();
+    auto cand_key = [&](int i) -> uint32_t { return __ldcg(ckey + i); };
+    auto cand_idx = [&](int i) -> int32_t { return __ldcg(cidx + i); };
+    // radix select on the 32-bit keys: digits of 11, 11 and 10 bits (skewed 2048-bin histogram)
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+      for (int j = threadIdx.x; j < 2048 + 64; j += blockDim.x) histk[j] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+        const uint32_t key = cand_key(i);
+        if ((key & pmask) == prefix) atomicAdd(&histk[skew((int)((key >> shift) & dmask))], 1);
+      }
+      __syncthreads();
+      find_digit_skewed<2048 / kSelThreads>(histk, 2048, remaining, res, scratch);
+      __syncthreads();
+      prefix |= (uint32_t)res[0] << shift;
+      pmask |= dmask << shift;
+      remaining -= res[1];
+      __syncthreads();
+    }
+    // selected = keys above K*, plus the `remaining` lowest indices among keys equal to K*.
+    // Slots come from warp-aggregated atomics (one per warp, or per distinct chunk within a
+    // warp) -- contended shared-memory atomics serialise lane by lane.
+    int32_t* eqlist = bucket;                              // keys equal to K* (scratch, before bucketing)
+    if (threadIdx.x == 0) {
+      lcount = 0;
+      gslot = 0;
+    }
+    __syncthreads();
+    for (int i0 = 0; i0 < nc; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      const uint32_t key = i < nc ? cand_key(i) : 0u;
+      const bool gt = i < nc && key > prefix;
+      const bool eq = i < nc && key == prefix;
+      const uint32_t mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
+      int bg = 0, be = 0;
+      if (lane_id() == 0) {
+        if (mg) bg = atomicAdd(&lcount, __popc(mg));
+        if (me) be = atomicAdd(&gslot, __popc(me));
+      }
+      bg = __shfl_sync(0xffffffffu, bg, 0);
+      be = __shfl_sync(0xffffffffu, be, 0);
+      const uint32_t below = (1u << lane_id()) - 1;
+      if (gt && bg + __popc(mg & below) < k) sel[bg + __popc(mg & below)] = cand_idx(i);
+      if (eq && be + __popc(me & below) < CSA_MAX_TOPK) eqlist[be + __popc(me & below)] = cand_idx(i);
+    }
+    __syncthreads();
+    const int ngt = lcount, neq = gslot;
+    // the `remaining` lowest indices among the equal keys (rank = equal keys with a lower index)
+    if (neq <= CSA_MAX_TOPK) {
+      for (int e = threadIdx.x; e < neq; e += blockDim.x) {
+        const int32_t j = eqlist[e];
+        int rank = 0;
+        for (int q = 0; q < neq; ++q) rank += eqlist[q] < j;
+        if (rank < remaining && ngt + rank < k) sel[ngt + rank] = j;
+      }
+    } else {
+      // more ties than the list holds (degenerate rows, e.g. constant scores): rank against
+      // the whole candidate list
+      for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+        if (cand_key(i) != prefix) continue;
+        const int32_t j = cand_idx(i);
+        int rank = 0;
+        for (int q = 0; q < nc && rank < remaining; ++q) rank += (cand_key(q) == prefix && cand_idx(q) < j);
+        if (rank < remaining && ngt + rank < k) sel[ngt + rank] = j;
+      }
+    }
+    __syncthreads();
+    int nsel = ngt + (remaining < neq ? remaining : neq);   // == k (nv > k)
+    nsel = nsel < k ? nsel : k;
+    // ascending order: chunks are contiguous index ranges, so order = (chunk, rank in chunk)
+    for (int i0 = 0; i0 < nsel; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      const bool act = i < nsel;
+      const int c = act ? sel[i] / chunk : -1;
+      const uint32_t m = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t peers = __match_any_sync(m, c);
+        if ((int)lane_id() == __ffs(peers) - 1) atomicAdd(&ccount[c], __popc(peers));
+      }
+    }
+    __syncthreads();
+    {
+      int total;
+      const int per = (nchunks + blockDim.x - 1) / blockDim.x;
+      int loc = 0;
+      for (int c = threadIdx.x * per; c < (int)(threadIdx.x + 1) * per && c < nchunks; ++c) loc += ccount[c];
+      int off = block_excl_scan(loc, scratch, &total);
+      __syncthreads();
+      for (int c = threadIdx.x * per; c < (int)(threadIdx.x + 1) * per && c < nchunks; ++c) {
+        const int n = ccount[c];
+        ccount[c] = off;                                   // start of chunk c's bucket
+        off += n;
+      }
+    }
+    __syncthreads();
+    for (int i0 = 0; i0 < nsel; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      const bool act = i < nsel;
+      const int32_t j = act ? sel[i] : 0;
+      const int c = act ? j / chunk : -1;
+      const uint32_t m = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t peers = __match_any_sync(m, c);
+        const int leader = __ffs(peers) - 1;
+        int base = 0;
+        if ((int)lane_id() == leader) base = atomicAdd(&ccount[c], __popc(peers));
+        base = __shfl_sync(peers, base, leader);
+        bucket[base + __popc(peers & ((1u << lane_id()) - 1))] = j;   // ccount ends at the bucket's end
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
+      const int32_t j = bucket[i];
+      const int c = j / chunk;
+      const int b_end = ccount[c];                         // end of this chunk's bucket
+      const int b_start = c > 0 ? ccount[c - 1] : 0;       // = end of the previous bucket
+      int rank = 0;
+      for (int q = b_start; q < b_end; ++q) rank += bucket[q] < j;
+      out[b_start + rank] = j;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
-    const int32_t j = bucket[i];
-    const int c = j / chunk;
-    const int b_end = ccount[c];                         // end of this chunk's bucket
-    const int b_start = c > 0 ? ccount[c - 1] : 0;       // = end of the previous bucket
-    int rank = 0;
-    for (int q = b_start; q < b_end; ++q) rank += bucket[q] < j;
-    out[b_start + rank] = j;
-  }
-  __syncthreads();
   // leave the row's header zeroed for the next call
   for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
   if (threadIdx.x == 0) {
-    *cand_count = 0;
-    *done = 0;
+    *fin = 0ull;
+    *slots = 0;
   }
 }
 

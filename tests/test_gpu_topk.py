@@ -117,7 +117,7 @@ def test_select_plain_matches_oracle(csa, B, N, k):
     hdr = ws.view(torch.int32)
     stride = csa.csa_select_workspace_size(1, N) // 4
     for b in range(B):
-        assert int(hdr[b * stride: b * stride + 4096 + 2].count_nonzero()) == 0
+        assert int(hdr[b * stride: b * stride + 4096 + 3].count_nonzero()) == 0
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
