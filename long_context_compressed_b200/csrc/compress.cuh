@@ -49,18 +49,48 @@ __device__ __forceinline__ void store8(float* p, const float* v) {
   reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-// CSA (ratio m = 4): one thread per (sequence, entry, group of 8 channels).
+__device__ __forceinline__ void load2(const __nv_bfloat16* p, float* v) {
+  const float2 f = __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162*>(p)));
+  v[0] = f.x;
+  v[1] = f.y;
+}
+__device__ __forceinline__ void load2(const float* p, float* v) {
+  const float2 f = __ldg(reinterpret_cast<const float2*>(p));
+  v[0] = f.x;
+  v[1] = f.y;
+}
+__device__ __forceinline__ void store2(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+}
+__device__ __forceinline__ void store2(float* p, const float* v) {
+  *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+}
+template <int CH, typename T>
+__device__ __forceinline__ void load_ch(const T* p, float* v) {
+  if constexpr (CH == 8) load8(p, v); else load2(p, v);
+}
+template <int CH, typename T>
+__device__ __forceinline__ void store_ch(T* p, const float* v) {
+  if constexpr (CH == 8) store8(p, v); else store2(p, v);
+}
+
+constexpr float kCompLog2e = 1.4426950408889634f;
+
+// CSA (ratio m = 4): one thread per (sequence, entry, group of CH channels):
+// CH = 8 (16-byte loads) when there are enough entries to fill the GPU, CH = 2
+// otherwise (a decode step compresses a single block per sequence).  All 2m
+// rows are loaded before use; the softmax runs in the base-2 domain.
 // Layouts: C_a, C_b, Z_a, Z_b [B, L, c]; prev_Cb, prev_Zb [B, m, c] or null;
 // out [B, L/m, c].
-template <typename Tin, typename Tout, int M>
+template <typename Tin, typename Tout, int M, int CH>
 __global__ void __launch_bounds__(256) compress_csa_kernel(const Tin* __restrict__ Ca, const Tin* __restrict__ Cb,
                                                            const Tin* __restrict__ Za, const Tin* __restrict__ Zb,
                                                            const Tin* __restrict__ pCb,
                                                            const Tin* __restrict__ pZb, int B, int64_t L, int c,
                                                            Tout* __restrict__ out) {
   griddep_sync();
-  // 32-bit index arithmetic (the host guarantees B * L/M * c/8 < 2^31)
-  const uint32_t groups = (uint32_t)c >> 3;
+  // 32-bit index arithmetic (the host guarantees B * L/M * c/CH < 2^31)
+  const uint32_t groups = (uint32_t)c / CH;
   const uint32_t n_entries = (uint32_t)(L / M);
   const uint32_t total = (uint32_t)B * n_entries * groups;
   for (uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x; gid < total; gid += gridDim.x * blockDim.x) {
@@ -68,125 +98,114 @@ __global__ void __launch_bounds__(256) compress_csa_kernel(const Tin* __restrict
     const uint32_t rest = gid / groups;
     const int64_t i = rest % n_entries;
     const int b = (int)(rest / n_entries);
-    const int ch = g * 8;
-    float z[2 * M][8], v[2 * M][8];
+    const int ch = g * CH;
+    float z[2 * M][CH], v[2 * M][CH];
     bool has_b = true;
 #pragma unroll
     for (int r = 0; r < M; ++r) {
       if (i > 0) {
         const int64_t off = ((int64_t)b * L + (i - 1) * M + r) * c + ch;
-        load8(Zb + off, z[r]);
-        load8(Cb + off, v[r]);
+        load_ch<CH>(Zb + off, z[r]);
+        load_ch<CH>(Cb + off, v[r]);
       } else if (pZb != nullptr) {
         const int64_t off = ((int64_t)b * M + r) * c + ch;
-        load8(pZb + off, z[r]);
-        load8(pCb + off, v[r]);
+        load_ch<CH>(pZb + off, z[r]);
+        load_ch<CH>(pCb + off, v[r]);
       } else {
         has_b = false;
       }
       const int64_t aoff = ((int64_t)b * L + i * M + r) * c + ch;
-      load8(Za + aoff, z[M + r]);
-      load8(Ca + aoff, v[M + r]);
+      load_ch<CH>(Za + aoff, z[M + r]);
+      load_ch<CH>(Ca + aoff, v[M + r]);
     }
     const int r0 = has_b ? 0 : M;
-    float res[8];
+    float res[CH];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < CH; ++j) {
       float mx = -INFINITY;
 #pragma unroll
       for (int r = 0; r < 2 * M; ++r)
-        if (r >= r0) mx = fmaxf(mx, z[r][j]);
+        if (r >= r0) {
+          z[r][j] *= kCompLog2e;
+          mx = fmaxf(mx, z[r][j]);
+        }
       float den = 0.f, acc = 0.f;
 #pragma unroll
       for (int r = 0; r < 2 * M; ++r) {
         if (r < r0) continue;
-        const float e = expf(z[r][j] - mx);
+        const float e = ex2_approx(z[r][j] - mx);
         den += e;
         acc = fmaf(e, v[r][j], acc);
       }
       res[j] = acc / den;
     }
-    store8(out + ((int64_t)b * n_entries + i) * c + ch, res);
+    store_ch<CH>(out + ((int64_t)b * n_entries + i) * c + ch, res);
   }
 }
 
-// HCA (ratio 128): one CTA per (sequence, entry, block of channels).  Inside
-// the CTA, 8-channel groups run along threadIdx.x (coalesced rows) and the 128
-// rows are split over row groups; each thread keeps an online softmax state
-// (running max, sum of exponentials, weighted sum) over chunks of 8 rows, and
-// the row groups merge through shared memory.
+// HCA (ratio 128): one CTA per (sequence, entry, block of 64 channels); 256
+// threads = 8 groups of 8 channels (16-byte loads, a warp covers 128-byte row
+// segments) x 32 row groups of 4 rows.  Every thread loads its 4 rows at once,
+// reduces them to a softmax state (max, sum of exponentials, weighted sum) per
+// channel, and 64 threads merge the 32 row-group states through shared memory.
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) compress_hca_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z,
                                                            int B, int64_t L, int c, Tout* __restrict__ out) {
   griddep_sync();
-  constexpr int M = 128;
-  constexpr int CH = 8;
-  const int groups = c >> 3;
-  const int G = groups < 64 ? groups : 64;       // channel groups per CTA
-  const int RG = 256 / G;                        // row groups
-  const int tg = threadIdx.x % G;
-  const int rg = threadIdx.x / G;
+  constexpr int M = 128, CH = 8, CG = 8, RG = 32, RPT = M / RG;
+  constexpr int PAD = CG * CH + 1;               // conflict-free partial stores and merge reads
+  __shared__ float pm[RG][PAD], ps[RG][PAD], pa[RG][PAD];
+  const int cg = threadIdx.x % CG, rg = threadIdx.x / CG;
   const int64_t n_entries = L / M;
   const int64_t i = blockIdx.y;
   const int b = blockIdx.z;
-  const int ch = (blockIdx.x * G + tg) * CH;
-  __shared__ float part[256][3 * CH];
-
-  float m[CH], s[CH], a[CH];
-#pragma unroll
-  for (int j = 0; j < CH; ++j) { m[j] = -INFINITY; s[j] = 0.f; a[j] = 0.f; }
-  const bool active = rg < RG && ch < c;
-  if (active) {
-    const int rows_per = M / RG;                 // RG divides 128
+  const int ch0 = blockIdx.x * CG * CH;
+  const int ch = ch0 + cg * CH;
+  if (ch < c) {
     const int64_t base = ((int64_t)b * L + i * M) * c + ch;
-    for (int r0 = 0; r0 < rows_per; r0 += 8) {
-      float z[8][CH], v[8][CH];
+    float z[RPT][CH], v[RPT][CH];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int row = rg + (r0 + u) * RG;
-        load8(Z + base + (int64_t)row * c, z[u]);
-        load8(C + base + (int64_t)row * c, v[u]);
-      }
-#pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        float cm = z[0][j];
-#pragma unroll
-        for (int u = 1; u < 8; ++u) cm = fmaxf(cm, z[u][j]);
-        const float nm = fmaxf(m[j], cm);
-        const float sc = expf(m[j] - nm);        // 0 on the first chunk (m = -inf)
-        float ss = s[j] * sc, aa = a[j] * sc;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float e = expf(z[u][j] - nm);
-          ss += e;
-          aa = fmaf(e, v[u][j], aa);
-        }
-        m[j] = nm; s[j] = ss; a[j] = aa;
-      }
+    for (int u = 0; u < RPT; ++u) {
+      const int64_t off = base + (int64_t)(rg + u * RG) * c;
+      load8(Z + off, z[u]);
+      load8(C + off, v[u]);
     }
-  }
-#pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    part[threadIdx.x][j] = m[j];
-    part[threadIdx.x][CH + j] = s[j];
-    part[threadIdx.x][2 * CH + j] = a[j];
-  }
-  __syncthreads();
-  if (rg == 0 && ch < c) {
-    float res[CH];
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-      float mx = -INFINITY;
-      for (int q = 0; q < RG; ++q) mx = fmaxf(mx, part[q * G + tg][j]);
-      float ss = 0.f, aa = 0.f;
-      for (int q = 0; q < RG; ++q) {
-        const float sc = expf(part[q * G + tg][j] - mx);
-        ss = fmaf(part[q * G + tg][CH + j], sc, ss);
-        aa = fmaf(part[q * G + tg][2 * CH + j], sc, aa);
+      float m = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < RPT; ++u) {
+        z[u][j] *= kCompLog2e;
+        m = fmaxf(m, z[u][j]);
       }
-      res[j] = aa / ss;
+      float sum = 0.f, acc = 0.f;
+#pragma unroll
+      for (int u = 0; u < RPT; ++u) {
+        const float e = ex2_approx(z[u][j] - m);
+        sum += e;
+        acc = fmaf(e, v[u][j], acc);
+      }
+      pm[rg][cg * CH + j] = m;
+      ps[rg][cg * CH + j] = sum;
+      pa[rg][cg * CH + j] = acc;
     }
-    store8(out + ((int64_t)b * n_entries + i) * c + ch, res);
+  }
+  __syncthreads();
+  const int t = threadIdx.x;
+  if (t < CG * CH && ch0 + t < c) {
+    float mx = -INFINITY;
+#pragma unroll 8
+    for (int q = 0; q < RG; ++q) mx = fmaxf(mx, pm[q][t]);
+    float sum = 0.f, acc = 0.f;
+#pragma unroll 8
+    for (int q = 0; q < RG; ++q) {
+      const float f = ex2_approx(pm[q][t] - mx);
+      sum = fmaf(ps[q][t], f, sum);
+      acc = fmaf(pa[q][t], f, acc);
+    }
+    const float r = acc / sum;
+    Tout* o = out + ((int64_t)b * n_entries + i) * c + ch0 + t;
+    if constexpr (sizeof(Tout) == 2) *o = __float2bfloat16_rn(r); else *o = r;
   }
 }
 

@@ -272,14 +272,22 @@ int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* 
   cudaStream_t st = as_stream(stream);
   const bool bf_in = in_dtype == CSA_BF16, bf_out = out_dtype == CSA_BF16;
   if (ratio == 4) {
-    const int64_t total = (int64_t)B * n_entries * (c / 8);
+    // 8 channels per thread once that still gives two waves of CTAs; 2 otherwise
+    const int64_t total8 = (int64_t)B * n_entries * (c / 8);
+    const bool wide = total8 >= (int64_t)sm_count() * 2 * 256;
+    const int64_t total = wide ? total8 : 4 * total8;
     if (total >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
     const int64_t blocks64 = (total + 255) / 256;
     const unsigned blocks = (unsigned)std::min<int64_t>(blocks64, (int64_t)sm_count() * 16);
-#define CSA_LAUNCH_CSA(TI, TO)                                                                              \
-  launch_k(csa::compress_csa_kernel<TI, TO, 4>, blocks, 256, 0, st,                                               \
-      (const TI*)C_a, (const TI*)C_b, (const TI*)Z_a, (const TI*)Z_b, (const TI*)prev_Cb, (const TI*)prev_Zb, \
-      B, L, c, (TO*)out)
+#define CSA_LAUNCH_CSA(TI, TO)                                                                                  \
+  do {                                                                                                          \
+    if (wide)                                                                                                   \
+      launch_k(csa::compress_csa_kernel<TI, TO, 4, 8>, blocks, 256, 0, st, (const TI*)C_a, (const TI*)C_b,      \
+               (const TI*)Z_a, (const TI*)Z_b, (const TI*)prev_Cb, (const TI*)prev_Zb, B, L, c, (TO*)out);      \
+    else                                                                                                        \
+      launch_k(csa::compress_csa_kernel<TI, TO, 4, 2>, blocks, 256, 0, st, (const TI*)C_a, (const TI*)C_b,      \
+               (const TI*)Z_a, (const TI*)Z_b, (const TI*)prev_Cb, (const TI*)prev_Zb, B, L, c, (TO*)out);      \
+  } while (0)
     if (bf_in && bf_out) CSA_LAUNCH_CSA(__nv_bfloat16, __nv_bfloat16);
     else if (bf_in) CSA_LAUNCH_CSA(__nv_bfloat16, float);
     else if (bf_out) CSA_LAUNCH_CSA(float, __nv_bfloat16);
@@ -287,8 +295,7 @@ int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* 
 #undef CSA_LAUNCH_CSA
   } else {
     if (n_entries > 65535 || B > 65535) return CSA_ERR_UNSUPPORTED;
-    const int G = std::min(c / 8, 64);
-    dim3 grid((unsigned)(c / 8 / G), (unsigned)n_entries, (unsigned)B);
+    dim3 grid((unsigned)((c + 63) / 64), (unsigned)n_entries, (unsigned)B);   // 64 channels per CTA
 #define CSA_LAUNCH_HCA(TI, TO) \
   launch_k(csa::compress_hca_kernel<TI, TO>, grid, 256, 0, st, (const TI*)C_a, (const TI*)Z_a, B, L, c, (TO*)out)
     if (bf_in && bf_out) CSA_LAUNCH_HCA(__nv_bfloat16, __nv_bfloat16);
@@ -357,7 +364,7 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
   const int key_bytes = fp8 ? csa::IndexCfg<true>::kKeyBytes : csa::IndexCfg<false>::kKeyBytes;
   const int qrow = fp8 ? 128 : 256;
   const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
-  const int fixed = 1024 + q_bytes + 2048 * p.TQ + 8 * (4 + 2 * csa::kMaxAcc) +
+  const int fixed = 1024 + q_bytes + 2048 * p.TQ + 8 * (4 + 2 * csa::kMaxAcc) + csa::kKsRing * 256 * 4 +
                     (select_ws ? 2 * csa::kHistBinsIdx * 4 : 0);
   p.stages = std::min(12, (kSmemLimit - fixed) / (key_bytes + 16));
   if (p.stages < 2) return CSA_ERR_UNSUPPORTED;

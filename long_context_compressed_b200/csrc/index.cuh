@@ -33,6 +33,8 @@ constexpr int kIdxDim = 128;
 constexpr int kIdxTileKeys = 128;
 constexpr int kMaxAcc = 4;
 constexpr int kIdxThreads = 320;                // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kKsAhead = 3;                     // key-scale prefetch distance (items of one epilogue set)
+constexpr int kKsRing = kKsAhead + 1;
 constexpr int kHistBinsIdx = 4096;              // 12-bit histogram of order-preserving score keys
 
 // Top 12 bits of the order-preserving uint32 key of a score (-0.0 folded to +0.0):
@@ -113,8 +115,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
   uint64_t* tempty = qfull + 2 + kMaxAcc;           // [kMaxAcc]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 2 + 2 * kMaxAcc);
   float* w_all = reinterpret_cast<float*>(qfull + 4 + 2 * kMaxAcc);  // [8 epilogue warps][TQ][64]
+  float* ks_all = w_all + 8 * TQ * kIdxHeads;                        // [kKsRing][256] key-scale ring
   // score histograms of the first two rows this CTA touches (when p.hist is set)
-  int* hist_s = reinterpret_cast<int*>(w_all + 8 * TQ * kIdxHeads);   // [2][kHistBinsIdx]
+  int* hist_s = reinterpret_cast<int*>(ks_all + kKsRing * 256);       // [2][kHistBinsIdx]
 
   const int QG = (p.T + TQ - 1) / TQ;
   const int64_t KT = (p.N + kIdxTileKeys - 1) / kIdxTileKeys;
@@ -242,22 +245,28 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
     const int acc_shift = NACC == 4 ? 2 : (NACC == 2 ? 1 : 0);
     float* w_s = w_all + (warp - 2) * TQ * kIdxHeads;
     int64_t nv_q[4] = {0, 0, 0, 0};
-    // key scales are fetched two of this set's items ahead along a second iterator
+    // key scales (e4m3) travel by cp.async into a per-thread ring in shared memory,
+    // kKsAhead of this set's items ahead along a second iterator: no register waits
+    // on a load in flight
+    float* ks_ring = ks_all + (threadIdx.x - 64);     // column of this epilogue thread
     IndexItem ahead = index_item(w0, QG, KT);
     int64_t w_ahead = w0;
     if (es) { index_next(ahead, QG, KT); ++w_ahead; }
-    auto ks_next = [&]() -> float {
-      float v = 1.f;
+    int ring_put = 0;
+    auto ks_fetch = [&]() {
       if (FP8 && w_ahead < w1) {
         const int64_t ii = ahead.kt * kIdxTileKeys + row;
-        if (ii < p.N) v = __ldg(p.k_scale + (int64_t)ahead.b * p.N + ii);
+        if (ii < p.N) cp_async_4(ks_ring + ring_put * 256, p.k_scale + (int64_t)ahead.b * p.N + ii);
       }
+      cp_async_commit();
+      ring_put = ring_put + 1 == kKsRing ? 0 : ring_put + 1;
       w_ahead += 2;
       index_next(ahead, QG, KT);
       index_next(ahead, QG, KT);
-      return v;
     };
-    float ks0 = ks_next(), ks1 = ks_next();
+    if (FP8)
+      for (int j = 0; j < kKsAhead; ++j) ks_fetch();
+    int ring_get = 0;
     int prev_b = -1, prev_qg = -1;
     IndexItem it = index_item(w0, QG, KT);
     int64_t w = w0;
@@ -265,32 +274,43 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
     if (es) { index_next(it, QG, KT); ++w; ++cnt; }
     for (; w < w1; w += 2, cnt += 2, index_next(it, QG, KT), index_next(it, QG, KT)) {
       if (it.b != prev_b || it.qg != prev_qg) {
-        // each epilogue warp keeps a private copy of the group's head weights
-        __syncwarp();
-        for (int j = (int)lane_id(); j < TQ * kIdxHeads; j += 32) {
+        // each epilogue warp keeps a private copy of the group's head weights; the
+        // weights, query scales and n_valid are all requested before any is used
+        // (one memory round trip, overlapping the wait for the first accumulator)
+        constexpr int PER = 4 * kIdxHeads / 32;
+        float wv[PER], sv[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+          const int j = (int)lane_id() + 32 * u;
           const int t = it.qg * TQ + j / kIdxHeads;
-          float v = 0.f;
-          if (t < p.T) {
-            const int64_t o = ((int64_t)it.b * p.T + t) * kIdxHeads + (j % kIdxHeads);
-            v = p.w[o];
-            if (FP8) v *= p.q_scale[o];
-          }
-          w_s[j] = v;
+          const bool in = j < TQ * kIdxHeads && t < p.T;
+          const int64_t o = ((int64_t)it.b * p.T + t) * kIdxHeads + (j % kIdxHeads);
+          wv[u] = in ? __ldg(p.w + o) : 0.f;
+          sv[u] = (FP8 && in) ? __ldg(p.q_scale + o) : 1.f;
         }
+        const int tq = it.qg * TQ + (int)lane_id();
+        const int nv_l = ((int)lane_id() < TQ && tq < p.T) ? __ldg(p.n_valid + (int64_t)it.b * p.T + tq) : 0;
         __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int t = it.qg * TQ + q;
-          nv_q[q] = (q < TQ && t < p.T) ? (int64_t)p.n_valid[(int64_t)it.b * p.T + t] : 0;
+        for (int u = 0; u < PER; ++u) {
+          const int j = (int)lane_id() + 32 * u;
+          if (j < TQ * kIdxHeads) w_s[j] = FP8 ? wv[u] * sv[u] : wv[u];
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) nv_q[q] = __shfl_sync(0xffffffffu, nv_l, q);
+        __syncwarp();
         prev_b = it.b;
         prev_qg = it.qg;
       }
       const int acc = cnt & (NACC - 1);
       const uint32_t aph = (uint32_t)(cnt >> acc_shift) & 1u;
-      const float ks = ks0;
-      ks0 = ks1;
-      ks1 = ks_next();
+      float ks = 1.f;
+      if (FP8) {
+        ks_fetch();                                 // item kKsAhead ahead
+        cp_async_wait_group<kKsAhead>();            // this item's copy has landed
+        ks = ks_ring[ring_get * 256];
+        ring_get = ring_get + 1 == kKsRing ? 0 : ring_get + 1;
+      }
       if (!mbar_wait(&tfull[acc], aph)) break;
       tc_fence_after();
       const int64_t i = it.kt * kIdxTileKeys + row;
@@ -337,6 +357,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&tempty[acc]);
     }
+    if (FP8) cp_async_wait_group<0>();              // no copy may land after the CTA has left
   }
 
   tc_fence_before();
