@@ -167,17 +167,15 @@ struct AttnCfg {
   static constexpr int kMaxStages = 4;
   static constexpr int kMaxCtaRows = 2048;                 // index values staged per CTA (larger lists stream)
   static constexpr int kBarBytes = 256 + 4 * kMaxCtaRows;
-  // Q rows held per 64-dim atom: 64 when H <= 64 (compact), else 128
-  static __host__ __device__ int q_rows(int H) { return H <= 64 ? 64 : 128; }
-  static __host__ __device__ int q_bytes(int H) { return q_rows(H) * D * 2; }
-  static __host__ __device__ int stages(int H) {
-    const int avail = 232448 - 1024 - kBarBytes - q_bytes(H) - 2 * kPBytes;
-    const int n = avail / kKVBytes;
-    return n >= kMaxStages ? kMaxStages : n;
-  }
-  static __host__ __device__ int smem(int H) {
-    return 1024 + q_bytes(H) + stages(H) * kKVBytes + 2 * kPBytes + kBarBytes;
-  }
+  // heads are taken in groups of kHeadGroup per CTA (more heads: more CTAs), so
+  // the Q tile is 64 rows per 64-dim atom and four KV stages always fit
+  static constexpr int kHeadGroup = 64;
+  static constexpr int kQBytes = kHeadGroup * D * 2;
+  static constexpr int kStages = ((232448 - 1024 - kBarBytes - kQBytes - 2 * kPBytes) / kKVBytes) >= kMaxStages
+                                     ? kMaxStages
+                                     : (232448 - 1024 - kBarBytes - kQBytes - 2 * kPBytes) / kKVBytes;
+  static constexpr int kSmem = 1024 + kQBytes + kStages * kKVBytes + 2 * kPBytes + kBarBytes;
+  static __host__ __device__ int head_groups(int H) { return (H + kHeadGroup - 1) / kHeadGroup; }
 };
 
 // Byte offset of 16-byte chunk c of row r in a K-major tile with 128-byte
@@ -186,8 +184,8 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
   return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-// Q [B*T, H, D] is loaded by TMA as D/64 boxes of {64 dims, QR rows}.  With
-// QR = 64 (H <= 64) the M = 128 MMA operand of atom a also spans the first 64
+// Q [B*T, H, D] is loaded by TMA as D/64 boxes of {64 dims, 64 head rows}
+// (head group blockIdx.y / NDH).  The M = 128 MMA operand of atom a also spans the first 64
 // rows of atom a+1 (or, for the last atom, the next 8 KB of shared memory):
 // finite values whose result rows (>= H) are never used.
 template <int D>
@@ -197,10 +195,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   constexpr int R = Cfg::R, DH = Cfg::DH;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int QR = Cfg::q_rows(p.H);
-  const int NS = Cfg::stages(p.H);
+  constexpr int QR = Cfg::kHeadGroup;
+  constexpr int NS = Cfg::kStages;
   uint8_t* q_s = smem;
-  uint8_t* kv_s = q_s + Cfg::q_bytes(p.H);                  // [NS][kKVBytes]
+  uint8_t* kv_s = q_s + Cfg::kQBytes;                       // [NS][kKVBytes]
   uint8_t* p_s = kv_s + NS * Cfg::kKVBytes;                 // [2][kPBytes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Cfg::kPBytes);
   uint64_t* full = bars;        // [4] KV stage loaded (128 cp.async arrivals)
@@ -215,9 +213,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 20);      // [4 stages][4 loader warps]
   int32_t* idx_s = reinterpret_cast<int32_t*>(bars + 32);         // [kMaxCtaRows] raw index values
 
+  __shared__ float epi_g[Cfg::kHeadGroup];   // per-head output scale (softmax -> epilogue warps)
+  __shared__ int epi_have_o;
   const int qi = blockIdx.z;                 // b * T + t
   const int b = qi / p.T, t = qi % p.T;
-  const int dh = blockIdx.y;
+  const int dh = blockIdx.y % Cfg::NDH;
+  const int h0 = (blockIdx.y / Cfg::NDH) * QR;  // first head of this CTA's group
   const int split = blockIdx.x;
   const int warp = warp_id();
   const int32_t* idx_row = p.sparse ? p.idx + ((int64_t)b * p.T + t) * p.k : nullptr;
@@ -320,13 +321,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
           mbar_arrive(&full[s]);
         }
       }
+      cp_async_wait_group<0>();                       // none may land after the CTA has left
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ Q by TMA, then the MMA issuer
     if (elect_one() && nt > 0) {
       prefetch_tmap(&qmap);
-      mbar_arrive_expect_tx(qfull, (uint32_t)Cfg::q_bytes(p.H));
-      for (int a = 0; a < Cfg::kAtoms; ++a) tma_load_3d(q_s + a * QR * 128, &qmap, qfull, a * 64, 0, qi);
+      mbar_arrive_expect_tx(qfull, (uint32_t)Cfg::kQBytes);
+      for (int a = 0; a < Cfg::kAtoms; ++a) tma_load_3d(q_s + a * QR * 128, &qmap, qfull, a * 64, h0, qi);
       const uint32_t idesc_s = make_idesc(128, R, 1, 0, 0);
       const uint32_t idesc_o = make_idesc(128, DH, 1, 0, 1);
       const uint32_t qb = smem_u32(q_s);
@@ -380,7 +382,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     // ------------------------------------------------------------ softmax / epilogue (warps 0..3)
     const int h = threadIdx.x;                 // TMEM lane = head row
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sinkL = (h < p.H) ? p.sink[h] * kLog2e : 0.f;
+    const bool head_ok = h < QR && h0 + h < p.H;    // rows >= QR are the operand's filler
+    const float sinkL = head_ok ? p.sink[h0 + h] * kLog2e : 0.f;
     const float zs = p.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -463,14 +466,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&pfull[sb]);
     }
-    // ---- epilogue
+    // ---- hand-over to the epilogue: per-head output scale and whether O is valid
     const bool have_o = ok && nt > 0 && mbar_wait(odone, 0);
-    tc_fence_after();
-    // O rows leave TMEM as 32-column chunks; each warp transposes its 32 x 32 chunk
-    // through shared memory (the KV stages are idle now) so that each store
-    // instruction writes four full 128-byte row segments.
-    float* stage = reinterpret_cast<float*>(kv_s) + warp * 32 * 36;
-    const int hw0 = warp * 32;                 // first head row of this warp
     float g = 1.f;
     if (p.nsplit == 1) {
       const float M = fmaxf(m_used, sinkL);
@@ -478,13 +475,38 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       const float den = l * fo + exp2f(sinkL - M);
       g = fo / den;
     }
+    if (h < QR) epi_g[h] = g;
+    if (h == 0) epi_have_o = have_o ? 1 : 0;
+    if (p.nsplit > 1 && head_ok && dh == 0) {
+      float* ml = p.ws_ml + (((int64_t)split * p.B * p.T + qi) * p.H + h0 + h) * 2;
+      ml[0] = have_o ? m_used : -INFINITY;
+      ml[1] = have_o ? l : 0.f;
+    }
+  }
+
+  // ------------------------------------------------------------ epilogue
+  // TMEM lanes 0..63 hold this CTA's heads; they are readable by warps 0, 1 and
+  // (same lane quarters) 4, 5, which split the O columns in two halves.  Each
+  // warp moves 32-column chunks out of TMEM and transposes them through shared
+  // memory (the KV stages are idle now) so that a store instruction writes four
+  // full 128-byte row segments.
+  if (warp == 0 || warp == 1 || warp == 4 || warp == 5) {
+    asm volatile("bar.sync 2, 128;" ::: "memory");   // epi_g / epi_have_o written by warps 0, 1
+    tc_fence_after();
+    const bool have_o = epi_have_o != 0;
+    const int rw = warp & 3;                           // lane quarter: head rows 32 * rw ..
+    const int hw0 = rw * 32;
+    const uint32_t lane_q = (uint32_t)(rw * 32) << 16;
+    const int c_begin = warp < 4 ? 0 : DH / 2, c_end = warp < 4 ? DH / 2 : DH;
+    float* stage = reinterpret_cast<float*>(kv_s) + warp * 32 * 36;
+    const float g = epi_g[hw0 + (int)lane_id()];
     const int sub = (int)lane_id() >> 3, q4 = ((int)lane_id() & 7) * 4;   // row within a group of 4, column
-    __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + hw0) * D + dh * DH;
-    float* wbase = p.ws_o + (((int64_t)split * p.B * p.T + qi) * p.H + hw0) * D + dh * DH;
-    for (int c0 = 0; c0 < DH; c0 += 32) {
+    __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hw0) * D + dh * DH;
+    float* wbase = p.ws_o + (((int64_t)split * p.B * p.T + qi) * p.H + h0 + hw0) * D + dh * DH;
+    for (int c0 = c_begin; c0 < c_end; c0 += 32) {
       float o[32];
       if (have_o) {
-        tmem_ld32(tmem + lane_base + c0, o);
+        tmem_ld32(tmem + lane_q + c0, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -499,7 +521,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
 #pragma unroll
       for (int r4 = 0; r4 < 32; r4 += 4) {
         const int r = r4 + sub;
-        if (hw0 + r < p.H) {
+        if (h0 + hw0 + r < p.H) {
           const float4 v = *reinterpret_cast<const float4*>(stage + r * 36 + q4);
           if (p.nsplit == 1) {
             __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), bb = __floats2bfloat162_rn(v.z, v.w);
@@ -512,11 +534,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
           }
         }
       }
-    }
-    if (p.nsplit > 1 && h < p.H && dh == 0) {
-      float* ml = p.ws_ml + (((int64_t)split * p.B * p.T + qi) * p.H + h) * 2;
-      ml[0] = have_o ? m_used : -INFINITY;
-      ml[1] = have_o ? l : 0.f;
+      __syncwarp();
     }
   }
 

@@ -144,20 +144,22 @@ int attn_rows_per_tile() { return AttnCfg<D>::R; }
 
 int attn_ndh(int D) { return D > 256 ? D / 256 : 1; }
 
-int attn_nsplit(int B, int T, int D, int64_t max_rows) {
-  const int64_t items = (int64_t)B * T * attn_ndh(D);
+// CTAs per (query, D-slice, head group) over the row list: one wave of CTAs, at
+// least four KV tiles each
+int attn_nsplit(int B, int T, int H, int D, int64_t max_rows) {
+  const int64_t items = (int64_t)B * T * attn_ndh(D) * ((H + 63) / 64);
   const int sms = sm_count();
   if (items <= 0 || items >= 2 * sms) return 1;
   const int R = D >= 512 ? 32 : 64;
   const int64_t tiles = (max_rows + R - 1) / R;
-  const int64_t want = (2 * sms + items - 1) / items;
+  const int64_t want = std::max<int64_t>(1, sms / items);
   const int64_t cap = std::max<int64_t>(1, tiles / 4);
   return (int)std::max<int64_t>(1, std::min(want, cap));
 }
 
 size_t attn_ws_bytes(int B, int T, int H, int D, int64_t max_rows, int dtype) {
   if (dtype != CSA_BF16) return 0;
-  const int ns = attn_nsplit(B, T, D, max_rows);
+  const int ns = attn_nsplit(B, T, H, D, max_rows);
   if (ns <= 1) return 0;
   const size_t per = (size_t)B * T * H;
   return (size_t)ns * per * ((size_t)D + 2) * sizeof(float) + 256;
@@ -177,26 +179,25 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     }
     return launch_status();
   }
-  p.nsplit = attn_nsplit(p.B, p.T, p.D, max_rows);
+  p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows);
   const size_t need = attn_ws_bytes(p.B, p.T, p.H, p.D, max_rows, dtype);
   if (need > 0) {
     if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return CSA_ERR_INVALID;
     p.ws_o = static_cast<float*>(ws);
     p.ws_ml = p.ws_o + (size_t)p.nsplit * p.B * p.T * p.H * p.D;
   }
-  dim3 grid(p.nsplit, attn_ndh(p.D), p.B * p.T);
-  // Q [B*T, H, D] by TMA: boxes of {64 dims, 64 or 128 rows}, rows past H zero-filled
+  // grid: (splits of the row list, D-slice x head group of 64, query)
+  dim3 grid(p.nsplit, attn_ndh(p.D) * ((p.H + 63) / 64), p.B * p.T);
+  // Q [B*T, H, D] by TMA: boxes of {64 dims, 64 head rows}, rows past H zero-filled
   CUtensorMap qmap;
-  const uint32_t qrows = p.H <= 64 ? 64 : 128;
   if (!make_map(&qmap, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D, (uint64_t)p.H,
-                (uint64_t)p.B * p.T, 64, qrows))
+                (uint64_t)p.B * p.T, 64, 64))
     return CSA_ERR_CUDA;
   switch (p.D) {
 #define CSA_LAUNCH_ATTN(DD)                                                                       \
   case DD: {                                                                                      \
-    const int sm = AttnCfg<DD>::smem(p.H);                                                        \
-    if (!set_smem(csa::attn_tc_kernel<DD>, std::max(AttnCfg<DD>::smem(1), AttnCfg<DD>::smem(128))))   \
-      return CSA_ERR_CUDA;                                                                        \
+    const int sm = AttnCfg<DD>::kSmem;                                                            \
+    if (!set_smem(csa::attn_tc_kernel<DD>, sm)) return CSA_ERR_CUDA;                              \
     launch_k(csa::attn_tc_kernel<DD>, grid, AttnCfg<DD>::kThreads, sm, st, qmap, p);                    \
     break;                                                                                        \
   }
