@@ -129,6 +129,26 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes (read + write) per indexer launch from the committed ncu summary, or None
+    when the indexer source has changed since that capture (the summary records a hash)."""
+    import hashlib
+    import re
+    try:
+        text = open(os.path.join(ROOT, "profiles", "index_tc_kernel_e4m3_decode.md")).read()
+        src = open(os.path.join(ROOT, "long_context_compressed_b200", "csrc", "index.cuh"), "rb").read()
+    except OSError:
+        return None
+    m = re.search(r"^traffic_bytes_per_launch: (.*)$", text, re.M)
+    if not m:
+        return None
+    fields = dict(kv.split("=", 1) for kv in m.group(1).split())
+    if hashlib.sha256(src).hexdigest()[:16] != fields.get("source_sha256_prefix"):
+        return None
+    v = fields.get(workload)
+    return int(v) if v is not None else None
+
+
 def measured_tflops():
     """Dense bf16 tensor peak (TFLOP/s): the burst figure, for kernels timed alone."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -778,7 +798,8 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if args.index == "e4m3"
                          else "index_tc_kernel (csa_index_scores, bf16)",
                          "achieved": idx_gbs, "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak,
-                         "peak_source": peak_kind + " (burst copy; the kernel is timed alone)", "traffic": None,
+                         "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
+                         "traffic": profiled_traffic(wl.name) if args.index == "e4m3" else None,
                          "bytes_per_launch": r["index_bytes"], "avg_launch_us": r["index_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays"},
