@@ -213,8 +213,10 @@ int csa_topk_select(const float *scores, const int32_t *n_valid, int B, int64_t 
  *   idx    : [B, T, k] int32;  out : [B, T, H, D] dtype
  *   dtype CSA_BF16 (tcgen05, fp32 softmax and accumulation; H <= 128,
  *   D in {128, 256, 512}) or CSA_F32 (fp32 FMA; D multiple of 32, <= 512).
- *   workspace : csa_attn_workspace_size(...) bytes (split-KV partials; may be
- *               0 bytes / NULL when that size is 0).
+ *   workspace : csa_attn_workspace_size(...) bytes; may be NULL when that size
+ *               is 0, which it is in this version: the row list of a query is
+ *               split over up to 8 CTAs that form one thread-block cluster and
+ *               merge their partial results in distributed shared memory.
  */
 size_t csa_attn_workspace_size(int B, int T, int H, int D, int64_t rows_per_query, int dtype);
 int sparse_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,

@@ -15,8 +15,9 @@
 //                [0, N) contributes nothing); hca_attn -> kv[e] for
 //                e < min(N, (pos+1)/ratio) (complete blocks only).
 //
-// attn_tc_kernel (bf16): one CTA per (split, D-slice, query).  The query block
-// (H heads padded to the M = 128 operand, all D dims) stays in shared memory;
+// attn_tc_kernel (bf16): one CTA per (split, D-slice x head group of 64, query).
+// The query block (64 heads, padded to the M = 128 operand, all D dims) stays in
+// shared memory;
 // KV rows are gathered with 16-byte cp.async into 128-byte-swizzled K-major
 // tiles of R rows; S = Q K^T (tcgen05, fp32 in TMEM, double buffered); four
 // softmax warps (one head per thread) run the online softmax in the log2
@@ -24,8 +25,11 @@
 // tile read as an MN-major operand, restricted to this CTA's D-slice of width
 // DH <= 256) accumulates in TMEM.  O is rescaled only when a tile's maximum
 // exceeds the running reference by more than 2^8, so exponentials stay <= 256.
-// With several splits the CTA writes (O, m, l) partials that attn_combine_kernel
-// merges together with the sink.
+// With several splits (<= 8) the split CTAs of one (query, D-slice, head group)
+// are one thread-block cluster: each parks its unnormalised O and (m, l) in its
+// own shared memory, and after a cluster barrier every CTA merges a slice of the
+// heads, sink included, reading the others' shared memory (no partials in HBM,
+// no second launch).
 //
 // attn_f32_kernel: fp32 SIMT (one warp per head), exact online softmax.
 #pragma once
@@ -46,10 +50,9 @@ struct AttnParams {
   const float* sink;      // [H]
   const int32_t* idx;     // [B, T, k] (sparse) or null (hca)
   void* out;              // [B, T, H, D]
-  float* ws_o;            // [nsplit, B*T, H, D] partial O (nsplit > 1)
-  float* ws_ml;           // [nsplit, B*T, H, 2] partial (m, l), log2 domain
   float scale;
   int B, T, H, D, W, k, ratio, nsplit;
+  int has_kvmap, has_swamap;   // tensor maps of kv [B, N, D] and swa_kv [B, W, D] were built
   int sparse;             // 1: memory rows from idx (sparse_attn); 0: dense prefix (hca_attn)
   int64_t N;
 };
@@ -190,6 +193,8 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
 // finite values whose result rows (>= H) are never used.
 template <int D>
 __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                           const __grid_constant__ CUtensorMap kvmap,
+                                                                           const __grid_constant__ CUtensorMap swamap,
                                                                            const AttnParams p) {
   using Cfg = AttnCfg<D>;
   constexpr int R = Cfg::R, DH = Cfg::DH;
@@ -215,6 +220,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
 
   __shared__ float epi_g[Cfg::kHeadGroup];   // per-head output scale (softmax -> epilogue warps)
   __shared__ int epi_have_o;
+  // split partials (nsplit > 1: the CTAs of one query / D-slice / head group form a
+  // cluster and merge through distributed shared memory)
+  __shared__ float cl_m[Cfg::kHeadGroup], cl_l[Cfg::kHeadGroup];   // running max (log2) and sum
+  __shared__ float cl_w[Cfg::kHeadGroup][8];                       // merge weights of the <= 8 splits
   const int qi = blockIdx.z;                 // b * T + t
   const int b = qi / p.T, t = qi % p.T;
   const int dh = blockIdx.y % Cfg::NDH;
@@ -294,24 +303,42 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       int ks = 0;
       uint32_t kph = 0;
       for (int jj = 0; jj < nt; ++jj) {
-        const int rg = (j0 + jj) * R + my_r;
+        const int rg0 = (j0 + jj) * R;
+        const int rg = rg0 + my_r;
         const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
         const int s = ks;
         const uint32_t ph = kph;
         if (++ks == NS) { ks = 0; kph ^= 1; }
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        const int64_t src_off = row_src(rg, raw);
-        const __nv_bfloat16* src = src_off >= 0 ? kv + src_off : (src_off <= -2 ? swa + (-2 - src_off) : nullptr);
         uint8_t* tile = kv_s + s * Cfg::kKVBytes;
+        // R consecutive rows of one buffer (SWA rows, or hca_attn's dense memory rows):
+        // one TMA box per 64-dim atom, same 128-byte-swizzled layout as the gather
+        const bool swa_tile = p.has_swamap && rg0 + R <= rl.n_swa;
+        const bool mem_tile = p.has_kvmap && !p.sparse && rg0 >= rl.n_swa && rg0 + R <= n_rows;
+        const __nv_bfloat16* src = nullptr;
+        if (swa_tile || mem_tile) {
+          src = kv;                                   // every row valid
+          if (lt == 0) {
+            mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKVBytes);
+            const int y = swa_tile ? (int)rl.swa_row0 + rg0 : rg0 - rl.n_swa;
+            for (int a = 0; a < Cfg::kAtoms; ++a)
+              tma_load_3d(tile + a * R * 128, swa_tile ? &swamap : &kvmap, &full[s], a * 64, y, b);
+          } else {
+            mbar_arrive(&full[s]);
+          }
+        } else {
+          const int64_t src_off = row_src(rg, raw);
+          src = src_off >= 0 ? kv + src_off : (src_off <= -2 ? swa + (-2 - src_off) : nullptr);
 #pragma unroll 4
-        for (int i = 0; i < CPT; ++i) {
-          const int ch = my_c + TPR * i;
-          uint8_t* dst = tile + sw128_off(my_r, ch, R);
-          if (src) cp_async_16(dst, src + ch * 8);
-          else st_shared_zero16(dst);                 // finite filler for rows that do not contribute
+          for (int i = 0; i < CPT; ++i) {
+            const int ch = my_c + TPR * i;
+            uint8_t* dst = tile + sw128_off(my_r, ch, R);
+            if (src) cp_async_16(dst, src + ch * 8);
+            else st_shared_zero16(dst);               // finite filler for rows that do not contribute
+          }
+          fence_proxy_async_smem();
+          cp_async_arrive_noinc(&full[s]);
         }
-        fence_proxy_async_smem();
-        cp_async_arrive_noinc(&full[s]);
         // validity of this warp's rows (TPR threads per row): one word per loader warp
         const uint32_t bal = __ballot_sync(0xffffffffu, src != nullptr);
         if (lane_id() == 0) {
@@ -477,10 +504,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     }
     if (h < QR) epi_g[h] = g;
     if (h == 0) epi_have_o = have_o ? 1 : 0;
-    if (p.nsplit > 1 && head_ok && dh == 0) {
-      float* ml = p.ws_ml + (((int64_t)split * p.B * p.T + qi) * p.H + h0 + h) * 2;
-      ml[0] = have_o ? m_used : -INFINITY;
-      ml[1] = have_o ? l : 0.f;
+    if (h < QR) {
+      cl_m[h] = have_o ? m_used : -INFINITY;
+      cl_l[h] = have_o ? l : 0.f;
     }
   }
 
@@ -502,7 +528,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     const float g = epi_g[hw0 + (int)lane_id()];
     const int sub = (int)lane_id() >> 3, q4 = ((int)lane_id() & 7) * 4;   // row within a group of 4, column
     __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hw0) * D + dh * DH;
-    float* wbase = p.ws_o + (((int64_t)split * p.B * p.T + qi) * p.H + h0 + hw0) * D + dh * DH;
+    float* obuf = reinterpret_cast<float*>(kv_s);   // clustered: raw O [64 heads][DH], float4 slots ^ (row & 7)
     for (int c0 = c_begin; c0 < c_end; c0 += 32) {
       float o[32];
       if (have_o) {
@@ -511,6 +537,17 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0.f;
+      }
+      if (p.nsplit > 1) {
+        const int row = hw0 + (int)lane_id();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int f = (c0 >> 2) + c;
+          const int phys = (f & ~7) | ((f ^ row) & 7);
+          *reinterpret_cast<float4*>(obuf + row * DH + phys * 4) =
+              make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        }
+        continue;
       }
       __syncwarp();
 #pragma unroll
@@ -523,66 +560,83 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         const int r = r4 + sub;
         if (h0 + hw0 + r < p.H) {
           const float4 v = *reinterpret_cast<const float4*>(stage + r * 36 + q4);
-          if (p.nsplit == 1) {
-            __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), bb = __floats2bfloat162_rn(v.z, v.w);
-            uint2 u;
-            u.x = *reinterpret_cast<uint32_t*>(&a);
-            u.y = *reinterpret_cast<uint32_t*>(&bb);
-            *reinterpret_cast<uint2*>(obase + (int64_t)r * D + c0 + q4) = u;
-          } else {
-            *reinterpret_cast<float4*>(wbase + (int64_t)r * D + c0 + q4) = v;
-          }
+          __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), bb = __floats2bfloat162_rn(v.z, v.w);
+          uint2 u;
+          u.x = *reinterpret_cast<uint32_t*>(&a);
+          u.y = *reinterpret_cast<uint32_t*>(&bb);
+          *reinterpret_cast<uint2*>(obase + (int64_t)r * D + c0 + q4) = u;
         }
       }
       __syncwarp();
     }
   }
 
+  if (p.nsplit > 1) {
+    // ------------------------------------------------------------ merge of the splits
+    // CTA `rank` of the cluster finishes heads [rank*64/ns, (rank+1)*64/ns): with
+    // M = max(sink, m_j), den = 2^(sink - M) + sum_j l_j 2^(m_j - M), the output is
+    // sum_j 2^(m_j - M) O_j / den, O_j read from CTA j's shared memory.
+    const int ns = p.nsplit;
+    const uint32_t rank = cluster_ctarank();
+    const int hb = (int)rank * QR / ns, he = ((int)rank + 1) * QR / ns;
+    cluster_sync();                                   // every split's O and (m, l) are in place
+    for (int hl = threadIdx.x; hl < he - hb; hl += blockDim.x) {
+      const int hh = hb + hl;
+      float mj[8], lj[8];
+      const float sinkL = (h0 + hh < p.H) ? p.sink[h0 + hh] * kLog2e : 0.f;
+      float M = sinkL;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        mj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_m[hh]), (uint32_t)j)) : -INFINITY;
+        lj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_l[hh]), (uint32_t)j)) : 0.f;
+        M = fmaxf(M, mj[j]);
+      }
+      float den = ex2_approx(sinkL - M);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        mj[j] = ex2_approx(mj[j] - M);                // m = -inf (no rows) -> weight 0
+        den = fmaf(lj[j], mj[j], den);
+      }
+      const float inv = 1.f / den;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cl_w[hh][j] = mj[j] * inv;
+    }
+    __syncthreads();
+    constexpr int F = DH / 4;                         // float4 slots per head row
+    const uint32_t ob = smem_u32(kv_s);
+    uint32_t peer[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) peer[j] = cluster_map(ob, (uint32_t)(j < ns ? j : 0));
+    for (int it = threadIdx.x; it < (he - hb) * F; it += blockDim.x) {
+      const int hh = hb + it / F, f = it % F;
+      if (h0 + hh >= p.H) continue;
+      const uint32_t off = (uint32_t)(hh * DH + (((f & ~7) | ((f ^ hh) & 7)) * 4)) * 4u;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < ns) {
+          const float4 v = ld_cluster_f4(peer[j] + off);
+          const float wj = cl_w[hh][j];
+          acc.x = fmaf(wj, v.x, acc.x);
+          acc.y = fmaf(wj, v.y, acc.y);
+          acc.z = fmaf(wj, v.z, acc.z);
+          acc.w = fmaf(wj, v.w, acc.w);
+        }
+      }
+      __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y), bb = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&a);
+      u.y = *reinterpret_cast<uint32_t*>(&bb);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hh) * D + dh * DH +
+                                f * 4) = u;
+    }
+    cluster_sync();                                   // no CTA leaves while its shared memory is read
+  }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 8) tmem_dealloc(tmem, Cfg::kTmemCols);
-}
-
-// Merge split partials with the sink: M = max(sink, m_s); den = e^(sink-M) +
-// sum_s l_s e^(m_s-M); o = sum_s O_s e^(m_s-M) / den  (log2 domain).  One
-// thread per (query, head, 8 dims).
-__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
-  griddep_sync();
-  const uint32_t gpr = (uint32_t)(p.D / 8);  // 32-bit index math: B*T*H*D/8 < 2^31 (host-checked)
-  const uint32_t groups = (uint32_t)(p.B * p.T * p.H) * gpr;
-  const uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= groups) return;
-  const int d0 = (int)(g % gpr) * 8;
-  const uint32_t qh = g / gpr;               // (b*T + t) * H + h
-  const int h = (int)(qh % (uint32_t)p.H);
-  const float sinkL = p.sink[h] * kLog2e;
-  const int64_t stride_ml = (int64_t)p.B * p.T * p.H * 2;
-  const int64_t stride_o = (int64_t)p.B * p.T * p.H * p.D;
-  float M = sinkL;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.ws_ml[s * stride_ml + qh * 2]);
-  float den = exp2f(sinkL - M);
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float ms = p.ws_ml[s * stride_ml + qh * 2];
-    if (ms == -INFINITY) continue;
-    const float f = exp2f(ms - M);
-    den = fmaf(p.ws_ml[s * stride_ml + qh * 2 + 1], f, den);
-    const float4* src = reinterpret_cast<const float4*>(p.ws_o + s * stride_o + qh * p.D + d0);
-    const float4 a = src[0], c = src[1];
-    acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
-    acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
-    acc[4] = fmaf(c.x, f, acc[4]); acc[5] = fmaf(c.y, f, acc[5]);
-    acc[6] = fmaf(c.z, f, acc[6]); acc[7] = fmaf(c.w, f, acc[7]);
-  }
-  const float inv = 1.f / den;
-  uint4 u;
-  __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) hv[e] = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + qh * p.D + d0) = u;
 }
 
 }  // namespace csa

@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <map>
+#include <tuple>
 #include <utility>
 #include <mutex>
 #include <vector>
@@ -123,19 +125,74 @@ bool use_pdl() {
   return on;
 }
 
+// Launch with programmatic dependent launch (unless disabled) and, for cluster_x > 1,
+// thread-block clusters of cluster_x CTAs along x.
 template <typename... KArgs, typename... Args>
-void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+void launch_kc(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+               Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (use_pdl()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = use_pdl() ? 1 : 0;
+  cfg.numAttrs = n;
   cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  launch_kc(kernel, grid, block, smem, st, 1, std::forward<Args>(args)...);
+}
+
+// Clusters of cluster_x CTAs of `kernel` that fit on the device at once (cached);
+// 0 if the occupancy query fails.
+template <typename... KArgs>
+int max_active_clusters(void (*kernel)(KArgs...), int threads, int smem, int cluster_x) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_tuple(reinterpret_cast<const void*>(kernel), dev, cluster_x);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  if (!set_smem(kernel, smem)) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cluster_x, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = n;
+  return n;
 }
 
 // ------------------------------------------------------------------ attention split policy
@@ -154,16 +211,11 @@ int attn_nsplit(int B, int T, int H, int D, int64_t max_rows) {
   const int64_t tiles = (max_rows + R - 1) / R;
   const int64_t want = std::max<int64_t>(1, sms / items);
   const int64_t cap = std::max<int64_t>(1, tiles / 4);
-  return (int)std::max<int64_t>(1, std::min(want, cap));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), 8));   // <= 8: one portable cluster
 }
 
-size_t attn_ws_bytes(int B, int T, int H, int D, int64_t max_rows, int dtype) {
-  if (dtype != CSA_BF16) return 0;
-  const int ns = attn_nsplit(B, T, H, D, max_rows);
-  if (ns <= 1) return 0;
-  const size_t per = (size_t)B * T * H;
-  return (size_t)ns * per * ((size_t)D + 2) * sizeof(float) + 256;
-}
+// The split partials merge inside the kernel (cluster shared memory): no workspace.
+size_t attn_ws_bytes(int, int, int, int, int64_t, int) { return 0; }
 
 int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_rows, cudaStream_t st) {
   if (p.B == 0 || p.T == 0) return CSA_OK;
@@ -180,25 +232,44 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     return launch_status();
   }
   p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows);
-  const size_t need = attn_ws_bytes(p.B, p.T, p.H, p.D, max_rows, dtype);
-  if (need > 0) {
-    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return CSA_ERR_INVALID;
-    p.ws_o = static_cast<float*>(ws);
-    p.ws_ml = p.ws_o + (size_t)p.nsplit * p.B * p.T * p.H * p.D;
-  }
+  (void)ws;
+  (void)ws_bytes;
   // grid: (splits of the row list, D-slice x head group of 64, query)
   dim3 grid(p.nsplit, attn_ndh(p.D) * ((p.H + 63) / 64), p.B * p.T);
+  // fewer splits while the clusters would not all be resident at once (one CTA per
+  // SM, a cluster's CTAs in one GPC)
+  const int64_t items = (int64_t)grid.y * grid.z;
+  while (p.nsplit > 1) {
+    int fit = 0;
+    switch (p.D) {
+      case 128: fit = max_active_clusters(csa::attn_tc_kernel<128>, AttnCfg<128>::kThreads, AttnCfg<128>::kSmem, p.nsplit); break;
+      case 256: fit = max_active_clusters(csa::attn_tc_kernel<256>, AttnCfg<256>::kThreads, AttnCfg<256>::kSmem, p.nsplit); break;
+      case 512: fit = max_active_clusters(csa::attn_tc_kernel<512>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit); break;
+      default: break;
+    }
+    if (fit >= items || fit == 0) break;   // 0: the query failed; keep the policy's choice
+    --p.nsplit;
+  }
+  grid.x = p.nsplit;
   // Q [B*T, H, D] by TMA: boxes of {64 dims, 64 head rows}, rows past H zero-filled
-  CUtensorMap qmap;
+  CUtensorMap qmap, kvmap, swamap;
   if (!make_map(&qmap, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D, (uint64_t)p.H,
                 (uint64_t)p.B * p.T, 64, 64))
     return CSA_ERR_CUDA;
+  // kv and swa_kv as boxes of {64 dims, R rows}: contiguous row tiles load by TMA
+  const uint32_t rows_per_tile = p.D >= 512 ? 32u : 64u;
+  std::memset(&kvmap, 0, sizeof(kvmap));
+  std::memset(&swamap, 0, sizeof(swamap));
+  p.has_kvmap = p.N > 0 && make_map(&kvmap, p.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D,
+                                    (uint64_t)p.N, (uint64_t)p.B, 64, rows_per_tile) ? 1 : 0;
+  p.has_swamap = p.W > 0 && make_map(&swamap, p.swa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D,
+                                     (uint64_t)p.W, (uint64_t)p.B, 64, rows_per_tile) ? 1 : 0;
   switch (p.D) {
 #define CSA_LAUNCH_ATTN(DD)                                                                       \
   case DD: {                                                                                      \
     const int sm = AttnCfg<DD>::kSmem;                                                            \
     if (!set_smem(csa::attn_tc_kernel<DD>, sm)) return CSA_ERR_CUDA;                              \
-    launch_k(csa::attn_tc_kernel<DD>, grid, AttnCfg<DD>::kThreads, sm, st, qmap, p);                    \
+    launch_kc(csa::attn_tc_kernel<DD>, grid, AttnCfg<DD>::kThreads, sm, st, p.nsplit, qmap, kvmap, swamap, p); \
     break;                                                                                        \
   }
     CSA_LAUNCH_ATTN(128)
@@ -207,10 +278,6 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
 #undef CSA_LAUNCH_ATTN
     default: return CSA_ERR_UNSUPPORTED;
   }
-  int rc = launch_status();
-  if (rc != CSA_OK || p.nsplit == 1) return rc;
-  const int64_t groups = (int64_t)p.B * p.T * p.H * (p.D / 8);
-  launch_k(csa::attn_combine_kernel, (unsigned)((groups + 255) / 256), 256, 0, st, p);
   return launch_status();
 }
 
