@@ -232,6 +232,13 @@ class DecodeSet:
             q = B * T * 64 * (256 + 4)
         return keys + q + B * T * N * 4
 
+    def attn_bytes(self):
+        """One sparse_attn launch: q, the gathered top-k and SWA rows, idx, sink, out."""
+        wl = self.wl
+        B, T, H, D, k = wl.B, wl.T, wl.H, wl.D, wl.topk
+        rows = B * T * (k + min(wl.W, 128)) * D * 2
+        return B * T * H * D * 2 * 2 + rows + B * T * k * 4 + H * 4
+
     def step_bytes(self):
         wl = self.wl
         B, T, N, H, D, k = wl.B, wl.T, wl.N, wl.H, wl.D, wl.topk
@@ -403,6 +410,41 @@ def index_alone_ms(sets, index, device, reps_per_set=8, replays=20):
     return ms
 
 
+def attn_alone_ms(sets, device, reps_per_set=8, replays=20):
+    """Average duration (ms) of one sparse_attn launch (attn_tc_kernel) timed alone:
+    back-to-back launches in one CUDA graph cycling over the input sets (cold in L2),
+    CUDA events around the graph replays."""
+    import torch
+
+    from long_context_compressed_b200 import csa
+    n = reps_per_set * len(sets)
+
+    def launch(i):
+        s = sets[i % len(sets)]
+        x = s.inputs
+        csa.sparse_attn(x["q"], s.kv, s.swa, s.swa_pos0, s.q_pos, s.sink, s.idx, 1.0 / math.sqrt(s.wl.D),
+                        out=s.out, workspace=s.attn_ws)
+    for i in range(len(sets)):
+        launch(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            launch(i)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (replays * n)
+    del g
+    return ms
+
+
 def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=None):
     import torch
 
@@ -416,7 +458,8 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     graphs, launches = capture(sets, side)
     t = timed_replays(graphs, steps, warmup, world)
     t = max_over_ranks(t, world, device)
-    idx_ms = index_alone_ms(sets, index, device)
+    idx_ms = index_alone_ms(sets, index, device, replays=max(3, min(20, steps // 100)))
+    attn_ms = attn_alone_ms(sets, device, replays=max(3, min(20, steps // 100)))
     # per-stage breakdown from a separate diagnostic graph with events between all stages
     diag, _ = capture(sets, side, timing_events="all")
     timed_replays(diag, min(steps, 200), 5, world)
@@ -437,6 +480,7 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     h2d, d2h = probe.per_step_io()
     res = {"wl": wl, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
            "index_ms": idx_ms, "index_bytes": probe.index_bytes(), "step_bytes": touched,
+           "attn_ms": attn_ms, "attn_bytes": probe.attn_bytes(),
            "e2e_seconds": t_e2e, "h2d": h2d, "d2h": d2h, "tokens_per_step": wl.B * wl.T,
            "breakdown": breakdown}
     del graphs, e2e_graphs, sets
@@ -598,6 +642,76 @@ def bench_hca(steps, warmup, device, hbm_peak):
 
 
 STAGES = ("compress", "quantize", "index", "select", "attn", "hcompress", "hca")
+BIG_STAGES = ("prefill_compress", "prefill_index", "prefill_index8", "prefill_topk", "prefill_attn",
+              "hca_compress", "hca_attn")
+
+
+def run_big_stage(stage, steps, warmup, device):
+    """One call of the chunked-prefill (flash_prefill) or HCA-decode (pro_hca) shapes,
+    eagerly, for profiling a single kernel on its measured workload.  Prints the mean
+    device time per call (CUDA events)."""
+    import torch
+
+    from long_context_compressed_b200 import csa, synth
+    dev = device
+    if stage.startswith("prefill"):
+        wl = synth.WORKLOADS["flash_prefill"]
+    else:
+        wl = synth.WORKLOADS["pro_hca"]
+    B, T, N, H, D, k = wl.B, wl.T, wl.N, wl.H, wl.D, wl.topk
+    g = lambda nm, shape: synth.store(synth.normal(0, f"bench/{wl.name}/{nm}", shape, device=dev), "bf16")
+    q_pos = (torch.arange(T, device=dev, dtype=torch.int64) + wl.q_pos0).view(1, T).repeat(B, 1)
+    swa_pos0 = torch.full((B,), wl.swa_pos0, dtype=torch.int64, device=dev)
+    sink = synth.normal(0, f"bench/{wl.name}/sink", (H,), device=dev)
+    if stage == "prefill_compress":
+        x = {nm: g(nm, (B, wl.comp_L, wl.comp_c)) for nm in ("C_a", "C_b", "Z_a", "Z_b")}
+        pr = {nm: g(nm, (B, 4, wl.comp_c)) for nm in ("prev_Cb", "prev_Zb")}
+        out = torch.empty((B, wl.comp_L // 4, wl.comp_c), dtype=torch.bfloat16, device=dev)
+        fn = lambda: csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], pr["prev_Cb"], pr["prev_Zb"], ratio=4,
+                                      out=out)
+    elif stage in ("prefill_index", "prefill_index8", "prefill_topk"):
+        qI, kI = g("qI", (B, T, 64, 128)), g("kI", (B, N, 128))
+        w = synth.normal(0, f"bench/{wl.name}/w", (B, T, 64), device=dev)
+        n_valid = csa.n_valid_for(q_pos, 4, N)
+        scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
+        if stage == "prefill_index8":
+            q8, qs = csa.csa_quantize_e4m3(qI)
+            k8, ks = csa.csa_quantize_e4m3(kI)
+            fn = lambda: csa.csa_index_scores(q8, w, k8, n_valid, q_scale=qs, k_scale=ks, scores=scores)
+        else:
+            csa.csa_index_scores(qI, w, kI, n_valid, scores=scores)
+            fn = lambda: csa.csa_index_scores(qI, w, kI, n_valid, scores=scores)
+        if stage == "prefill_topk":
+            idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
+            ws = csa.topk_workspace(B, T, N, k, dev)
+            fn = lambda: csa.csa_topk(scores, n_valid, k, idx=idx, workspace=ws)
+    elif stage == "prefill_attn":
+        q, kv, swa = g("q", (B, T, H, D)), g("kv", (B, N, D)), g("swa", (B, wl.W, D))
+        idx = synth.random_subset(0, f"bench/{wl.name}/idx", csa.n_valid_for(q_pos, 4, N).cpu(), k, device=dev)
+        out = torch.empty_like(q)
+        fn = lambda: csa.sparse_attn(q, kv, swa, swa_pos0, q_pos, sink, idx, 1.0 / math.sqrt(D), out=out)
+    elif stage == "hca_compress":
+        C, Z = g("C", (B, wl.comp_L, wl.comp_c)), g("Z", (B, wl.comp_L, wl.comp_c))
+        out = torch.empty((B, wl.comp_L // 128, wl.comp_c), dtype=torch.bfloat16, device=dev)
+        fn = lambda: csa.csa_compress(C, None, Z, None, ratio=128, out=out)
+    elif stage == "hca_attn":
+        q, kv, swa = g("q", (B, T, H, D)), g("kv", (B, N, D)), g("swa", (B, wl.W, D))
+        out = torch.empty_like(q)
+        fn = lambda: csa.hca_attn(q, kv, swa, swa_pos0, q_pos, sink, 1.0 / math.sqrt(D), out=out)
+    else:
+        raise SystemExit(f"unknown stage {stage}")
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    assert csa.csa_poll_status() == csa.CSA_OK
+    print(json.dumps({"stage": stage, "workload": wl.name, "steps": steps,
+                      "us_per_call": 1e3 * a.elapsed_time(b) / steps}), flush=True)
 
 
 def run_stage(name, stage, index, steps, warmup, device):
@@ -722,7 +836,7 @@ def main():
     ap.add_argument("--index", default="e4m3", choices=["e4m3", "bf16"])
     ap.add_argument("--no-extra", action="store_true", help="skip the pro1m measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=STAGES, help="time one stage alone (eager calls), e.g. under ncu")
+    ap.add_argument("--stage", choices=STAGES + BIG_STAGES, help="time one stage alone (eager calls), e.g. under ncu")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_env()
@@ -765,6 +879,9 @@ def main():
     __graft_entry__.build()
     from long_context_compressed_b200 import csa  # noqa: F401  (fails loudly if libcsa.so is missing)
 
+    if args.stage in BIG_STAGES:
+        run_big_stage(args.stage, args.steps, args.warmup, device)
+        return
     if args.stage:
         run_stage(args.workload, args.stage, args.index, args.steps, args.warmup, device)
         return
@@ -790,12 +907,21 @@ def main():
         tok = r["tokens_per_step"] * world
         steps = args.steps
         idx_gbs = r["index_bytes"] / (r["index_ms"] * 1e-3) / 1e9
+        attn_gbs = r["attn_bytes"] / (r["attn_ms"] * 1e-3) / 1e9
         step_gbs = r["step_bytes"] / (r["step_ms"] * 1e-3) / 1e9
         return {
             "value": tok * steps / r["seconds"], "ms_per_step": r["step_ms"],
             "e2e": {"value": tok * steps / r["e2e_seconds"], "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-            "roofline": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if args.index == "e4m3"
+            "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (sparse_attn: top-k + SWA rows, cluster merge)",
+                         "achieved": attn_gbs, "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak,
+                         "peak_source": peak_kind + " (burst copy; the kernel is timed alone)", "traffic": None,
+                         "bytes_per_launch": r["attn_bytes"], "avg_launch_us": r["attn_ms"] * 1e3,
+                         "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
+                                   "CUDA events around the graph replays",
+                         "why_this_kernel": "largest share of the step in the ncu launch list (two launches per "
+                                            "step: CSA sparse_attn and HCA hca_attn)"},
+            "roofline_indexer": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if args.index == "e4m3"
                          else "index_tc_kernel (csa_index_scores, bf16)",
                          "achieved": idx_gbs, "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak,
                          "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
@@ -825,7 +951,8 @@ def main():
                                f"{wl.ctx // 128}+128 rows)" if with_hca else ""),
                    "l2": f"{m['input_sets']} rotating input sets, > 2x L2 touched between reuses",
                    "parallelism": f"replicas x{world}"},
-        "e2e": m["e2e"], "roofline": m["roofline"], "step_roofline": m["step_roofline"],
+        "e2e": m["e2e"], "roofline": m["roofline"], "roofline_indexer": m["roofline_indexer"],
+        "step_roofline": m["step_roofline"],
         "indexer_keys_per_s": m["indexer_keys_per_s"], "gpu_launches": m["gpu_launches"],
         "launches_per_step": m["launches_per_step"], "clocks": clocks,
         "breakdown_us_diagnostic": m["breakdown_us"],
@@ -833,7 +960,8 @@ def main():
     if extra is not None:
         e = summarise(extra)
         line["pro1m"] = {"value": e["value"], "unit": "tokens/s", "ms_per_step": e["ms_per_step"],
-                         "step_roofline": e["step_roofline"], "roofline": e["roofline"], "e2e": e["e2e"],
+                         "step_roofline": e["step_roofline"], "roofline": e["roofline"],
+                         "roofline_indexer": e["roofline_indexer"], "e2e": e["e2e"],
                          "indexer_keys_per_s": e["indexer_keys_per_s"], "launches_per_step": e["launches_per_step"],
                          "breakdown_us": e["breakdown_us"]}
         line["gpu_launches"] += e["gpu_launches"]
