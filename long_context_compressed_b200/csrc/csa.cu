@@ -433,7 +433,8 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
   const int key_bytes = fp8 ? csa::IndexCfg<true>::kKeyBytes : csa::IndexCfg<false>::kKeyBytes;
   const int qrow = fp8 ? 128 : 256;
   const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
-  const int fixed = 1024 + q_bytes + 2048 * p.TQ + 8 * (4 + 2 * csa::kMaxAcc) + csa::kKsRing * 256 * 4 +
+  const int fixed = 1024 + q_bytes + csa::kIdxEpiWarps * p.TQ * csa::kIdxHeads * 4 + 8 * (4 + 2 * csa::kMaxAcc) +
+                    csa::kKsRing * 32 * csa::kIdxEpiWarps * 4 +
                     (select_ws ? 2 * csa::kHistBinsIdx * 4 : 0);
   p.stages = std::min(12, (kSmemLimit - fixed) / (key_bytes + 16));
   if (p.stages < 2) return CSA_ERR_UNSUPPORTED;

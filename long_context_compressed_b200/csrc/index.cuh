@@ -9,7 +9,8 @@
 // TQ queries x 64 heads of a query group are the N = 64*TQ operand, K = 128.
 // Both are staged by TMA (128-byte swizzle, K-major) into shared memory;
 // one elected thread issues tcgen05.mma into a double-buffered fp32 TMEM
-// accumulator; eight epilogue warps (two sets taking alternate tiles) read
+// accumulator; sixteen epilogue warps (4 sets taking tiles in turn, or 2 sets of
+// 8 warps that split the group's queries when only 2 accumulators fit) read
 // their 32 TMEM lanes (one key per
 // thread), apply ReLU and the head weights, reduce over the 64 heads and store
 // one fp32 score per (query, key).  Persistent: one CTA per SM walks a
@@ -32,7 +33,8 @@ constexpr int kIdxHeads = 64;
 constexpr int kIdxDim = 128;
 constexpr int kIdxTileKeys = 128;
 constexpr int kMaxAcc = 4;
-constexpr int kIdxThreads = 320;                // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kIdxEpiWarps = 16;
+constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;   // TMA warp, MMA warp, 16 epilogue warps
 constexpr int kKsAhead = 3;                     // key-scale prefetch distance (items of one epilogue set)
 constexpr int kKsRing = kKsAhead + 1;
 constexpr int kHistBinsIdx = 4096;              // 12-bit histogram of order-preserving score keys
@@ -115,16 +117,20 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
   uint64_t* tempty = qfull + 2 + kMaxAcc;           // [kMaxAcc]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 2 + 2 * kMaxAcc);
   float* w_all = reinterpret_cast<float*>(qfull + 4 + 2 * kMaxAcc);  // [8 epilogue warps][TQ][64]
-  float* ks_all = w_all + 8 * TQ * kIdxHeads;                        // [kKsRing][256] key-scale ring
+  float* ks_all = w_all + kIdxEpiWarps * TQ * kIdxHeads;             // [kKsRing][epilogue threads] key-scale ring
   // score histograms of the first two rows this CTA touches (when p.hist is set)
-  int* hist_s = reinterpret_cast<int*>(ks_all + kKsRing * 256);       // [2][kHistBinsIdx]
+  int* hist_s = reinterpret_cast<int*>(ks_all + kKsRing * 32 * kIdxEpiWarps);   // [2][kHistBinsIdx]
 
   const int QG = (p.T + TQ - 1) / TQ;
   const int64_t KT = (p.N + kIdxTileKeys - 1) / kIdxTileKeys;
   const int64_t items = (int64_t)p.B * QG * KT;
   const int64_t w0 = items * blockIdx.x / gridDim.x;
   const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
-  const int NACC = (512 / NQ) < kMaxAcc ? (512 / NQ) : kMaxAcc;   // TMEM accumulators in flight
+  const int NACC = (512 / NQ) < kMaxAcc ? (512 / NQ) : kMaxAcc;   // TMEM accumulators in flight (2 or 4)
+  // epilogue sets: one per accumulator; with 2 accumulators each set has 8 warps, two
+  // per TMEM lane quarter, splitting the group's queries
+  const int nsets = NACC >= 4 ? 4 : 2;
+  const int set_warps = kIdxEpiWarps / nsets;
   const uint32_t tmem_cols = (uint32_t)(NACC * NQ) < 32 ? 32u : (uint32_t)(NACC * NQ);
 
   const int warp = warp_id();
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
     mbar_init(qempty, 1);
     for (int a = 0; a < kMaxAcc; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);                     // one arrive per epilogue warp
+      mbar_init(&tempty[a], set_warps);             // one arrive per epilogue warp of the set
     }
     fence_mbar_init();
     prefetch_tmap(&kmap);
@@ -236,33 +242,37 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       }
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2..9)
-    // Two sets of four warps take alternate tiles; within a set, warp w owns TMEM
-    // lanes 32*(w%4) .. +31, i.e. one key per thread.
+    // ---------------------------------------------------------------- epilogue (warps 2..17)
+    // nsets sets take the work items in turn (set s: items w0 + s, w0 + s + nsets, ..);
+    // warp w owns TMEM lanes 32*(w%4) .. +31, i.e. one key per thread, and the
+    // queries [q_lo, q_hi) of the group.
+    const int e = warp - 2;
     const int quarter = warp & 3;                   // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + (int)lane_id();  // key within the tile
-    const int es = (warp - 2) >> 2;                 // epilogue set: 0 or 1
+    const int es = (e >> 2) % nsets;                // epilogue set
+    const int qpart = (e >> 2) / nsets;             // 0, or 0/1 with 2 sets
+    const int q_lo = qpart * TQ * nsets / 4, q_hi = (qpart + 1) * TQ * nsets / 4;
     const int acc_shift = NACC == 4 ? 2 : (NACC == 2 ? 1 : 0);
-    float* w_s = w_all + (warp - 2) * TQ * kIdxHeads;
-    int64_t nv_q[4] = {0, 0, 0, 0};
+    float* w_s = w_all + e * TQ * kIdxHeads;
+    int nv_q[4] = {0, 0, 0, 0};
     // key scales (e4m3) travel by cp.async into a per-thread ring in shared memory,
     // kKsAhead of this set's items ahead along a second iterator: no register waits
     // on a load in flight
+    constexpr int kEpiThreads = 32 * kIdxEpiWarps;
     float* ks_ring = ks_all + (threadIdx.x - 64);     // column of this epilogue thread
     IndexItem ahead = index_item(w0, QG, KT);
     int64_t w_ahead = w0;
-    if (es) { index_next(ahead, QG, KT); ++w_ahead; }
+    for (int j = 0; j < es; ++j) { index_next(ahead, QG, KT); ++w_ahead; }
     int ring_put = 0;
     auto ks_fetch = [&]() {
       if (FP8 && w_ahead < w1) {
         const int64_t ii = ahead.kt * kIdxTileKeys + row;
-        if (ii < p.N) cp_async_4(ks_ring + ring_put * 256, p.k_scale + (int64_t)ahead.b * p.N + ii);
+        if (ii < p.N) cp_async_4(ks_ring + ring_put * kEpiThreads, p.k_scale + (int64_t)ahead.b * p.N + ii);
       }
       cp_async_commit();
       ring_put = ring_put + 1 == kKsRing ? 0 : ring_put + 1;
-      w_ahead += 2;
-      index_next(ahead, QG, KT);
-      index_next(ahead, QG, KT);
+      w_ahead += nsets;
+      for (int j = 0; j < nsets; ++j) index_next(ahead, QG, KT);
     };
     if (FP8)
       for (int j = 0; j < kKsAhead; ++j) ks_fetch();
@@ -271,30 +281,35 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
     IndexItem it = index_item(w0, QG, KT);
     int64_t w = w0;
     int cnt = 0;
-    if (es) { index_next(it, QG, KT); ++w; ++cnt; }
-    for (; w < w1; w += 2, cnt += 2, index_next(it, QG, KT), index_next(it, QG, KT)) {
+    for (int j = 0; j < es; ++j) { index_next(it, QG, KT); ++w; ++cnt; }
+    for (; w < w1; w += nsets, cnt += nsets) {
+      if (cnt >= nsets)
+        for (int j = 0; j < nsets; ++j) index_next(it, QG, KT);
       if (it.b != prev_b || it.qg != prev_qg) {
         // each epilogue warp keeps a private copy of the group's head weights; the
         // weights, query scales and n_valid are all requested before any is used
         // (one memory round trip, overlapping the wait for the first accumulator)
         constexpr int PER = 4 * kIdxHeads / 32;
-        float wv[PER], sv[PER];
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const int j = (int)lane_id() + 32 * u;
-          const int t = it.qg * TQ + j / kIdxHeads;
-          const bool in = j < TQ * kIdxHeads && t < p.T;
-          const int64_t o = ((int64_t)it.b * p.T + t) * kIdxHeads + (j % kIdxHeads);
-          wv[u] = in ? __ldg(p.w + o) : 0.f;
-          sv[u] = (FP8 && in) ? __ldg(p.q_scale + o) : 1.f;
-        }
         const int tq = it.qg * TQ + (int)lane_id();
         const int nv_l = ((int)lane_id() < TQ && tq < p.T) ? __ldg(p.n_valid + (int64_t)it.b * p.T + tq) : 0;
         __syncwarp();
 #pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const int j = (int)lane_id() + 32 * u;
-          if (j < TQ * kIdxHeads) w_s[j] = FP8 ? wv[u] * sv[u] : wv[u];
+        for (int u0 = 0; u0 < PER; u0 += PER / 2) {     // two batches of loads (register budget)
+          float wv[PER / 2], sv[PER / 2];
+#pragma unroll
+          for (int u = 0; u < PER / 2; ++u) {
+            const int j = (int)lane_id() + 32 * (u0 + u);
+            const int t = it.qg * TQ + j / kIdxHeads;
+            const bool in = j < TQ * kIdxHeads && t < p.T;
+            const int64_t o = ((int64_t)it.b * p.T + t) * kIdxHeads + (j % kIdxHeads);
+            wv[u] = in ? __ldg(p.w + o) : 0.f;
+            sv[u] = (FP8 && in) ? __ldg(p.q_scale + o) : 1.f;
+          }
+#pragma unroll
+          for (int u = 0; u < PER / 2; ++u) {
+            const int j = (int)lane_id() + 32 * (u0 + u);
+            if (j < TQ * kIdxHeads) w_s[j] = FP8 ? wv[u] * sv[u] : wv[u];
+          }
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) nv_q[q] = __shfl_sync(0xffffffffu, nv_l, q);
@@ -308,7 +323,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       if (FP8) {
         ks_fetch();                                 // item kKsAhead ahead
         cp_async_wait_group<kKsAhead>();            // this item's copy has landed
-        ks = ks_ring[ring_get * 256];
+        ks = ks_ring[ring_get * kEpiThreads];
         ring_get = ring_get + 1 == kKsRing ? 0 : ring_get + 1;
       }
       if (!mbar_wait(&tfull[acc], aph)) break;
@@ -316,29 +331,25 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       const int64_t i = it.kt * kIdxTileKeys + row;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        if (q >= TQ) break;
+        if (q < q_lo) continue;
+        if (q >= q_hi) break;
         const int t = it.qg * TQ + q;
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NQ + q * 64);
-        float v0[32], v1[32];
-        tmem_ld32(taddr, v0);
-        tmem_ld32(taddr + 32, v1);
-        tmem_wait_ld();
-        if (t >= p.T) continue;
+        if (t >= p.T) continue;                       // uniform over the warp
         const float* wq = w_s + q * kIdxHeads;
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;   // independent chains
 #pragma unroll
-        for (int h = 0; h < 32; h += 4) {
-          s0 = fmaf(wq[h], fmaxf(v0[h], 0.f), s0);
-          s1 = fmaf(wq[h + 1], fmaxf(v0[h + 1], 0.f), s1);
-          s2 = fmaf(wq[h + 2], fmaxf(v0[h + 2], 0.f), s2);
-          s3 = fmaf(wq[h + 3], fmaxf(v0[h + 3], 0.f), s3);
-        }
+        for (int half = 0; half < 2; ++half) {          // 32 heads at a time (register budget)
+          float v[32];
+          tmem_ld32(taddr + 32 * half, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 32; h += 4) {
-          s0 = fmaf(wq[32 + h], fmaxf(v1[h], 0.f), s0);
-          s1 = fmaf(wq[33 + h], fmaxf(v1[h + 1], 0.f), s1);
-          s2 = fmaf(wq[34 + h], fmaxf(v1[h + 2], 0.f), s2);
-          s3 = fmaf(wq[35 + h], fmaxf(v1[h + 3], 0.f), s3);
+          for (int h = 0; h < 32; h += 4) {
+            s0 = fmaf(wq[32 * half + h], fmaxf(v[h], 0.f), s0);
+            s1 = fmaf(wq[32 * half + h + 1], fmaxf(v[h + 1], 0.f), s1);
+            s2 = fmaf(wq[32 * half + h + 2], fmaxf(v[h + 2], 0.f), s2);
+            s3 = fmaf(wq[32 * half + h + 3], fmaxf(v[h + 3], 0.f), s3);
+          }
         }
         const float sc = (s0 + s1) + (s2 + s3);
         if (i < p.N) {

@@ -136,6 +136,37 @@ __device__ __forceinline__ void find_digit_block(const int* hist, int nbins, int
   }
 }
 
+// Skewed shared-memory histogram index: bin h lives at h + h/32, so threads that
+// own consecutive groups of 8 or 16 bins read them without bank conflicts.
+__device__ __forceinline__ int skew(int h) { return h + (h >> 5); }
+
+// find_digit_block over a skewed histogram (nbins == BPT * blockDim.x).
+template <int BPT>
+__device__ __forceinline__ void find_digit_skewed(const int* hist, int nbins, int remaining, int* res,
+                                                  int* scratch) {
+  const int hi = nbins - 1 - BPT * (int)threadIdx.x;
+  int c[BPT], local = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    c[j] = hist[skew(hi - j)];
+    local += c[j];
+  }
+  int total;
+  const int exc = block_excl_scan(local, scratch, &total);
+  if (exc < remaining && remaining <= exc + local) {
+    int above = exc;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (above + c[j] >= remaining) {
+        res[0] = hi - j;
+        res[1] = above;
+        break;
+      }
+      above += c[j];
+    }
+  }
+}
+
 // Write the selection of a segment in index order.  Every thread owns the
 // contiguous index range [lo, hi) and calls get(i) -> key.
 template <typename GetKey>
@@ -177,7 +208,7 @@ __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict_
                                                         const int32_t* __restrict__ map) {
   griddep_sync();
   extern __shared__ __align__(16) uint32_t keys[];  // [min(N, kRowSmemMax)]
-  __shared__ int hist[256];
+  __shared__ __align__(16) int rhist[kHistBins + kHistBins / 32];   // skewed
   __shared__ int scratch[33];
   __shared__ int res[2];
   const int64_t row = blockIdx.x;
@@ -190,28 +221,44 @@ __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict_
     return;
   }
   const float* s = scores + row * N;
-  for (int i = threadIdx.x; i < nv; i += blockDim.x) keys[i] = order_key(s[i]);
+  // every score of this thread is requested before any is used (one memory round trip)
+  {
+    constexpr int kPer = kRowSmemMax / 1024;
+    float v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = u * 1024 + (int)threadIdx.x;
+      v[u] = i < nv ? __ldg(s + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = u * 1024 + (int)threadIdx.x;
+      if (i < nv) keys[i] = order_key(v[u]);
+    }
+  }
+  // radix select with digits of 12, 10 and 10 bits on a skewed histogram
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int j = threadIdx.x; j < 256; j += blockDim.x) hist[j] = 0;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 20 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 0 ? 4095u : 1023u;
+    for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) rhist[j] = 0;
     __syncthreads();
-    for (int i0 = 0; i0 < nv; i0 += blockDim.x) {
-      const int i = i0 + threadIdx.x;
-      const uint32_t key = i < nv ? keys[i] : 0u;
-      const bool act = i < nv && (key & pmask) == prefix;
-      warp_hist_add(hist, (key >> shift) & 255u, act);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      const uint32_t key = keys[i];
+      if ((key & pmask) == prefix) atomicAdd(&rhist[skew((int)((key >> shift) & dmask))], 1);
     }
     __syncthreads();
-    find_digit(hist, 256, remaining, res);
+    if (pass == 0) find_digit_skewed<kHistBins / 1024>(rhist, kHistBins, remaining, res, scratch);
+    else find_digit_skewed<1>(rhist, 1024, remaining, res, scratch);
     __syncthreads();
     prefix |= (uint32_t)res[0] << shift;
-    pmask |= 255u << shift;
+    pmask |= dmask << shift;
     remaining -= res[1];
     __syncthreads();
   }
-  const int per = (nv + blockDim.x - 1) / blockDim.x;
+  // contiguous index ranges of odd length per thread: conflict-free shared-memory reads
+  const int per = ((nv + (int)blockDim.x - 1) / (int)blockDim.x) | 1;
   const int64_t lo = (int64_t)threadIdx.x * per;
   const int64_t hi = lo + per < nv ? lo + per : nv;
   write_selection(lo < nv ? lo : nv, hi, [&](int64_t i) { return keys[i]; }, prefix, remaining, out, scratch);
@@ -453,37 +500,6 @@ template <>
 __device__ __forceinline__ void unpack_vec<float>(uint4 v, float* f) {  // 4 fp32
   f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
   f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
-}
-
-// Skewed shared-memory histogram index: bin h lives at h + h/32, so threads that
-// own consecutive groups of 8 or 16 bins read them without bank conflicts.
-__device__ __forceinline__ int skew(int h) { return h + (h >> 5); }
-
-// find_digit_block over a skewed histogram (nbins == BPT * blockDim.x).
-template <int BPT>
-__device__ __forceinline__ void find_digit_skewed(const int* hist, int nbins, int remaining, int* res,
-                                                  int* scratch) {
-  const int hi = nbins - 1 - BPT * (int)threadIdx.x;
-  int c[BPT], local = 0;
-#pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    c[j] = hist[skew(hi - j)];
-    local += c[j];
-  }
-  int total;
-  const int exc = block_excl_scan(local, scratch, &total);
-  if (exc < remaining && remaining <= exc + local) {
-    int above = exc;
-#pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      if (above + c[j] >= remaining) {
-        res[0] = hi - j;
-        res[1] = above;
-        break;
-      }
-      above += c[j];
-    }
-  }
 }
 
 // Row r (one query per sequence: T == 1) of scores [rows, N].  Candidates are the
