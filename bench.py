@@ -160,6 +160,24 @@ def measured_tflops():
 
 
 # ----------------------------------------------------------------------------- the step
+def _pack(tensors, device):
+    """One uint8 device buffer holding copies of `tensors` at 16-byte aligned offsets,
+    and typed views of it in the same order."""
+    import torch
+    nbytes = [t.numel() * t.element_size() for t in tensors]
+    offs, total = [], 0
+    for n in nbytes:
+        offs.append(total)
+        total += (n + 15) // 16 * 16
+    buf = torch.empty(max(total, 16), dtype=torch.uint8, device=device)
+    views = []
+    for t, o, n in zip(tensors, offs, nbytes):
+        v = buf[o:o + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+    return buf, views
+
+
 class DecodeSet:
     """One input set of a decode workload: resident caches, per-step inputs, outputs and
     workspaces on the device, plus pinned host copies of the per-step inputs/outputs."""
@@ -214,11 +232,19 @@ class DecodeSet:
             self.hcomp = torch.empty((B, 1, D), dtype=torch.bfloat16, device=dev)
             self.hattn_ws = csa.attn_workspace(B, T, H, D, 128 + Nh, device=dev)
             self.hout = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
-        self.outputs = [self.out] + ([self.hout] if with_hca else [])
-        self.host_in = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in self.inputs.items()}
-        for n, t in self.inputs.items():
-            self.host_in[n].copy_(t)
-        self.host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in self.outputs]
+        # per-step inputs and outputs live in one contiguous device buffer each (views at
+        # 16-byte aligned offsets), so a step moves them with one copy per direction
+        self.in_buf, views = _pack(list(self.inputs.values()), dev)
+        self.inputs = dict(zip(self.inputs.keys(), views))
+        outs = [self.out] + ([self.hout] if with_hca else [])
+        self.out_buf, outs = _pack(outs, dev)
+        self.out = outs[0]
+        if with_hca:
+            self.hout = outs[1]
+        self.outputs = outs
+        self.host_in = torch.empty(self.in_buf.numel(), dtype=torch.uint8, pin_memory=True)
+        self.host_in.copy_(self.in_buf)
+        self.host_out = torch.empty(self.out_buf.numel(), dtype=torch.uint8, pin_memory=True)
 
     # -- byte accounting (algorithmic: inputs read once, outputs written once, intermediates excluded)
     def index_bytes(self):
@@ -256,7 +282,7 @@ class DecodeSet:
 
     def per_step_io(self):
         nb = lambda t: t.numel() * t.element_size()
-        return sum(nb(t) for t in self.inputs.values()), sum(nb(o) for o in self.outputs)
+        return nb(self.in_buf), nb(self.out_buf)
 
     # -- the step
     def run(self, side_streams, timing_events: bool = False, copies: bool = False):
@@ -267,8 +293,7 @@ class DecodeSet:
         x = self.inputs
         main = torch.cuda.current_stream()
         if copies:
-            for n, t in x.items():
-                t.copy_(self.host_in[n], non_blocking=True)
+            self.in_buf.copy_(self.host_in, non_blocking=True)
         def side_branch():
             # compressors and the HCA layer: independent of the indexer chain and of each
             # other within a step, so they run on side streams, started once the
@@ -328,8 +353,7 @@ class DecodeSet:
         if timing_events:
             self.marks = marks
         if copies:
-            for h, o in zip(self.host_out, self.outputs):
-                h.copy_(o, non_blocking=True)
+            self.host_out.copy_(self.out_buf, non_blocking=True)
 
 
 def capture(sets, sides, **kw):
