@@ -477,6 +477,7 @@ constexpr int kSelPerThread = 4;     // scores each thread loads per pass of the
 constexpr int kSelTcRows = 128;      // candidates rescored per tensor-core batch (bf16)
 constexpr int kSelKeyBatch = 64;     // candidate key rows per SIMT batch (fp32)
 constexpr int kSelCandSmem = 8192;   // candidates the last CTA stages in shared memory
+constexpr int kSelPrefetch = 2048;   // chunk entries whose scores are fetched with the histogram
 constexpr int kSelMaxChunkLen = 16384;  // entries per chunk (shared-memory candidate list)
 static_assert(kSelPerThread * (kSelThreads / 32) == 32, "one scan lane per (pass, warp)");
 static_assert(kSelMaxChunks % kSelThreads == 0, "chunk table split evenly over the threads");
@@ -571,6 +572,30 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   float* wsm = reinterpret_cast<float*>(lkey + chunk);               // [64]
   if (active) {
     const int kk = RESCORE ? (kc < nv ? kc : nv) : k;
+    const float* srow = scores + row * N;
+    const int64_t c0 = (int64_t)blockIdx.x * chunk;
+    const int64_t c1 = c0 + chunk < nv ? c0 + chunk : nv;
+    // Every load the front half needs is issued here, before any is used: the
+    // histogram, this chunk's scores (chunks up to kSelPrefetch entries) and, for the
+    // tensor-core rescoring, the query tile and head weights.
+    constexpr int kPre = kSelPrefetch / kSelThreads;
+    const bool prefetched = c1 - c0 <= kSelPrefetch;
+    float pre[kPre];
+    if (prefetched) {
+#pragma unroll
+      for (int u = 0; u < kPre; ++u) {
+        const int64_t i = c0 + (int64_t)u * kSelThreads + threadIdx.x;
+        pre[u] = i < c1 ? __ldg(srow + i) : 0.f;
+      }
+    }
+    uint4 qv[TC ? 4 : 1];
+    float wv = 0.f;
+    if (TC) {
+      const uint4* q4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(qI) + row * 64 * 128);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) qv[u] = __ldg(q4 + threadIdx.x + u * kSelThreads);
+      if (threadIdx.x < 64) wv = w[row * 64 + threadIdx.x];
+    }
     // ---- threshold bin b*: count(bins > b*) < kk <= count(bins >= b*)
     {
       const int4* g4 = reinterpret_cast<const int4*>(ghist);
@@ -586,23 +611,37 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         histk[skew(h + 3)] = v[u].w;
       }
     }
+    if (TC) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = threadIdx.x + u * kSelThreads, r = j >> 4, c = j & 15;
+        *reinterpret_cast<uint4*>(qt_s + (c >> 3) * 64 * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = qv[u];
+      }
+      if (threadIdx.x < 64) wsm[threadIdx.x] = wv;
+    }
     if (threadIdx.x == 0) lcount = 0;
     __syncthreads();
     find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, kk, res, scratch);
     __syncthreads();
     const uint32_t bstar = (uint32_t)res[0];
-    // ---- this chunk's candidates, compacted in index order (each thread loads its
-    // scores before using them; one warp scans the 32 (pass, warp) counts)
-    const float* srow = scores + row * N;
-    const int64_t c0 = (int64_t)blockIdx.x * chunk;
-    const int64_t c1 = c0 + chunk < nv ? c0 + chunk : nv;
+    // ---- this chunk's candidates, compacted in index order (one warp scans the 32
+    // (pass, warp) counts)
     int lbase = 0;
-    for (int64_t base0 = c0; base0 < c1; base0 += (int64_t)kSelPerThread * blockDim.x) {
+    int pass = 0;
+    for (int64_t base0 = c0; base0 < c1; base0 += (int64_t)kSelPerThread * blockDim.x, ++pass) {
       float v[kSelPerThread];
+      if (prefetched) {
 #pragma unroll
-      for (int u = 0; u < kSelPerThread; ++u) {
-        const int64_t i = base0 + (int64_t)u * blockDim.x + threadIdx.x;
-        v[u] = i < c1 ? __ldg(srow + i) : 0.f;
+        for (int pp = 0; pp < kPre / kSelPerThread; ++pp)   // static register indices
+          if (pp == pass)
+#pragma unroll
+            for (int u = 0; u < kSelPerThread; ++u) v[u] = pre[pp * kSelPerThread + u];
+      } else {
+#pragma unroll
+        for (int u = 0; u < kSelPerThread; ++u) {
+          const int64_t i = base0 + (int64_t)u * blockDim.x + threadIdx.x;
+          v[u] = i < c1 ? __ldg(srow + i) : 0.f;
+        }
       }
       uint32_t key[kSelPerThread], m[kSelPerThread];
 #pragma unroll
@@ -635,19 +674,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   }
   if (TC && active && nloc > 0) {
     // ---- exact rescoring on tcgen05: candidates (M = 128 per batch) x 64 heads, K = 128
-    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qI) + row * 64 * 128;
+    // (the query tile and head weights were staged with the front-half loads)
     const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(kI) + row * N * 128;
-    {
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(qrow) + threadIdx.x + u * kSelThreads);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = threadIdx.x + u * kSelThreads, r = j >> 4, c = j & 15;
-        *reinterpret_cast<uint4*>(qt_s + (c >> 3) * 64 * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v[u];
-      }
-    }
-    if (threadIdx.x < 64) wsm[threadIdx.x] = w[row * 64 + threadIdx.x];
     const uint32_t idesc = make_idesc(128, 64, 1, 0, 0);
     uint32_t mph = 0;
     for (int cb = 0; cb < nloc; cb += kSelTcRows) {

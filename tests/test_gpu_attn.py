@@ -79,6 +79,24 @@ def test_bf16_ragged(csa, D, H, B, T):
     check_attn_bf16(g, ref, what=f"bf16 D={D} H={H} B={B} T={T}")
 
 
+@pytest.mark.parametrize("D,H,k", [(512, 64, 128), (512, 100, 224), (512, 128, 352), (512, 64, 480),
+                                   (512, 128, 1024), (256, 72, 400), (128, 16, 900)])
+def test_bf16_split_clusters(csa, D, H, k):
+    """Few queries with long row lists: the row list is split over 2..8 CTAs that merge
+    their partials inside a thread-block cluster; H not a multiple of 64 leaves the
+    last head group partly empty."""
+    B, T, N = 2, 1, 4096
+    wl = synth.Workload(f"attn_split_{D}_{H}_{k}", "bf16", B=B, ctx=2 * N, T=T, q_pos0=2 * N - 1, ratio=1, N=N,
+                        H=H, D=D)
+    at, q_pos, swa_pos0, _ = _case(wl, seed=k + H)
+    idx = synth.random_subset(k, "attn/split/idx", torch.full((B, T), N), k).numpy()
+    scale = 1 / math.sqrt(D)
+    g = _gpu_sparse(csa, at, q_pos, swa_pos0, idx, scale)
+    ref = oracle.sparse_attn(_np(at["q"]), _np(at["kv"]), _np(at["swa_kv"]), swa_pos0, q_pos,
+                             at["sink"].numpy(), idx, scale)
+    check_attn_bf16(g, ref, what=f"split D={D} H={H} k={k}")
+
+
 @pytest.mark.parametrize("name", ["flash64k", "pro1m"])
 def test_bf16_decode_full(csa, name):
     wl = synth.WORKLOADS[name]
