@@ -21,7 +21,8 @@
 // KV rows are gathered with 16-byte cp.async into 128-byte-swizzled K-major
 // tiles of R rows; S = Q K^T (tcgen05, fp32 in TMEM, double buffered); four
 // softmax warps (one head per thread) run the online softmax in the log2
-// domain, writing P (bf16) to shared memory; O += P V (tcgen05; the same KV
+// domain, writing P (bf16) back into TMEM over the tile's S columns; O += P V
+// (tcgen05 with the A operand read from TMEM; the same KV
 // tile read as an MN-major operand, restricted to this CTA's D-slice of width
 // DH <= 256) accumulates in TMEM.  O is rescaled only when a tile's maximum
 // exceeds the running reference by more than 2^8, so exponentials stay <= 256.
@@ -160,10 +161,6 @@ struct AttnCfg {
   static constexpr int NDH = D / DH;
   static constexpr int kAtoms = D / 64;                    // 128-byte atoms per row
   static constexpr int kKVBytes = R * D * 2;
-  static constexpr int kPRowBytes = R * 2;                 // 64 (SW64) or 128 (SW128)
-  static constexpr int kPBytes = 128 * kPRowBytes;
-  static constexpr uint32_t kPLayout = (kPRowBytes == 128) ? kLayoutSW128 : kLayoutSW64;
-  static constexpr int kPSBO = 8 * kPRowBytes;
   static constexpr int kTmemCols = (DH + 2 * R) <= 256 ? 256 : 512;  // O slice + two S buffers
   static constexpr int kSCol0 = DH;                        // S buffers after O
   static constexpr int kThreads = 288;                     // 4 softmax + 4 loader + 1 MMA warps
@@ -174,10 +171,10 @@ struct AttnCfg {
   // the Q tile is 64 rows per 64-dim atom and four KV stages always fit
   static constexpr int kHeadGroup = 64;
   static constexpr int kQBytes = kHeadGroup * D * 2;
-  static constexpr int kStages = ((232448 - 1024 - kBarBytes - kQBytes - 2 * kPBytes) / kKVBytes) >= kMaxStages
+  static constexpr int kStages = ((232448 - 1024 - kBarBytes - kQBytes) / kKVBytes) >= kMaxStages
                                      ? kMaxStages
-                                     : (232448 - 1024 - kBarBytes - kQBytes - 2 * kPBytes) / kKVBytes;
-  static constexpr int kSmem = 1024 + kQBytes + kStages * kKVBytes + 2 * kPBytes + kBarBytes;
+                                     : (232448 - 1024 - kBarBytes - kQBytes) / kKVBytes;
+  static constexpr int kSmem = 1024 + kQBytes + kStages * kKVBytes + kBarBytes;
   static __host__ __device__ int head_groups(int H) { return (H + kHeadGroup - 1) / kHeadGroup; }
 };
 
@@ -204,12 +201,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   constexpr int NS = Cfg::kStages;
   uint8_t* q_s = smem;
   uint8_t* kv_s = q_s + Cfg::kQBytes;                       // [NS][kKVBytes]
-  uint8_t* p_s = kv_s + NS * Cfg::kKVBytes;                 // [2][kPBytes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Cfg::kPBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kv_s + NS * Cfg::kKVBytes);
   uint64_t* full = bars;        // [4] KV stage loaded (128 cp.async arrivals)
   uint64_t* empty = bars + 4;   // [4] KV stage consumed by PV
   uint64_t* sfull = bars + 8;   // [2] S ready
-  uint64_t* sfree = bars + 10;  // [2] S read by softmax
+  uint64_t* sfree = bars + 10;  // [2] (unused: S buffer reuse waits for the PV that read its P)
   uint64_t* pfull = bars + 12;  // [2] P written
   uint64_t* pdone = bars + 14;  // [2] PV done (P buffer free, O consistent)
   uint64_t* qfull = bars + 16;
@@ -369,7 +365,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         const int s = ks;
         const uint32_t ph = kph;
         if (!mbar_wait(&full[s], ph)) return false;
-        if (!mbar_wait(&sfree[sb], sph ^ 1)) return false;
+        // S buffer sb holds P of tile jj-2 until that tile's PV has run
+        if (!mbar_wait(&pdone[sb], sph ^ 1)) return false;
         fence_proxy_async_smem();                   // cp.async data -> tensor core reads
         tc_fence_after();
         const uint32_t kb = smem_u32(kv_s + s * Cfg::kKVBytes);
@@ -392,13 +389,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         const int sb = jj & 1;
         if (!mbar_wait(&pfull[sb], (jj >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t pb = smem_u32(p_s + sb * Cfg::kPBytes);
+        // P (bf16, two per column) sits in TMEM over the S columns of its tile
+        const uint32_t pt = tmem + Cfg::kSCol0 + sb * R;
         const uint32_t vb = smem_u32(kv_s + s * Cfg::kKVBytes) + dh * (DH / 64) * R * 128;
 #pragma unroll
         for (int kk = 0; kk < R / 16; ++kk) {
-          const uint64_t ad = smem_desc(pb + kk * 32, 16, Cfg::kPSBO, Cfg::kPLayout);
           const uint64_t bd = smem_desc(vb + kk * 2048, R * 128, 1024, kLayoutSW128);
-          mma_bf16(tmem, ad, bd, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem, pt + kk * 8, bd, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&pdone[sb]);
         mma_commit(&empty[s]);
@@ -419,7 +416,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     int ks = 0;
     uint32_t kph = 0;
     constexpr int RPW = R / 4;                 // tile rows covered by one loader warp
-    for (int jj = 0; jj < nt; ++jj) {
+    // warps 2, 3 own the operand's filler rows (64..127): no softmax for them, only the
+    // hand-overs, in the same order as the real rows so every barrier phase stays exact
+    // (their P rows stay as they are: O rows 64..127 are never read)
+    const int jj_end = warp < 2 ? nt : 0;
+    for (int jj = 0; ok && jj < nt && warp >= 2; ++jj) {
+      const int sb = jj & 1;
+      const uint32_t ph = (jj >> 1) & 1;
+      if (!mbar_wait(&sfull[sb], ph)) { ok = false; break; }
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&pfull[sb]);
+    }
+    for (int jj = 0; jj < jj_end; ++jj) {
       const int sb = jj & 1;
       const uint32_t ph = (jj >> 1) & 1;
       const int s = ks;
@@ -436,17 +444,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       tmem_ld32(tmem + lane_base + Cfg::kSCol0 + sb * R, z);
       if constexpr (R == 64) tmem_ld32(tmem + lane_base + Cfg::kSCol0 + sb * R + 32, z + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane_id() == 0) mbar_arrive(&sfree[sb]);
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < R; ++c) {
         z[c] = ((valid >> c) & 1) ? z[c] * zs : -INFINITY;
         mt = fmaxf(mt, z[c]);
       }
-      // P buffer sb is free once PV of tile jj-2 completed
-      if (!mbar_wait(&pdone[sb], ph ^ 1)) { ok = false; break; }
       if (mt > m_used + 8.f) {
         const float m_new = mt;
         if (m_used != -INFINITY && jj > 0) {
@@ -481,14 +484,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         packed[c / 2] = *reinterpret_cast<uint32_t*>(&v);
       }
       l += ps0 + ps1;
-      uint8_t* prow = p_s + sb * Cfg::kPBytes + h * Cfg::kPRowBytes;
-#pragma unroll
-      for (int c = 0; c < R / 8; ++c) {
-        const int phys = (R == 64) ? (c ^ (h & 7)) : (c ^ ((h >> 1) & 3));
-        *reinterpret_cast<uint4*>(prow + phys * 16) =
-            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      // P over this tile's S columns (the PV operand A is read from TMEM)
+      const uint32_t pt = tmem + lane_base + Cfg::kSCol0 + sb * R;
+      if constexpr (R == 32) {
+        tmem_st16u(pt, packed);
+      } else {
+        tmem_st16u(pt, packed);
+        tmem_st16u(pt + 16, packed + 16);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&pfull[sb]);
