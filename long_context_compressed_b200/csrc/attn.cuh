@@ -255,9 +255,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   const RowList rl = make_row_list(p, b, t);
   const int n_rows = rl.n_swa + rl.n_mem;
   const int n_tiles_all = (n_rows + R - 1) / R;
-  const int tps = (n_tiles_all + p.nsplit - 1) / p.nsplit;
-  const int j0 = split * tps;
-  const int j1 = min(n_tiles_all, j0 + tps);
+  // balanced tile ranges: the splits' tile counts differ by at most one
+  const int j0 = (int)((int64_t)split * n_tiles_all / p.nsplit);
+  const int j1 = (int)((int64_t)(split + 1) * n_tiles_all / p.nsplit);
   const int nt = j1 > j0 ? j1 - j0 : 0;      // tiles of this CTA
   // the index value behind list row rg (only memory rows of sparse_attn read memory)
   auto fetch_raw = [&](int rg) -> int32_t {
@@ -278,6 +278,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ loaders (128 threads)
     const int lt = threadIdx.x - 128;
+    if (lt == 0) {
+      if (p.has_kvmap) prefetch_tmap(&kvmap);
+      if (p.has_swamap) prefetch_tmap(&swamap);
+    }
     if (nt > 0) {
       const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(p.kv);
       const __nv_bfloat16* swa = static_cast<const __nv_bfloat16*>(p.swa);
@@ -315,10 +319,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         if (swa_tile || mem_tile) {
           src = kv;                                   // every row valid
           if (lt == 0) {
+            // one box of {64 dims, R rows, all 64-dim atoms}: the atoms land R rows apart,
+            // the K-major layout the MMA reads
             mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKVBytes);
             const int y = swa_tile ? (int)rl.swa_row0 + rg0 : rg0 - rl.n_swa;
-            for (int a = 0; a < Cfg::kAtoms; ++a)
-              tma_load_3d(tile + a * R * 128, swa_tile ? &swamap : &kvmap, &full[s], a * 64, y, b);
+            tma_load_4d(tile, swa_tile ? &swamap : &kvmap, &full[s], 0, y, 0, b);
           } else {
             mbar_arrive(&full[s]);
           }

@@ -113,6 +113,22 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-tile map of a [dim2, rows, D] bf16 tensor seen as {64 elements, rows, D/64
+// atoms, dim2}: one box of {64, box_rows, D/64, 1} holds box_rows full rows with
+// each 64-element atom stored box_rows rows apart (128-byte swizzle).
+bool make_row_tile_map(CUtensorMap* m, const void* ptr, uint64_t D, uint64_t rows, uint64_t dim2,
+                       uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn || D % 64 != 0 || D / 64 > 256) return false;
+  cuuint64_t dims[4] = {64, rows, D / 64, dim2};
+  cuuint64_t strides[3] = {D * 2, 128, rows * D * 2};
+  cuuint32_t box[4] = {64, box_rows, (cuuint32_t)(D / 64), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Kernel launch with programmatic stream serialization (PDL): the kernel may begin
 // launching while its predecessor in the stream finishes; every kernel of this
 // library waits for the predecessor (griddepcontrol.wait) before touching global
@@ -260,10 +276,10 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
   const uint32_t rows_per_tile = p.D >= 512 ? 32u : 64u;
   std::memset(&kvmap, 0, sizeof(kvmap));
   std::memset(&swamap, 0, sizeof(swamap));
-  p.has_kvmap = p.N > 0 && make_map(&kvmap, p.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D,
-                                    (uint64_t)p.N, (uint64_t)p.B, 64, rows_per_tile) ? 1 : 0;
-  p.has_swamap = p.W > 0 && make_map(&swamap, p.swa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.D,
-                                     (uint64_t)p.W, (uint64_t)p.B, 64, rows_per_tile) ? 1 : 0;
+  p.has_kvmap = p.N > 0 && make_row_tile_map(&kvmap, p.kv, (uint64_t)p.D, (uint64_t)p.N, (uint64_t)p.B,
+                                             rows_per_tile) ? 1 : 0;
+  p.has_swamap = p.W > 0 && make_row_tile_map(&swamap, p.swa, (uint64_t)p.D, (uint64_t)p.W, (uint64_t)p.B,
+                                              rows_per_tile) ? 1 : 0;
   switch (p.D) {
 #define CSA_LAUNCH_ATTN(DD)                                                                       \
   case DD: {                                                                                      \
