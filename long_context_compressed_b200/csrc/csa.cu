@@ -356,10 +356,11 @@ int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* 
   cudaStream_t st = as_stream(stream);
   const bool bf_in = in_dtype == CSA_BF16, bf_out = out_dtype == CSA_BF16;
   if (ratio == 4) {
-    // 8 channels per thread (16-byte loads, 4x fewer requests) once that still fills
-    // every SM with a CTA; 2 otherwise
+    // 8 channels per thread (16-byte loads) only once that still gives two waves of
+    // CTAs: its 2m x 8 live values per thread cap residency at one CTA per SM, which
+    // on smaller inputs loses to the 2-channel variant's occupancy
     const int64_t total8 = (int64_t)B * n_entries * (c / 8);
-    const bool wide = total8 >= (int64_t)sm_count() * 256;
+    const bool wide = total8 >= (int64_t)sm_count() * 2 * 256;
     const int64_t total = wide ? total8 : 4 * total8;
     if (total >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
     const int64_t blocks64 = (total + 255) / 256;
