@@ -57,6 +57,17 @@ def test_csa_workloads(csa, name):
         check_bf16_store(gpu, ref, mag, what=name + " index keys")
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_csa_wide_variant(csa, out_dtype):
+    """Enough entries for the 8-channels-per-thread (16-byte load) variant: B = 4 sequences
+    of a 4,096-token chunk at c = 512, with the carry."""
+    wl = synth.Workload("csa_wide", "bf16", B=4, ctx=4096, T=1, q_pos0=4095, ratio=4, N=1024, H=16, D=128,
+                        comp_L=4096, comp_c=512)
+    d = synth.draw_compressor(wl, seed=19)
+    gpu, ref, mag = _run_csa(csa, d, out_dtype, True)
+    (check_f32 if out_dtype == torch.float32 else check_bf16_store)(gpu, ref, mag, what="csa wide")
+
+
 def test_csa_chunked_equals_whole(csa):
     """Compressing in two chunks with the carry equals one pass, bit-exact on the GPU too."""
     wl = synth.Workload("chunk", "bf16", B=2, ctx=512, T=1, q_pos0=511, ratio=4, N=128, H=16, D=128,
