@@ -337,7 +337,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NQ + q * 64);
         if (t >= p.T) continue;                       // uniform over the warp
         const float* wq = w_s + q * kIdxHeads;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;   // independent chains
+        // four independent chains (heads = 0, 1, 2, 3 mod 4) held as two packed fp32 pairs:
+        // one f32x2 FMA per pair of heads, each half rounded as its own fmaf
+        unsigned long long a01 = 0ull, a23 = 0ull;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {          // 32 heads at a time (register budget)
           float v[32];
@@ -345,13 +347,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
           tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < 32; h += 4) {
-            s0 = fmaf(wq[32 * half + h], fmaxf(v[h], 0.f), s0);
-            s1 = fmaf(wq[32 * half + h + 1], fmaxf(v[h + 1], 0.f), s1);
-            s2 = fmaf(wq[32 * half + h + 2], fmaxf(v[h + 2], 0.f), s2);
-            s3 = fmaf(wq[32 * half + h + 3], fmaxf(v[h + 3], 0.f), s3);
+            const float2 w01 = *reinterpret_cast<const float2*>(wq + 32 * half + h);
+            const float2 w23 = *reinterpret_cast<const float2*>(wq + 32 * half + h + 2);
+            f32x2_fma(a01, f32x2_pack(w01.x, w01.y), f32x2_pack(fmaxf(v[h], 0.f), fmaxf(v[h + 1], 0.f)));
+            f32x2_fma(a23, f32x2_pack(w23.x, w23.y), f32x2_pack(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)));
           }
         }
-        const float sc = (s0 + s1) + (s2 + s3);
+        const float2 s01 = f32x2_unpack(a01), s23 = f32x2_unpack(a23);
+        const float sc = (s01.x + s01.y) + (s23.x + s23.y);
         if (i < p.N) {
           const bool valid = i < nv_q[q];
           const float val = valid ? sc * ks : -INFINITY;
