@@ -26,7 +26,7 @@
 // tile read as an MN-major operand, restricted to this CTA's D-slice of width
 // DH <= 256) accumulates in TMEM.  O is rescaled only when a tile's maximum
 // exceeds the running reference by more than 2^8, so exponentials stay <= 256.
-// With several splits (<= 8) the split CTAs of one (query, D-slice, head group)
+// With several splits (<= 16) the split CTAs of one (query, D-slice, head group)
 // are one thread-block cluster: each parks its unnormalised O and (m, l) in its
 // own shared memory, and after a cluster barrier every CTA merges a slice of the
 // heads, sink included, reading the others' shared memory (no partials in HBM,
@@ -40,6 +40,7 @@
 namespace csa {
 
 constexpr int kSwaWindow = 128;
+constexpr int kMaxSplits = 16;   // CTAs of one query's cluster (sizes above 8 are non-portable)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnParams {
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   // split partials (nsplit > 1: the CTAs of one query / D-slice / head group form a
   // cluster and merge through distributed shared memory)
   __shared__ float cl_m[Cfg::kHeadGroup], cl_l[Cfg::kHeadGroup];   // running max (log2) and sum
-  __shared__ float cl_w[Cfg::kHeadGroup][8];                       // merge weights of the <= 8 splits
+  __shared__ float cl_w[Cfg::kHeadGroup][kMaxSplits];              // merge weights of the splits
   const int qi = blockIdx.z;                 // b * T + t
   const int b = qi / p.T, t = qi % p.T;
   const int dh = blockIdx.y % Cfg::NDH;
@@ -591,38 +592,38 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     cluster_sync();                                   // every split's O and (m, l) are in place
     for (int hl = threadIdx.x; hl < he - hb; hl += blockDim.x) {
       const int hh = hb + hl;
-      float mj[8], lj[8];
+      float mj[kMaxSplits], lj[kMaxSplits];
       const float sinkL = (h0 + hh < p.H) ? p.sink[h0 + hh] * kLog2e : 0.f;
       float M = sinkL;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < kMaxSplits; ++j) {
         mj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_m[hh]), (uint32_t)j)) : -INFINITY;
         lj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_l[hh]), (uint32_t)j)) : 0.f;
         M = fmaxf(M, mj[j]);
       }
       float den = ex2_approx(sinkL - M);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < kMaxSplits; ++j) {
         mj[j] = ex2_approx(mj[j] - M);                // m = -inf (no rows) -> weight 0
         den = fmaf(lj[j], mj[j], den);
       }
       const float inv = 1.f / den;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) cl_w[hh][j] = mj[j] * inv;
+      for (int j = 0; j < kMaxSplits; ++j) cl_w[hh][j] = mj[j] * inv;
     }
     __syncthreads();
     constexpr int F = DH / 4;                         // float4 slots per head row
     const uint32_t ob = smem_u32(kv_s);
-    uint32_t peer[8];
+    uint32_t peer[kMaxSplits];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) peer[j] = cluster_map(ob, (uint32_t)(j < ns ? j : 0));
+    for (int j = 0; j < kMaxSplits; ++j) peer[j] = cluster_map(ob, (uint32_t)(j < ns ? j : 0));
     for (int it = threadIdx.x; it < (he - hb) * F; it += blockDim.x) {
       const int hh = hb + it / F, f = it % F;
       if (h0 + hh >= p.H) continue;
       const uint32_t off = (uint32_t)(hh * DH + (((f & ~7) | ((f ^ hh) & 7)) * 4)) * 4u;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < kMaxSplits; ++j) {
         if (j < ns) {
           const float4 v = ld_cluster_f4(peer[j] + off);
           const float wj = cl_w[hh][j];

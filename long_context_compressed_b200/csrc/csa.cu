@@ -190,6 +190,11 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, int smem, int clu
     if (it != cache.end()) return it->second;
   }
   if (!set_smem(kernel, smem)) return 0;
+  if (cluster_x > 8 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)cluster_x, 1, 1);
   cfg.blockDim = dim3((unsigned)threads, 1, 1);
@@ -227,7 +232,7 @@ int attn_nsplit(int B, int T, int H, int D, int64_t max_rows) {
   const int64_t tiles = (max_rows + R - 1) / R;
   const int64_t want = std::max<int64_t>(1, sms / items);
   const int64_t cap = std::max<int64_t>(1, tiles / 4);
-  return (int)std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), 8));   // <= 8: one portable cluster
+  return (int)std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), csa::kMaxSplits));   // one cluster
 }
 
 // The split partials merge inside the kernel (cluster shared memory): no workspace.
@@ -263,7 +268,11 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
       case 512: fit = max_active_clusters(csa::attn_tc_kernel<512>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit); break;
       default: break;
     }
-    if (fit >= items || fit == 0) break;   // 0: the query failed; keep the policy's choice
+    if (fit == 0 && p.nsplit > 8) {        // a non-portable size the device does not take
+      p.nsplit = 8;
+      continue;
+    }
+    if (fit >= items || fit == 0) break;   // 0: the query failed; keep the portable choice
     --p.nsplit;
   }
   grid.x = p.nsplit;
