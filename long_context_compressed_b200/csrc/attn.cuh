@@ -27,7 +27,7 @@
 // DH <= 256) accumulates in TMEM.  O is rescaled only when a tile's maximum
 // exceeds the running reference by more than 2^8, so exponentials stay <= 256.
 // With several splits (<= 16) the split CTAs of one (query, D-slice, head group)
-// are one thread-block cluster: each parks its unnormalised O and (m, l) in its
+// are one thread-block cluster: each parks its unnormalised O (bf16) and (m, l) in its
 // own shared memory, and after a cluster barrier every CTA merges a slice of the
 // heads, sink included, reading the others' shared memory (no partials in HBM,
 // no second launch).
@@ -549,13 +549,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         for (int c = 0; c < 32; ++c) o[c] = 0.f;
       }
       if (p.nsplit > 1) {
+        // raw O as bf16, 8 values per 16-byte slot, slots ^ (row & 7) within each 128 bytes
         const int row = hw0 + (int)lane_id();
+        uint8_t* orow = reinterpret_cast<uint8_t*>(obuf) + row * DH * 2;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int f = (c0 >> 2) + c;
+        for (int c = 0; c < 4; ++c) {
+          const int f = (c0 >> 3) + c;
           const int phys = (f & ~7) | ((f ^ row) & 7);
-          *reinterpret_cast<float4*>(obuf + row * DH + phys * 4) =
-              make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          uint4 u;
+          __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) hv[e] = __floats2bfloat162_rn(o[8 * c + 2 * e], o[8 * c + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(orow + phys * 16) = u;
         }
         continue;
       }
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       for (int j = 0; j < kMaxSplits; ++j) cl_w[hh][j] = mj[j] * inv;
     }
     __syncthreads();
-    constexpr int F = DH / 4;                         // float4 slots per head row
+    constexpr int F = DH / 8;                         // 16-byte slots (8 bf16) per head row
     const uint32_t ob = smem_u32(kv_s);
     uint32_t peer[kMaxSplits];
 #pragma unroll
@@ -620,25 +625,33 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     for (int it = threadIdx.x; it < (he - hb) * F; it += blockDim.x) {
       const int hh = hb + it / F, f = it % F;
       if (h0 + hh >= p.H) continue;
-      const uint32_t off = (uint32_t)(hh * DH + (((f & ~7) | ((f ^ hh) & 7)) * 4)) * 4u;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const uint32_t off = (uint32_t)(hh * DH * 2 + (((f & ~7) | ((f ^ hh) & 7)) * 16));
+      uint4 v[kMaxSplits];
+#pragma unroll
+      for (int j = 0; j < kMaxSplits; ++j)
+        if (j < ns) v[j] = ld_cluster_u4(peer[j] + off);
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
         if (j < ns) {
-          const float4 v = ld_cluster_f4(peer[j] + off);
           const float wj = cl_w[hh][j];
-          acc.x = fmaf(wj, v.x, acc.x);
-          acc.y = fmaf(wj, v.y, acc.y);
-          acc.z = fmaf(wj, v.z, acc.z);
-          acc.w = fmaf(wj, v.w, acc.w);
+          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(hv[e]);
+            acc[2 * e] = fmaf(wj, x.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wj, x.y, acc[2 * e + 1]);
+          }
         }
       }
-      __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y), bb = __floats2bfloat162_rn(acc.z, acc.w);
-      uint2 u;
-      u.x = *reinterpret_cast<uint32_t*>(&a);
-      u.y = *reinterpret_cast<uint32_t*>(&bb);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hh) * D + dh * DH +
-                                f * 4) = u;
+      uint4 u;
+      __nv_bfloat162* ho = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ho[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hh) * D + dh * DH +
+                                f * 8) = u;
     }
     cluster_sync();                                   // no CTA leaves while its shared memory is read
   }
