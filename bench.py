@@ -129,14 +129,15 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes (read + write) per indexer launch from the committed ncu summary, or None
-    when the indexer source has changed since that capture (the summary records a hash)."""
+def profiled_traffic(profile: str, source: str, workload: str):
+    """DRAM bytes (read + write) per launch of one kernel on one workload, from the committed
+    ncu summary `profiles/<profile>`, or None when the kernel's source file `csrc/<source>` has
+    changed since that capture (the summary records a hash of it)."""
     import hashlib
     import re
     try:
-        text = open(os.path.join(ROOT, "profiles", "index_tc_kernel_e4m3_decode.md")).read()
-        src = open(os.path.join(ROOT, "long_context_compressed_b200", "csrc", "index.cuh"), "rb").read()
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        src = open(os.path.join(ROOT, "long_context_compressed_b200", "csrc", source), "rb").read()
     except OSError:
         return None
     m = re.search(r"^traffic_bytes_per_launch: (.*)$", text, re.M)
@@ -939,7 +940,8 @@ def main():
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (sparse_attn: top-k + SWA rows, cluster merge)",
                          "achieved": attn_gbs, "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak,
-                         "peak_source": peak_kind + " (burst copy; the kernel is timed alone)", "traffic": None,
+                         "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
+                         "traffic": profiled_traffic("attn_tc_kernel_decode_prefill_hca.md", "attn.cuh", wl.name),
                          "bytes_per_launch": r["attn_bytes"], "avg_launch_us": r["attn_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays",
@@ -949,7 +951,8 @@ def main():
                          else "index_tc_kernel (csa_index_scores, bf16)",
                          "achieved": idx_gbs, "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak,
                          "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
-                         "traffic": profiled_traffic(wl.name) if args.index == "e4m3" else None,
+                         "traffic": profiled_traffic("index_tc_kernel_e4m3_decode.md", "index.cuh", wl.name)
+                         if args.index == "e4m3" else None,
                          "bytes_per_launch": r["index_bytes"], "avg_launch_us": r["index_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays"},

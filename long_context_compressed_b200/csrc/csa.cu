@@ -223,15 +223,17 @@ int attn_rows_per_tile() { return AttnCfg<D>::R; }
 int attn_ndh(int D) { return D > 256 ? D / 256 : 1; }
 
 // CTAs per (query, D-slice, head group) over the row list: one wave of CTAs, at
-// least four KV tiles each
-int attn_nsplit(int B, int T, int H, int D, int64_t max_rows) {
+// least two KV tiles each for sparse_attn (gathered rows: the more SMs issue the
+// gathers, the sooner the rows are in) and four for hca_attn (contiguous rows by TMA,
+// and it shares the GPU with the chain of the CSA layer)
+int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse) {
   const int64_t items = (int64_t)B * T * attn_ndh(D) * ((H + 63) / 64);
   const int sms = sm_count();
   if (items <= 0 || items >= 2 * sms) return 1;
   const int R = D >= 512 ? 32 : 64;
   const int64_t tiles = (max_rows + R - 1) / R;
   const int64_t want = std::max<int64_t>(1, sms / items);
-  const int64_t cap = std::max<int64_t>(1, tiles / 4);
+  const int64_t cap = std::max<int64_t>(1, tiles / (sparse ? 2 : 4));
   return (int)std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), csa::kMaxSplits));   // one cluster
 }
 
@@ -252,7 +254,7 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     }
     return launch_status();
   }
-  p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows);
+  p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows, p.sparse != 0);
   (void)ws;
   (void)ws_bytes;
   // grid: (splits of the row list, D-slice x head group of 64, query)
