@@ -605,7 +605,8 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
   const int phase3 = csa::kSelTileBytes + csa::kSelQBytes + chunk * 8 + 64 * 4 +
                      (rescore && !tc ? (64 * 129 + csa::kSelKeyBatch * 128) * 4 : 0);
   // last CTA: staged candidates + chunk table, or (overflow) the bucketed selection
-  const int phase4 = (int)std::max<int64_t>(2 * csa::kSelCandSmem * 4 + 2 * csa::kSelMaxChunks * 4,
+  const int phase4 = (int)std::max<int64_t>(2 * csa::kSelCandSmem * 4 + 2 * csa::kSelMaxChunks * 4 +
+                                                csa::kSelPivot * 4,
                                             2 * CSA_MAX_TOPK * 4 + (nchunks + 1) * 4);
   const int smem = 1024 + std::max(phase3, phase4);
   cudaStream_t st = as_stream(stream);

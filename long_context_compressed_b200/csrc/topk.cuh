@@ -477,6 +477,8 @@ constexpr int kSelPerThread = 4;     // scores each thread loads per pass of the
 constexpr int kSelTcRows = 128;      // candidates rescored per tensor-core batch (bf16)
 constexpr int kSelKeyBatch = 64;     // candidate key rows per SIMT batch (fp32)
 constexpr int kSelCandSmem = 8192;   // candidates the last CTA stages in shared memory
+// keys the last CTA ranks directly once a radix digit has narrowed the k-th key to one bin
+constexpr int kSelPivot = 256;
 constexpr int kSelPrefetch = 2048;   // chunk entries whose scores are fetched with the histogram
 constexpr int kSelMaxChunkLen = 16384;  // entries per chunk (shared-memory candidate list)
 static_assert(kSelPerThread * (kSelThreads / 32) == 32, "one scan lane per (pass, warp)");
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   __shared__ __align__(16) int histk[kHistBins + kHistBins / 32];   // skewed
   __shared__ int scratch[33];
   __shared__ int res[2];
-  __shared__ int lcount, gslot, is_last;
+  __shared__ int lcount, gslot, is_last, pcount;
   __shared__ int wcnt[32], wexc[33];
   __shared__ uint32_t kext[2];
   __shared__ uint64_t mma_bar;
@@ -900,9 +902,14 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
       const uint32_t dmask = (1u << (hi - lo)) - 1;
       for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) histk[j] = 0;
       __syncthreads();
-      for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-        const uint32_t u = okey[i] - kmin;
-        if ((u & pmask) == prefix) atomicAdd(&histk[skew((int)((u >> lo) & dmask))], 1);
+      for (int i0 = threadIdx.x; i0 < nc; i0 += 4 * kSelThreads) {   // 4 keys requested at once
+        uint32_t uu[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) uu[q] = i0 + q * kSelThreads < nc ? okey[i0 + q * kSelThreads] - kmin : 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (i0 + q * kSelThreads < nc && (uu[q] & pmask) == prefix)
+            atomicAdd(&histk[skew((int)((uu[q] >> lo) & dmask))], 1);
       }
       __syncthreads();
       find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, remaining, res, scratch);
@@ -911,6 +918,55 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
       pmask |= dmask << lo;
       remaining -= res[1];
       hi = lo;
+      // When the chosen bin holds few keys (the usual case after the first digit), rank
+      // them directly: the k-th key K* is the key with fewer than `remaining` keys above
+      // it and at least `remaining` at or above it, among the keys of the bin.
+      const int nb = histk[skew(res[0])];
+      if (hi > 0 && nb <= kSelPivot) {
+        uint32_t* piv = reinterpret_cast<uint32_t*>(tpre + kSelMaxChunks);   // [kSelPivot]
+        if (threadIdx.x == 0) pcount = 0;
+        __syncthreads();
+        const uint32_t below = (1u << lane_id()) - 1;
+        for (int i0 = 0; i0 < nc; i0 += kSelThreads) {      // one slot claim per warp
+          const int i = i0 + threadIdx.x;
+          const uint32_t u = i < nc ? okey[i] - kmin : 0u;
+          const bool m = i < nc && (u & pmask) == prefix;
+          const uint32_t bal = __ballot_sync(0xffffffffu, m);
+          int base = 0;
+          if (lane_id() == 0 && bal) base = atomicAdd(&pcount, __popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (m) piv[base + __popc(bal & below)] = u;
+        }
+        __syncthreads();
+        if ((int)threadIdx.x < nb) {
+          const uint32_t v = piv[threadIdx.x];
+          int gt = 0, ge = 0;
+          int j = 0;
+          for (; j + 16 <= nb; j += 16) {                    // 16 keys requested at once
+            uint4 x[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) x[q] = *reinterpret_cast<const uint4*>(piv + j + 4 * q);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              gt += (x[q].x > v) + (x[q].y > v) + (x[q].z > v) + (x[q].w > v);
+              ge += (x[q].x >= v) + (x[q].y >= v) + (x[q].z >= v) + (x[q].w >= v);
+            }
+          }
+          for (; j < nb; ++j) {
+            gt += piv[j] > v;
+            ge += piv[j] >= v;
+          }
+          if (gt < remaining && remaining <= ge) {       // every key equal to K* writes the same
+            res[0] = (int)v;
+            res[1] = gt;
+          }
+        }
+        __syncthreads();
+        prefix = (uint32_t)res[0];
+        pmask = 0xffffffffu;
+        remaining -= res[1];
+        break;
+      }
     }
     // ordered emit: every key above K*, and the first `remaining` keys equal to K* (the
     // staged order is index order); each thread walks a contiguous run of odd length
@@ -919,23 +975,38 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     const int p0 = (int)threadIdx.x * per;
     const int p1 = p0 + per < nc ? p0 + per : nc;
     int cg = 0, ce = 0;
-    for (int i = p0; i < p1; ++i) {
-      const uint32_t u = okey[i] - kmin;
-      cg += u > prefix;
-      ce += u == prefix;
+    for (int i0 = p0; i0 < p1; i0 += 4) {                 // 4 keys requested at once
+      uint32_t uu[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) uu[q] = i0 + q < p1 ? okey[i0 + q] - kmin : 0u;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        cg += i0 + q < p1 && uu[q] > prefix;
+        ce += i0 + q < p1 && uu[q] == prefix;
+      }
     }
     int total;
     const int ex = block_excl_scan((cg << 16) | ce, scratch, &total);
     int g = ex >> 16, e = ex & 0xffff;
-    for (int i = p0; i < p1; ++i) {
-      const uint32_t u = okey[i] - kmin;
-      if (u > prefix) {
-        const int o = g + (e < remaining ? e : remaining);
-        if (o < k) out[o] = oidx[i];                     // (bound holds unless the histogram is stale)
-        ++g;
-      } else if (u == prefix) {
-        if (e < remaining && g + e < k) out[g + e] = oidx[i];
-        ++e;
+    for (int i0 = p0; i0 < p1; i0 += 4) {
+      uint32_t uu[4];
+      int32_t ii[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uu[q] = i0 + q < p1 ? okey[i0 + q] - kmin : 0u;
+        ii[q] = i0 + q < p1 ? oidx[i0 + q] : 0;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (i0 + q >= p1) break;
+        if (uu[q] > prefix) {
+          const int o = g + (e < remaining ? e : remaining);
+          if (o < k) out[o] = ii[q];                       // (bound holds unless the histogram is stale)
+          ++g;
+        } else if (uu[q] == prefix) {
+          if (e < remaining && g + e < k) out[g + e] = ii[q];
+          ++e;
+        }
       }
     }
     __syncthreads();
