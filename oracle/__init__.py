@@ -17,8 +17,8 @@ cited in ``oracle.c``:
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
 (tests/test_oracle_pins.py) except the FP8 *recall* statistic, which the pages
-do not fix ("parity unpinned" for recall only; the e4m3 codec and the FP8
-score definition are pinned).
+do not fix ("parity unpinned" for recall only; the e4m3 codec, the FP8 score
+definition and the mixed-precision KV storage codec are pinned).
 """
 from __future__ import annotations
 
@@ -69,13 +69,18 @@ def _load():
     lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_quantize_rows_e4m3.argtypes = [_f32p, i64, i32, _u8p, _f32p]
+    lib.oracle_kv8_entry_bytes.argtypes = [i32]
+    lib.oracle_kv8_entry_bytes.restype = i64
+    lib.oracle_kv8_quantize.argtypes = [_f32p, i64, i32, _u8p]
+    lib.oracle_kv8_dequantize.argtypes = [_u8p, i64, i32, _f32p]
     lib.oracle_topk.argtypes = [_f32p, _i32p, i32, i64, i32, _i32p]
     lib.oracle_sparse_attn.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _f32p, _i32p, i32, dbl, i32,
                                        i32, i32, i32, i64, _f64p, _f64p]
     lib.oracle_hca_attn.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _f32p, i32, dbl, i32,
                                     i32, i32, i32, i64, _f64p, _f64p]
     for name in ("oracle_compress_csa", "oracle_compress_hca", "oracle_index_scores",
-                 "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_topk",
+                 "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_kv8_quantize",
+                 "oracle_kv8_dequantize", "oracle_topk",
                  "oracle_sparse_attn", "oracle_hca_attn"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -212,6 +217,35 @@ def quantize_rows_e4m3(x):
     scale = np.empty(x.shape[:-1], np.float32)
     _check(lib.oracle_quantize_rows_e4m3(x, rows, cols, codes, scale), "quantize_rows_e4m3")
     return codes, scale
+
+
+def kv8_entry_bytes(D: int) -> int:
+    """Bytes of one mixed-precision compressed entry (FP8 dims, BF16 RoPE dims, scales)."""
+    return int(_load().oracle_kv8_entry_bytes(int(D)))
+
+
+def kv8_quantize(kv):
+    """Mixed-precision storage of compressed entries ([HA] §4.2 storage precision):
+    kv [..., D] (BF16 values) -> entries [..., kv8_entry_bytes(D)] uint8."""
+    lib = _load()
+    x = _f32(kv)
+    D = x.shape[-1]
+    rows = x.size // D
+    out = np.empty(x.shape[:-1] + (kv8_entry_bytes(D),), np.uint8)
+    _check(lib.oracle_kv8_quantize(x, rows, D, out), "kv8_quantize")
+    return out
+
+
+def kv8_dequantize(entries, D: int):
+    """entries [..., kv8_entry_bytes(D)] uint8 -> kv [..., D] float32 (exact values)."""
+    lib = _load()
+    e = np.ascontiguousarray(np.asarray(entries, np.uint8))
+    eb = kv8_entry_bytes(D)
+    assert e.shape[-1] == eb
+    rows = e.size // eb
+    out = np.empty(e.shape[:-1] + (D,), np.float32)
+    _check(lib.oracle_kv8_dequantize(e, rows, D, out), "kv8_dequantize")
+    return out
 
 
 # --------------------------------------------------------------------------- top-k

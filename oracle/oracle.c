@@ -238,6 +238,90 @@ int oracle_quantize_rows_e4m3(const float *x, int64_t rows, int cols, uint8_t *c
     return ORC_OK;
 }
 
+/* ---- Mixed-precision storage of the compressed KV entries ([HA] §4.2, the
+ * paragraph on storage precision: the RoPE dims stay BF16, the rest of each
+ * compressed entry is FP8).  Readings (the pages give no granularity or layout):
+ *   - the RoPE dims are the last 64 of D; the first D-64 dims are e4m3 codes;
+ *   - one scale per block of 64 FP8 dims, a power of two s = 2^e with e the
+ *     smallest integer such that amax <= 448 * 2^e (an all-zero block: e = 0), so
+ *     x / s is exact and code * s is exactly representable in BF16;
+ *   - code = e4m3(x / s), nearest value, ties to the even mantissa;
+ *   - entry bytes: [D-64 codes][64 BF16 RoPE dims][(D-64)/64 fp32 scales], zero
+ *     padding to a multiple of 16 bytes (608 bytes for D = 512).
+ * kv holds BF16 values widened exactly to float. */
+int64_t oracle_kv8_entry_bytes(int D)
+{
+    int64_t b = (int64_t)(D - 64) + 128 + 4 * (int64_t)((D - 64) / 64);
+    return (b + 15) / 16 * 16;
+}
+
+static uint16_t orc_bf16_bits(float x)      /* x is a BF16 value widened exactly */
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    return (uint16_t)(u >> 16);
+}
+
+int oracle_kv8_quantize(const float *kv, int64_t rows, int D, uint8_t *entries)
+{
+    if (D < 128 || D % 64 != 0) return ORC_BAD;
+    const int nf = D - 64, nb = nf / 64;
+    const int64_t eb = oracle_kv8_entry_bytes(D);
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *x = kv + r * D;
+        uint8_t *e = entries + r * eb;
+        memset(e, 0, (size_t)eb);
+        for (int blk = 0; blk < nb; ++blk) {
+            double amax = 0.0;
+            for (int j = 0; j < 64; ++j) {
+                double a = fabs((double)x[blk * 64 + j]);
+                if (a > amax) amax = a;
+            }
+            int ex = 0;
+            if (amax > 0.0) {
+                ex = (int)ceil(log2(amax / 448.0));
+                while (ldexp(448.0, ex) < amax) ++ex;          /* smallest e with amax <= 448 * 2^e */
+                while (ldexp(448.0, ex - 1) >= amax) --ex;
+            }
+            const double sc = ldexp(1.0, ex);
+            for (int j = 0; j < 64; ++j)
+                e[blk * 64 + j] = oracle_e4m3_encode((float)((double)x[blk * 64 + j] / sc));
+            const float fs = (float)sc;
+            memcpy(e + nf + 128 + 4 * blk, &fs, 4);
+        }
+        for (int j = 0; j < 64; ++j) {
+            uint16_t h = orc_bf16_bits(x[nf + j]);
+            memcpy(e + nf + 2 * j, &h, 2);
+        }
+    }
+    return ORC_OK;
+}
+
+/* Inverse of the storage above: x = code * s for the FP8 dims, the BF16 bits for
+ * the RoPE dims.  Every value is exact in float. */
+int oracle_kv8_dequantize(const uint8_t *entries, int64_t rows, int D, float *kv)
+{
+    if (D < 128 || D % 64 != 0) return ORC_BAD;
+    const int nf = D - 64;
+    const int64_t eb = oracle_kv8_entry_bytes(D);
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint8_t *e = entries + r * eb;
+        float *x = kv + r * D;
+        for (int j = 0; j < nf; ++j) {
+            float fs;
+            memcpy(&fs, e + nf + 128 + 4 * (j / 64), 4);
+            x[j] = (float)(oracle_e4m3_decode(e[j]) * (double)fs);
+        }
+        for (int j = 0; j < 64; ++j) {
+            uint16_t h;
+            memcpy(&h, e + nf + 2 * j, 2);
+            uint32_t u = (uint32_t)h << 16;
+            memcpy(&x[nf + j], &u, 4);
+        }
+    }
+    return ORC_OK;
+}
+
 /* [HA] §4.2 on dequantised e4m3 inputs: q = code * q_scale[t,h],
  * k = code * k_scale[i]; the score is the plain definition on those values. */
 int oracle_index_scores_e4m3(const uint8_t *q8, const float *q_scale, const float *w,

@@ -469,3 +469,102 @@ def test_generator_moments_and_independence():
     assert 0 <= u.min().item() and u.max().item() < 1 and abs(u.mean().item() - 0.5) < 0.01
     # order-independence: drawing a prefix gives the same values
     assert torch.equal(synth.normal(3, "p", (10,)), synth.normal(3, "p", (1000,))[:10])
+
+
+# ----------------------------------------------------------------------------- mixed-precision KV storage
+def _bf16(x):
+    return torch.tensor(np.asarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def test_kv8_worked_block_and_layout():
+    """[HA] §4.2 storage precision, on D = 128 (one FP8 block of 64 dims + 64 BF16 RoPE dims).
+
+    Hand-derived expectations:
+      - amax = 448 gives the scale 2^0 = 1.  Codes: 448 = 1.75 * 2^8 -> 0 1111 110 = 0x7E;
+        -1.0 = 2^0 -> 1 0111 000 = 0xB8; 0.5 = 2^-1 -> 0 0110 000 = 0x30;
+        3.0 = 1.5 * 2^1 -> 0 1000 100 = 0x44; 0 -> 0x00.
+      - amax = 452 (a BF16 value) needs 2^1: 452 / 2 = 226 lies between 224 (0x76) and
+        240 (0x77), so the code is 0x76, which decodes back to 448.
+      - amax = 2^-10 (0.0009765625) gives e = ceil(log2(2^-10 / 448)) = -18: 448 * 2^-18 >= 2^-10
+        and 448 * 2^-19 < 2^-10.  Then 2^-10 / 2^-18 = 256 = 2^8 -> 0 1111 000 = 0x78.
+      - Layout: 64 codes, then 64 BF16 RoPE values, then one fp32 scale, zero padding to 208 bytes.
+    """
+    assert oracle.kv8_entry_bytes(128) == 208
+    assert oracle.kv8_entry_bytes(512) == 608
+    rope = _bf16(np.linspace(-3, 3, 64))
+    x = np.zeros((3, 128), np.float32)
+    x[0, :5] = [448.0, -1.0, 0.5, 3.0, 0.0]
+    x[1, 0] = 452.0
+    x[2, 7] = 2.0 ** -10
+    x[:, 64:] = rope
+    e = oracle.kv8_quantize(x)
+    assert e.shape == (3, 208)
+    assert list(e[0, :5]) == [0x7E, 0xB8, 0x30, 0x44, 0x00]
+    assert np.all(e[0, 5:64] == 0)
+    assert e[0, 64:192].view(np.uint16).tolist() == (rope.view(np.uint32) >> 16).astype(np.uint16).tolist()
+    scales = [float(e[r, 192:196].view(np.float32)[0]) for r in range(3)]
+    assert scales == [1.0, 2.0, 2.0 ** -18]
+    assert np.all(e[:, 196:] == 0)
+    assert e[1, 0] == 0x76 and e[2, 7] == 0x78
+    y = oracle.kv8_dequantize(e, 128)
+    assert y[0, :5].tolist() == [448.0, -1.0, 0.5, 3.0, 0.0]
+    assert y[1, 0] == 448.0 and y[2, 7] == 2.0 ** -10
+    np.testing.assert_array_equal(y[:, 64:], x[:, 64:])
+
+
+def test_kv8_scale_is_the_smallest_power_of_two():
+    """s = 2^e with amax <= 448 s < 2 amax (e minimal), per block of 64 dims; zero block -> 1."""
+    D = 512
+    mags = [1e-6, 3e-3, 0.7, 1.0, 5.0, 448.0, 449.0, 3e4]
+    x = np.zeros((len(mags) + 1, D), np.float32)
+    for r, mg in enumerate(mags):
+        x[r] = _bf16(rnd(D) * mg)
+    x[-1, :448] = 0.0                                    # all FP8 blocks zero
+    e = oracle.kv8_quantize(x)
+    for r in range(x.shape[0]):
+        sc = e[r, 448 + 128:448 + 128 + 28].view(np.float32)
+        for blk in range(7):
+            s = float(sc[blk])
+            m, ex = math.frexp(s)
+            assert m == 0.5, (r, blk, s)                 # a power of two
+            amax = float(np.abs(x[r, blk * 64:(blk + 1) * 64]).max())
+            if amax == 0.0:
+                assert s == 1.0
+            else:
+                assert amax <= 448.0 * s and amax > 224.0 * s, (r, blk, amax, s)
+
+
+def test_kv8_exact_roundtrip_of_every_code():
+    """Values code * s for every finite e4m3 code come back with the same code."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    for s in (2.0 ** -12, 1.0, 2.0 ** 5):
+        x = np.zeros((len(codes), 128), np.float32)
+        x[:, 0] = (vals * s).astype(np.float32)
+        x[:, 1] = 448.0 * s                                # pins the block's scale to s
+        e = oracle.kv8_quantize(x)
+        np.testing.assert_array_equal(e[:, 0], codes)
+        assert np.all(e[:, 192:196].view(np.float32) == np.float32(s))
+        y = oracle.kv8_dequantize(e, 128)
+        np.testing.assert_array_equal(y[:, 0], x[:, 0])
+
+
+def test_kv8_error_bound_and_block_independence():
+    """|x - x'| <= max(|x| 2^-4, s 2^-10) (half an e4m3 step); blocks quantise independently;
+    the RoPE dims are bit-exact."""
+    D = 512
+    x = _bf16(rnd(64, D) * np.exp(rnd(64, 1) * 2))
+    e = oracle.kv8_quantize(x)
+    y = oracle.kv8_dequantize(e, D)
+    sc = e[:, 576:604].view(np.float32)                  # [64, 7]
+    s_full = np.repeat(sc, 64, axis=1)
+    err = np.abs(x[:, :448].astype(np.float64) - y[:, :448])
+    bound = np.maximum(np.abs(x[:, :448]) * 2.0 ** -4, s_full * 2.0 ** -10)
+    assert np.all(err <= bound * (1 + 1e-12))
+    np.testing.assert_array_equal(y[:, 448:], x[:, 448:])
+    x2 = x.copy()
+    x2[:, 64:128] *= 16.0                                # change block 1 only
+    e2 = oracle.kv8_quantize(x2)
+    np.testing.assert_array_equal(e2[:, :64], e[:, :64])
+    np.testing.assert_array_equal(e2[:, 128:448], e[:, 128:448])
+    assert np.all(e2[:, 580:584].view(np.float32) == e[:, 580:584].view(np.float32) * 16)
