@@ -20,7 +20,8 @@
  *   - Kernels never wait without bound: a wait that runs out records
  *     CSA_ERR_TIMEOUT in a device status word that csa_poll_status() returns.
  *   - dtype codes: CSA_F32 (fp32), CSA_BF16 (bfloat16), CSA_E4M3 (OCP FP8 e4m3,
- *     one byte per element).
+ *     one byte per element), CSA_BF16_KV8 (attention only: bf16 q / swa_kv / out,
+ *     memory rows kv stored as mixed-precision entries, see csa_quantize_kv8).
  */
 #ifndef CSA_H_
 #define CSA_H_
@@ -40,7 +41,7 @@ enum {
   CSA_ERR_TIMEOUT = 4      /* a kernel gave up a bounded wait (see csa_poll_status) */
 };
 
-enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2 };
+enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2, CSA_BF16_KV8 = 3 };
 
 #define CSA_INDEX_HEADS 64   /* index heads per query ([HA] §2 table, §4.2) */
 #define CSA_INDEX_DIM 128    /* dims per index head */
@@ -199,6 +200,26 @@ int csa_topk_select(const float *scores, const int32_t *n_valid, int B, int64_t 
                     void *stream);
 
 /*
+ * csa_quantize_kv8 -- mixed-precision storage of compressed KV entries ([HA] §4.2,
+ * storage precision: the RoPE dims stay BF16, the rest of each compressed entry
+ * is FP8).  D = 512 only; the last 64 dims are the RoPE dims.
+ *   kv      : [rows, 512] bf16 (device), 16-byte aligned
+ *   entries : [rows, csa_kv8_entry_bytes(512) = 608] bytes (device), 16-byte aligned:
+ *             bytes [0, 448)   e4m3 codes of dims 0..447,
+ *                   [448, 576) bf16 dims 448..511 (bit copy),
+ *                   [576, 604) seven fp32 block scales s = 2^e (block = 64 dims), e the
+ *                              smallest integer with max|x| <= 448 * 2^e (0 for a zero block),
+ *                   [604, 608) zero.
+ *             code = e4m3 of x / s, nearest, ties to even (x / s is exact), so code * s is
+ *             exactly a bf16 value.
+ *   CSA_ERR_UNSUPPORTED for D != 512; CSA_ERR_INVALID for null or misaligned pointers.
+ * Such entries are the kv argument of sparse_attn / hca_attn with dtype CSA_BF16_KV8,
+ * which attend over the dequantised rows (code * s, and the bf16 dims as stored).
+ */
+long long csa_kv8_entry_bytes(int D);
+int csa_quantize_kv8(const void *kv, int64_t rows, int D, void *entries, void *stream);
+
+/*
  * sparse_attn -- CSA core attention ([P2] sparse_attn(q, kv, attn_sink,
  * topk_idxs, softmax_scale); [HA] §4.2 Shared-KV MQA, §6 SWA + sink, §7 call chain):
  *   for query (b,t) at absolute position pos = q_pos[b,t] and head h:
@@ -212,10 +233,11 @@ int csa_topk_select(const float *scores, const int32_t *n_valid, int B, int64_t 
  *   swa_pos0 : [B] int64;  q_pos : [B, T] int64;  sink : [H] fp32 (unscaled logit)
  *   idx    : [B, T, k] int32;  out : [B, T, H, D] dtype
  *   dtype CSA_BF16 (tcgen05, fp32 softmax and accumulation; H <= 128,
- *   D in {128, 256, 512}) or CSA_F32 (fp32 FMA; D multiple of 32, <= 512).
+ *   D in {128, 256, 512}), CSA_BF16_KV8 (as CSA_BF16 with kv [B, N, 608] bytes of
+ *   csa_quantize_kv8 entries; D = 512) or CSA_F32 (fp32 FMA; D multiple of 32, <= 512).
  *   workspace : csa_attn_workspace_size(...) bytes; may be NULL when that size
  *               is 0, which it is in this version: the row list of a query is
- *               split over up to 8 CTAs that form one thread-block cluster and
+ *               split over up to 16 CTAs that form one thread-block cluster and
  *               merge their partial results in distributed shared memory.
  */
 size_t csa_attn_workspace_size(int B, int T, int H, int D, int64_t rows_per_query, int dtype);

@@ -22,7 +22,8 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 CSA_OK, CSA_ERR_INVALID, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA, CSA_ERR_TIMEOUT = range(5)
-CSA_F32, CSA_BF16, CSA_E4M3 = 0, 1, 2
+CSA_F32, CSA_BF16, CSA_E4M3, CSA_BF16_KV8 = 0, 1, 2, 3
+KV8_DIMS, KV8_BYTES = 512, 608   # mixed-precision compressed entry: 448 e4m3 dims, 64 bf16 RoPE dims, 7 scales
 INDEX_HEADS, INDEX_DIM, SWA_WINDOW, MAX_TOPK = 64, 128, 128, 2048
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -32,6 +33,8 @@ _SIGS = {
     "csa_version": ([], _i32),
     "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
+    "csa_kv8_entry_bytes": ([_i32], ctypes.c_longlong),
+    "csa_quantize_kv8": ([_vp, _i64, _i32, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
     "csa_select_workspace_size": ([_i32, _i64], _sz),
     "csa_score_histogram": ([_vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
@@ -235,13 +238,33 @@ def attn_workspace(B, T, H, D, rows_per_query, dtype=CSA_BF16, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
+def quantize_kv8(kv, entries=None, stream=None):
+    """Mixed-precision storage of compressed entries (FP8 dims, BF16 RoPE dims):
+    kv [..., 512] bf16 -> entries [..., 608] uint8 (layout in include/csa.h)."""
+    assert kv.dtype == torch.bfloat16 and kv.shape[-1] == KV8_DIMS
+    kv = kv.contiguous()
+    rows = kv.numel() // KV8_DIMS
+    if entries is None:
+        entries = torch.empty(kv.shape[:-1] + (KV8_BYTES,), dtype=torch.uint8, device=kv.device)
+    _check(_lib.csa_quantize_kv8(_ptr(kv), rows, KV8_DIMS, _ptr(entries), _stream(stream)), "csa_quantize_kv8")
+    return entries
+
+
+def _attn_dtype(q, kv) -> int:
+    # uint8 kv of 608-byte rows: quantize_kv8 entries (bf16 q, swa_kv and out)
+    if kv.dtype == torch.uint8:
+        assert q.dtype == torch.bfloat16 and kv.shape[-1] == KV8_BYTES
+        return CSA_BF16_KV8
+    return _dtype_code(q)
+
+
 def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale: float, *, out=None, workspace=None,
                 stream=None):
-    """CSA core attention.  q [B,T,H,D], kv [B,N,D], swa_kv [B,W,D], swa_pos0 [B] int64, q_pos [B,T] int64,
-    sink [H] fp32, idx [B,T,k] int32 -> out [B,T,H,D]."""
+    """CSA core attention.  q [B,T,H,D], kv [B,N,D] (or [B,N,608] uint8 quantize_kv8 entries), swa_kv [B,W,D],
+    swa_pos0 [B] int64, q_pos [B,T] int64, sink [H] fp32, idx [B,T,k] int32 -> out [B,T,H,D]."""
     B, T, H, D = q.shape
     N, W, k = kv.shape[1], swa_kv.shape[1], idx.shape[2]
-    dt = _dtype_code(q)
+    dt = _attn_dtype(q, kv)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
@@ -257,7 +280,7 @@ def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int =
     """HCA core attention: dense over kv[b, :min(N, (pos+1)//ratio)] plus the SWA rows."""
     B, T, H, D = q.shape
     N, W = kv.shape[1], swa_kv.shape[1]
-    dt = _dtype_code(q)
+    dt = _attn_dtype(q, kv)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:

@@ -35,6 +35,7 @@
 // attn_f32_kernel: fp32 SIMT (one warp per head), exact online softmax.
 #pragma once
 #include <cuda_bf16.h>
+#include "kv8.cuh"
 #include "ptx.cuh"
 
 namespace csa {
@@ -189,7 +190,12 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
 // (head group blockIdx.y / NDH).  The M = 128 MMA operand of atom a also spans the first 64
 // rows of atom a+1 (or, for the last atom, the next 8 KB of shared memory):
 // finite values whose result rows (>= H) are never used.
-template <int D>
+// KV8: memory rows are csa_quantize_kv8 entries (FP8 dims + BF16 RoPE dims, D = 512);
+// the loader warps stage each 608-byte entry at the tail of its tile's buffer by
+// cp.async and convert it to the bf16 tile (exact: code * 2^e is a bf16 value) before
+// the MMA reads it.  The memory rows then start at a tile boundary of the row list
+// (the SWA rows are padded with masked rows), so a tile is all SWA or all memory.
+template <int D, bool KV8>
 __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                            const __grid_constant__ CUtensorMap kvmap,
                                                                            const __grid_constant__ CUtensorMap swamap,
@@ -254,7 +260,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   const uint32_t tmem = *tmem_holder;
   griddep_sync();
   const RowList rl = make_row_list(p, b, t);
-  const int n_rows = rl.n_swa + rl.n_mem;
+  const int mem0 = KV8 ? (rl.n_swa + R - 1) / R * R : rl.n_swa;   // list row of the first memory row
+  const int n_rows = mem0 + rl.n_mem;
   const int n_tiles_all = (n_rows + R - 1) / R;
   // balanced tile ranges: the splits' tile counts differ by at most one
   const int j0 = (int)((int64_t)split * n_tiles_all / p.nsplit);
@@ -262,17 +269,19 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   const int nt = j1 > j0 ? j1 - j0 : 0;      // tiles of this CTA
   // the index value behind list row rg (only memory rows of sparse_attn read memory)
   auto fetch_raw = [&](int rg) -> int32_t {
-    if (!p.sparse || rg < rl.n_swa || rg >= n_rows) return 0;
-    return __ldg(idx_row + (rg - rl.n_swa));
+    if (!p.sparse || rg < mem0 || rg >= n_rows) return 0;
+    return __ldg(idx_row + (rg - mem0));
   };
   // element offset of list row rg given its raw index; -1 if it contributes nothing;
   // SWA rows are encoded as -2 - offset
+  // (KV8: offset in entries, i.e. the memory row's entry number)
   auto row_src = [&](int rg, int32_t raw) -> int64_t {
     if (rg >= n_rows) return -1;
     if (rg < rl.n_swa) return -2 - ((int64_t)b * p.W + rl.swa_row0 + rg) * D;
-    const int64_t i = p.sparse ? (int64_t)raw : (int64_t)(rg - rl.n_swa);
+    if (rg < mem0) return -1;                        // padding between the SWA and memory rows
+    const int64_t i = p.sparse ? (int64_t)raw : (int64_t)(rg - mem0);
     if (i < 0 || i >= p.N) return -1;
-    return ((int64_t)b * p.N + i) * D;
+    return KV8 ? (int64_t)b * p.N + i : ((int64_t)b * p.N + i) * D;
   };
 
 
@@ -297,58 +306,177 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       if (staged) {
         for (int r = lt; r < nrow; r += 128) {
           const int rg = row0 + r;
-          idx_s[r] = (rg >= rl.n_swa && rg < n_rows) ? __ldg(idx_row + (rg - rl.n_swa)) : 0;
+          idx_s[r] = (rg >= mem0 && rg < n_rows) ? __ldg(idx_row + (rg - mem0)) : 0;
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
-      int ks = 0;
-      uint32_t kph = 0;
-      for (int jj = 0; jj < nt; ++jj) {
-        const int rg0 = (j0 + jj) * R;
-        const int rg = rg0 + my_r;
-        const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
-        const int s = ks;
-        const uint32_t ph = kph;
-        if (++ks == NS) { ks = 0; kph ^= 1; }
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        uint8_t* tile = kv_s + s * Cfg::kKVBytes;
-        // R consecutive rows of one buffer (SWA rows, or hca_attn's dense memory rows):
-        // one TMA box per 64-dim atom, same 128-byte-swizzled layout as the gather
-        const bool swa_tile = p.has_swamap && rg0 + R <= rl.n_swa;
-        const bool mem_tile = p.has_kvmap && !p.sparse && rg0 >= rl.n_swa && rg0 + R <= n_rows;
-        const __nv_bfloat16* src = nullptr;
-        if (swa_tile || mem_tile) {
-          src = kv;                                   // every row valid
-          if (lt == 0) {
-            // one box of {64 dims, R rows, all 64-dim atoms}: the atoms land R rows apart,
-            // the K-major layout the MMA reads
-            mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKVBytes);
-            const int y = swa_tile ? (int)rl.swa_row0 + rg0 : rg0 - rl.n_swa;
-            tma_load_4d(tile, swa_tile ? &swamap : &kvmap, &full[s], 0, y, 0, b);
+      if constexpr (!KV8) {
+        int ks = 0;
+        uint32_t kph = 0;
+        for (int jj = 0; jj < nt; ++jj) {
+          const int rg0 = (j0 + jj) * R;
+          const int rg = rg0 + my_r;
+          const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
+          const int s = ks;
+          const uint32_t ph = kph;
+          if (++ks == NS) { ks = 0; kph ^= 1; }
+          if (!mbar_wait(&empty[s], ph ^ 1)) break;
+          uint8_t* tile = kv_s + s * Cfg::kKVBytes;
+          // R consecutive rows of one buffer (SWA rows, or hca_attn's dense memory rows):
+          // one TMA box per 64-dim atom, same 128-byte-swizzled layout as the gather
+          const bool swa_tile = p.has_swamap && rg0 + R <= rl.n_swa;
+          const bool mem_tile = !KV8 && p.has_kvmap && !p.sparse && rg0 >= mem0 && rg0 + R <= n_rows;
+          const __nv_bfloat16* src = nullptr;
+          if (swa_tile || mem_tile) {
+            src = kv;                                   // every row valid
+            if (lt == 0) {
+              // one box of {64 dims, R rows, all 64-dim atoms}: the atoms land R rows apart,
+              // the K-major layout the MMA reads
+              mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKVBytes);
+              const int y = swa_tile ? (int)rl.swa_row0 + rg0 : rg0 - mem0;
+              tma_load_4d(tile, swa_tile ? &swamap : &kvmap, &full[s], 0, y, 0, b);
+            } else {
+              mbar_arrive(&full[s]);
+            }
           } else {
+            const int64_t src_off = row_src(rg, raw);
+            src = src_off >= 0 ? kv + src_off : (src_off <= -2 ? swa + (-2 - src_off) : nullptr);
+#pragma unroll 4
+            for (int i = 0; i < CPT; ++i) {
+              const int ch = my_c + TPR * i;
+              uint8_t* dst = tile + sw128_off(my_r, ch, R);
+              if (src) cp_async_16(dst, src + ch * 8);
+              else st_shared_zero16(dst);               // finite filler for rows that do not contribute
+            }
+            fence_proxy_async_smem();
+            cp_async_arrive_noinc(&full[s]);
+          }
+          // validity of this warp's rows (TPR threads per row): one word per loader warp
+          const uint32_t bal = __ballot_sync(0xffffffffu, src != nullptr);
+          if (lane_id() == 0) {
+            uint32_t rows = 0;                          // bit j: row (warp's first row + j)
+            for (int j = 0; j < 32 / TPR; ++j) rows |= ((bal >> (j * TPR)) & 1u) << j;
+            mask_s[s * 4 + (lt >> 5)] = rows;
             mbar_arrive(&full[s]);
           }
-        } else {
-          const int64_t src_off = row_src(rg, raw);
-          src = src_off >= 0 ? kv + src_off : (src_off <= -2 ? swa + (-2 - src_off) : nullptr);
-#pragma unroll 4
-          for (int i = 0; i < CPT; ++i) {
-            const int ch = my_c + TPR * i;
-            uint8_t* dst = tile + sw128_off(my_r, ch, R);
-            if (src) cp_async_16(dst, src + ch * 8);
-            else st_shared_zero16(dst);               // finite filler for rows that do not contribute
+        }
+      } else {
+        // ---- memory rows as KV8 entries: 608-byte entries are copied to the tail of the
+        // tile's buffer; LAG tiles later (all copies of the tile have landed) the loader
+        // threads convert them in place to the bf16 swizzled tile and arrive on full[s].
+        // SWA rows (by TMA, or copied in place) and the padding rows arrive as before.
+        static_assert(D == kKv8Dims && R == 32 && TPR == 4, "KV8 entries: D = 512, 32-row tiles");
+        constexpr int kEC = kKv8Bytes / 16;                 // 16-byte chunks per entry
+        constexpr int kStg = Cfg::kKVBytes - R * kKv8Bytes; // staged entries at the buffer's tail
+        constexpr int LAG = NS - 1;
+        const uint8_t* kv8 = static_cast<const uint8_t*>(p.kv);
+        // completion of memory tile jc (called by all 128 loader threads together)
+        auto complete = [&](int jc) {
+          const int rg0c = (j0 + jc) * R;
+          if (rg0c < mem0) return;                          // SWA / padding tile: arrived at issue
+          const int s = jc % NS;
+          uint8_t* tile = kv_s + s * Cfg::kKVBytes;
+          asm volatile("bar.sync 1, 128;" ::: "memory");   // every thread's copies of tile jc landed
+          const int rg = rg0c + my_r;
+          const int32_t raw = staged ? idx_s[jc * R + my_r] : fetch_raw(rg);
+          const bool ok = row_src(rg, raw) >= 0;
+          const uint8_t* stg = tile + kStg + my_r * kKv8Bytes;
+          uint4 v[7], rp[2];
+          float sc[7];
+          if (ok) {
+#pragma unroll
+            for (int i = 0; i < 7; ++i) v[i] = *reinterpret_cast<const uint4*>(stg + 16 * (my_c + 4 * i));
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              rp[i] = *reinterpret_cast<const uint4*>(stg + kKv8Fp8Dims + 16 * (my_c + 4 * i));
+#pragma unroll
+            for (int i = 0; i < 7; ++i) sc[i] = *reinterpret_cast<const float*>(stg + kKv8ScaleOff + 4 * i);
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");   // staged bytes read: the tile may be written
+          if (ok) {
+#pragma unroll
+            for (int i = 0; i < 7; ++i) {                   // 16 FP8 dims of block i -> two bf16 chunks
+              const int f = 2 * (my_c + 4 * i);
+              const uint4 o0 = make_uint4(e4m3x2_to_bf16x2(v[i].x, sc[i]), e4m3x2_to_bf16x2(v[i].x >> 16, sc[i]),
+                                          e4m3x2_to_bf16x2(v[i].y, sc[i]), e4m3x2_to_bf16x2(v[i].y >> 16, sc[i]));
+              const uint4 o1 = make_uint4(e4m3x2_to_bf16x2(v[i].z, sc[i]), e4m3x2_to_bf16x2(v[i].z >> 16, sc[i]),
+                                          e4m3x2_to_bf16x2(v[i].w, sc[i]), e4m3x2_to_bf16x2(v[i].w >> 16, sc[i]));
+              *reinterpret_cast<uint4*>(tile + sw128_off(my_r, f, R)) = o0;
+              *reinterpret_cast<uint4*>(tile + sw128_off(my_r, f + 1, R)) = o1;
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)                     // RoPE dims: bf16 as stored
+              *reinterpret_cast<uint4*>(tile + sw128_off(my_r, kKv8Fp8Dims / 8 + my_c + 4 * i, R)) = rp[i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) st_shared_zero16(tile + sw128_off(my_r, my_c + TPR * i, R));
           }
           fence_proxy_async_smem();
-          cp_async_arrive_noinc(&full[s]);
-        }
-        // validity of this warp's rows (TPR threads per row): one word per loader warp
-        const uint32_t bal = __ballot_sync(0xffffffffu, src != nullptr);
-        if (lane_id() == 0) {
-          uint32_t rows = 0;                          // bit j: row (warp's first row + j)
-          for (int j = 0; j < 32 / TPR; ++j) rows |= ((bal >> (j * TPR)) & 1u) << j;
-          mask_s[s * 4 + (lt >> 5)] = rows;
           mbar_arrive(&full[s]);
+        };
+        int ks = 0;
+        uint32_t kph = 0;
+        bool go = true;
+        for (int jj = 0; jj < nt; ++jj) {
+          if (jj >= LAG) {
+            cp_async_wait_group<LAG - 1>();                 // this thread's copies of tile jj - LAG
+            complete(jj - LAG);
+          }
+          const int rg0 = (j0 + jj) * R;
+          const int rg = rg0 + my_r;
+          const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
+          const int s = ks;
+          const uint32_t ph = kph;
+          if (++ks == NS) { ks = 0; kph ^= 1; }
+          // every loader thread leaves together (named barriers follow)
+          if (!bar_and_128<1>(mbar_wait(&empty[s], ph ^ 1))) {
+            go = false;
+            break;
+          }
+          uint8_t* tile = kv_s + s * Cfg::kKVBytes;
+          const bool swa_tile = p.has_swamap && rg0 + R <= rl.n_swa;
+          bool valid = true;
+          if (swa_tile) {
+            if (lt == 0) {
+              mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKVBytes);
+              tma_load_4d(tile, &swamap, &full[s], 0, (int)rl.swa_row0 + rg0, 0, b);
+            } else {
+              mbar_arrive(&full[s]);
+            }
+          } else if (rg0 < mem0) {
+            const int64_t so = row_src(rg, raw);              // SWA row (-2 - offset) or padding (-1)
+            const __nv_bfloat16* src = so <= -2 ? swa + (-2 - so) : nullptr;
+            valid = src != nullptr;
+#pragma unroll 4
+            for (int i = 0; i < CPT; ++i) {
+              const int ch = my_c + TPR * i;
+              uint8_t* dst = tile + sw128_off(my_r, ch, R);
+              if (src) cp_async_16(dst, src + ch * 8);
+              else st_shared_zero16(dst);
+            }
+            fence_proxy_async_smem();
+            cp_async_arrive_noinc(&full[s]);
+          } else {
+            const int64_t so = row_src(rg, raw);              // entry number, or -1
+            valid = so >= 0;
+            if (valid) {
+              const uint8_t* e = kv8 + so * kKv8Bytes;
+              uint8_t* dst = tile + kStg + my_r * kKv8Bytes;
+              for (int c = my_c; c < kEC; c += TPR) cp_async_16(dst + 16 * c, e + 16 * c);
+            }
+          }
+          cp_async_commit();                                // one group per tile
+          const uint32_t bal = __ballot_sync(0xffffffffu, valid);
+          if (lane_id() == 0) {
+            uint32_t rows = 0;
+            for (int j = 0; j < 32 / TPR; ++j) rows |= ((bal >> (j * TPR)) & 1u) << j;
+            mask_s[s * 4 + (lt >> 5)] = rows;
+            mbar_arrive(&full[s]);
+          }
         }
+        cp_async_wait_group<0>();
+        if (go)
+          for (int jc = nt > LAG ? nt - LAG : 0; jc < nt; ++jc) complete(jc);
       }
       cp_async_wait_group<0>();                       // none may land after the CTA has left
     }

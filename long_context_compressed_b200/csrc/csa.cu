@@ -21,6 +21,7 @@
 #include "attn.cuh"
 #include "compress.cuh"
 #include "index.cuh"
+#include "kv8.cuh"
 #include "quantize.cuh"
 #include "topk.cuh"
 
@@ -254,6 +255,7 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     }
     return launch_status();
   }
+  const bool kv8 = dtype == CSA_BF16_KV8;
   p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows, p.sparse != 0);
   (void)ws;
   (void)ws_bytes;
@@ -265,9 +267,12 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
   while (p.nsplit > 1) {
     int fit = 0;
     switch (p.D) {
-      case 128: fit = max_active_clusters(csa::attn_tc_kernel<128>, AttnCfg<128>::kThreads, AttnCfg<128>::kSmem, p.nsplit); break;
-      case 256: fit = max_active_clusters(csa::attn_tc_kernel<256>, AttnCfg<256>::kThreads, AttnCfg<256>::kSmem, p.nsplit); break;
-      case 512: fit = max_active_clusters(csa::attn_tc_kernel<512>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit); break;
+      case 128: fit = max_active_clusters(csa::attn_tc_kernel<128, false>, AttnCfg<128>::kThreads, AttnCfg<128>::kSmem, p.nsplit); break;
+      case 256: fit = max_active_clusters(csa::attn_tc_kernel<256, false>, AttnCfg<256>::kThreads, AttnCfg<256>::kSmem, p.nsplit); break;
+      case 512:
+        fit = kv8 ? max_active_clusters(csa::attn_tc_kernel<512, true>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit)
+                  : max_active_clusters(csa::attn_tc_kernel<512, false>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit);
+        break;
       default: break;
     }
     if (fit == 0 && p.nsplit > 8) {        // a non-portable size the device does not take
@@ -287,16 +292,24 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
   const uint32_t rows_per_tile = p.D >= 512 ? 32u : 64u;
   std::memset(&kvmap, 0, sizeof(kvmap));
   std::memset(&swamap, 0, sizeof(swamap));
-  p.has_kvmap = p.N > 0 && make_row_tile_map(&kvmap, p.kv, (uint64_t)p.D, (uint64_t)p.N, (uint64_t)p.B,
-                                             rows_per_tile) ? 1 : 0;
+  // (KV8 entries are not bf16 rows: they are always copied and converted by the loaders)
+  p.has_kvmap = !kv8 && p.N > 0 && make_row_tile_map(&kvmap, p.kv, (uint64_t)p.D, (uint64_t)p.N, (uint64_t)p.B,
+                                                     rows_per_tile) ? 1 : 0;
   p.has_swamap = p.W > 0 && make_row_tile_map(&swamap, p.swa, (uint64_t)p.D, (uint64_t)p.W, (uint64_t)p.B,
                                               rows_per_tile) ? 1 : 0;
+  if (kv8) {
+    if (p.D != 512) return CSA_ERR_UNSUPPORTED;
+    const int sm = AttnCfg<512>::kSmem;
+    if (!set_smem(csa::attn_tc_kernel<512, true>, sm)) return CSA_ERR_CUDA;
+    launch_kc(csa::attn_tc_kernel<512, true>, grid, AttnCfg<512>::kThreads, sm, st, p.nsplit, qmap, kvmap, swamap, p);
+    return launch_status();
+  }
   switch (p.D) {
 #define CSA_LAUNCH_ATTN(DD)                                                                       \
   case DD: {                                                                                      \
     const int sm = AttnCfg<DD>::kSmem;                                                            \
-    if (!set_smem(csa::attn_tc_kernel<DD>, sm)) return CSA_ERR_CUDA;                              \
-    launch_kc(csa::attn_tc_kernel<DD>, grid, AttnCfg<DD>::kThreads, sm, st, p.nsplit, qmap, kvmap, swamap, p); \
+    if (!set_smem(csa::attn_tc_kernel<DD, false>, sm)) return CSA_ERR_CUDA;                       \
+    launch_kc(csa::attn_tc_kernel<DD, false>, grid, AttnCfg<DD>::kThreads, sm, st, p.nsplit, qmap, kvmap, swamap, p); \
     break;                                                                                        \
   }
     CSA_LAUNCH_ATTN(128)
@@ -314,7 +327,7 @@ int check_attn_common(const void* q, const void* kv, const void* swa_kv, const i
   if (B < 0 || T < 0 || H <= 0 || D <= 0 || N < 0 || W < 0) return CSA_ERR_INVALID;
   if ((int64_t)B * T * H * (D / 8) >= (int64_t(1) << 31) || (int64_t)B * T > 65535 * 1024)
     return CSA_ERR_UNSUPPORTED;
-  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_BF16_KV8) return CSA_ERR_INVALID;
   if (!(scale == scale)) return CSA_ERR_INVALID;
   if (B == 0 || T == 0) return CSA_OK;
   if (!q || !out || !swa_pos0 || !q_pos || !sink) return CSA_ERR_INVALID;
@@ -324,6 +337,9 @@ int check_attn_common(const void* q, const void* kv, const void* swa_kv, const i
     return CSA_ERR_INVALID;
   if (dtype == CSA_BF16) {
     if (D != 128 && D != 256 && D != 512) return CSA_ERR_UNSUPPORTED;
+    if (H > 128) return CSA_ERR_UNSUPPORTED;
+  } else if (dtype == CSA_BF16_KV8) {
+    if (D != csa::kKv8Dims) return CSA_ERR_UNSUPPORTED;
     if (H > 128) return CSA_ERR_UNSUPPORTED;
   } else {
     if (D % 32 != 0 || D > 512) return CSA_ERR_UNSUPPORTED;
@@ -417,6 +433,20 @@ int csa_quantize_e4m3(const void* x, int x_dtype, int64_t rows, int cols, uint8_
     launch_k(csa::quantize_e4m3_kernel<__nv_bfloat16>, blocks, 256, 0, st, (const __nv_bfloat16*)x, rows, cols, codes, scale);
   else
     launch_k(csa::quantize_e4m3_kernel<float>, blocks, 256, 0, st, (const float*)x, rows, cols, codes, scale);
+  return launch_status();
+}
+
+long long csa_kv8_entry_bytes(int D) { return D == csa::kKv8Dims ? (long long)csa::kKv8Bytes : 0; }
+
+int csa_quantize_kv8(const void* kv, int64_t rows, int D, void* entries, void* stream) {
+  if (rows < 0) return CSA_ERR_INVALID;
+  if (D != csa::kKv8Dims) return CSA_ERR_UNSUPPORTED;
+  if (rows == 0) return CSA_OK;
+  if (!kv || !entries || !aligned16(kv) || !aligned16(entries)) return CSA_ERR_INVALID;
+  const int64_t blocks64 = (rows + 7) / 8;
+  const unsigned blocks = (unsigned)std::min<int64_t>(blocks64, (int64_t)sm_count() * 32);
+  launch_k(csa::kv8_quantize_kernel, blocks, 256, 0, as_stream(stream), (const __nv_bfloat16*)kv, rows,
+           (uint8_t*)entries);
   return launch_status();
 }
 
@@ -643,7 +673,8 @@ int sparse_attn(const void* q, const void* kv, const void* swa_kv, const int64_t
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
   p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale;
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = k; p.ratio = 1; p.N = N; p.nsplit = 1;
-  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k;
+  // (KV8: the memory rows start at a 32-row tile boundary after the SWA rows)
+  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k + (dtype == CSA_BF16_KV8 ? 31 : 0);
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
 
@@ -657,7 +688,7 @@ int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* s
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
   p.idx = nullptr; p.sparse = 0; p.out = out; p.scale = scale;
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = 0; p.ratio = ratio; p.N = N; p.nsplit = 1;
-  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + N;
+  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + N + (dtype == CSA_BF16_KV8 ? 31 : 0);
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
 

@@ -359,4 +359,21 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Named barrier `ID` over 128 threads that also ANDs a predicate across them: every
+// participant gets true only if all passed true (a uniform decision, e.g. to leave a
+// loop together before further named barriers).
+template <int ID>
+__device__ __forceinline__ bool bar_and_128(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(ID)
+      : "memory");
+  return r != 0;
+}
+
 }  // namespace csa

@@ -112,3 +112,30 @@ def test_index_and_attention_reject_bad_arguments(lib):
     # NaN scale, negative k
     assert g(p, p, p, p, 128, p, p, p, 8, float("nan"), 1, 1, 16, 128, 100, 1, p, None, 0, None) == 1
     assert g(p, p, p, p, 128, p, p, p, -1, 0.1, 1, 1, 16, 128, 100, 1, p, None, 0, None) == 1
+
+
+def test_kv8_storage_host_checks(lib):
+    """Mixed-precision entries: 608 bytes at D = 512, nothing else; bad arguments rejected."""
+    eb = lib.csa_kv8_entry_bytes
+    eb.restype = ctypes.c_longlong
+    eb.argtypes = [ctypes.c_int]
+    assert eb(512) == 608 and eb(128) == 0 and eb(256) == 0
+    q = lib.csa_quantize_kv8
+    q.restype = ctypes.c_int
+    q.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    p = 16
+    assert q(p, 4, 256, p, None) == 2            # D other than 512
+    assert q(None, 4, 512, p, None) == 1         # null source
+    assert q(p, 4, 512, 8, None) == 1            # misaligned destination
+    assert q(p, -1, 512, p, None) == 1
+    assert q(p, 0, 512, p, None) == 0            # nothing to do
+    g = lib.sparse_attn
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    # CSA_BF16_KV8 (3) needs D = 512 and H <= 128; an unknown dtype is invalid
+    assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 16, 256, 100, 3, p, None, 0, None) == 2
+    assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 256, 512, 100, 3, p, None, 0, None) == 2
+    assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 16, 512, 100, 4, p, None, 0, None) == 1
