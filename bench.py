@@ -183,11 +183,11 @@ class DecodeSet:
     """One input set of a decode workload: resident caches, per-step inputs, outputs and
     workspaces on the device, plus pinned host copies of the per-step inputs/outputs."""
 
-    def __init__(self, wl, seed: int, index: str, with_hca: bool, device):
+    def __init__(self, wl, seed: int, index: str, with_hca: bool, device, kv8: bool = False):
         import torch
 
         from long_context_compressed_b200 import csa, synth
-        self.wl, self.index, self.with_hca = wl, index, with_hca
+        self.wl, self.index, self.with_hca, self.kv8 = wl, index, with_hca, kv8
         B, T, N, H, D, k = wl.B, wl.T, wl.N, wl.H, wl.D, wl.topk
         dev = device
         g = lambda nm, shape: synth.store(synth.normal(seed, f"bench/{wl.name}/{nm}", shape, device=dev), "bf16")
@@ -224,6 +224,13 @@ class DecodeSet:
         self.select_ws = csa.select_workspace(B, N, dev)
         self.attn_ws = csa.attn_workspace(B, T, H, D, 128 + k, device=dev)
         self.out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+        # the attention's memory rows: bf16 rows, or (kv8) mixed-precision entries, in which
+        # case the step also quantises the entries its compressor produces
+        self.kv_store = self.kv
+        if kv8:
+            self.kv_store = csa.quantize_kv8(self.kv)
+            self.kv = None
+            self.comp_kv8 = torch.empty(self.comp_kv.shape[:-1] + (csa.KV8_BYTES,), dtype=torch.uint8, device=dev)
         if with_hca:
             Nh = wl.ctx // 128
             self.hkv = g("hkv", (B, Nh, D))
@@ -233,6 +240,11 @@ class DecodeSet:
             self.hcomp = torch.empty((B, 1, D), dtype=torch.bfloat16, device=dev)
             self.hattn_ws = csa.attn_workspace(B, T, H, D, 128 + Nh, device=dev)
             self.hout = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+            self.hkv_store = self.hkv
+            if kv8:
+                self.hkv_store = csa.quantize_kv8(self.hkv)
+                self.hkv = None
+                self.hcomp8 = torch.empty((B, 1, csa.KV8_BYTES), dtype=torch.uint8, device=dev)
         # per-step inputs and outputs live in one contiguous device buffer each (views at
         # 16-byte aligned offsets), so a step moves them with one copy per direction
         self.in_buf, views = _pack(list(self.inputs.values()), dev)
@@ -259,11 +271,15 @@ class DecodeSet:
             q = B * T * 64 * (256 + 4)
         return keys + q + B * T * N * 4
 
+    def row_bytes(self):
+        """Bytes of one memory row of the attention: bf16 row or mixed-precision entry."""
+        return 608 if self.kv8 else self.wl.D * 2
+
     def attn_bytes(self):
         """One sparse_attn launch: q, the gathered top-k and SWA rows, idx, sink, out."""
         wl = self.wl
         B, T, H, D, k = wl.B, wl.T, wl.H, wl.D, wl.topk
-        rows = B * T * (k + min(wl.W, 128)) * D * 2
+        rows = B * T * (k * self.row_bytes() + min(wl.W, 128) * D * 2)
         return B * T * H * D * 2 * 2 + rows + B * T * k * 4 + H * 4
 
     def step_bytes(self):
@@ -275,10 +291,15 @@ class DecodeSet:
         total += B * N * (132 if self.index == "e4m3" else 256)               # index keys (+ scales)
         if self.index == "e4m3":
             total += B * T * 2 * k * 256                                      # rerank: bf16 keys of candidates
-        total += B * T * (k + min(wl.W, 128)) * D * 2                          # gathered latent + SWA rows
+        total += B * T * (k * self.row_bytes() + min(wl.W, 128) * D * 2)      # gathered latent + SWA rows
         total += nb(self.out)
+        if self.kv8:
+            total += nb(self.comp_kv) + nb(self.comp_kv8)                      # quantise the new entries
         if self.with_hca:
-            total += B * (wl.ctx // 128) * D * 2 + B * min(wl.W, 128) * D * 2 + nb(self.hcomp) + nb(self.hout)
+            total += B * (wl.ctx // 128) * self.row_bytes() + B * min(wl.W, 128) * D * 2 + nb(self.hcomp)
+            total += nb(self.hout)
+            if self.kv8:
+                total += nb(self.hcomp) + nb(self.hcomp8)
         return total
 
     def per_step_io(self):
@@ -306,15 +327,19 @@ class DecodeSet:
             with torch.cuda.stream(sa):
                 csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"], ratio=4,
                                  out=self.comp_kv)
+                if self.kv8:
+                    csa.quantize_kv8(self.comp_kv, entries=self.comp_kv8)
             with torch.cuda.stream(sb):
                 if wl.comp_ci:
                     csa.csa_compress(x["iC_a"], x["iC_b"], x["iZ_a"], x["iZ_b"], x["iprev_Cb"], x["iprev_Zb"],
                                      ratio=4, out=self.comp_ki)
                 if self.with_hca:
                     csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=self.hcomp)
+                    if self.kv8:
+                        csa.quantize_kv8(self.hcomp, entries=self.hcomp8)
             if self.with_hca:
                 with torch.cuda.stream(sc):
-                    csa.hca_attn(x["hq"], self.hkv, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
+                    csa.hca_attn(x["hq"], self.hkv_store, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
                                  1.0 / math.sqrt(wl.D), out=self.hout, workspace=self.hattn_ws)
         # stage boundaries on the main stream (event record nodes inside the graph)
         # timing_events: False (the timed graphs) or "all" (every stage: a diagnostic graph;
@@ -345,7 +370,7 @@ class DecodeSet:
             side_branch()
             csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, idx=self.idx)
             mark("select")
-        csa.sparse_attn(x["q"], self.kv, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
+        csa.sparse_attn(x["q"], self.kv_store, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
                         1.0 / math.sqrt(wl.D), out=self.out, workspace=self.attn_ws)
         mark("sparse_attn")
         for ss in side_streams:
@@ -447,7 +472,7 @@ def attn_alone_ms(sets, device, reps_per_set=8, replays=20):
     def launch(i):
         s = sets[i % len(sets)]
         x = s.inputs
-        csa.sparse_attn(x["q"], s.kv, s.swa, s.swa_pos0, s.q_pos, s.sink, s.idx, 1.0 / math.sqrt(s.wl.D),
+        csa.sparse_attn(x["q"], s.kv_store, s.swa, s.swa_pos0, s.q_pos, s.sink, s.idx, 1.0 / math.sqrt(s.wl.D),
                         out=s.out, workspace=s.attn_ws)
     for i in range(len(sets)):
         launch(i)
@@ -470,15 +495,15 @@ def attn_alone_ms(sets, device, reps_per_set=8, replays=20):
     return ms
 
 
-def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=None):
+def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=None, kv8=False):
     import torch
 
     from long_context_compressed_b200 import csa, synth
     wl = synth.WORKLOADS[name]
-    probe = DecodeSet(wl, 0, index, with_hca, device)
+    probe = DecodeSet(wl, 0, index, with_hca, device, kv8=kv8)
     touched = probe.step_bytes()
     n_sets = n_sets or max(2, math.ceil(2 * L2_BYTES / touched) + 1)
-    sets = [probe] + [DecodeSet(wl, s, index, with_hca, device) for s in range(1, n_sets)]
+    sets = [probe] + [DecodeSet(wl, s, index, with_hca, device, kv8=kv8) for s in range(1, n_sets)]
     side = [torch.cuda.Stream(device=device) for _ in range(3)]
     graphs, launches = capture(sets, side)
     t = timed_replays(graphs, steps, warmup, world)
@@ -608,7 +633,7 @@ def bench_prefill(steps, warmup, device, tflops_peak):
     return res
 
 
-def bench_hca(steps, warmup, device, hbm_peak):
+def bench_hca(steps, warmup, device, hbm_peak, kv8=False):
     """Pro-shaped HCA decode at 1M context, B = 4: compress the newest 16,384-token tail
     128:1 (c = 512) and hca_attn (128 heads, D = 512) over all 8,192 entries + 128 SWA rows.
     Input sets rotate so that more than 2x the L2 is touched between reuses."""
@@ -629,6 +654,9 @@ def bench_hca(steps, warmup, device, hbm_peak):
         st["comp"] = torch.empty((B, wl.comp_L // 128, D), dtype=torch.bfloat16, device=dev)
         st["out"] = torch.empty_like(st["q"])
         st["ws"] = csa.attn_workspace(B, T, H, D, 128 + N, device=dev)
+        if kv8:                     # memory rows as mixed-precision entries; new entries quantised
+            st["kv"] = csa.quantize_kv8(st["kv"])
+            st["comp8"] = torch.empty((B, wl.comp_L // 128, csa.KV8_BYTES), dtype=torch.uint8, device=dev)
         sets.append(st)
         touched = sum(nb(st[n]) for n in ("C", "Z", "kv", "swa", "q", "comp", "out"))
         if len(sets) * touched > 2 * L2_BYTES and len(sets) >= 2:
@@ -639,6 +667,8 @@ def bench_hca(steps, warmup, device, hbm_peak):
 
     def step(st):
         csa.csa_compress(st["C"], None, st["Z"], None, ratio=128, out=st["comp"])
+        if kv8:
+            csa.quantize_kv8(st["comp"], entries=st["comp8"])
         csa.hca_attn(st["q"], st["kv"], st["swa"], swa_pos0, q_pos, st["sink"], scale, out=st["out"],
                      workspace=st["ws"])
     c0 = csa.csa_launch_count()
@@ -654,9 +684,13 @@ def bench_hca(steps, warmup, device, hbm_peak):
     t = timed_replays(graphs, steps, warmup, 1)
     assert csa.csa_poll_status() == csa.CSA_OK
     ms = 1e3 * t / steps
-    algo = sum(nb(sets[0][n]) for n in ("C", "Z", "q", "comp", "out")) + B * (N + 128) * D * 2
+    algo = sum(nb(sets[0][n]) for n in ("C", "Z", "q", "comp", "out")) + B * N * (608 if kv8 else D * 2)
+    algo += B * 128 * D * 2
+    if kv8:
+        algo += nb(sets[0]["comp"]) + nb(sets[0]["comp8"])
     res = {"workload": f"pro_hca: B={B} decode at 1M, compress 128:1 over [{B},{wl.comp_L},{wl.comp_c}], "
-                       f"hca_attn H={H} D={D} over {N}+128 rows",
+                       f"hca_attn H={H} D={D} over {N}+128 rows"
+                       + (", memory rows as 608-byte FP8/BF16 entries" if kv8 else ""),
            "tokens_per_s": B * T / (ms * 1e-3), "ms_per_step": ms, "launches_per_step": launches,
            "input_sets": len(sets),
            "step_roofline": {"bytes_per_step": algo, "achieved_gbs": algo / (ms * 1e-3) / 1e9,
@@ -739,14 +773,14 @@ def run_big_stage(stage, steps, warmup, device):
                       "us_per_call": 1e3 * a.elapsed_time(b) / steps}), flush=True)
 
 
-def run_stage(name, stage, index, steps, warmup, device):
+def run_stage(name, stage, index, steps, warmup, device, kv8=False):
     """One stage of the step (one ABI call), eagerly, for profiling a single kernel.
     Prints the mean device time per call measured with CUDA events."""
     import torch
 
     from long_context_compressed_b200 import csa, synth
     wl = synth.WORKLOADS[name]
-    st = DecodeSet(wl, 0, index, name == "flash64k", device)
+    st = DecodeSet(wl, 0, index, name == "flash64k", device, kv8=kv8)
     x = st.inputs
     calls = {
         "compress": lambda: csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"],
@@ -761,10 +795,10 @@ def run_stage(name, stage, index, steps, warmup, device):
                   if index == "e4m3" else
                   (lambda: (csa.csa_score_histogram(st.scores, st.n_valid, st.select_ws),
                             csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws, idx=st.idx))),
-        "attn": lambda: csa.sparse_attn(x["q"], st.kv, st.swa, st.swa_pos0, st.q_pos, st.sink, st.idx,
+        "attn": lambda: csa.sparse_attn(x["q"], st.kv_store, st.swa, st.swa_pos0, st.q_pos, st.sink, st.idx,
                                         1.0 / math.sqrt(wl.D), out=st.out, workspace=st.attn_ws),
         "hcompress": lambda: csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=st.hcomp),
-        "hca": lambda: csa.hca_attn(x["hq"], st.hkv, st.hswa, st.swa_pos0, st.q_pos, st.hsink,
+        "hca": lambda: csa.hca_attn(x["hq"], st.hkv_store, st.hswa, st.swa_pos0, st.q_pos, st.hsink,
                                     1.0 / math.sqrt(wl.D), out=st.hout, workspace=st.hattn_ws),
     }
     # inputs of the later stages come from the earlier ones
@@ -862,6 +896,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the pro1m measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", choices=STAGES + BIG_STAGES, help="time one stage alone (eager calls), e.g. under ncu")
+    ap.add_argument("--kv8", action="store_true", help="with --stage: memory rows as mixed-precision KV8 entries")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_env()
@@ -908,7 +943,7 @@ def main():
         run_big_stage(args.stage, args.steps, args.warmup, device)
         return
     if args.stage:
-        run_stage(args.workload, args.stage, args.index, args.steps, args.warmup, device)
+        run_stage(args.workload, args.stage, args.index, args.steps, args.warmup, device, kv8=args.kv8)
         return
     peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
@@ -918,16 +953,22 @@ def main():
     if not args.no_extra and args.workload != "pro1m":
         extra = bench_workload("pro1m", args.index, False, args.steps, args.warmup, world, device)
     prefill = hca = None
+    kv8_runs = {}
     if not args.no_extra:
         prefill = bench_prefill(max(5, min(20, args.steps // 100)), 3, device, measured_tflops())
         hca = bench_hca(args.steps, args.warmup, device, peak)
+        # the same decode steps with the memory rows stored as mixed-precision entries
+        for nm in ([args.workload] + (["pro1m"] if args.workload != "pro1m" else [])):
+            kv8_runs[nm] = bench_workload(nm, args.index, nm == "flash64k", args.steps, args.warmup, world, device,
+                                          kv8=True)
+        kv8_runs["pro_hca"] = bench_hca(args.steps, args.warmup, device, peak, kv8=True)
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         cpu = oracle_baseline(main_res["wl"], args.index, with_hca)
     if rank != 0:
         return
 
-    def summarise(r):
+    def summarise(r, kv8=False):
         wl = r["wl"]
         tok = r["tokens_per_step"] * world
         steps = args.steps
@@ -938,10 +979,12 @@ def main():
             "value": tok * steps / r["seconds"], "ms_per_step": r["step_ms"],
             "e2e": {"value": tok * steps / r["e2e_seconds"], "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-            "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (sparse_attn: top-k + SWA rows, cluster merge)",
+            "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (sparse_attn: top-k + SWA rows, cluster merge"
+                                                   + (", memory rows as KV8 entries)" if kv8 else ")"),
                          "achieved": attn_gbs, "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak,
                          "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
-                         "traffic": profiled_traffic("attn_tc_kernel_decode_prefill_hca.md", "attn.cuh", wl.name),
+                         "traffic": profiled_traffic("attn_tc_kernel_decode_prefill_hca.md", "attn.cuh",
+                                                     wl.name + ("_kv8" if kv8 else "")),
                          "bytes_per_launch": r["attn_bytes"], "avg_launch_us": r["attn_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays",
@@ -996,6 +1039,19 @@ def main():
         line["prefill"] = prefill
     if hca is not None:
         line["pro_hca"] = hca
+    if kv8_runs:
+        kv = {"storage": "memory rows as 608-byte entries: 448 e4m3 dims with a power-of-two scale per 64 dims, "
+                         "64 bf16 RoPE dims; the step also quantises the entries its compressors produce"}
+        for nm, r in kv8_runs.items():
+            if nm == "pro_hca":
+                kv[nm] = r
+                continue
+            e = summarise(r, kv8=True)
+            kv[nm] = {"value": e["value"], "unit": "tokens/s", "ms_per_step": e["ms_per_step"],
+                      "roofline": e["roofline"], "step_roofline": e["step_roofline"], "e2e": e["e2e"],
+                      "launches_per_step": e["launches_per_step"]}
+            line["gpu_launches"] += e["gpu_launches"]
+        line["kv8"] = kv
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
