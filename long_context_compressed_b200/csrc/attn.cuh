@@ -156,9 +156,13 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
 }
 
 // ------------------------------------------------------------------ tcgen05 bf16
-template <int D>
+// RT: rows per KV tile.  One S = Q K^T MMA instruction (N = RT rows) costs about the same
+// for N = 32 and N = 64 (~46 cycles), so a 32-row tile of D = 512 spends ~0.75 us issuing
+// its 32 S instructions; 64-row tiles would halve that per row but leave two stages in
+// shared memory at D = 512, which measured slower.
+template <int D, int RT = (D >= 512 ? 32 : 64)>
 struct AttnCfg {
-  static constexpr int R = (D >= 512) ? 32 : 64;           // rows per KV tile
+  static constexpr int R = RT;                             // rows per KV tile
   static constexpr int DH = (D > 256) ? 256 : D;           // D-slice per CTA
   static constexpr int NDH = D / DH;
   static constexpr int kAtoms = D / 64;                    // 128-byte atoms per row
@@ -180,6 +184,12 @@ struct AttnCfg {
   static __host__ __device__ int head_groups(int H) { return (H + kHeadGroup - 1) / kHeadGroup; }
 };
 
+// KV8 launches 13 warps: warps 9..12 are the converters.
+__host__ __device__ constexpr int attn_threads(bool kv8) { return kv8 ? 416 : 288; }
+
+// A zero entry: the source of the staged bytes of KV8 rows that contribute nothing.
+__device__ __align__(16) uint8_t g_kv8_zero_entry[kKv8Bytes];
+
 // Byte offset of 16-byte chunk c of row r in a K-major tile with 128-byte
 // swizzle, whose 64-element atoms are `rows` rows tall.
 __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
@@ -190,17 +200,20 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
 // (head group blockIdx.y / NDH).  The M = 128 MMA operand of atom a also spans the first 64
 // rows of atom a+1 (or, for the last atom, the next 8 KB of shared memory):
 // finite values whose result rows (>= H) are never used.
-// KV8: memory rows are csa_quantize_kv8 entries (FP8 dims + BF16 RoPE dims, D = 512);
-// the loader warps stage each 608-byte entry at the tail of its tile's buffer by
-// cp.async and convert it to the bf16 tile (exact: code * 2^e is a bf16 value) before
-// the MMA reads it.  The memory rows then start at a tile boundary of the row list
-// (the SWA rows are padded with masked rows), so a tile is all SWA or all memory.
-template <int D, bool KV8>
-__global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+// KV8: memory rows are csa_quantize_kv8 entries (FP8 dims + BF16 RoPE dims, D = 512).
+// The loader warps stage each tile's 608-byte entries at the tail of its buffer (one
+// bulk copy for a contiguous tile of hca_attn, cp.async per entry otherwise; rows that
+// contribute nothing copy a zero entry), counted on the stage's `staged` barrier; four
+// converter warps (9..12) then rewrite the tile in place as the bf16 swizzled tile
+// (exact: code * 2^e is a bf16 value) and arrive on `full`.  The memory rows start at a
+// tile boundary of the row list (the SWA rows are padded with masked rows), so a tile
+// is all SWA or all memory.
+template <int D, bool KV8, int RT>
+__global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                            const __grid_constant__ CUtensorMap kvmap,
                                                                            const __grid_constant__ CUtensorMap swamap,
                                                                            const AttnParams p) {
-  using Cfg = AttnCfg<D>;
+  using Cfg = AttnCfg<D, RT>;
   constexpr int R = Cfg::R, DH = Cfg::DH;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -219,6 +232,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
   uint64_t* odone = bars + 17;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 20);      // [4 stages][4 loader warps]
+  uint64_t* staged = bars + 28;  // [4] KV8: a memory tile's entries are in its buffer's tail
   int32_t* idx_s = reinterpret_cast<int32_t*>(bars + 32);         // [kMaxCtaRows] raw index values
 
   __shared__ float epi_g[Cfg::kHeadGroup];   // per-head output scale (softmax -> epilogue warps)
@@ -239,6 +253,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
     for (int i = 0; i < 4; ++i) {
       mbar_init(&full[i], 128 + 4);          // cp.async of 128 threads + a mask word per loader warp
       mbar_init(&empty[i], 1);
+      if (KV8) mbar_init(&staged[i], 128);   // cp.async arrivals of the 128 loader threads
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
@@ -302,8 +317,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       // stage this CTA's index values in shared memory once (coalesced), so no
       // global load sits between the tiles
       const int row0 = j0 * R, nrow = nt * R;
-      const bool staged = p.sparse && nrow <= Cfg::kMaxCtaRows;
-      if (staged) {
+      const bool staged_idx = p.sparse && nrow <= Cfg::kMaxCtaRows;
+      if (staged_idx) {
         for (int r = lt; r < nrow; r += 128) {
           const int rg = row0 + r;
           idx_s[r] = (rg >= mem0 && rg < n_rows) ? __ldg(idx_row + (rg - mem0)) : 0;
@@ -316,7 +331,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
         for (int jj = 0; jj < nt; ++jj) {
           const int rg0 = (j0 + jj) * R;
           const int rg = rg0 + my_r;
-          const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
+          const int32_t raw = staged_idx ? idx_s[jj * R + my_r] : fetch_raw(rg);
           const int s = ks;
           const uint32_t ph = kph;
           if (++ks == NS) { ks = 0; kph ^= 1; }
@@ -361,78 +376,23 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
           }
         }
       } else {
-        // ---- memory rows as KV8 entries: 608-byte entries are copied to the tail of the
-        // tile's buffer; LAG tiles later (all copies of the tile have landed) the loader
-        // threads convert them in place to the bf16 swizzled tile and arrive on full[s].
+        // ---- memory rows as KV8 entries, staged at the tail of the tile's buffer and
+        // counted on staged[s]; the converter warps arrive on full[s] for those tiles.
         // SWA rows (by TMA, or copied in place) and the padding rows arrive as before.
-        static_assert(D == kKv8Dims && R == 32 && TPR == 4, "KV8 entries: D = 512, 32-row tiles");
+        static_assert(D == kKv8Dims && (TPR == 2 || TPR == 4), "KV8 entries: D = 512, 32- or 64-row tiles");
         constexpr int kEC = kKv8Bytes / 16;                 // 16-byte chunks per entry
         constexpr int kStg = Cfg::kKVBytes - R * kKv8Bytes; // staged entries at the buffer's tail
-        constexpr int LAG = NS - 1;
         const uint8_t* kv8 = static_cast<const uint8_t*>(p.kv);
-        // completion of memory tile jc (called by all 128 loader threads together)
-        auto complete = [&](int jc) {
-          const int rg0c = (j0 + jc) * R;
-          if (rg0c < mem0) return;                          // SWA / padding tile: arrived at issue
-          const int s = jc % NS;
-          uint8_t* tile = kv_s + s * Cfg::kKVBytes;
-          asm volatile("bar.sync 1, 128;" ::: "memory");   // every thread's copies of tile jc landed
-          const int rg = rg0c + my_r;
-          const int32_t raw = staged ? idx_s[jc * R + my_r] : fetch_raw(rg);
-          const bool ok = row_src(rg, raw) >= 0;
-          const uint8_t* stg = tile + kStg + my_r * kKv8Bytes;
-          uint4 v[7], rp[2];
-          float sc[7];
-          if (ok) {
-#pragma unroll
-            for (int i = 0; i < 7; ++i) v[i] = *reinterpret_cast<const uint4*>(stg + 16 * (my_c + 4 * i));
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-              rp[i] = *reinterpret_cast<const uint4*>(stg + kKv8Fp8Dims + 16 * (my_c + 4 * i));
-#pragma unroll
-            for (int i = 0; i < 7; ++i) sc[i] = *reinterpret_cast<const float*>(stg + kKv8ScaleOff + 4 * i);
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");   // staged bytes read: the tile may be written
-          if (ok) {
-#pragma unroll
-            for (int i = 0; i < 7; ++i) {                   // 16 FP8 dims of block i -> two bf16 chunks
-              const int f = 2 * (my_c + 4 * i);
-              const uint4 o0 = make_uint4(e4m3x2_to_bf16x2(v[i].x, sc[i]), e4m3x2_to_bf16x2(v[i].x >> 16, sc[i]),
-                                          e4m3x2_to_bf16x2(v[i].y, sc[i]), e4m3x2_to_bf16x2(v[i].y >> 16, sc[i]));
-              const uint4 o1 = make_uint4(e4m3x2_to_bf16x2(v[i].z, sc[i]), e4m3x2_to_bf16x2(v[i].z >> 16, sc[i]),
-                                          e4m3x2_to_bf16x2(v[i].w, sc[i]), e4m3x2_to_bf16x2(v[i].w >> 16, sc[i]));
-              *reinterpret_cast<uint4*>(tile + sw128_off(my_r, f, R)) = o0;
-              *reinterpret_cast<uint4*>(tile + sw128_off(my_r, f + 1, R)) = o1;
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i)                     // RoPE dims: bf16 as stored
-              *reinterpret_cast<uint4*>(tile + sw128_off(my_r, kKv8Fp8Dims / 8 + my_c + 4 * i, R)) = rp[i];
-          } else {
-#pragma unroll
-            for (int i = 0; i < CPT; ++i) st_shared_zero16(tile + sw128_off(my_r, my_c + TPR * i, R));
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&full[s]);
-        };
         int ks = 0;
         uint32_t kph = 0;
-        bool go = true;
         for (int jj = 0; jj < nt; ++jj) {
-          if (jj >= LAG) {
-            cp_async_wait_group<LAG - 1>();                 // this thread's copies of tile jj - LAG
-            complete(jj - LAG);
-          }
           const int rg0 = (j0 + jj) * R;
           const int rg = rg0 + my_r;
-          const int32_t raw = staged ? idx_s[jj * R + my_r] : fetch_raw(rg);
+          const int32_t raw = staged_idx ? idx_s[jj * R + my_r] : fetch_raw(rg);
           const int s = ks;
           const uint32_t ph = kph;
           if (++ks == NS) { ks = 0; kph ^= 1; }
-          // every loader thread leaves together (named barriers follow)
-          if (!bar_and_128<1>(mbar_wait(&empty[s], ph ^ 1))) {
-            go = false;
-            break;
-          }
+          if (!mbar_wait(&empty[s], ph ^ 1)) break;
           uint8_t* tile = kv_s + s * Cfg::kKVBytes;
           const bool swa_tile = p.has_swamap && rg0 + R <= rl.n_swa;
           bool valid = true;
@@ -456,16 +416,22 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
             }
             fence_proxy_async_smem();
             cp_async_arrive_noinc(&full[s]);
+          } else if (!p.sparse && rg0 + R <= n_rows) {
+            // hca_attn: R consecutive entries, one bulk copy
+            if (lt == 0) {
+              mbar_arrive_expect_tx(&staged[s], (uint32_t)(R * kKv8Bytes));
+              bulk_load(tile + kStg, kv8 + ((int64_t)b * p.N + (rg0 - mem0)) * kKv8Bytes, R * kKv8Bytes, &staged[s]);
+            } else {
+              mbar_arrive(&staged[s]);
+            }
           } else {
             const int64_t so = row_src(rg, raw);              // entry number, or -1
             valid = so >= 0;
-            if (valid) {
-              const uint8_t* e = kv8 + so * kKv8Bytes;
-              uint8_t* dst = tile + kStg + my_r * kKv8Bytes;
-              for (int c = my_c; c < kEC; c += TPR) cp_async_16(dst + 16 * c, e + 16 * c);
-            }
+            const uint8_t* e = valid ? kv8 + so * kKv8Bytes : g_kv8_zero_entry;
+            uint8_t* dst = tile + kStg + my_r * kKv8Bytes;
+            for (int c = my_c; c < kEC; c += TPR) cp_async_16(dst + 16 * c, e + 16 * c);
+            cp_async_arrive_noinc(&staged[s]);
           }
-          cp_async_commit();                                // one group per tile
           const uint32_t bal = __ballot_sync(0xffffffffu, valid);
           if (lane_id() == 0) {
             uint32_t rows = 0;
@@ -474,9 +440,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
             mbar_arrive(&full[s]);
           }
         }
-        cp_async_wait_group<0>();
-        if (go)
-          for (int jc = nt > LAG ? nt - LAG : 0; jc < nt; ++jc) complete(jc);
       }
       cp_async_wait_group<0>();                       // none may land after the CTA has left
     }
@@ -536,7 +499,60 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1) attn_tc_kernel(const 
       }
       mma_commit(odone);
     }
-  } else {
+  } else if (KV8 && warp >= 9) {
+    // ------------------------------------------------------------ converters (warps 9..12, KV8)
+    // A memory tile's staged entries -> the bf16 swizzled tile, in place: every thread
+    // reads its row's share of the entry, the 128 converters meet, then write.
+    if constexpr (KV8) {
+      constexpr int TPR = 128 / R;
+      constexpr int kStg = Cfg::kKVBytes - R * kKv8Bytes;
+      const int lc = (int)threadIdx.x - 288;
+      const int my_r = lc / TPR, my_c = lc % TPR;
+      uint32_t sph = 0;                                     // bit s: parity of staged[s]'s next phase
+      int ks = 0;
+      for (int jj = 0; jj < nt; ++jj) {
+        const int s = ks;
+        if (++ks == NS) ks = 0;
+        if ((j0 + jj) * R < mem0) continue;                 // SWA / padding tile
+        const bool got = mbar_wait(&staged[s], (sph >> s) & 1u);
+        sph ^= 1u << s;
+        if (!bar_and_128<3>(got)) break;                    // leave together (named barrier below)
+        uint8_t* tile = kv_s + s * Cfg::kKVBytes;
+        const uint8_t* stg = tile + kStg + my_r * kKv8Bytes;
+        // this thread's share of the row: FP8 chunks q = my_c + TPR * i (16 dims each,
+        // block q / 4) and RoPE chunks my_c + TPR * i (8 dims each)
+        constexpr int NQ = (kKv8Fp8Dims / 16) / TPR, NRP = 8 / TPR;
+        uint4 v[NQ], rp[NRP];
+        float sc[7];
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) v[i] = *reinterpret_cast<const uint4*>(stg + 16 * (my_c + TPR * i));
+#pragma unroll
+        for (int i = 0; i < NRP; ++i)
+          rp[i] = *reinterpret_cast<const uint4*>(stg + kKv8Fp8Dims + 16 * (my_c + TPR * i));
+#pragma unroll
+        for (int i = 0; i < 7; ++i) sc[i] = *reinterpret_cast<const float*>(stg + kKv8ScaleOff + 4 * i);
+        asm volatile("bar.sync 3, 128;" ::: "memory");     // staged bytes read: the tile may be written
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {                      // 16 FP8 dims -> two bf16 chunks
+          const int q = my_c + TPR * i;
+          float c;
+          if constexpr (TPR == 4) c = sc[i];                // q / 4 == i: a static register index
+          else c = sc[q >> 2];
+          const uint4 o0 = make_uint4(e4m3x2_to_bf16x2(v[i].x, c), e4m3x2_to_bf16x2(v[i].x >> 16, c),
+                                      e4m3x2_to_bf16x2(v[i].y, c), e4m3x2_to_bf16x2(v[i].y >> 16, c));
+          const uint4 o1 = make_uint4(e4m3x2_to_bf16x2(v[i].z, c), e4m3x2_to_bf16x2(v[i].z >> 16, c),
+                                      e4m3x2_to_bf16x2(v[i].w, c), e4m3x2_to_bf16x2(v[i].w >> 16, c));
+          *reinterpret_cast<uint4*>(tile + sw128_off(my_r, 2 * q, R)) = o0;
+          *reinterpret_cast<uint4*>(tile + sw128_off(my_r, 2 * q + 1, R)) = o1;
+        }
+#pragma unroll
+        for (int i = 0; i < NRP; ++i)                       // RoPE dims: bf16 as stored
+          *reinterpret_cast<uint4*>(tile + sw128_off(my_r, kKv8Fp8Dims / 8 + my_c + TPR * i, R)) = rp[i];
+        fence_proxy_async_smem();
+        mbar_arrive(&full[s]);
+      }
+    }
+  } else if (warp < 4) {
     // ------------------------------------------------------------ softmax / epilogue (warps 0..3)
     const int h = threadIdx.x;                 // TMEM lane = head row
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;

@@ -218,20 +218,16 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, int smem, int clu
 }
 
 // ------------------------------------------------------------------ attention split policy
-template <int D>
-int attn_rows_per_tile() { return AttnCfg<D>::R; }
-
 int attn_ndh(int D) { return D > 256 ? D / 256 : 1; }
 
 // CTAs per (query, D-slice, head group) over the row list: one wave of CTAs, at
 // least two KV tiles each for sparse_attn (gathered rows: the more SMs issue the
 // gathers, the sooner the rows are in) and four for hca_attn (contiguous rows by TMA,
 // and it shares the GPU with the chain of the CSA layer)
-int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse) {
+int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse, int R) {
   const int64_t items = (int64_t)B * T * attn_ndh(D) * ((H + 63) / 64);
   const int sms = sm_count();
   if (items <= 0 || items >= 2 * sms) return 1;
-  const int R = D >= 512 ? 32 : 64;
   const int64_t tiles = (max_rows + R - 1) / R;
   const int64_t want = std::max<int64_t>(1, sms / items);
   const int64_t cap = std::max<int64_t>(1, tiles / (sparse ? 2 : 4));
@@ -256,7 +252,10 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     return launch_status();
   }
   const bool kv8 = dtype == CSA_BF16_KV8;
-  p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows, p.sparse != 0);
+  // rows per KV tile: 32 at D = 512 (four stages in shared memory), else 64.  Measured:
+  // 64-row tiles at D = 512 (two stages) were slower for gathered, dense and KV8 rows.
+  const int R = p.D < 512 ? 64 : 32;
+  p.nsplit = attn_nsplit(p.B, p.T, p.H, p.D, max_rows, p.sparse != 0, R);
   (void)ws;
   (void)ws_bytes;
   // grid: (splits of the row list, D-slice x head group of 64, query)
@@ -267,11 +266,12 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
   while (p.nsplit > 1) {
     int fit = 0;
     switch (p.D) {
-      case 128: fit = max_active_clusters(csa::attn_tc_kernel<128, false>, AttnCfg<128>::kThreads, AttnCfg<128>::kSmem, p.nsplit); break;
-      case 256: fit = max_active_clusters(csa::attn_tc_kernel<256, false>, AttnCfg<256>::kThreads, AttnCfg<256>::kSmem, p.nsplit); break;
+      case 128: fit = max_active_clusters(csa::attn_tc_kernel<128, false, 64>, 288, AttnCfg<128, 64>::kSmem, p.nsplit); break;
+      case 256: fit = max_active_clusters(csa::attn_tc_kernel<256, false, 64>, 288, AttnCfg<256, 64>::kSmem, p.nsplit); break;
       case 512:
-        fit = kv8 ? max_active_clusters(csa::attn_tc_kernel<512, true>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit)
-                  : max_active_clusters(csa::attn_tc_kernel<512, false>, AttnCfg<512>::kThreads, AttnCfg<512>::kSmem, p.nsplit);
+        fit = kv8 ? max_active_clusters(csa::attn_tc_kernel<512, true, 32>, csa::attn_threads(true),
+                                        AttnCfg<512, 32>::kSmem, p.nsplit)
+                  : max_active_clusters(csa::attn_tc_kernel<512, false, 32>, 288, AttnCfg<512, 32>::kSmem, p.nsplit);
         break;
       default: break;
     }
@@ -289,7 +289,7 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
                 (uint64_t)p.B * p.T, 64, 64))
     return CSA_ERR_CUDA;
   // kv and swa_kv as boxes of {64 dims, R rows}: contiguous row tiles load by TMA
-  const uint32_t rows_per_tile = p.D >= 512 ? 32u : 64u;
+  const uint32_t rows_per_tile = (uint32_t)R;
   std::memset(&kvmap, 0, sizeof(kvmap));
   std::memset(&swamap, 0, sizeof(swamap));
   // (KV8 entries are not bf16 rows: they are always copied and converted by the loaders)
@@ -297,27 +297,22 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
                                                      rows_per_tile) ? 1 : 0;
   p.has_swamap = p.W > 0 && make_row_tile_map(&swamap, p.swa, (uint64_t)p.D, (uint64_t)p.W, (uint64_t)p.B,
                                               rows_per_tile) ? 1 : 0;
+  auto launch = [&](auto kernel, int threads, int smem) -> int {
+    if (!set_smem(kernel, smem)) return CSA_ERR_CUDA;
+    launch_kc(kernel, grid, threads, smem, st, p.nsplit, qmap, kvmap, swamap, p);
+    return CSA_OK;
+  };
+  int rc = CSA_ERR_UNSUPPORTED;
   if (kv8) {
-    if (p.D != 512) return CSA_ERR_UNSUPPORTED;
-    const int sm = AttnCfg<512>::kSmem;
-    if (!set_smem(csa::attn_tc_kernel<512, true>, sm)) return CSA_ERR_CUDA;
-    launch_kc(csa::attn_tc_kernel<512, true>, grid, AttnCfg<512>::kThreads, sm, st, p.nsplit, qmap, kvmap, swamap, p);
-    return launch_status();
+    if (p.D == 512) rc = launch(csa::attn_tc_kernel<512, true, 32>, csa::attn_threads(true), AttnCfg<512, 32>::kSmem);
+  } else if (p.D == 512) {
+    rc = launch(csa::attn_tc_kernel<512, false, 32>, 288, AttnCfg<512, 32>::kSmem);
+  } else if (p.D == 256) {
+    rc = launch(csa::attn_tc_kernel<256, false, 64>, 288, AttnCfg<256, 64>::kSmem);
+  } else if (p.D == 128) {
+    rc = launch(csa::attn_tc_kernel<128, false, 64>, 288, AttnCfg<128, 64>::kSmem);
   }
-  switch (p.D) {
-#define CSA_LAUNCH_ATTN(DD)                                                                       \
-  case DD: {                                                                                      \
-    const int sm = AttnCfg<DD>::kSmem;                                                            \
-    if (!set_smem(csa::attn_tc_kernel<DD, false>, sm)) return CSA_ERR_CUDA;                       \
-    launch_kc(csa::attn_tc_kernel<DD, false>, grid, AttnCfg<DD>::kThreads, sm, st, p.nsplit, qmap, kvmap, swamap, p); \
-    break;                                                                                        \
-  }
-    CSA_LAUNCH_ATTN(128)
-    CSA_LAUNCH_ATTN(256)
-    CSA_LAUNCH_ATTN(512)
-#undef CSA_LAUNCH_ATTN
-    default: return CSA_ERR_UNSUPPORTED;
-  }
+  if (rc != CSA_OK) return rc;
   return launch_status();
 }
 
@@ -673,7 +668,7 @@ int sparse_attn(const void* q, const void* kv, const void* swa_kv, const int64_t
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
   p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale;
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = k; p.ratio = 1; p.N = N; p.nsplit = 1;
-  // (KV8: the memory rows start at a 32-row tile boundary after the SWA rows)
+  // (KV8: the memory rows start at a tile boundary, at most 31 rows after the SWA rows)
   const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k + (dtype == CSA_BF16_KV8 ? 31 : 0);
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
