@@ -402,6 +402,75 @@ def capture(sets, sides, **kw):
     return graphs, launches
 
 
+def capture_steps(sets, sides, copies: bool):
+    """One CUDA graph that runs the given input sets once each, in order, as a serving loop
+    would.  With copies, the host->device copy of step j+1's inputs (pinned host buffer, its
+    own stream) and the device->host read of step j's outputs (another stream) overlap step
+    j's compute; every step still moves its own inputs and outputs inside the graph."""
+    import torch
+    main = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    for s in sets:
+        s.run(sides)                                          # eager warm-up
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        if not copies:
+            for s in sets:
+                s.run(sides)
+        else:
+            ev_in = [torch.cuda.Event() for _ in sets]
+            ev_done = [torch.cuda.Event() for _ in sets]
+            h2d.wait_stream(main)
+            d2h.wait_stream(main)
+            with torch.cuda.stream(h2d):
+                sets[0].in_buf.copy_(sets[0].host_in, non_blocking=True)
+                ev_in[0].record(h2d)
+            for j, s in enumerate(sets):
+                if j + 1 < len(sets):
+                    with torch.cuda.stream(h2d):
+                        sets[j + 1].in_buf.copy_(sets[j + 1].host_in, non_blocking=True)
+                        ev_in[j + 1].record(h2d)
+                main.wait_event(ev_in[j])
+                s.run(sides)
+                ev_done[j].record(main)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(ev_done[j])
+                    s.host_out.copy_(s.out_buf, non_blocking=True)
+            main.wait_stream(h2d)
+            main.wait_stream(d2h)
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_steps(sets, sides, steps: int, warmup: int, world: int, copies: bool = False):
+    """Seconds for exactly `steps` steps: replays of a graph over all input sets (each step
+    on the next set, so a set is reused only after every other set has been touched) and one
+    graph over the first steps % len(sets) sets; warm-up covers at least `warmup` steps."""
+    import torch
+    n = len(sets)
+    g_all = capture_steps(sets, sides, copies)
+    rem = steps % n
+    g_rem = capture_steps(sets[:rem], sides, copies) if rem else None
+    for _ in range(max(1, -(-warmup // n))):
+        g_all.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps // n):
+        g_all.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    del g_all, g_rem
+    return a.elapsed_time(b) / 1e3          # seconds
+
+
 def timed_replays(graphs, steps: int, warmup: int, world: int):
     import torch
     for i in range(warmup):
@@ -506,8 +575,9 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     sets = [probe] + [DecodeSet(wl, s, index, with_hca, device, kv8=kv8) for s in range(1, n_sets)]
     side = [torch.cuda.Stream(device=device) for _ in range(3)]
     graphs, launches = capture(sets, side)
-    t = timed_replays(graphs, steps, warmup, world)
+    t = timed_replays(graphs, steps, warmup, world)           # one graph per step, sets in rotation
     t = max_over_ranks(t, world, device)
+    del graphs
     idx_ms = index_alone_ms(sets, index, device, replays=max(3, min(20, steps // 100)))
     attn_ms = attn_alone_ms(sets, device, replays=max(3, min(20, steps // 100)))
     # per-stage breakdown from a separate diagnostic graph with events between all stages
@@ -524,8 +594,8 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     del diag
     # end to end: the same step with its inputs copied in from pinned host memory and its
     # outputs read back, inside every timed step
-    e2e_graphs, _ = capture(sets, side, copies=True)
-    t_e2e = max_over_ranks(timed_replays(e2e_graphs, steps, warmup, world), world, device)
+    # (the next step's input copy and the previous outputs' read overlap each step's compute)
+    t_e2e = max_over_ranks(timed_steps(sets, side, steps, warmup, world, copies=True), world, device)
     assert csa.csa_poll_status() == csa.CSA_OK
     h2d, d2h = probe.per_step_io()
     res = {"wl": wl, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
@@ -533,7 +603,7 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
            "attn_ms": attn_ms, "attn_bytes": probe.attn_bytes(),
            "e2e_seconds": t_e2e, "h2d": h2d, "d2h": d2h, "tokens_per_step": wl.B * wl.T,
            "breakdown": breakdown}
-    del graphs, e2e_graphs, sets
+    del sets
     torch.cuda.empty_cache()
     return res
 
