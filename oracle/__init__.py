@@ -69,6 +69,9 @@ def _load():
     lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_quantize_rows_e4m3.argtypes = [_f32p, i64, i32, _u8p, _f32p]
+    lib.oracle_sparse_attn_partial.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _i32p, i32, dbl, i32,
+                                               i32, i32, i32, i64, _f64p, _f64p, _f64p]
+    lib.oracle_attn_combine.argtypes = [i32, i32, i32, i32, _f64p, _f64p, _f64p, _f32p, _f64p]
     lib.oracle_kv8_entry_bytes.argtypes = [i32]
     lib.oracle_kv8_entry_bytes.restype = i64
     lib.oracle_kv8_quantize.argtypes = [_f32p, i64, i32, _u8p]
@@ -80,7 +83,7 @@ def _load():
                                     i32, i32, i32, i64, _f64p, _f64p]
     for name in ("oracle_compress_csa", "oracle_compress_hca", "oracle_index_scores",
                  "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_kv8_quantize",
-                 "oracle_kv8_dequantize", "oracle_topk",
+                 "oracle_kv8_dequantize", "oracle_sparse_attn_partial", "oracle_attn_combine", "oracle_topk",
                  "oracle_sparse_attn", "oracle_hca_attn"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -284,6 +287,44 @@ def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale, window: int = 
                                       k, float(scale), window, T, H, D, N, ob, mb), "sparse_attn")
         out[b], mag[b] = ob, mb
     return (out, mag) if with_mag else out
+
+
+def sparse_attn_partial(q, kv, swa_kv, swa_pos0, q_pos, idx, scale, window: int = 128, with_swa: bool = True):
+    """Attention pieces over one row set without the sink: (m [B,T,H], l [B,T,H], o [B,T,H,D]),
+    m = max z, l = sum e^(z - m), o = sum e^(z - m) row / l.  The SWA rows count only if
+    with_swa; the memory rows are kv[idx] for idx in [0, N)."""
+    lib = _load()
+    q, kv, swa_kv = _f32(q), _f32(kv), _f32(swa_kv)
+    B, T, H, D = q.shape
+    N, W, k = kv.shape[1], swa_kv.shape[1], idx.shape[2]
+    idx = np.ascontiguousarray(np.asarray(idx, np.int32))
+    s0 = np.asarray(swa_pos0, np.int64).reshape(B)
+    qp = np.ascontiguousarray(np.asarray(q_pos, np.int64))
+    m = np.empty((B, T, H)); l = np.empty((B, T, H)); o = np.empty((B, T, H, D))
+    for b in range(B):
+        mb, lb, ob = np.empty((T, H)), np.empty((T, H)), np.empty((T, H, D))
+        _check(lib.oracle_sparse_attn_partial(np.ascontiguousarray(q[b]), np.ascontiguousarray(kv[b]),
+                                              np.ascontiguousarray(swa_kv[b]), int(s0[b]), W if with_swa else 0,
+                                              np.ascontiguousarray(qp[b]), np.ascontiguousarray(idx[b]), k,
+                                              float(scale), window, T, H, D, N, mb, lb, ob), "sparse_attn_partial")
+        m[b], l[b], o[b] = mb, lb, ob
+    return m, l, o
+
+
+def attn_combine(m, l, o, sink):
+    """Pieces of G disjoint row sets (m, l [G,B,T,H]; o [G,B,T,H,D]) -> attention output
+    [B,T,H,D] with the sink added once."""
+    lib = _load()
+    m, l, o = (np.ascontiguousarray(np.asarray(a, np.float64)) for a in (m, l, o))
+    G, B, T, H, D = o.shape
+    sk = _f32(sink)
+    out = np.empty((B, T, H, D))
+    for b in range(B):
+        ob = np.empty((T, H, D))
+        _check(lib.oracle_attn_combine(G, T, H, D, np.ascontiguousarray(m[:, b]), np.ascontiguousarray(l[:, b]),
+                                       np.ascontiguousarray(o[:, b]), sk, ob), "attn_combine")
+        out[b] = ob
+    return out
 
 
 def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale, ratio: int = 128, window: int = 128,

@@ -504,3 +504,79 @@ int oracle_hca_attn(const float *q, const float *kv, const float *swa, int64_t s
     free(rows); free(z);
     return ORC_OK;
 }
+
+/* ---- Attention over disjoint row sets, put back together.  The [HA] §6 probability
+ * p_i = e^{z_i} / (e^{z_s} + sum_j e^{z_j}) over a union of disjoint row sets splits
+ * into per-set pieces without the sink: m = max_j z_j (-inf if the set is empty),
+ * l = sum_j e^{z_j - m} (0 if empty), o = sum_j e^{z_j - m} row_j / l (0 if empty).
+ * sparse_attn's rows for one query restricted to one set: the SWA rows only if W > 0,
+ * and the entries kv[idx] with idx in [0, N).  q [T, H, D] -> m, l [T, H], o [T, H, D]. */
+int oracle_sparse_attn_partial(const float *q, const float *kv, const float *swa, int64_t swa_pos0, int W,
+                               const int64_t *q_pos, const int32_t *idx, int k, double scale, int window,
+                               int T, int H, int D, int64_t N, double *m, double *l, double *o)
+{
+    int64_t cap = (int64_t)k + window;
+    const float **rows = (const float **)malloc(sizeof(float *) * (cap > 0 ? cap : 1));
+    double *z = (double *)malloc(sizeof(double) * (cap > 0 ? cap : 1));
+    if (!rows || !z) { free(rows); free(z); return ORC_BAD; }
+    for (int t = 0; t < T; ++t) {
+        int64_t n = W > 0 ? orc_swa_rows(swa, swa_pos0, W, D, q_pos[t], window, rows) : 0;
+        for (int j = 0; j < k; ++j) {
+            int64_t i = idx[(int64_t)t * k + j];
+            if (i < 0 || i >= N) continue;
+            rows[n++] = kv + i * D;
+        }
+        for (int h = 0; h < H; ++h) {
+            const float *qh = q + ((int64_t)t * H + h) * D;
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < n; ++j) {
+                double dot = 0.0;
+                for (int e = 0; e < D; ++e) dot += (double)qh[e] * (double)rows[j][e];
+                z[j] = scale * dot;
+                if (z[j] > mx) mx = z[j];
+            }
+            double sum = 0.0;
+            for (int64_t j = 0; j < n; ++j) sum += exp(z[j] - mx);
+            double *oh = o + ((int64_t)t * H + h) * D;
+            for (int e = 0; e < D; ++e) oh[e] = 0.0;
+            for (int64_t j = 0; j < n; ++j) {
+                double p = exp(z[j] - mx) / sum;
+                for (int e = 0; e < D; ++e) oh[e] += p * (double)rows[j][e];
+            }
+            m[(int64_t)t * H + h] = mx;
+            l[(int64_t)t * H + h] = sum;
+        }
+    }
+    free(rows); free(z);
+    return ORC_OK;
+}
+
+/* The pieces of G disjoint row sets -> the attention output with the sink added once:
+ * M = max(z_s, m_g), den = e^{z_s - M} + sum_g l_g e^{m_g - M},
+ * out = sum_g l_g e^{m_g - M} o_g / den.  m, l [G, T, H]; o [G, T, H, D]; out [T, H, D]. */
+int oracle_attn_combine(int G, int T, int H, int D, const double *m, const double *l, const double *o,
+                        const float *sink, double *out)
+{
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h) {
+            double M = (double)sink[h];
+            for (int g = 0; g < G; ++g) {
+                double mg = m[((int64_t)g * T + t) * H + h];
+                if (mg > M) M = mg;
+            }
+            double den = exp((double)sink[h] - M);
+            for (int g = 0; g < G; ++g) {
+                int64_t gi = ((int64_t)g * T + t) * H + h;
+                if (l[gi] > 0.0) den += l[gi] * exp(m[gi] - M);
+            }
+            double *oh = out + ((int64_t)t * H + h) * D;
+            for (int e = 0; e < D; ++e) oh[e] = 0.0;
+            for (int g = 0; g < G; ++g) {
+                int64_t gi = ((int64_t)g * T + t) * H + h;
+                if (!(l[gi] > 0.0)) continue;
+                double wgt = l[gi] * exp(m[gi] - M) / den;
+                for (int e = 0; e < D; ++e) oh[e] += wgt * o[gi * D + e];
+            }
+        }
+    return ORC_OK;
+}

@@ -568,3 +568,85 @@ def test_kv8_error_bound_and_block_independence():
     np.testing.assert_array_equal(e2[:, :64], e[:, :64])
     np.testing.assert_array_equal(e2[:, 128:448], e[:, 128:448])
     assert np.all(e2[:, 580:584].view(np.float32) == e[:, 580:584].view(np.float32) * 16)
+
+
+# ----------------------------------------------------------------------------- sharded decode pieces
+@pytest.mark.parametrize("G", [1, 2, 3, 5])
+def test_partial_pieces_recombine_to_full_attention(G):
+    """Rows split into G disjoint sets (the SWA rows in set 0, memory rows by a contiguous
+    partition of the entries, some sets empty): combining the per-set (m, l, o) with the
+    sink added once gives the full attention, checked against the full oracle and against
+    torch scaled_dot_product_attention (float64) with the sink as an extra zero row."""
+    H, D, N, k, T = 4, 32, 60, 16, 2
+    q = rnd(1, T, H, D)
+    kv = rnd(1, N, D)
+    swa = rnd(1, 130, D)
+    sink = rnd(H)
+    q_pos, swa_pos0 = np.array([[400, 401]]), 400 - 127
+    idx = np.stack([np.sort(RNG.choice(N, k, replace=False)) for _ in range(T)]).astype(np.int32)[None]
+    idx[0, 1, -2:] = -1
+    scale = 1 / math.sqrt(D)
+    bounds = np.linspace(0, N, G + 1).astype(int)
+    if G == 3:
+        bounds = np.array([0, 0, 30, N])                 # an empty shard
+    ms, ls, os_ = [], [], []
+    for g in range(G):
+        part = np.where((idx >= bounds[g]) & (idx < bounds[g + 1]), idx, -1).astype(np.int32)
+        m, l, o = oracle.sparse_attn_partial(q, kv, swa, [swa_pos0], q_pos, part, scale, with_swa=(g == 0))
+        ms.append(m); ls.append(l); os_.append(o)
+    out = oracle.attn_combine(np.stack(ms), np.stack(ls), np.stack(os_), sink)
+    full = oracle.sparse_attn(q, kv, swa, [swa_pos0], q_pos, sink, idx, scale)
+    np.testing.assert_allclose(out, full, rtol=1e-12, atol=1e-13)
+    for t in range(T):
+        p = q_pos[0, t]
+        rows = np.concatenate([swa[0, (p - 127 - swa_pos0):(p - swa_pos0 + 1)], kv[0, [i for i in idx[0, t] if i >= 0]]])
+        np.testing.assert_allclose(out[0, t], _sdpa_with_sink(q[0, t], rows, sink, scale), rtol=1e-12, atol=1e-13)
+
+
+def test_partial_pieces_empty_set_and_single_set():
+    """An empty set gives m = -inf, l = 0, o = 0; a single set reproduces the softmax
+    without sink (o = sum softmax(z) row), and adding a sink of -inf changes nothing."""
+    H, D, N, T = 2, 16, 10, 1
+    q, kv, swa = rnd(1, T, H, D), rnd(1, N, D), rnd(1, 4, D)
+    idx = np.full((1, T, 3), -1, np.int32)
+    m, l, o = oracle.sparse_attn_partial(q, kv, swa, [1000], np.array([[5]]), idx, 0.3, with_swa=False)
+    assert np.all(m == -np.inf) and np.all(l == 0) and np.all(o == 0)
+    idx = np.array([[[1, 4, 7]]], np.int32)
+    m, l, o = oracle.sparse_attn_partial(q, kv, swa, [1000], np.array([[5]]), idx, 0.3, with_swa=False)
+    rows = kv[0, [1, 4, 7]].astype(np.float64)
+    z = 0.3 * q[0, 0].astype(np.float64) @ rows.T                       # [H, 3]
+    p = np.exp(z - z.max(1, keepdims=True))
+    np.testing.assert_allclose(o[0, 0], (p / p.sum(1, keepdims=True)) @ rows, rtol=1e-12)
+    np.testing.assert_allclose(m[0, 0], z.max(1), rtol=1e-14)
+    np.testing.assert_allclose(l[0, 0], p.sum(1), rtol=1e-14)
+    out = oracle.attn_combine(m[None], l[None], o[None], np.full(H, -np.inf, np.float32))
+    np.testing.assert_allclose(out, o, rtol=1e-14)
+
+
+@pytest.mark.parametrize("G", [2, 4])
+def test_sharded_topk_equals_full_topk(G):
+    """Local top-k of each contiguous shard, then the top-k of the gathered (score, global
+    index) lists taken in shard order, equals the top-k of the whole row, ties included
+    (the gathered list is ascending in global index, so the lower index still wins)."""
+    N, k = 4000, 300
+    s = (RNG.standard_normal((1, 2, N)) * 64).astype(np.float32)
+    s[0, 1, ::7] = 3.0                                    # many exact ties around the threshold
+    s[0, 1, 100:400] = 50.0
+    nv = np.array([[N, 3333]], np.int32)
+    full = oracle.topk(s, nv, k)
+    bounds = np.linspace(0, N, G + 1).astype(int)
+    cand_s, cand_i = [], []
+    for g in range(G):
+        lo, hi = bounds[g], bounds[g + 1]
+        nvl = np.clip(nv - lo, 0, hi - lo).astype(np.int32)
+        loc = oracle.topk(np.ascontiguousarray(s[..., lo:hi]), nvl, k)
+        sc = np.where(loc >= 0, np.take_along_axis(s[..., lo:hi], np.maximum(loc, 0), -1), -np.inf)
+        cand_s.append(sc.astype(np.float32)); cand_i.append(np.where(loc >= 0, loc + lo, -1))
+    cs, ci = np.concatenate(cand_s, -1), np.concatenate(cand_i, -1)
+    pos = oracle.topk(np.ascontiguousarray(cs), np.full((1, 2), cs.shape[-1], np.int32), k)
+    got = np.where(pos >= 0, np.take_along_axis(ci, np.maximum(pos, 0), -1), -1)
+    got = np.where(np.take_along_axis(cs, np.maximum(pos, 0), -1) == -np.inf, -1, got)
+    for t in range(2):
+        a = sorted(x for x in got[0, t] if x >= 0)
+        b = sorted(x for x in full[0, t] if x >= 0)
+        assert a == b
