@@ -47,6 +47,7 @@ enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2, CSA_BF16_KV8 = 3 };
 #define CSA_INDEX_DIM 128    /* dims per index head */
 #define CSA_SWA_WINDOW 128   /* SWA tokens per query ([HA] §6; [P1] window_size 128) */
 #define CSA_MAX_TOPK 2048
+#define CSA_MAX_SHARDS 16    /* GPUs one sequence's entries may be sharded over */
 
 /* Human-readable name of a status code (static string). */
 const char *csa_status_string(int status);
@@ -253,6 +254,62 @@ int sparse_attn(const void *q, const void *kv, const void *swa_kv, const int64_t
 int hca_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
              const int64_t *q_pos, const float *sink, int ratio, float scale, int B, int T, int H, int D, int64_t N,
              int dtype, void *out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Sharded decode of one long sequence over G GPUs (the compressed entries split into
+ * G contiguous ranges, one per GPU).  Per step, on every GPU g owning entries [lo, hi):
+ *   1. csa_index_scores + top-k over the local entries (local indices), the exact
+ *      scores of the local winners (csa_index_rerank's cand_scores), and their global
+ *      indices (csa_shard_remap);
+ *   2. all-gather of the (score, global index = local + lo) lists, shard-major
+ *      [G][B][k]; csa_shard_select -> the global top-k, the same on every GPU;
+ *   3. csa_shard_remap -> the winners inside [lo, hi) as local indices;
+ *      sparse_attn_partial over them (the SWA rows on one GPU only: W = 0 elsewhere);
+ *   4. all-gather of the partial results; csa_attn_combine adds the sink once.
+ * The attention identity behind 3-4: [HA] §6 p_i = e^{z_i} / (e^{z_s} + sum_j e^{z_j})
+ * over a union of disjoint row sets, put together from per-set pieces.
+ */
+
+/*
+ * sparse_attn_partial -- sparse_attn over this GPU's rows without the sink:
+ *   out[b,t,h,:] = sum_j e^{z_j - m} row_j / l,  l = sum_j e^{z_j - m},
+ *   ml[b,t,h] = (m, l) as two fp32 (natural-log units; m is a reference value near the
+ *   largest z, so m + ln(l) is the log-sum-exp of the z_j); no rows -> (-inf, 0), out 0.
+ *   Arguments as sparse_attn (no sink); W = 0 leaves the SWA rows out.
+ *   dtype CSA_BF16 or CSA_BF16_KV8 (CSA_F32: CSA_ERR_UNSUPPORTED).
+ *   out [B,T,H,D] bf16; ml [B,T,H,2] fp32, 8-byte aligned.
+ */
+int sparse_attn_partial(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
+                        const int64_t *q_pos, const int32_t *idx, int k, float scale, int B, int T, int H, int D,
+                        int64_t N, int dtype, void *out, float *ml, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * csa_attn_combine -- G partial results -> the attention output with the sink added once:
+ *   M = max(sink[h], m_g), den = e^{sink[h] - M} + sum_g l_g e^{m_g - M},
+ *   out = sum_g l_g e^{m_g - M} o_g / den   (pieces with l_g = 0 are skipped).
+ *   parts [G][B,T,H,D] bf16 (sparse_attn_partial outputs), ml [G][B,T,H,2] fp32,
+ *   sink [H] fp32, out [B,T,H,D] bf16; 1 <= G <= CSA_MAX_SHARDS, D a multiple of 8.
+ */
+int csa_attn_combine(const void *parts, const float *ml, const float *sink, int G, int B, int T, int H, int D,
+                     void *out, void *stream);
+
+/*
+ * csa_shard_select -- global top-k from the gathered per-GPU lists: scores [G][B][k]
+ * fp32 and global indices gidx [G][B][k] int32 (each list ascending, -1 padded; the
+ * shards in ascending entry order) -> idx [B][k], the k best by score, ties toward the
+ * lower global index (position order), padding entries never before a real one.
+ * workspace: csa_shard_select_workspace_size(G, B, k) bytes.  G * k <= 32768.
+ */
+size_t csa_shard_select_workspace_size(int G, int B, int k);
+int csa_shard_select(const float *scores, const int32_t *gidx, int G, int B, int k, int32_t *idx, void *workspace,
+                     size_t ws_bytes, void *stream);
+
+/*
+ * csa_shard_remap -- out[i] = in[i] - lo + add if lo <= in[i] < hi, else -1 (n entries,
+ * int32).  Global -> local indices: the shard's [lo, hi), add = 0; local -> global:
+ * lo = 0, hi = the shard's entry count, add = its first entry.
+ */
+int csa_shard_remap(const int32_t *in, int64_t n, int64_t lo, int64_t hi, int64_t add, int32_t *out, void *stream);
 
 /*
  * csa_launch_count -- number of kernels this library has enqueued in this

@@ -48,6 +48,12 @@ _SIGS = {
                      _vp, _vp, _sz, _vp], _i32),
     "hca_attn": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                   _vp, _vp, _sz, _vp], _i32),
+    "sparse_attn_partial": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
+                             _vp, _vp, _vp, _sz, _vp], _i32),
+    "csa_attn_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
+    "csa_shard_select_workspace_size": ([_i32, _i32, _i32], _sz),
+    "csa_shard_select": ([_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
+    "csa_shard_remap": ([_vp, _i64, _i64, _i64, _i64, _vp, _vp], _i32),
     "csa_launch_count": ([], ctypes.c_ulonglong),
     "csa_poll_status": ([_vp], _i32),
 }
@@ -288,6 +294,57 @@ def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int =
     _check(_lib.hca_attn(_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), ratio,
                          float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream)), "hca_attn")
+    return out
+
+
+def sparse_attn_partial(q, kv, swa_kv, swa_pos0, q_pos, idx, scale: float, *, with_swa: bool = True, out=None,
+                        ml=None, workspace=None, stream=None):
+    """sparse_attn over these rows without the sink -> (out [B,T,H,D] bf16, ml [B,T,H,2] fp32 (m, l))."""
+    B, T, H, D = q.shape
+    N, W, k = kv.shape[1], swa_kv.shape[1], idx.shape[2]
+    dt = _attn_dtype(q, kv)
+    if out is None:
+        out = torch.empty_like(q)
+    if ml is None:
+        ml = torch.empty((B, T, H, 2), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = attn_workspace(B, T, H, D, min(W, SWA_WINDOW) + k, dt, q.device)
+    _check(_lib.sparse_attn_partial(_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W if with_swa else 0,
+                                    _ptr(q_pos), _ptr(idx), k, float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(ml),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sparse_attn_partial")
+    return out, ml
+
+
+def attn_combine(parts, ml, sink, out=None, stream=None):
+    """parts [G,B,T,H,D] bf16, ml [G,B,T,H,2] fp32, sink [H] -> out [B,T,H,D] bf16 (sink added once)."""
+    G, B, T, H, D = parts.shape
+    if out is None:
+        out = torch.empty(parts.shape[1:], dtype=parts.dtype, device=parts.device)
+    _check(_lib.csa_attn_combine(_ptr(parts), _ptr(ml), _ptr(sink), G, B, T, H, D, _ptr(out), _stream(stream)),
+           "csa_attn_combine")
+    return out
+
+
+def shard_select(scores, gidx, k: int, idx=None, workspace=None, stream=None):
+    """Gathered lists scores / gidx [G,B,k] -> global top-k indices [B,k] (ties to the lower index)."""
+    G, B, kk = scores.shape
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    if workspace is None:
+        workspace = torch.empty(int(_lib.csa_shard_select_workspace_size(G, B, kk)), dtype=torch.uint8,
+                                device=scores.device)
+    _check(_lib.csa_shard_select(_ptr(scores), _ptr(gidx), G, B, kk, _ptr(idx), _ptr(workspace),
+                                 workspace.numel(), _stream(stream)), "csa_shard_select")
+    return idx
+
+
+def shard_remap(idx_in, lo: int, hi: int, add: int = 0, out=None, stream=None):
+    """out = idx_in - lo + add where lo <= idx_in < hi, else -1 (int32, any shape)."""
+    if out is None:
+        out = torch.empty_like(idx_in)
+    _check(_lib.csa_shard_remap(_ptr(idx_in), idx_in.numel(), int(lo), int(hi), int(add), _ptr(out),
+                                _stream(stream)), "csa_shard_remap")
     return out
 
 

@@ -43,6 +43,7 @@ namespace csa {
 constexpr int kSwaWindow = 128;
 constexpr int kMaxSplits = 16;   // CTAs of one query's cluster (sizes above 8 are non-portable)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 struct AttnParams {
   const void* q;          // [B, T, H, D]
@@ -57,6 +58,7 @@ struct AttnParams {
   int B, T, H, D, W, k, ratio, nsplit;
   int has_kvmap, has_swamap;   // tensor maps of kv [B, N, D] and swa_kv [B, W, D] were built
   int sparse;             // 1: memory rows from idx (sparse_attn); 0: dense prefix (hca_attn)
+  float* ml;              // [B, T, H, 2] or null: partial mode (no sink; write (m, l) per head)
   int64_t N;
 };
 
@@ -557,7 +559,8 @@ __global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __g
     const int h = threadIdx.x;                 // TMEM lane = head row
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const bool head_ok = h < QR && h0 + h < p.H;    // rows >= QR are the operand's filler
-    const float sinkL = head_ok ? p.sink[h0 + h] * kLog2e : 0.f;
+    // (partial mode: no sink, i.e. a sink logit of -inf)
+    const float sinkL = !head_ok ? 0.f : (p.ml ? -INFINITY : p.sink[h0 + h] * kLog2e);
     const float zs = p.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -651,10 +654,19 @@ __global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __g
     const bool have_o = ok && nt > 0 && mbar_wait(odone, 0);
     float g = 1.f;
     if (p.nsplit == 1) {
-      const float M = fmaxf(m_used, sinkL);
-      const float fo = (m_used == -INFINITY) ? 0.f : exp2f(m_used - M);
-      const float den = l * fo + exp2f(sinkL - M);
-      g = fo / den;
+      if (p.ml) {
+        // partial mode: O / l and (m, l) in natural-log units, l = sum_j e^(z_j - m)
+        g = (have_o && l > 0.f) ? 1.f / l : 0.f;
+        if (head_ok) {
+          float2* mlh = reinterpret_cast<float2*>(p.ml) + ((int64_t)qi * p.H + h0 + h);
+          *mlh = (have_o && l > 0.f) ? make_float2(m_used * kLn2, l) : make_float2(-INFINITY, 0.f);
+        }
+      } else {
+        const float M = fmaxf(m_used, sinkL);
+        const float fo = (m_used == -INFINITY) ? 0.f : exp2f(m_used - M);
+        const float den = l * fo + exp2f(sinkL - M);
+        g = fo / den;
+      }
     }
     if (h < QR) epi_g[h] = g;
     if (h == 0) epi_have_o = have_o ? 1 : 0;
@@ -742,7 +754,7 @@ __global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __g
     for (int hl = threadIdx.x; hl < he - hb; hl += blockDim.x) {
       const int hh = hb + hl;
       float mj[kMaxSplits], lj[kMaxSplits];
-      const float sinkL = (h0 + hh < p.H) ? p.sink[h0 + hh] * kLog2e : 0.f;
+      const float sinkL = (h0 + hh >= p.H) ? 0.f : (p.ml ? -INFINITY : p.sink[h0 + hh] * kLog2e);
       float M = sinkL;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
@@ -750,13 +762,17 @@ __global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __g
         lj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_l[hh]), (uint32_t)j)) : 0.f;
         M = fmaxf(M, mj[j]);
       }
-      float den = ex2_approx(sinkL - M);
+      const bool any = M > -INFINITY;                 // (partial mode: some split has rows)
+      float den = any ? ex2_approx(sinkL - M) : 0.f;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
-        mj[j] = ex2_approx(mj[j] - M);                // m = -inf (no rows) -> weight 0
+        mj[j] = any ? ex2_approx(mj[j] - M) : 0.f;    // m = -inf (no rows) -> weight 0
         den = fmaf(lj[j], mj[j], den);
       }
-      const float inv = 1.f / den;
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      if (p.ml && h0 + hh < p.H)
+        reinterpret_cast<float2*>(p.ml)[(int64_t)qi * p.H + h0 + hh] =
+            den > 0.f ? make_float2(M * kLn2, den) : make_float2(-INFINITY, 0.f);
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) cl_w[hh][j] = mj[j] * inv;
     }
@@ -804,6 +820,56 @@ __global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __g
   __syncthreads();
   tc_fence_after();
   if (warp == 8) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// ------------------------------------------------------------------ sharded decode
+// G partial results over disjoint row sets (sparse_attn_partial) -> the attention output,
+// with the sink added once ([HA] §6 probability over the union of the sets):
+// M = max(sink, m_g), den = e^(sink - M) + sum_g l_g e^(m_g - M),
+// out = sum_g l_g e^(m_g - M) o_g / den.  One warp per (query, head); 8 dims per 16-byte load.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* __restrict__ parts,
+                                                           const float2* __restrict__ ml,
+                                                           const float* __restrict__ sink, int G, int64_t rows,
+                                                           int H, int D, __nv_bfloat16* __restrict__ out) {
+  griddep_sync();
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int h = (int)(r % H);
+  const float sinkL = sink[h] * kLog2e;
+  float M = sinkL;
+  for (int g = 0; g < G; ++g) {
+    const float2 v = ml[(int64_t)g * rows + r];
+    if (v.y > 0.f) M = fmaxf(M, v.x * kLog2e);
+  }
+  float den = exp2f(sinkL - M);
+  for (int g = 0; g < G; ++g) {
+    const float2 v = ml[(int64_t)g * rows + r];
+    if (v.y > 0.f) den += v.y * exp2f(v.x * kLog2e - M);
+  }
+  const float inv = 1.f / den;
+  for (int c = lane_id(); c < D / 8; c += 32) {
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int g = 0; g < G; ++g) {
+      const float2 v = ml[(int64_t)g * rows + r];
+      if (!(v.y > 0.f)) continue;
+      const float wg = v.y * exp2f(v.x * kLog2e - M) * inv;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(parts + ((int64_t)g * rows + r) * D) + c);
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(hv[e]);
+        acc[2 * e] = fmaf(wg, x.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wg, x.y, acc[2 * e + 1]);
+      }
+    }
+    uint4 o;
+    __nv_bfloat162* ho = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ho[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+    reinterpret_cast<uint4*>(out + r * D)[c] = o;
+  }
 }
 
 }  // namespace csa

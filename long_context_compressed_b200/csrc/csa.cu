@@ -687,6 +687,73 @@ int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* s
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
 
+int sparse_attn_partial(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                        const int64_t* q_pos, const int32_t* idx, int k, float scale, int B, int T, int H, int D,
+                        int64_t N, int dtype, void* out, float* ml, void* workspace, size_t ws_bytes, void* stream) {
+  if (dtype != CSA_BF16 && dtype != CSA_BF16_KV8) return dtype == CSA_F32 ? CSA_ERR_UNSUPPORTED : CSA_ERR_INVALID;
+  // (the sink is not used here: pass a non-null stand-in to the common checks)
+  static const float no_sink = 0.f;
+  int rc = check_attn_common(q, kv, swa_kv, swa_pos0, W, q_pos, &no_sink, scale, B, T, H, D, N, dtype, out);
+  if (rc != CSA_OK || B == 0 || T == 0) return rc;
+  if (k < 0 || (k > 0 && !idx) || !ml || (reinterpret_cast<uintptr_t>(ml) & 7)) return CSA_ERR_INVALID;
+  AttnParams p{};
+  p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = nullptr;
+  p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale; p.ml = ml;
+  p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = k; p.ratio = 1; p.N = N; p.nsplit = 1;
+  const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k + (dtype == CSA_BF16_KV8 ? 31 : 0);
+  return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
+}
+
+int csa_attn_combine(const void* parts, const float* ml, const float* sink, int G, int B, int T, int H, int D,
+                     void* out, void* stream) {
+  if (G < 1 || G > CSA_MAX_SHARDS || B < 0 || T < 0 || H <= 0 || D <= 0 || D % 8 != 0) return CSA_ERR_INVALID;
+  const int64_t rows = (int64_t)B * T * H;
+  if (rows == 0) return CSA_OK;
+  if (!parts || !ml || !sink || !out || !aligned16(parts) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(ml) & 7))
+    return CSA_ERR_INVALID;
+  const int64_t blocks = (rows + 7) / 8;
+  if (blocks > INT32_MAX) return CSA_ERR_UNSUPPORTED;
+  launch_k(csa::attn_combine_kernel, (unsigned)blocks, 256, 0, as_stream(stream),
+           (const __nv_bfloat16*)parts, (const float2*)ml, sink, G, rows, H, D, (__nv_bfloat16*)out);
+  return launch_status();
+}
+
+size_t csa_shard_select_workspace_size(int G, int B, int k) {
+  if (G < 1 || B < 1 || k < 1) return 0;
+  return (size_t)G * B * k * 8;
+}
+
+int csa_shard_select(const float* scores, const int32_t* gidx, int G, int B, int k, int32_t* idx, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  if (G < 1 || G > CSA_MAX_SHARDS || B < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (B == 0) return CSA_OK;
+  const int64_t n = (int64_t)G * k;
+  if (n > csa::kRowSmemMax) return CSA_ERR_UNSUPPORTED;
+  if (!scores || !gidx || !idx || !workspace || ws_bytes < csa_shard_select_workspace_size(G, B, k))
+    return CSA_ERR_INVALID;
+  cudaStream_t st = as_stream(stream);
+  float* row_scores = static_cast<float*>(workspace);
+  int32_t* row_idx = reinterpret_cast<int32_t*>(row_scores + (size_t)B * n);
+  const int64_t total = (int64_t)B * n;
+  launch_k(csa::shard_gather_kernel, (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8), 256, 0,
+           st, scores, gidx, G, B, k, row_scores, row_idx);
+  const int smem = (int)std::max<int64_t>(4, n * 4);
+  if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
+  launch_k(csa::topk_row_kernel, (unsigned)B, 1024, smem, st, (const float*)row_scores, (const int32_t*)nullptr, n, k,
+           idx, (const int32_t*)row_idx);
+  return launch_status();
+}
+
+int csa_shard_remap(const int32_t* in, int64_t n, int64_t lo, int64_t hi, int64_t add, int32_t* out, void* stream) {
+  if (n < 0 || lo < 0 || hi < lo || hi > INT32_MAX || add < 0 || hi - lo + add > INT32_MAX) return CSA_ERR_INVALID;
+  if (n == 0) return CSA_OK;
+  if (!in || !out) return CSA_ERR_INVALID;
+  launch_k(csa::shard_remap_kernel, (unsigned)std::min<int64_t>((n + 255) / 256, (int64_t)sm_count() * 8), 256, 0,
+           as_stream(stream), in, n, lo, hi, add, out);
+  return launch_status();
+}
+
 unsigned long long csa_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

@@ -1152,4 +1152,36 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   }
 }
 
+// ---------------------------------------------------------------- sharded decode
+// The gathered per-shard lists, shard-major [G][B][k] (scores and global indices), as one
+// row per sequence [B][G * k]: in shard order the valid global indices are ascending, so a
+// top-k over positions keeps the lower-index tie rule.
+__global__ void __launch_bounds__(256) shard_gather_kernel(const float* __restrict__ scores,
+                                                           const int32_t* __restrict__ gidx, int G, int B, int k,
+                                                           float* __restrict__ row_scores,
+                                                           int32_t* __restrict__ row_idx) {
+  griddep_sync();
+  const int64_t n = (int64_t)G * B * k;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t g = i / ((int64_t)B * k), rem = i % ((int64_t)B * k);
+    const int64_t b = rem / k, j = rem % k;
+    const int64_t o = b * (int64_t)G * k + g * k + j;
+    const int32_t gi = gidx[i];
+    row_scores[o] = gi >= 0 ? scores[i] : -INFINITY;   // padding never outranks an entry
+    row_idx[o] = gi;
+  }
+}
+
+// Index remap between global and shard-local entry numbers: in in [lo, hi) ->
+// in - lo + add, else -1 (order kept).  Global -> local: (lo, hi) of the shard, add 0;
+// local -> global: (0, shard size), add = the shard's first entry.
+__global__ void __launch_bounds__(256) shard_remap_kernel(const int32_t* __restrict__ in, int64_t n, int64_t lo,
+                                                          int64_t hi, int64_t add, int32_t* __restrict__ out) {
+  griddep_sync();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t g = in[i];
+    out[i] = (g >= lo && g < hi) ? (int32_t)(g - lo + add) : -1;
+  }
+}
+
 }  // namespace csa
