@@ -259,13 +259,14 @@ int hca_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *s
  * Sharded decode of one long sequence over G GPUs (the compressed entries split into
  * G contiguous ranges, one per GPU).  Per step, on every GPU g owning entries [lo, hi):
  *   1. csa_index_scores + top-k over the local entries (local indices), the exact
- *      scores of the local winners (csa_index_rerank's cand_scores), and their global
- *      indices (csa_shard_remap);
- *   2. all-gather of the (score, global index = local + lo) lists, shard-major
- *      [G][B][k]; csa_shard_select -> the global top-k, the same on every GPU;
+ *      scores of the local winners (csa_index_rerank's cand_scores), and csa_shard_pack
+ *      -> (score, global index) pairs;
+ *   2. one all-gather of the pairs, shard-major [G][B][k]; csa_shard_select -> the
+ *      global top-k, the same on every GPU;
  *   3. csa_shard_remap -> the winners inside [lo, hi) as local indices;
- *      sparse_attn_partial over them (the SWA rows on one GPU only: W = 0 elsewhere);
- *   4. all-gather of the partial results; csa_attn_combine adds the sink once.
+ *      sparse_attn_partial over them (the SWA rows on one GPU only: W = 0 elsewhere),
+ *      its output and (m, l) written into one buffer;
+ *   4. one all-gather of those buffers; csa_attn_combine adds the sink once.
  * The attention identity behind 3-4: [HA] §6 p_i = e^{z_i} / (e^{z_s} + sum_j e^{z_j})
  * over a union of disjoint row sets, put together from per-set pieces.
  */
@@ -287,22 +288,33 @@ int sparse_attn_partial(const void *q, const void *kv, const void *swa_kv, const
  * csa_attn_combine -- G partial results -> the attention output with the sink added once:
  *   M = max(sink[h], m_g), den = e^{sink[h] - M} + sum_g l_g e^{m_g - M},
  *   out = sum_g l_g e^{m_g - M} o_g / den   (pieces with l_g = 0 are skipped).
- *   parts [G][B,T,H,D] bf16 (sparse_attn_partial outputs), ml [G][B,T,H,2] fp32,
- *   sink [H] fp32, out [B,T,H,D] bf16; 1 <= G <= CSA_MAX_SHARDS, D a multiple of 8.
+ *   Shard g's outputs o_g [B,T,H,D] bf16 start at parts + g * part_stride bytes and its
+ *   (m, l) [B,T,H,2] fp32 at ml + g * ml_stride bytes (e.g. one gathered buffer per shard:
+ *   the same stride for both); sink [H] fp32; out [B,T,H,D] bf16.
+ *   1 <= G <= CSA_MAX_SHARDS; D a multiple of 8; parts, out 16-byte aligned, part_stride a
+ *   multiple of 16, ml and ml_stride multiples of 8.
  */
-int csa_attn_combine(const void *parts, const float *ml, const float *sink, int G, int B, int T, int H, int D,
-                     void *out, void *stream);
+int csa_attn_combine(const void *parts, int64_t part_stride, const float *ml, int64_t ml_stride, const float *sink,
+                     int G, int B, int T, int H, int D, void *out, void *stream);
 
 /*
- * csa_shard_select -- global top-k from the gathered per-GPU lists: scores [G][B][k]
- * fp32 and global indices gidx [G][B][k] int32 (each list ascending, -1 padded; the
- * shards in ascending entry order) -> idx [B][k], the k best by score, ties toward the
- * lower global index (position order), padding entries never before a real one.
+ * csa_shard_pack -- this shard's winners as (score, global index) pairs: n entries,
+ *   loc[i] in [0, ns) -> (scores[i], loc[i] + lo); anything else -> (-inf, -1).
+ *   pairs: n x {fp32 score, int32 index}, 8-byte aligned.
+ */
+int csa_shard_pack(const float *scores, const int32_t *loc, int64_t n, int64_t ns, int64_t lo, void *pairs,
+                   void *stream);
+
+/*
+ * csa_shard_select -- global top-k from the gathered pairs [G][B][k] (csa_shard_pack's
+ * layout; each shard's list ascending, -1 padded; the shards in ascending entry order)
+ * -> idx [B][k], the k best by score, ties toward the lower global index (position
+ * order), padding never before a real entry.
  * workspace: csa_shard_select_workspace_size(G, B, k) bytes.  G * k <= 32768.
  */
 size_t csa_shard_select_workspace_size(int G, int B, int k);
-int csa_shard_select(const float *scores, const int32_t *gidx, int G, int B, int k, int32_t *idx, void *workspace,
-                     size_t ws_bytes, void *stream);
+int csa_shard_select(const void *pairs, int G, int B, int k, int32_t *idx, void *workspace, size_t ws_bytes,
+                     void *stream);
 
 /*
  * csa_shard_remap -- out[i] = in[i] - lo + add if lo <= in[i] < hi, else -1 (n entries,

@@ -50,9 +50,10 @@ _SIGS = {
                   _vp, _vp, _sz, _vp], _i32),
     "sparse_attn_partial": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                              _vp, _vp, _vp, _sz, _vp], _i32),
-    "csa_attn_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
+    "csa_attn_combine": ([_vp, _i64, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "csa_shard_select_workspace_size": ([_i32, _i32, _i32], _sz),
-    "csa_shard_select": ([_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
+    "csa_shard_pack": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp], _i32),
+    "csa_shard_select": ([_vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "csa_shard_remap": ([_vp, _i64, _i64, _i64, _i64, _vp, _vp], _i32),
     "csa_launch_count": ([], ctypes.c_ulonglong),
     "csa_poll_status": ([_vp], _i32),
@@ -317,25 +318,58 @@ def sparse_attn_partial(q, kv, swa_kv, swa_pos0, q_pos, idx, scale: float, *, wi
 
 
 def attn_combine(parts, ml, sink, out=None, stream=None):
-    """parts [G,B,T,H,D] bf16, ml [G,B,T,H,2] fp32, sink [H] -> out [B,T,H,D] bf16 (sink added once)."""
+    """parts [G,B,T,H,D] bf16 and ml [G,B,T,H,2] fp32 (stacked) -> out [B,T,H,D] bf16, the sink added once."""
     G, B, T, H, D = parts.shape
     if out is None:
         out = torch.empty(parts.shape[1:], dtype=parts.dtype, device=parts.device)
-    _check(_lib.csa_attn_combine(_ptr(parts), _ptr(ml), _ptr(sink), G, B, T, H, D, _ptr(out), _stream(stream)),
-           "csa_attn_combine")
+    _check(_lib.csa_attn_combine(_ptr(parts), parts[0].numel() * 2, _ptr(ml), ml[0].numel() * 4, _ptr(sink), G, B,
+                                 T, H, D, _ptr(out), _stream(stream)), "csa_attn_combine")
     return out
 
 
-def shard_select(scores, gidx, k: int, idx=None, workspace=None, stream=None):
-    """Gathered lists scores / gidx [G,B,k] -> global top-k indices [B,k] (ties to the lower index)."""
-    G, B, kk = scores.shape
+def attn_combine_packed(gathered, shape, sink, out=None, stream=None):
+    """gathered [G, nbytes] uint8, each row one shard's packed (output, (m, l)) buffer of
+    pack_partial_views(shape) -> out [B,T,H,D] bf16."""
+    G = gathered.shape[0]
+    B, T, H, D = shape
+    rows = B * T * H
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=gathered.device)
+    stride = gathered.shape[1]
+    base = gathered.data_ptr()
+    _check(_lib.csa_attn_combine(base, stride, base + rows * D * 2, stride, _ptr(sink), G, B, T, H, D, _ptr(out),
+                                 _stream(stream)), "csa_attn_combine")
+    return out
+
+
+def pack_partial_views(shape, device):
+    """One uint8 buffer holding a partial output [B,T,H,D] bf16 followed by its (m, l)
+    [B,T,H,2] fp32 -> (buffer, out view, ml view)."""
+    B, T, H, D = shape
+    ob = B * T * H * D * 2
+    buf = torch.empty(ob + B * T * H * 8, dtype=torch.uint8, device=device)
+    return buf, buf[:ob].view(torch.bfloat16).view(B, T, H, D), buf[ob:].view(torch.float32).view(B, T, H, 2)
+
+
+def shard_pack(scores, loc, ns: int, lo: int, pairs=None, stream=None):
+    """Winners (scores [..], local indices [..], same shape) -> pairs [.., 2] int32 (score bits, global index)."""
+    if pairs is None:
+        pairs = torch.empty(tuple(loc.shape) + (2,), dtype=torch.int32, device=loc.device)
+    _check(_lib.csa_shard_pack(_ptr(scores), _ptr(loc), loc.numel(), int(ns), int(lo), _ptr(pairs), _stream(stream)),
+           "csa_shard_pack")
+    return pairs
+
+
+def shard_select(pairs, k: int, idx=None, workspace=None, stream=None):
+    """Gathered pairs [G,B,kk,2] int32 (csa_shard_pack) -> global top-k indices [B,k] (ties to the lower index)."""
+    G, B, kk = pairs.shape[0], pairs.shape[1], pairs.shape[2]
     if idx is None:
-        idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+        idx = torch.empty((B, k), dtype=torch.int32, device=pairs.device)
     if workspace is None:
         workspace = torch.empty(int(_lib.csa_shard_select_workspace_size(G, B, kk)), dtype=torch.uint8,
-                                device=scores.device)
-    _check(_lib.csa_shard_select(_ptr(scores), _ptr(gidx), G, B, kk, _ptr(idx), _ptr(workspace),
-                                 workspace.numel(), _stream(stream)), "csa_shard_select")
+                                device=pairs.device)
+    _check(_lib.csa_shard_select(_ptr(pairs), G, B, kk, _ptr(idx), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "csa_shard_select")
     return idx
 
 

@@ -827,8 +827,10 @@ __global__ void __launch_bounds__(attn_threads(KV8), 1) attn_tc_kernel(const __g
 // with the sink added once ([HA] §6 probability over the union of the sets):
 // M = max(sink, m_g), den = e^(sink - M) + sum_g l_g e^(m_g - M),
 // out = sum_g l_g e^(m_g - M) o_g / den.  One warp per (query, head); 8 dims per 16-byte load.
-__global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* __restrict__ parts,
-                                                           const float2* __restrict__ ml,
+// Shard g's output rows start at parts + g * part_stride bytes and its (m, l) at
+// ml + g * ml_stride bytes (one gathered buffer per shard, or two stacked arrays).
+__global__ void __launch_bounds__(256) attn_combine_kernel(const uint8_t* __restrict__ parts_b, int64_t part_stride,
+                                                           const uint8_t* __restrict__ ml_b, int64_t ml_stride,
                                                            const float* __restrict__ sink, int G, int64_t rows,
                                                            int H, int D, __nv_bfloat16* __restrict__ out) {
   griddep_sync();
@@ -837,13 +839,14 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* 
   const int h = (int)(r % H);
   const float sinkL = sink[h] * kLog2e;
   float M = sinkL;
+  auto mlg = [&](int g) { return reinterpret_cast<const float2*>(ml_b + (int64_t)g * ml_stride)[r]; };
   for (int g = 0; g < G; ++g) {
-    const float2 v = ml[(int64_t)g * rows + r];
+    const float2 v = mlg(g);
     if (v.y > 0.f) M = fmaxf(M, v.x * kLog2e);
   }
   float den = exp2f(sinkL - M);
   for (int g = 0; g < G; ++g) {
-    const float2 v = ml[(int64_t)g * rows + r];
+    const float2 v = mlg(g);
     if (v.y > 0.f) den += v.y * exp2f(v.x * kLog2e - M);
   }
   const float inv = 1.f / den;
@@ -852,10 +855,10 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* 
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     for (int g = 0; g < G; ++g) {
-      const float2 v = ml[(int64_t)g * rows + r];
+      const float2 v = mlg(g);
       if (!(v.y > 0.f)) continue;
       const float wg = v.y * exp2f(v.x * kLog2e - M) * inv;
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(parts + ((int64_t)g * rows + r) * D) + c);
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(parts_b + (int64_t)g * part_stride + r * D * 2) + c);
       const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

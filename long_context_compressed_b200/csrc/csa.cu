@@ -704,18 +704,19 @@ int sparse_attn_partial(const void* q, const void* kv, const void* swa_kv, const
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
 
-int csa_attn_combine(const void* parts, const float* ml, const float* sink, int G, int B, int T, int H, int D,
-                     void* out, void* stream) {
+int csa_attn_combine(const void* parts, int64_t part_stride, const float* ml, int64_t ml_stride, const float* sink,
+                     int G, int B, int T, int H, int D, void* out, void* stream) {
   if (G < 1 || G > CSA_MAX_SHARDS || B < 0 || T < 0 || H <= 0 || D <= 0 || D % 8 != 0) return CSA_ERR_INVALID;
   const int64_t rows = (int64_t)B * T * H;
   if (rows == 0) return CSA_OK;
   if (!parts || !ml || !sink || !out || !aligned16(parts) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(ml) & 7))
+      (reinterpret_cast<uintptr_t>(ml) & 7) || (G > 1 && ((part_stride & 15) || (ml_stride & 7))) ||
+      (G > 1 && (part_stride < rows * D * 2 || ml_stride < rows * 8)))
     return CSA_ERR_INVALID;
   const int64_t blocks = (rows + 7) / 8;
   if (blocks > INT32_MAX) return CSA_ERR_UNSUPPORTED;
-  launch_k(csa::attn_combine_kernel, (unsigned)blocks, 256, 0, as_stream(stream),
-           (const __nv_bfloat16*)parts, (const float2*)ml, sink, G, rows, H, D, (__nv_bfloat16*)out);
+  launch_k(csa::attn_combine_kernel, (unsigned)blocks, 256, 0, as_stream(stream), (const uint8_t*)parts, part_stride,
+           (const uint8_t*)ml, ml_stride, sink, G, rows, H, D, (__nv_bfloat16*)out);
   return launch_status();
 }
 
@@ -724,20 +725,31 @@ size_t csa_shard_select_workspace_size(int G, int B, int k) {
   return (size_t)G * B * k * 8;
 }
 
-int csa_shard_select(const float* scores, const int32_t* gidx, int G, int B, int k, int32_t* idx, void* workspace,
-                     size_t ws_bytes, void* stream) {
+int csa_shard_pack(const float* scores, const int32_t* loc, int64_t n, int64_t ns, int64_t lo, void* pairs,
+                   void* stream) {
+  if (n < 0 || ns < 0 || lo < 0 || lo + ns > INT32_MAX) return CSA_ERR_INVALID;
+  if (n == 0) return CSA_OK;
+  if (!scores || !loc || !pairs || (reinterpret_cast<uintptr_t>(pairs) & 7)) return CSA_ERR_INVALID;
+  launch_k(csa::shard_pack_kernel, (unsigned)std::min<int64_t>((n + 255) / 256, (int64_t)sm_count() * 8), 256, 0,
+           as_stream(stream), scores, loc, n, ns, lo, (csa::ShardPair*)pairs);
+  return launch_status();
+}
+
+int csa_shard_select(const void* pairs, int G, int B, int k, int32_t* idx, void* workspace, size_t ws_bytes,
+                     void* stream) {
   if (G < 1 || G > CSA_MAX_SHARDS || B < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
   if (B == 0) return CSA_OK;
   const int64_t n = (int64_t)G * k;
   if (n > csa::kRowSmemMax) return CSA_ERR_UNSUPPORTED;
-  if (!scores || !gidx || !idx || !workspace || ws_bytes < csa_shard_select_workspace_size(G, B, k))
+  if (!pairs || !idx || !workspace || ws_bytes < csa_shard_select_workspace_size(G, B, k) ||
+      (reinterpret_cast<uintptr_t>(pairs) & 7))
     return CSA_ERR_INVALID;
   cudaStream_t st = as_stream(stream);
   float* row_scores = static_cast<float*>(workspace);
   int32_t* row_idx = reinterpret_cast<int32_t*>(row_scores + (size_t)B * n);
   const int64_t total = (int64_t)B * n;
   launch_k(csa::shard_gather_kernel, (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8), 256, 0,
-           st, scores, gidx, G, B, k, row_scores, row_idx);
+           st, (const csa::ShardPair*)pairs, G, B, k, row_scores, row_idx);
   const int smem = (int)std::max<int64_t>(4, n * 4);
   if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
   launch_k(csa::topk_row_kernel, (unsigned)B, 1024, smem, st, (const float*)row_scores, (const int32_t*)nullptr, n, k,

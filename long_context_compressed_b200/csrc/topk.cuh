@@ -1153,11 +1153,29 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
 }
 
 // ---------------------------------------------------------------- sharded decode
-// The gathered per-shard lists, shard-major [G][B][k] (scores and global indices), as one
-// row per sequence [B][G * k]: in shard order the valid global indices are ascending, so a
-// top-k over positions keeps the lower-index tie rule.
-__global__ void __launch_bounds__(256) shard_gather_kernel(const float* __restrict__ scores,
-                                                           const int32_t* __restrict__ gidx, int G, int B, int k,
+// One shard's k best entries as (score, global index) pairs, the unit every GPU
+// contributes to the all-gather: local index i in [0, ns) -> (score, i + lo); -1 ->
+// (-inf, -1).
+struct ShardPair {
+  float score;
+  int32_t gidx;
+};
+
+__global__ void __launch_bounds__(256) shard_pack_kernel(const float* __restrict__ scores,
+                                                         const int32_t* __restrict__ loc, int64_t n, int64_t ns,
+                                                         int64_t lo, ShardPair* __restrict__ pairs) {
+  griddep_sync();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t l = loc[i];
+    const bool ok = l >= 0 && l < ns;
+    pairs[i] = ok ? ShardPair{scores[i], (int32_t)(l + lo)} : ShardPair{-INFINITY, -1};
+  }
+}
+
+// The gathered pairs, shard-major [G][B][k], as one row per sequence [B][G * k] of scores
+// and global indices: in shard order the valid global indices are ascending, so a top-k
+// over positions keeps the lower-index tie rule.
+__global__ void __launch_bounds__(256) shard_gather_kernel(const ShardPair* __restrict__ pairs, int G, int B, int k,
                                                            float* __restrict__ row_scores,
                                                            int32_t* __restrict__ row_idx) {
   griddep_sync();
@@ -1166,9 +1184,9 @@ __global__ void __launch_bounds__(256) shard_gather_kernel(const float* __restri
     const int64_t g = i / ((int64_t)B * k), rem = i % ((int64_t)B * k);
     const int64_t b = rem / k, j = rem % k;
     const int64_t o = b * (int64_t)G * k + g * k + j;
-    const int32_t gi = gidx[i];
-    row_scores[o] = gi >= 0 ? scores[i] : -INFINITY;   // padding never outranks an entry
-    row_idx[o] = gi;
+    const ShardPair pr = pairs[i];
+    row_scores[o] = pr.gidx >= 0 ? pr.score : -INFINITY;   // padding never outranks an entry
+    row_idx[o] = pr.gidx;
   }
 }
 

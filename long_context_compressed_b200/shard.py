@@ -7,14 +7,14 @@ library's kernels; this module only orders the calls and the exchanges):
 1. the indexer over the local entries, the local top-k (e4m3 scores, exact bf16
    rescoring of the kc = 2k candidates as in the single-GPU step), the exact scores of
    the local winners and their global entry numbers;
-2. one all-gather of the (score, global index) lists, then the global top-k
+2. one all-gather of the (score, global index) pairs, then the global top-k
    (csa_shard_select), the same on every GPU.  Every global winner is a local winner of
    its shard, so the gathered lists hold the whole-row top-k, and with the shards in
    entry order the lower-index tie rule still holds;
 3. the winners inside [lo, hi) as local indices, and the attention over them without
    the sink (sparse_attn_partial); the SWA rows are attended on GPU 0 only;
-4. one all-gather of the partial results, then csa_attn_combine adds the sink once and
-   every GPU holds the output.
+4. one all-gather of the partial results (output and (m, l) in one buffer), then
+   csa_attn_combine adds the sink once and every GPU holds the output.
 
 The identity behind 3-4 is the attention-sink probability of "DeepSeek-V4 混合注意力：
 从压缩记忆到百万上下文" §6 over a union of disjoint row sets.  The exchanges go through an
@@ -89,7 +89,7 @@ class GpuKernels:
         return t
 
     def local_topk(self, sh: Shard, qI, w):
-        """(scores [B, k] fp32, global indices [B, k] int32) of the shard's k best entries."""
+        """The shard's k best entries as (score, global index) pairs [B, k, 2] int32."""
         from . import csa
         B, Ns, dev, k = sh.kI.shape[0], sh.kI.shape[1], sh.kI.device, self.k
         if sh.k8 is None:
@@ -107,33 +107,34 @@ class GpuKernels:
         exact = self._b("exact", (B, 1, k), torch.float32, dev)
         kept = self._b("kept", (B, 1, k), torch.int32, dev)
         csa.csa_index_rerank(qI, w, sh.kI, loc, k, cand_scores=exact, idx=kept)
-        gidx = csa.shard_remap(loc, 0, Ns, sh.lo, out=self._b("gidx", (B, 1, k), torch.int32, dev))
-        return exact.view(B, k), gidx.view(B, k)
+        pairs = csa.shard_pack(exact, loc, Ns, sh.lo, pairs=self._b("pairs", (B, k, 2), torch.int32, dev))
+        return pairs
 
-    def attend(self, sh: Shard, q, all_scores, all_gidx):
-        """This shard's part of the attention over the global top-k -> (part, ml)."""
+    def attend(self, sh: Shard, q, all_pairs):
+        """This shard's part of the attention over the global top-k, written into one
+        buffer (output, then (m, l)) -> uint8 [nbytes]."""
         from . import csa
         B, dev, k = q.shape[0], q.device, self.k
-        g = csa.shard_select(all_scores, all_gidx, k, idx=self._b("glob", (B, k), torch.int32, dev))
+        g = csa.shard_select(all_pairs, k, idx=self._b("glob", (B, k), torch.int32, dev))
         loc = csa.shard_remap(g, sh.lo, sh.hi, 0, out=self._b("sel", (B, 1, k), torch.int32, dev))
-        return csa.sparse_attn_partial(q, sh.kv, sh.swa, sh.swa_pos0, sh.q_pos, loc, self.scale,
-                                       with_swa=(sh.rank == 0))
+        if "part" not in self.buf or self.buf["part"][1].shape != q.shape:
+            self.buf["part"] = csa.pack_partial_views(tuple(q.shape), dev)
+        buf, out, ml = self.buf["part"]
+        csa.sparse_attn_partial(q, sh.kv, sh.swa, sh.swa_pos0, sh.q_pos, loc, self.scale, with_swa=(sh.rank == 0),
+                                out=out, ml=ml)
+        return buf
 
-    def combine(self, sh: Shard, parts, mls):
+    def combine(self, sh: Shard, gathered, shape):
         from . import csa
-        return csa.attn_combine(parts, mls, sh.sink)
+        return csa.attn_combine_packed(gathered, shape, sh.sink)
 
 
 def decode_step(sh: Shard, kernels, exchange, q, qI, w):
     """One decode step of the sharded sequence(s) on this GPU; returns the full output
-    [B, 1, H, D] (identical on every GPU)."""
-    scores, gidx = kernels.local_topk(sh, qI, w)
-    all_scores = exchange.all_gather(scores)
-    all_gidx = exchange.all_gather(gidx)
-    part, ml = kernels.attend(sh, q, all_scores, all_gidx)
-    parts = exchange.all_gather(part)
-    mls = exchange.all_gather(ml)
-    return kernels.combine(sh, parts, mls)
+    [B, 1, H, D] (identical on every GPU).  Two all-gathers per step."""
+    pairs = kernels.local_topk(sh, qI, w)
+    part = kernels.attend(sh, q, exchange.all_gather(pairs))
+    return kernels.combine(sh, exchange.all_gather(part), tuple(q.shape))
 
 
 def default_scale(D: int) -> float:

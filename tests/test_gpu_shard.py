@@ -88,9 +88,8 @@ def test_shard_select_and_remap(csa, G, k):
         loc = oracle.topk(np.ascontiguousarray(s[..., lo:hi]), nvl, k)[:, 0]
         cs.append(np.where(loc >= 0, np.take_along_axis(s[:, 0, lo:hi], np.maximum(loc, 0), -1), -np.inf))
         ci.append(np.where(loc >= 0, loc + lo, -1))
-    cs = torch.from_numpy(np.stack(cs).astype(np.float32)).cuda()
-    ci = torch.from_numpy(np.stack(ci).astype(np.int32)).cuda()
-    got = csa.shard_select(cs, ci, k).cpu().numpy()
+    pairs = np.stack([np.stack(cs).astype(np.float32).view(np.int32), np.stack(ci).astype(np.int32)], -1)
+    got = csa.shard_select(torch.from_numpy(pairs).cuda(), k).cpu().numpy()
     ref = oracle.topk(s, nv, k)[:, 0]
     for b in range(B):
         assert sorted(x for x in got[b] if x >= 0) == sorted(x for x in ref[b] if x >= 0)
@@ -99,6 +98,11 @@ def test_shard_select_and_remap(csa, G, k):
     np.testing.assert_array_equal(loc, np.where((ref >= lo) & (ref < hi), ref - lo, -1))
     back = csa.shard_remap(torch.from_numpy(loc).cuda(), 0, hi - lo, lo).cpu().numpy()
     np.testing.assert_array_equal(back, np.where((ref >= lo) & (ref < hi), ref, -1))
+    sc = rng.standard_normal(loc.shape).astype(np.float32)
+    pk = csa.shard_pack(torch.from_numpy(sc).cuda(), torch.from_numpy(loc).cuda(), hi - lo, lo).cpu().numpy()
+    ok = loc >= 0
+    np.testing.assert_array_equal(pk[..., 1], np.where(ok, loc + lo, -1))
+    np.testing.assert_array_equal(np.ascontiguousarray(pk[..., 0]).view(np.float32), np.where(ok, sc, -np.inf))
 
 
 @pytest.mark.parametrize("G", [1, 2, 4])
@@ -122,11 +126,9 @@ def test_sharded_decode_emulated(csa, G):
                                   n_valid=shard.local_n_valid(nv, lo, hi).cuda()))
         kern.append(shard.GpuKernels(k, scale))
     qI, w, q = ix["qI"].cuda(), ix["w"].cuda(), at["q"].cuda()
-    lt = [kern[g].local_topk(shards[g], qI, w) for g in range(G)]
-    all_s = torch.stack([a for a, _ in lt])
-    all_i = torch.stack([b for _, b in lt])
-    att = [kern[g].attend(shards[g], q, all_s, all_i) for g in range(G)]
-    out = kern[0].combine(shards[0], torch.stack([a for a, _ in att]), torch.stack([b for _, b in att]))
+    all_pairs = torch.stack([kern[g].local_topk(shards[g], qI, w) for g in range(G)])      # the first all-gather
+    gathered = torch.stack([kern[g].attend(shards[g], q, all_pairs).clone() for g in range(G)])  # the second
+    out = kern[0].combine(shards[0], gathered, tuple(q.shape))
     glob = kern[0].buf["glob"].cpu().numpy()
     s_ref, smag = oracle.index_scores(_np(ix["qI"]), ix["w"].numpy(), _np(ix["kI"]), nv.numpy(), with_mag=True)
     for b in range(B):

@@ -32,25 +32,31 @@ class OracleKernels:
         import oracle
         s = oracle.index_scores(qI.numpy(), w.numpy(), sh.kI.numpy(), sh.n_valid.numpy())
         loc = oracle.topk(s.astype(np.float32), sh.n_valid.numpy(), self.k)[:, 0]     # [B, k]
-        sc = np.where(loc >= 0, np.take_along_axis(s[:, 0], np.maximum(loc, 0), -1), -np.inf)
-        return torch.from_numpy(sc.astype(np.float32)), torch.from_numpy(np.where(loc >= 0, loc + sh.lo, -1).astype(np.int32))
+        sc = np.where(loc >= 0, np.take_along_axis(s[:, 0], np.maximum(loc, 0), -1), -np.inf).astype(np.float32)
+        gi = np.where(loc >= 0, loc + sh.lo, -1).astype(np.int32)
+        return torch.from_numpy(np.stack([sc.view(np.int32), gi], -1))             # (score bits, index)
 
-    def attend(self, sh, q, all_scores, all_gidx):
+    def attend(self, sh, q, all_pairs):
         import oracle
-        G, B, k = all_scores.shape
-        cs = all_scores.permute(1, 0, 2).reshape(B, 1, G * k).numpy()
-        ci = all_gidx.permute(1, 0, 2).reshape(B, 1, G * k).numpy()
+        G, B, k, _ = all_pairs.shape
+        ap = all_pairs.numpy()
+        cs = np.ascontiguousarray(ap[..., 0]).view(np.float32).transpose(1, 0, 2).reshape(B, 1, G * k)
+        ci = ap[..., 1].transpose(1, 0, 2).reshape(B, 1, G * k)
         pos = oracle.topk(np.ascontiguousarray(cs), np.full((B, 1), G * k, np.int32), k)
         glob = np.where(pos >= 0, np.take_along_axis(ci, np.maximum(pos, 0), -1), -1)
         loc = np.where((glob >= sh.lo) & (glob < sh.hi), glob - sh.lo, -1).astype(np.int32)
         m, l, o = oracle.sparse_attn_partial(q.numpy(), sh.kv.numpy(), sh.swa.numpy(), sh.swa_pos0.numpy(),
                                              sh.q_pos.numpy(), loc, self.scale, with_swa=(sh.rank == 0))
-        return torch.from_numpy(o), torch.from_numpy(np.stack([m, l], -1))
+        return torch.from_numpy(np.concatenate([o.reshape(-1), np.stack([m, l], -1).reshape(-1)]))
 
-    def combine(self, sh, parts, mls):
+    def combine(self, sh, gathered, shape):
         import oracle
-        return torch.from_numpy(oracle.attn_combine(mls[..., 0].numpy(), mls[..., 1].numpy(), parts.numpy(),
-                                                    sh.sink.numpy()))
+        B, T, H, D = shape
+        n = B * T * H * D
+        g = gathered.numpy()
+        o = g[:, :n].reshape((-1,) + tuple(shape))
+        ml = g[:, n:].reshape(-1, B, T, H, 2)
+        return torch.from_numpy(oracle.attn_combine(ml[..., 0], ml[..., 1], o, sh.sink.numpy()))
 
 
 def _inputs(B=2, N=900, H=8, D=64, W=140, seed=3):
