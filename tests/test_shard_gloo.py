@@ -93,7 +93,7 @@ def _worker(rank, world, port, k, out):
 def test_sharded_decode_equals_whole_sequence(world):
     import oracle
     k = 64
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, _free_port(), k, out), nprocs=world, join=True)
     x = _inputs()
     s = oracle.index_scores(x["qI"].numpy(), x["w"].numpy(), x["kI"].numpy(), x["n_valid"].numpy())
