@@ -226,6 +226,23 @@ def draw_indexer(wl: Workload, seed: int = 0, device="cpu", N=None):
     return {"qI": qI, "w": w, "kI": kI}
 
 
+def draw_indexer_outliers(seed: int, B: int, T: int, N: int, Hi: int = 64, di: int = 128,
+                          channels=(3, 40, 77, 100), key_offset: float = 20.0, q_gain: float = 8.0,
+                          device="cpu"):
+    """Index inputs with outlier channels, the regime a rotation before low-precision
+    scoring is for: N(0,1) draws, then on the given channels every key gets a common
+    offset and every query head a larger gain; bf16 storage.  w ~ N(0, 0.1^2) fp32.
+    Returns {"qI" [B,T,Hi,di], "w" [B,T,Hi], "kI" [B,N,di]}."""
+    tag = f"outliers/{B}x{T}x{N}"
+    qI = normal(seed, f"{tag}/qI", (B, T, Hi, di), device=device)
+    kI = normal(seed, f"{tag}/kI", (B, N, di), device=device)
+    ch = torch.tensor(list(channels), dtype=torch.long, device=device)
+    kI[..., ch] += key_offset
+    qI[..., ch] *= q_gain
+    w = normal(seed, f"{tag}/w", (B, T, Hi), std=0.1, device=device)
+    return {"qI": store(qI, "bf16"), "w": w, "kI": store(kI, "bf16")}
+
+
 def draw_attention(wl: Workload, seed: int = 0, device="cpu", N=None, tag="attn"):
     """Queries q [B,T,H,D], latent cache kv [B,N,D], raw SWA rows swa_kv [B,W,D]
     (absolute positions swa_pos0..swa_pos0+W-1), per-head sink logits [H] (fp32)."""

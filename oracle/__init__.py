@@ -18,7 +18,8 @@ cited in ``oracle.c``:
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
 (tests/test_oracle_pins.py) except the FP8 *recall* statistic, which the pages
 do not fix ("parity unpinned" for recall only; the e4m3 codec, the FP8 score
-definition and the mixed-precision KV storage codec are pinned).
+definition, the Hadamard rotation of the index vectors and the mixed-precision KV
+storage codec are pinned).
 """
 from __future__ import annotations
 
@@ -69,6 +70,8 @@ def _load():
     lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_quantize_rows_e4m3.argtypes = [_f32p, i64, i32, _u8p, _f32p]
+    lib.oracle_hadamard_rotate.argtypes = [_f64p, i64, i32, _f64p]
+    lib.oracle_quantize_rows_e4m3_hadamard.argtypes = [_f32p, i64, i32, _u8p, _f32p]
     lib.oracle_sparse_attn_partial.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _i32p, i32, dbl, i32,
                                                i32, i32, i32, i64, _f64p, _f64p, _f64p]
     lib.oracle_attn_combine.argtypes = [i32, i32, i32, i32, _f64p, _f64p, _f64p, _f32p, _f64p]
@@ -82,7 +85,8 @@ def _load():
     lib.oracle_hca_attn.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _f32p, i32, dbl, i32,
                                     i32, i32, i32, i64, _f64p, _f64p]
     for name in ("oracle_compress_csa", "oracle_compress_hca", "oracle_index_scores",
-                 "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_kv8_quantize",
+                 "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_hadamard_rotate",
+                 "oracle_quantize_rows_e4m3_hadamard", "oracle_kv8_quantize",
                  "oracle_kv8_dequantize", "oracle_sparse_attn_partial", "oracle_attn_combine", "oracle_topk",
                  "oracle_sparse_attn", "oracle_hca_attn"):
         getattr(lib, name).restype = ctypes.c_int
@@ -219,6 +223,28 @@ def quantize_rows_e4m3(x):
     codes = np.empty(x.shape, np.uint8)
     scale = np.empty(x.shape[:-1], np.float32)
     _check(lib.oracle_quantize_rows_e4m3(x, rows, cols, codes, scale), "quantize_rows_e4m3")
+    return codes, scale
+
+
+def hadamard_rotate(x):
+    """Orthonormal Sylvester Walsh-Hadamard rotation of the last axis ([P1], Indexer
+    paragraph).  x [..., n], n a power of two -> float64 [..., n]."""
+    lib = _load()
+    x = np.ascontiguousarray(np.asarray(x, np.float64))
+    n = x.shape[-1]
+    y = np.empty(x.shape, np.float64)
+    _check(lib.oracle_hadamard_rotate(x, x.size // n if n else 0, n, y), "hadamard_rotate")
+    return y
+
+
+def quantize_rows_e4m3_hadamard(x):
+    """Rotate each row, round to fp32, then quantize_rows_e4m3.  x [..., n] -> (codes u8, scale f32)."""
+    lib = _load()
+    x = _f32(x)
+    n = x.shape[-1]
+    codes = np.empty(x.shape, np.uint8)
+    scale = np.empty(x.shape[:-1], np.float32)
+    _check(lib.oracle_quantize_rows_e4m3_hadamard(x, x.size // n, n, codes, scale), "quantize_rows_e4m3_hadamard")
     return codes, scale
 
 

@@ -238,6 +238,63 @@ int oracle_quantize_rows_e4m3(const float *x, int64_t rows, int cols, uint8_t *c
     return ORC_OK;
 }
 
+/* ---- Hadamard rotation of the index vectors ([P1], the paragraph on the
+ * Indexer: the index query passes through RoPE and a Hadamard rotation before
+ * its dot products with the compressed keys).  Readings: the rotation is the
+ * orthonormal Sylvester-ordered Walsh-Hadamard matrix R = H_n / sqrt(n), with
+ * H_1 = [1] and H_2m = [[H_m, H_m], [H_m, -H_m]]; the index keys get the same
+ * rotation, so <Rq, Rk> = <q, k> and the scores keep their meaning; it comes
+ * before the e4m3 quantisation, as an aid to it.
+ * x, y: [rows, n] double, n a power of two <= 1024.  y = R x, summed in
+ * double in index order, then multiplied by c = 1 / sqrt(n) (both IEEE
+ * double, round to nearest). */
+static int orc_is_pow2(int n) { return n > 0 && (n & (n - 1)) == 0; }
+
+int oracle_hadamard_rotate(const double *x, int64_t rows, int n, double *y)
+{
+    if (!orc_is_pow2(n) || n > 1024 || rows < 0) return ORC_BAD;
+    signed char *H = (signed char *)malloc((size_t)n * n);
+    if (!H) return ORC_BAD;
+    H[0] = 1;
+    for (int m = 1; m < n; m *= 2)          /* Sylvester doubling of the m x m block */
+        for (int i = 0; i < m; ++i)
+            for (int j = 0; j < m; ++j) {
+                signed char h = H[(size_t)i * n + j];
+                H[(size_t)i * n + (j + m)] = h;
+                H[(size_t)(i + m) * n + j] = h;
+                H[(size_t)(i + m) * n + (j + m)] = (signed char)-h;
+            }
+    const double c = 1.0 / sqrt((double)n);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int i = 0; i < n; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < n; ++j) acc += H[(size_t)i * n + j] * x[r * n + j];
+            y[r * n + i] = acc * c;
+        }
+    free(H);
+    return ORC_OK;
+}
+
+/* Rotated e4m3 quantisation: each row is rotated (oracle_hadamard_rotate on the
+ * row widened to double), rounded to fp32, then quantised exactly as in
+ * oracle_quantize_rows_e4m3.  x [rows, n] float -> codes [rows, n], scale [rows]. */
+int oracle_quantize_rows_e4m3_hadamard(const float *x, int64_t rows, int n, uint8_t *codes, float *scale)
+{
+    if (!orc_is_pow2(n) || n > 1024 || rows < 0) return ORC_BAD;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)n);
+    double *yd = (double *)malloc(sizeof(double) * (size_t)n);
+    float *yf = (float *)malloc(sizeof(float) * (size_t)n);
+    int rc = (xd && yd && yf) ? ORC_OK : ORC_BAD;
+    for (int64_t r = 0; r < rows && rc == ORC_OK; ++r) {
+        for (int j = 0; j < n; ++j) xd[j] = x[r * n + j];
+        rc = oracle_hadamard_rotate(xd, 1, n, yd);
+        for (int j = 0; j < n; ++j) yf[j] = (float)yd[j];
+        if (rc == ORC_OK) rc = oracle_quantize_rows_e4m3(yf, 1, n, codes + r * n, scale + r);
+    }
+    free(xd); free(yd); free(yf);
+    return rc;
+}
+
 /* ---- Mixed-precision storage of the compressed KV entries ([HA] §4.2, the
  * paragraph on storage precision: the RoPE dims stay BF16, the rest of each
  * compressed entry is FP8).  Readings (the pages give no granularity or layout):

@@ -650,3 +650,119 @@ def test_sharded_topk_equals_full_topk(G):
         a = sorted(x for x in got[0, t] if x >= 0)
         b = sorted(x for x in full[0, t] if x >= 0)
         assert a == b
+
+
+# ----------------------------------------------------------------------------- Hadamard rotation
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024])
+def test_hadamard_rows_are_scipy_sylvester(n):
+    """Rotating the identity gives H_n / sqrt(n), with H_n the Sylvester matrix of scipy.linalg.hadamard."""
+    import scipy.linalg
+    y = oracle.hadamard_rotate(np.eye(n))
+    assert np.max(np.abs(y * math.sqrt(n) - scipy.linalg.hadamard(n))) < 1e-12
+
+
+def test_hadamard_textbook_h4():
+    """The 4 x 4 Walsh-Hadamard matrix in natural (Sylvester) order, written out."""
+    H4 = np.array([[1, 1, 1, 1], [1, -1, 1, -1], [1, 1, -1, -1], [1, -1, -1, 1]], np.float64) / 2.0
+    assert np.array_equal(oracle.hadamard_rotate(np.eye(4)), H4)
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    assert np.array_equal(oracle.hadamard_rotate(x), np.array([[5.0, -1.0, -2.0, 0.0]]))
+
+
+def test_hadamard_is_an_orthogonal_involution():
+    """H_n is symmetric with H_n^2 = n I, so R = H_n / sqrt(n) is its own inverse and keeps
+    norms and inner products: <Rq, Rk> = <q, k>."""
+    q = RNG.standard_normal((6, 128))
+    k = RNG.standard_normal((6, 128))
+    rq, rk = oracle.hadamard_rotate(q), oracle.hadamard_rotate(k)
+    assert np.max(np.abs(oracle.hadamard_rotate(rq) - q)) < 1e-13
+    assert np.allclose(np.sum(rq * rk, -1), np.sum(q * k, -1), rtol=1e-13, atol=1e-13)
+    assert np.allclose(np.linalg.norm(rq, axis=-1), np.linalg.norm(q, axis=-1), rtol=1e-14)
+
+
+def test_hadamard_spreads_a_spike():
+    """A one-hot row c e_j becomes a row of +-c/sqrt(n), the sign of entry i being
+    (-1)^popcount(i & j): the energy of one channel spreads evenly over all of them."""
+    n = 128
+    for j, c in ((0, 3.0), (5, -2.5), (127, 1.0)):
+        x = np.zeros((1, n))
+        x[0, j] = c
+        y = oracle.hadamard_rotate(x)[0]
+        sign = np.array([(-1) ** bin(i & j).count("1") for i in range(n)], np.float64)
+        assert np.allclose(y, sign * c / math.sqrt(n), rtol=1e-15, atol=0)
+
+
+def test_hadamard_quantize_worked_rows():
+    """Rotated e4m3 quantisation on hand-worked rows of n = 128 (c = 1/sqrt(128)):
+    2 e_0 -> 2c everywhere -> every code 448 (0x7E);  e_0 + e_1 -> 2c, 0, 2c, 0, ...;
+    e_0 - e_1 -> 0, 2c, ...;  -3 e_5 -> -3c (-1)^popcount(i & 5) -> 0xFE / 0x7E."""
+    n = 128
+    x = np.zeros((4, n), np.float32)
+    x[0, 0] = 2.0
+    x[1, 0] = x[1, 1] = 1.0
+    x[2, 0], x[2, 1] = 1.0, -1.0
+    x[3, 5] = -3.0
+    codes, scale = oracle.quantize_rows_e4m3_hadamard(x)
+    two_c = np.float32(2.0 / math.sqrt(n))
+    assert np.all(codes[0] == 0x7E) and scale[0] == np.float32(two_c / np.float32(448.0))
+    assert np.array_equal(codes[1], np.tile([0x7E, 0x00], n // 2))
+    assert np.array_equal(codes[2], np.tile([0x00, 0x7E], n // 2))
+    assert scale[1] == scale[2] == scale[0]
+    neg = np.array([bin(i & 5).count("1") % 2 == 0 for i in range(n)])
+    assert np.array_equal(codes[3], np.where(neg, 0xFE, 0x7E))
+    assert scale[3] == np.float32(np.float32(3.0 / math.sqrt(n)) / np.float32(448.0))
+    z, zs = oracle.quantize_rows_e4m3_hadamard(np.zeros((1, n), np.float32))
+    assert np.all(z == 0) and zs[0] == 1.0
+
+
+def test_hadamard_quantize_is_rotate_then_quantize():
+    """The rotated quantiser equals the pinned rotation, rounded to fp32, fed to the pinned
+    per-row quantiser; rows are independent."""
+    x = torch.randn(5, 64, generator=torch.Generator().manual_seed(7)).bfloat16().float().numpy()
+    c, s = oracle.quantize_rows_e4m3_hadamard(x)
+    c2, s2 = oracle.quantize_rows_e4m3(oracle.hadamard_rotate(x).astype(np.float32))
+    assert np.array_equal(c, c2) and np.array_equal(s, s2)
+    c3, s3 = oracle.quantize_rows_e4m3_hadamard(x[2:3])
+    assert np.array_equal(c3[0], c[2]) and s3[0] == s[2]
+
+
+def test_hadamard_rejects_bad_width():
+    for n in (0, 3, 96, 2048):
+        with pytest.raises(ValueError):
+            oracle.hadamard_rotate(np.ones((1, n)))
+    with pytest.raises(ValueError):
+        oracle.quantize_rows_e4m3_hadamard(np.ones((1, 96), np.float32))
+
+
+def test_hadamard_keeps_index_scores():
+    """Rotating queries and keys together leaves the Lightning Indexer scores unchanged."""
+    x = synth.draw_indexer_outliers(3, 1, 2, 96, Hi=8, di=128)
+    qI, w, kI = (x[k].float().numpy() for k in ("qI", "w", "kI"))
+    nv = np.array([[96, 50]], np.int32)
+    s0 = oracle.index_scores(qI, w, kI, nv)
+    s1 = oracle.index_scores(oracle.hadamard_rotate(qI).astype(np.float32), w,
+                             oracle.hadamard_rotate(kI).astype(np.float32), nv)
+    fin = np.isfinite(s0)
+    assert np.array_equal(fin, np.isfinite(s1))
+    assert np.max(np.abs(s1[fin] - s0[fin])) < 1e-4 * np.max(np.abs(s0[fin]))
+
+
+def test_hadamard_cuts_e4m3_score_error_on_outlier_channels():
+    """The point of the rotation: with outlier channels shared by queries and keys, the
+    e4m3 scores of the rotated operands are much closer to the exact scores than those of
+    the unrotated ones (rms error about 0.3x over seeds); on plain N(0,1) inputs both are
+    alike (1.00 +- 0.02)."""
+    def rel_err(x, quant):
+        qI, w, kI = (x[k].float().numpy() for k in ("qI", "w", "kI"))
+        nv = np.full((1, qI.shape[1]), kI.shape[1], np.int32)
+        exact = oracle.index_scores(qI, w, kI, nv)
+        q8, qs = quant(qI)
+        k8, ks = quant(kI)
+        d = oracle.index_scores_e4m3(q8, qs, w, k8, ks, nv) - exact
+        return float(np.sqrt(np.mean(d * d)) / np.std(exact))
+    out = synth.draw_indexer_outliers(11, 1, 8, 512)
+    plain, rot = rel_err(out, oracle.quantize_rows_e4m3), rel_err(out, oracle.quantize_rows_e4m3_hadamard)
+    assert rot < 0.5 * plain, (plain, rot)
+    flat = synth.draw_indexer_outliers(11, 1, 8, 512, channels=(), key_offset=0.0, q_gain=1.0)
+    plain, rot = rel_err(flat, oracle.quantize_rows_e4m3), rel_err(flat, oracle.quantize_rows_e4m3_hadamard)
+    assert 0.9 < rot / plain < 1.1, (plain, rot)
