@@ -6,7 +6,8 @@ at 65,536 tokens of context, through one CSA layer and one HCA layer, as the
 Flash configuration alternates them ("DeepSeek-V4 混合注意力：从压缩记忆到百万上下文"
 §2 configuration table, §4-§7):
   CSA: compress the newest 4-token block (latent c=512 and index keys c=128, with
-       the carry of the previous block) -> quantise the index queries (e4m3) ->
+       the carry of the previous block) -> Hadamard-rotate and quantise the index
+       queries (e4m3; the index keys are held rotated and quantised) ->
        e4m3 index scores over 16,384 keys -> top-1024 candidates -> exact rerank
        (bf16) to top-512 -> sparse_attn (64 heads, D=512, 512 + 128 SWA rows).
   HCA: compress the newest 128-token block (c=512) -> hca_attn over 512 summaries
@@ -36,6 +37,15 @@ if ROOT not in sys.path:
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+# e4m3 index path: queries and keys are Walsh-Hadamard-rotated before quantisation
+# (the Indexer paragraph of the MXFP4 sparse-attention page); --no-hadamard turns it off.
+INDEX_ROTATION = True
+
+
+def oracle_quantizer():
+    """The oracle's e4m3 quantiser matching INDEX_ROTATION (CPU-baseline / reference leg)."""
+    import oracle
+    return oracle.quantize_rows_e4m3_hadamard if INDEX_ROTATION else oracle.quantize_rows_e4m3
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -197,7 +207,7 @@ class DecodeSet:
         self.swa = g("swa", (B, wl.W, D))
         self.kI = g("kI", (B, N, 128))
         if index == "e4m3":
-            self.k8, self.ks = csa.csa_quantize_e4m3(self.kI)
+            self.k8, self.ks = csa.csa_quantize_e4m3(self.kI, hadamard=INDEX_ROTATION)
         self.sink = f32("sink", (H,))
         self.q_pos = torch.full((B, T), wl.q_pos0, dtype=torch.int64, device=dev)
         self.swa_pos0 = torch.full((B,), wl.swa_pos0, dtype=torch.int64, device=dev)
@@ -353,7 +363,7 @@ class DecodeSet:
                 marks.append((name, ev))
         mark("start")
         if self.index == "e4m3":
-            csa.csa_quantize_e4m3(x["qI"], codes=self.q8, scale=self.qs)
+            csa.csa_quantize_e4m3(x["qI"], codes=self.q8, scale=self.qs, hadamard=INDEX_ROTATION)
             mark("quantize_q")
             csa.csa_index_scores(self.q8, x["w"], self.k8, self.n_valid, q_scale=self.qs, k_scale=self.ks,
                                  scores=self.scores, select_ws=self.select_ws)
@@ -660,7 +670,7 @@ def bench_prefill(steps, warmup, device, tflops_peak):
     topk_ws = csa.topk_workspace(B, T, N, k, dev)
     attn_ws = csa.attn_workspace(B, T, H, D, 128 + k, device=dev)
     out = torch.empty_like(q)
-    k8, ks = csa.csa_quantize_e4m3(kI)
+    k8, ks = csa.csa_quantize_e4m3(kI, hadamard=INDEX_ROTATION)
     q8 = torch.empty((B, T, 64, 128), dtype=torch.uint8, device=dev)
     qs = torch.empty((B, T, 64), dtype=torch.float32, device=dev)
     scale = 1.0 / math.sqrt(D)
@@ -679,7 +689,7 @@ def bench_prefill(steps, warmup, device, tflops_peak):
         fn()
     launches = csa.csa_launch_count() - c0
     per, step_ms = _stage_times(stages, steps, warmup)
-    e4m3 = [("quantize_q", lambda: csa.csa_quantize_e4m3(qI, codes=q8, scale=qs)),
+    e4m3 = [("quantize_q", lambda: csa.csa_quantize_e4m3(qI, codes=q8, scale=qs, hadamard=INDEX_ROTATION)),
             ("index_e4m3", lambda: csa.csa_index_scores(q8, w, k8, n_valid, q_scale=qs, k_scale=ks, scores=scores))]
     per8, _ = _stage_times(e4m3, steps, warmup)
     assert csa.csa_poll_status() == csa.CSA_OK
@@ -804,8 +814,8 @@ def run_big_stage(stage, steps, warmup, device):
         n_valid = csa.n_valid_for(q_pos, 4, N)
         scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         if stage == "prefill_index8":
-            q8, qs = csa.csa_quantize_e4m3(qI)
-            k8, ks = csa.csa_quantize_e4m3(kI)
+            q8, qs = csa.csa_quantize_e4m3(qI, hadamard=INDEX_ROTATION)
+            k8, ks = csa.csa_quantize_e4m3(kI, hadamard=INDEX_ROTATION)
             fn = lambda: csa.csa_index_scores(q8, w, k8, n_valid, q_scale=qs, k_scale=ks, scores=scores)
         else:
             csa.csa_index_scores(qI, w, kI, n_valid, scores=scores)
@@ -855,7 +865,7 @@ def run_stage(name, stage, index, steps, warmup, device, kv8=False):
     calls = {
         "compress": lambda: csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"],
                                              ratio=4, out=st.comp_kv),
-        "quantize": lambda: csa.csa_quantize_e4m3(x["qI"], codes=st.q8, scale=st.qs),
+        "quantize": lambda: csa.csa_quantize_e4m3(x["qI"], codes=st.q8, scale=st.qs, hadamard=INDEX_ROTATION),
         "index": (lambda: csa.csa_index_scores(st.q8, x["w"], st.k8, st.n_valid, q_scale=st.qs, k_scale=st.ks,
                                                scores=st.scores)) if index == "e4m3" else
                  (lambda: csa.csa_index_scores(x["qI"], x["w"], st.kI, st.n_valid, scores=st.scores)),
@@ -907,13 +917,13 @@ def oracle_decode_token(wl, seed, index, with_hca):
     sink = f32("sink", (H,))
     comp = {nm: g(nm, (1, cL, cc)) for nm in ("C_a", "C_b", "Z_a", "Z_b")}
     prev = {nm: g(nm, (1, 4, cc)) for nm in ("prev_Cb", "prev_Zb")}
-    k8, ks = oracle.quantize_rows_e4m3(kI) if index == "e4m3" else (None, None)
+    k8, ks = oracle_quantizer()(kI) if index == "e4m3" else (None, None)
     q_pos = np.array([[one.q_pos0]], np.int64)
     nv = oracle.n_visible(q_pos, 4, N)
     t0 = time.perf_counter()
     oracle.compress_csa(comp["C_a"], comp["C_b"], comp["Z_a"], comp["Z_b"], prev["prev_Cb"], prev["prev_Zb"])
     if index == "e4m3":
-        q8, qs = oracle.quantize_rows_e4m3(qI)
+        q8, qs = oracle_quantizer()(qI)
         s8 = oracle.index_scores_e4m3(q8, qs, w, k8, ks, nv)
         cand = oracle.topk(s8.astype(np.float32), nv, 2 * k)[0, 0]
         cand = cand[cand >= 0]
@@ -954,6 +964,15 @@ def oracle_baseline(wl, index, with_hca, budget_s=12.0, max_tokens=24):
                       f"{cpu_model()}"}
 
 
+def workload_text(wl, index, with_hca):
+    """The JSON line's config.workload, the same for both arms."""
+    return (f"{wl.name}: B={wl.B} decode tokens/GPU at ctx {wl.ctx}; CSA layer (compress 4:1 c=512+128, "
+            f"{index} index over N={wl.N}, top-{wl.topk}"
+            + ((" (Hadamard-rotated q/k)" if INDEX_ROTATION else "") + " via 2k rerank" if index == "e4m3" else "")
+            + f", sparse_attn H={wl.H} D={wl.D})"
+            + (f" + HCA layer (compress 128:1, hca_attn over {wl.ctx // 128}+128 rows)" if with_hca else ""))
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -963,12 +982,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="flash64k", choices=["flash64k", "pro1m"])
     ap.add_argument("--index", default="e4m3", choices=["e4m3", "bf16"])
+    ap.add_argument("--no-hadamard", action="store_true",
+                    help="e4m3 index path without the Hadamard rotation of queries and keys")
     ap.add_argument("--no-extra", action="store_true", help="skip the pro1m measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", choices=STAGES + BIG_STAGES, help="time one stage alone (eager calls), e.g. under ncu")
     ap.add_argument("--kv8", action="store_true", help="with --stage: memory rows as mixed-precision KV8 entries")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    global INDEX_ROTATION
+    INDEX_ROTATION = not args.no_hadamard
     rank, world, local = dist_env()
     with_hca = args.workload == "flash64k"
 
@@ -989,8 +1012,7 @@ def main():
                 "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * sum(times) / steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": f"{wl.name}: B={wl.B} decode, ctx {wl.ctx}, N={wl.N}, top-{wl.topk}, "
-                                       f"H={wl.H}, D={wl.D}, index {args.index}" + (" + HCA layer" if with_hca else ""),
+                "config": {"workload": workload_text(wl, args.index, with_hca),
                            "sample": "one sequence per step"},
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                  "sample": f"{steps} steps of one single-sequence decode token each "
@@ -1084,11 +1106,7 @@ def main():
         "value": m["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16+e4m3" if args.index == "e4m3" else "bf16", "data": "synthetic",
-        "config": {"workload": f"{wl.name}: B={wl.B} decode tokens/GPU at ctx {wl.ctx}; CSA layer (compress 4:1 "
-                               f"c=512+128, {args.index} index over N={wl.N}, top-{wl.topk}"
-                               + (" via 2k rerank" if args.index == "e4m3" else "") +
-                               f", sparse_attn H={wl.H} D={wl.D})" + (" + HCA layer (compress 128:1, hca_attn over "
-                               f"{wl.ctx // 128}+128 rows)" if with_hca else ""),
+        "config": {"workload": workload_text(wl, args.index, with_hca),
                    "l2": f"{m['input_sets']} rotating input sets, > 2x L2 touched between reuses",
                    "parallelism": f"replicas x{world}"},
         "e2e": m["e2e"], "roofline": m["roofline"], "roofline_indexer": m["roofline_indexer"],

@@ -92,6 +92,27 @@ int csa_quantize_e4m3(const void *x, int x_dtype, int64_t rows, int cols, uint8_
                       void *stream);
 
 /*
+ * csa_quantize_e4m3_hadamard -- csa_quantize_e4m3 of the Hadamard-rotated rows
+ * ([P1], the Indexer paragraph: the index query is Hadamard-rotated before it is
+ * scored against the compressed keys).  Give the index keys the same rotation: the
+ * rotation is orthonormal, so <Rq, Rk> = <q, k> and the scores keep their value,
+ * while channels that dominate q and k are spread over all dims before the e4m3
+ * rounding.  The exact bf16 rerank (csa_topk_select, csa_index_rerank) takes the
+ * UNROTATED bf16 operands.
+ *   y = H_n x / sqrt(n) per row, H_n the Walsh-Hadamard matrix in Sylvester (natural)
+ *       order, H[i][j] = (-1)^popcount(i & j); the sums are taken in fp64 (exact while
+ *       a row spans at most 53 - 8 - log2(n) binary orders for BF16 input, 53 - 24 -
+ *       log2(n) for F32), times 1/sqrt(n) in fp64, rounded to fp32; a zero is +0
+ *   then codes / scale exactly as csa_quantize_e4m3 computes them from y.
+ *   x     : [rows, cols] F32 or BF16 (x_dtype), 16-byte aligned;  cols = 32, 64, 128 or 256
+ *   codes : [rows, cols] uint8 e4m3, 16-byte aligned;  scale : [rows] fp32
+ * NaN inputs are not supported.  Returns CSA_ERR_INVALID for any other cols or dtype,
+ * or for an x or codes pointer that is not 16-byte aligned.
+ */
+int csa_quantize_e4m3_hadamard(const void *x, int x_dtype, int64_t rows, int cols, uint8_t *codes, float *scale,
+                               void *stream);
+
+/*
  * csa_index_scores -- Lightning Indexer ([HA] §4.2):
  *   scores[b,t,i] = sum_{h<64} w[b,t,h] * ReLU(<qI[b,t,h,:], kI[b,i,:]>)   for i < n_valid[b,t]
  *   scores[b,t,i] = -inf                                                   for n_valid[b,t] <= i < N

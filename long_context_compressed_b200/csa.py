@@ -33,6 +33,7 @@ _SIGS = {
     "csa_version": ([], _i32),
     "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
+    "csa_quantize_e4m3_hadamard": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_kv8_entry_bytes": ([_i32], ctypes.c_longlong),
     "csa_quantize_kv8": ([_vp, _i64, _i32, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
@@ -120,16 +121,19 @@ def csa_compress(C_a, C_b=None, Z_a=None, Z_b=None, prev_Cb=None, prev_Zb=None, 
     return out
 
 
-def csa_quantize_e4m3(x, codes=None, scale=None, stream=None):
-    """Per-row e4m3 quantisation of x [..., cols] -> (codes uint8 [..., cols], scale fp32 [...])."""
+def csa_quantize_e4m3(x, codes=None, scale=None, stream=None, hadamard=False):
+    """Per-row e4m3 quantisation of x [..., cols] -> (codes uint8 [..., cols], scale fp32 [...]).
+    hadamard=True quantises the Walsh-Hadamard-rotated rows instead (csa_quantize_e4m3_hadamard;
+    give queries and keys the same setting)."""
     cols = x.shape[-1]
     rows = x.numel() // cols
     if codes is None:
         codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scale is None:
         scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
-    _check(_lib.csa_quantize_e4m3(_ptr(x), _dtype_code(x), rows, cols, _ptr(codes), _ptr(scale),
-                                  _stream(stream)), "csa_quantize_e4m3")
+    name = "csa_quantize_e4m3_hadamard" if hadamard else "csa_quantize_e4m3"
+    _check(getattr(_lib, name)(_ptr(x), _dtype_code(x), rows, cols, _ptr(codes), _ptr(scale), _stream(stream)),
+           name)
     return codes, scale
 
 

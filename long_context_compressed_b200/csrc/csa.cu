@@ -431,6 +431,38 @@ int csa_quantize_e4m3(const void* x, int x_dtype, int64_t rows, int cols, uint8_
   return launch_status();
 }
 
+int csa_quantize_e4m3_hadamard(const void* x, int x_dtype, int64_t rows, int cols, uint8_t* codes, float* scale,
+                               void* stream) {
+  if (rows < 0 || !(cols == 32 || cols == 64 || cols == 128 || cols == 256)) return CSA_ERR_INVALID;
+  if (x_dtype != CSA_F32 && x_dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (rows == 0) return CSA_OK;
+  if (!x || !codes || !scale) return CSA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(codes)) & 15) return CSA_ERR_INVALID;
+  cudaStream_t st = as_stream(stream);
+  // 8 warps per block, a warp takes HadamardCfg<N>::RPW rows per pass; two blocks per SM
+#define CSA_LAUNCH_HAD(T, N)                                                                              \
+  do {                                                                                                    \
+    const int64_t rpb = 8 * csa::HadamardCfg<N>::RPW;                                                     \
+    const unsigned blocks = (unsigned)std::min<int64_t>((rows + rpb - 1) / rpb, (int64_t)sm_count() * 2); \
+    launch_k(csa::hadamard_quantize_e4m3_kernel<T, N>, blocks, 256, 0, st, (const T*)x, rows, codes, scale); \
+  } while (0)
+#define CSA_LAUNCH_HAD_COLS(T)            \
+  switch (cols) {                         \
+    case 32: CSA_LAUNCH_HAD(T, 32); break;   \
+    case 64: CSA_LAUNCH_HAD(T, 64); break;   \
+    case 128: CSA_LAUNCH_HAD(T, 128); break; \
+    default: CSA_LAUNCH_HAD(T, 256); break;  \
+  }
+  if (x_dtype == CSA_BF16) {
+    CSA_LAUNCH_HAD_COLS(__nv_bfloat16)
+  } else {
+    CSA_LAUNCH_HAD_COLS(float)
+  }
+#undef CSA_LAUNCH_HAD_COLS
+#undef CSA_LAUNCH_HAD
+  return launch_status();
+}
+
 long long csa_kv8_entry_bytes(int D) { return D == csa::kKv8Dims ? (long long)csa::kKv8Bytes : 0; }
 
 int csa_quantize_kv8(const void* kv, int64_t rows, int D, void* entries, void* stream) {

@@ -37,4 +37,124 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const Tin* __restric
   }
 }
 
+// Hadamard-rotated variant for the index vectors ("揭秘DeepSeek-V4-Pro-MXFP4稀疏注意力：
+// 哈希索引与DSA如何撑起1M超长上下文？", the Indexer paragraph: the index query is
+// Hadamard-rotated before it is scored; the keys take the same rotation, which leaves
+// <q, k> unchanged and spreads outlier channels before the e4m3 rounding).
+// Row of N values: y = H_N x with H_N the Sylvester-ordered Walsh-Hadamard matrix, by
+// the fast transform in fp64.  LPR = N / E lanes share a row, lane g of the row holding
+// the E contiguous elements g*E .. g*E+E-1 (16-byte loads and stores): the log2(E)
+// butterflies over the low index bits run inside the lane, the log2(LPR) over the high
+// bits across lanes (shuffles); butterflies over different bits commute.  Every partial
+// sum is an exact fp64 value while the row spans at most 53 - (significand bits) -
+// log2(N) binary orders, so the order of the additions does not matter.  Then
+// y * (1/sqrt(N)) in fp64, rounded to fp32 (a zero becomes +0), and the per-row
+// quantiser above.  x and codes are 16-byte aligned (checked by the caller).  Each pass of
+// the grid-stride loop requests the next pass's rows before it transforms its own.
+template <int N>
+struct HadamardCfg {
+  static constexpr int E = N / 4 < 16 ? N / 4 : 16;   // elements per lane (registers)
+  static constexpr int LPR = N / E;                    // lanes per row: 4, 8 or 16
+  static constexpr int RPW = 32 / LPR;              // rows per warp
+};
+
+// 16 raw bytes -> doubles (exact widening)
+__device__ __forceinline__ void widen16(const uint4 u, double* v, const __nv_bfloat16*) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[2 * j] = (double)__uint_as_float(w[j] << 16);
+    v[2 * j + 1] = (double)__uint_as_float(w[j] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void widen16(const uint4 u, double* v, const float*) {
+  v[0] = (double)__uint_as_float(u.x);
+  v[1] = (double)__uint_as_float(u.y);
+  v[2] = (double)__uint_as_float(u.z);
+  v[3] = (double)__uint_as_float(u.w);
+}
+
+template <typename Tin, int N>
+__global__ void __launch_bounds__(256, 2) hadamard_quantize_e4m3_kernel(const Tin* __restrict__ x, int64_t rows,
+                                                                        uint8_t* __restrict__ codes,
+                                                                        float* __restrict__ scale) {
+  using C = HadamardCfg<N>;
+  constexpr int E = C::E, LPR = C::LPR, RPW = C::RPW;
+  constexpr int VEC = 16 / (int)sizeof(Tin);   // elements per 16-byte load
+  constexpr int NV = E / VEC;                  // 16-byte loads per lane and row
+  griddep_sync();
+  const double c = __ddiv_rn(1.0, __dsqrt_rn((double)N));
+  const int lane = (int)lane_id();
+  const int g = lane % LPR;
+  const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5) * RPW;
+  // the raw bytes of the next rows are requested before the current rows are transformed
+  auto fetch = [&](int64_t rr, uint4* dst) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+      dst[k] = rr < rows ? __ldg(reinterpret_cast<const uint4*>(x + rr * N + g * E + k * VEC)) : make_uint4(0, 0, 0, 0);
+  };
+  int64_t r0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+  uint4 raw[NV];
+  fetch(r0 + lane / LPR, raw);
+  for (; r0 < rows; r0 += step) {
+    const int64_t r = r0 + lane / LPR;
+    uint4 nxt[NV];
+    fetch(r + step, nxt);
+    double v[E];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) widen16(raw[k], v + k * VEC, x);
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        if ((e & h) == 0) {
+          const double a = v[e], b = v[e + h];
+          v[e] = __dadd_rn(a, b);
+          v[e + h] = __dsub_rn(a, b);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 1; m < LPR; m <<= 1) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const double o = __shfl_xor_sync(0xffffffffu, v[e], m);
+        v[e] = (g & m) ? __dsub_rn(o, v[e]) : __dadd_rn(v[e], o);
+      }
+    }
+    float y[E];
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      y[e] = __double2float_rn(__dadd_rn(__dmul_rn(v[e], c), 0.0));
+      amax = fmaxf(amax, fabsf(y[e]));
+    }
+#pragma unroll
+    for (int m = 1; m < LPR; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+    if (r < rows) {
+      uint32_t packed[E / 4];
+#pragma unroll
+      for (int q = 0; q < E / 4; ++q) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          word |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(y[4 * q + j], s), __NV_SATFINITE, __NV_E4M3) << (8 * j);
+        packed[q] = word;
+      }
+      uint8_t* cr = codes + r * N + g * E;
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint2*>(cr) = make_uint2(packed[0], packed[1]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < E / 4; q += 4)
+          *reinterpret_cast<uint4*>(cr + 4 * q) = make_uint4(packed[q], packed[q + 1], packed[q + 2], packed[q + 3]);
+      }
+      if (g == 0) scale[r] = s;
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) raw[k] = nxt[k];
+  }
+}
+
 }  // namespace csa

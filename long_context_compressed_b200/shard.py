@@ -4,8 +4,9 @@ Each GPU holds a contiguous range [lo, hi) of the compressed entries (index keys
 latent rows).  One decode step, on every GPU (all of its arithmetic runs in the
 library's kernels; this module only orders the calls and the exchanges):
 
-1. the indexer over the local entries, the local top-k (e4m3 scores, exact bf16
-   rescoring of the kc = 2k candidates as in the single-GPU step), the exact scores of
+1. the indexer over the local entries, the local top-k (e4m3 scores of Hadamard-rotated
+   queries and keys, exact bf16 rescoring of the kc = 2k candidates as in the single-GPU
+   step), the exact scores of
    the local winners and their global entry numbers;
 2. one all-gather of the (score, global index) pairs, then the global top-k
    (csa_shard_select), the same on every GPU.  Every global winner is a local winner of
@@ -77,8 +78,8 @@ class Shard:
 class GpuKernels:
     """The library's calls for one shard; buffers are allocated on first use and kept."""
 
-    def __init__(self, k: int, scale: float):
-        self.k, self.scale = k, scale
+    def __init__(self, k: int, scale: float, hadamard: bool = True):
+        self.k, self.scale, self.hadamard = k, scale, hadamard
         self.buf: dict = {}
 
     def _b(self, name, shape, dtype, device, zero=False):
@@ -93,10 +94,10 @@ class GpuKernels:
         from . import csa
         B, Ns, dev, k = sh.kI.shape[0], sh.kI.shape[1], sh.kI.device, self.k
         if sh.k8 is None:
-            sh.k8, sh.ks = csa.csa_quantize_e4m3(sh.kI)
+            sh.k8, sh.ks = csa.csa_quantize_e4m3(sh.kI, hadamard=self.hadamard)
         q8 = self._b("q8", qI.shape, torch.uint8, dev)
         qs = self._b("qs", qI.shape[:-1], torch.float32, dev)
-        csa.csa_quantize_e4m3(qI, codes=q8, scale=qs)
+        csa.csa_quantize_e4m3(qI, codes=q8, scale=qs, hadamard=self.hadamard)
         scores = self._b("scores", (B, 1, Ns), torch.float32, dev)
         ws = self.buf.get("select_ws")
         if ws is None:

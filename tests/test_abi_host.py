@@ -139,3 +139,22 @@ def test_kv8_storage_host_checks(lib):
     assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 16, 256, 100, 3, p, None, 0, None) == 2
     assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 256, 512, 100, 3, p, None, 0, None) == 2
     assert g(p, p, p, p, 128, p, p, p, 8, 0.1, 1, 1, 16, 512, 100, 4, p, None, 0, None) == 1
+
+
+def test_hadamard_quantizer_host_checks(lib):
+    """The rotated quantiser takes rows of 32, 64, 128 or 256 F32 / BF16 values only."""
+    f = lib.csa_quantize_e4m3_hadamard
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p]
+    p = 16
+    for cols in (0, 16, 96, 512, 1024):
+        assert f(p, 1, 4, cols, p, p, None) == 1, cols
+    assert f(p, 2, 4, 128, p, p, None) == 1          # e4m3 input
+    assert f(p, 1, -1, 128, p, p, None) == 1
+    assert f(None, 1, 4, 128, p, p, None) == 1
+    assert f(p, 1, 4, 128, None, p, None) == 1
+    assert f(p + 8, 1, 4, 128, p, p, None) == 1      # x not 16-byte aligned
+    assert f(p, 1, 4, 128, p + 4, p, None) == 1      # codes not 16-byte aligned
+    for cols in (32, 64, 128, 256):
+        assert f(p, 1, 0, cols, p, p, None) == 0     # nothing to do
