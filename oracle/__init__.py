@@ -18,8 +18,8 @@ cited in ``oracle.c``:
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
 (tests/test_oracle_pins.py) except the FP8 *recall* statistic, which the pages
 do not fix ("parity unpinned" for recall only; the e4m3 codec, the FP8 score
-definition, the Hadamard rotation of the index vectors and the mixed-precision KV
-storage codec are pinned).
+definition, the Hadamard rotation of the index vectors, the MXFP4 codec of the FP4
+index operands and the mixed-precision KV storage codec are pinned).
 """
 from __future__ import annotations
 
@@ -71,6 +71,12 @@ def _load():
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_quantize_rows_e4m3.argtypes = [_f32p, i64, i32, _u8p, _f32p]
     lib.oracle_hadamard_rotate.argtypes = [_f64p, i64, i32, _f64p]
+    lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e2m1_decode.restype = dbl
+    lib.oracle_e2m1_encode.argtypes = [dbl]
+    lib.oracle_e2m1_encode.restype = ctypes.c_uint8
+    lib.oracle_quantize_rows_mxfp4.argtypes = [_f32p, i64, i32, _u8p, _u8p]
+    lib.oracle_mxfp4_dequantize.argtypes = [_u8p, _u8p, i64, i32, _f32p]
     lib.oracle_quantize_rows_e4m3_hadamard.argtypes = [_f32p, i64, i32, _u8p, _f32p]
     lib.oracle_sparse_attn_partial.argtypes = [_f32p, _f32p, _f32p, i64, i32, _i64p, _i32p, i32, dbl, i32,
                                                i32, i32, i32, i64, _f64p, _f64p, _f64p]
@@ -86,7 +92,8 @@ def _load():
                                     i32, i32, i32, i64, _f64p, _f64p]
     for name in ("oracle_compress_csa", "oracle_compress_hca", "oracle_index_scores",
                  "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_hadamard_rotate",
-                 "oracle_quantize_rows_e4m3_hadamard", "oracle_kv8_quantize",
+                 "oracle_quantize_rows_e4m3_hadamard", "oracle_quantize_rows_mxfp4", "oracle_mxfp4_dequantize",
+                 "oracle_kv8_quantize",
                  "oracle_kv8_dequantize", "oracle_sparse_attn_partial", "oracle_attn_combine", "oracle_topk",
                  "oracle_sparse_attn", "oracle_hca_attn"):
         getattr(lib, name).restype = ctypes.c_int
@@ -246,6 +253,46 @@ def quantize_rows_e4m3_hadamard(x):
     scale = np.empty(x.shape[:-1], np.float32)
     _check(lib.oracle_quantize_rows_e4m3_hadamard(x, x.size // n, n, codes, scale), "quantize_rows_e4m3_hadamard")
     return codes, scale
+
+
+def e2m1_decode(codes):
+    """FP4 E2M1 code (low nibble) -> value."""
+    lib = _load()
+    c = np.asarray(codes, np.uint8)
+    return np.asarray([lib.oracle_e2m1_decode(int(b)) for b in c.reshape(-1)], np.float64).reshape(c.shape)
+
+
+def e2m1_encode(x):
+    """Nearest E2M1 code (ties to the even mantissa, saturating at 6)."""
+    lib = _load()
+    a = np.asarray(x, np.float64)
+    return np.asarray([lib.oracle_e2m1_encode(float(v)) for v in a.reshape(-1)], np.uint8).reshape(a.shape)
+
+
+def quantize_rows_mxfp4(x, hadamard: bool = False):
+    """MXFP4 of the last axis ([HA] §4.2 FP4 index QK; OCP MX reading): x [..., n], n a
+    multiple of 32 -> (codes u8 [..., n] one E2M1 code per byte, scale u8 [..., n/32] E8M0).
+    hadamard=True quantises the Walsh-Hadamard-rotated rows, rounded to fp32 first."""
+    lib = _load()
+    x = _f32(x)
+    if hadamard:
+        x = hadamard_rotate(x).astype(np.float32)
+    n = x.shape[-1]
+    codes = np.empty(x.shape, np.uint8)
+    scale = np.empty(x.shape[:-1] + (n // 32 if n % 32 == 0 else 0,), np.uint8)
+    _check(lib.oracle_quantize_rows_mxfp4(x, x.size // n if n else 0, n, codes, scale), "quantize_rows_mxfp4")
+    return codes, scale
+
+
+def mxfp4_dequantize(codes, scale):
+    """codes [..., n], scale [..., n/32] -> float32 [..., n], exactly code * 2^(scale-127)."""
+    lib = _load()
+    c = np.ascontiguousarray(np.asarray(codes, np.uint8))
+    s = np.ascontiguousarray(np.asarray(scale, np.uint8))
+    n = c.shape[-1]
+    out = np.empty(c.shape, np.float32)
+    _check(lib.oracle_mxfp4_dequantize(c, s, c.size // n, n, out), "mxfp4_dequantize")
+    return out
 
 
 def kv8_entry_bytes(D: int) -> int:

@@ -295,6 +295,76 @@ int oracle_quantize_rows_e4m3_hadamard(const float *x, int64_t rows, int n, uint
     return rc;
 }
 
+/* ---- FP4 index QK ([HA] §2 configuration table and §4.2: the index QK path
+ * runs in FP4).  Readings (the pages name no FP4 format for the indexer): OCP
+ * MXFP4, i.e. FP4 E2M1 elements (1 sign, 2 exponent bits with bias 1, 1 mantissa
+ * bit; no infinities or NaN; largest magnitude 6) with one shared E8M0 scale
+ * (2^(c-127)) per block of 32 consecutive dims.  The block scale is
+ * X = 2^(floor(log2 amax) - 2), 2 being the exponent of E2M1's largest binade,
+ * clamped to 2^-127 .. 2^127; an all-zero block gets X = 1.  Elements are
+ * x / X rounded to the nearest E2M1 value, ties to the even mantissa, magnitudes
+ * beyond 6 saturating to 6.  The score is the plain definition on the values
+ * code * X, as for e4m3. */
+double oracle_e2m1_decode(uint8_t c)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    return (c & 8) ? -mag[c & 7] : mag[c & 7];
+}
+
+/* Nearest E2M1 value by search over the 8 non-negative codes (increasing in
+ * magnitude); on a tie the code with mantissa bit 0 (an even code) wins. */
+uint8_t oracle_e2m1_encode(double x)
+{
+    uint8_t sign = signbit(x) ? 8 : 0;
+    double a = fabs(x);
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        double d = fabs(oracle_e2m1_decode((uint8_t)c) - a);
+        double db = fabs(oracle_e2m1_decode((uint8_t)best) - a);
+        if (d < db || (d == db && (c & 1) == 0)) best = c;
+    }
+    return sign | (uint8_t)best;
+}
+
+/* x [rows, n] (n a multiple of 32) -> codes [rows, n] (one E2M1 code per byte,
+ * low nibble) and scale [rows, n/32] (E8M0 codes). */
+int oracle_quantize_rows_mxfp4(const float *x, int64_t rows, int n, uint8_t *codes, uint8_t *scale)
+{
+    if (n <= 0 || n % 32 != 0 || rows < 0) return ORC_BAD;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int b = 0; b < n / 32; ++b) {
+            const float *xb = x + r * n + 32 * b;
+            double amax = 0.0;
+            for (int j = 0; j < 32; ++j)
+                if (fabs((double)xb[j]) > amax) amax = fabs((double)xb[j]);
+            int e = 0;
+            if (amax > 0.0) {
+                int E;
+                frexp(amax, &E);            /* amax = f 2^E, f in [0.5, 1): floor(log2 amax) = E - 1 */
+                e = E - 1 - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            scale[r * (n / 32) + b] = (uint8_t)(e + 127);
+            for (int j = 0; j < 32; ++j)
+                codes[r * n + 32 * b + j] = oracle_e2m1_encode(ldexp((double)xb[j], -e));
+        }
+    return ORC_OK;
+}
+
+/* codes / scale as above -> x [rows, n] float (code * 2^(scale-127), exact). */
+int oracle_mxfp4_dequantize(const uint8_t *codes, const uint8_t *scale, int64_t rows, int n, float *x)
+{
+    if (n <= 0 || n % 32 != 0 || rows < 0) return ORC_BAD;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int j = 0; j < n; ++j) {
+            uint8_t s = scale[r * (n / 32) + j / 32];
+            if (s == 0xFF) return ORC_BAD;     /* E8M0 NaN */
+            x[r * n + j] = (float)ldexp(oracle_e2m1_decode(codes[r * n + j] & 15), (int)s - 127);
+        }
+    return ORC_OK;
+}
+
 /* ---- Mixed-precision storage of the compressed KV entries ([HA] §4.2, the
  * paragraph on storage precision: the RoPE dims stay BF16, the rest of each
  * compressed entry is FP8).  Readings (the pages give no granularity or layout):

@@ -766,3 +766,100 @@ def test_hadamard_cuts_e4m3_score_error_on_outlier_channels():
     flat = synth.draw_indexer_outliers(11, 1, 8, 512, channels=(), key_offset=0.0, q_gain=1.0)
     plain, rot = rel_err(flat, oracle.quantize_rows_e4m3), rel_err(flat, oracle.quantize_rows_e4m3_hadamard)
     assert 0.9 < rot / plain < 1.1, (plain, rot)
+
+
+# ----------------------------------------------------------------------------- FP4 (MXFP4) index operands
+def test_e2m1_decode_is_the_bit_field_formula():
+    """E2M1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0; exponent 0 is
+    subnormal (m / 2), otherwise 2^(e-1) (1 + m/2).  All 16 codes from the fields."""
+    for c in range(16):
+        s, e, m = c >> 3, (c >> 1) & 3, c & 1
+        v = (m / 2.0) if e == 0 else 2.0 ** (e - 1) * (1 + m / 2.0)
+        got = oracle.e2m1_decode([c])[0]
+        assert got == (-v if s else v) and (np.signbit(got) == bool(s)), c
+
+
+def test_e2m1_encode_is_nearest_with_even_ties():
+    """Brute force over a dense grid: the code is the nearest of the 8 magnitudes, ties go
+    to mantissa bit 0, magnitudes beyond 6 give 6; the sign is kept (also for -0)."""
+    mags = oracle.e2m1_decode(np.arange(8))
+    xs = np.concatenate([np.arange(-800, 801) / 100.0, [-0.0, 1e-30, 50.0, -1e9]])
+    got = oracle.e2m1_encode(xs)
+    for x, c in zip(xs, got):
+        d = np.abs(mags - abs(x))
+        best = [i for i in range(8) if d[i] == d.min()]
+        want = best[0] if len(best) == 1 else [i for i in best if i % 2 == 0][0]
+        assert c == (want | (8 if np.signbit(x) else 0)), (x, c, want)
+    # hand-worked ties
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6, 7.0: 7, -5.0: 14}
+    for x, c in ties.items():
+        assert oracle.e2m1_encode([x])[0] == c, x
+
+
+def test_mxfp4_block_scale_and_layout():
+    """Per block of 32: X = 2^(floor(log2 amax) - 2), so amax / X lies in [4, 8); E8M0 code
+    = log2 X + 127; blocks are independent; an all-zero block gets X = 1 (code 127)."""
+    for amax in (1e-3, 0.3, 1.0, 4.0, 6.0, 7.99, 8.0, 1000.0, 3e30):
+        x = np.zeros((1, 64), np.float32)
+        x[0, 5] = -amax
+        x[0, 40] = 1.0
+        c, s = oracle.quantize_rows_mxfp4(x)
+        e = math.floor(math.log2(np.float32(amax))) - 2
+        assert s[0, 0] == e + 127 and s[0, 1] == 127 - 2       # second block: amax 1 -> X = 1/4
+        assert 4.0 <= np.float32(amax) / 2.0 ** e < 8.0
+        assert c[0, 40] == 6                                    # 1 / (1/4) = 4
+    z, zs = oracle.quantize_rows_mxfp4(np.zeros((2, 32), np.float32))
+    assert np.all(z == 0) and np.all(zs == 127)
+    x = rnd(3, 128)
+    c, s = oracle.quantize_rows_mxfp4(x)
+    x2 = x.copy()
+    x2[:, 32:64] *= 100.0
+    c2, s2 = oracle.quantize_rows_mxfp4(x2)
+    keep = np.r_[0:32, 64:128]
+    assert np.array_equal(c[:, keep], c2[:, keep]) and np.array_equal(s[:, [0, 2, 3]], s2[:, [0, 2, 3]])
+
+
+def test_mxfp4_round_trip_and_error_bound():
+    """Values code * 2^k with a 4 or 6 in the block round-trip exactly; otherwise each
+    element is off by at most half a grid step of its binade (times X), or by the
+    saturation to 6 X."""
+    rng = np.random.default_rng(5)
+    for k in (-20, -3, 0, 7):
+        codes = rng.integers(0, 16, (4, 64)).astype(np.uint8)
+        codes[:, 0] = 7
+        codes[:, 32] = 14
+        x = (oracle.e2m1_decode(codes) * 2.0 ** k).astype(np.float32)
+        c, s = oracle.quantize_rows_mxfp4(x)
+        assert np.array_equal(oracle.mxfp4_dequantize(c, s), x)
+    x = rnd(16, 128, scale=3.0)
+    c, s = oracle.quantize_rows_mxfp4(x)
+    X = 2.0 ** (s.astype(np.float64) - 127).repeat(32, axis=1)
+    y = np.abs(x / X)
+    err = np.abs(oracle.mxfp4_dequantize(c, s) - x) / X
+    half_step = np.where(y < 2, 0.25, np.where(y < 4, 0.5, 1.0))
+    assert np.all(err <= np.maximum(half_step, y - 6.0) + 1e-12)
+
+
+def test_mxfp4_scores_are_the_definition_on_dequantised_values():
+    """The FP4 score is the pinned index score of the dequantised operands; with the
+    rotation, rotating q and k first leaves the exact scores unchanged, so the FP4 error
+    on outlier-channel inputs drops as it does for e4m3."""
+    x = synth.draw_indexer_outliers(4, 1, 4, 256)
+    qI, w, kI = (x[k].float().numpy() for k in ("qI", "w", "kI"))
+    nv = np.full((1, 4), 256, np.int32)
+    exact = oracle.index_scores(qI, w, kI, nv)
+    errs = []
+    for had in (False, True):
+        qc, qs = oracle.quantize_rows_mxfp4(qI, hadamard=had)
+        kc, ks = oracle.quantize_rows_mxfp4(kI, hadamard=had)
+        s4 = oracle.index_scores(oracle.mxfp4_dequantize(qc, qs), w, oracle.mxfp4_dequantize(kc, ks), nv)
+        errs.append(float(np.sqrt(np.mean((s4 - exact) ** 2)) / np.std(exact)))
+    assert errs[1] < 0.7 * errs[0], errs
+
+
+def test_mxfp4_rejects_bad_width():
+    for n in (16, 48, 0):
+        with pytest.raises(ValueError):
+            oracle.quantize_rows_mxfp4(np.ones((1, n), np.float32) if n else np.ones((1, 0), np.float32))
+    with pytest.raises(ValueError):
+        oracle.mxfp4_dequantize(np.zeros((1, 32), np.uint8), np.full((1, 1), 255, np.uint8))
