@@ -19,7 +19,7 @@ Parity status: every function here is pinned by a ``-m "not gpu"`` test
 (tests/test_oracle_pins.py) except the FP8 *recall* statistic, which the pages
 do not fix ("parity unpinned" for recall only; the e4m3 codec, the FP8 score
 definition, the Hadamard rotation of the index vectors, the MXFP4 codec of the FP4
-index operands and the mixed-precision KV storage codec are pinned).
+index operands, the partial RoPE and the mixed-precision KV storage codec are pinned).
 """
 from __future__ import annotations
 
@@ -71,6 +71,7 @@ def _load():
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_quantize_rows_e4m3.argtypes = [_f32p, i64, i32, _u8p, _f32p]
     lib.oracle_hadamard_rotate.argtypes = [_f64p, i64, i32, _f64p]
+    lib.oracle_rope.argtypes = [_f64p, _i64p, i64, i32, dbl, i32, _f64p]
     lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
     lib.oracle_e2m1_decode.restype = dbl
     lib.oracle_e2m1_encode.argtypes = [dbl]
@@ -93,6 +94,7 @@ def _load():
     for name in ("oracle_compress_csa", "oracle_compress_hca", "oracle_index_scores",
                  "oracle_index_scores_e4m3", "oracle_quantize_rows_e4m3", "oracle_hadamard_rotate",
                  "oracle_quantize_rows_e4m3_hadamard", "oracle_quantize_rows_mxfp4", "oracle_mxfp4_dequantize",
+                 "oracle_rope",
                  "oracle_kv8_quantize",
                  "oracle_kv8_dequantize", "oracle_sparse_attn_partial", "oracle_attn_combine", "oracle_topk",
                  "oracle_sparse_attn", "oracle_hca_attn"):
@@ -293,6 +295,46 @@ def mxfp4_dequantize(codes, scale):
     out = np.empty(c.shape, np.float32)
     _check(lib.oracle_mxfp4_dequantize(c, s, c.size // n, n, out), "mxfp4_dequantize")
     return out
+
+
+def rope(x, pos, theta: float, inverse: bool = False):
+    """Partial RoPE of the last 64 dims ([HA] §6; RoFormer pairs (2i, 2i+1), angle
+    pos * theta^(-2i/64)).  x [..., D] (taken as float64), pos broadcastable to
+    x.shape[:-1] (int) -> float64 [..., D].  inverse turns the other way."""
+    lib = _load()
+    x = np.ascontiguousarray(np.asarray(x, np.float64))
+    D = x.shape[-1]
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, np.int64), x.shape[:-1]).reshape(-1))
+    y = np.empty(x.shape, np.float64)
+    _check(lib.oracle_rope(x, p, x.size // D if D else 0, D, float(theta), int(inverse), y), "rope")
+    return y
+
+
+def compressed_entry_positions(N: int, m: int):
+    """Position of compressed entry i for RoPE: i * m, the first token of its own block
+    (a reading: the pages do not say which token an entry stands for)."""
+    return np.arange(N, dtype=np.int64) * m
+
+
+def sparse_attn_rope(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale, theta: float, m: int,
+                     window: int = 128, kv_pos=None):
+    """sparse_attn with the partial RoPE of [HA] §6 around it: the query rotated at its
+    position, memory entry i at compressed_entry_positions (or kv_pos [B, N]), SWA row j at
+    its token position swa_pos0 + j; attention on the rotated rows (rounded to fp32 for
+    the attention definition); the output's last 64 dims turned back at the query's
+    position.  Shapes as sparse_attn -> float64 [B, T, H, D]."""
+    q = np.asarray(q, np.float64)
+    B, T, H, D = q.shape
+    N, W = np.asarray(kv).shape[1], np.asarray(swa_kv).shape[1]
+    q_pos = np.asarray(q_pos, np.int64)
+    if kv_pos is None:
+        kv_pos = np.broadcast_to(compressed_entry_positions(N, m), (B, N))
+    swa_pos = np.asarray(swa_pos0, np.int64).reshape(B, 1) + np.arange(W, dtype=np.int64)
+    qr = rope(q, q_pos[:, :, None], theta)
+    kvr = rope(kv, kv_pos, theta)
+    swar = rope(swa_kv, swa_pos, theta)
+    o = sparse_attn(qr, kvr, swar, swa_pos0, q_pos, sink, idx, scale, window)
+    return rope(o, q_pos[:, :, None], theta, inverse=True)
 
 
 def kv8_entry_bytes(D: int) -> int:

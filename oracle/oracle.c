@@ -365,6 +365,35 @@ int oracle_mxfp4_dequantize(const uint8_t *codes, const uint8_t *scale, int64_t 
     return ORC_OK;
 }
 
+/* ---- Partial RoPE ([HA] §6: only the last 64 dims of each head are rotated by
+ * position; after the core attention the same dims of the output get the inverse
+ * rotation, before the grouped output projection).  Readings (the pages give no
+ * pairing, base or position rule for compressed entries): the rotary embedding of
+ * the RoFormer paper on dims D-64..D-1, pairs (D-64+2i, D-64+2i+1) for i < 32
+ * turned by the angle pos * theta^(-2i/64); theta is a parameter (the MXFP4 page
+ * gives compress_rope_theta = 160000 for the compressed layers; its YaRN extension
+ * has no stated parameters and is not applied).  inverse != 0 turns by -angle.
+ * x [rows, D] double, pos [rows] int64 -> y [rows, D] double; dims below D-64 are
+ * copied unchanged.  cos / sin of the angle in double. */
+int oracle_rope(const double *x, const int64_t *pos, int64_t rows, int D, double theta, int inverse, double *y)
+{
+    if (D < 64 || D % 2 != 0 || rows < 0 || !(theta > 1.0)) return ORC_BAD;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *xr = x + r * D;
+        double *yr = y + r * D;
+        for (int j = 0; j < D - 64; ++j) yr[j] = xr[j];
+        for (int i = 0; i < 32; ++i) {
+            double ang = (double)pos[r] * pow(theta, -2.0 * i / 64.0);
+            if (inverse) ang = -ang;
+            double c = cos(ang), s = sin(ang);
+            double a = xr[D - 64 + 2 * i], b = xr[D - 64 + 2 * i + 1];
+            yr[D - 64 + 2 * i] = a * c - b * s;
+            yr[D - 64 + 2 * i + 1] = a * s + b * c;
+        }
+    }
+    return ORC_OK;
+}
+
 /* ---- Mixed-precision storage of the compressed KV entries ([HA] §4.2, the
  * paragraph on storage precision: the RoPE dims stay BF16, the rest of each
  * compressed entry is FP8).  Readings (the pages give no granularity or layout):

@@ -863,3 +863,104 @@ def test_mxfp4_rejects_bad_width():
             oracle.quantize_rows_mxfp4(np.ones((1, n), np.float32) if n else np.ones((1, 0), np.float32))
     with pytest.raises(ValueError):
         oracle.mxfp4_dequantize(np.zeros((1, 32), np.uint8), np.full((1, 1), 255, np.uint8))
+
+
+# ----------------------------------------------------------------------------- partial RoPE
+THETA = 160000.0
+
+
+def test_rope_matches_transformers_rotary_embedding():
+    """Library pin: transformers' Llama rotary embedding (its own inverse frequencies, fp32)
+    and apply_rotary_pos_emb rotate pairs (i, i + 32) of a 64-dim head; after moving the
+    interleaved pairs (2i, 2i+1) of the last 64 dims into that layout the two agree."""
+    from transformers import LlamaConfig
+    from transformers.models.llama import modeling_llama as ml
+    cfg = LlamaConfig(hidden_size=64, num_attention_heads=1, head_dim=64, rope_theta=THETA,
+                      max_position_embeddings=1 << 20)
+    emb = ml.LlamaRotaryEmbedding(cfg)
+    pos = np.array([0, 1, 2, 7, 100, 1000, 4095], np.int64)
+    x = RNG.standard_normal((len(pos), 96))
+    got = oracle.rope(x, pos, THETA)
+    assert np.array_equal(got[:, :32], x[:, :32])
+    perm = np.r_[np.arange(0, 64, 2), np.arange(1, 64, 2)]        # interleaved -> half layout
+    xh = torch.from_numpy(x[:, 32:][:, perm]).view(1, 1, len(pos), 64)
+    cos, sin = emb(xh, torch.from_numpy(pos).view(1, -1))
+    ref_h, _ = ml.apply_rotary_pos_emb(xh, xh, cos.double(), sin.double())
+    ref = np.empty((len(pos), 64))
+    ref[:, perm] = ref_h.view(len(pos), 64).numpy()
+    tol = 2e-7 * (pos[:, None] + 1) * np.abs(x[:, 32:]).max()
+    assert np.all(np.abs(got[:, 32:] - ref) <= tol)
+
+
+def test_rope_identity_inverse_norm():
+    """Position 0 is the identity; the inverse undoes the rotation; norms are kept; only the
+    last 64 dims move."""
+    x = RNG.standard_normal((5, 512))
+    pos = np.array([0, 3, 4000, 262143, 1 << 20])
+    y = oracle.rope(x, pos, THETA)
+    assert np.array_equal(y[0], x[0])
+    assert np.array_equal(y[:, :448], x[:, :448])
+    assert np.max(np.abs(oracle.rope(y, pos, THETA, inverse=True) - x)) < 1e-12
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+
+
+def test_rope_relative_position_and_composition():
+    """<R(a) q, R(b) k> depends on a - b only, and R(a) R(b) = R(a + b)."""
+    q, k = RNG.standard_normal((2, 4, 128))
+    a, b, s = np.array([5, 900, 77, 0]), np.array([2, 1000, 77, 65535]), 12345
+    d0 = np.sum(oracle.rope(q, a, THETA) * oracle.rope(k, b, THETA), -1)
+    d1 = np.sum(oracle.rope(q, a + s, THETA) * oracle.rope(k, b + s, THETA), -1)
+    assert np.allclose(d0, d1, rtol=1e-9, atol=1e-9)
+    assert np.allclose(oracle.rope(oracle.rope(q, a, THETA), b, THETA), oracle.rope(q, a + b, THETA), atol=1e-9)
+
+
+def test_rope_pair_frequencies():
+    """RoFormer frequencies: pair 0 turns 1 rad per position, and each next pair turns
+    theta^(-1/32) times slower (a geometric ladder ending at theta^(-62/64))."""
+    x = np.zeros((32, 64))
+    x[np.arange(32), 2 * np.arange(32)] = 1.0
+    y = oracle.rope(x, 1, THETA)
+    ang = np.arctan2(y[np.arange(32), 2 * np.arange(32) + 1], y[np.arange(32), 2 * np.arange(32)])
+    assert abs(ang[0] - 1.0) < 1e-15
+    assert np.allclose(ang[1:] / ang[:-1], THETA ** (-1.0 / 32), rtol=1e-12)
+    assert np.allclose(oracle.rope(x, 1, 10000.0)[1, 2:4], [math.cos(0.01 ** (1 / 16)), math.sin(0.01 ** (1 / 16))])
+
+
+def _rope_case(seed=3, B=2, N=40, k=12, H=4, D=128, W=150):
+    g = np.random.default_rng(seed)
+    t = 4 * N + 3
+    return dict(q=g.standard_normal((B, 1, H, D)), kv=g.standard_normal((B, N, D)), swa=g.standard_normal((B, W, D)),
+                swa_pos0=np.full(B, t - W + 1), q_pos=np.full((B, 1), t), sink=g.standard_normal(H),
+                idx=np.stack([np.sort(g.choice(N, k, replace=False)) for _ in range(B)])[:, None].astype(np.int32))
+
+
+def test_sparse_attn_rope_is_shift_invariant():
+    """Moving every position (query, memory entries, SWA rows) by the same amount leaves the
+    RoPE attention output unchanged: scores see position differences only, and the output
+    is turned back at the query's position."""
+    c = _rope_case()
+    N = c["kv"].shape[1]
+    kv_pos = np.broadcast_to(oracle.compressed_entry_positions(N, 4), (2, N))
+    o0 = oracle.sparse_attn_rope(c["q"], c["kv"], c["swa"], c["swa_pos0"], c["q_pos"], c["sink"], c["idx"], 0.1,
+                                 THETA, 4, kv_pos=kv_pos)
+    s = 100000
+    o1 = oracle.sparse_attn_rope(c["q"], c["kv"], c["swa"], c["swa_pos0"] + s, c["q_pos"] + s, c["sink"], c["idx"],
+                                 0.1, THETA, 4, kv_pos=kv_pos + s)
+    assert np.max(np.abs(o1 - o0)) < 1e-5 * np.max(np.abs(o0))
+
+
+def test_sparse_attn_rope_reduces_to_plain_attention_at_one_position():
+    """With every attended row at the query's own position the rotations cancel: the RoPE
+    attention equals the plain attention of the unrotated inputs (SWA buffer placed outside
+    the window so that only the memory rows count)."""
+    c = _rope_case(seed=9)
+    N = c["kv"].shape[1]
+    t = int(c["q_pos"][0, 0])
+    swa_pos0 = np.full(2, t - 1000)
+    kv_pos = np.full((2, N), t)
+    o = oracle.sparse_attn_rope(c["q"], c["kv"], c["swa"], swa_pos0, c["q_pos"], c["sink"], c["idx"], 0.1, THETA, 4,
+                                kv_pos=kv_pos)
+    plain = oracle.sparse_attn(c["q"], c["kv"], c["swa"], swa_pos0, c["q_pos"], c["sink"], c["idx"], 0.1)
+    assert np.max(np.abs(o - plain)) < 1e-5 * np.max(np.abs(plain))
+    o_far = oracle.sparse_attn_rope(c["q"], c["kv"], c["swa"], swa_pos0, c["q_pos"], c["sink"], c["idx"], 0.1, THETA, 4)
+    assert np.max(np.abs(o_far - plain)) > 1e-3          # real positions do change the result
