@@ -113,6 +113,25 @@ int csa_quantize_e4m3_hadamard(const void *x, int x_dtype, int64_t rows, int col
                                void *stream);
 
 /*
+ * csa_quantize_mxfp4 -- MXFP4 operands for the FP4 index QK ([HA] §2 table and §4.2:
+ * the index QK path runs in FP4; the format is this library's reading, OCP MXFP4).
+ *   per block of 32 consecutive values of a row: X = 2^(floor(log2 amax) - 2), clamped
+ *   to 2^-127 .. 2^127, X = 1 for an all-zero block; element = nearest FP4 E2M1 value
+ *   of v / X (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the even mantissa,
+ *   saturating at 6; the sign is kept (also for zero).
+ *   hadamard != 0: the rows are first rotated as in csa_quantize_e4m3_hadamard (the
+ *   rounded fp32 rotated values are the v above).
+ *   x      : [rows, cols] F32 or BF16 (x_dtype), 16-byte aligned;  cols = 32, 64, 128 or 256
+ *   codes  : [rows, cols/2] bytes, 16-byte aligned; value 2j in the low nibble, 2j+1 in
+ *            the high nibble (sign bit 3, exponent bits 2..1, mantissa bit 0)
+ *   scales : [rows, cols/32] E8M0 bytes (X = 2^(byte - 127))
+ * NaN inputs are not supported.  Returns CSA_ERR_INVALID for any other cols or dtype,
+ * or for an x or codes pointer that is not 16-byte aligned.
+ */
+int csa_quantize_mxfp4(const void *x, int x_dtype, int64_t rows, int cols, int hadamard, uint8_t *codes,
+                       uint8_t *scales, void *stream);
+
+/*
  * csa_index_scores -- Lightning Indexer ([HA] §4.2):
  *   scores[b,t,i] = sum_{h<64} w[b,t,h] * ReLU(<qI[b,t,h,:], kI[b,i,:]>)   for i < n_valid[b,t]
  *   scores[b,t,i] = -inf                                                   for n_valid[b,t] <= i < N

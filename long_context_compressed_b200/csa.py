@@ -34,6 +34,7 @@ _SIGS = {
     "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_quantize_e4m3_hadamard": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
+    "csa_quantize_mxfp4": ([_vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp], _i32),
     "csa_kv8_entry_bytes": ([_i32], ctypes.c_longlong),
     "csa_quantize_kv8": ([_vp, _i64, _i32, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
@@ -119,6 +120,20 @@ def csa_compress(C_a, C_b=None, Z_a=None, Z_b=None, prev_Cb=None, prev_Zb=None, 
     _check(_lib.csa_compress(_ptr(C_a), _ptr(C_b), _ptr(Z_a), _ptr(Z_b), _ptr(prev_Cb), _ptr(prev_Zb), B, L, c,
                              ratio, _dtype_code(C_a), _dtype_code(out), _ptr(out), _stream(stream)), "csa_compress")
     return out
+
+
+def csa_quantize_mxfp4(x, codes=None, scales=None, stream=None, hadamard=False):
+    """MXFP4 of x [..., cols] -> (codes uint8 [..., cols/2] two E2M1 values per byte,
+    scales uint8 [..., cols/32] E8M0); hadamard=True rotates the rows first."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    if codes is None:
+        codes = torch.empty(x.shape[:-1] + (cols // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (cols // 32,), dtype=torch.uint8, device=x.device)
+    _check(_lib.csa_quantize_mxfp4(_ptr(x), _dtype_code(x), rows, cols, int(bool(hadamard)), _ptr(codes),
+                                   _ptr(scales), _stream(stream)), "csa_quantize_mxfp4")
+    return codes, scales
 
 
 def csa_quantize_e4m3(x, codes=None, scale=None, stream=None, hadamard=False):

@@ -463,6 +463,43 @@ int csa_quantize_e4m3_hadamard(const void* x, int x_dtype, int64_t rows, int col
   return launch_status();
 }
 
+int csa_quantize_mxfp4(const void* x, int x_dtype, int64_t rows, int cols, int hadamard, uint8_t* codes,
+                       uint8_t* scales, void* stream) {
+  if (rows < 0 || !(cols == 32 || cols == 64 || cols == 128 || cols == 256)) return CSA_ERR_INVALID;
+  if (x_dtype != CSA_F32 && x_dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (rows == 0) return CSA_OK;
+  if (!x || !codes || !scales) return CSA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(codes)) & 15) return CSA_ERR_INVALID;
+  cudaStream_t st = as_stream(stream);
+#define CSA_LAUNCH_MX(T, N, ROT)                                                                              \
+  do {                                                                                                        \
+    const int64_t rpb = 8 * csa::HadamardCfg<N>::RPW;                                                         \
+    const unsigned blocks = (unsigned)std::min<int64_t>((rows + rpb - 1) / rpb, (int64_t)sm_count() * 2);     \
+    launch_k(csa::quantize_mxfp4_kernel<T, N, ROT>, blocks, 256, 0, st, (const T*)x, rows, codes, scales);     \
+  } while (0)
+#define CSA_LAUNCH_MX_ROT(T, N)        \
+  do {                                 \
+    if (hadamard) CSA_LAUNCH_MX(T, N, true); \
+    else CSA_LAUNCH_MX(T, N, false);   \
+  } while (0)
+#define CSA_LAUNCH_MX_COLS(T)                  \
+  switch (cols) {                              \
+    case 32: CSA_LAUNCH_MX_ROT(T, 32); break;   \
+    case 64: CSA_LAUNCH_MX_ROT(T, 64); break;   \
+    case 128: CSA_LAUNCH_MX_ROT(T, 128); break; \
+    default: CSA_LAUNCH_MX_ROT(T, 256); break;  \
+  }
+  if (x_dtype == CSA_BF16) {
+    CSA_LAUNCH_MX_COLS(__nv_bfloat16)
+  } else {
+    CSA_LAUNCH_MX_COLS(float)
+  }
+#undef CSA_LAUNCH_MX_COLS
+#undef CSA_LAUNCH_MX_ROT
+#undef CSA_LAUNCH_MX
+  return launch_status();
+}
+
 long long csa_kv8_entry_bytes(int D) { return D == csa::kKv8Dims ? (long long)csa::kKv8Bytes : 0; }
 
 int csa_quantize_kv8(const void* kv, int64_t rows, int D, void* entries, void* stream) {

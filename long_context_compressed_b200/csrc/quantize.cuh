@@ -74,6 +74,33 @@ __device__ __forceinline__ void widen16(const uint4 u, double* v, const float*) 
   v[3] = (double)__uint_as_float(u.w);
 }
 
+// The butterflies of one row part (E elements per lane, LPR lanes per row, g = lane in the
+// row), then y = v * c rounded to fp32 with a zero as +0.
+template <int E, int LPR>
+__device__ __forceinline__ void hadamard_lane_part(double* v, int g, double c, float* y) {
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if ((e & h) == 0) {
+        const double a = v[e], b = v[e + h];
+        v[e] = __dadd_rn(a, b);
+        v[e + h] = __dsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < LPR; m <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const double o = __shfl_xor_sync(0xffffffffu, v[e], m);
+      v[e] = (g & m) ? __dsub_rn(o, v[e]) : __dadd_rn(v[e], o);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) y[e] = __double2float_rn(__dadd_rn(__dmul_rn(v[e], c), 0.0));
+}
+
 template <typename Tin, int N>
 __global__ void __launch_bounds__(256, 2) hadamard_quantize_e4m3_kernel(const Tin* __restrict__ x, int64_t rows,
                                                                         uint8_t* __restrict__ codes,
@@ -103,32 +130,11 @@ __global__ void __launch_bounds__(256, 2) hadamard_quantize_e4m3_kernel(const Ti
     double v[E];
 #pragma unroll
     for (int k = 0; k < NV; ++k) widen16(raw[k], v + k * VEC, x);
-#pragma unroll
-    for (int h = 1; h < E; h <<= 1) {
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        if ((e & h) == 0) {
-          const double a = v[e], b = v[e + h];
-          v[e] = __dadd_rn(a, b);
-          v[e + h] = __dsub_rn(a, b);
-        }
-      }
-    }
-#pragma unroll
-    for (int m = 1; m < LPR; m <<= 1) {
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const double o = __shfl_xor_sync(0xffffffffu, v[e], m);
-        v[e] = (g & m) ? __dsub_rn(o, v[e]) : __dadd_rn(v[e], o);
-      }
-    }
     float y[E];
+    hadamard_lane_part<E, LPR>(v, g, c, y);
     float amax = 0.f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      y[e] = __double2float_rn(__dadd_rn(__dmul_rn(v[e], c), 0.0));
-      amax = fmaxf(amax, fabsf(y[e]));
-    }
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
 #pragma unroll
     for (int m = 1; m < LPR; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
     const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
@@ -151,6 +157,94 @@ __global__ void __launch_bounds__(256, 2) hadamard_quantize_e4m3_kernel(const Ti
           *reinterpret_cast<uint4*>(cr + 4 * q) = make_uint4(packed[q], packed[q + 1], packed[q + 2], packed[q + 3]);
       }
       if (g == 0) scale[r] = s;
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) raw[k] = nxt[k];
+  }
+}
+
+// MXFP4 operands for the FP4 index QK ("DeepSeek-V4 混合注意力：从压缩记忆到百万上下文" §2
+// table and §4.2: the index QK runs in FP4).  OCP MX: E2M1 elements with one E8M0 scale
+// per 32 consecutive values, X = 2^(floor(log2 amax) - 2) clamped to 2^-127 .. 2^127 (an
+// all-zero block: X = 1); element = nearest E2M1 value of y / X, ties to the even
+// mantissa, saturating at 6.  With ROT the rows are first Walsh-Hadamard-rotated exactly
+// as in hadamard_quantize_e4m3_kernel.  Layout: codes [rows, N/2] bytes, element 2j in
+// the low nibble and 2j+1 in the high nibble; scales [rows, N/32] E8M0 bytes.
+
+// Nearest E2M1 magnitude code of a >= 0: the count of rounding thresholds passed, where a
+// tie (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) goes to the code with mantissa bit 0.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  const uint32_t m = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+                     (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) + (uint32_t)(a > 5.0f);
+  return (signbit(v) ? 8u : 0u) | m;
+}
+
+template <typename Tin, int N, bool ROT>
+__global__ void __launch_bounds__(256, 2) quantize_mxfp4_kernel(const Tin* __restrict__ x, int64_t rows,
+                                                                uint8_t* __restrict__ codes,
+                                                                uint8_t* __restrict__ scales) {
+  using C = HadamardCfg<N>;
+  constexpr int E = C::E, LPR = C::LPR, RPW = C::RPW;
+  constexpr int VEC = 16 / (int)sizeof(Tin);
+  constexpr int NV = E / VEC;
+  constexpr int LPB = 32 / E;                  // lanes per 32-value block
+  static_assert(E % 8 == 0 && 32 % E == 0, "a lane holds a whole number of bytes of one block");
+  griddep_sync();
+  const double c = __ddiv_rn(1.0, __dsqrt_rn((double)N));
+  const int lane = (int)lane_id();
+  const int g = lane % LPR;
+  const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5) * RPW;
+  auto fetch = [&](int64_t rr, uint4* dst) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+      dst[k] = rr < rows ? __ldg(reinterpret_cast<const uint4*>(x + rr * N + g * E + k * VEC)) : make_uint4(0, 0, 0, 0);
+  };
+  int64_t r0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+  uint4 raw[NV];
+  fetch(r0 + lane / LPR, raw);
+  for (; r0 < rows; r0 += step) {
+    const int64_t r = r0 + lane / LPR;
+    uint4 nxt[NV];
+    fetch(r + step, nxt);
+    double v[E];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) widen16(raw[k], v + k * VEC, x);
+    float y[E];
+    if constexpr (ROT) {
+      hadamard_lane_part<E, LPR>(v, g, c, y);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) y[e] = (float)v[e];      // exact: v holds widened inputs
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
+#pragma unroll
+    for (int m = 1; m < LPB; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    int ex = 0;
+    if (amax > 0.f) {
+      int E2;
+      frexpf(amax, &E2);                          // amax = f 2^E2, f in [0.5, 1)
+      ex = E2 - 3;
+      ex = ex < -127 ? -127 : (ex > 127 ? 127 : ex);
+    }
+    if (r < rows) {
+      uint32_t packed[E / 8];
+#pragma unroll
+      for (int q = 0; q < E / 8; ++q) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) word |= e2m1_code(ldexpf(y[8 * q + j], -ex)) << (4 * j);
+        packed[q] = word;
+      }
+      uint8_t* cr = codes + (r * N + g * E) / 2;
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint32_t*>(cr) = packed[0];
+      } else {
+        *reinterpret_cast<uint2*>(cr) = make_uint2(packed[0], packed[1]);
+      }
+      if (g % LPB == 0) scales[r * (N / 32) + g / LPB] = (uint8_t)(ex + 127);
     }
 #pragma unroll
     for (int k = 0; k < NV; ++k) raw[k] = nxt[k];

@@ -158,3 +158,21 @@ def test_hadamard_quantizer_host_checks(lib):
     assert f(p, 1, 4, 128, p + 4, p, None) == 1      # codes not 16-byte aligned
     for cols in (32, 64, 128, 256):
         assert f(p, 1, 0, cols, p, p, None) == 0     # nothing to do
+
+
+def test_mxfp4_quantizer_host_checks(lib):
+    f = lib.csa_quantize_mxfp4
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    p = 16
+    for cols in (0, 16, 48, 96, 512):
+        assert f(p, 1, 4, cols, 0, p, p, None) == 1, cols
+    assert f(p, 2, 4, 128, 0, p, p, None) == 1          # e4m3 input
+    assert f(p, 1, -1, 128, 1, p, p, None) == 1
+    assert f(None, 1, 4, 128, 1, p, p, None) == 1
+    assert f(p, 1, 4, 128, 1, p, None, None) == 1
+    assert f(p + 8, 1, 4, 128, 0, p, p, None) == 1      # x not 16-byte aligned
+    assert f(p, 1, 4, 128, 0, p + 8, p, None) == 1      # codes not 16-byte aligned
+    for cols in (32, 64, 128, 256):
+        assert f(p, 1, 0, cols, 1, p, p, None) == 0
