@@ -967,6 +967,73 @@ def oracle_baseline(wl, index, with_hca, budget_s=12.0, max_tokens=24):
                       f"{cpu_model()}"}
 
 
+def oracle_config_timings(seed=2000):
+    """The CPU oracle (single-threaded fp64 C) on the other configurations, one bounded
+    sample each: the whole tiny step (8 queries); one pro1m decode token (the same chain as
+    the GPU step: rotated e4m3 scores, 2k candidates, exact rerank, sparse_attn); one
+    pro_hca sequence (128:1 compressor over the 16,384-token tail, hca_attn over 8,192 + 128
+    rows); the flash_prefill chunk's compressors in full plus 8 of its 4,096 queries (index,
+    top-512, sparse_attn), extrapolated to the chunk.  Input preparation is not timed."""
+    import numpy as np
+
+    import oracle
+    from long_context_compressed_b200 import synth
+    W = synth.WORKLOADS
+    np32 = lambda t: t.float().numpy()
+    out = {}
+    # tiny: the whole step
+    wl = W["tiny"]
+    cz, ix, at = synth.draw_compressor(wl, seed), synth.draw_indexer(wl, seed), synth.draw_attention(wl, seed)
+    q_pos = np.array([wl.q_pos], np.int64)
+    nv = oracle.n_visible(q_pos, 4, wl.N)
+    t0 = time.perf_counter()
+    oracle.compress_csa(*(np32(cz[n]) for n in ("C_a", "C_b", "Z_a", "Z_b")))
+    s = oracle.index_scores(np32(ix["qI"]), np32(ix["w"]), np32(ix["kI"]), nv)
+    idx = oracle.topk(s.astype(np.float32), nv, wl.topk)
+    oracle.sparse_attn(np32(at["q"]), np32(at["kv"]), np32(at["swa_kv"]), [wl.swa_pos0], q_pos, np32(at["sink"]),
+                       idx, 1 / math.sqrt(wl.D))
+    dt = time.perf_counter() - t0
+    out["tiny"] = {"ms_per_step": 1e3 * dt, "tokens_per_s": wl.T / dt, "sample": "the whole 8-query step"}
+    # pro1m: one decode token
+    dt = oracle_decode_token(W["pro1m"], seed, "e4m3", False)
+    out["pro1m"] = {"ms_per_step": 1e3 * dt, "tokens_per_s": 1 / dt, "sample": "one decode token (B=1)"}
+    # pro_hca: one of the 4 sequences
+    wl = W["pro_hca"]
+    one = synth.Workload(**{**wl.__dict__, "B": 1, "extra": {}})
+    hz, at = synth.draw_compressor(one, seed), synth.draw_attention(one, seed)
+    q_pos = np.array([[one.q_pos0]], np.int64)
+    t0 = time.perf_counter()
+    oracle.compress_hca(np32(hz["C"]), np32(hz["Z"]))
+    oracle.hca_attn(np32(at["q"]), np32(at["kv"]), np32(at["swa_kv"]), [one.swa_pos0], q_pos, np32(at["sink"]),
+                    1 / math.sqrt(one.D))
+    dt = time.perf_counter() - t0
+    out["pro_hca"] = {"ms_per_step": 1e3 * dt * wl.B, "tokens_per_s": 1 / dt,
+                      "sample": f"one of the {wl.B} sequences, x{wl.B} for the step"}
+    # flash_prefill: compressors in full, 8 sampled queries, extrapolated
+    wl = W["flash_prefill"]
+    cz = synth.draw_compressor(wl, seed)
+    czi = synth.draw_compressor(wl, seed, c=wl.comp_ci, tag="ki")
+    ix, at = synth.draw_indexer(wl, seed), synth.draw_attention(wl, seed)
+    rows = np.linspace(0, wl.T - 1, 8).round().astype(int)
+    q_pos = np.array([[wl.q_pos0 + int(r) for r in rows]], np.int64)
+    nv = oracle.n_visible(q_pos, 4, wl.N)
+    t0 = time.perf_counter()
+    for z in (cz, czi):
+        oracle.compress_csa(*(np32(z[n]) for n in ("C_a", "C_b", "Z_a", "Z_b", "prev_Cb", "prev_Zb")))
+    t_comp = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    s = oracle.index_scores(np32(ix["qI"][:, rows]), np32(ix["w"][:, rows]), np32(ix["kI"]), nv)
+    idx = oracle.topk(s.astype(np.float32), nv, wl.topk)
+    oracle.sparse_attn(np32(at["q"][:, rows]), np32(at["kv"]), np32(at["swa_kv"]), [wl.swa_pos0], q_pos,
+                       np32(at["sink"]), idx, 1 / math.sqrt(wl.D))
+    t_q = (time.perf_counter() - t0) / len(rows)
+    total = t_comp + t_q * wl.T
+    out["flash_prefill"] = {"ms_per_step": 1e3 * total, "tokens_per_s": wl.T / total, "extrapolated": True,
+                            "sample": f"both chunk compressors in full ({1e3 * t_comp:.1f} ms) plus {len(rows)} of "
+                                      f"the {wl.T} queries ({1e3 * t_q:.1f} ms each), scaled to {wl.T} queries"}
+    return {"cores": 1, "kind": "oracle", "cpu": cpu_model(), "configs": out}
+
+
 def workload_text(wl, index, with_hca):
     """The JSON line's config.workload, the same for both arms."""
     return (f"{wl.name}: B={wl.B} decode tokens/GPU at ctx {wl.ctx}; CSA layer (compress 4:1 c=512+128, "
@@ -1057,9 +1124,11 @@ def main():
             kv8_runs[nm] = bench_workload(nm, args.index, nm == "flash64k", args.steps, args.warmup, world, device,
                                           kv8=True)
         kv8_runs["pro_hca"] = bench_hca(args.steps, args.warmup, device, peak, kv8=True)
-    cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    cpu = oracle_cfg = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:       # the oracle leg: one process, N = 1
         cpu = oracle_baseline(main_res["wl"], args.index, with_hca)
+        if not args.no_extra:
+            oracle_cfg = oracle_config_timings()
     if rank != 0:
         return
 
@@ -1145,6 +1214,8 @@ def main():
         line["kv8"] = kv
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if oracle_cfg is not None:
+        line["oracle_configs"] = oracle_cfg
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
