@@ -43,13 +43,24 @@ _vp = ctypes.c_void_p
 
 
 def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so (gcc, -O2, no fast-math, no FMA contraction)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+    """Compile oracle.c into liboracle.so (gcc, -O2, no fast-math, no FMA contraction).
+
+    With CSA_ORACLE_SANITIZE=1 in the environment the library is built with AddressSanitizer
+    and UndefinedBehaviorSanitizer instead (liboracle_san.so); the process then needs the
+    sanitizer runtimes preloaded, e.g.
+    LD_PRELOAD="$(gcc -print-file-name=libasan.so):$(gcc -print-file-name=libubsan.so)"
+    ASAN_OPTIONS=detect_leaks=0 UBSAN_OPTIONS=halt_on_error=1 CSA_ORACLE_SANITIZE=1 \
+        python -m pytest tests/test_oracle_pins.py"""
+    lib, flags = _LIB, ["-O2"]
+    if os.environ.get("CSA_ORACLE_SANITIZE"):
+        lib = os.path.join(_HERE, "liboracle_san.so")
+        flags = ["-O1", "-g", "-fsanitize=address,undefined", "-fno-omit-frame-pointer"]
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(_SRC):
+        tmp = lib + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *flags, "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
                                "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 def _load():
