@@ -214,7 +214,7 @@ class DecodeSet:
         self.sink = f32("sink", (H,))
         self.q_pos = torch.full((B, T), wl.q_pos0, dtype=torch.int64, device=dev)
         self.swa_pos0 = torch.full((B,), wl.swa_pos0, dtype=torch.int64, device=dev)
-        self.n_valid = csa.n_valid_for(self.q_pos, 4, N)
+        self.n_valid = csa.csa_n_valid(self.q_pos, 4, 0, N)
         # per-step inputs
         cL, cc = wl.comp_L, wl.comp_c
         self.inputs = {
@@ -229,7 +229,9 @@ class DecodeSet:
                                 "iprev_Cb": g("iprev_Cb", (B, 4, ci)), "iprev_Zb": g("iprev_Zb", (B, 4, ci))})
         # outputs and scratch
         self.comp_kv = torch.empty((B, cL // 4, cc), dtype=torch.bfloat16, device=dev)
-        self.comp_ki = torch.empty((B, cL // 4, wl.comp_ci or 8), dtype=torch.bfloat16, device=dev)
+        # new index-key entries go straight into the caches' newest rows (bf16 keys and, on
+        # the e4m3 path, their rotated e4m3 codes and scales): rows N - L/4 .. N - 1
+        self.new_key_pos = N - cL // 4
         self.scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         self.q8 = torch.empty((B, T, 64, 128), dtype=torch.uint8, device=dev)
         self.qs = torch.empty((B, T, 64), dtype=torch.float32, device=dev)
@@ -300,7 +302,9 @@ class DecodeSet:
         B, T, N, H, D, k = wl.B, wl.T, wl.N, wl.H, wl.D, wl.topk
         nb = lambda t: t.numel() * t.element_size()
         total = sum(nb(t) for t in self.inputs.values())                       # per-step inputs
-        total += nb(self.comp_kv) + (nb(self.comp_ki) if wl.comp_ci else 0)   # compressor outputs
+        total += nb(self.comp_kv)                                             # latent compressor output
+        if wl.comp_ci:                                                        # new index keys (+ e4m3)
+            total += B * (wl.comp_L // 4) * (256 + (132 if self.index == "e4m3" else 0))
         total += B * N * (132 if self.index == "e4m3" else 256)               # index keys (+ scales)
         if self.index == "e4m3":
             total += B * T * 2 * k * 256                                      # rerank: bf16 keys of candidates
@@ -330,30 +334,40 @@ class DecodeSet:
         if copies:
             self.in_buf.copy_(self.host_in, non_blocking=True)
         def side_branch():
-            # compressors and the HCA layer: independent of the indexer chain and of each
-            # other within a step, so they run on side streams, started once the
+            # the latent compressor and the HCA layer: independent of the indexer chain and
+            # of each other within a step, so they run on side streams, started once the
             # bandwidth-bound indexer is done and overlapping the latency-bound top-k /
             # rerank / attention kernels
             sa, sb, sc = side_streams
-            for ss in side_streams:
-                ss.wait_stream(main)
+            sa.wait_stream(main)
+            sc.wait_stream(main)
             with torch.cuda.stream(sa):
                 csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"], ratio=4,
                                  out=self.comp_kv)
                 if self.kv8:
                     csa.quantize_kv8(self.comp_kv, entries=self.comp_kv8)
-            with torch.cuda.stream(sb):
-                if wl.comp_ci:
-                    csa.csa_compress(x["iC_a"], x["iC_b"], x["iZ_a"], x["iZ_b"], x["iprev_Cb"], x["iprev_Zb"],
-                                     ratio=4, out=self.comp_ki)
-                if self.with_hca:
+            if self.with_hca:
+                with torch.cuda.stream(sc):
                     csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=self.hcomp)
                     if self.kv8:
                         csa.quantize_kv8(self.hcomp, entries=self.hcomp8)
-            if self.with_hca:
-                with torch.cuda.stream(sc):
                     csa.hca_attn(x["hq"], self.hkv_store, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
                                  1.0 / math.sqrt(wl.D), out=self.hout, workspace=self.hattn_ws)
+
+        def append_index_keys():
+            # the step's new index-key entries, compressed, rotated and quantised in one launch
+            # into the caches' newest rows; after the select, the last reader of the bf16 keys
+            # in this step, so the next step's indexer scans them
+            sb = side_streams[1]
+            sb.wait_stream(main)
+            if wl.comp_ci:
+                with torch.cuda.stream(sb):
+                    e4 = self.index == "e4m3"
+                    csa.csa_compress_index_keys(x["iC_a"], x["iC_b"], x["iZ_a"], x["iZ_b"], x["iprev_Cb"],
+                                                x["iprev_Zb"], self.kI, pos0=self.new_key_pos,
+                                                k8=self.k8 if e4 else None, k_scale=self.ks if e4 else None,
+                                                hadamard=INDEX_ROTATION)
+
         # stage boundaries on the main stream (event record nodes inside the graph)
         # timing_events: False (the timed graphs) or "all" (every stage: a diagnostic graph;
         # event nodes break the programmatic-launch overlap and add their own latency)
@@ -383,6 +397,7 @@ class DecodeSet:
             side_branch()
             csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, idx=self.idx)
             mark("select")
+        append_index_keys()
         csa.sparse_attn(x["q"], self.kv_store, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
                         1.0 / math.sqrt(wl.D), out=self.out, workspace=self.attn_ws)
         mark("sparse_attn")
@@ -611,7 +626,7 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     t_e2e = max_over_ranks(timed_steps(sets, side, steps, warmup, world, copies=True), world, device)
     assert csa.csa_poll_status() == csa.CSA_OK
     h2d, d2h = probe.per_step_io()
-    res = {"wl": wl, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
+    res = {"wl": wl, "index": index, "with_hca": with_hca, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
            "index_ms": idx_ms, "index_bytes": probe.index_bytes(), "step_bytes": touched,
            "attn_ms": attn_ms, "attn_bytes": probe.attn_bytes(),
            "e2e_seconds": t_e2e, "h2d": h2d, "d2h": d2h, "tokens_per_step": wl.B * wl.T,
@@ -665,9 +680,8 @@ def bench_prefill(steps, warmup, device, tflops_peak):
     ip = {nm: g("i" + nm, (B, 4, ci)) for nm in ("prev_Cb", "prev_Zb")}
     q_pos = (torch.arange(T, device=dev, dtype=torch.int64) + wl.q_pos0).view(1, T).repeat(B, 1)
     swa_pos0 = torch.full((B,), wl.swa_pos0, dtype=torch.int64, device=dev)
-    n_valid = csa.n_valid_for(q_pos, 4, N)
+    n_valid = csa.csa_n_valid(q_pos, 4, 0, N)
     comp_kv = torch.empty((B, cL // 4, cc), dtype=torch.bfloat16, device=dev)
-    comp_ki = torch.empty((B, cL // 4, ci), dtype=torch.bfloat16, device=dev)
     scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
     idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
     topk_ws = csa.topk_workspace(B, T, N, k, dev)
@@ -680,8 +694,10 @@ def bench_prefill(steps, warmup, device, tflops_peak):
     stages = [
         ("compress", lambda: (csa.csa_compress(cz["C_a"], cz["C_b"], cz["Z_a"], cz["Z_b"], cp["prev_Cb"],
                                                cp["prev_Zb"], ratio=4, out=comp_kv),
-                              csa.csa_compress(iz["C_a"], iz["C_b"], iz["Z_a"], iz["Z_b"], ip["prev_Cb"],
-                                               ip["prev_Zb"], ratio=4, out=comp_ki))),
+                              # the chunk's index keys, into the caches' newest rows (bf16 + e4m3)
+                              csa.csa_compress_index_keys(iz["C_a"], iz["C_b"], iz["Z_a"], iz["Z_b"],
+                                                          ip["prev_Cb"], ip["prev_Zb"], kI, pos0=N - cL // 4,
+                                                          k8=k8, k_scale=ks, hadamard=INDEX_ROTATION))),
         ("index", lambda: csa.csa_index_scores(qI, w, kI, n_valid, scores=scores)),
         ("topk", lambda: csa.csa_topk(scores, n_valid, k, idx=idx, workspace=topk_ws)),
         ("sparse_attn", lambda: csa.sparse_attn(q, kv, swa, swa_pos0, q_pos, sink, idx, scale, out=out,
@@ -814,7 +830,7 @@ def run_big_stage(stage, steps, warmup, device):
     elif stage in ("prefill_index", "prefill_index8", "prefill_topk"):
         qI, kI = g("qI", (B, T, 64, 128)), g("kI", (B, N, 128))
         w = synth.normal(0, f"bench/{wl.name}/w", (B, T, 64), device=dev)
-        n_valid = csa.n_valid_for(q_pos, 4, N)
+        n_valid = csa.csa_n_valid(q_pos, 4, 0, N)
         scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         if stage == "prefill_index8":
             q8, qs = csa.csa_quantize_e4m3(qI, hadamard=INDEX_ROTATION)
@@ -829,7 +845,7 @@ def run_big_stage(stage, steps, warmup, device):
             fn = lambda: csa.csa_topk(scores, n_valid, k, idx=idx, workspace=ws)
     elif stage == "prefill_attn":
         q, kv, swa = g("q", (B, T, H, D)), g("kv", (B, N, D)), g("swa", (B, wl.W, D))
-        idx = synth.random_subset(0, f"bench/{wl.name}/idx", csa.n_valid_for(q_pos, 4, N).cpu(), k, device=dev)
+        idx = synth.random_subset(0, f"bench/{wl.name}/idx", csa.csa_n_valid(q_pos, 4, 0, N).cpu(), k, device=dev)
         out = torch.empty_like(q)
         fn = lambda: csa.sparse_attn(q, kv, swa, swa_pos0, q_pos, sink, idx, 1.0 / math.sqrt(D), out=out)
     elif stage == "hca_compress":
@@ -1114,6 +1130,15 @@ def main():
     extra = None
     if not args.no_extra and args.workload != "pro1m":
         extra = bench_workload("pro1m", args.index, False, args.steps, args.warmup, world, device)
+    variants = {}
+    if not args.no_extra and args.workload == "flash64k":
+        # the same configuration with the bf16 indexer (BASELINE's FP8 and BF16 variants),
+        # and the plain CSA layer without the HCA layer beside it
+        other = "bf16" if args.index == "e4m3" else "e4m3"
+        variants[f"flash64k_{other}_index"] = bench_workload("flash64k", other, True, args.steps, args.warmup, world,
+                                                             device)
+        variants["flash64k_csa_only"] = bench_workload("flash64k", args.index, False, args.steps, args.warmup, world,
+                                                       device)
     prefill = hca = None
     kv8_runs = {}
     if not args.no_extra:
@@ -1154,12 +1179,12 @@ def main():
                                    "CUDA events around the graph replays",
                          "why_this_kernel": "largest share of the step in the ncu launch list (two launches per "
                                             "step: CSA sparse_attn and HCA hca_attn)"},
-            "roofline_indexer": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if args.index == "e4m3"
+            "roofline_indexer": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if r["index"] == "e4m3"
                          else "index_tc_kernel (csa_index_scores, bf16)",
                          "achieved": idx_gbs, "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak,
                          "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
                          "traffic": profiled_traffic("index_tc_kernel_e4m3_decode.md", "index.cuh", wl.name)
-                         if args.index == "e4m3" else None,
+                         if r["index"] == "e4m3" else None,
                          "bytes_per_launch": r["index_bytes"], "avg_launch_us": r["index_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays"},
@@ -1194,6 +1219,13 @@ def main():
                          "roofline_indexer": e["roofline_indexer"], "e2e": e["e2e"],
                          "indexer_keys_per_s": e["indexer_keys_per_s"], "launches_per_step": e["launches_per_step"],
                          "breakdown_us": e["breakdown_us"]}
+        line["gpu_launches"] += e["gpu_launches"]
+    for nm, r in variants.items():
+        e = summarise(r)
+        line[nm] = {"value": e["value"], "unit": "tokens/s", "ms_per_step": e["ms_per_step"],
+                    "workload": workload_text(r["wl"], r["index"], r["with_hca"]),
+                    "step_roofline": e["step_roofline"], "roofline_indexer": e["roofline_indexer"], "e2e": e["e2e"],
+                    "launches_per_step": e["launches_per_step"], "breakdown_us": e["breakdown_us"]}
         line["gpu_launches"] += e["gpu_launches"]
     if prefill is not None:
         line["prefill"] = prefill

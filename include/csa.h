@@ -56,6 +56,21 @@ const char *csa_status_string(int status);
 int csa_version(void);
 
 /*
+ * csa_n_valid -- how many compressed entries each query may see ([HA] §6: a query at
+ * absolute position t attends to entry i only once its block of `ratio` raw tokens
+ * is complete, (i + 1) * ratio <= t + 1):
+ *   n_valid[i] = clamp(floor((q_pos[i] + 1) / ratio) - lo, 0, hi - lo)   (0 for q_pos[i] < 0)
+ * for a device that holds the sequence's entries [lo, hi); a device that holds all N
+ * entries passes lo = 0, hi = N.  The result is the n_valid argument of
+ * csa_index_scores, csa_topk and csa_topk_select.
+ *   q_pos   : [count] int64 absolute positions (device)
+ *   n_valid : [count] int32 (device)
+ *   ratio >= 1, 0 <= lo <= hi, hi - lo <= INT32_MAX; CSA_ERR_INVALID otherwise.
+ */
+int csa_n_valid(const int64_t *q_pos, int64_t count, int ratio, int64_t lo, int64_t hi, int32_t *n_valid,
+                void *stream);
+
+/*
  * csa_compress -- token-level Compressor ([HA] §4.1 for ratio 4, §5 for 128).
  *
  * ratio 4 (CSA, overlapped two-branch pooling):
@@ -77,6 +92,24 @@ int csa_version(void);
 int csa_compress(const void *C_a, const void *C_b, const void *Z_a, const void *Z_b, const void *prev_Cb,
                  const void *prev_Zb, int B, int64_t L, int c, int ratio, int in_dtype, int out_dtype, void *out,
                  void *stream);
+
+/*
+ * csa_compress_index_keys -- a step's new index-key entries, written straight into the
+ * indexer's caches in one launch ([HA] §4.1 compressor over the index keys; §7: the
+ * Indexer compresses its own keys; §4.2: its QK runs in low precision):
+ *   entry i of sequence b = csa_compress(ratio 4) of the c = 128 index-key channels, bit
+ *   for bit, rounded to bf16 and stored at row pos0 + i of kI [B, n_cap, 128] bf16;
+ *   with k8 != NULL that stored bf16 row is also quantised exactly as
+ *   csa_quantize_e4m3_hadamard (hadamard != 0) or csa_quantize_e4m3 (hadamard == 0)
+ *   quantises it, into row pos0 + i of k8 [B, n_cap, 128] e4m3 and k_scale [B, n_cap] fp32.
+ *   C_a, C_b, Z_a, Z_b : [B, L, 128] in_dtype (F32|BF16); prev_Cb, prev_Zb : [B, 4, 128] or
+ *   both NULL (see csa_compress); L / 4 entries per sequence (a partial block makes none);
+ *   0 <= pos0, pos0 + L/4 <= n_cap.  k8 and k_scale are both NULL or both set.
+ *   Pointers 16-byte aligned.  CSA_ERR_INVALID otherwise.
+ */
+int csa_compress_index_keys(const void *C_a, const void *C_b, const void *Z_a, const void *Z_b, const void *prev_Cb,
+                            const void *prev_Zb, int B, int64_t L, int in_dtype, int hadamard, int64_t n_cap,
+                            int64_t pos0, void *kI, uint8_t *k8, float *k_scale, void *stream);
 
 /*
  * csa_quantize_e4m3 -- per-row symmetric e4m3 quantisation for the
@@ -141,7 +174,7 @@ int csa_quantize_mxfp4(const void *x, int x_dtype, int64_t rows, int cols, int h
  *   w       : [B, T, 64] fp32
  *   kI      : [B, N, 128] dtype   (keys shared by the 64 heads)
  *   k_scale : [B, N] fp32 (E4M3 only, else NULL)
- *   n_valid : [B, T] int32, 0 <= n_valid <= N (visible complete entries, (t+1)/4)
+ *   n_valid : [B, T] int32, 0 <= n_valid <= N (visible complete entries: csa_n_valid)
  *   scores  : [B, T, N] fp32
  *   select_ws : NULL, or (T == 1 only) a csa_topk_select workspace: the call then
  *               also accumulates each row's 4096-bin histogram of its valid scores
@@ -172,24 +205,28 @@ int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t 
              void *workspace, size_t ws_bytes, void *stream);
 
 /*
- * csa_topk_noalloc -- csa_topk without a caller-provided workspace.  The pages
- * have no counterpart: this entry point exists for callers that cannot allocate
- * device memory -- code that runs while a CUDA stream is being captured (an
- * allocation there breaks or is refused by the capture), embedded or real-time
- * hosts that fix their device memory at start-up, and C callers with no device
- * allocator of their own.
- *   Same arguments and results as csa_topk, minus the workspace.  Rows that need
- *   scratch (see csa_topk_workspace_size) use a library-owned device array of
+ * csa_topk_noalloc -- csa_topk without a caller-provided workspace.  The pages have
+ * no counterpart: this entry point is for callers that cannot allocate device
+ * memory themselves -- a host that reserves its whole device-memory budget at
+ * start-up and forbids allocation afterwards (embedded or latency-critical
+ * serving), a plug-in that runs inside another application which owns the device
+ * allocator, or plain C code with no device allocator of its own.
+ *   Same arguments, checks and results as csa_topk, minus the workspace.  Rows that
+ *   need scratch (see csa_topk_workspace_size) use a library-owned device array of
  *   CSA_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads the library
  *   holds until the process exits; a call whose csa_topk_workspace_size exceeds
- *   it returns CSA_ERR_UNSUPPORTED and launches nothing.  No cudaMalloc / cudaFree
- *   is ever made: the array is cleared with cudaMemsetAsync on `stream` at the
- *   start of each call.
+ *   it returns CSA_ERR_UNSUPPORTED.  Every argument is checked before the array is
+ *   touched: a rejected call enqueues nothing.  No cudaMalloc / cudaFree (or any
+ *   allocating routine) is ever made; each call clears the part of the array it
+ *   uses with cudaMemsetAsync on `stream`, since the array keeps whatever the
+ *   previous call left in it.
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  All calls share the one array: calls that may
- *   overlap on the GPU (different streams, or graphs replayed concurrently)
- *   race and give wrong results -- order them on one stream.
+ *   (cudaGetSymbolAddress) with that device current and keeps it for later calls;
+ *   make that first call before any stream capture, and do not use this entry
+ *   point after cudaDeviceReset (the kept address would be stale).  All calls share
+ *   the one array: calls that may overlap on the GPU (different streams, or work
+ *   replayed concurrently) race on it and give wrong results -- order them on one
+ *   stream.
  */
 #define CSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 int csa_topk_noalloc(const float *scores, const int32_t *n_valid, int B, int T, int64_t N, int k, int32_t *idx,
@@ -375,6 +412,17 @@ unsigned long long csa_launch_count(void);
  * wait since the last poll).  CSA_ERR_CUDA if synchronisation fails.
  */
 int csa_poll_status(void *stream);
+
+/*
+ * csa_test_bounded_wait -- a check of the failure-detection path (no counterpart in
+ * the pages): one kernel thread waits on a shared-memory barrier that completes only
+ * if `complete` is non-zero, with the bound limit_ns nanoseconds of the GPU's global
+ * timer.  If the bound runs out the kernel records CSA_ERR_TIMEOUT in the device status
+ * word and returns, exactly as every wait inside the library's kernels does; the
+ * next csa_poll_status returns that code and clears it.  No GPU fault is involved.
+ *   1000 <= limit_ns <= 10^9; CSA_ERR_INVALID otherwise.
+ */
+int csa_test_bounded_wait(int complete, long long limit_ns, void *stream);
 
 #ifdef __cplusplus
 }

@@ -31,7 +31,10 @@ _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctyp
 _SIGS = {
     "csa_status_string": ([_i32], ctypes.c_char_p),
     "csa_version": ([], _i32),
+    "csa_n_valid": ([_vp, _i64, _i32, _i64, _i64, _vp, _vp], _i32),
     "csa_compress": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
+    "csa_compress_index_keys": ([_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i64, _i64, _vp, _vp, _vp,
+                                 _vp], _i32),
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_quantize_e4m3_hadamard": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_quantize_mxfp4": ([_vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp], _i32),
@@ -59,6 +62,7 @@ _SIGS = {
     "csa_shard_remap": ([_vp, _i64, _i64, _i64, _i64, _vp, _vp], _i32),
     "csa_launch_count": ([], ctypes.c_ulonglong),
     "csa_poll_status": ([_vp], _i32),
+    "csa_test_bounded_wait": ([_i32, ctypes.c_longlong, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -110,6 +114,16 @@ def csa_version() -> int:
     return _lib.csa_version()
 
 
+def csa_n_valid(q_pos, ratio: int, lo: int = 0, hi: int = 0, *, out=None, stream=None):
+    """Visible compressed entries per query, q_pos [...] int64 -> n_valid [...] int32, computed by
+    the library (entries [lo, hi) held here; pass hi = N for a whole sequence)."""
+    if out is None:
+        out = torch.empty(q_pos.shape, dtype=torch.int32, device=q_pos.device)
+    _check(_lib.csa_n_valid(_ptr(q_pos), q_pos.numel(), int(ratio), int(lo), int(hi), _ptr(out), _stream(stream)),
+           "csa_n_valid")
+    return out
+
+
 def csa_compress(C_a, C_b=None, Z_a=None, Z_b=None, prev_Cb=None, prev_Zb=None, *, ratio=4, out=None,
                  out_dtype=None, stream=None):
     """Compressor.  ratio 4: C_a, C_b, Z_a, Z_b [B, L, c] (+ carry [B, 4, c]); ratio 128: C_a = C,
@@ -120,6 +134,18 @@ def csa_compress(C_a, C_b=None, Z_a=None, Z_b=None, prev_Cb=None, prev_Zb=None, 
     _check(_lib.csa_compress(_ptr(C_a), _ptr(C_b), _ptr(Z_a), _ptr(Z_b), _ptr(prev_Cb), _ptr(prev_Zb), B, L, c,
                              ratio, _dtype_code(C_a), _dtype_code(out), _ptr(out), _stream(stream)), "csa_compress")
     return out
+
+
+def csa_compress_index_keys(C_a, C_b, Z_a, Z_b, prev_Cb, prev_Zb, kI, *, pos0: int, k8=None, k_scale=None,
+                            hadamard: bool = True, stream=None):
+    """New index-key entries of raw rows C_a, C_b, Z_a, Z_b [B, L, 128] (+ carry [B, 4, 128]) into
+    rows pos0 .. pos0 + L/4 - 1 of the caches kI [B, Ncap, 128] bf16 and, if given, k8 [B, Ncap, 128]
+    uint8 e4m3 / k_scale [B, Ncap] fp32 (Hadamard-rotated before the quantisation when `hadamard`)."""
+    B, L, c = C_a.shape
+    _check(_lib.csa_compress_index_keys(_ptr(C_a), _ptr(C_b), _ptr(Z_a), _ptr(Z_b), _ptr(prev_Cb), _ptr(prev_Zb), B, L,
+                                        _dtype_code(C_a), int(bool(hadamard)), kI.shape[1], int(pos0), _ptr(kI),
+                                        _ptr(k8), _ptr(k_scale), _stream(stream)), "csa_compress_index_keys")
+    return kI
 
 
 def csa_quantize_mxfp4(x, codes=None, scales=None, stream=None, hadamard=False):
@@ -411,6 +437,7 @@ def csa_poll_status(stream=None) -> int:
     return int(_lib.csa_poll_status(_stream(stream)))
 
 
-def n_valid_for(q_pos: torch.Tensor, ratio: int, N: int) -> torch.Tensor:
-    """Visible complete entries per query, min(N, (pos + 1) // ratio), as int32 (host-side helper)."""
-    return torch.clamp((q_pos.to(torch.int64) + 1) // ratio, max=N).to(torch.int32)
+def csa_test_bounded_wait(complete: bool, limit_ns: int, stream=None) -> None:
+    """Enqueue the bounded-wait check: a kernel waits on a barrier that completes only if
+    `complete`; if the limit runs out it records CSA_ERR_TIMEOUT (read by csa_poll_status)."""
+    _check(_lib.csa_test_bounded_wait(int(bool(complete)), int(limit_ns), _stream(stream)), "csa_test_bounded_wait")

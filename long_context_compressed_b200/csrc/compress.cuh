@@ -76,6 +76,29 @@ __device__ __forceinline__ void store_ch(T* p, const float* v) {
 
 constexpr float kCompLog2e = 1.4426950408889634f;
 
+// One channel j of one CSA entry: softmax over positions r0 .. 2M-1 of the logits z[r][j]
+// (base-2 domain), weighted sum of the contents v[r][j].  Every CSA compressor kernel
+// takes its entries from here, so they agree bit for bit.
+template <int M, int CH>
+__device__ __forceinline__ float pool_channel(float (&z)[2 * M][CH], const float (&v)[2 * M][CH], int j, int r0) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < 2 * M; ++r)
+    if (r >= r0) {
+      z[r][j] *= kCompLog2e;
+      mx = fmaxf(mx, z[r][j]);
+    }
+  float den = 0.f, acc = 0.f;
+#pragma unroll
+  for (int r = 0; r < 2 * M; ++r) {
+    if (r < r0) continue;
+    const float e = ex2_approx(z[r][j] - mx);
+    den += e;
+    acc = fmaf(e, v[r][j], acc);
+  }
+  return acc / den;
+}
+
 // CSA (ratio m = 4): one thread per (sequence, entry, group of CH channels):
 // CH = 8 (16-byte loads) when there are enough entries to fill the GPU, CH = 2
 // otherwise (a decode step compresses a single block per sequence).  All 2m
@@ -121,24 +144,7 @@ __global__ void __launch_bounds__(256) compress_csa_kernel(const Tin* __restrict
     const int r0 = has_b ? 0 : M;
     float res[CH];
 #pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < 2 * M; ++r)
-        if (r >= r0) {
-          z[r][j] *= kCompLog2e;
-          mx = fmaxf(mx, z[r][j]);
-        }
-      float den = 0.f, acc = 0.f;
-#pragma unroll
-      for (int r = 0; r < 2 * M; ++r) {
-        if (r < r0) continue;
-        const float e = ex2_approx(z[r][j] - mx);
-        den += e;
-        acc = fmaf(e, v[r][j], acc);
-      }
-      res[j] = acc / den;
-    }
+    for (int j = 0; j < CH; ++j) res[j] = pool_channel<M, CH>(z, v, j, r0);
     store_ch<CH>(out + ((int64_t)b * n_entries + i) * c + ch, res);
   }
 }

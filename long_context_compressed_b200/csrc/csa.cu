@@ -18,7 +18,9 @@
 #include <vector>
 
 #include "../../include/csa.h"
+#include "append.cuh"
 #include "attn.cuh"
+#include "causal.cuh"
 #include "compress.cuh"
 #include "index.cuh"
 #include "kv8.cuh"
@@ -357,7 +359,23 @@ const char* csa_status_string(int status) {
   }
 }
 
-int csa_version(void) { return 100; }
+int csa_version(void) { return 101; }
+
+int csa_n_valid(const int64_t* q_pos, int64_t count, int ratio, int64_t lo, int64_t hi, int32_t* n_valid,
+                void* stream) {
+  if (count < 0 || ratio < 1 || lo < 0 || hi < lo || hi - lo > INT32_MAX) return CSA_ERR_INVALID;
+  if (count == 0) return CSA_OK;
+  if (!q_pos || !n_valid) return CSA_ERR_INVALID;
+  const unsigned blocks = (unsigned)std::min<int64_t>((count + 255) / 256, (int64_t)sm_count() * 4);
+  launch_k(csa::n_valid_kernel, blocks, 256, 0, as_stream(stream), q_pos, count, ratio, lo, hi, n_valid);
+  return launch_status();
+}
+
+int csa_test_bounded_wait(int complete, long long limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000LL) return CSA_ERR_INVALID;
+  launch_k(csa::bounded_wait_kernel, 1, 32, 0, as_stream(stream), complete ? 1 : 0, (uint64_t)limit_ns);
+  return launch_status();
+}
 
 int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* Z_b, const void* prev_Cb,
                  const void* prev_Zb, int B, int64_t L, int c, int ratio, int in_dtype, int out_dtype, void* out,
@@ -412,6 +430,34 @@ int csa_compress(const void* C_a, const void* C_b, const void* Z_a, const void* 
     else CSA_LAUNCH_HCA(float, float);
 #undef CSA_LAUNCH_HCA
   }
+  return launch_status();
+}
+
+int csa_compress_index_keys(const void* C_a, const void* C_b, const void* Z_a, const void* Z_b, const void* prev_Cb,
+                            const void* prev_Zb, int B, int64_t L, int in_dtype, int hadamard, int64_t n_cap,
+                            int64_t pos0, void* kI, uint8_t* k8, float* k_scale, void* stream) {
+  if (B < 0 || L < 0 || n_cap < 0 || pos0 < 0) return CSA_ERR_INVALID;
+  if (in_dtype != CSA_F32 && in_dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if ((prev_Cb == nullptr) != (prev_Zb == nullptr) || (k8 == nullptr) != (k_scale == nullptr)) return CSA_ERR_INVALID;
+  const int64_t n_entries = L / 4;
+  if (pos0 + n_entries > n_cap) return CSA_ERR_INVALID;
+  if (B == 0 || n_entries == 0) return CSA_OK;
+  if (!C_a || !C_b || !Z_a || !Z_b || !kI) return CSA_ERR_INVALID;
+  const void* ptrs[] = {C_a, C_b, Z_a, Z_b, prev_Cb, prev_Zb, kI, k8};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CSA_ERR_INVALID;
+  const int64_t warps = (int64_t)B * n_entries;
+  const unsigned blocks = (unsigned)std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8);
+  cudaStream_t st = as_stream(stream);
+  if (in_dtype == CSA_BF16)
+    launch_k(csa::compress_index_keys_kernel<__nv_bfloat16>, blocks, 256, 0, st, (const __nv_bfloat16*)C_a,
+             (const __nv_bfloat16*)C_b, (const __nv_bfloat16*)Z_a, (const __nv_bfloat16*)Z_b,
+             (const __nv_bfloat16*)prev_Cb, (const __nv_bfloat16*)prev_Zb, B, L, hadamard ? 1 : 0, n_cap, pos0,
+             (__nv_bfloat16*)kI, k8, k_scale);
+  else
+    launch_k(csa::compress_index_keys_kernel<float>, blocks, 256, 0, st, (const float*)C_a, (const float*)C_b,
+             (const float*)Z_a, (const float*)Z_b, (const float*)prev_Cb, (const float*)prev_Zb, B, L,
+             hadamard ? 1 : 0, n_cap, pos0, (__nv_bfloat16*)kI, k8, k_scale);
   return launch_status();
 }
 
@@ -622,8 +668,10 @@ size_t csa_topk_workspace_size(int B, int T, int64_t N, int k) {
   return (size_t)B * T * (size_t)csa::TopkWs::row_bytes(N);
 }
 
-int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t N, int k, int32_t* idx,
-             void* workspace, size_t ws_bytes, void* stream) {
+// Checks of csa_topk's arguments other than the workspace: CSA_OK, or the status to
+// return before anything is enqueued.
+static int topk_check(const float* scores, const int32_t* n_valid, int B, int T, int64_t N, int k,
+                      const int32_t* idx) {
   if (B < 0 || T < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
   if (N > (int64_t(1) << 20)) return CSA_ERR_UNSUPPORTED;
   if (B == 0 || T == 0) return CSA_OK;
@@ -631,6 +679,14 @@ int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t 
   const int64_t rows = (int64_t)B * T;
   if (rows > 65535 && topk_long_path(B, T, N)) return CSA_ERR_UNSUPPORTED;
   if (rows > (int64_t(1) << 31) - 1) return CSA_ERR_UNSUPPORTED;
+  return CSA_OK;
+}
+
+int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t N, int k, int32_t* idx,
+             void* workspace, size_t ws_bytes, void* stream) {
+  const int chk = topk_check(scores, n_valid, B, T, N, k, idx);
+  if (chk != CSA_OK || B == 0 || T == 0) return chk;
+  const int64_t rows = (int64_t)B * T;
   cudaStream_t st = as_stream(stream);
   if (!topk_long_path(B, T, N)) {
     const int smem = (int)std::max<int64_t>(4, std::min<int64_t>(N, csa::kRowSmemMax) * 4);
@@ -868,14 +924,19 @@ extern "C" {
 
 int csa_topk_noalloc(const float* scores, const int32_t* n_valid, int B, int T, int64_t N, int k, int32_t* idx,
                      void* stream) {
-  if (B < 0 || T < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
-  if (N > (int64_t(1) << 20)) return CSA_ERR_UNSUPPORTED;
+  // every argument is checked before the shared array is touched: a rejected call
+  // enqueues nothing
+  const int chk = topk_check(scores, n_valid, B, T, N, k, idx);
+  if (chk != CSA_OK || B == 0 || T == 0) return chk;
   const size_t need = csa_topk_workspace_size(B, T, N, k);
   if (need == 0) return csa_topk(scores, n_valid, B, T, N, k, idx, nullptr, 0, stream);   // needs no scratch
   if (need > (size_t)CSA_NOALLOC_SCRATCH_BYTES) return CSA_ERR_UNSUPPORTED;                 // beyond the array
   void* scratch = noalloc_scratch_ptr();
   if (scratch == nullptr) return CSA_ERR_CUDA;
-  // the array keeps the previous call's contents: clear the part this call relies on being zero
+  // A completed call leaves the part of the array it used zero-filled, and the
+  // chunked top-k needs exactly that at its start; a call cut short, or one that
+  // overlapped another on the GPU, would not leave it so.  Clearing the `need`
+  // bytes here makes every call independent of what the previous one left behind.
   if (cudaMemsetAsync(scratch, 0, need, as_stream(stream)) != cudaSuccess) return CSA_ERR_CUDA;
   return csa_topk(scores, n_valid, B, T, N, k, idx, scratch, need, stream);
 }

@@ -37,12 +37,6 @@ def shard_range(N: int, G: int, g: int) -> tuple[int, int]:
     return g * N // G, (g + 1) * N // G
 
 
-def local_n_valid(n_valid: torch.Tensor, lo: int, hi: int) -> torch.Tensor:
-    """Visible entries of the shard [lo, hi) for visible global counts n_valid (host helper,
-    computed once per position like n_valid itself)."""
-    return torch.clamp(n_valid.to(torch.int64) - lo, min=0, max=hi - lo).to(torch.int32)
-
-
 class TorchDistExchange:
     """all_gather over a torch.distributed process group (NCCL for CUDA tensors)."""
 
@@ -70,7 +64,7 @@ class Shard:
     swa_pos0: torch.Tensor    # [B] int64
     q_pos: torch.Tensor       # [B, 1] int64
     sink: torch.Tensor        # [H] fp32
-    n_valid: torch.Tensor     # [B, 1] int32, visible entries of this shard
+    n_valid: torch.Tensor     # [B, 1] int32, visible entries of this shard (csa_n_valid with [lo, hi))
     k8: torch.Tensor | None = None
     ks: torch.Tensor | None = None
 

@@ -20,3 +20,17 @@ def golden():
         with open(os.path.join(ROOT, "tests", "golden", name), encoding="utf-8") as f:
             return json.load(f)
     return load
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The fp32 parity checks' literal relative errors next to the 1e-5 * mag reading."""
+    try:
+        import tolerances
+    except ImportError:
+        return
+    if not tolerances.REPORTS:
+        return
+    tr = terminalreporter
+    tr.write_line("fp32 parity: max |gpu-ref|/mag (bound 1e-5) | max |gpu-ref|/|ref| where |ref| >= 1e-2 mag")
+    for what, c21, lit, n in tolerances.REPORTS:
+        tr.write_line(f"  {what}: {c21:.3g} | {lit:.3g} over {n} outputs")

@@ -43,7 +43,7 @@ def test_status_strings(lib):
     lib.csa_status_string.restype = ctypes.c_char_p
     assert lib.csa_status_string(0) == b"CSA_OK"
     assert b"INVALID" in lib.csa_status_string(1)
-    assert lib.csa_version() == 100
+    assert lib.csa_version() == 101
 
 
 def _vp(x=16):
@@ -176,3 +176,26 @@ def test_mxfp4_quantizer_host_checks(lib):
     assert f(p, 1, 4, 128, 0, p + 8, p, None) == 1      # codes not 16-byte aligned
     for cols in (32, 64, 128, 256):
         assert f(p, 1, 0, cols, 1, p, p, None) == 0
+
+
+def test_n_valid_and_bounded_wait_host_checks(lib):
+    """csa_n_valid: ratio >= 1, 0 <= lo <= hi, non-null pointers; csa_test_bounded_wait:
+    a limit between 1 us and 1 s.  Rejected calls launch nothing."""
+    f = lib.csa_n_valid
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p]
+    p = 16
+    assert f(p, 4, 0, 0, 10, p, None) == 1            # ratio 0
+    assert f(p, 4, 4, 5, 3, p, None) == 1             # hi < lo
+    assert f(p, 4, 4, -1, 3, p, None) == 1            # negative lo
+    assert f(p, -1, 4, 0, 3, p, None) == 1            # negative count
+    assert f(None, 4, 4, 0, 3, p, None) == 1          # null q_pos
+    assert f(p, 4, 4, 0, 3, None, None) == 1          # null output
+    assert f(p, 4, 4, 0, 1 << 32, p, None) == 1       # range beyond int32
+    assert f(None, 0, 4, 0, 3, None, None) == 0       # nothing to do
+    g = lib.csa_test_bounded_wait
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_int, ctypes.c_longlong, ctypes.c_void_p]
+    for bad in (0, 999, 10 ** 9 + 1, -5):
+        assert g(0, bad, None) == 1

@@ -1,7 +1,13 @@
 """End-to-end chains on the GPU (compress -> index -> top-k -> sparse_attn; compress ->
-hca_attn) against the same chain in the oracle.  Index sets are compared with the tie
-window of the measured score error; attention outputs are compared where the GPU
-chain selected the same set as the oracle chain."""
+hca_attn) against the same chain in the oracle.
+
+Index sets: the GPU chain must select exactly the oracle chain's set for every query.
+That is stricter than the fp32 rule alone, which only bounds each score's error by
+1e-5 * mag (mag: the oracle's sum of |terms|; differences inside that a-priori window
+would be allowed by check_topk_sets).  On these seeded inputs the gap between the k-th
+and (k+1)-th exact score is at least 0.036 (tiny) and 6e-4 (pro1m), above the fp32
+rounding the chains actually carry, so any difference at all is a failure.  Attention
+outputs are then compared element by element for every query."""
 import math
 
 import numpy as np
@@ -28,7 +34,7 @@ def test_tiny_chain_fp32(csa):
     cz = synth.draw_compressor(wl)
     comp = csa.csa_compress(*(cz[k].cuda() for k in ("C_a", "C_b", "Z_a", "Z_b")), ratio=4)      # [1, 1024, 128]
     comp_ref, cmag = oracle.compress_csa(*(cz[k].numpy() for k in ("C_a", "C_b", "Z_a", "Z_b")), with_mag=True)
-    check_f32(comp.cpu().numpy(), comp_ref, cmag, what="tiny compressor")
+    check_f32(comp.cpu().numpy(), comp_ref, cmag, what="tiny compressor", literal=True)
     ix = synth.draw_indexer(wl)
     q_pos = np.array([wl.q_pos], np.int64)
     nv = oracle.n_visible(q_pos, 4, wl.N)
@@ -36,23 +42,22 @@ def test_tiny_chain_fp32(csa):
     idx = csa.csa_topk(s, torch.from_numpy(nv).cuda(), wl.topk)
     comp_np = comp_ref.astype(np.float32)              # the oracle chain uses its own compressed cache
     s_ref, smag = oracle.index_scores(ix["qI"].numpy(), ix["w"].numpy(), comp_np, nv, with_mag=True)
-    E = float(np.max(np.abs(s.cpu().numpy()[np.isfinite(s_ref)] - s_ref[np.isfinite(s_ref)])))
     idx_np = idx.cpu().numpy()
     idx_ref = oracle.topk(s_ref.astype(np.float32), nv, wl.topk)
     for t in range(wl.T):
-        check_topk_sets(idx_np[0, t], s_ref[0, t, :nv[0, t]], wl.topk, E, what=f"tiny chain t={t}")
+        check_topk_sets(idx_np[0, t], s_ref[0, t, :nv[0, t]], wl.topk, 1e-5 * smag[0, t].max(),
+                        what=f"tiny chain t={t}")
+    assert np.array_equal(idx_np, idx_ref), "tiny chain: index sets differ from the oracle chain's"
     at = synth.draw_attention(wl)
     swa_pos0 = np.array([wl.swa_pos0], np.int64)
     scale = 1 / math.sqrt(wl.D)
     o = csa.sparse_attn(at["q"].cuda(), comp, at["swa_kv"].cuda(), torch.from_numpy(swa_pos0).cuda(),
                         torch.from_numpy(q_pos).cuda(), at["sink"].cuda(), idx, scale).cpu().numpy()
-    same = [t for t in range(wl.T) if np.array_equal(idx_np[0, t], idx_ref[0, t])]
-    assert len(same) >= wl.T - 1
     # attention on the GPU's own (compressed) cache vs the oracle's: both caches agree
     # within 1e-5 of their magnitude, which the fp32 attention tolerance absorbs
     ref, mag = oracle.sparse_attn(at["q"].numpy(), comp_np, at["swa_kv"].numpy(), swa_pos0, q_pos,
                                   at["sink"].numpy(), idx_ref, scale, with_mag=True)
-    check_f32(o[:, same], ref[:, same], np.maximum(mag, np.abs(ref))[:, same], what="tiny chain attention")
+    check_f32(o, ref, np.maximum(mag, np.abs(ref)), what="tiny chain attention")
 
 
 def test_pro1m_chain_fp8_rerank(csa):
@@ -73,20 +78,16 @@ def test_pro1m_chain_fp8_rerank(csa):
                                       with_mag=True)
     idx_np = idx.cpu().numpy()
     rec = check_topk_sets(idx_np[0, 0], s_ref[0, 0], wl.topk, 1e-5 * smag.max(), what="pro1m chain")
-    assert rec >= 0.99
+    idx_ref = oracle.topk(s_ref.astype(np.float32), nv, wl.topk)
+    assert np.array_equal(idx_np, idx_ref), f"pro1m chain: the reranked set differs from the oracle's (recall {rec})"
     at = synth.draw_attention(wl)
     swa_pos0 = np.array([wl.swa_pos0], np.int64)
     scale = 1 / math.sqrt(wl.D)
     o = csa.sparse_attn(at["q"].cuda(), at["kv"].cuda(), at["swa_kv"].cuda(), torch.from_numpy(swa_pos0).cuda(),
                         torch.from_numpy(q_pos).cuda(), at["sink"].cuda(), idx, scale).float().cpu().numpy()
-    idx_ref = oracle.topk(s_ref.astype(np.float32), nv, wl.topk)
     ref = oracle.sparse_attn(at["q"].float().numpy(), at["kv"].float().numpy(), at["swa_kv"].float().numpy(),
                              swa_pos0, q_pos, at["sink"].numpy(), idx_ref, scale)
-    if np.array_equal(idx_np, idx_ref):
-        check_attn_bf16(o, ref, what="pro1m chain attention")
-    else:
-        # near-tie swaps only: the swapped rows carry little weight
-        assert np.max(np.abs(o - ref)) < 0.1
+    check_attn_bf16(o, ref, what="pro1m chain attention")
 
 
 def test_hca_chain(csa):

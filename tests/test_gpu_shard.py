@@ -123,7 +123,7 @@ def test_sharded_decode_emulated(csa, G):
         shards.append(shard.Shard(rank=g, world=G, lo=lo, hi=hi, kI=ix["kI"][:, lo:hi].contiguous().cuda(),
                                   kv=at["kv"][:, lo:hi].contiguous().cuda(), swa=at["swa_kv"].cuda(),
                                   swa_pos0=swa_pos0.cuda(), q_pos=q_pos.cuda(), sink=at["sink"].cuda(),
-                                  n_valid=shard.local_n_valid(nv, lo, hi).cuda()))
+                                  n_valid=csa.csa_n_valid(q_pos.cuda(), 4, lo, hi)))
         kern.append(shard.GpuKernels(k, scale))
     qI, w, q = ix["qI"].cuda(), ix["w"].cuda(), at["q"].cuda()
     all_pairs = torch.stack([kern[g].local_topk(shards[g], qI, w) for g in range(G)])      # the first all-gather
@@ -131,14 +131,11 @@ def test_sharded_decode_emulated(csa, G):
     out = kern[0].combine(shards[0], gathered, tuple(q.shape))
     glob = kern[0].buf["glob"].cpu().numpy()
     s_ref, smag = oracle.index_scores(_np(ix["qI"]), ix["w"].numpy(), _np(ix["kI"]), nv.numpy(), with_mag=True)
-    for b in range(B):
-        rec = check_topk_sets(glob[b], s_ref[b, 0], k, 1e-5 * smag.max(), what=f"sharded G={G} b={b}")
-        assert rec >= 0.99
     idx_ref = oracle.topk(s_ref.astype(np.float32), nv.numpy(), k)
+    for b in range(B):
+        check_topk_sets(glob[b], s_ref[b, 0], k, 1e-5 * smag.max(), what=f"sharded G={G} b={b}")
+        # the exact rescoring makes the global selection the oracle's, index for index
+        assert np.array_equal(glob[b], idx_ref[b, 0]), f"sharded G={G} b={b}: set differs from the oracle's"
     ref = oracle.sparse_attn(_np(at["q"]), _np(at["kv"]), _np(at["swa_kv"]), swa_pos0.numpy(), q_pos.numpy(),
                              at["sink"].numpy(), idx_ref, scale)
-    same = all(sorted(x for x in glob[b] if x >= 0) == sorted(x for x in idx_ref[b, 0] if x >= 0) for b in range(B))
-    if same:
-        check_attn_bf16(_np(out), ref, what=f"sharded G={G}")
-    else:
-        assert np.max(np.abs(_np(out) - ref)) < 0.1        # near-tie swaps only
+    check_attn_bf16(_np(out), ref, what=f"sharded G={G}")

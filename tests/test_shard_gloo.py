@@ -82,7 +82,7 @@ def _worker(rank, world, port, k, out):
     lo, hi = shard.shard_range(N, world, rank)
     sh = shard.Shard(rank=rank, world=world, lo=lo, hi=hi, kI=x["kI"][:, lo:hi].contiguous(),
                      kv=x["kv"][:, lo:hi].contiguous(), swa=x["swa"], swa_pos0=x["swa_pos0"], q_pos=x["q_pos"],
-                     sink=x["sink"], n_valid=shard.local_n_valid(x["n_valid"], lo, hi))
+                     sink=x["sink"], n_valid=torch.clamp(x["n_valid"] - lo, 0, hi - lo).to(torch.int32))
     y = shard.decode_step(sh, OracleKernels(k, 1 / math.sqrt(x["q"].shape[-1])), shard.TorchDistExchange(),
                           x["q"], x["qI"], x["w"])
     out[rank] = y.numpy()
@@ -114,6 +114,3 @@ def test_shard_ranges_cover_the_entries():
             assert rs[0][0] == 0 and rs[-1][1] == N
             assert all(a[1] == b[0] for a, b in zip(rs[:-1], rs[1:]))
             assert max(h - l for l, h in rs) - min(h - l for l, h in rs) <= 1
-    nv = torch.tensor([[0], [5], [10], [25]], dtype=torch.int32)
-    assert shard.local_n_valid(nv, 10, 20).view(-1).tolist() == [0, 0, 0, 10]
-    assert shard.local_n_valid(nv, 0, 10).view(-1).tolist() == [0, 5, 10, 10]

@@ -8,11 +8,18 @@ bf16-stored outputs of fp32 arithmetic (the compressor): the stored value must
     the exact result, i.e. RN(ref - tol) <= gpu <= RN(ref + tol).
 bf16 attention: |gpu - ref| <= 2e-2 + 1e-2 * |ref|.
 Indices: bit-exact.
+
+Every fp32 check also reports the literal figure next to that reading: the largest
+|gpu - ref| / |ref| over the outputs with |ref| >= 1e-2 * mag (outputs that are not
+mostly cancellation).  check_f32(..., literal=True) asserts it is <= 1e-5 as well; the
+reports are printed at the end of the pytest run (tests/conftest.py).
 """
 import numpy as np
 
 F32_REL = 1e-5
 ATTN_ABS, ATTN_REL = 2e-2, 1e-2
+LITERAL_FLOOR = 1e-2
+REPORTS = []       # (what, max err/mag, max err/|ref| where |ref| >= 1e-2 mag, entries counted)
 
 
 def bf16_round(x):
@@ -22,8 +29,10 @@ def bf16_round(x):
     return np.ldexp(np.rint(m * 256.0) / 256.0, e)
 
 
-def check_f32(gpu, ref, mag, rel=F32_REL, what=""):
+def check_f32(gpu, ref, mag, rel=F32_REL, what="", literal=False):
     gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    mag = np.asarray(mag, np.float64)
     err = np.abs(gpu - ref)
     tol = rel * mag + 1e-30
     bad = ~(err <= tol)
@@ -31,6 +40,13 @@ def check_f32(gpu, ref, mag, rel=F32_REL, what=""):
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside 1e-5*mag; first at {tuple(i)}: "
                              f"gpu={gpu[tuple(i)]!r} ref={ref[tuple(i)]!r} mag={mag[tuple(i)]!r}")
+    sel = np.abs(ref) >= LITERAL_FLOOR * mag
+    lit = float(np.max(err[sel] / np.abs(ref[sel]))) if sel.any() else 0.0
+    c21 = float(np.max(err / (mag + 1e-300)))
+    REPORTS.append((what, c21, lit, int(sel.sum())))
+    if literal:
+        assert lit <= rel, f"{what}: literal relative error {lit:.3g} > {rel} where |ref| >= 1e-2 mag"
+    return lit
 
 
 def check_bf16_store(gpu, ref, mag, rel=F32_REL, what=""):
