@@ -41,6 +41,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # e4m3 index path: queries and keys are Walsh-Hadamard-rotated before quantisation
 # (the Indexer paragraph of the MXFP4 sparse-attention page); --no-hadamard turns it off.
 INDEX_ROTATION = True
+# partial RoPE of the attention ("DeepSeek-V4 混合注意力：从压缩记忆到百万上下文" §6; the MXFP4 page's
+# compress_rope_theta): q turned and the output turned back inside the attention kernel, new
+# compressed entries turned when the step appends them.  Not applied to mixed-precision KV8 rows.
+ROPE_THETA = 160000.0
 
 
 def oracle_quantizer():
@@ -232,6 +236,9 @@ class DecodeSet:
         # new index-key entries go straight into the caches' newest rows (bf16 keys and, on
         # the e4m3 path, their rotated e4m3 codes and scales): rows N - L/4 .. N - 1
         self.new_key_pos = N - cL // 4
+        self.theta = 0.0 if kv8 else ROPE_THETA
+        # RoPE positions of the step's new entries: latent entry i at 4 (N - L/4 + i)
+        self.new_entry_pos = torch.full((B,), 4 * (N - cL // 4), dtype=torch.int64, device=dev)
         self.scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         self.q8 = torch.empty((B, T, 64, 128), dtype=torch.uint8, device=dev)
         self.qs = torch.empty((B, T, 64), dtype=torch.float32, device=dev)
@@ -253,6 +260,7 @@ class DecodeSet:
             self.hsink = f32("hsink", (H,))
             self.inputs.update({"hq": g("hq", (B, T, H, D)), "hC": g("hC", (B, 128, D)), "hZ": g("hZ", (B, 128, D))})
             self.hcomp = torch.empty((B, 1, D), dtype=torch.bfloat16, device=dev)
+            self.hnew_pos = torch.full((B,), 128 * (Nh - 1), dtype=torch.int64, device=dev)
             self.hattn_ws = csa.attn_workspace(B, T, H, D, 128 + Nh, device=dev)
             self.hout = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
             self.hkv_store = self.hkv
@@ -344,15 +352,20 @@ class DecodeSet:
             with torch.cuda.stream(sa):
                 csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"], ratio=4,
                                  out=self.comp_kv)
+                if self.theta:
+                    csa.csa_rope(self.comp_kv, self.theta, stride=4, pos_base=self.new_entry_pos, out=self.comp_kv)
                 if self.kv8:
                     csa.quantize_kv8(self.comp_kv, entries=self.comp_kv8)
             if self.with_hca:
                 with torch.cuda.stream(sc):
                     csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=self.hcomp)
+                    if self.theta:
+                        csa.csa_rope(self.hcomp, self.theta, stride=128, pos_base=self.hnew_pos, out=self.hcomp)
                     if self.kv8:
                         csa.quantize_kv8(self.hcomp, entries=self.hcomp8)
                     csa.hca_attn(x["hq"], self.hkv_store, self.hswa, self.swa_pos0, self.q_pos, self.hsink,
-                                 1.0 / math.sqrt(wl.D), out=self.hout, workspace=self.hattn_ws)
+                                 1.0 / math.sqrt(wl.D), rope_theta=self.theta, out=self.hout,
+                                 workspace=self.hattn_ws)
 
         def append_index_keys():
             # the step's new index-key entries, compressed, rotated and quantised in one launch
@@ -399,7 +412,7 @@ class DecodeSet:
             mark("select")
         append_index_keys()
         csa.sparse_attn(x["q"], self.kv_store, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
-                        1.0 / math.sqrt(wl.D), out=self.out, workspace=self.attn_ws)
+                        1.0 / math.sqrt(wl.D), rope_theta=self.theta, out=self.out, workspace=self.attn_ws)
         mark("sparse_attn")
         for ss in side_streams:
             main.wait_stream(ss)
@@ -436,13 +449,15 @@ def capture_steps(sets, sides, copies: bool):
     own stream) and the device->host read of step j's outputs (another stream) overlap step
     j's compute; every step still moves its own inputs and outputs inside the graph."""
     import torch
-    main = torch.cuda.current_stream()
+    # the capturing stream itself is "main": the copy streams join the capture by waiting on
+    # it, so the copies are nodes of the graph and run on every replay
+    main = torch.cuda.Stream()
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
     for s in sets:
         s.run(sides)                                          # eager warm-up
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    with torch.cuda.graph(g, stream=main):
         if not copies:
             for s in sets:
                 s.run(sides)
@@ -570,6 +585,7 @@ def attn_alone_ms(sets, device, reps_per_set=8, replays=20):
         s = sets[i % len(sets)]
         x = s.inputs
         csa.sparse_attn(x["q"], s.kv_store, s.swa, s.swa_pos0, s.q_pos, s.sink, s.idx, 1.0 / math.sqrt(s.wl.D),
+                        rope_theta=s.theta,
                         out=s.out, workspace=s.attn_ws)
     for i in range(len(sets)):
         launch(i)

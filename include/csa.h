@@ -41,7 +41,7 @@ enum {
   CSA_ERR_TIMEOUT = 4      /* a kernel gave up a bounded wait (see csa_poll_status) */
 };
 
-enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2, CSA_BF16_KV8 = 3 };
+enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2, CSA_BF16_KV8 = 3, CSA_MXFP4 = 4 };
 
 #define CSA_INDEX_HEADS 64   /* index heads per query ([HA] §2 table, §4.2) */
 #define CSA_INDEX_DIM 128    /* dims per index head */
@@ -165,16 +165,34 @@ int csa_quantize_mxfp4(const void *x, int x_dtype, int64_t rows, int cols, int h
                        uint8_t *scales, void *stream);
 
 /*
+ * csa_quantize_mxfp4_sf128 -- csa_quantize_mxfp4 of rows of 128 values (cols = 128) with the
+ * E8M0 scales written in the layout the block-scaled tensor-core MMA reads, the operands of
+ * csa_index_scores with dtype CSA_MXFP4: the rows of each of `batches` batches (rows_per_batch
+ * each) in tiles of 128; tile j of batch b is one 512-byte atom at byte (b * ceil(rpb/128) + j) *
+ * 512, holding row i = 128 j + m0 + 32 m1 (m0 < 32, m1 < 4) at byte 16 m0 + 4 m1 + s for its
+ * scale s < 4 (dims 32 s .. 32 s + 31).  Bytes of rows past rows_per_batch are not written.
+ *   codes : [batches * rows_per_batch, 64] bytes as csa_quantize_mxfp4; sf : 16-byte aligned,
+ *   csa_mxfp4_sf128_bytes(batches, rows_per_batch) bytes.
+ */
+size_t csa_mxfp4_sf128_bytes(int64_t batches, int64_t rows_per_batch);
+int csa_quantize_mxfp4_sf128(const void *x, int x_dtype, int64_t batches, int64_t rows_per_batch, int hadamard,
+                             uint8_t *codes, uint8_t *sf, void *stream);
+
+/*
  * csa_index_scores -- Lightning Indexer ([HA] §4.2):
  *   scores[b,t,i] = sum_{h<64} w[b,t,h] * ReLU(<qI[b,t,h,:], kI[b,i,:]>)   for i < n_valid[b,t]
  *   scores[b,t,i] = -inf                                                   for n_valid[b,t] <= i < N
- * with dequantised values (code * scale) when dtype = CSA_E4M3.
+ * with dequantised values (code * scale) when dtype = CSA_E4M3, and (code * 2^(e - 127)) per
+ * block of 32 dims when dtype = CSA_MXFP4 (the FP4 index QK of [HA] §2 / §4.2).
  *   qI      : [B, T, 64, 128] dtype
  *   q_scale : [B, T, 64] fp32 (E4M3 only, else NULL)
  *   w       : [B, T, 64] fp32
  *   kI      : [B, N, 128] dtype   (keys shared by the 64 heads)
  *   k_scale : [B, N] fp32 (E4M3 only, else NULL)
  *   n_valid : [B, T] int32, 0 <= n_valid <= N (visible complete entries: csa_n_valid)
+ *   CSA_MXFP4: qI [B, T, 64, 64] and kI [B, N, 64] packed E2M1 codes (csa_quantize_mxfp4_sf128);
+ *              q_scale / k_scale are the byte arrays of their scales in the tensor-core layout
+ *              (rows_per_batch T * 64 and N), 16-byte aligned.
  *   scores  : [B, T, N] fp32
  *   select_ws : NULL, or (T == 1 only) a csa_topk_select workspace: the call then
  *               also accumulates each row's 4096-bin histogram of its valid scores
@@ -331,6 +349,41 @@ int sparse_attn(const void *q, const void *kv, const void *swa_kv, const int64_t
 int hca_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
              const int64_t *q_pos, const float *sink, int ratio, float scale, int B, int T, int H, int D, int64_t N,
              int dtype, void *out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Partial RoPE ([HA] §6: only the last 64 dims of each head carry the rotary position
+ * embedding; after the core attention the output's same dims get the inverse rotation,
+ * before the grouped output projection).  The pages give no pairing, base or position
+ * rule; this library's reading: the RoFormer rotation of the pairs (D-64+2i, D-64+2i+1),
+ * i < 32, by the angle pos * theta^(-2i/64) (theta > 1; the MXFP4 page's
+ * compress_rope_theta is 160000), a compressed entry i standing at position i * ratio,
+ * SWA rows and queries at their token positions.  Angles and their cos / sin are formed
+ * in fp64, the rotation runs in fp32.
+ *
+ * csa_rope -- rows x [B, R, D] (F32|BF16) -> out (the same pointer for in place): dims
+ *   D-64.. turned at position pos(b, r) = (pos_base ? pos_base[b] : 0) + r * stride, the
+ *   others copied; inverse != 0 turns the other way.  Use it when rows enter a cache:
+ *   compressed entries (pos_base NULL, stride = ratio) and raw SWA rows (pos_base =
+ *   swa_pos0, stride 1).  D even and >= 64.
+ */
+int csa_rope(const void *x, int dtype, int B, int64_t R, int D, const int64_t *pos_base, int64_t stride,
+             double theta, int inverse, void *out, void *stream);
+
+/*
+ * sparse_attn_rope / hca_attn_rope -- sparse_attn / hca_attn with the partial RoPE around
+ * the attention: q (as given, not rotated) is turned at q_pos inside the kernel, the memory
+ * and SWA rows are taken as stored (rotated when they entered the cache, csa_rope), and the
+ * output's last 64 dims are turned back at q_pos.  So out = inverse_rope(attn(rope(q),
+ * rows)) ([HA] §7 call chain).  rope_theta > 1; dtype CSA_BF16 or CSA_F32 (CSA_BF16_KV8:
+ * CSA_ERR_UNSUPPORTED); D >= 64.  Other arguments as sparse_attn / hca_attn.
+ */
+int sparse_attn_rope(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
+                     const int64_t *q_pos, const float *sink, const int32_t *idx, int k, float scale,
+                     double rope_theta, int B, int T, int H, int D, int64_t N, int dtype, void *out, void *workspace,
+                     size_t ws_bytes, void *stream);
+int hca_attn_rope(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,
+                  const int64_t *q_pos, const float *sink, int ratio, float scale, double rope_theta, int B, int T,
+                  int H, int D, int64_t N, int dtype, void *out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Sharded decode of one long sequence over G GPUs (the compressed entries split into

@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 CSA_OK, CSA_ERR_INVALID, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA, CSA_ERR_TIMEOUT = range(5)
-CSA_F32, CSA_BF16, CSA_E4M3, CSA_BF16_KV8 = 0, 1, 2, 3
+CSA_F32, CSA_BF16, CSA_E4M3, CSA_BF16_KV8, CSA_MXFP4 = 0, 1, 2, 3, 4
 KV8_DIMS, KV8_BYTES = 512, 608   # mixed-precision compressed entry: 448 e4m3 dims, 64 bf16 RoPE dims, 7 scales
 INDEX_HEADS, INDEX_DIM, SWA_WINDOW, MAX_TOPK = 64, 128, 128, 2048
 
@@ -38,6 +38,8 @@ _SIGS = {
     "csa_quantize_e4m3": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_quantize_e4m3_hadamard": ([_vp, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_quantize_mxfp4": ([_vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp], _i32),
+    "csa_mxfp4_sf128_bytes": ([_i64, _i64], _sz),
+    "csa_quantize_mxfp4_sf128": ([_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_kv8_entry_bytes": ([_i32], ctypes.c_longlong),
     "csa_quantize_kv8": ([_vp, _i64, _i32, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
@@ -53,6 +55,11 @@ _SIGS = {
                      _vp, _vp, _sz, _vp], _i32),
     "hca_attn": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                   _vp, _vp, _sz, _vp], _i32),
+    "csa_rope": ([_vp, _i32, _i32, _i64, _i32, _vp, _i64, ctypes.c_double, _i32, _vp, _vp], _i32),
+    "sparse_attn_rope": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _f32, ctypes.c_double, _i32, _i32, _i32,
+                          _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
+    "hca_attn_rope": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, ctypes.c_double, _i32, _i32, _i32, _i32,
+                       _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "sparse_attn_partial": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                              _vp, _vp, _vp, _sz, _vp], _i32),
     "csa_attn_combine": ([_vp, _i64, _vp, _i64, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
@@ -179,18 +186,35 @@ def csa_quantize_e4m3(x, codes=None, scale=None, stream=None, hadamard=False):
 
 
 def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=None, select_ws=None,
-                     stream=None):
+                     mxfp4: bool = False, stream=None):
     """Indexer scores.  qI [B, T, 64, 128] (fp32 | bf16 | uint8 e4m3 codes), w [B, T, 64] fp32,
     kI [B, N, 128] same dtype, n_valid [B, T] int32 -> scores [B, T, N] fp32.  With select_ws
-    (T == 1) the per-row score histogram for csa_topk_select is accumulated there."""
+    (T == 1) the per-row score histogram for csa_topk_select is accumulated there.
+    mxfp4=True: qI [B, T, 64, 64] / kI [B, N, 64] packed E2M1 codes and q_scale / k_scale their
+    tensor-core-layout scales (csa_quantize_mxfp4_sf128)."""
     B, T = qI.shape[0], qI.shape[1]
     N = kI.shape[1]
     if scores is None:
         scores = torch.empty((B, T, N), dtype=torch.float32, device=qI.device)
-    _check(_lib.csa_index_scores(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), _dtype_code(qI),
+    dt = CSA_MXFP4 if mxfp4 else _dtype_code(qI)
+    _check(_lib.csa_index_scores(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), dt,
                                  _ptr(n_valid), B, T, N, _ptr(scores), _ptr(select_ws), _stream(stream)),
            "csa_index_scores")
     return scores
+
+
+def csa_quantize_mxfp4_sf128(x, batches: int, *, hadamard: bool = True, codes=None, sf=None, stream=None):
+    """MXFP4 index operands with the scales in the tensor-core layout: x [..., 128] (fp32 | bf16) whose
+    rows form `batches` equal batches -> (codes uint8 [..., 64], sf uint8 [csa_mxfp4_sf128_bytes])."""
+    rows = x.numel() // 128
+    rpb = rows // batches
+    if codes is None:
+        codes = torch.empty(x.shape[:-1] + (64,), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.zeros(max(16, int(_lib.csa_mxfp4_sf128_bytes(batches, rpb))), dtype=torch.uint8, device=x.device)
+    _check(_lib.csa_quantize_mxfp4_sf128(_ptr(x), _dtype_code(x), batches, rpb, int(bool(hadamard)), _ptr(codes),
+                                         _ptr(sf), _stream(stream)), "csa_quantize_mxfp4_sf128")
+    return codes, sf
 
 
 def csa_select_workspace_size(B: int, N: int) -> int:
@@ -310,10 +334,11 @@ def _attn_dtype(q, kv) -> int:
     return _dtype_code(q)
 
 
-def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale: float, *, out=None, workspace=None,
-                stream=None):
+def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale: float, *, rope_theta: float = 0.0, out=None,
+                workspace=None, stream=None):
     """CSA core attention.  q [B,T,H,D], kv [B,N,D] (or [B,N,608] uint8 quantize_kv8 entries), swa_kv [B,W,D],
-    swa_pos0 [B] int64, q_pos [B,T] int64, sink [H] fp32, idx [B,T,k] int32 -> out [B,T,H,D]."""
+    swa_pos0 [B] int64, q_pos [B,T] int64, sink [H] fp32, idx [B,T,k] int32 -> out [B,T,H,D].
+    rope_theta > 0: sparse_attn_rope (q turned at q_pos inside, output turned back; rows as stored)."""
     B, T, H, D = q.shape
     N, W, k = kv.shape[1], swa_kv.shape[1], idx.shape[2]
     dt = _attn_dtype(q, kv)
@@ -321,15 +346,20 @@ def sparse_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, idx, scale: float, *, out=
         out = torch.empty_like(q)
     if workspace is None:
         workspace = attn_workspace(B, T, H, D, min(W, SWA_WINDOW) + k, dt, q.device)
-    _check(_lib.sparse_attn(_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), _ptr(idx),
-                            k, float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(workspace),
-                            workspace.numel() * workspace.element_size(), _stream(stream)), "sparse_attn")
+    args = (_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), _ptr(idx), k, float(scale))
+    tail = (B, T, H, D, N, dt, _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream))
+    if rope_theta:
+        _check(_lib.sparse_attn_rope(*args, float(rope_theta), *tail), "sparse_attn_rope")
+    else:
+        _check(_lib.sparse_attn(*args, *tail), "sparse_attn")
     return out
 
 
-def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int = 128, out=None, workspace=None,
-             stream=None):
-    """HCA core attention: dense over kv[b, :min(N, (pos+1)//ratio)] plus the SWA rows."""
+def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int = 128, rope_theta: float = 0.0,
+             out=None, workspace=None, stream=None):
+    """HCA core attention: dense over kv[b, :min(N, (pos+1)//ratio)] plus the SWA rows
+    (rope_theta > 0: hca_attn_rope)."""
     B, T, H, D = q.shape
     N, W = kv.shape[1], swa_kv.shape[1]
     dt = _attn_dtype(q, kv)
@@ -337,9 +367,24 @@ def hca_attn(q, kv, swa_kv, swa_pos0, q_pos, sink, scale: float, *, ratio: int =
         out = torch.empty_like(q)
     if workspace is None:
         workspace = attn_workspace(B, T, H, D, min(W, SWA_WINDOW) + N, dt, q.device)
-    _check(_lib.hca_attn(_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), ratio,
-                         float(scale), B, T, H, D, N, dt, _ptr(out), _ptr(workspace),
-                         workspace.numel() * workspace.element_size(), _stream(stream)), "hca_attn")
+    args = (_ptr(q), _ptr(kv), _ptr(swa_kv), _ptr(swa_pos0), W, _ptr(q_pos), _ptr(sink), ratio, float(scale))
+    tail = (B, T, H, D, N, dt, _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream))
+    if rope_theta:
+        _check(_lib.hca_attn_rope(*args, float(rope_theta), *tail), "hca_attn_rope")
+    else:
+        _check(_lib.hca_attn(*args, *tail), "hca_attn")
+    return out
+
+
+def csa_rope(x, theta: float, *, stride: int = 1, pos_base=None, inverse: bool = False, out=None, stream=None):
+    """Partial RoPE of rows x [B, R, D] (fp32 | bf16): dims D-64.. turned at position
+    pos_base[b] + r * stride (pos_base [B] int64 or None for 0) -> out (pass out=x for in place)."""
+    B, R, D = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(_lib.csa_rope(_ptr(x), _dtype_code(x), B, R, D, _ptr(pos_base), int(stride), float(theta), int(inverse),
+                         _ptr(out), _stream(stream)), "csa_rope")
     return out
 
 

@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include "kv8.cuh"
 #include "ptx.cuh"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -60,6 +61,7 @@ struct AttnParams {
   int sparse;             // 1: memory rows from idx (sparse_attn); 0: dense prefix (hca_attn)
   float* ml;              // [B, T, H, 2] or null: partial mode (no sink; write (m, l) per head)
   int64_t N;
+  double rope_theta;      // > 0: partial RoPE around the attention (rope.cuh); 0: none
 };
 
 struct RowList {
@@ -126,6 +128,21 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
     qv[j] = q[lane_id() + 32 * j];
     o[j] = 0.f;
   }
+  // partial RoPE: dims D-64.. of q turned at the query's position (pairs in adjacent lanes)
+  const int64_t qpos = p.q_pos[(int64_t)b * p.T + t];
+  const bool rope = p.rope_theta > 0.0;
+  float2 rcs[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) {
+    const int d = lane_id() + 32 * j;
+    rcs[j] = make_float2(1.f, 0.f);
+    if (rope && d >= p.D - kRopeDims) {
+      rcs[j] = rope_cs(qpos, (d - (p.D - kRopeDims)) >> 1, p.rope_theta, false);
+      const float other = __shfl_xor_sync(0xffffffffu, qv[j], 1);
+      const float2 y = (d & 1) ? rope_turn(other, qv[j], rcs[j]) : rope_turn(qv[j], other, rcs[j]);
+      qv[j] = (d & 1) ? y.y : y.x;                    // (d >= D - 64 holds for the whole warp)
+    }
+  }
   float m = p.sink[h], l = 1.f;
   const RowList rl = make_row_list(p, b, t);
   const int n = rl.n_swa + rl.n_mem;
@@ -154,7 +171,19 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
   float* out = static_cast<float*>(p.out) + (((int64_t)b * p.T + t) * p.H + h) * p.D;
   const float inv = 1.f / l;
 #pragma unroll
-  for (int j = 0; j < DPL; ++j) out[lane_id() + 32 * j] = o[j] * inv;
+  for (int j = 0; j < DPL; ++j) {
+    float v = o[j] * inv;
+    const int d = lane_id() + 32 * j;
+    if (rope) {                                        // inverse RoPE of the output at the query's position
+      const float other = __shfl_xor_sync(0xffffffffu, v, 1);
+      if (d >= p.D - kRopeDims) {
+        const float2 cs = make_float2(rcs[j].x, -rcs[j].y);
+        const float2 y = (d & 1) ? rope_turn(other, v, cs) : rope_turn(v, other, cs);
+        v = (d & 1) ? y.y : y.x;
+      }
+    }
+    out[d] = v;
+  }
 }
 
 // ------------------------------------------------------------------ tcgen05 bf16

@@ -20,6 +20,7 @@
 #include "../../include/csa.h"
 #include "append.cuh"
 #include "attn.cuh"
+#include "attn_t.cuh"
 #include "causal.cuh"
 #include "compress.cuh"
 #include "index.cuh"
@@ -102,18 +103,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map over [dim2][dim1][inner] with a 128-byte-swizzled box {box0, box1, 1}.
+// 3-D map over [dim2][dim1][inner] with a swizzled box {box0, box1, 1} (128-byte swizzle
+// unless another is given).
 bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t dim1,
-              uint64_t dim2, uint32_t box0, uint32_t box1) {
+              uint64_t dim2, uint32_t box0, uint32_t box1,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, dim1, dim2};
   cuuint64_t strides[2] = {inner * esize, inner * dim1 * esize};
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Row-tile map of a [dim2, rows, D] bf16 tensor seen as {64 elements, rows, D/64
@@ -239,6 +241,55 @@ int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse, int R
 // The split partials merge inside the kernel (cluster shared memory): no workspace.
 size_t attn_ws_bytes(int, int, int, int, int64_t, int) { return 0; }
 
+// bf16 rows: attn_t_kernel (rows as the MMA's M dimension, 64 heads per CTA, all of D).
+// Splits of a query's row list (units of 64 rows) form one cluster: as many as the SMs
+// allow for one wave, at most one per unit and at most kMaxSplits, and fewer while the
+// clusters would not all be resident at once.
+template <int D>
+int launch_attn_t(AttnParams p, int64_t max_rows, cudaStream_t st) {
+  using Cfg = csa::AttnTCfg<D>;
+  const int groups = (p.H + Cfg::HG - 1) / Cfg::HG;
+  const int64_t items = (int64_t)p.B * p.T * groups;
+  const int64_t units = std::max<int64_t>(1, (max_rows + Cfg::U - 1) / Cfg::U);
+  const int sms = sm_count();
+  int ns = 1;
+  if (items < sms) ns = (int)std::min<int64_t>(std::min<int64_t>(csa::kMaxSplits, units), std::max<int64_t>(1, sms / items));
+  auto kernel = csa::attn_t_kernel<D>;
+  while (ns > 1) {
+    const int fit = max_active_clusters(kernel, Cfg::kThreads, Cfg::kSmem, ns);
+    if (fit == 0 && ns > 8) {              // a non-portable size the device does not take
+      ns = 8;
+      continue;
+    }
+    if (fit >= items || fit == 0) break;   // 0: the query failed; keep the portable choice
+    --ns;
+  }
+  p.nsplit = ns;
+  CUtensorMap qmap, kvmap, swamap;
+  if (!make_map(&qmap, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)D, (uint64_t)p.H, (uint64_t)p.B * p.T,
+                64, 64))
+    return CSA_ERR_CUDA;
+  std::memset(&kvmap, 0, sizeof(kvmap));
+  std::memset(&swamap, 0, sizeof(swamap));
+  p.has_kvmap = p.N > 0 && make_row_tile_map(&kvmap, p.kv, (uint64_t)D, (uint64_t)p.N, (uint64_t)p.B, 8) ? 1 : 0;
+  p.has_swamap = p.W > 0 && make_row_tile_map(&swamap, p.swa, (uint64_t)D, (uint64_t)p.W, (uint64_t)p.B, 8) ? 1 : 0;
+  if (!set_smem(kernel, Cfg::kSmem)) return CSA_ERR_CUDA;
+  if (ns > 8 && cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return CSA_ERR_CUDA;
+  dim3 grid((unsigned)ns, (unsigned)groups, (unsigned)(p.B * p.T));
+  launch_kc(kernel, grid, Cfg::kThreads, Cfg::kSmem, st, ns, qmap, kvmap, swamap, p);
+  return launch_status();
+}
+
+int run_attn_t(const AttnParams& p, int64_t max_rows, cudaStream_t st) {
+  switch (p.D) {
+    case 128: return launch_attn_t<128>(p, max_rows, st);
+    case 256: return launch_attn_t<256>(p, max_rows, st);
+    case 512: return launch_attn_t<512>(p, max_rows, st);
+    default: return CSA_ERR_UNSUPPORTED;
+  }
+}
+
 int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_rows, cudaStream_t st) {
   if (p.B == 0 || p.T == 0) return CSA_OK;
   if (dtype == CSA_F32) {
@@ -254,6 +305,7 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     return launch_status();
   }
   const bool kv8 = dtype == CSA_BF16_KV8;
+  if (!kv8) return run_attn_t(p, max_rows, st);
   // rows per KV tile: 32 at D = 512 (four stages in shared memory), else 64.  Measured:
   // 64-row tiles at D = 512 (two stages) were slower for gathered, dense and KV8 rows.
   const int R = p.D < 512 ? 64 : 32;
@@ -509,8 +561,29 @@ int csa_quantize_e4m3_hadamard(const void* x, int x_dtype, int64_t rows, int col
   return launch_status();
 }
 
+static int quantize_mxfp4_impl(const void* x, int x_dtype, int64_t rows, int cols, int hadamard, uint8_t* codes,
+                               uint8_t* scales, int64_t rpb, void* stream);
+
 int csa_quantize_mxfp4(const void* x, int x_dtype, int64_t rows, int cols, int hadamard, uint8_t* codes,
                        uint8_t* scales, void* stream) {
+  return quantize_mxfp4_impl(x, x_dtype, rows, cols, hadamard, codes, scales, 0, stream);
+}
+
+size_t csa_mxfp4_sf128_bytes(int64_t batches, int64_t rows_per_batch) {
+  if (batches <= 0 || rows_per_batch <= 0) return 0;
+  return (size_t)batches * (size_t)((rows_per_batch + 127) / 128) * 512;
+}
+
+int csa_quantize_mxfp4_sf128(const void* x, int x_dtype, int64_t batches, int64_t rows_per_batch, int hadamard,
+                             uint8_t* codes, uint8_t* sf, void* stream) {
+  if (batches < 0 || rows_per_batch < 0) return CSA_ERR_INVALID;
+  if (batches == 0 || rows_per_batch == 0) return CSA_OK;
+  if (!sf || (reinterpret_cast<uintptr_t>(sf) & 15)) return CSA_ERR_INVALID;
+  return quantize_mxfp4_impl(x, x_dtype, batches * rows_per_batch, 128, hadamard, codes, sf, rows_per_batch, stream);
+}
+
+static int quantize_mxfp4_impl(const void* x, int x_dtype, int64_t rows, int cols, int hadamard, uint8_t* codes,
+                               uint8_t* scales, int64_t rpb, void* stream) {
   if (rows < 0 || !(cols == 32 || cols == 64 || cols == 128 || cols == 256)) return CSA_ERR_INVALID;
   if (x_dtype != CSA_F32 && x_dtype != CSA_BF16) return CSA_ERR_INVALID;
   if (rows == 0) return CSA_OK;
@@ -519,9 +592,9 @@ int csa_quantize_mxfp4(const void* x, int x_dtype, int64_t rows, int cols, int h
   cudaStream_t st = as_stream(stream);
 #define CSA_LAUNCH_MX(T, N, ROT)                                                                              \
   do {                                                                                                        \
-    const int64_t rpb = 8 * csa::HadamardCfg<N>::RPW;                                                         \
-    const unsigned blocks = (unsigned)std::min<int64_t>((rows + rpb - 1) / rpb, (int64_t)sm_count() * 2);     \
-    launch_k(csa::quantize_mxfp4_kernel<T, N, ROT>, blocks, 256, 0, st, (const T*)x, rows, codes, scales);     \
+    const int64_t rows_pb = 8 * csa::HadamardCfg<N>::RPW;                                                     \
+    const unsigned blocks = (unsigned)std::min<int64_t>((rows + rows_pb - 1) / rows_pb, (int64_t)sm_count() * 2); \
+    launch_k(csa::quantize_mxfp4_kernel<T, N, ROT>, blocks, 256, 0, st, (const T*)x, rows, codes, scales, rpb); \
   } while (0)
 #define CSA_LAUNCH_MX_ROT(T, N)        \
   do {                                 \
@@ -564,11 +637,12 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
                      int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* select_ws,
                      void* stream) {
   if (B < 0 || T < 0 || N < 0) return CSA_ERR_INVALID;
-  if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3) return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3 && dtype != CSA_MXFP4) return CSA_ERR_INVALID;
   if (B == 0 || T == 0 || N == 0) return CSA_OK;
   if (!qI || !w || !kI || !n_valid || !scores) return CSA_ERR_INVALID;
-  if (dtype == CSA_E4M3 && (!q_scale || !k_scale)) return CSA_ERR_INVALID;
+  if ((dtype == CSA_E4M3 || dtype == CSA_MXFP4) && (!q_scale || !k_scale)) return CSA_ERR_INVALID;
   if (!aligned16(qI) || !aligned16(kI)) return CSA_ERR_INVALID;
+  if (dtype == CSA_MXFP4 && (!aligned16(q_scale) || !aligned16(k_scale))) return CSA_ERR_INVALID;
   if (N >= (int64_t(1) << 31) || (int64_t)T * csa::kIdxHeads >= (int64_t(1) << 31) || B > 65535)
     return CSA_ERR_UNSUPPORTED;
   cudaStream_t st = as_stream(stream);
@@ -576,21 +650,25 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
     if (T > 65535) return CSA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)((N + 63) / 64), (unsigned)T, (unsigned)B);
     if (!set_smem(csa::index_simt_kernel<float, false>, csa::kIdxSimtSmem)) return CSA_ERR_CUDA;
-    launch_k(csa::index_simt_kernel<float, false>, grid, 256, csa::kIdxSimtSmem, st, 
+    launch_k(csa::index_simt_kernel<float, false>, grid, 256, csa::kIdxSimtSmem, st,
         (const float*)qI, w, (const float*)kI, n_valid, nullptr, 0, T, N, scores);
     return launch_status();
   }
-  const bool fp8 = dtype == CSA_E4M3;
+  const int mode = dtype == CSA_BF16 ? csa::kIdxBf16 : (dtype == CSA_E4M3 ? csa::kIdxE4m3 : csa::kIdxMxfp4);
+  const bool fp4 = mode == csa::kIdxMxfp4;
   IndexParams p;
   p.w = w;
-  p.q_scale = q_scale;
-  p.k_scale = k_scale;
+  p.q_scale = mode == csa::kIdxE4m3 ? q_scale : nullptr;
+  p.k_scale = mode == csa::kIdxE4m3 ? k_scale : nullptr;
+  p.q_sf = fp4 ? reinterpret_cast<const uint8_t*>(q_scale) : nullptr;
+  p.k_sf = fp4 ? reinterpret_cast<const uint8_t*>(k_scale) : nullptr;
   p.n_valid = n_valid;
   p.scores = scores;
   p.B = B;
   p.T = T;
   p.N = N;
-  p.TQ = T >= 4 ? 4 : (T >= 2 ? 2 : 1);
+  // queries per group: up to 4 (mxfp4: 2, so that a group's query scales are one atom)
+  p.TQ = (T >= 4 && !fp4) ? 4 : (T >= 2 ? 2 : 1);
   p.hist = nullptr;
   p.hist_stride = 0;
   if (select_ws != nullptr) {
@@ -598,34 +676,38 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
     p.hist = reinterpret_cast<int*>(select_ws);
     p.hist_stride = csa::SelectWs::row_bytes(N) / 4;
   }
-  const int key_bytes = fp8 ? csa::IndexCfg<true>::kKeyBytes : csa::IndexCfg<false>::kKeyBytes;
-  const int qrow = fp8 ? 128 : 256;
+  const int key_bytes = mode == csa::kIdxBf16 ? csa::IndexCfg<csa::kIdxBf16>::kKeyBytes
+                        : mode == csa::kIdxE4m3 ? csa::IndexCfg<csa::kIdxE4m3>::kKeyBytes
+                                                : csa::IndexCfg<csa::kIdxMxfp4>::kKeyBytes;
+  const int qrow = mode == csa::kIdxBf16 ? 256 : (mode == csa::kIdxE4m3 ? 128 : 64);
   const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
-  const int fixed = 1024 + q_bytes + csa::kIdxEpiWarps * p.TQ * csa::kIdxHeads * 4 + 8 * (4 + 2 * csa::kMaxAcc) +
-                    csa::kKsRing * 32 * csa::kIdxEpiWarps * 4 +
-                    (select_ws ? 2 * csa::kHistBinsIdx * 4 : 0);
-  p.stages = std::min(12, (kSmemLimit - fixed) / (key_bytes + 16));
+  const int fixed = 1024 + (q_bytes + 1023) / 1024 * 1024 + (fp4 ? 1024 : 0) +
+                    csa::kIdxEpiWarps * p.TQ * csa::kIdxHeads * 4 + 8 * (4 + 2 * csa::kMaxAcc) +
+                    csa::kKsRing * 32 * csa::kIdxEpiWarps * 4 + (select_ws ? 2 * csa::kHistBinsIdx * 4 : 0);
+  p.stages = std::min(fp4 ? 16 : 12, (kSmemLimit - fixed) / (key_bytes + 16));
   if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
   const int smem = fixed + p.stages * (key_bytes + 16);
   CUtensorMap kmap, qmap;
-  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int es = fp8 ? 1 : 2;
-  const uint32_t box0 = fp8 ? 128 : 64;
-  if (!make_map(&kmap, kI, dt, es, csa::kIdxDim, (uint64_t)N, (uint64_t)B, box0, csa::kIdxTileKeys) ||
-      !make_map(&qmap, qI, dt, es, csa::kIdxDim, (uint64_t)T * csa::kIdxHeads, (uint64_t)B, box0,
-                (uint32_t)(p.TQ * csa::kIdxHeads)))
+  const CUtensorMapDataType dt = mode == csa::kIdxBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const int es = mode == csa::kIdxBf16 ? 2 : 1;
+  const uint32_t box0 = mode == csa::kIdxBf16 ? 64 : (fp4 ? 64 : 128);        // elements of one swizzle row
+  const uint64_t inner = fp4 ? 64 : csa::kIdxDim;                             // elements per row in memory
+  const CUtensorMapSwizzle swz = fp4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_map(&kmap, kI, dt, es, inner, (uint64_t)N, (uint64_t)B, box0, csa::kIdxTileKeys, swz) ||
+      !make_map(&qmap, qI, dt, es, inner, (uint64_t)T * csa::kIdxHeads, (uint64_t)B, box0,
+                (uint32_t)(p.TQ * csa::kIdxHeads), swz))
     return CSA_ERR_CUDA;
   const int QG = (T + p.TQ - 1) / p.TQ;
   const int64_t items = (int64_t)B * QG * ((N + csa::kIdxTileKeys - 1) / csa::kIdxTileKeys);
   const unsigned grid = (unsigned)std::min<int64_t>(items, sm_count());
-  if (fp8) {
-    if (!set_smem(csa::index_tc_kernel<true>, smem)) return CSA_ERR_CUDA;
-    launch_k(csa::index_tc_kernel<true>, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
-  } else {
-    if (!set_smem(csa::index_tc_kernel<false>, smem)) return CSA_ERR_CUDA;
-    launch_k(csa::index_tc_kernel<false>, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
-  }
-  return launch_status();
+  auto go = [&](auto kernel) -> int {
+    if (!set_smem(kernel, smem)) return CSA_ERR_CUDA;
+    launch_k(kernel, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
+    return launch_status();
+  };
+  if (mode == csa::kIdxE4m3) return go(csa::index_tc_kernel<csa::kIdxE4m3>);
+  if (mode == csa::kIdxBf16) return go(csa::index_tc_kernel<csa::kIdxBf16>);
+  return go(csa::index_tc_kernel<csa::kIdxMxfp4>);
 }
 
 int csa_index_rerank(const void* qI, const float* w, const void* kI, int dtype, const int32_t* cand, int kc, int B,
@@ -783,33 +865,90 @@ size_t csa_attn_workspace_size(int B, int T, int H, int D, int64_t rows_per_quer
   return attn_ws_bytes(B, T, H, D, rows_per_query, dtype);
 }
 
-int sparse_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
-                const int64_t* q_pos, const float* sink, const int32_t* idx, int k, float scale, int B, int T,
-                int H, int D, int64_t N, int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+static int sparse_attn_impl(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                            const int64_t* q_pos, const float* sink, const int32_t* idx, int k, float scale,
+                            double theta, int B, int T, int H, int D, int64_t N, int dtype, void* out,
+                            void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_attn_common(q, kv, swa_kv, swa_pos0, W, q_pos, sink, scale, B, T, H, D, N, dtype, out);
-  if (rc != CSA_OK || B == 0 || T == 0) return rc;
+  if (rc != CSA_OK) return rc;
+  if (theta != 0.0 && (!(theta > 1.0) || D < csa::kRopeDims || dtype == CSA_BF16_KV8))
+    return !(theta > 1.0) ? CSA_ERR_INVALID : CSA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return rc;
   if (k < 0 || (k > 0 && !idx)) return CSA_ERR_INVALID;
   AttnParams p{};
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
-  p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale;
+  p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale; p.rope_theta = theta;
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = k; p.ratio = 1; p.N = N; p.nsplit = 1;
   // (KV8: the memory rows start at a tile boundary, at most 31 rows after the SWA rows)
   const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k + (dtype == CSA_BF16_KV8 ? 31 : 0);
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
 }
 
-int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
-             const int64_t* q_pos, const float* sink, int ratio, float scale, int B, int T, int H, int D, int64_t N,
-             int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+static int hca_attn_impl(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                         const int64_t* q_pos, const float* sink, int ratio, float scale, double theta, int B, int T,
+                         int H, int D, int64_t N, int dtype, void* out, void* workspace, size_t ws_bytes,
+                         void* stream) {
   int rc = check_attn_common(q, kv, swa_kv, swa_pos0, W, q_pos, sink, scale, B, T, H, D, N, dtype, out);
-  if (rc != CSA_OK || B == 0 || T == 0) return rc;
+  if (rc != CSA_OK) return rc;
+  if (theta != 0.0 && (!(theta > 1.0) || D < csa::kRopeDims || dtype == CSA_BF16_KV8))
+    return !(theta > 1.0) ? CSA_ERR_INVALID : CSA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return rc;
   if (ratio < 1) return CSA_ERR_INVALID;
   AttnParams p{};
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
-  p.idx = nullptr; p.sparse = 0; p.out = out; p.scale = scale;
+  p.idx = nullptr; p.sparse = 0; p.out = out; p.scale = scale; p.rope_theta = theta;
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = 0; p.ratio = ratio; p.N = N; p.nsplit = 1;
   const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + N + (dtype == CSA_BF16_KV8 ? 31 : 0);
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
+}
+
+int sparse_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                const int64_t* q_pos, const float* sink, const int32_t* idx, int k, float scale, int B, int T,
+                int H, int D, int64_t N, int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  return sparse_attn_impl(q, kv, swa_kv, swa_pos0, W, q_pos, sink, idx, k, scale, 0.0, B, T, H, D, N, dtype, out,
+                          workspace, ws_bytes, stream);
+}
+
+int sparse_attn_rope(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                     const int64_t* q_pos, const float* sink, const int32_t* idx, int k, float scale,
+                     double rope_theta, int B, int T, int H, int D, int64_t N, int dtype, void* out, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  if (!(rope_theta > 1.0)) return CSA_ERR_INVALID;
+  return sparse_attn_impl(q, kv, swa_kv, swa_pos0, W, q_pos, sink, idx, k, scale, rope_theta, B, T, H, D, N, dtype,
+                          out, workspace, ws_bytes, stream);
+}
+
+int hca_attn(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+             const int64_t* q_pos, const float* sink, int ratio, float scale, int B, int T, int H, int D, int64_t N,
+             int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  return hca_attn_impl(q, kv, swa_kv, swa_pos0, W, q_pos, sink, ratio, scale, 0.0, B, T, H, D, N, dtype, out,
+                       workspace, ws_bytes, stream);
+}
+
+int hca_attn_rope(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,
+                  const int64_t* q_pos, const float* sink, int ratio, float scale, double rope_theta, int B, int T,
+                  int H, int D, int64_t N, int dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!(rope_theta > 1.0)) return CSA_ERR_INVALID;
+  return hca_attn_impl(q, kv, swa_kv, swa_pos0, W, q_pos, sink, ratio, scale, rope_theta, B, T, H, D, N, dtype, out,
+                       workspace, ws_bytes, stream);
+}
+
+int csa_rope(const void* x, int dtype, int B, int64_t R, int D, const int64_t* pos_base, int64_t stride,
+             double theta, int inverse, void* out, void* stream) {
+  if (B < 0 || R < 0 || D < csa::kRopeDims || D % 2 != 0 || !(theta > 1.0)) return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_ERR_INVALID;
+  if (B == 0 || R == 0) return CSA_OK;
+  if (!x || !out) return CSA_ERR_INVALID;
+  const int64_t total = (int64_t)B * R * (csa::kRopeDims / 2);
+  const unsigned blocks = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
+  cudaStream_t st = as_stream(stream);
+  if (dtype == CSA_BF16)
+    launch_k(csa::rope_rows_kernel<__nv_bfloat16>, blocks, 256, 0, st, (const __nv_bfloat16*)x, (int64_t)B, R, D,
+             pos_base, stride, theta, inverse ? 1 : 0, (__nv_bfloat16*)out);
+  else
+    launch_k(csa::rope_rows_kernel<float>, blocks, 256, 0, st, (const float*)x, (int64_t)B, R, D, pos_base, stride,
+             theta, inverse ? 1 : 0, (float*)out);
+  return launch_status();
 }
 
 int sparse_attn_partial(const void* q, const void* kv, const void* swa_kv, const int64_t* swa_pos0, int W,

@@ -20,6 +20,12 @@
 //   e4m3 : kind::f8f6f4 with a per-key scale ks[b,i] and a per-(query, head)
 //          scale qs[b,t,h]; both are positive so they commute with ReLU:
 //          s = ks * sum_h (w * qs)_h * ReLU(<q8, k8>).
+//   mxfp4: kind::mxf4.block_scale (the FP4 index QK of §2 / §4.2): packed E2M1 codes
+//          (64 bytes per 128-dim row, 64-byte swizzle) with one E8M0 scale per 32 dims
+//          applied inside the MMA.  Scales are stored in the tensor-core layout
+//          (csa_quantize_mxfp4_sf128: 512 bytes per 128 rows), copied next to the codes
+//          into shared memory by a bulk copy and from there into tensor memory by
+//          tcgen05.cp; two MMAs of K = 64 per tile.
 //
 // index_simt_kernel: fp32 SIMT path (FMA), used for fp32 inputs and for the
 // exact rescoring of a candidate list.
@@ -54,6 +60,8 @@ struct IndexParams {
   const float* k_scale;  // [B, N] or null (bf16)
   const int32_t* n_valid;  // [B, T]
   float* scores;         // [B, T, N]
+  const uint8_t* q_sf;   // mxfp4: query scales [B][ceil(T*64/128)][512] (tensor-core layout)
+  const uint8_t* k_sf;   // mxfp4: key scales [B][ceil(N/128)][512]
   int* hist;             // per-row 4096-bin histogram of the score keys (T == 1), row stride hist_stride, or null
   int64_t hist_stride;   // ints between consecutive rows' histograms
   int B, T;
@@ -62,13 +70,23 @@ struct IndexParams {
   int stages;            // key pipeline depth
 };
 
-template <bool FP8>
+// Operand modes of index_tc_kernel.
+enum : int { kIdxBf16 = 0, kIdxE4m3 = 1, kIdxMxfp4 = 2 };
+
+template <int MODE>
 struct IndexCfg {
-  static constexpr int kKeyBytes = kIdxTileKeys * kIdxDim * (FP8 ? 1 : 2);  // one key tile
-  static constexpr int kQRowBytes = kIdxDim * (FP8 ? 1 : 2);               // one (t, h) row
-  static constexpr int kAtoms = FP8 ? 1 : 2;                                // 128-byte K atoms per row
-  static constexpr int kKInstr = FP8 ? 32 : 16;                             // K per MMA instruction
+  static constexpr bool FP4 = MODE == kIdxMxfp4;
+  static constexpr int kRowBytes = MODE == kIdxBf16 ? 256 : (MODE == kIdxE4m3 ? 128 : 64);   // one 128-dim row
+  static constexpr int kCodeBytes = kIdxTileKeys * kRowBytes;               // codes of one key tile
+  static constexpr int kSfBytes = FP4 ? 512 : 0;                            // scales of one key tile
+  static constexpr int kKeyBytes = kCodeBytes + (FP4 ? 1024 : 0);           // one pipeline stage (1 KiB aligned)
+  static constexpr int kQRowBytes = kRowBytes;                              // one (t, h) row
+  static constexpr int kAtomBytes = FP4 ? 64 : 128;                         // swizzle width
+  static constexpr int kAtoms = kRowBytes / kAtomBytes;                     // K atoms per row
+  static constexpr uint32_t kLayout = FP4 ? kLayoutSW64 : kLayoutSW128;
+  static constexpr int kKInstr = MODE == kIdxBf16 ? 16 : (MODE == kIdxE4m3 ? 32 : 64);   // K per MMA
   static constexpr int kKSteps = kIdxDim / kKInstr;
+  static constexpr int kKBytes = kKInstr * kRowBytes / kIdxDim;             // bytes of K per MMA
 };
 
 // Work item w -> (b, query group, key tile), ordered with the key tile fastest.
@@ -96,18 +114,22 @@ __device__ __forceinline__ void index_next(IndexItem& it, int QG, int64_t KT) {
   }
 }
 
-template <bool FP8>
+template <int MODE>
 __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap qmap,
                                                           const IndexParams p) {
-  using Cfg = IndexCfg<FP8>;
+  using Cfg = IndexCfg<MODE>;
+  constexpr bool FP8 = MODE == kIdxE4m3;            // per-row scales applied in the epilogue
+  constexpr bool FP4 = Cfg::FP4;                    // block scales applied by the MMA
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int TQ = p.TQ;
   const int NQ = TQ * kIdxHeads;                    // MMA N
   const int q_bytes = NQ * Cfg::kQRowBytes;
   uint8_t* q_smem = smem;
-  uint8_t* k_smem = smem + q_bytes;
+  // (mxfp4: the group's 512-byte scale atom after the codes, 1 KiB aligned)
+  uint8_t* qsf_smem = smem + ((q_bytes + 1023) & ~1023);
+  uint8_t* k_smem = qsf_smem + (FP4 ? 1024 : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(k_smem + (size_t)p.stages * Cfg::kKeyBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + p.stages;
@@ -126,12 +148,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
   const int64_t items = (int64_t)p.B * QG * KT;
   const int64_t w0 = items * blockIdx.x / gridDim.x;
   const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
-  const int NACC = (512 / NQ) < kMaxAcc ? (512 / NQ) : kMaxAcc;   // TMEM accumulators in flight (2 or 4)
+  // TMEM accumulators in flight (2 or 4); mxfp4 keeps 32 columns for the block scales
+  const int acc_fit = (FP4 ? 480 : 512) / NQ;
+  const int NACC = acc_fit >= kMaxAcc ? kMaxAcc : (acc_fit >= 2 ? 2 : 1);
   // epilogue sets: one per accumulator; with 2 accumulators each set has 8 warps, two
   // per TMEM lane quarter, splitting the group's queries
   const int nsets = NACC >= 4 ? 4 : 2;
   const int set_warps = kIdxEpiWarps / nsets;
-  const uint32_t tmem_cols = (uint32_t)(NACC * NQ) < 32 ? 32u : (uint32_t)(NACC * NQ);
+  const uint32_t tmem_cols = FP4 ? 512u : ((uint32_t)(NACC * NQ) < 32 ? 32u : (uint32_t)(NACC * NQ));
+  const uint32_t sfa_col0 = (uint32_t)(NACC * NQ);          // mxfp4: [acc] key scales, 4 columns each
+  const uint32_t sfb_col0 = sfa_col0 + 4 * kMaxAcc;        // mxfp4: [2] query scales, 4 columns each
 
   const int warp = warp_id();
   if (threadIdx.x == 0) {
@@ -177,9 +203,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
             if (!mbar_wait(qempty, qe_phase)) break;
             qe_phase ^= 1;
           }
-          mbar_arrive_expect_tx(qfull, (uint32_t)q_bytes);
+          mbar_arrive_expect_tx(qfull, (uint32_t)(q_bytes + Cfg::kSfBytes));
           for (int a = 0; a < Cfg::kAtoms; ++a)
             tma_load_3d(q_smem + (size_t)a * NQ * 128, &qmap, qfull, a * 64, it.qg * NQ, it.b);
+          if (FP4) {
+            const int64_t qtiles = ((int64_t)p.T * kIdxHeads + 127) / 128;
+            bulk_load(qsf_smem, p.q_sf + ((int64_t)it.b * qtiles + (int64_t)it.qg * NQ / 128) * 512, 512, qfull);
+          }
           prev_b = it.b;
           prev_qg = it.qg;
         }
@@ -187,11 +217,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
         const uint32_t ph = st_ph;
         if (++st_i == p.stages) { st_i = 0; st_ph ^= 1; }
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kKeyBytes);
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(Cfg::kCodeBytes + Cfg::kSfBytes));
         uint8_t* dst = k_smem + (size_t)s * Cfg::kKeyBytes;
         for (int a = 0; a < Cfg::kAtoms; ++a)
           tma_load_3d(dst + (size_t)a * kIdxTileKeys * 128, &kmap, &full[s], a * 64, (int)(it.kt * kIdxTileKeys),
                       it.b);
+        if (FP4) bulk_load(dst + Cfg::kCodeBytes, p.k_sf + ((int64_t)it.b * KT + it.kt) * 512, 512, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -200,6 +231,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       const uint32_t idesc = make_idesc(128, NQ, FP8 ? 0u : 1u, 0, 0);
       int prev_b = -1, prev_qg = -1;
       uint32_t qf_phase = 0;
+      uint32_t sfb_col = sfb_col0;                   // mxfp4: this group's query-scale columns
       int64_t cnt = 0;
       int st_i = 0, ac_i = 0;
       uint32_t st_ph = 0, ac_ph = 0;
@@ -211,6 +243,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
           qf_phase ^= 1;
           prev_b = it.b;
           prev_qg = it.qg;
+          if (FP4) {
+            // the group's query scales into tensor memory (alternating column sets, so the
+            // previous group's MMAs still read theirs)
+            sfb_col = sfb_col0 + (qf_phase ? 0u : 4u);
+            tc_fence_after();
+            tmem_cp_sf128(tmem_base + sfb_col, smem_desc(smem_u32(qsf_smem), 16, 128, 0));
+          }
         }
         const int s = st_i;
         const uint32_t ph = st_ph;
@@ -224,18 +263,31 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
         const uint32_t kbase = smem_u32(k_smem + (size_t)s * Cfg::kKeyBytes);
         const uint32_t qbase = smem_u32(q_smem);
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NQ);
+        if (FP4) {
+          // the tile's key scales into this accumulator's columns (freed with the accumulator)
+          tmem_cp_sf128(tmem_base + sfa_col0 + 4u * (uint32_t)acc,
+                        smem_desc(kbase + Cfg::kCodeBytes, 16, 128, 0));
+        }
 #pragma unroll
         for (int kk = 0; kk < Cfg::kKSteps; ++kk) {
-          const int byte_k = kk * Cfg::kKInstr * (FP8 ? 1 : 2);   // byte offset along K
-          const int atom = byte_k / 128;
-          const int inner = byte_k % 128;
+          const int byte_k = kk * Cfg::kKBytes;          // byte offset along K
+          const int atom = byte_k / Cfg::kAtomBytes;
+          const int inner = byte_k % Cfg::kAtomBytes;
+          const uint32_t sbo = 8 * Cfg::kAtomBytes;
           const uint64_t adesc =
-              smem_desc(kbase + atom * kIdxTileKeys * 128 + inner, 16, 1024, kLayoutSW128);
-          const uint64_t bdesc = smem_desc(qbase + atom * NQ * 128 + inner, 16, 1024, kLayoutSW128);
-          if (FP8)
+              smem_desc(kbase + atom * kIdxTileKeys * Cfg::kAtomBytes + inner, 16, sbo, Cfg::kLayout);
+          const uint64_t bdesc = smem_desc(qbase + atom * NQ * Cfg::kAtomBytes + inner, 16, sbo, Cfg::kLayout);
+          if constexpr (FP4) {
+            // scales of dims 64 kk .. 64 kk + 63: bytes 2 kk, 2 kk + 1 of each row's scale word
+            const uint32_t sf_byte = 2u * (uint32_t)kk;
+            mma_mxf4(d_tmem, adesc, bdesc, make_idesc_mxf4(128, NQ, sf_byte, sf_byte),
+                     tmem_base + sfa_col0 + 4u * (uint32_t)acc + (sf_byte << 30), tmem_base + sfb_col + (sf_byte << 30),
+                     kk > 0 ? 1u : 0u);
+          } else if (FP8) {
             mma_f8(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-          else
+          } else {
             mma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          }
         }
         mma_commit(&empty[s]);
         mma_commit(&tfull[acc]);

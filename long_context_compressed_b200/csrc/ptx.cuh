@@ -192,6 +192,26 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// Block-scaled FP4: D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T, kind::mxf4 with one E8M0
+// scale per 32 values of K (K = 64 per instruction).  sfa / sfb are the tensor-memory
+// addresses of the scales, the byte of the 32-bit scale word in bits 30..31.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy a 512-byte scale atom (32 rows of 16 bytes in shared memory, described by a
+// no-swizzle matrix descriptor) into 4 tensor-memory columns of lanes 0..31, replicated to
+// the other three lane quarters.
+__device__ __forceinline__ void tmem_cp_sf128(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive on the mbarrier once every tcgen05.mma issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -283,6 +303,14 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t ab_form
                                                   uint32_t b_mn_major) {
   return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor of the block-scaled kind::mxf4 MMA: E2M1 A and B (format 1),
+// E8M0 scales (bit 23), K-major operands, dense K = 64; the scale byte selectors of B
+// (bits 4..5) and A (bits 29..30); N >> 3 in bits 17..22, M >> 4 in bits 24..28.
+__host__ __device__ constexpr uint32_t make_idesc_mxf4(int M, int N, uint32_t a_sf_byte, uint32_t b_sf_byte) {
+  return ((b_sf_byte & 3u) << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(M >> 4) << 24) | ((a_sf_byte & 3u) << 29);
 }
 
 // 2^x with the SFU instruction (approximate, ~2 ulp; flushes subnormal results

@@ -180,10 +180,21 @@ __device__ __forceinline__ uint32_t e2m1_code(float v) {
   return (signbit(v) ? 8u : 0u) | m;
 }
 
+// Byte offset of E8M0 scale s (block of 32 values) of row i of a sequence's rows in the
+// tensor-core scale layout: rows in tiles of 128, each tile one 512-byte atom holding row
+// m = m0 + 32 m1 at byte 16 m0 + 4 m1 + s (the layout tcgen05.cp .32x128b.warpx4 moves into
+// tensor memory as 4 columns: row m's four scales in column m1 of lane m0).
+__device__ __forceinline__ int64_t sf128_offset(int64_t b, int64_t i, int s, int64_t tiles_per_batch) {
+  const int m = (int)(i & 127);
+  return (b * tiles_per_batch + (i >> 7)) * 512 + 16 * (m & 31) + 4 * (m >> 5) + s;
+}
+
+// rpb > 0: the scales go to the tensor-core layout above, rows counted per batch of rpb
+// rows (N = 128 only); rpb == 0: scales [rows, N/32].
 template <typename Tin, int N, bool ROT>
 __global__ void __launch_bounds__(256, 2) quantize_mxfp4_kernel(const Tin* __restrict__ x, int64_t rows,
                                                                 uint8_t* __restrict__ codes,
-                                                                uint8_t* __restrict__ scales) {
+                                                                uint8_t* __restrict__ scales, int64_t rpb) {
   using C = HadamardCfg<N>;
   constexpr int E = C::E, LPR = C::LPR, RPW = C::RPW;
   constexpr int VEC = 16 / (int)sizeof(Tin);
@@ -244,7 +255,12 @@ __global__ void __launch_bounds__(256, 2) quantize_mxfp4_kernel(const Tin* __res
       } else {
         *reinterpret_cast<uint2*>(cr) = make_uint2(packed[0], packed[1]);
       }
-      if (g % LPB == 0) scales[r * (N / 32) + g / LPB] = (uint8_t)(ex + 127);
+      if (g % LPB == 0) {
+        if (rpb > 0)
+          scales[sf128_offset(r / rpb, r % rpb, g / LPB, (rpb + 127) >> 7)] = (uint8_t)(ex + 127);
+        else
+          scales[r * (N / 32) + g / LPB] = (uint8_t)(ex + 127);
+      }
     }
 #pragma unroll
     for (int k = 0; k < NV; ++k) raw[k] = nxt[k];

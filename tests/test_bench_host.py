@@ -26,17 +26,19 @@ def test_traffic_records_follow_the_source_hash():
 
 
 def test_traffic_is_null_once_the_source_changes(tmp_path, monkeypatch):
-    """A copy of the tree whose kernel source differs by one byte gets no traffic figure."""
+    """A traffic record keyed on a source's hash is used while that source is unchanged, and
+    not once the source differs by one byte."""
     (tmp_path / "profiles").mkdir()
     (tmp_path / "long_context_compressed_b200" / "csrc").mkdir(parents=True)
-    prof = open(os.path.join(ROOT, "profiles", "attn_tc_kernel_decode_prefill_hca.md")).read()
     src = open(os.path.join(ROOT, "long_context_compressed_b200", "csrc", "attn.cuh"), "rb").read()
-    (tmp_path / "profiles" / "p.md").write_text(prof)
+    h = hashlib.sha256(src).hexdigest()[:16]
+    (tmp_path / "profiles" / "p.md").write_text(f"# x\ntraffic_bytes_per_launch: source_sha256_prefix={h} "
+                                                f"flash64k=123456 pro1m=789\n")
     (tmp_path / "long_context_compressed_b200" / "csrc" / "attn.cuh").write_bytes(src)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.profiled_traffic("p.md", "attn.cuh", "flash64k") is not None
+    assert bench.profiled_traffic("p.md", "attn.cuh", "flash64k") == 123456
+    assert bench.profiled_traffic("p.md", "attn.cuh", "pro1m") == 789
     (tmp_path / "long_context_compressed_b200" / "csrc" / "attn.cuh").write_bytes(src + b" ")
-    assert hashlib.sha256(src + b" ").hexdigest()[:16] not in prof
     assert bench.profiled_traffic("p.md", "attn.cuh", "flash64k") is None
 
 
