@@ -911,10 +911,12 @@ def run_stage(name, stage, index, steps, warmup, device, kv8=False):
                   (lambda: (csa.csa_score_histogram(st.scores, st.n_valid, st.select_ws),
                             csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws, idx=st.idx))),
         "attn": lambda: csa.sparse_attn(x["q"], st.kv_store, st.swa, st.swa_pos0, st.q_pos, st.sink, st.idx,
-                                        1.0 / math.sqrt(wl.D), out=st.out, workspace=st.attn_ws),
+                                        1.0 / math.sqrt(wl.D), rope_theta=st.theta, out=st.out,
+                                        workspace=st.attn_ws),
         "hcompress": lambda: csa.csa_compress(x["hC"], None, x["hZ"], None, ratio=128, out=st.hcomp),
         "hca": lambda: csa.hca_attn(x["hq"], st.hkv_store, st.hswa, st.swa_pos0, st.q_pos, st.hsink,
-                                    1.0 / math.sqrt(wl.D), out=st.hout, workspace=st.hattn_ws),
+                                    1.0 / math.sqrt(wl.D), rope_theta=st.theta, out=st.hout,
+                                    workspace=st.hattn_ws),
     }
     # inputs of the later stages come from the earlier ones
     order = ["quantize", "index", "select"] if index == "e4m3" else ["index", "select"]

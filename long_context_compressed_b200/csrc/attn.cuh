@@ -62,6 +62,7 @@ struct AttnParams {
   float* ml;              // [B, T, H, 2] or null: partial mode (no sink; write (m, l) per head)
   int64_t N;
   double rope_theta;      // > 0: partial RoPE around the attention (rope.cuh); 0: none
+  RopeFreqs rope_freq;    // theta^(-2i/64), i < 32 (when rope_theta > 0)
 };
 
 struct RowList {
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
     const int d = lane_id() + 32 * j;
     rcs[j] = make_float2(1.f, 0.f);
     if (rope && d >= p.D - kRopeDims) {
-      rcs[j] = rope_cs(qpos, (d - (p.D - kRopeDims)) >> 1, p.rope_theta, false);
+      rcs[j] = rope_cs(qpos, p.rope_freq.f[(d - (p.D - kRopeDims)) >> 1], false);
       const float other = __shfl_xor_sync(0xffffffffu, qv[j], 1);
       const float2 y = (d & 1) ? rope_turn(other, qv[j], rcs[j]) : rope_turn(qv[j], other, rcs[j]);
       qv[j] = (d & 1) ? y.y : y.x;                    // (d >= D - 64 holds for the whole warp)

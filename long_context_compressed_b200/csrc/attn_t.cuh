@@ -51,11 +51,13 @@ struct AttnTCfg {
   static constexpr int kStage = U * D * 2;         // bytes of one stage (8 groups)
   static constexpr int kQ = HG * D * 2;            // q tile: [atom][64 heads][128 B]
   static constexpr int kP = 128 * 128;             // P^T: 128 rows x 64 heads bf16
-  static constexpr int kMaxCtaRows = 2048;         // index values staged per CTA
-  static constexpr int kMisc = 512 + 4 * kMaxCtaRows;
+  static constexpr int kMaxCtaRows = 1024;         // index values staged per CTA
+  static constexpr int kOnes = 4096;               // 128 x 16 bf16 ones: the A operand of the row sums
+  static constexpr int kMisc = 512 + 4 * kMaxCtaRows + kOnes;
   static constexpr int kSmem = 1024 + NS * kStage + kQ + kP + kMisc;
   static constexpr int kMT = D / 128;              // O^T M-tiles
   static constexpr int kSCol = 256;                // S^T buffers at TMEM columns 256 and 320
+  static constexpr int kLCol = 384;                // per-head sums of P (every lane the same) at 384..447
   static constexpr int kThreads = 288;             // 4 softmax + 4 loader + 1 MMA warps
   static constexpr float kRescaleLog2 = 64.f;      // raise a head's reference max beyond this
   static_assert(D == 128 || D == 256 || D == 512, "D");
@@ -111,15 +113,17 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
   uint64_t* qfull = bars + 10;
   uint64_t* odone = bars + 11;
   uint64_t* qrot = bars + 13;     // RoPE dims of q turned (4 softmax warps)
+  uint64_t* recv_bar = bars + 18; // cluster merge: the peers' slices of this CTA's heads arrived
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 14);   // [2 stages][4 loader warps], 16 rows each
   int32_t* idx_s = reinterpret_cast<int32_t*>(bars + 64);      // [kMaxCtaRows]
+  uint8_t* ones_s = reinterpret_cast<uint8_t*>(idx_s + Cfg::kMaxCtaRows);   // [kOnes] bf16 1.0
 
-  __shared__ float red_max[4][HG], red_sum[4][HG];
+  __shared__ float red_max[4][HG];
   __shared__ float m_use[HG], fscale[HG];
   __shared__ float epi_g[HG];
   __shared__ int epi_have_o;
-  __shared__ float cl_m[HG], cl_l[HG];
+  __shared__ __align__(16) float2 cl_ml[HG];       // per head (m, l) of this CTA's rows
   __shared__ float cl_w[HG][kMaxSplits];
   __shared__ float2 rope_tab[kRopeDims / 2];   // cos, sin of the query position's angles
 
@@ -141,12 +145,16 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     mbar_init(qfull, 1);
     mbar_init(odone, 1);
     mbar_init(qrot, 4);
+    mbar_init(recv_bar, 1);
     fence_mbar_init();
   }
   if (warp == 8) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
+  for (int i = threadIdx.x; i < Cfg::kOnes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(ones_s)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async_smem();                        // generic-proxy writes -> tensor-core reads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -254,6 +262,9 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       for (int a = 0; a < Cfg::kAtoms; ++a) tma_load_3d(q_s + a * HG * 128, &qmap, qfull, a * 64, h0, qi);
       const uint32_t idesc_s = make_idesc(128, HG, 1, 0, 0);
       const uint32_t idesc_o = make_idesc(128, HG, 1, 1, 1);
+      const uint32_t idesc_l = make_idesc(128, HG, 1, 0, 1);
+      // all-ones A (128 x 16, no swizzle): ones . P^T = the per-head sum of P in every lane
+      const uint64_t ones_desc = smem_desc(smem_u32(ones_s), 128, 256, 0);
       const uint32_t qb = smem_u32(q_s);
       const uint32_t pb = smem_u32(p_s);
       bool ok = rope ? mbar_wait(qrot, 0) : mbar_wait(qfull, 0);
@@ -293,12 +304,13 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
         const uint32_t vb = smem_u32(kv_s + (pair ? 0 : sb) * Cfg::kStage);
         const uint32_t pt = pb + (pair ? 0 : sb * (Cfg::kP / 2));
         for (int kk = 0; kk < nk; ++kk) {
+          const uint64_t bd = smem_desc(pt + kk * 2048, 8192, 1024, kLayoutSW128);
 #pragma unroll
           for (int m = 0; m < Cfg::kMT; ++m) {
             const uint64_t ad = smem_desc(vb + 2 * m * 1024 + kk * 2 * Cfg::kGroup, 1024, Cfg::kGroup, kLayoutSW128);
-            const uint64_t bd = smem_desc(pt + kk * 2048, 8192, 1024, kLayoutSW128);
             mma_bf16(tmem + m * HG, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
           }
+          mma_bf16(tmem + Cfg::kLCol, ones_desc, bd, idesc_l, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&pdone[sb]);
         if (pair) {
@@ -318,13 +330,13 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     const bool owner = r < HG;                   // owner of head h0 + r's running statistics
     const bool head_ok = owner && h0 + r < p.H;
     const float zs = p.scale * kLog2e;
-    float m_run = -INFINITY, l_run = 0.f;        // owners: running max (log2 domain) and sum
+    float m_run = -INFINITY;                     // owners: running max (log2 domain)
     bool ok = true;
     if (rope) {
       // partial RoPE of q at the query's position: the last 64-dim atom of every head row,
       // turned in shared memory before the first S^T MMA reads it
       const int64_t qpos = p.q_pos[(int64_t)b * p.T + t];
-      if (r < kRopeDims / 2) rope_tab[r] = rope_cs(qpos, r, p.rope_theta, false);
+      if (r < kRopeDims / 2) rope_tab[r] = rope_cs(qpos, p.rope_freq.f[r], false);
       asm volatile("bar.sync 2, 128;" ::: "memory");
       if (nu > 0) {
         if (!mbar_wait(qfull, 0)) ok = false;
@@ -365,20 +377,24 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       tmem_ld32(s_addr, z);
       tmem_ld32(s_addr + 32, z + 32);
       tmem_wait_ld();
+      // per-head maximum over this warp's 32 rows (every lane gets each head's maximum)
+      float mine0 = -INFINITY, mine1 = -INFINITY;      // heads lane and lane + 32
 #pragma unroll
-      for (int h = 0; h < HG; ++h) z[h] = valid ? z[h] * zs : -INFINITY;
-      const float2 wm = warp_reduce64<true>(z);          // (S^T is read again below)
-      reinterpret_cast<float2*>(red_max[warp])[lane_id()] = wm;
+      for (int h = 0; h < HG; ++h) {
+        const float m = warp_max_f32(valid ? z[h] * zs : -INFINITY);
+        if (h == (int)lane_id()) mine0 = m;
+        if (h == (int)lane_id() + 32) mine1 = m;
+      }
+      red_max[warp][lane_id()] = mine0;
+      red_max[warp][lane_id() + 32] = mine1;
       asm volatile("bar.sync 2, 128;" ::: "memory");
       bool need = false;
       if (owner) {
-        if (j > 0) l_run += red_sum[0][r] + red_sum[1][r] + red_sum[2][r] + red_sum[3][r];
         const float tm = fmaxf(fmaxf(red_max[0][r], red_max[1][r]), fmaxf(red_max[2][r], red_max[3][r]));
         float f = 1.f;
         if (tm > m_run + Cfg::kRescaleLog2 || (m_run == -INFINITY && tm > -INFINITY)) {
           if (m_run != -INFINITY) {
             f = ex2_approx(m_run - tm);
-            l_run *= f;
             need = true;
           }
           m_run = tm;
@@ -391,14 +407,16 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       if (any && j > 0) {
         if (!mbar_wait(&pdone[(j - 1) & 1], ((j - 1) >> 1) & 1)) ok = false;
         tc_fence_after();
-        for (int m = 0; m < Cfg::kMT; ++m) {
+        // O^T's M-tiles and the sums of P (columns kLCol..) turn by the same per-head factors
+        for (int m = 0; m <= Cfg::kMT; ++m) {
+          const uint32_t col0 = m < Cfg::kMT ? (uint32_t)(m * HG) : (uint32_t)Cfg::kLCol;
           for (int c0 = 0; c0 < HG; c0 += 32) {
             float o[32];
-            tmem_ld32(tmem + lane_base + m * HG + c0, o);
+            tmem_ld32(tmem + lane_base + col0 + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] *= fscale[c0 + c];
-            tmem_st32(tmem + lane_base + m * HG + c0, o);
+            tmem_st32(tmem + lane_base + col0 + c0, o);
           }
         }
         tmem_wait_st();
@@ -430,16 +448,24 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
           *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = u;
         }
       }
-      const float2 ws = warp_reduce64<false>(z);
-      reinterpret_cast<float2*>(red_sum[warp])[lane_id()] = ws;
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&pfull[sb]);
     }
-    asm volatile("bar.sync 2, 128;" ::: "memory");  // the last unit's sums are in place
-    if (owner && ntiles > 0) l_run += red_sum[0][r] + red_sum[1][r] + red_sum[2][r] + red_sum[3][r];
     const bool have_o = ok && ntiles > 0 && mbar_wait(odone, 0);
+    // the per-head sum of P over every unit (the same in every TMEM lane): head r from lane r
+    float l_run = 0.f;
+    if (warp < 2) {
+      tc_fence_after();
+      float lv[32];
+      tmem_ld32(tmem + lane_base + Cfg::kLCol + (uint32_t)(warp * 32), lv);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (c == (int)lane_id()) l_run = lv[c];
+      if (!have_o) l_run = 0.f;
+    }
     if (owner) {
       float g = 1.f;
       if (p.nsplit == 1) {
@@ -457,8 +483,7 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
         }
       }
       epi_g[r] = g;
-      cl_m[r] = have_o ? m_run : -INFINITY;
-      cl_l[r] = have_o ? l_run : 0.f;
+      cl_ml[r] = have_o ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
     }
     if (r == 0) epi_have_o = have_o ? 1 : 0;
     tc_fence_before();
@@ -482,19 +507,28 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     for (int m = warp >> 2; m < Cfg::kMT; m += 2) {
       const int d = m * 128 + quarter * 32 + lane;
       if (p.nsplit == 1) __syncwarp();
+      float oall[HG];
+      if (have_o) {
+        tmem_ld32(tmem + lane_q + m * HG, oall);
+        tmem_ld32(tmem + lane_q + m * HG + 32, oall + 32);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int h = 0; h < HG; ++h) oall[h] = 0.f;
+      }
 #pragma unroll
       for (int hh = 0; hh < HG; hh += 32) {
-        float o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_q + m * HG + hh, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int h = 0; h < 32; ++h) o[h] = 0.f;
-        }
+        float* o = oall + hh;
         if (p.nsplit > 1) {
+          // [head][D] bf16: lanes d, d ^ 1 pair up, the even lane storing even heads and the
+          // odd lane odd heads as two adjacent values (one 4-byte store each)
+          const bool odd = (d & 1) != 0;
 #pragma unroll
-          for (int h = 0; h < 32; ++h) obuf[(hh + h) * D + d] = __float2bfloat16_rn(o[h]);
+          for (int h = 0; h < 32; h += 2) {
+            const float got = __shfl_xor_sync(0xffffffffu, odd ? o[h] : o[h + 1], 1);
+            const __nv_bfloat162 v = odd ? __floats2bfloat162_rn(got, o[h + 1]) : __floats2bfloat162_rn(o[h], got);
+            *reinterpret_cast<__nv_bfloat162*>(obuf + (hh + h + (odd ? 1 : 0)) * D + (d & ~1)) = v;
+          }
         } else {
 #pragma unroll
           for (int h = 0; h < 32; ++h) o[h] *= epi_g[hh + h];
@@ -530,20 +564,42 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
   if (p.nsplit > 1) {
     // ------------------------------------------------------------ merge of the splits
     // CTA `rank` finishes heads [rank*64/ns, (rank+1)*64/ns): M = max(sink, m_j),
-    // den = 2^(sink - M) + sum_j l_j 2^(m_j - M), out = sum_j 2^(m_j - M) O_j / den.
+    // den = 2^(sink - M) + sum_j l_j 2^(m_j - M), out = sum_j 2^(m_j - M) O_j / den.  Every
+    // CTA pushes each peer's heads of its raw O (bf16 [64][D] in stage 0) into that peer's
+    // receive area by one bulk shared-to-shared copy; the peer sums locally.
     const int ns = p.nsplit;
     const uint32_t rank = cluster_ctarank();
     const int hb = (int)rank * HG / ns, he = ((int)rank + 1) * HG / ns;
+    const int hpc = (HG + ns - 1) / ns;               // receive slot of one peer: hpc head rows
+    const __nv_bfloat16* part = reinterpret_cast<const __nv_bfloat16*>(kv_s);        // own raw O [64][D]
+    __nv_bfloat16* recv = reinterpret_cast<__nv_bfloat16*>(kv_s + Cfg::kStage);   // [ns][hpc][D]
+    float2* recv_ml = reinterpret_cast<float2*>(recv + (size_t)ns * hpc * D);       // [ns][64] (m, l)
     cluster_sync();                                   // every split's O and (m, l) are in place
-    for (int hl = threadIdx.x; hl < he - hb; hl += blockDim.x) {
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(recv_bar, (uint32_t)((ns - 1) * ((he - hb) * D * 2 + HG * 8)));
+      const uint32_t src = smem_u32(kv_s);
+      const uint32_t dst_o = smem_u32(recv + (size_t)rank * hpc * D);
+      const uint32_t dst_ml = smem_u32(recv_ml + rank * HG);
+      for (int j = 0; j < ns; ++j) {
+        if (j == (int)rank) continue;
+        const int hbj = j * HG / ns, hej = (j + 1) * HG / ns;
+        const uint32_t bar_j = cluster_map(smem_u32(recv_bar), (uint32_t)j);
+        bulk_s2cluster(cluster_map(dst_o, (uint32_t)j), src + (uint32_t)(hbj * D * 2), (uint32_t)((hej - hbj) * D * 2),
+                       bar_j);
+        bulk_s2cluster(cluster_map(dst_ml, (uint32_t)j), smem_u32(cl_ml), (uint32_t)(HG * 8), bar_j);
+      }
+    }
+    const bool arrived = mbar_wait(recv_bar, 0);
+    for (int hl = threadIdx.x; arrived && hl < he - hb; hl += blockDim.x) {
       const int hh = hb + hl;
       float mj[kMaxSplits], lj[kMaxSplits];
       const float sinkL = (h0 + hh >= p.H) ? 0.f : (p.ml ? -INFINITY : p.sink[h0 + hh] * kLog2e);
       float M = sinkL;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
-        mj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_m[hh]), (uint32_t)j)) : -INFINITY;
-        lj[j] = j < ns ? ld_cluster_f32(cluster_map(smem_u32(&cl_l[hh]), (uint32_t)j)) : 0.f;
+        const float2 v = j < ns ? (j == (int)rank ? cl_ml[hh] : recv_ml[j * HG + hh]) : make_float2(-INFINITY, 0.f);
+        mj[j] = v.x;
+        lj[j] = v.y;
         M = fmaxf(M, mj[j]);
       }
       const bool any = M > -INFINITY;
@@ -562,18 +618,9 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     }
     __syncthreads();
     constexpr int F = D / 8;                          // 16-byte slots (8 bf16) per head row
-    const uint32_t ob = smem_u32(kv_s);
-    uint32_t peer[kMaxSplits];
-#pragma unroll
-    for (int j = 0; j < kMaxSplits; ++j) peer[j] = cluster_map(ob, (uint32_t)(j < ns ? j : 0));
-    for (int it = threadIdx.x; it < (he - hb) * F; it += blockDim.x) {
-      const int hh = hb + it / F, f = it % F;
+    for (int it = threadIdx.x; arrived && it < (he - hb) * F; it += blockDim.x) {
+      const int hl = it / F, hh = hb + hl, f = it % F;
       if (h0 + hh >= p.H) continue;
-      const uint32_t off = (uint32_t)((hh * D + f * 8) * 2);
-      uint4 v[kMaxSplits];
-#pragma unroll
-      for (int j = 0; j < kMaxSplits; ++j)
-        if (j < ns) v[j] = ld_cluster_u4(peer[j] + off);
       float acc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -581,7 +628,9 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       for (int j = 0; j < kMaxSplits; ++j) {
         if (j < ns) {
           const float wj = cl_w[hh][j];
-          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
+          const __nv_bfloat16* srcj = j == (int)rank ? part + (size_t)hh * D : recv + ((size_t)j * hpc + hl) * D;
+          const uint4 v = *reinterpret_cast<const uint4*>(srcj + f * 8);
+          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 x = __bfloat1622float2(hv[e]);
@@ -605,7 +654,9 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       for (int e = 0; e < 4; ++e) ho[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hh) * D + f * 8) = u;
     }
-    cluster_sync();                                   // no CTA leaves while its shared memory is read
+    // no CTA leaves while a copy into or out of its shared memory, or a read of its (m, l),
+    // is still in flight
+    cluster_sync();
   }
 
   tc_fence_before();

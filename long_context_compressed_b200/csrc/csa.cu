@@ -878,6 +878,7 @@ static int sparse_attn_impl(const void* q, const void* kv, const void* swa_kv, c
   AttnParams p{};
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
   p.idx = idx; p.sparse = 1; p.out = out; p.scale = scale; p.rope_theta = theta;
+  if (theta > 0.0) p.rope_freq = csa::rope_freqs(theta);
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = k; p.ratio = 1; p.N = N; p.nsplit = 1;
   // (KV8: the memory rows start at a tile boundary, at most 31 rows after the SWA rows)
   const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + k + (dtype == CSA_BF16_KV8 ? 31 : 0);
@@ -897,6 +898,7 @@ static int hca_attn_impl(const void* q, const void* kv, const void* swa_kv, cons
   AttnParams p{};
   p.q = q; p.kv = kv; p.swa = swa_kv; p.swa_pos0 = swa_pos0; p.q_pos = q_pos; p.sink = sink;
   p.idx = nullptr; p.sparse = 0; p.out = out; p.scale = scale; p.rope_theta = theta;
+  if (theta > 0.0) p.rope_freq = csa::rope_freqs(theta);
   p.B = B; p.T = T; p.H = H; p.D = D; p.W = W; p.k = 0; p.ratio = ratio; p.N = N; p.nsplit = 1;
   const int64_t max_rows = (int64_t)std::min(W, CSA_SWA_WINDOW) + N + (dtype == CSA_BF16_KV8 ? 31 : 0);
   return run_attn(p, dtype, workspace, ws_bytes, max_rows, as_stream(stream));
@@ -944,10 +946,10 @@ int csa_rope(const void* x, int dtype, int B, int64_t R, int D, const int64_t* p
   cudaStream_t st = as_stream(stream);
   if (dtype == CSA_BF16)
     launch_k(csa::rope_rows_kernel<__nv_bfloat16>, blocks, 256, 0, st, (const __nv_bfloat16*)x, (int64_t)B, R, D,
-             pos_base, stride, theta, inverse ? 1 : 0, (__nv_bfloat16*)out);
+             pos_base, stride, csa::rope_freqs(theta), inverse ? 1 : 0, (__nv_bfloat16*)out);
   else
     launch_k(csa::rope_rows_kernel<float>, blocks, 256, 0, st, (const float*)x, (int64_t)B, R, D, pos_base, stride,
-             theta, inverse ? 1 : 0, (float*)out);
+             csa::rope_freqs(theta), inverse ? 1 : 0, (float*)out);
   return launch_status();
 }
 

@@ -373,6 +373,24 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to shared memory of
+// a CTA of the cluster (dst_cluster from cluster_map), completion counted in bytes on the
+// destination CTA's mbarrier (bar_cluster, from cluster_map).  A unicast shared-to-shared copy.
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                               uint32_t bar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+               : "memory");
+}
+
+// Maximum of x over the 32 lanes of the warp, returned to every lane.
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // ------------------------------------------------------------------ packed fp32 pairs
 __device__ __forceinline__ unsigned long long f32x2_pack(float lo, float hi) {
   unsigned long long r;

@@ -467,11 +467,26 @@ __global__ void __launch_bounds__(1024) topk_gather_select_kernel(const float* _
 constexpr int kSelMaxChunks = 1024;   // chunks per row (table in the row header)
 struct SelectWs {
   static constexpr int64_t kTableInt = kHistBins + 64;            // [chunk] -> (first slot, count)
-  static constexpr int64_t kHeaderInts = kTableInt + 2 * kSelMaxChunks;
+  static constexpr int64_t kFineInt = kTableInt + 2 * kSelMaxChunks;   // fine histogram of the candidates
+  static constexpr int64_t kHeaderInts = kFineInt + kHistBins;
   static __host__ __device__ int64_t row_bytes(int64_t N) {
     return ((kHeaderInts + 2 * N) * 4 + 15) / 16 * 16;
   }
 };
+// Fine histogram of the candidates' (rescored) keys: 4096 bins of 2^12 keys each, from two
+// threshold bins (2 * 2^20 keys) below the kk-th score's bin -- every candidate's score
+// lies in that bin or above, and a rescored score near it -- with keys outside the range
+// clamped to the end bins.  The last CTA finds the k-th key's fine bin with one scan of
+// this histogram and ranks that bin's few keys directly.
+__device__ __forceinline__ uint32_t fine_base(uint32_t bstar, bool rescore) {
+  const uint32_t below = rescore ? 2u : 0u;
+  return (bstar >= below ? bstar - below : 0u) << 20;
+}
+__device__ __forceinline__ int fine_bin(uint32_t key, uint32_t base) {
+  if (key < base) return 0;
+  const uint32_t f = (key - base) >> 12;
+  return f > (uint32_t)(kHistBins - 1) ? kHistBins - 1 : (int)f;
+}
 constexpr int kSelThreads = 256;
 constexpr int kSelPerThread = 4;     // scores each thread loads per pass of the chunk scan
 constexpr int kSelTcRows = 128;      // candidates rescored per tensor-core batch (bf16)
@@ -555,6 +570,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   unsigned long long* fin = reinterpret_cast<unsigned long long*>(ghist + kHistBins);
   int* slots = ghist + kHistBins + 2;
   int* ctab = reinterpret_cast<int*>(rws) + SelectWs::kTableInt;
+  int* gfine = reinterpret_cast<int*>(rws) + SelectWs::kFineInt;
   uint32_t* ckey = reinterpret_cast<uint32_t*>(rws + SelectWs::kHeaderInts * 4);
   int32_t* cidx = reinterpret_cast<int32_t*>(ckey + N);
   int32_t* out = idx + row * k;
@@ -565,6 +581,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
   }
   int nloc = 0;
+  uint32_t fbase = 0;                                // this row's fine-histogram base key
   // shared-memory map: [key tile 32 KB][q tile 16 KB] (tensor-core rescoring) then
   // lidx / lkey [chunk] and the fp32 rescoring scratch; the last CTA reuses all of it
   uint8_t* tile_s = sel_smem;
@@ -626,6 +643,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, kk, res, scratch);
     __syncthreads();
     const uint32_t bstar = (uint32_t)res[0];
+    fbase = fine_base(bstar, RESCORE);
     // ---- this chunk's candidates, compacted in index order (one warp scans the 32
     // (pass, warp) counts)
     int lbase = 0;
@@ -790,7 +808,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     if (warp_id() == 0) tmem_dealloc(tmem_holder, 64);
   }
   if (!active) return;
-  // ---- append to the row's candidate list
+  // ---- append to the row's candidate list, and the candidates' keys to the fine histogram
   if (threadIdx.x == 0) {
     const int g = nloc > 0 ? atomicAdd(slots, nloc) : 0;
     gslot = g;
@@ -798,8 +816,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   }
   __syncthreads();
   for (int c = threadIdx.x; c < nloc; c += blockDim.x) {
-    ckey[gslot + c] = lkey[c];
+    const uint32_t key = lkey[c];
+    ckey[gslot + c] = key;
     cidx[gslot + c] = lidx[c];
+    atomicAdd(&gfine[fine_bin(key, fbase)], 1);
   }
   __syncthreads();
   const int nchunks = (int)((nv + chunk - 1) / chunk);
@@ -893,11 +913,67 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     __syncthreads();
     kmin = kext[0];
     const uint32_t span = kext[1] - kmin;
-    // radix select on u = key - kmin, 12-bit digits from the highest bit of the span down
-    // (the candidates share their leading key bits, so the digits spread over the bins)
     uint32_t prefix = 0, pmask = 0;
     int remaining = k;
-    for (int hi = span ? 32 - __clz(span) : 0; hi > 0;) {
+    // The k-th key's bin of the fine histogram the chunks accumulated; if it is an inner
+    // bin holding at most kSelPivot keys, rank those keys directly and skip the radix.
+    bool located = false;
+    {
+      const int4* g4 = reinterpret_cast<const int4*>(gfine);
+#pragma unroll
+      for (int u = 0; u < kHistBins / 4 / kSelThreads; ++u) {
+        const int4 v = __ldcg(g4 + threadIdx.x + u * kSelThreads);
+        const int h = 4 * (threadIdx.x + u * kSelThreads);
+        histk[skew(h)] = v.x;
+        histk[skew(h + 1)] = v.y;
+        histk[skew(h + 2)] = v.z;
+        histk[skew(h + 3)] = v.w;
+      }
+      __syncthreads();
+      find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, k, res, scratch);
+      __syncthreads();
+      const int fstar = res[0], above = res[1];
+      const int nb = histk[skew(fstar)];
+      if (fstar > 0 && fstar < kHistBins - 1 && nb <= kSelPivot) {
+        uint32_t* piv = reinterpret_cast<uint32_t*>(tpre + kSelMaxChunks);   // [kSelPivot]
+        if (threadIdx.x == 0) pcount = 0;
+        __syncthreads();
+        const uint32_t below = (1u << lane_id()) - 1;
+        for (int i0 = 0; i0 < nc; i0 += kSelThreads) {       // one slot claim per warp
+          const int i = i0 + threadIdx.x;
+          const uint32_t key = i < nc ? okey[i] : 0u;
+          const bool m = i < nc && fine_bin(key, fbase) == fstar;
+          const uint32_t bal = __ballot_sync(0xffffffffu, m);
+          int base = 0;
+          if (lane_id() == 0 && bal) base = atomicAdd(&pcount, __popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (m) piv[base + __popc(bal & below)] = key;
+        }
+        __syncthreads();
+        const int want = k - above;                          // keys of this bin to take
+        if ((int)threadIdx.x < nb) {
+          const uint32_t v = piv[threadIdx.x];
+          int gt = 0, ge = 0;
+          for (int j = 0; j < nb; ++j) {
+            gt += piv[j] > v;
+            ge += piv[j] >= v;
+          }
+          if (gt < want && want <= ge) {                     // every key equal to K* writes the same
+            res[0] = (int)(v - kmin);
+            res[1] = gt;
+          }
+        }
+        __syncthreads();
+        prefix = (uint32_t)res[0];
+        pmask = 0xffffffffu;
+        remaining = want - res[1];
+        located = true;
+      }
+      __syncthreads();
+    }
+    // otherwise: radix select on u = key - kmin, 12-bit digits from the highest bit of the
+    // span down (the candidates share their leading key bits, so the digits spread over the bins)
+    for (int hi = (located || !span) ? 0 : 32 - __clz(span); hi > 0;) {
       const int lo = hi > kHistBits ? hi - kHistBits : 0;
       const uint32_t dmask = (1u << (hi - lo)) - 1;
       for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) histk[j] = 0;
@@ -1145,7 +1221,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     __syncthreads();
   }
   // leave the row's header zeroed for the next call
-  for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
+  for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) {
+    ghist[j] = 0;
+    gfine[j] = 0;
+  }
   if (threadIdx.x == 0) {
     *fin = 0ull;
     *slots = 0;

@@ -73,14 +73,19 @@ def test_compress_index_keys(csa, name, B, L, dtype, carry, hadamard, ncap, pos0
     unique = ~amb.any(-1)
     assert np.array_equal(c_gpu[unique], c_ref[unique]) and np.array_equal(s_gpu[unique], s_ref[unique])
     if (~unique).any():
+        # each ambiguous stored key may sit anywhere in its admissible bf16 range; the
+        # rotation spreads those ranges over the row (|H| = 1 / sqrt(128) per entry)
+        width = (hi - lo)[~unique]
+        slack = (width.sum(-1, keepdims=True) / np.sqrt(128.0)) if hadamard else width
         dq_gpu = oracle.e4m3_decode(c_gpu[~unique]) * s_gpu[~unique][:, None]
         dq_ref = oracle.e4m3_decode(c_ref[~unique]) * s_ref[~unique][:, None]
         smax = np.maximum(s_gpu[~unique], s_ref[~unique])[:, None]
-        step = 0.125 * np.maximum(np.abs(dq_ref), np.abs(dq_gpu)) + 2.0 ** -9 * smax * 1.001
-        bad = np.abs(dq_gpu - dq_ref) > step
-        assert not bad.any(), (f"{bad.sum()} codes beyond one e4m3 step of the oracle's, e.g. gpu "
-                               f"{dq_gpu[bad][:4]} ref {dq_ref[bad][:4]} scales {s_gpu[~unique][:2]} {s_ref[~unique][:2]}")
-        assert np.all(np.abs(s_gpu[~unique] / s_ref[~unique] - 1) <= 1e-3)
+        step = 0.125 * (np.maximum(np.abs(dq_ref), np.abs(dq_gpu)) + slack) + 2.0 ** -9 * smax * 1.001
+        bad = np.abs(dq_gpu - dq_ref) > step + slack
+        assert not bad.any(), (f"{bad.sum()} codes beyond the admissible keys' reach, e.g. gpu "
+                               f"{dq_gpu[bad][:4]} ref {dq_ref[bad][:4]}")
+        ds = np.abs(s_gpu[~unique] - s_ref[~unique])
+        assert np.all(ds <= slack.max(-1) / 448.0 * 1.01 + 1e-6 * s_ref[~unique])
 
 
 def test_compress_index_keys_bf16_only(csa):

@@ -6,8 +6,9 @@ index QK path runs in FP4; format reading c25, OCP MXFP4) on the block-scaled te
 - csa_index_scores with dtype CSA_MXFP4 against oracle.index_scores on the oracle's own
   dequantised operands (code * 2^(e - 127) per block of 32), fp32 rule 1e-5 * mag, at the
   decode shapes, ragged key counts and several queries per sequence;
-- the decode top-k fed by the FP4 scores with the exact bf16 rescoring of the 2k-bin
-  candidates: recall against the oracle's exact top-k (>= 0.99)."""
+- the decode top-k fed by the FP4 scores with the exact bf16 rescoring of the candidates
+  of the 4k-th score's bin: recall against the oracle's exact top-k (>= 0.99).  FP4 scores
+  are coarser than e4m3 ones, so the candidate list is twice the e4m3 path's."""
 import numpy as np
 import pytest
 import torch
@@ -75,7 +76,7 @@ def test_fp4_scores_match_oracle_on_dequantised_operands(csa, B, T, N):
 
 @pytest.mark.parametrize("name", ["flash64k", "pro1m"])
 def test_fp4_decode_topk_recall_after_rescoring(csa, name):
-    """FP4 scores with the score histogram -> the candidates of the 2k-th score's bin,
+    """FP4 scores with the score histogram -> the candidates of the 4k-th score's bin,
     rescored exactly on the bf16 operands -> top-k; recall of the oracle's exact top-k."""
     wl = synth.WORKLOADS[name]
     ix = synth.draw_indexer(wl)
@@ -87,9 +88,9 @@ def test_fp4_decode_topk_recall_after_rescoring(csa, name):
     k4, ksf = csa.csa_quantize_mxfp4_sf128(kI, wl.B)
     ws = csa.select_workspace(wl.B, wl.N)
     s4 = csa.csa_index_scores(q4, w, k4, g_nv, q_scale=qsf, k_scale=ksf, select_ws=ws, mxfp4=True)
-    got = csa.csa_topk_select(s4, g_nv, wl.topk, ws, kc=2 * wl.topk, qI=qI, w=w, kI=kI).cpu().numpy()
+    got = csa.csa_topk_select(s4, g_nv, wl.topk, ws, kc=4 * wl.topk, qI=qI, w=w, kI=kI).cpu().numpy()
     ref = oracle.index_scores(ix["qI"].float().numpy(), ix["w"].numpy(), ix["kI"].float().numpy(), nv)
     idx_ref = oracle.topk(ref.astype(np.float32), nv, wl.topk)
     recall = min(len(np.intersect1d(got[b, 0], idx_ref[b, 0])) / wl.topk for b in range(wl.B))
-    print(f"{name} FP4 + 2k rescoring recall {recall:.4f}")
+    print(f"{name} FP4 + 4k rescoring recall {recall:.4f}")
     assert recall >= 0.99
