@@ -215,6 +215,9 @@ class DecodeSet:
         self.kI = g("kI", (B, N, 128))
         if index == "e4m3":
             self.k8, self.ks = csa.csa_quantize_e4m3(self.kI, hadamard=INDEX_ROTATION)
+        if index == "mxfp4":
+            # packed E2M1 codes of the rotated keys, scales in the tensor-core layout
+            self.k4, self.ksf = csa.csa_quantize_mxfp4_sf128(self.kI, B)
         self.sink = f32("sink", (H,))
         self.q_pos = torch.full((B, T), wl.q_pos0, dtype=torch.int64, device=dev)
         self.swa_pos0 = torch.full((B,), wl.swa_pos0, dtype=torch.int64, device=dev)
@@ -242,6 +245,9 @@ class DecodeSet:
         self.scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         self.q8 = torch.empty((B, T, 64, 128), dtype=torch.uint8, device=dev)
         self.qs = torch.empty((B, T, 64), dtype=torch.float32, device=dev)
+        if index == "mxfp4":
+            self.q4 = torch.empty((B, T, 64, 64), dtype=torch.uint8, device=dev)
+            self.qsf = torch.zeros(csa.csa_mxfp4_sf128_bytes(B, T * 64), dtype=torch.uint8, device=dev)
         self.idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
         self.select_ws = csa.select_workspace(B, N, dev)
         self.attn_ws = csa.attn_workspace(B, T, H, D, 128 + k, device=dev)
@@ -289,6 +295,9 @@ class DecodeSet:
         if self.index == "e4m3":
             keys = B * N * (128 + 4)
             q = B * T * 64 * (128 + 4 + 4)
+        elif self.index == "mxfp4":
+            keys = B * N * (64 + 4)                 # 128 E2M1 codes + 4 E8M0 scales per key
+            q = B * T * 64 * (64 + 4 + 4)
         else:
             keys = B * N * 256
             q = B * T * 64 * (256 + 4)
@@ -311,11 +320,12 @@ class DecodeSet:
         nb = lambda t: t.numel() * t.element_size()
         total = sum(nb(t) for t in self.inputs.values())                       # per-step inputs
         total += nb(self.comp_kv)                                             # latent compressor output
-        if wl.comp_ci:                                                        # new index keys (+ e4m3)
-            total += B * (wl.comp_L // 4) * (256 + (132 if self.index == "e4m3" else 0))
-        total += B * N * (132 if self.index == "e4m3" else 256)               # index keys (+ scales)
-        if self.index == "e4m3":
-            total += B * T * 2 * k * 256                                      # rerank: bf16 keys of candidates
+        low = {"e4m3": 132, "mxfp4": 68}.get(self.index, 0)                 # low-precision key bytes
+        if wl.comp_ci:                                                        # new index keys (+ quantised)
+            total += B * (wl.comp_L // 4) * (256 + low)
+        total += B * N * (low if low else 256)                                # index keys (+ scales)
+        if low:
+            total += B * T * self.kc_factor() * k * 256                       # rescoring: bf16 keys of candidates
         total += B * T * (k * self.row_bytes() + min(wl.W, 128) * D * 2)      # gathered latent + SWA rows
         total += nb(self.out)
         if self.kv8:
@@ -326,6 +336,10 @@ class DecodeSet:
             if self.kv8:
                 total += nb(self.hcomp) + nb(self.hcomp8)
         return total
+
+    def kc_factor(self):
+        """Candidate list of the rescoring select, in units of k (FP4 scores are coarser)."""
+        return 4 if self.index == "mxfp4" else 2
 
     def per_step_io(self):
         nb = lambda t: t.numel() * t.element_size()
@@ -380,6 +394,15 @@ class DecodeSet:
                                                 x["iprev_Zb"], self.kI, pos0=self.new_key_pos,
                                                 k8=self.k8 if e4 else None, k_scale=self.ks if e4 else None,
                                                 hadamard=INDEX_ROTATION)
+                    if self.index == "mxfp4":
+                        # re-quantise the 128-row tiles that hold the new entries (N is a multiple
+                        # of 128): their codes and tensor-core-layout scales
+                        p0, n_new, tiles = self.new_key_pos, wl.comp_L // 4, wl.N // 128
+                        r0, r1 = (p0 // 128) * 128, -(-(p0 + n_new) // 128) * 128
+                        for b in range(wl.B):
+                            csa.csa_quantize_mxfp4_sf128(self.kI[b, r0:r1], (r1 - r0) // 128,
+                                                         codes=self.k4[b, r0:r1],
+                                                         sf=self.ksf[(b * tiles + r0 // 128) * 512:])
 
         # stage boundaries on the main stream (event record nodes inside the graph)
         # timing_events: False (the timed graphs) or "all" (every stage: a diagnostic graph;
@@ -401,6 +424,17 @@ class DecodeSet:
             side_branch()
             # top-2k bin of the e4m3 scores, exact bf16 rescoring, best k -- one launch
             csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, kc=2 * wl.topk, qI=x["qI"],
+                                w=x["w"], kI=self.kI, idx=self.idx)
+            mark("select")
+        elif self.index == "mxfp4":
+            csa.csa_quantize_mxfp4_sf128(x["qI"], wl.B, codes=self.q4, sf=self.qsf)
+            mark("quantize_q")
+            csa.csa_index_scores(self.q4, x["w"], self.k4, self.n_valid, q_scale=self.qsf, k_scale=self.ksf,
+                                 scores=self.scores, select_ws=self.select_ws, mxfp4=True)
+            mark("index")
+            side_branch()
+            # top-4k bin of the FP4 scores, exact bf16 rescoring, best k -- one launch
+            csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, kc=4 * wl.topk, qI=x["qI"],
                                 w=x["w"], kI=self.kI, idx=self.idx)
             mark("select")
         else:
@@ -549,6 +583,9 @@ def index_alone_ms(sets, index, device, reps_per_set=8, replays=20):
         if index == "e4m3":
             csa.csa_index_scores(s.q8, x["w"], s.k8, s.n_valid, q_scale=s.qs, k_scale=s.ks, scores=s.scores,
                                  select_ws=scratch[i % len(sets)])
+        elif index == "mxfp4":
+            csa.csa_index_scores(s.q4, x["w"], s.k4, s.n_valid, q_scale=s.qsf, k_scale=s.ksf, scores=s.scores,
+                                 select_ws=scratch[i % len(sets)], mxfp4=True)
         else:
             csa.csa_index_scores(x["qI"], x["w"], s.kI, s.n_valid, scores=s.scores, select_ws=scratch[i % len(sets)])
     for i in range(len(sets)):
@@ -573,7 +610,8 @@ def index_alone_ms(sets, index, device, reps_per_set=8, replays=20):
 
 
 def attn_alone_ms(sets, device, reps_per_set=8, replays=20):
-    """Average duration (ms) of one sparse_attn launch (attn_tc_kernel) timed alone:
+    """Average duration (ms) of one sparse_attn launch timed alone (attn_t_kernel for bf16
+    rows, attn_tc_kernel for KV8 entries):
     back-to-back launches in one CUDA graph cycling over the input sets (cold in L2),
     CUDA events around the graph replays."""
     import torch
@@ -900,14 +938,19 @@ def run_stage(name, stage, index, steps, warmup, device, kv8=False):
     calls = {
         "compress": lambda: csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], x["prev_Cb"], x["prev_Zb"],
                                              ratio=4, out=st.comp_kv),
-        "quantize": lambda: csa.csa_quantize_e4m3(x["qI"], codes=st.q8, scale=st.qs, hadamard=INDEX_ROTATION),
+        "quantize": (lambda: csa.csa_quantize_mxfp4_sf128(x["qI"], wl.B, codes=st.q4, sf=st.qsf))
+                    if index == "mxfp4" else
+                    (lambda: csa.csa_quantize_e4m3(x["qI"], codes=st.q8, scale=st.qs, hadamard=INDEX_ROTATION)),
         "index": (lambda: csa.csa_index_scores(st.q8, x["w"], st.k8, st.n_valid, q_scale=st.qs, k_scale=st.ks,
                                                scores=st.scores)) if index == "e4m3" else
+                 (lambda: csa.csa_index_scores(st.q4, x["w"], st.k4, st.n_valid, q_scale=st.qsf, k_scale=st.ksf,
+                                               scores=st.scores, mxfp4=True)) if index == "mxfp4" else
                  (lambda: csa.csa_index_scores(x["qI"], x["w"], st.kI, st.n_valid, scores=st.scores)),
         "select": (lambda: (csa.csa_score_histogram(st.scores, st.n_valid, st.select_ws),
-                            csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws, kc=2 * wl.topk,
-                                                qI=x["qI"], w=x["w"], kI=st.kI, idx=st.idx)))
-                  if index == "e4m3" else
+                            csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws,
+                                                kc=st.kc_factor() * wl.topk, qI=x["qI"], w=x["w"], kI=st.kI,
+                                                idx=st.idx)))
+                  if index in ("e4m3", "mxfp4") else
                   (lambda: (csa.csa_score_histogram(st.scores, st.n_valid, st.select_ws),
                             csa.csa_topk_select(st.scores, st.n_valid, wl.topk, st.select_ws, idx=st.idx))),
         "attn": lambda: csa.sparse_attn(x["q"], st.kv_store, st.swa, st.swa_pos0, st.q_pos, st.sink, st.idx,
@@ -919,7 +962,7 @@ def run_stage(name, stage, index, steps, warmup, device, kv8=False):
                                     workspace=st.hattn_ws),
     }
     # inputs of the later stages come from the earlier ones
-    order = ["quantize", "index", "select"] if index == "e4m3" else ["index", "select"]
+    order = ["quantize", "index", "select"] if index in ("e4m3", "mxfp4") else ["index", "select"]
     if stage in ("select", "attn"):
         for pre in order[:order.index(stage)] if stage in order else order:
             calls[pre]()
@@ -1073,6 +1116,8 @@ def workload_text(wl, index, with_hca):
     return (f"{wl.name}: B={wl.B} decode tokens/GPU at ctx {wl.ctx}; CSA layer (compress 4:1 c=512+128, "
             f"{index} index over N={wl.N}, top-{wl.topk}"
             + ((" (Hadamard-rotated q/k)" if INDEX_ROTATION else "") + " via 2k rerank" if index == "e4m3" else "")
+            + ((" (Hadamard-rotated q/k, MXFP4)" if INDEX_ROTATION else " (MXFP4)") + " via 4k rescoring"
+               if index == "mxfp4" else "")
             + f", sparse_attn H={wl.H} D={wl.D})"
             + (f" + HCA layer (compress 128:1, hca_attn over {wl.ctx // 128}+128 rows)" if with_hca else ""))
 
@@ -1085,7 +1130,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="flash64k", choices=["flash64k", "pro1m"])
-    ap.add_argument("--index", default="e4m3", choices=["e4m3", "bf16"])
+    ap.add_argument("--index", default="e4m3", choices=["e4m3", "bf16", "mxfp4"])
     ap.add_argument("--no-hadamard", action="store_true",
                     help="e4m3 index path without the Hadamard rotation of queries and keys")
     ap.add_argument("--no-extra", action="store_true", help="skip the pro1m measurement")
@@ -1157,6 +1202,9 @@ def main():
                                                              device)
         variants["flash64k_csa_only"] = bench_workload("flash64k", args.index, False, args.steps, args.warmup, world,
                                                        device)
+    if not args.no_extra:
+        # the FP4 index QK: MXFP4 scores, 4k candidates rescored exactly in bf16
+        variants["pro1m_mxfp4_index"] = bench_workload("pro1m", "mxfp4", False, args.steps, args.warmup, world, device)
     prefill = hca = None
     kv8_runs = {}
     if not args.no_extra:
@@ -1186,23 +1234,25 @@ def main():
             "value": tok * steps / r["seconds"], "ms_per_step": r["step_ms"],
             "e2e": {"value": tok * steps / r["e2e_seconds"], "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-            "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (sparse_attn: top-k + SWA rows, cluster merge"
-                                                   + (", memory rows as KV8 entries)" if kv8 else ")"),
+            "roofline": {"bound": "hbm", "kernel": ("attn_tc_kernel (sparse_attn: top-k + SWA rows, cluster merge, "
+                                                    "memory rows as KV8 entries)") if kv8 else
+                         ("attn_t_kernel (sparse_attn: top-k + SWA rows as the MMA's M, split over a cluster, "
+                          "partials merged through L2, partial RoPE)"),
                          "achieved": attn_gbs, "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak,
                          "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
                          "traffic": profiled_traffic("attn_tc_kernel_decode_prefill_hca.md", "attn.cuh",
-                                                     wl.name + ("_kv8" if kv8 else "")),
+                                                     wl.name + "_kv8") if kv8 else
+                                    profiled_traffic("attn_t_kernel_decode.md", "attn_t.cuh", wl.name),
                          "bytes_per_launch": r["attn_bytes"], "avg_launch_us": r["attn_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays",
                          "why_this_kernel": "largest share of the step in the ncu launch list (two launches per "
                                             "step: CSA sparse_attn and HCA hca_attn)"},
-            "roofline_indexer": {"bound": "hbm", "kernel": "index_tc_kernel (csa_index_scores, e4m3)" if r["index"] == "e4m3"
-                         else "index_tc_kernel (csa_index_scores, bf16)",
+            "roofline_indexer": {"bound": "hbm", "kernel": f"index_tc_kernel (csa_index_scores, {r['index']})",
                          "achieved": idx_gbs, "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak,
                          "peak_source": peak_kind + " (burst copy; the kernel is timed alone)",
-                         "traffic": profiled_traffic("index_tc_kernel_e4m3_decode.md", "index.cuh", wl.name)
-                         if r["index"] == "e4m3" else None,
+                         "traffic": profiled_traffic(f"index_tc_kernel_{r['index']}_decode.md", "index.cuh",
+                                                     wl.name) if r["index"] in ("e4m3", "mxfp4") else None,
                          "bytes_per_launch": r["index_bytes"], "avg_launch_us": r["index_ms"] * 1e3,
                          "timing": "back-to-back launches in one CUDA graph over rotating input sets (cold in L2), "
                                    "CUDA events around the graph replays"},
@@ -1243,6 +1293,7 @@ def main():
         line[nm] = {"value": e["value"], "unit": "tokens/s", "ms_per_step": e["ms_per_step"],
                     "workload": workload_text(r["wl"], r["index"], r["with_hca"]),
                     "step_roofline": e["step_roofline"], "roofline_indexer": e["roofline_indexer"], "e2e": e["e2e"],
+                    "roofline": e["roofline"],
                     "launches_per_step": e["launches_per_step"], "breakdown_us": e["breakdown_us"]}
         line["gpu_launches"] += e["gpu_launches"]
     if prefill is not None:

@@ -331,10 +331,17 @@ int csa_quantize_kv8(const void *kv, int64_t rows, int D, void *entries, void *s
  *   dtype CSA_BF16 (tcgen05, fp32 softmax and accumulation; H <= 128,
  *   D in {128, 256, 512}), CSA_BF16_KV8 (as CSA_BF16 with kv [B, N, 608] bytes of
  *   csa_quantize_kv8 entries; D = 512) or CSA_F32 (fp32 FMA; D multiple of 32, <= 512).
- *   workspace : csa_attn_workspace_size(...) bytes; may be NULL when that size
- *               is 0, which it is in this version: the row list of a query is
- *               split over up to 16 CTAs that form one thread-block cluster and
- *               merge their partial results in distributed shared memory.
+ *   workspace : csa_attn_workspace_size(B, T, H, D, rows_per_query, dtype) bytes
+ *               (16-byte aligned, device memory, owned by the caller, contents
+ *               need not be kept between calls), rows_per_query = min(W, 128) + k
+ *               for sparse_attn and min(W, 128) + N for hca_attn (a larger value
+ *               gives a size that is also enough); may be NULL when that size is 0.
+ *               With few queries (B * T * ceil(H / 64) below the SM count) the
+ *               CSA_BF16 row list of a query is split over up to 16 CTAs of one
+ *               thread-block cluster that write their unnormalised partial
+ *               outputs and (m, l) there and merge them after a cluster barrier;
+ *               CSA_BF16_KV8 and CSA_F32 need none (size 0).  Too small or
+ *               misaligned -> CSA_ERR_INVALID, nothing launched.
  */
 size_t csa_attn_workspace_size(int B, int T, int H, int D, int64_t rows_per_query, int dtype);
 int sparse_attn(const void *q, const void *kv, const void *swa_kv, const int64_t *swa_pos0, int W,

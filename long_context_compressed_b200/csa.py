@@ -203,6 +203,11 @@ def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=N
     return scores
 
 
+def csa_mxfp4_sf128_bytes(batches: int, rows_per_batch: int) -> int:
+    """Bytes of the tensor-core-layout scales of `batches` x `rows_per_batch` MXFP4 rows."""
+    return int(_lib.csa_mxfp4_sf128_bytes(batches, rows_per_batch))
+
+
 def csa_quantize_mxfp4_sf128(x, batches: int, *, hadamard: bool = True, codes=None, sf=None, stream=None):
     """MXFP4 index operands with the scales in the tensor-core layout: x [..., 128] (fp32 | bf16) whose
     rows form `batches` equal batches -> (codes uint8 [..., 64], sf uint8 [csa_mxfp4_sf128_bytes])."""
@@ -211,7 +216,7 @@ def csa_quantize_mxfp4_sf128(x, batches: int, *, hadamard: bool = True, codes=No
     if codes is None:
         codes = torch.empty(x.shape[:-1] + (64,), dtype=torch.uint8, device=x.device)
     if sf is None:
-        sf = torch.zeros(max(16, int(_lib.csa_mxfp4_sf128_bytes(batches, rpb))), dtype=torch.uint8, device=x.device)
+        sf = torch.zeros(max(16, csa_mxfp4_sf128_bytes(batches, rpb)), dtype=torch.uint8, device=x.device)
     _check(_lib.csa_quantize_mxfp4_sf128(_ptr(x), _dtype_code(x), batches, rpb, int(bool(hadamard)), _ptr(codes),
                                          _ptr(sf), _stream(stream)), "csa_quantize_mxfp4_sf128")
     return codes, sf

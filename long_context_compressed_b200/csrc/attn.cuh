@@ -63,6 +63,8 @@ struct AttnParams {
   int64_t N;
   double rope_theta;      // > 0: partial RoPE around the attention (rope.cuh); 0: none
   RopeFreqs rope_freq;    // theta^(-2i/64), i < 32 (when rope_theta > 0)
+  void* part_o;           // attn_t_kernel with splits: bf16 [B*T*groups][nsplit][64][D] unnormalised O
+  void* part_ml;          // ... and float2 [B*T*groups][nsplit][64] (m (log2), l) of each split
 };
 
 struct RowList {

@@ -31,8 +31,11 @@
 // shared memory.  The reference maximum of a head is raised only when a unit's maximum
 // exceeds it by more than 2^64 (base 2), so exponentials stay <= 2^64 and O^T is rescaled
 // in tensor memory only in that rare case.  With several splits the split CTAs of one
-// (query, head group) form a thread-block cluster and merge their unnormalised O and
-// (m, l) through distributed shared memory, sink included.
+// (query, head group) form a thread-block cluster: each stores its unnormalised O (bf16)
+// and per-head (m, l) straight from tensor memory into a workspace, one cluster barrier
+// (release / acquire) orders those stores before the reads, and CTA r then bulk-copies
+// heads [r*64/ns, (r+1)*64/ns) of every split into its idle KV stages and merges them
+// there, sink included.
 #pragma once
 #include <cuda_bf16.h>
 #include "attn.cuh"
@@ -62,6 +65,8 @@ struct AttnTCfg {
   static constexpr float kRescaleLog2 = 64.f;      // raise a head's reference max beyond this
   static_assert(D == 128 || D == 256 || D == 512, "D");
   static_assert(kStage == kQ, "a stage's upper-half filler reads stay inside shared memory");
+  static_assert(NS * kStage >= (HG + kMaxSplits - 1) * D * 2 + kMaxSplits * HG * 8,
+                "the merge's copies of every split's heads fit in the KV stages");
 };
 
 // Byte offset of 16-byte chunk c of row r inside a stage (8-row groups, atoms of 128 B).
@@ -113,7 +118,7 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
   uint64_t* qfull = bars + 10;
   uint64_t* odone = bars + 11;
   uint64_t* qrot = bars + 13;     // RoPE dims of q turned (4 softmax warps)
-  uint64_t* recv_bar = bars + 18; // cluster merge: the peers' slices of this CTA's heads arrived
+  uint64_t* merge_bar = bars + 18; // the splits' pieces of this CTA's heads copied in
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 14);   // [2 stages][4 loader warps], 16 rows each
   int32_t* idx_s = reinterpret_cast<int32_t*>(bars + 64);      // [kMaxCtaRows]
@@ -123,14 +128,13 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
   __shared__ float m_use[HG], fscale[HG];
   __shared__ float epi_g[HG];
   __shared__ int epi_have_o;
-  __shared__ __align__(16) float2 cl_ml[HG];       // per head (m, l) of this CTA's rows
-  __shared__ float cl_w[HG][kMaxSplits];
   __shared__ float2 rope_tab[kRopeDims / 2];   // cos, sin of the query position's angles
 
   const int qi = blockIdx.z;                     // b * T + t
   const int b = qi / p.T, t = qi % p.T;
   const int h0 = blockIdx.y * HG;
   const int split = blockIdx.x;
+  const int64_t item = (int64_t)qi * gridDim.y + blockIdx.y;   // (query, head group)
   const int warp = warp_id();
   const int32_t* idx_row = p.sparse ? p.idx + ((int64_t)b * p.T + t) * p.k : nullptr;
 
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     mbar_init(qfull, 1);
     mbar_init(odone, 1);
     mbar_init(qrot, 4);
-    mbar_init(recv_bar, 1);
+    mbar_init(merge_bar, 1);
     fence_mbar_init();
   }
   if (warp == 8) {
@@ -190,9 +194,11 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     if (nu > 0) {
       const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(p.kv);
       const __nv_bfloat16* swa = static_cast<const __nv_bfloat16*>(p.swa);
-      constexpr int CPR = D / 8;                 // 16-byte chunks per row
-      constexpr int CPT = CPR / 2;               // chunks per thread and unit (2 threads per row)
-      const int my_r = lt >> 1, my_c = lt & 1;
+      // warp w fills rows 16w .. 16w+15 of a unit, four rows per pass: lane l copies 16-byte
+      // chunk l % 8 of every 128-byte atom of row 4 * pass + l / 8, so one cp.async of the
+      // warp reads four whole 128-byte lines
+      const int wl = lt >> 5, lane = (int)lane_id();
+      const int sub = lane >> 3, c8 = lane & 7;
       const int nrow = nu * U;
       const bool staged_idx = p.sparse && nrow <= Cfg::kMaxCtaRows;
       if (staged_idx) {
@@ -208,12 +214,10 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
         uint8_t* stage = kv_s + s * Cfg::kStage;
         const int rg0 = row0 + u * U;
-        const int rg = rg0 + my_r;
         const bool swa_tile = p.has_swamap && rg0 + U <= rl.n_swa;
         const bool mem_tile = p.has_kvmap && !p.sparse && rg0 >= mem0 && rg0 + U <= n_rows;
-        bool valid;
+        uint32_t rows = 0xFFFFu;                  // validity of this warp's 16 rows
         if (swa_tile || mem_tile) {
-          valid = true;
           // eight boxes of {64 dims, 8 rows, all atoms}: each lands as one 8-row group
           if (lt < 32) {
             if (lt == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kStage);
@@ -227,28 +231,41 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
             mbar_arrive(&full[s]);
           }
         } else {
-          int32_t raw = 0;
-          if (p.sparse && rg >= mem0 && rg < n_rows)
-            raw = staged_idx ? idx_s[u * U + my_r] : __ldg(idx_row + (rg - mem0));
-          const int64_t so = row_src(rg, raw);
-          const __nv_bfloat16* src = so >= 0 ? kv + so : (so <= -2 ? swa + (-2 - so) : nullptr);
-          valid = src != nullptr;
-#pragma unroll 8
-          for (int i = 0; i < CPT; ++i) {
-            const int ch = my_c + 2 * i;
-            uint8_t* dst = stage + st_off<D>(my_r, ch);
-            if (src) cp_async_16(dst, src + ch * 8);
-            else st_shared_zero16(dst);           // finite filler for rows that do not contribute
+          const __nv_bfloat16* src[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = 16 * wl + 4 * j + sub;
+            const int rg = rg0 + r;
+            int32_t raw = 0;
+            if (p.sparse && rg >= mem0 && rg < n_rows)
+              raw = staged_idx ? idx_s[u * U + r] : __ldg(idx_row + (rg - mem0));
+            const int64_t so = row_src(rg, raw);
+            src[j] = so >= 0 ? kv + so : (so <= -2 ? swa + (-2 - so) : nullptr);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = 16 * wl + 4 * j + sub;
+#pragma unroll
+            for (int a = 0; a < Cfg::kAtoms; ++a) {
+              const int ch = a * 8 + c8;
+              uint8_t* dst = stage + st_off<D>(r, ch);
+              if (src[j]) cp_async_16(dst, src[j] + ch * 8);
+              else st_shared_zero16(dst);         // finite filler for rows that do not contribute
+            }
           }
           fence_proxy_async_smem();
           cp_async_arrive_noinc(&full[s]);
+          rows = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t bal = __ballot_sync(0xffffffffu, src[j] != nullptr);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rows |= ((bal >> (8 * q)) & 1u) << (4 * j + q);
+          }
         }
-        // row validity, one word per loader warp (16 rows, 2 threads per row)
-        const uint32_t bal = __ballot_sync(0xffffffffu, valid);
-        if (lane_id() == 0) {
-          uint32_t rows = 0;
-          for (int j = 0; j < 16; ++j) rows |= ((bal >> (2 * j)) & 1u) << j;
-          mask_s[s * 4 + (lt >> 5)] = rows;
+        // row validity, one word per loader warp (16 rows)
+        if (lane == 0) {
+          mask_s[s * 4 + wl] = rows;
           mbar_arrive(&full[s]);
         }
       }
@@ -483,7 +500,9 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
         }
       }
       epi_g[r] = g;
-      cl_ml[r] = have_o ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
+      if (p.nsplit > 1)
+        reinterpret_cast<float2*>(p.part_ml)[(item * p.nsplit + split) * HG + r] =
+            have_o ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
     }
     if (r == 0) epi_have_o = have_o ? 1 : 0;
     tc_fence_before();
@@ -499,14 +518,14 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     const int quarter = warp & 3;
     const uint32_t lane_q = (uint32_t)(quarter * 32) << 16;
     const int lane = (int)lane_id();
-    // the KV stages are idle: this warp's transpose buffer (64 heads x 32 dims bf16), or the
-    // cluster's parked partials [64 heads][D] bf16
+    // the KV stages are idle: this warp's transpose buffer (64 heads x 32 dims bf16); with
+    // splits, this split's partial O [64 heads][D] bf16 in the workspace
     uint8_t* stage = kv_s + warp * (HG * 64);
-    __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(kv_s);
+    __nv_bfloat16* obuf = static_cast<__nv_bfloat16*>(p.part_o) + (item * p.nsplit + split) * HG * D;
     const int nh = min(HG, p.H - h0);
     for (int m = warp >> 2; m < Cfg::kMT; m += 2) {
       const int d = m * 128 + quarter * 32 + lane;
-      if (p.nsplit == 1) __syncwarp();
+      __syncwarp();
       float oall[HG];
       if (have_o) {
         tmem_ld32(tmem + lane_q + m * HG, oall);
@@ -521,7 +540,8 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
         float* o = oall + hh;
         if (p.nsplit > 1) {
           // [head][D] bf16: lanes d, d ^ 1 pair up, the even lane storing even heads and the
-          // odd lane odd heads as two adjacent values (one 4-byte store each)
+          // odd lane odd heads as two adjacent values (one 4-byte store each; per store the
+          // warp writes 64 contiguous bytes of two head rows)
           const bool odd = (d & 1) != 0;
 #pragma unroll
           for (int h = 0; h < 32; h += 2) {
@@ -564,78 +584,64 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
   if (p.nsplit > 1) {
     // ------------------------------------------------------------ merge of the splits
     // CTA `rank` finishes heads [rank*64/ns, (rank+1)*64/ns): M = max(sink, m_j),
-    // den = 2^(sink - M) + sum_j l_j 2^(m_j - M), out = sum_j 2^(m_j - M) O_j / den.  Every
-    // CTA pushes each peer's heads of its raw O (bf16 [64][D] in stage 0) into that peer's
-    // receive area by one bulk shared-to-shared copy; the peer sums locally.
+    // den = 2^(sink - M) + sum_j l_j 2^(m_j - M), out = sum_j 2^(m_j - M) O_j / den.
     const int ns = p.nsplit;
-    const uint32_t rank = cluster_ctarank();
-    const int hb = (int)rank * HG / ns, he = ((int)rank + 1) * HG / ns;
-    const int hpc = (HG + ns - 1) / ns;               // receive slot of one peer: hpc head rows
-    const __nv_bfloat16* part = reinterpret_cast<const __nv_bfloat16*>(kv_s);        // own raw O [64][D]
-    __nv_bfloat16* recv = reinterpret_cast<__nv_bfloat16*>(kv_s + Cfg::kStage);   // [ns][hpc][D]
-    float2* recv_ml = reinterpret_cast<float2*>(recv + (size_t)ns * hpc * D);       // [ns][64] (m, l)
-    cluster_sync();                                   // every split's O and (m, l) are in place
+    const int rank = (int)cluster_ctarank();
+    const int hb = rank * HG / ns, he = (rank + 1) * HG / ns, nhl = he - hb;
+    const __nv_bfloat16* po = static_cast<const __nv_bfloat16*>(p.part_o) + item * ns * HG * D;
+    const float2* pml = static_cast<const float2*>(p.part_ml) + item * ns * HG;
+    // the idle KV stages receive [ns][nhl][D] bf16 (split j's rows of heads hb..he-1), then
+    // [ns][64] (m, l)
+    const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(kv_s);
+    const float2* recv_ml = reinterpret_cast<const float2*>(kv_s + (size_t)ns * nhl * D * 2);
+    cluster_sync();                                   // release / acquire: every split's O and (m, l) are stored
     if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(recv_bar, (uint32_t)((ns - 1) * ((he - hb) * D * 2 + HG * 8)));
-      const uint32_t src = smem_u32(kv_s);
-      const uint32_t dst_o = smem_u32(recv + (size_t)rank * hpc * D);
-      const uint32_t dst_ml = smem_u32(recv_ml + rank * HG);
-      for (int j = 0; j < ns; ++j) {
-        if (j == (int)rank) continue;
-        const int hbj = j * HG / ns, hej = (j + 1) * HG / ns;
-        const uint32_t bar_j = cluster_map(smem_u32(recv_bar), (uint32_t)j);
-        bulk_s2cluster(cluster_map(dst_o, (uint32_t)j), src + (uint32_t)(hbj * D * 2), (uint32_t)((hej - hbj) * D * 2),
-                       bar_j);
-        bulk_s2cluster(cluster_map(dst_ml, (uint32_t)j), smem_u32(cl_ml), (uint32_t)(HG * 8), bar_j);
-      }
+      fence_proxy_async_global();                     // those generic stores -> the bulk copies' reads
+      const uint32_t bytes_o = (uint32_t)(nhl * D * 2);
+      mbar_arrive_expect_tx(merge_bar, (uint32_t)ns * (bytes_o + HG * 8));
+      for (int j = 0; j < ns; ++j)
+        bulk_load(kv_s + (size_t)j * bytes_o, po + ((int64_t)j * HG + hb) * D, bytes_o, merge_bar);
+      bulk_load(kv_s + (size_t)ns * bytes_o, pml, (uint32_t)ns * HG * 8, merge_bar);
     }
-    const bool arrived = mbar_wait(recv_bar, 0);
-    for (int hl = threadIdx.x; arrived && hl < he - hb; hl += blockDim.x) {
-      const int hh = hb + hl;
-      float mj[kMaxSplits], lj[kMaxSplits];
-      const float sinkL = (h0 + hh >= p.H) ? 0.f : (p.ml ? -INFINITY : p.sink[h0 + hh] * kLog2e);
+    const bool arrived = mbar_wait(merge_bar, 0);
+    // one thread per 8 output dims of a head; each forms its head's split weights itself
+    // (no further barrier)
+    constexpr int F = D / 8;                          // 16-byte pieces (8 bf16) per head row
+    for (int it = threadIdx.x; arrived && it < nhl * F; it += blockDim.x) {
+      const int hl = it / F, hh = hb + hl, f = it % F;
+      if (h0 + hh >= p.H) continue;
+      float2 ml[kMaxSplits];
+#pragma unroll
+      for (int j = 0; j < kMaxSplits; ++j) ml[j] = j < ns ? recv_ml[j * HG + hh] : make_float2(-INFINITY, 0.f);
+      const float sinkL = p.ml ? -INFINITY : p.sink[h0 + hh] * kLog2e;
       float M = sinkL;
 #pragma unroll
-      for (int j = 0; j < kMaxSplits; ++j) {
-        const float2 v = j < ns ? (j == (int)rank ? cl_ml[hh] : recv_ml[j * HG + hh]) : make_float2(-INFINITY, 0.f);
-        mj[j] = v.x;
-        lj[j] = v.y;
-        M = fmaxf(M, mj[j]);
-      }
+      for (int j = 0; j < kMaxSplits; ++j) M = fmaxf(M, ml[j].x);
       const bool any = M > -INFINITY;
       float den = any ? ex2_approx(sinkL - M) : 0.f;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
-        mj[j] = any ? ex2_approx(mj[j] - M) : 0.f;
-        den = fmaf(lj[j], mj[j], den);
+        ml[j].x = any ? ex2_approx(ml[j].x - M) : 0.f;
+        den = fmaf(ml[j].y, ml[j].x, den);
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
-      if (p.ml && h0 + hh < p.H)
+      if (p.ml && f == 0)
         reinterpret_cast<float2*>(p.ml)[(int64_t)qi * p.H + h0 + hh] =
             den > 0.f ? make_float2(M * kLn2, den) : make_float2(-INFINITY, 0.f);
-#pragma unroll
-      for (int j = 0; j < kMaxSplits; ++j) cl_w[hh][j] = mj[j] * inv;
-    }
-    __syncthreads();
-    constexpr int F = D / 8;                          // 16-byte slots (8 bf16) per head row
-    for (int it = threadIdx.x; arrived && it < (he - hb) * F; it += blockDim.x) {
-      const int hl = it / F, hh = hb + hl, f = it % F;
-      if (h0 + hh >= p.H) continue;
       float acc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
         if (j < ns) {
-          const float wj = cl_w[hh][j];
-          const __nv_bfloat16* srcj = j == (int)rank ? part + (size_t)hh * D : recv + ((size_t)j * hpc + hl) * D;
-          const uint4 v = *reinterpret_cast<const uint4*>(srcj + f * 8);
+          const float w = ml[j].x * inv;
+          const uint4 v = *reinterpret_cast<const uint4*>(recv + ((size_t)j * nhl + hl) * D + f * 8);
           const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 x = __bfloat1622float2(hv[e]);
-            acc[2 * e] = fmaf(wj, x.x, acc[2 * e]);
-            acc[2 * e + 1] = fmaf(wj, x.y, acc[2 * e + 1]);
+            acc[2 * e] = fmaf(w, x.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(w, x.y, acc[2 * e + 1]);
           }
         }
       }
@@ -654,9 +660,6 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       for (int e = 0; e < 4; ++e) ho[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((int64_t)qi * p.H + h0 + hh) * D + f * 8) = u;
     }
-    // no CTA leaves while a copy into or out of its shared memory, or a read of its (m, l),
-    // is still in flight
-    cluster_sync();
   }
 
   tc_fence_before();

@@ -238,22 +238,38 @@ int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse, int R
   return (int)std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), csa::kMaxSplits));   // one cluster
 }
 
-// The split partials merge inside the kernel (cluster shared memory): no workspace.
-size_t attn_ws_bytes(int, int, int, int, int64_t, int) { return 0; }
+// bf16 rows (attn_t_kernel): splits of a query's row list (units of 64 rows) form one
+// cluster: as many as the SMs allow for one wave, at most one per unit and at most
+// kMaxSplits (the launch may take fewer, while the clusters would not all be resident).
+int attn_t_splits(int B, int T, int H, int64_t max_rows) {
+  const int64_t items = (int64_t)B * T * ((H + 63) / 64);
+  const int64_t units = std::max<int64_t>(1, (max_rows + 63) / 64);
+  const int sms = sm_count();
+  if (items <= 0 || items >= sms) return 1;
+  return (int)std::min<int64_t>(std::min<int64_t>(csa::kMaxSplits, units), std::max<int64_t>(1, sms / items));
+}
+
+// Workspace of a split launch: each split's unnormalised O (bf16, 64 heads x D) and its
+// per-head (m, l) (two floats), per (query, head group).  The KV8 and fp32 kernels merge
+// without one (cluster shared memory; no splits).
+size_t attn_t_ws_bytes(int B, int T, int H, int D, int ns) {
+  if (ns <= 1) return 0;
+  const size_t items = (size_t)B * T * ((H + 63) / 64);
+  return items * ns * 64 * ((size_t)D * 2 + 8);
+}
+
+size_t attn_ws_bytes(int B, int T, int H, int D, int64_t rows, int dtype) {
+  if (dtype != CSA_BF16) return 0;
+  return attn_t_ws_bytes(B, T, H, D, attn_t_splits(B, T, H, rows));
+}
 
 // bf16 rows: attn_t_kernel (rows as the MMA's M dimension, 64 heads per CTA, all of D).
-// Splits of a query's row list (units of 64 rows) form one cluster: as many as the SMs
-// allow for one wave, at most one per unit and at most kMaxSplits, and fewer while the
-// clusters would not all be resident at once.
 template <int D>
-int launch_attn_t(AttnParams p, int64_t max_rows, cudaStream_t st) {
+int launch_attn_t(AttnParams p, int64_t max_rows, void* ws, size_t ws_bytes, cudaStream_t st) {
   using Cfg = csa::AttnTCfg<D>;
   const int groups = (p.H + Cfg::HG - 1) / Cfg::HG;
   const int64_t items = (int64_t)p.B * p.T * groups;
-  const int64_t units = std::max<int64_t>(1, (max_rows + Cfg::U - 1) / Cfg::U);
-  const int sms = sm_count();
-  int ns = 1;
-  if (items < sms) ns = (int)std::min<int64_t>(std::min<int64_t>(csa::kMaxSplits, units), std::max<int64_t>(1, sms / items));
+  int ns = attn_t_splits(p.B, p.T, p.H, max_rows);
   auto kernel = csa::attn_t_kernel<D>;
   while (ns > 1) {
     const int fit = max_active_clusters(kernel, Cfg::kThreads, Cfg::kSmem, ns);
@@ -265,6 +281,12 @@ int launch_attn_t(AttnParams p, int64_t max_rows, cudaStream_t st) {
     --ns;
   }
   p.nsplit = ns;
+  if (ns > 1) {
+    const size_t need = attn_t_ws_bytes(p.B, p.T, p.H, D, ns);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return CSA_ERR_INVALID;
+    p.part_o = ws;
+    p.part_ml = static_cast<uint8_t*>(ws) + items * ns * 64 * (size_t)D * 2;
+  }
   CUtensorMap qmap, kvmap, swamap;
   if (!make_map(&qmap, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)D, (uint64_t)p.H, (uint64_t)p.B * p.T,
                 64, 64))
@@ -281,11 +303,11 @@ int launch_attn_t(AttnParams p, int64_t max_rows, cudaStream_t st) {
   return launch_status();
 }
 
-int run_attn_t(const AttnParams& p, int64_t max_rows, cudaStream_t st) {
+int run_attn_t(const AttnParams& p, int64_t max_rows, void* ws, size_t ws_bytes, cudaStream_t st) {
   switch (p.D) {
-    case 128: return launch_attn_t<128>(p, max_rows, st);
-    case 256: return launch_attn_t<256>(p, max_rows, st);
-    case 512: return launch_attn_t<512>(p, max_rows, st);
+    case 128: return launch_attn_t<128>(p, max_rows, ws, ws_bytes, st);
+    case 256: return launch_attn_t<256>(p, max_rows, ws, ws_bytes, st);
+    case 512: return launch_attn_t<512>(p, max_rows, ws, ws_bytes, st);
     default: return CSA_ERR_UNSUPPORTED;
   }
 }
@@ -305,7 +327,7 @@ int run_attn(AttnParams p, int dtype, void* ws, size_t ws_bytes, int64_t max_row
     return launch_status();
   }
   const bool kv8 = dtype == CSA_BF16_KV8;
-  if (!kv8) return run_attn_t(p, max_rows, st);
+  if (!kv8) return run_attn_t(p, max_rows, ws, ws_bytes, st);
   // rows per KV tile: 32 at D = 512 (four stages in shared memory), else 64.  Measured:
   // 64-row tiles at D = 512 (two stages) were slower for gathered, dense and KV8 rows.
   const int R = p.D < 512 ? 64 : 32;

@@ -90,6 +90,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders earlier generic-proxy accesses of global memory with later async-proxy ones (a
+// bulk copy that reads what other threads stored).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 // 2-D / 3-D TMA tile load into this CTA's shared memory, completion counted on
 // the mbarrier in bytes.  Plain loads only: no cluster multicast anywhere.
