@@ -33,9 +33,10 @@
 // in tensor memory only in that rare case.  With several splits the split CTAs of one
 // (query, head group) form a thread-block cluster: each stores its unnormalised O (bf16)
 // and per-head (m, l) straight from tensor memory into a workspace, one cluster barrier
-// (release / acquire) orders those stores before the reads, and CTA r then bulk-copies
-// heads [r*64/ns, (r+1)*64/ns) of every split into its idle KV stages and merges them
-// there, sink included.
+// (release / acquire) orders those stores before the reads, and CTA r then merges heads
+// [r*64/ns, (r+1)*64/ns) of every split from L2, sink included.  (Measured against this:
+// bulk copies of the slices into shared memory, and a push of bf16 slices between the
+// CTAs' shared memories; both slower.)
 #pragma once
 #include <cuda_bf16.h>
 #include "attn.cuh"
@@ -65,8 +66,6 @@ struct AttnTCfg {
   static constexpr float kRescaleLog2 = 64.f;      // raise a head's reference max beyond this
   static_assert(D == 128 || D == 256 || D == 512, "D");
   static_assert(kStage == kQ, "a stage's upper-half filler reads stay inside shared memory");
-  static_assert(NS * kStage >= (HG + kMaxSplits - 1) * D * 2 + kMaxSplits * HG * 8,
-                "the merge's copies of every split's heads fit in the KV stages");
 };
 
 // Byte offset of 16-byte chunk c of row r inside a stage (8-row groups, atoms of 128 B).
@@ -118,7 +117,6 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
   uint64_t* qfull = bars + 10;
   uint64_t* odone = bars + 11;
   uint64_t* qrot = bars + 13;     // RoPE dims of q turned (4 softmax warps)
-  uint64_t* merge_bar = bars + 18; // the splits' pieces of this CTA's heads copied in
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 14);   // [2 stages][4 loader warps], 16 rows each
   int32_t* idx_s = reinterpret_cast<int32_t*>(bars + 64);      // [kMaxCtaRows]
@@ -149,7 +147,6 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     mbar_init(qfull, 1);
     mbar_init(odone, 1);
     mbar_init(qrot, 4);
-    mbar_init(merge_bar, 1);
     fence_mbar_init();
   }
   if (warp == 8) {
@@ -585,34 +582,30 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     // ------------------------------------------------------------ merge of the splits
     // CTA `rank` finishes heads [rank*64/ns, (rank+1)*64/ns): M = max(sink, m_j),
     // den = 2^(sink - M) + sum_j l_j 2^(m_j - M), out = sum_j 2^(m_j - M) O_j / den.
+    // One thread per 8 output dims of a head: it loads the ns (m, l) pairs and the ns
+    // 16-byte pieces of O at once (L2 only: they were written by other SMs) and sums.
     const int ns = p.nsplit;
     const int rank = (int)cluster_ctarank();
-    const int hb = rank * HG / ns, he = (rank + 1) * HG / ns, nhl = he - hb;
+    const int hb = rank * HG / ns, he = (rank + 1) * HG / ns;
     const __nv_bfloat16* po = static_cast<const __nv_bfloat16*>(p.part_o) + item * ns * HG * D;
     const float2* pml = static_cast<const float2*>(p.part_ml) + item * ns * HG;
-    // the idle KV stages receive [ns][nhl][D] bf16 (split j's rows of heads hb..he-1), then
-    // [ns][64] (m, l)
-    const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(kv_s);
-    const float2* recv_ml = reinterpret_cast<const float2*>(kv_s + (size_t)ns * nhl * D * 2);
     cluster_sync();                                   // release / acquire: every split's O and (m, l) are stored
-    if (threadIdx.x == 0) {
-      fence_proxy_async_global();                     // those generic stores -> the bulk copies' reads
-      const uint32_t bytes_o = (uint32_t)(nhl * D * 2);
-      mbar_arrive_expect_tx(merge_bar, (uint32_t)ns * (bytes_o + HG * 8));
-      for (int j = 0; j < ns; ++j)
-        bulk_load(kv_s + (size_t)j * bytes_o, po + ((int64_t)j * HG + hb) * D, bytes_o, merge_bar);
-      bulk_load(kv_s + (size_t)ns * bytes_o, pml, (uint32_t)ns * HG * 8, merge_bar);
-    }
-    const bool arrived = mbar_wait(merge_bar, 0);
-    // one thread per 8 output dims of a head; each forms its head's split weights itself
-    // (no further barrier)
     constexpr int F = D / 8;                          // 16-byte pieces (8 bf16) per head row
-    for (int it = threadIdx.x; arrived && it < nhl * F; it += blockDim.x) {
-      const int hl = it / F, hh = hb + hl, f = it % F;
+    for (int it = threadIdx.x; it < (he - hb) * F; it += blockDim.x) {
+      const int hh = hb + it / F, f = it % F;
       if (h0 + hh >= p.H) continue;
       float2 ml[kMaxSplits];
+      uint4 v[kMaxSplits];
 #pragma unroll
-      for (int j = 0; j < kMaxSplits; ++j) ml[j] = j < ns ? recv_ml[j * HG + hh] : make_float2(-INFINITY, 0.f);
+      for (int j = 0; j < kMaxSplits; ++j) {
+        if (j < ns) {
+          ml[j] = __ldcg(pml + j * HG + hh);
+          v[j] = __ldcg(reinterpret_cast<const uint4*>(po + ((int64_t)j * HG + hh) * D + f * 8));
+        } else {
+          ml[j] = make_float2(-INFINITY, 0.f);
+          v[j] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       const float sinkL = p.ml ? -INFINITY : p.sink[h0 + hh] * kLog2e;
       float M = sinkL;
 #pragma unroll
@@ -633,16 +626,13 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
       for (int j = 0; j < kMaxSplits; ++j) {
-        if (j < ns) {
-          const float w = ml[j].x * inv;
-          const uint4 v = *reinterpret_cast<const uint4*>(recv + ((size_t)j * nhl + hl) * D + f * 8);
-          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
+        const float w = ml[j].x * inv;
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x = __bfloat1622float2(hv[e]);
-            acc[2 * e] = fmaf(w, x.x, acc[2 * e]);
-            acc[2 * e + 1] = fmaf(w, x.y, acc[2 * e + 1]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = __bfloat1622float2(hv[e]);
+          acc[2 * e] = fmaf(w, x.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(w, x.y, acc[2 * e + 1]);
         }
       }
       if (rope && f * 8 >= D - kRopeDims) {          // inverse RoPE of the merged output

@@ -90,11 +90,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Orders earlier generic-proxy accesses of global memory with later async-proxy ones (a
-// bulk copy that reads what other threads stored).
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 // 2-D / 3-D TMA tile load into this CTA's shared memory, completion counted on
 // the mbarrier in bytes.  Plain loads only: no cluster multicast anywhere.
@@ -376,17 +371,6 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
-}
-
-// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to shared memory of
-// a CTA of the cluster (dst_cluster from cluster_map), completion counted in bytes on the
-// destination CTA's mbarrier (bar_cluster, from cluster_map).  A unicast shared-to-shared copy.
-__device__ __forceinline__ void bulk_s2cluster(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                               uint32_t bar_cluster) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dst_cluster),
-               "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-               : "memory");
 }
 
 // Maximum of x over the 32 lanes of the warp, returned to every lane.

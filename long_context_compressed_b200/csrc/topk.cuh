@@ -857,9 +857,15 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
       ck[u] = i < nc ? __ldcg(ckey + i) : 0u;
       ci[u] = i < nc ? __ldcg(cidx + i) : 0;
     }
+    // the fine histogram the chunks accumulated, requested with the first candidates
+    int4 gf[kHistBins / 4 / kSelThreads];
+#pragma unroll
+    for (int u = 0; u < kHistBins / 4 / kSelThreads; ++u)
+      gf[u] = __ldcg(reinterpret_cast<const int4*>(gfine) + threadIdx.x + u * kSelThreads);
     if (threadIdx.x == 0) {
       kext[0] = 0xffffffffu;
       kext[1] = 0u;
+      pcount = 0;
     }
     {
       int local = 0;
@@ -877,7 +883,25 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         off += ct[u].y;
       }
     }
+#pragma unroll
+    for (int u = 0; u < kHistBins / 4 / kSelThreads; ++u) {
+      const int h = 4 * (threadIdx.x + u * kSelThreads);
+      histk[skew(h)] = gf[u].x;
+      histk[skew(h + 1)] = gf[u].y;
+      histk[skew(h + 2)] = gf[u].z;
+      histk[skew(h + 3)] = gf[u].w;
+    }
     __syncthreads();
+    // The k-th key's bin of the fine histogram; if it is an inner bin holding at most
+    // kSelPivot keys, the staging pass below also collects that bin's keys (the pivots),
+    // which are then ranked directly instead of a radix select.
+    find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, k, res, scratch);
+    __syncthreads();
+    const int fstar = res[0], fabove = res[1];
+    const int fnb = histk[skew(fstar)];
+    const bool pivots = fstar > 0 && fstar < kHistBins - 1 && fnb <= kSelPivot;
+    uint32_t* piv = reinterpret_cast<uint32_t*>(tpre + kSelMaxChunks);   // [kSelPivot]
+    const uint32_t lane_below = (1u << lane_id()) - 1;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     const float inv_chunk = 1.f / (float)chunk;
     for (int i0 = 0;;) {
@@ -893,6 +917,14 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
           oidx[pos] = ci[u];
           kmin = min(kmin, ck[u]);
           kmax = max(kmax, ck[u]);
+        }
+        if (pivots) {                                     // one slot claim per warp
+          const bool m = i < nc && fine_bin(ck[u], fbase) == fstar;
+          const uint32_t bal = __ballot_sync(0xffffffffu, m);
+          int base = 0;
+          if (lane_id() == 0 && bal) base = atomicAdd(&pcount, __popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (m) piv[base + __popc(bal & lane_below)] = ck[u];
         }
       }
       i0 += U * kSelThreads;
@@ -915,60 +947,26 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     const uint32_t span = kext[1] - kmin;
     uint32_t prefix = 0, pmask = 0;
     int remaining = k;
-    // The k-th key's bin of the fine histogram the chunks accumulated; if it is an inner
-    // bin holding at most kSelPivot keys, rank those keys directly and skip the radix.
     bool located = false;
-    {
-      const int4* g4 = reinterpret_cast<const int4*>(gfine);
-#pragma unroll
-      for (int u = 0; u < kHistBins / 4 / kSelThreads; ++u) {
-        const int4 v = __ldcg(g4 + threadIdx.x + u * kSelThreads);
-        const int h = 4 * (threadIdx.x + u * kSelThreads);
-        histk[skew(h)] = v.x;
-        histk[skew(h + 1)] = v.y;
-        histk[skew(h + 2)] = v.z;
-        histk[skew(h + 3)] = v.w;
+    if (pivots) {
+      const int want = k - fabove;                         // keys of the pivot bin to take
+      if ((int)threadIdx.x < fnb) {
+        const uint32_t v = piv[threadIdx.x];
+        int gt = 0, ge = 0;
+        for (int j = 0; j < fnb; ++j) {
+          gt += piv[j] > v;
+          ge += piv[j] >= v;
+        }
+        if (gt < want && want <= ge) {                     // every key equal to K* writes the same
+          res[0] = (int)(v - kmin);
+          res[1] = gt;
+        }
       }
       __syncthreads();
-      find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, k, res, scratch);
-      __syncthreads();
-      const int fstar = res[0], above = res[1];
-      const int nb = histk[skew(fstar)];
-      if (fstar > 0 && fstar < kHistBins - 1 && nb <= kSelPivot) {
-        uint32_t* piv = reinterpret_cast<uint32_t*>(tpre + kSelMaxChunks);   // [kSelPivot]
-        if (threadIdx.x == 0) pcount = 0;
-        __syncthreads();
-        const uint32_t below = (1u << lane_id()) - 1;
-        for (int i0 = 0; i0 < nc; i0 += kSelThreads) {       // one slot claim per warp
-          const int i = i0 + threadIdx.x;
-          const uint32_t key = i < nc ? okey[i] : 0u;
-          const bool m = i < nc && fine_bin(key, fbase) == fstar;
-          const uint32_t bal = __ballot_sync(0xffffffffu, m);
-          int base = 0;
-          if (lane_id() == 0 && bal) base = atomicAdd(&pcount, __popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (m) piv[base + __popc(bal & below)] = key;
-        }
-        __syncthreads();
-        const int want = k - above;                          // keys of this bin to take
-        if ((int)threadIdx.x < nb) {
-          const uint32_t v = piv[threadIdx.x];
-          int gt = 0, ge = 0;
-          for (int j = 0; j < nb; ++j) {
-            gt += piv[j] > v;
-            ge += piv[j] >= v;
-          }
-          if (gt < want && want <= ge) {                     // every key equal to K* writes the same
-            res[0] = (int)(v - kmin);
-            res[1] = gt;
-          }
-        }
-        __syncthreads();
-        prefix = (uint32_t)res[0];
-        pmask = 0xffffffffu;
-        remaining = want - res[1];
-        located = true;
-      }
+      prefix = (uint32_t)res[0];
+      pmask = 0xffffffffu;
+      remaining = want - res[1];
+      located = true;
       __syncthreads();
     }
     // otherwise: radix select on u = key - kmin, 12-bit digits from the highest bit of the
