@@ -45,6 +45,10 @@ INDEX_ROTATION = True
 # compress_rope_theta): q turned and the output turned back inside the attention kernel, new
 # compressed entries turned when the step appends them.  Not applied to mixed-precision KV8 rows.
 ROPE_THETA = 160000.0
+# How a decode step's launches are laid out: "streams" puts the compressors and the HCA
+# layer on side streams beside the indexer -> select -> attention chain; "serial" issues
+# every launch on one stream.
+SCHEDULE = "streams"
 
 
 def oracle_quantizer():
@@ -353,6 +357,8 @@ class DecodeSet:
         wl = self.wl
         x = self.inputs
         main = torch.cuda.current_stream()
+        if SCHEDULE == "serial":
+            side_streams = (main,) * len(side_streams)
         if copies:
             self.in_buf.copy_(self.host_in, non_blocking=True)
         def side_branch():
@@ -1124,6 +1130,7 @@ def workload_text(wl, index, with_hca):
 
 # ----------------------------------------------------------------------------- main
 def main():
+    global SCHEDULE
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -1137,8 +1144,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", choices=STAGES + BIG_STAGES, help="time one stage alone (eager calls), e.g. under ncu")
     ap.add_argument("--kv8", action="store_true", help="with --stage: memory rows as mixed-precision KV8 entries")
+    ap.add_argument("--schedule", choices=["streams", "serial"], default=SCHEDULE,
+                    help="streams: compressors / HCA layer on side streams beside the indexer chain; "
+                         "serial: every launch of the step on one stream")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    SCHEDULE = args.schedule
     global INDEX_ROTATION
     INDEX_ROTATION = not args.no_hadamard
     rank, world, local = dist_env()

@@ -240,8 +240,8 @@ int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t 
  *   previous call left in it.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current and keeps it for later calls;
- *   make that first call before any stream capture, and do not use this entry
- *   point after cudaDeviceReset (the kept address would be stale).  All calls share
+ *   do not use this entry point after cudaDeviceReset (the kept address would be
+ *   stale).  All calls share
  *   the one array: calls that may overlap on the GPU (different streams, or work
  *   replayed concurrently) race on it and give wrong results -- order them on one
  *   stream.
