@@ -46,8 +46,9 @@ INDEX_ROTATION = True
 # compressed entries turned when the step appends them.  Not applied to mixed-precision KV8 rows.
 ROPE_THETA = 160000.0
 # How a decode step's launches are laid out: "streams" puts the compressors and the HCA
-# layer on side streams beside the indexer -> select -> attention chain; "serial" issues
-# every launch on one stream.
+# layer on side streams beside the indexer -> select -> attention chain, forked after the
+# indexer ("early": at the step's start, "late": after the select); "serial" issues every
+# launch on one stream.
 SCHEDULE = "streams"
 
 
@@ -421,13 +422,16 @@ class DecodeSet:
                 ev.record()
                 marks.append((name, ev))
         mark("start")
+        if SCHEDULE == "early":
+            side_branch()
         if self.index == "e4m3":
             csa.csa_quantize_e4m3(x["qI"], codes=self.q8, scale=self.qs, hadamard=INDEX_ROTATION)
             mark("quantize_q")
             csa.csa_index_scores(self.q8, x["w"], self.k8, self.n_valid, q_scale=self.qs, k_scale=self.ks,
                                  scores=self.scores, select_ws=self.select_ws)
             mark("index")
-            side_branch()
+            if SCHEDULE in ("streams", "serial"):
+                side_branch()
             # top-2k bin of the e4m3 scores, exact bf16 rescoring, best k -- one launch
             csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, kc=2 * wl.topk, qI=x["qI"],
                                 w=x["w"], kI=self.kI, idx=self.idx)
@@ -438,7 +442,8 @@ class DecodeSet:
             csa.csa_index_scores(self.q4, x["w"], self.k4, self.n_valid, q_scale=self.qsf, k_scale=self.ksf,
                                  scores=self.scores, select_ws=self.select_ws, mxfp4=True)
             mark("index")
-            side_branch()
+            if SCHEDULE in ("streams", "serial"):
+                side_branch()
             # top-4k bin of the FP4 scores, exact bf16 rescoring, best k -- one launch
             csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, kc=4 * wl.topk, qI=x["qI"],
                                 w=x["w"], kI=self.kI, idx=self.idx)
@@ -447,9 +452,12 @@ class DecodeSet:
             csa.csa_index_scores(x["qI"], x["w"], self.kI, self.n_valid, scores=self.scores,
                                  select_ws=self.select_ws)
             mark("index")
-            side_branch()
+            if SCHEDULE in ("streams", "serial"):
+                side_branch()
             csa.csa_topk_select(self.scores, self.n_valid, wl.topk, self.select_ws, idx=self.idx)
             mark("select")
+        if SCHEDULE == "late":
+            side_branch()
         append_index_keys()
         csa.sparse_attn(x["q"], self.kv_store, self.swa, self.swa_pos0, self.q_pos, self.sink, self.idx,
                         1.0 / math.sqrt(wl.D), rope_theta=self.theta, out=self.out, workspace=self.attn_ws)
@@ -663,9 +671,12 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     sets = [probe] + [DecodeSet(wl, s, index, with_hca, device, kv8=kv8) for s in range(1, n_sets)]
     side = [torch.cuda.Stream(device=device) for _ in range(3)]
     graphs, launches = capture(sets, side)
-    t = timed_replays(graphs, steps, warmup, world)           # one graph per step, sets in rotation
-    t = max_over_ranks(t, world, device)
+    # one graph per step, sets in rotation (reported beside the value)
+    t_single = max_over_ranks(timed_replays(graphs, steps, warmup, world), world, device)
     del graphs
+    # the value: one graph running a step on every input set in turn, as a serving loop
+    # runs steps back to back (no graph launch between consecutive steps)
+    t = max_over_ranks(timed_steps(sets, side, steps, warmup, world, copies=False), world, device)
     idx_ms = index_alone_ms(sets, index, device, replays=max(3, min(20, steps // 100)))
     attn_ms = attn_alone_ms(sets, device, replays=max(3, min(20, steps // 100)))
     # per-stage breakdown from a separate diagnostic graph with events between all stages
@@ -684,6 +695,7 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
     # outputs read back, inside every timed step
     # (the next step's input copy and the previous outputs' read overlap each step's compute)
     t_e2e = max_over_ranks(timed_steps(sets, side, steps, warmup, world, copies=True), world, device)
+    breakdown["one_graph_per_step_us"] = round(1e6 * t_single / steps, 2)
     assert csa.csa_poll_status() == csa.CSA_OK
     h2d, d2h = probe.per_step_io()
     res = {"wl": wl, "index": index, "with_hca": with_hca, "sets": n_sets, "seconds": t, "step_ms": 1e3 * t / steps, "launches": launches,
@@ -1144,8 +1156,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", choices=STAGES + BIG_STAGES, help="time one stage alone (eager calls), e.g. under ncu")
     ap.add_argument("--kv8", action="store_true", help="with --stage: memory rows as mixed-precision KV8 entries")
-    ap.add_argument("--schedule", choices=["streams", "serial"], default=SCHEDULE,
-                    help="streams: compressors / HCA layer on side streams beside the indexer chain; "
+    ap.add_argument("--schedule", choices=["streams", "early", "late", "serial"], default=SCHEDULE,
+                    help="streams: compressors / HCA layer on side streams, forked after the indexer; "
+                         "early / late: the same, forked at the step's start / after the select; "
                          "serial: every launch of the step on one stream")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -1284,6 +1297,8 @@ def main():
         "dtype": "bf16+e4m3" if args.index == "e4m3" else "bf16", "data": "synthetic",
         "config": {"workload": workload_text(wl, args.index, with_hca),
                    "l2": f"{m['input_sets']} rotating input sets, > 2x L2 touched between reuses",
+                   "graph": "one CUDA graph runs a step on every input set in turn, replayed; "
+                            "steps % sets more by a second graph",
                    "parallelism": f"replicas x{world}"},
         "e2e": m["e2e"], "roofline": m["roofline"], "roofline_indexer": m["roofline_indexer"],
         "step_roofline": m["step_roofline"],
