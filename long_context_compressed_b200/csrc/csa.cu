@@ -769,7 +769,7 @@ int csa_index_rerank(const void* qI, const float* w, const void* kI, int dtype, 
   if (rc != CSA_OK) return rc;
   const int smem = kc * 4;
   if (!set_smem(csa::topk_row_kernel, std::max(smem, 4))) return CSA_ERR_CUDA;
-  launch_k(csa::topk_row_kernel, (unsigned)((int64_t)B * T), 1024, smem, st, cand_scores, nullptr, kc, k, idx, cand);
+  launch_k(csa::topk_row_kernel, (unsigned)((int64_t)B * T), 1024, smem, st, cand_scores, nullptr, kc, k, idx, cand, 0);
   return launch_status();
 }
 
@@ -806,9 +806,12 @@ int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t 
   const int64_t rows = (int64_t)B * T;
   cudaStream_t st = as_stream(stream);
   if (!topk_long_path(B, T, N)) {
-    const int smem = (int)std::max<int64_t>(4, std::min<int64_t>(N, csa::kRowSmemMax) * 4);
+    // keys, then (rows of kRowFastMin or more) the sampled path's candidates
+    const int smem = (int)std::max<int64_t>(4, std::min<int64_t>(N, csa::kRowSmemMax) * 4) +
+                     (N >= csa::kRowFastMin ? csa::kRowCand * 8 : 0);
     if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
-    launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, smem, st, scores, n_valid, N, k, idx, nullptr);
+    launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, smem, st, scores, n_valid, N, k, idx, nullptr,
+             N >= csa::kRowFastMin ? 1 : 0);
     return launch_status();
   }
   const size_t need = csa_topk_workspace_size(B, T, N, k);
@@ -857,7 +860,7 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
   const size_t need = csa_select_workspace_size(B, N);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSA_ERR_INVALID;
   if (N == 0) {
-    launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr);
+    launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr, 0);
     return launch_status();
   }
   // chunks: one wave (at most one CTA per SM over all rows), at least 512 entries each,
@@ -1054,7 +1057,7 @@ int csa_shard_select(const void* pairs, int G, int B, int k, int32_t* idx, void*
   const int smem = (int)std::max<int64_t>(4, n * 4);
   if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
   launch_k(csa::topk_row_kernel, (unsigned)B, 1024, smem, st, (const float*)row_scores, (const int32_t*)nullptr, n, k,
-           idx, (const int32_t*)row_idx);
+           idx, (const int32_t*)row_idx, 0);
   return launch_status();
 }
 

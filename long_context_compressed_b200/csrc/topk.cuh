@@ -28,6 +28,8 @@
 namespace csa {
 
 constexpr int kRowSmemMax = 32768;
+constexpr int kRowFastMin = 8192;               // rows this long try the sampled threshold first
+constexpr int kRowCand = 8192;                  // candidates of that path (shared memory)
 constexpr int kHistBits = 12;
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kChunk = 4096;
@@ -201,16 +203,19 @@ __device__ __forceinline__ void write_all_valid(int32_t* out, int nv, int k) {
 // n_valid may be null (every row has N valid entries); map may be null, else the
 // output holds map[row, position] instead of the position (used to return the
 // original indices of a rescored candidate list; map rows must be ascending so
-// that the output stays ascending).
+// that the output stays ascending).  cand_smem: the dynamic shared memory also holds
+// kRowCand candidate keys and indices after the row's keys (rows of kRowFastMin or more
+// then try the sampled threshold first).
 __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict__ scores,
                                                         const int32_t* __restrict__ n_valid, int64_t N, int k,
                                                         int32_t* __restrict__ idx,
-                                                        const int32_t* __restrict__ map) {
+                                                        const int32_t* __restrict__ map, int cand_smem) {
   griddep_sync();
-  extern __shared__ __align__(16) uint32_t keys[];  // [min(N, kRowSmemMax)]
+  extern __shared__ __align__(16) uint32_t keys[];  // [min(N, kRowSmemMax)], then (long rows) the candidates
   __shared__ __align__(16) int rhist[kHistBins + kHistBins / 32];   // skewed
   __shared__ int scratch[33];
   __shared__ int res[2];
+  __shared__ uint32_t ext[2];
   const int64_t row = blockIdx.x;
   int nv = n_valid ? n_valid[row] : (int)N;
   nv = nv < 0 ? 0 : (nv > (int)N ? (int)N : nv);
@@ -235,6 +240,98 @@ __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict_
       const int i = u * 1024 + (int)threadIdx.x;
       if (i < nv) keys[i] = order_key(v[u]);
     }
+  }
+  // ---- long rows: a strided sample of 1024 keys places a threshold t (the lower edge of the
+  // sample-histogram bin that holds the sample's 2k*1024/nv-th key, plus a margin) whose count
+  // over the row usually lies in [k, kRowCand].  Then only the keys >= t, compacted in index
+  // order, enter the radix select, over their own key span (the tail of a row spreads over
+  // the histogram instead of piling into the few bins the row's bulk falls in).  Otherwise
+  // the full radix below runs.
+  if (cand_smem && nv >= kRowFastMin && blockDim.x == 1024) {
+    uint32_t* ckey = keys + (N < kRowSmemMax ? N : kRowSmemMax);
+    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kRowCand);
+    const int stride = nv / 1024;
+    const uint32_t sk = keys[threadIdx.x * stride];
+    for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) rhist[j] = 0;
+    if (threadIdx.x == 0) {
+      ext[0] = 0xffffffffu;
+      ext[1] = 0u;
+    }
+    const uint32_t wmin = __reduce_min_sync(0xffffffffu, sk), wmax = __reduce_max_sync(0xffffffffu, sk);
+    __syncthreads();
+    if (lane_id() == 0) {
+      atomicMin(&ext[0], wmin);
+      atomicMax(&ext[1], wmax);
+    }
+    __syncthreads();
+    const uint32_t smin = ext[0];
+    const uint32_t sspan = ext[1] - smin;
+    const int sbits = sspan ? 32 - __clz(sspan) : 0;
+    const int sh = sbits > kHistBits ? sbits - kHistBits : 0;
+    atomicAdd(&rhist[skew((int)((sk - smin) >> sh))], 1);
+    __syncthreads();
+    const int64_t want64 = 2 * (int64_t)k * 1024 / nv + 16;
+    const int want = want64 < 1024 ? (int)want64 : 1024;
+    find_digit_skewed<kHistBins / 1024>(rhist, kHistBins, want, res, scratch);
+    __syncthreads();
+    const uint32_t t = smin + ((uint32_t)res[0] << sh);
+    // the row's keys >= t, counted and then compacted over contiguous index ranges
+    const int per = ((nv + 1023) / 1024) | 1;
+    const int lo = min((int)threadIdx.x * per, nv), hi = min(lo + per, nv);
+    int c = 0;
+    uint32_t cmax = 0u;
+    for (int i = lo; i < hi; ++i) {
+      const uint32_t key = keys[i];
+      c += key >= t;
+      cmax = max(cmax, key);
+    }
+    int C;
+    const int off = block_excl_scan(c, scratch, &C);
+    if (C >= k && C <= kRowCand) {                       // the whole block takes the same branch
+      int o = off;
+      for (int i = lo; i < hi; ++i) {
+        const uint32_t key = keys[i];
+        if (key >= t) {
+          ckey[o] = key;
+          cidx[o] = i;
+          ++o;
+        }
+      }
+      cmax = __reduce_max_sync(0xffffffffu, cmax);
+      if (lane_id() == 0) atomicMax(&ext[1], cmax);       // ext[1] already holds the sample max
+      __syncthreads();
+      const uint32_t cspan = ext[1] - t;
+      uint32_t prefix = 0, pmask = 0;
+      int remaining = k;
+      for (int hb = cspan ? 32 - __clz(cspan) : 0; hb > 0;) {
+        const int lb = hb > kHistBits ? hb - kHistBits : 0;
+        const uint32_t dmask = (1u << (hb - lb)) - 1;
+        for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) rhist[j] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {
+          const uint32_t u = ckey[i] - t;
+          if ((u & pmask) == prefix) atomicAdd(&rhist[skew((int)((u >> lb) & dmask))], 1);
+        }
+        __syncthreads();
+        find_digit_skewed<kHistBins / 1024>(rhist, kHistBins, remaining, res, scratch);
+        __syncthreads();
+        prefix |= (uint32_t)res[0] << lb;
+        pmask |= dmask << lb;
+        remaining -= res[1];
+        hb = lb;
+        __syncthreads();
+      }
+      const int cper = ((C + 1023) / 1024) | 1;
+      const int clo = min((int)threadIdx.x * cper, C), chi = min(clo + cper, C);
+      write_selection(clo, chi, [&](int64_t i) { return ckey[i]; }, t + prefix, remaining, out, scratch);
+      __syncthreads();
+      for (int j = threadIdx.x; j < k; j += blockDim.x) {
+        const int32_t ci = cidx[out[j]];
+        out[j] = mrow ? mrow[ci] : ci;
+      }
+      return;
+    }
+    __syncthreads();
   }
   // radix select with digits of 12, 10 and 10 bits on a skewed histogram
   uint32_t prefix = 0, pmask = 0;

@@ -66,6 +66,24 @@ def test_topk_all_equal_and_signed_zero(csa, N):
     assert g[0, 1].tolist() == list(range(k))
 
 
+def test_topk_row_sampled_threshold_and_its_fallbacks(csa):
+    """Rows of 8,192..32,768 scores try a threshold placed by a strided sample of 1,024
+    keys first.  Rows where that cannot work must fall back to the full radix: every score
+    equal (the count above the threshold exceeds the candidate space), and a row whose
+    sampled positions hold its largest values (too few keys reach the threshold).  Plus a
+    plain row and a heavy-tailed one; all bit for bit against the oracle."""
+    B, T, N, k = 1, 4, 20000, 512
+    s = synth.draw_scores(13, "topk/sampled", B, T, N, ties=4)
+    s[0, 0] = 7.5                                            # all equal
+    stride = N // 1024
+    s[0, 1] = synth.normal(13, "topk/sampled/small", (N,))
+    s[0, 1, 0:1024 * stride:stride] = 1000.0 + torch.arange(1024, dtype=torch.float32)
+    s[0, 3] = torch.exp(4 * synth.normal(13, "topk/sampled/tail", (N,)))   # heavy tail
+    nv = np.array([[N, N, N - 3, N]], np.int32)
+    g = _run(csa, s, nv, k)
+    assert g[0, 0].tolist() == list(range(k))
+
+
 def test_topk_workloads_chunk_and_row_paths_agree(csa):
     """The same rows through both paths (as one batch of many rows and as few rows)."""
     N, k = 16384, 512
