@@ -989,16 +989,15 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
       histk[skew(h + 3)] = gf[u].w;
     }
     __syncthreads();
-    // The k-th key's bin of the fine histogram; if it is an inner bin holding at most
-    // kSelPivot keys, the staging pass below also collects that bin's keys (the pivots),
-    // which are then ranked directly instead of a radix select.
+    // The k-th key's bin of the fine histogram (bins of 2^12 keys).  If it is an inner bin,
+    // the staging pass below also histograms the low 12 bits of that bin's keys, which
+    // gives the k-th key itself; an edge bin (keys clamped into it) takes the radix select.
     find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, k, res, scratch);
     __syncthreads();
     const int fstar = res[0], fabove = res[1];
-    const int fnb = histk[skew(fstar)];
-    const bool pivots = fstar > 0 && fstar < kHistBins - 1 && fnb <= kSelPivot;
-    uint32_t* piv = reinterpret_cast<uint32_t*>(tpre + kSelMaxChunks);   // [kSelPivot]
-    const uint32_t lane_below = (1u << lane_id()) - 1;
+    const bool pivots = fstar > 0 && fstar < kHistBins - 1;
+    for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) histk[j] = 0;
+    __syncthreads();
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     const float inv_chunk = 1.f / (float)chunk;
     for (int i0 = 0;;) {
@@ -1015,14 +1014,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
           kmin = min(kmin, ck[u]);
           kmax = max(kmax, ck[u]);
         }
-        if (pivots) {                                     // one slot claim per warp
-          const bool m = i < nc && fine_bin(ck[u], fbase) == fstar;
-          const uint32_t bal = __ballot_sync(0xffffffffu, m);
-          int base = 0;
-          if (lane_id() == 0 && bal) base = atomicAdd(&pcount, __popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (m) piv[base + __popc(bal & lane_below)] = ck[u];
-        }
+        if (pivots && i < nc && fine_bin(ck[u], fbase) == fstar)
+          atomicAdd(&histk[skew((int)((ck[u] - fbase) & (kHistBins - 1)))], 1);
       }
       i0 += U * kSelThreads;
       if (i0 >= nc) break;
@@ -1046,21 +1039,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     int remaining = k;
     bool located = false;
     if (pivots) {
-      const int want = k - fabove;                         // keys of the pivot bin to take
-      if ((int)threadIdx.x < fnb) {
-        const uint32_t v = piv[threadIdx.x];
-        int gt = 0, ge = 0;
-        for (int j = 0; j < fnb; ++j) {
-          gt += piv[j] > v;
-          ge += piv[j] >= v;
-        }
-        if (gt < want && want <= ge) {                     // every key equal to K* writes the same
-          res[0] = (int)(v - kmin);
-          res[1] = gt;
-        }
-      }
+      const int want = k - fabove;                         // keys of the k-th key's bin to take
+      find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, want, res, scratch);
       __syncthreads();
-      prefix = (uint32_t)res[0];
+      prefix = fbase + ((uint32_t)fstar << 12) + (uint32_t)res[0] - kmin;   // K* - kmin
       pmask = 0xffffffffu;
       remaining = want - res[1];
       located = true;
