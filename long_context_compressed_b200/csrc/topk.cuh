@@ -595,6 +595,7 @@ constexpr int kSelPrefetch = 2048;   // chunk entries whose scores are fetched w
 constexpr int kSelMaxChunkLen = 16384;  // entries per chunk (shared-memory candidate list)
 static_assert(kSelPerThread * (kSelThreads / 32) == 32, "one scan lane per (pass, warp)");
 static_assert(kSelMaxChunks % kSelThreads == 0, "chunk table split evenly over the threads");
+static_assert(2 * kSelMaxChunks >= CSA_MAX_TOPK, "the last CTA stages k indices in the chunk table's space");
 constexpr int64_t kSelMaxN = int64_t(1) << 19;
 constexpr int kSelTileBytes = 2 * kSelTcRows * 128;    // candidate key tile, 2 x 128-byte K atoms (bf16)
 constexpr int kSelQBytes = 2 * 64 * 128;               // q tile: 64 heads x 128 dims bf16
@@ -1141,6 +1142,9 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     int total;
     const int ex = block_excl_scan((cg << 16) | ce, scratch, &total);
     int g = ex >> 16, e = ex & 0xffff;
+    // the k indices land in shared memory first (the chunk table's space, free now), then
+    // go out as coalesced 16-byte stores
+    int32_t* sout = tslot;                                 // [k]; kSelMaxChunks * 2 >= CSA_MAX_TOPK
     for (int i0 = p0; i0 < p1; i0 += 4) {
       uint32_t uu[4];
       int32_t ii[4];
@@ -1154,13 +1158,20 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         if (i0 + q >= p1) break;
         if (uu[q] > prefix) {
           const int o = g + (e < remaining ? e : remaining);
-          if (o < k) out[o] = ii[q];                       // (bound holds unless the histogram is stale)
+          if (o < k) sout[o] = ii[q];                      // (bound holds unless the histogram is stale)
           ++g;
         } else if (uu[q] == prefix) {
-          if (e < remaining && g + e < k) out[g + e] = ii[q];
+          if (e < remaining && g + e < k) sout[g + e] = ii[q];
           ++e;
         }
       }
+    }
+    __syncthreads();
+    if ((k & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) {
+      for (int j = threadIdx.x; j < k / 4; j += blockDim.x)
+        reinterpret_cast<int4*>(out)[j] = reinterpret_cast<const int4*>(sout)[j];
+    } else {
+      for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = sout[j];
     }
     __syncthreads();
   } else {
