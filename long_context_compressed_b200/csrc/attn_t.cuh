@@ -19,7 +19,8 @@
 // of D across CTAs.
 //
 // CTA = (split of the row list, group of 64 heads, query).  Rows arrive in units of 64
-// (one shared-memory stage each, two stages): gathered rows by cp.async (16-byte pieces),
+// (one shared-memory stage each, two stages; the softmax warps load unit 1 beside the
+// loader warps' unit 0): gathered rows by cp.async (16-byte pieces),
 // 64 consecutive rows of one buffer (SWA rows, hca_attn's memory rows) by eight TMA boxes
 // of 8 rows.  A stage is stored as eight 8-row groups, each group holding its rows' D/64
 // 128-byte-swizzled atoms: two adjacent stages are then one 128-row operand, so a CTA with
@@ -181,6 +182,84 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     return ((int64_t)b * p.N + i) * D;
   };
 
+  // One unit's rows into its stage by 128 threads (lt = 0..127): warp w of the group fills
+  // rows 16w .. 16w+15, four rows per pass: lane l copies 16-byte chunk l % 8 of every
+  // 128-byte atom of row 4 * pass + l / 8, so one cp.async of the warp reads four whole
+  // 128-byte lines.  A unit of 64 consecutive rows of one buffer goes by eight TMA boxes
+  // instead.  Arrives 128 + 4 times on full[s] (the copies of every thread, one validity
+  // word per warp).
+  const bool staged_idx = p.sparse && nu * U <= Cfg::kMaxCtaRows;
+  auto load_unit = [&](int u, int lt, bool use_staged) -> bool {
+    const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(p.kv);
+    const __nv_bfloat16* swa = static_cast<const __nv_bfloat16*>(p.swa);
+    const int wl = lt >> 5, lane = (int)lane_id();
+    const int sub = lane >> 3, c8 = lane & 7;
+    const int s = u & 1;
+    const uint32_t ph = (u >> 1) & 1;
+    if (!mbar_wait(&empty[s], ph ^ 1)) return false;
+    uint8_t* stage = kv_s + s * Cfg::kStage;
+    const int rg0 = row0 + u * U;
+    const bool swa_tile = p.has_swamap && rg0 + U <= rl.n_swa;
+    const bool mem_tile = p.has_kvmap && !p.sparse && rg0 >= mem0 && rg0 + U <= n_rows;
+    uint32_t rows = 0xFFFFu;                      // validity of this warp's 16 rows
+    if (swa_tile || mem_tile) {
+      // eight boxes of {64 dims, 8 rows, all atoms}: each lands as one 8-row group
+      if (lt < 32) {
+        if (lt == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kStage);
+        __syncwarp();
+        if (lt < 8) {
+          const int y = swa_tile ? (int)rl.swa_row0 + rg0 + 8 * lt : rg0 - mem0 + 8 * lt;
+          tma_load_4d(stage + lt * Cfg::kGroup, swa_tile ? &swamap : &kvmap, &full[s], 0, y, 0, b);
+        }
+        if (lt != 0) mbar_arrive(&full[s]);
+      } else {
+        mbar_arrive(&full[s]);
+      }
+    } else {
+      const __nv_bfloat16* src[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = 16 * wl + 4 * j + sub;
+        const int rg = rg0 + r;
+        int32_t raw = 0;
+        if (p.sparse && rg >= mem0 && rg < n_rows)
+          raw = use_staged ? idx_s[u * U + r] : __ldg(idx_row + (rg - mem0));
+        const int64_t so = row_src(rg, raw);
+        src[j] = so >= 0 ? kv + so : (so <= -2 ? swa + (-2 - so) : nullptr);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = 16 * wl + 4 * j + sub;
+#pragma unroll
+        for (int a = 0; a < Cfg::kAtoms; ++a) {
+          const int ch = a * 8 + c8;
+          uint8_t* dst = stage + st_off<D>(r, ch);
+          if (src[j]) cp_async_16(dst, src[j] + ch * 8);
+          else st_shared_zero16(dst);             // finite filler for rows that do not contribute
+        }
+      }
+      fence_proxy_async_smem();
+      cp_async_arrive_noinc(&full[s]);
+      rows = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, src[j] != nullptr);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) rows |= ((bal >> (8 * q)) & 1u) << (4 * j + q);
+      }
+    }
+    // row validity, one word per warp of the group (16 rows)
+    if (lane == 0) {
+      mask_s[s * 4 + wl] = rows;
+      mbar_arrive(&full[s]);
+    }
+    return true;
+  };
+  // With two or more units the softmax warps, idle until the first S^T lands, fill stage 1
+  // (unit 1) while the loader warps fill stage 0: the first two units' copies are issued
+  // by 256 threads at once.
+  const bool helped = nu >= 2;
+
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ loaders (128 threads)
     const int lt = threadIdx.x - 128;
@@ -189,82 +268,16 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       if (p.has_swamap) prefetch_tmap(&swamap);
     }
     if (nu > 0) {
-      const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(p.kv);
-      const __nv_bfloat16* swa = static_cast<const __nv_bfloat16*>(p.swa);
-      // warp w fills rows 16w .. 16w+15 of a unit, four rows per pass: lane l copies 16-byte
-      // chunk l % 8 of every 128-byte atom of row 4 * pass + l / 8, so one cp.async of the
-      // warp reads four whole 128-byte lines
-      const int wl = lt >> 5, lane = (int)lane_id();
-      const int sub = lane >> 3, c8 = lane & 7;
-      const int nrow = nu * U;
-      const bool staged_idx = p.sparse && nrow <= Cfg::kMaxCtaRows;
       if (staged_idx) {
-        for (int r = lt; r < nrow; r += 128) {
+        for (int r = lt; r < nu * U; r += 128) {
           const int rg = row0 + r;
           idx_s[r] = (rg >= mem0 && rg < n_rows) ? __ldg(idx_row + (rg - mem0)) : 0;
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
       for (int u = 0; u < nu; ++u) {
-        const int s = u & 1;
-        const uint32_t ph = (u >> 1) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        uint8_t* stage = kv_s + s * Cfg::kStage;
-        const int rg0 = row0 + u * U;
-        const bool swa_tile = p.has_swamap && rg0 + U <= rl.n_swa;
-        const bool mem_tile = p.has_kvmap && !p.sparse && rg0 >= mem0 && rg0 + U <= n_rows;
-        uint32_t rows = 0xFFFFu;                  // validity of this warp's 16 rows
-        if (swa_tile || mem_tile) {
-          // eight boxes of {64 dims, 8 rows, all atoms}: each lands as one 8-row group
-          if (lt < 32) {
-            if (lt == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)Cfg::kStage);
-            __syncwarp();
-            if (lt < 8) {
-              const int y = swa_tile ? (int)rl.swa_row0 + rg0 + 8 * lt : rg0 - mem0 + 8 * lt;
-              tma_load_4d(stage + lt * Cfg::kGroup, swa_tile ? &swamap : &kvmap, &full[s], 0, y, 0, b);
-            }
-            if (lt != 0) mbar_arrive(&full[s]);
-          } else {
-            mbar_arrive(&full[s]);
-          }
-        } else {
-          const __nv_bfloat16* src[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = 16 * wl + 4 * j + sub;
-            const int rg = rg0 + r;
-            int32_t raw = 0;
-            if (p.sparse && rg >= mem0 && rg < n_rows)
-              raw = staged_idx ? idx_s[u * U + r] : __ldg(idx_row + (rg - mem0));
-            const int64_t so = row_src(rg, raw);
-            src[j] = so >= 0 ? kv + so : (so <= -2 ? swa + (-2 - so) : nullptr);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = 16 * wl + 4 * j + sub;
-#pragma unroll
-            for (int a = 0; a < Cfg::kAtoms; ++a) {
-              const int ch = a * 8 + c8;
-              uint8_t* dst = stage + st_off<D>(r, ch);
-              if (src[j]) cp_async_16(dst, src[j] + ch * 8);
-              else st_shared_zero16(dst);         // finite filler for rows that do not contribute
-            }
-          }
-          fence_proxy_async_smem();
-          cp_async_arrive_noinc(&full[s]);
-          rows = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t bal = __ballot_sync(0xffffffffu, src[j] != nullptr);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) rows |= ((bal >> (8 * q)) & 1u) << (4 * j + q);
-          }
-        }
-        // row validity, one word per loader warp (16 rows)
-        if (lane == 0) {
-          mask_s[s * 4 + wl] = rows;
-          mbar_arrive(&full[s]);
-        }
+        if (u == 1 && helped) continue;           // the softmax warps' unit
+        if (!load_unit(u, lt, staged_idx)) break;
       }
       cp_async_wait_group<0>();                   // none may land after the CTA has left
     }
@@ -339,6 +352,7 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
     __syncwarp();                                  // the warp is converged again before the cluster barriers
   } else if (warp < 4) {
     // ------------------------------------------------------------ softmax (warps 0..3, TMEM lane = row)
+    if (helped) load_unit(1, threadIdx.x, false);  // unit 1 into stage 1 (its index values read directly)
     const int r = threadIdx.x;                   // row of the 128-row operand
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const bool owner = r < HG;                   // owner of head h0 + r's running statistics
@@ -467,6 +481,7 @@ __global__ void __launch_bounds__(288, 1) attn_t_kernel(const __grid_constant__ 
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&pfull[sb]);
     }
+    if (helped) cp_async_wait_group<0>();         // (unit 1's copies landed before its S^T was issued)
     const bool have_o = ok && ntiles > 0 && mbar_wait(odone, 0);
     // the per-head sum of P over every unit (the same in every TMEM lane): head r from lane r
     float l_run = 0.f;
