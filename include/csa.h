@@ -279,6 +279,11 @@ int csa_index_rerank(const void *qI, const float *w, const void *kI, int dtype, 
  *                full-precision qI [B, 64, 128] / kI [B, N, 128] (dtype F32 or BF16)
  *                and w [B, 64], and idx = the k best rescored candidates.
  *   Ties go to the lower index; rows are ascending and -1 padded (n_valid < k).
+ *   idx_scores : NULL, or [B, k] fp32 (caller-owned): beside each idx entry the score
+ *               that ranked it -- the rescored exact score when qI != NULL, else the
+ *               input score -- and -inf beside a -1 pad.  With qI != NULL a row of
+ *               0 < n_valid <= k entries is then rescored too (every entry is taken).
+ *               The sharded decode packs these scores for its all-gather.
  *   k <= CSA_MAX_TOPK, k <= kc, N <= 2^19.
  *   workspace : csa_select_workspace_size(B, N) bytes, 16-byte aligned, ZERO-FILLED
  *               before first use; csa_index_scores(..., workspace) fills the
@@ -292,8 +297,8 @@ size_t csa_select_workspace_size(int B, int64_t N);
 int csa_score_histogram(const float *scores, const int32_t *n_valid, int B, int64_t N, void *workspace,
                         size_t ws_bytes, void *stream);
 int csa_topk_select(const float *scores, const int32_t *n_valid, int B, int64_t N, int k, int kc, const void *qI,
-                    const float *w, const void *kI, int dtype, int32_t *idx, void *workspace, size_t ws_bytes,
-                    void *stream);
+                    const float *w, const void *kI, int dtype, int32_t *idx, float *idx_scores, void *workspace,
+                    size_t ws_bytes, void *stream);
 
 /*
  * csa_quantize_kv8 -- mixed-precision storage of compressed KV entries ([HA] §4.2,
@@ -395,8 +400,8 @@ int hca_attn_rope(const void *q, const void *kv, const void *swa_kv, const int64
 /*
  * Sharded decode of one long sequence over G GPUs (the compressed entries split into
  * G contiguous ranges, one per GPU).  Per step, on every GPU g owning entries [lo, hi):
- *   1. csa_index_scores + top-k over the local entries (local indices), the exact
- *      scores of the local winners (csa_index_rerank's cand_scores), and csa_shard_pack
+ *   1. csa_index_scores + csa_topk_select over the local entries (local indices, with
+ *      the exact rescored scores of the local winners in idx_scores), and csa_shard_pack
  *      -> (score, global index) pairs;
  *   2. one all-gather of the pairs, shard-major [G][B][k]; csa_shard_select -> the
  *      global top-k, the same on every GPU;

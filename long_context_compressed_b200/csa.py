@@ -45,7 +45,7 @@ _SIGS = {
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
     "csa_select_workspace_size": ([_i32, _i64], _sz),
     "csa_score_histogram": ([_vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
-    "csa_topk_select": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp], _i32),
+    "csa_topk_select": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "csa_topk_noalloc": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp], _i32),
     "csa_index_rerank": ([_vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp], _i32),
     "csa_topk_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
@@ -240,17 +240,19 @@ def csa_score_histogram(scores, n_valid, workspace, stream=None):
 
 
 def csa_topk_select(scores, n_valid, k: int, workspace, *, kc=None, qI=None, w=None, kI=None, idx=None,
-                    stream=None):
+                    idx_scores=None, stream=None):
     """Decode top-k from the histogram csa_index_scores(select_ws=workspace) accumulated.
     scores [B, 1, N] (or [B, N]), n_valid [B, 1] -> idx [B, 1, k].  With qI/w/kI (full precision)
-    the candidates of the kc-th score's bin are rescored exactly and the best k kept."""
+    the candidates of the kc-th score's bin are rescored exactly and the best k kept.
+    idx_scores (optional, fp32 with idx's shape) receives the score that ranked each entry."""
     B, N = scores.shape[0], scores.shape[-1]
     if idx is None:
         idx = torch.empty((B, 1, k), dtype=torch.int32, device=scores.device)
     kc = k if kc is None else kc
     dt = _dtype_code(qI) if qI is not None else CSA_F32
     _check(_lib.csa_topk_select(_ptr(scores), _ptr(n_valid), B, N, k, kc, _ptr(qI), _ptr(w), _ptr(kI), dt, _ptr(idx),
-                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+                                _ptr(idx_scores), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream)),
            "csa_topk_select")
     return idx
 

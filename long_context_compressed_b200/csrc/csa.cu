@@ -848,8 +848,8 @@ int csa_score_histogram(const float* scores, const int32_t* n_valid, int B, int6
 }
 
 int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t N, int k, int kc, const void* qI,
-                    const float* w, const void* kI, int dtype, int32_t* idx, void* workspace, size_t ws_bytes,
-                    void* stream) {
+                    const float* w, const void* kI, int dtype, int32_t* idx, float* idx_scores, void* workspace,
+                    size_t ws_bytes, void* stream) {
   if (B < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
   if (N > csa::kSelMaxN || B > 65535) return CSA_ERR_UNSUPPORTED;
   const bool rescore = qI != nullptr;
@@ -861,6 +861,9 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSA_ERR_INVALID;
   if (N == 0) {
     launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr, 0);
+    if (idx_scores)
+      launch_k(csa::fill_f32_kernel, (unsigned)std::min<int64_t>(((int64_t)B * k + 255) / 256, 1024), 256, 0,
+               as_stream(stream), idx_scores, (int64_t)B * k, -INFINITY);
     return launch_status();
   }
   // chunks: one wave (at most one CTA per SM over all rows), at least 512 entries each,
@@ -877,7 +880,7 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
   // last CTA: staged candidates + chunk table, or (overflow) the bucketed selection
   const int phase4 = (int)std::max<int64_t>(2 * csa::kSelCandSmem * 4 + 2 * csa::kSelMaxChunks * 4 +
                                                 csa::kSelPivot * 4,
-                                            2 * CSA_MAX_TOPK * 4 + (nchunks + 1) * 4);
+                                            4 * CSA_MAX_TOPK * 4 + (nchunks + 1) * 4);
   const int smem = 1024 + std::max(phase3, phase4);
   cudaStream_t st = as_stream(stream);
   dim3 grid((unsigned)nchunks, (unsigned)B);
@@ -885,15 +888,15 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
   if (!rescore) {
     if (!set_smem(csa::topk_select_kernel<false, float>, smem)) return CSA_ERR_CUDA;
     launch_k(csa::topk_select_kernel<false, float>, grid, csa::kSelThreads, smem, st, scores, n_valid, N, k, k,
-             chunk, (const float*)nullptr, w, (const float*)nullptr, idx, ws);
+             chunk, (const float*)nullptr, w, (const float*)nullptr, idx, idx_scores, ws);
   } else if (dtype == CSA_BF16) {
     if (!set_smem(csa::topk_select_kernel<true, __nv_bfloat16>, smem)) return CSA_ERR_CUDA;
     launch_k(csa::topk_select_kernel<true, __nv_bfloat16>, grid, csa::kSelThreads, smem, st, scores, n_valid, N,
-             k, kc, chunk, (const __nv_bfloat16*)qI, w, (const __nv_bfloat16*)kI, idx, ws);
+             k, kc, chunk, (const __nv_bfloat16*)qI, w, (const __nv_bfloat16*)kI, idx, idx_scores, ws);
   } else {
     if (!set_smem(csa::topk_select_kernel<true, float>, smem)) return CSA_ERR_CUDA;
     launch_k(csa::topk_select_kernel<true, float>, grid, csa::kSelThreads, smem, st, scores, n_valid, N, k, kc,
-             chunk, (const float*)qI, w, (const float*)kI, idx, ws);
+             chunk, (const float*)qI, w, (const float*)kI, idx, idx_scores, ws);
   }
   return launch_status();
 }

@@ -41,6 +41,11 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float an order key came from (-0.0 comes back as +0.0).
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 // Inclusive warp scan.
 __device__ __forceinline__ int warp_incl_scan(int v) {
 #pragma unroll
@@ -197,6 +202,10 @@ __device__ __forceinline__ void write_selection(int64_t lo, int64_t hi, GetKey g
 
 __device__ __forceinline__ void write_all_valid(int32_t* out, int nv, int k) {
   for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < nv ? j : -1;
+}
+
+__global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) p[i] = v;
 }
 
 // ---------------------------------------------------------------- row kernel
@@ -626,6 +635,10 @@ __device__ __forceinline__ void unpack_vec<float>(uint4 v, float* f) {  // 4 fp3
 // exact top-k of the (re)scored candidates, lower index first among equal scores, is
 // written in ascending index order by the last CTA of the row (chunks are contiguous
 // index ranges: the k indices are bucketed by chunk and ranked inside their bucket).
+// sel_scores (may be null) receives, beside each index, the score that ranked it: the
+// rescored one with RESCORE, else the input score; -inf beside a -1 pad.  With RESCORE
+// and sel_scores, a row of n_valid <= k entries is rescored too (all its entries are
+// candidates, and the last CTA takes them all).
 template <bool RESCORE, typename Tin>
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* __restrict__ scores,
                                                                   const int32_t* __restrict__ n_valid, int64_t N,
@@ -633,6 +646,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
                                                                   const Tin* __restrict__ qI,
                                                                   const float* __restrict__ w,
                                                                   const Tin* __restrict__ kI, int32_t* __restrict__ idx,
+                                                                  float* __restrict__ sel_scores,
                                                                   uint8_t* __restrict__ ws) {
   constexpr bool TC = RESCORE && sizeof(Tin) == 2;
   extern __shared__ __align__(1024) uint8_t sel_raw[];
@@ -672,10 +686,13 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
   uint32_t* ckey = reinterpret_cast<uint32_t*>(rws + SelectWs::kHeaderInts * 4);
   int32_t* cidx = reinterpret_cast<int32_t*>(ckey + N);
   int32_t* out = idx + row * k;
-  const bool all_valid = nv <= k;
+  float* oscore = sel_scores ? sel_scores + row * k : nullptr;
+  const bool all_valid = nv <= k && !(RESCORE && oscore && nv > 0);
   const bool active = !all_valid && (int64_t)blockIdx.x * chunk < nv;
   if (all_valid && blockIdx.x == 0) {
     write_all_valid(out, nv, k);
+    if (oscore)
+      for (int j = threadIdx.x; j < k; j += blockDim.x) oscore[j] = j < nv ? scores[row * N + j] : -INFINITY;
     for (int j = threadIdx.x; j < kHistBins; j += blockDim.x) ghist[j] = 0;
   }
   int nloc = 0;
@@ -993,9 +1010,15 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     // The k-th key's bin of the fine histogram (bins of 2^12 keys).  If it is an inner bin,
     // the staging pass below also histograms the low 12 bits of that bin's keys, which
     // gives the k-th key itself; an edge bin (keys clamped into it) takes the radix select.
-    find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, k, res, scratch);
-    __syncthreads();
-    const int fstar = res[0], fabove = res[1];
+    // No more candidates than k: every one is taken.
+    const bool take_all = nc <= k;
+    int fstar = 0, fabove = 0;
+    if (!take_all) {
+      find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, k, res, scratch);
+      __syncthreads();
+      fstar = res[0];
+      fabove = res[1];
+    }
     const bool pivots = fstar > 0 && fstar < kHistBins - 1;
     for (int j = threadIdx.x; j < kHistBins + kHistBins / 32; j += blockDim.x) histk[j] = 0;
     __syncthreads();
@@ -1039,6 +1062,11 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     uint32_t prefix = 0, pmask = 0;
     int remaining = k;
     bool located = false;
+    if (take_all) {                                        // K* = the smallest key, all of them taken
+      pmask = 0xffffffffu;
+      remaining = nc;
+      located = true;
+    }
     if (pivots) {
       const int want = k - fabove;                         // keys of the k-th key's bin to take
       find_digit_skewed<kHistBins / kSelThreads>(histk, kHistBins, want, res, scratch);
@@ -1158,13 +1186,23 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         if (i0 + q >= p1) break;
         if (uu[q] > prefix) {
           const int o = g + (e < remaining ? e : remaining);
-          if (o < k) sout[o] = ii[q];                      // (bound holds unless the histogram is stale)
+          if (o < k) {                                     // (bound holds unless the histogram is stale)
+            sout[o] = ii[q];
+            if (oscore) oscore[o] = key_value(uu[q] + kmin);
+          }
           ++g;
         } else if (uu[q] == prefix) {
-          if (e < remaining && g + e < k) sout[g + e] = ii[q];
+          if (e < remaining && g + e < k) {
+            sout[g + e] = ii[q];
+            if (oscore) oscore[g + e] = key_value(uu[q] + kmin);
+          }
           ++e;
         }
       }
+    }
+    for (int j = nc + threadIdx.x; j < k; j += blockDim.x) {   // take_all with nc < k: -1 pads
+      sout[j] = -1;
+      if (oscore) oscore[j] = -INFINITY;
     }
     __syncthreads();
     if ((k & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) {
@@ -1179,9 +1217,14 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
     // candidate list in global memory
     int32_t* sel = reinterpret_cast<int32_t*>(sel_smem);   // [k] selected indices, then bucketed
     int32_t* bucket = sel + CSA_MAX_TOPK;                  // [k] indices grouped by chunk
-    int* ccount = bucket + CSA_MAX_TOPK;                   // [nchunks + 1] per-chunk counts -> offsets
+    uint32_t* selk = reinterpret_cast<uint32_t*>(bucket + CSA_MAX_TOPK);   // [k] their keys (sel_scores)
+    uint32_t* bucketk = selk + CSA_MAX_TOPK;               // [k] keys beside bucket
+    int* ccount = reinterpret_cast<int*>(bucketk + CSA_MAX_TOPK);   // [nchunks + 1] per-chunk counts -> offsets
     for (int j = threadIdx.x; j <= nchunks; j += blockDim.x) ccount[j] = 0;
-    for (int j = threadIdx.x; j < k; j += blockDim.x) sel[j] = 0;   // in range even if a slot stays unset
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {   // in range even if a slot stays unset
+      sel[j] = 0;
+      selk[j] = 0u;
+    }
     __syncthreads();
     auto cand_key = [&](int i) -> uint32_t { return __ldcg(ckey + i); };
     auto cand_idx = [&](int i) -> int32_t { return __ldcg(cidx + i); };
@@ -1228,7 +1271,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
       bg = __shfl_sync(0xffffffffu, bg, 0);
       be = __shfl_sync(0xffffffffu, be, 0);
       const uint32_t below = (1u << lane_id()) - 1;
-      if (gt && bg + __popc(mg & below) < k) sel[bg + __popc(mg & below)] = cand_idx(i);
+      if (gt && bg + __popc(mg & below) < k) {
+        sel[bg + __popc(mg & below)] = cand_idx(i);
+        selk[bg + __popc(mg & below)] = key;
+      }
       if (eq && be + __popc(me & below) < CSA_MAX_TOPK) eqlist[be + __popc(me & below)] = cand_idx(i);
     }
     __syncthreads();
@@ -1239,7 +1285,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         const int32_t j = eqlist[e];
         int rank = 0;
         for (int q = 0; q < neq; ++q) rank += eqlist[q] < j;
-        if (rank < remaining && ngt + rank < k) sel[ngt + rank] = j;
+        if (rank < remaining && ngt + rank < k) {
+          sel[ngt + rank] = j;
+          selk[ngt + rank] = prefix;
+        }
       }
     } else {
       // more ties than the list holds (degenerate rows, e.g. constant scores): rank against
@@ -1249,7 +1298,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         const int32_t j = cand_idx(i);
         int rank = 0;
         for (int q = 0; q < nc && rank < remaining; ++q) rank += (cand_key(q) == prefix && cand_idx(q) < j);
-        if (rank < remaining && ngt + rank < k) sel[ngt + rank] = j;
+        if (rank < remaining && ngt + rank < k) {
+          sel[ngt + rank] = j;
+          selk[ngt + rank] = prefix;
+        }
       }
     }
     __syncthreads();
@@ -1294,6 +1346,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
         if ((int)lane_id() == leader) base = atomicAdd(&ccount[c], __popc(peers));
         base = __shfl_sync(peers, base, leader);
         bucket[base + __popc(peers & ((1u << lane_id()) - 1))] = j;   // ccount ends at the bucket's end
+        bucketk[base + __popc(peers & ((1u << lane_id()) - 1))] = selk[i];
       }
     }
     __syncthreads();
@@ -1305,6 +1358,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* _
       int rank = 0;
       for (int q = b_start; q < b_end; ++q) rank += bucket[q] < j;
       out[b_start + rank] = j;
+      if (oscore) oscore[b_start + rank] = key_value(bucketk[i]);
     }
     __syncthreads();
   }

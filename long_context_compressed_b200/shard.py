@@ -6,8 +6,8 @@ library's kernels; this module only orders the calls and the exchanges):
 
 1. the indexer over the local entries, the local top-k (e4m3 scores of Hadamard-rotated
    queries and keys, exact bf16 rescoring of the kc = 2k candidates as in the single-GPU
-   step), the exact scores of
-   the local winners and their global entry numbers;
+   step), which also returns the exact scores of the local winners, and their global
+   entry numbers;
 2. one all-gather of the (score, global index) pairs, then the global top-k
    (csa_shard_select), the same on every GPU.  Every global winner is a local winner of
    its shard, so the gathered lists hold the whole-row top-k, and with the shards in
@@ -98,10 +98,8 @@ class GpuKernels:
             ws = self.buf["select_ws"] = csa.select_workspace(B, Ns, dev)
         csa.csa_index_scores(q8, w, sh.k8, sh.n_valid, q_scale=qs, k_scale=sh.ks, scores=scores, select_ws=ws)
         loc = self._b("loc", (B, 1, k), torch.int32, dev)
-        csa.csa_topk_select(scores, sh.n_valid, k, ws, kc=2 * k, qI=qI, w=w, kI=sh.kI, idx=loc)
         exact = self._b("exact", (B, 1, k), torch.float32, dev)
-        kept = self._b("kept", (B, 1, k), torch.int32, dev)
-        csa.csa_index_rerank(qI, w, sh.kI, loc, k, cand_scores=exact, idx=kept)
+        csa.csa_topk_select(scores, sh.n_valid, k, ws, kc=2 * k, qI=qI, w=w, kI=sh.kI, idx=loc, idx_scores=exact)
         pairs = csa.shard_pack(exact, loc, Ns, sh.lo, pairs=self._b("pairs", (B, k, 2), torch.int32, dev))
         return pairs
 

@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from long_context_compressed_b200 import synth
-from tolerances import check_topk_sets
+from tolerances import check_f32, check_topk_sets
 
 pytestmark = pytest.mark.gpu
 
@@ -165,6 +165,69 @@ def test_select_rescore_semantics(csa, dtype):
         pos = [int(np.searchsorted(cand, i)) for i in got[b, 0] if i >= 0]
         assert np.all(np.isin(got[b, 0], cand))
         check_topk_sets(pos, ex[0, 0], k, 1e-5 * mag.max(), what=f"select rescore b={b}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_select_exported_scores(csa, dtype):
+    """idx_scores: beside each selected index the rescored score that ranked it, equal to the
+    plain indexer score of that entry (oracle, fp32 rule); -inf beside the -1 pads.  Rows:
+    full, ragged, n_valid <= k (every entry taken, rescored too) and n_valid = 0.  The
+    selection itself is the one the call makes without idx_scores."""
+    B, N, k, kc = 4, 3000, 100, 200
+    wl = synth.Workload("sel_scores", dtype, B=B, ctx=4 * N, T=1, q_pos0=4 * N - 1, ratio=4, N=N, H=16, D=128,
+                        index_dtype=dtype)
+    ix = synth.draw_indexer(wl, seed=37)
+    s = synth.draw_scores(37, "select/scores", B, 1, N)
+    nv = np.array([[N], [N - 777], [k - 9], [0]], np.int32)
+    ws = csa.select_workspace(B, N)
+    g_s, g_nv = s.cuda(), torch.from_numpy(nv).cuda()
+    qI, w, kI = ix["qI"].cuda(), ix["w"].cuda(), ix["kI"].cuda()
+    csa.csa_score_histogram(g_s, g_nv, ws)
+    plain = csa.csa_topk_select(g_s, g_nv, k, ws, kc=kc, qI=qI, w=w, kI=kI).cpu().numpy()
+    sc = torch.empty((B, 1, k), dtype=torch.float32, device="cuda")
+    csa.csa_score_histogram(g_s, g_nv, ws)
+    got = csa.csa_topk_select(g_s, g_nv, k, ws, kc=kc, qI=qI, w=w, kI=kI, idx_scores=sc).cpu().numpy()
+    sc = sc.cpu().numpy()
+    assert np.array_equal(got, plain)
+    for b in range(B):
+        n = min(int(nv[b, 0]), k)
+        sel = got[b, 0, :n]
+        if nv[b, 0] <= k:
+            assert sel.tolist() == list(range(n))
+        assert np.all(got[b, 0, n:] == -1) and np.all(np.isneginf(sc[b, 0, n:]))
+        if n == 0:
+            continue
+        ex, mag = oracle.index_scores(ix["qI"][b:b + 1].float().numpy(), ix["w"][b:b + 1].numpy(),
+                                      ix["kI"][b:b + 1, sel].float().numpy(), np.array([[n]], np.int32),
+                                      with_mag=True)
+        check_f32(sc[b, 0, :n], ex[0, 0], mag[0, 0], what=f"select exported scores {dtype} b={b}")
+
+
+def test_select_exported_scores_plain(csa):
+    """Without rescoring idx_scores holds the input score of each selected index, bit for
+    bit (the order key maps back to the float; -0.0 comes back as +0.0), on the shared-memory
+    path, on a constant row (the global-memory path) and on a row of n_valid < k; N = 0 gives
+    -1 and -inf throughout."""
+    B, N, k = 3, 50000, 512
+    s = synth.draw_scores(41, "select/scores_plain", B, 1, N, ties=6)
+    s[1, 0] = 3.25
+    nv = np.array([[N], [N], [k - 3]], np.int32)
+    ws = csa.select_workspace(B, N)
+    g_s, g_nv = s.cuda(), torch.from_numpy(nv).cuda()
+    csa.csa_score_histogram(g_s, g_nv, ws)
+    sc = torch.empty((B, 1, k), dtype=torch.float32, device="cuda")
+    got = csa.csa_topk_select(g_s, g_nv, k, ws, idx_scores=sc).cpu().numpy()
+    sc = sc.cpu().numpy()
+    assert np.array_equal(got, oracle.topk(s.numpy(), nv, k))
+    for b in range(B):
+        ok = got[b, 0] >= 0
+        assert np.array_equal(sc[b, 0, ok], s[b, 0].numpy()[got[b, 0, ok]])
+        assert np.all(np.isneginf(sc[b, 0, ~ok]))
+    e = torch.empty((2, 1, 0), device="cuda")
+    nv0 = torch.zeros((2, 1), dtype=torch.int32, device="cuda")
+    sc0 = torch.zeros((2, 1, 8), dtype=torch.float32, device="cuda")
+    i0 = csa.csa_topk_select(e, nv0, 8, csa.select_workspace(2, 0), idx_scores=sc0).cpu().numpy()
+    assert np.all(i0 == -1) and np.all(np.isneginf(sc0.cpu().numpy()))
 
 
 def test_select_fed_by_indexer_histogram(csa):
