@@ -227,7 +227,10 @@ int attn_ndh(int D) { return D > 256 ? D / 256 : 1; }
 // CTAs per (query, D-slice, head group) over the row list: one wave of CTAs, at
 // least two KV tiles each for sparse_attn (gathered rows: the more SMs issue the
 // gathers, the sooner the rows are in) and four for hca_attn (contiguous rows by TMA,
-// and it shares the GPU with the chain of the CSA layer)
+// and it shares the GPU with the chain of the CSA layer).  When that leaves at most four
+// tiles per split, the launch takes at most half the SMs, with the fewest splits that
+// give the same largest share (the rule of the bf16 kernel below: the step's other
+// attention then runs beside it).
 int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse, int R) {
   const int64_t items = (int64_t)B * T * attn_ndh(D) * ((H + 63) / 64);
   const int sms = sm_count();
@@ -235,7 +238,14 @@ int attn_nsplit(int B, int T, int H, int D, int64_t max_rows, bool sparse, int R
   const int64_t tiles = (max_rows + R - 1) / R;
   const int64_t want = std::max<int64_t>(1, sms / items);
   const int64_t cap = std::max<int64_t>(1, tiles / (sparse ? 2 : 4));
-  return (int)std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), csa::kMaxSplits));   // one cluster
+  int64_t ns = std::max<int64_t>(1, std::min<int64_t>(std::min(want, cap), csa::kMaxSplits));   // one cluster
+  const int64_t half = std::max<int64_t>(1, sms / 2 / items);
+  if (tiles <= 4 * ns && ns > half) {
+    ns = half;
+    const int64_t share = (tiles + ns - 1) / ns;
+    while (ns > 1 && (tiles + ns - 2) / (ns - 1) == share) --ns;
+  }
+  return (int)ns;
 }
 
 // bf16 rows (attn_t_kernel): splits of a query's row list (units of 64 rows) form one
