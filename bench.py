@@ -710,8 +710,9 @@ def bench_workload(name, index, with_hca, steps, warmup, world, device, n_sets=N
 
 def _stage_times(stages, steps, warmup):
     """Eager calls, CUDA events between stages on the current stream: mean device time
-    per stage (us) and per step (ms).  Every step writes hundreds of MB (scores,
-    outputs), so no input stays in L2 from one step to the next."""
+    per stage (us) and per step (ms).  Every step reads and writes hundreds of MB (the
+    attention's 256 MB of queries and of outputs), so no input stays in L2 from one step
+    to the next."""
     import torch
     for _ in range(warmup):
         for _, fn in stages:
@@ -733,8 +734,10 @@ def _stage_times(stages, steps, warmup):
 def bench_prefill(steps, warmup, device, tflops_peak):
     """Flash-shaped chunked prefill (4,096 query tokens at 126,976..131,071 of a 131,072-token
     context, B = 1): compress the chunk (c = 512 latent + 128 index keys), bf16 index scores
-    over 32,768 keys, top-512 per query, sparse_attn (64 heads, D = 512).  Also the indexer
-    alone in e4m3 (quantised queries and keys).  Indexer FLOPs = 2 x 64 x 128 x sum(n_valid)."""
+    over 32,768 keys, top-512 per query, sparse_attn (64 heads, D = 512).  Also timed: the
+    indexer and top-k in one call without the score matrix (csa_index_topk; its indices are
+    checked equal to the step's), and the indexer alone in e4m3 (quantised queries and
+    keys).  Indexer FLOPs = 2 x 64 x 128 x sum(n_valid)."""
     import torch
 
     from long_context_compressed_b200 import csa, synth
@@ -757,6 +760,8 @@ def bench_prefill(steps, warmup, device, tflops_peak):
     scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
     idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
     topk_ws = csa.topk_workspace(B, T, N, k, dev)
+    fused_ws = csa.index_topk_workspace(B, T, N, k, csa.CSA_BF16, dev)
+    failed = torch.zeros((1,), dtype=torch.int32, device=dev)
     attn_ws = csa.attn_workspace(B, T, H, D, 128 + k, device=dev)
     out = torch.empty_like(q)
     k8, ks = csa.csa_quantize_e4m3(kI, hadamard=INDEX_ROTATION)
@@ -780,6 +785,12 @@ def bench_prefill(steps, warmup, device, tflops_peak):
         fn()
     launches = csa.csa_launch_count() - c0
     per, step_ms = _stage_times(stages, steps, warmup)
+    idx_fused = torch.empty_like(idx)
+    fused = [("index_topk", lambda: csa.csa_index_topk(qI, w, kI, n_valid, k, idx=idx_fused, workspace=fused_ws,
+                                                       failed_rows=failed))]
+    per_f, _ = _stage_times(fused, steps, warmup)
+    assert torch.equal(idx, idx_fused), "fused and unfused prefill top-k differ"
+    failed_rows = int(failed.item())
     e4m3 = [("quantize_q", lambda: csa.csa_quantize_e4m3(qI, codes=q8, scale=qs, hadamard=INDEX_ROTATION)),
             ("index_e4m3", lambda: csa.csa_index_scores(q8, w, k8, n_valid, q_scale=qs, k_scale=ks, scores=scores))]
     per8, _ = _stage_times(e4m3, steps, warmup)
@@ -791,6 +802,10 @@ def bench_prefill(steps, warmup, device, tflops_peak):
                        f"N={N} keys, top-{k}, H={H}, D={D}",
            "tokens_per_s": B * T / (step_ms * 1e-3), "ms_per_step": step_ms, "steps": steps,
            "launches_per_step": launches, "breakdown_us": {n: round(v, 1) for n, v in per.items()},
+           "index_topk": {"fused_us": per_f["index_topk"], "unfused_us": per["index"] + per["topk"],
+                          "failed_rows": failed_rows,
+                          "note": "csa_index_topk (no score matrix) on the step's inputs, same indices; "
+                                  "the step keeps the faster unfused pair"},
            "indexer": {"keys_per_s": float(n_valid.sum().item()) / (per["index"] * 1e-6),
                        "bf16": {"achieved": tf_bf16, "peak": tflops_peak, "unit": "TFLOP/s",
                                 "frac": tf_bf16 / tflops_peak, "peak_source": "measured bf16 (burst)",
@@ -799,7 +814,7 @@ def bench_prefill(steps, warmup, device, tflops_peak):
                                 "frac": tf_e4m3 / (2 * tflops_peak),
                                 "peak_source": "measured bf16 (burst) x 2 (nominal e4m3:bf16 ratio)",
                                 "us": per8["index_e4m3"], "quantize_q_us": per8["quantize_q"]}}}
-    del scores, out, q, topk_ws, attn_ws
+    del scores, out, q, topk_ws, attn_ws, fused_ws
     torch.cuda.empty_cache()
     return res
 
@@ -872,8 +887,8 @@ def bench_hca(steps, warmup, device, hbm_peak, kv8=False):
 
 
 STAGES = ("compress", "quantize", "index", "select", "attn", "hcompress", "hca")
-BIG_STAGES = ("prefill_compress", "prefill_index", "prefill_index8", "prefill_topk", "prefill_attn",
-              "hca_compress", "hca_attn")
+BIG_STAGES = ("prefill_compress", "prefill_index", "prefill_index8", "prefill_topk", "prefill_index_topk",
+              "prefill_attn", "hca_compress", "hca_attn")
 
 
 def run_big_stage(stage, steps, warmup, device):
@@ -899,6 +914,13 @@ def run_big_stage(stage, steps, warmup, device):
         out = torch.empty((B, wl.comp_L // 4, wl.comp_c), dtype=torch.bfloat16, device=dev)
         fn = lambda: csa.csa_compress(x["C_a"], x["C_b"], x["Z_a"], x["Z_b"], pr["prev_Cb"], pr["prev_Zb"], ratio=4,
                                       out=out)
+    elif stage == "prefill_index_topk":
+        qI, kI = g("qI", (B, T, 64, 128)), g("kI", (B, N, 128))
+        w = synth.normal(0, f"bench/{wl.name}/w", (B, T, 64), device=dev)
+        n_valid = csa.csa_n_valid(q_pos, 4, 0, N)
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=dev)
+        ws = csa.index_topk_workspace(B, T, N, k, csa.CSA_BF16, dev)
+        fn = lambda: csa.csa_index_topk(qI, w, kI, n_valid, k, idx=idx, workspace=ws)
     elif stage in ("prefill_index", "prefill_index8", "prefill_topk"):
         qI, kI = g("qI", (B, T, 64, 128)), g("kI", (B, N, 128))
         w = synth.normal(0, f"bench/{wl.name}/w", (B, T, 64), device=dev)

@@ -205,6 +205,39 @@ int csa_index_scores(const void *qI, const float *q_scale, const float *w, const
                      void *stream);
 
 /*
+ * csa_index_topk -- the indexer and the top-k in one call, without writing the score
+ * matrix ([HA] §4.2: a cheap scan of every compressed key, the expensive work only for
+ * the top-k; the chunked-prefill shapes).  The result equals, index for index,
+ * csa_index_scores followed by csa_topk on the same arguments (the same kernel computes
+ * every score, so the values are bit-identical).  Steps, in stream order:
+ *   1. every 16th key of each sequence (and its scale) is gathered and scored;
+ *   2. per row, the r-th largest sampled score (r = ceil(4k / 16)) is the row's
+ *      threshold: about 4k keys are expected at or above it, and at least r are (a
+ *      row with r samples or fewer takes every valid key);
+ *   3. the indexer scores every key; each valid score at or above its row's threshold
+ *      goes into the row's candidate list (score key, index); nothing else is written;
+ *   4. per row with at least k and at most cap = min(8192, max(2048, 16k)) candidates, the exact
+ *      top-k of the list (ties toward the lower index), ascending; other rows are
+ *      counted as failed;
+ *   5. a fallback, launched every time and doing nothing unless a row failed: the
+ *      scores of every row into the workspace, then the row top-k of csa_topk.
+ *   Arguments as csa_index_scores / csa_topk; dtype CSA_BF16 or CSA_E4M3 (others:
+ *   CSA_ERR_UNSUPPORTED); k <= 1024, N <= 32768 (the fallback's row top-k holds a row in
+ *   shared memory).
+ *   idx         : [B, T, k] int32, ascending, -1 padded when n_valid < k.
+ *   failed_rows : NULL, or one device int32 (caller-owned): the number of rows that
+ *                 took the fallback (0 unless the sample misled a row's threshold or
+ *                 the row is dominated by ties).
+ *   workspace   : csa_index_topk_workspace_size(B, T, N, k, dtype) bytes, 256-byte
+ *                 aligned, no initial contents.  It includes room for the fallback's
+ *                 [B, T, N] fp32 scores, which only a failed row makes the call write.
+ */
+size_t csa_index_topk_workspace_size(int B, int T, int64_t N, int k, int dtype);
+int csa_index_topk(const void *qI, const float *q_scale, const float *w, const void *kI, const float *k_scale,
+                   int dtype, const int32_t *n_valid, int B, int T, int64_t N, int k, int32_t *idx,
+                   int32_t *failed_rows, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * csa_topk -- top-k of each score row ([HA] §4.2 / §7 topk(scores, k);
  * k = 512 Flash, 1024 Pro):
  *   idx[b,t,:] = the k indices i < n_valid[b,t] with the largest scores[b,t,i],

@@ -43,6 +43,8 @@ _SIGS = {
     "csa_kv8_entry_bytes": ([_i32], ctypes.c_longlong),
     "csa_quantize_kv8": ([_vp, _i64, _i32, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
+    "csa_index_topk_workspace_size": ([_i32, _i32, _i64, _i32, _i32], _sz),
+    "csa_index_topk": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "csa_select_workspace_size": ([_i32, _i64], _sz),
     "csa_score_histogram": ([_vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
     "csa_topk_select": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
@@ -201,6 +203,34 @@ def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=N
                                  _ptr(n_valid), B, T, N, _ptr(scores), _ptr(select_ws), _stream(stream)),
            "csa_index_scores")
     return scores
+
+
+def index_topk_workspace(B: int, T: int, N: int, k: int, dtype, device="cuda") -> torch.Tensor:
+    """A csa_index_topk workspace (256-byte aligned; no initial contents needed)."""
+    n = int(_lib.csa_index_topk_workspace_size(B, T, N, k, dtype))
+    buf = torch.empty(max(n, 16) + 256, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 256
+    return buf[off:off + max(n, 16)]
+
+
+def csa_index_topk(qI, w, kI, n_valid, k: int, *, q_scale=None, k_scale=None, idx=None, workspace=None,
+                   failed_rows=None, stream=None):
+    """Indexer scores and their top-k without the score matrix: idx [B, T, k] int32 equal to
+    csa_topk(csa_index_scores(...), n_valid, k).  qI [B, T, 64, 128] bf16 (or uint8 e4m3 codes
+    with q_scale / k_scale), kI [B, N, 128].  failed_rows: optional int32 [1] device tensor that
+    receives the number of rows that took the fallback."""
+    B, T = qI.shape[0], qI.shape[1]
+    N = kI.shape[1]
+    dt = _dtype_code(qI)
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=qI.device)
+    if workspace is None:
+        workspace = index_topk_workspace(B, T, N, k, dt, qI.device)
+    _check(_lib.csa_index_topk(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), dt, _ptr(n_valid), B, T,
+                               N, k, _ptr(idx), _ptr(failed_rows), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)),
+           "csa_index_topk")
+    return idx
 
 
 def csa_mxfp4_sf128_bytes(batches: int, rows_per_batch: int) -> int:

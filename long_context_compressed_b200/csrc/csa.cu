@@ -24,6 +24,7 @@
 #include "causal.cuh"
 #include "compress.cuh"
 #include "index.cuh"
+#include "index_topk.cuh"
 #include "kv8.cuh"
 #include "quantize.cuh"
 #include "topk.cuh"
@@ -678,6 +679,78 @@ int csa_quantize_kv8(const void* kv, int64_t rows, int D, void* entries, void* s
   return launch_status();
 }
 
+// Parameters of index_tc_kernel for one call (scores written, no histogram, no candidates).
+static IndexParams index_params(int mode, const float* q_scale, const float* w, const float* k_scale,
+                                const int32_t* n_valid, float* scores, int B, int T, int64_t N) {
+  const bool fp4 = mode == csa::kIdxMxfp4;
+  IndexParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.w = w;
+  p.q_scale = mode == csa::kIdxE4m3 ? q_scale : nullptr;
+  p.k_scale = mode == csa::kIdxE4m3 ? k_scale : nullptr;
+  p.q_sf = fp4 ? reinterpret_cast<const uint8_t*>(q_scale) : nullptr;
+  p.k_sf = fp4 ? reinterpret_cast<const uint8_t*>(k_scale) : nullptr;
+  p.n_valid = n_valid;
+  p.scores = scores;
+  p.B = B;
+  p.T = T;
+  p.N = N;
+  // queries per group: up to 4 (mxfp4: 2, so that a group's query scales are one atom)
+  p.TQ = (T >= 4 && !fp4) ? 4 : (T >= 2 ? 2 : 1);
+  return p;
+}
+
+// One launch of index_tc_kernel (emit: the candidate mode) over p's B x T queries and N keys.
+static int launch_index_tc(const void* qI, const void* kI, int mode, IndexParams p, bool emit, cudaStream_t st) {
+  const bool fp4 = mode == csa::kIdxMxfp4;
+  const int B = p.B, T = p.T;
+  const int64_t N = p.N;
+  const int key_bytes = mode == csa::kIdxBf16 ? csa::IndexCfg<csa::kIdxBf16>::kKeyBytes
+                        : mode == csa::kIdxE4m3 ? csa::IndexCfg<csa::kIdxE4m3>::kKeyBytes
+                                                : csa::IndexCfg<csa::kIdxMxfp4>::kKeyBytes;
+  const int qrow = mode == csa::kIdxBf16 ? 256 : (mode == csa::kIdxE4m3 ? 128 : 64);
+  const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
+  const int fixed = 1024 + (q_bytes + 1023) / 1024 * 1024 + (fp4 ? 1024 : 0) +
+                    csa::kIdxEpiWarps * p.TQ * csa::kIdxHeads * 4 + 8 * (4 + 2 * csa::kMaxAcc) +
+                    csa::kKsRing * 32 * csa::kIdxEpiWarps * 4 + (p.hist ? 2 * csa::kHistBinsIdx * 4 : 0) +
+                    (emit ? csa::kIdxEpiWarps * 12 * 4 : 0);
+  if (emit && p.hist) return CSA_ERR_INVALID;      // (the two share their shared memory)
+  p.stages = std::min(fp4 ? 16 : 12, (kSmemLimit - fixed) / (key_bytes + 16));
+  if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
+  const int smem = fixed + p.stages * (key_bytes + 16);
+  CUtensorMap kmap, qmap;
+  const CUtensorMapDataType dt = mode == csa::kIdxBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const int es = mode == csa::kIdxBf16 ? 2 : 1;
+  const uint32_t box0 = mode == csa::kIdxBf16 ? 64 : (fp4 ? 64 : 128);        // elements of one swizzle row
+  const uint64_t inner = fp4 ? 64 : csa::kIdxDim;                             // elements per row in memory
+  const CUtensorMapSwizzle swz = fp4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_map(&kmap, kI, dt, es, inner, (uint64_t)N, (uint64_t)B, box0, csa::kIdxTileKeys, swz) ||
+      !make_map(&qmap, qI, dt, es, inner, (uint64_t)T * csa::kIdxHeads, (uint64_t)B, box0,
+                (uint32_t)(p.TQ * csa::kIdxHeads), swz))
+    return CSA_ERR_CUDA;
+  const int QG = (T + p.TQ - 1) / p.TQ;
+  const int64_t KT = (N + csa::kIdxTileKeys - 1) / csa::kIdxTileKeys;
+  const int64_t items = (int64_t)B * QG * KT;
+  const unsigned grid = (unsigned)std::min<int64_t>(items, sm_count());
+  // candidate mode: 32-slot chunks when a CTA walks at least one whole row of key tiles
+  // (a row then spans at most two CTAs: at most 2 x 16 warps x 31 unused slots); exact
+  // reservations otherwise
+  if (emit) p.cand_chunk = items / grid >= KT ? 32 : 1;
+  auto go = [&](auto kernel) -> int {
+    if (!set_smem(kernel, smem)) return CSA_ERR_CUDA;
+    launch_k(kernel, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
+    return launch_status();
+  };
+  if (emit) {
+    if (mode == csa::kIdxE4m3) return go(csa::index_tc_kernel<csa::kIdxE4m3, true>);
+    if (mode == csa::kIdxBf16) return go(csa::index_tc_kernel<csa::kIdxBf16, true>);
+    return CSA_ERR_UNSUPPORTED;
+  }
+  if (mode == csa::kIdxE4m3) return go(csa::index_tc_kernel<csa::kIdxE4m3>);
+  if (mode == csa::kIdxBf16) return go(csa::index_tc_kernel<csa::kIdxBf16>);
+  return go(csa::index_tc_kernel<csa::kIdxMxfp4>);
+}
+
 int csa_index_scores(const void* qI, const float* q_scale, const float* w, const void* kI, const float* k_scale,
                      int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* select_ws,
                      void* stream) {
@@ -700,59 +773,145 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
     return launch_status();
   }
   const int mode = dtype == CSA_BF16 ? csa::kIdxBf16 : (dtype == CSA_E4M3 ? csa::kIdxE4m3 : csa::kIdxMxfp4);
-  const bool fp4 = mode == csa::kIdxMxfp4;
-  IndexParams p;
-  p.w = w;
-  p.q_scale = mode == csa::kIdxE4m3 ? q_scale : nullptr;
-  p.k_scale = mode == csa::kIdxE4m3 ? k_scale : nullptr;
-  p.q_sf = fp4 ? reinterpret_cast<const uint8_t*>(q_scale) : nullptr;
-  p.k_sf = fp4 ? reinterpret_cast<const uint8_t*>(k_scale) : nullptr;
-  p.n_valid = n_valid;
-  p.scores = scores;
-  p.B = B;
-  p.T = T;
-  p.N = N;
-  // queries per group: up to 4 (mxfp4: 2, so that a group's query scales are one atom)
-  p.TQ = (T >= 4 && !fp4) ? 4 : (T >= 2 ? 2 : 1);
-  p.hist = nullptr;
-  p.hist_stride = 0;
+  IndexParams p = index_params(mode, q_scale, w, k_scale, n_valid, scores, B, T, N);
   if (select_ws != nullptr) {
     if (T != 1 || !aligned16(select_ws)) return CSA_ERR_INVALID;
     p.hist = reinterpret_cast<int*>(select_ws);
     p.hist_stride = csa::SelectWs::row_bytes(N) / 4;
   }
-  const int key_bytes = mode == csa::kIdxBf16 ? csa::IndexCfg<csa::kIdxBf16>::kKeyBytes
-                        : mode == csa::kIdxE4m3 ? csa::IndexCfg<csa::kIdxE4m3>::kKeyBytes
-                                                : csa::IndexCfg<csa::kIdxMxfp4>::kKeyBytes;
-  const int qrow = mode == csa::kIdxBf16 ? 256 : (mode == csa::kIdxE4m3 ? 128 : 64);
-  const int q_bytes = p.TQ * csa::kIdxHeads * qrow;
-  const int fixed = 1024 + (q_bytes + 1023) / 1024 * 1024 + (fp4 ? 1024 : 0) +
-                    csa::kIdxEpiWarps * p.TQ * csa::kIdxHeads * 4 + 8 * (4 + 2 * csa::kMaxAcc) +
-                    csa::kKsRing * 32 * csa::kIdxEpiWarps * 4 + (select_ws ? 2 * csa::kHistBinsIdx * 4 : 0);
-  p.stages = std::min(fp4 ? 16 : 12, (kSmemLimit - fixed) / (key_bytes + 16));
-  if (p.stages < 2) return CSA_ERR_UNSUPPORTED;
-  const int smem = fixed + p.stages * (key_bytes + 16);
-  CUtensorMap kmap, qmap;
-  const CUtensorMapDataType dt = mode == csa::kIdxBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  const int es = mode == csa::kIdxBf16 ? 2 : 1;
-  const uint32_t box0 = mode == csa::kIdxBf16 ? 64 : (fp4 ? 64 : 128);        // elements of one swizzle row
-  const uint64_t inner = fp4 ? 64 : csa::kIdxDim;                             // elements per row in memory
-  const CUtensorMapSwizzle swz = fp4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_map(&kmap, kI, dt, es, inner, (uint64_t)N, (uint64_t)B, box0, csa::kIdxTileKeys, swz) ||
-      !make_map(&qmap, qI, dt, es, inner, (uint64_t)T * csa::kIdxHeads, (uint64_t)B, box0,
-                (uint32_t)(p.TQ * csa::kIdxHeads), swz))
-    return CSA_ERR_CUDA;
-  const int QG = (T + p.TQ - 1) / p.TQ;
-  const int64_t items = (int64_t)B * QG * ((N + csa::kIdxTileKeys - 1) / csa::kIdxTileKeys);
-  const unsigned grid = (unsigned)std::min<int64_t>(items, sm_count());
-  auto go = [&](auto kernel) -> int {
-    if (!set_smem(kernel, smem)) return CSA_ERR_CUDA;
-    launch_k(kernel, grid, csa::kIdxThreads, smem, st, kmap, qmap, p);
-    return launch_status();
+  return launch_index_tc(qI, kI, mode, p, false, st);
+}
+
+// ---------------------------------------------------------------- csa_index_topk
+// Workspace pieces, each 256-byte aligned: sample keys, sample key scales, sample
+// n_valid, sample scores, thresholds, candidate counts, failure count, candidate lists,
+// and the score matrix the fallback writes.
+struct IndexTopkWs {
+  size_t kI_s, ks_s, nv_s, s_scores, thr, cnt, fail, cand, scores, total;
+  int64_t Ns;
+  int cap, r0;
+};
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+static IndexTopkWs index_topk_layout(int B, int T, int64_t N, int k, int dtype) {
+  IndexTopkWs L;
+  const int64_t rows = (int64_t)B * T;
+  L.Ns = (N + csa::kSampleStride - 1) / csa::kSampleStride;
+  L.r0 = (4 * k + csa::kSampleStride - 1) / csa::kSampleStride;
+  L.cap = std::min(csa::kCandCapMax, std::max(2048, 16 * k));
+  const size_t row_bytes = dtype == CSA_BF16 ? 256 : 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
   };
-  if (mode == csa::kIdxE4m3) return go(csa::index_tc_kernel<csa::kIdxE4m3>);
-  if (mode == csa::kIdxBf16) return go(csa::index_tc_kernel<csa::kIdxBf16>);
-  return go(csa::index_tc_kernel<csa::kIdxMxfp4>);
+  L.kI_s = take((size_t)B * L.Ns * row_bytes);
+  L.ks_s = take(dtype == CSA_E4M3 ? (size_t)B * L.Ns * 4 : 0);
+  L.nv_s = take((size_t)rows * 4);
+  L.s_scores = take((size_t)rows * L.Ns * 4);
+  L.thr = take((size_t)rows * 4);
+  L.cnt = take((size_t)rows * 4);
+  L.fail = take(16);
+  L.cand = take((size_t)rows * L.cap * 8);
+  L.scores = take((size_t)rows * N * 4);
+  L.total = off;
+  return L;
+}
+
+size_t csa_index_topk_workspace_size(int B, int T, int64_t N, int k, int dtype) {
+  if (B <= 0 || T <= 0 || N <= 0 || k < 1) return 0;
+  return index_topk_layout(B, T, N, k, dtype).total;
+}
+
+int csa_index_topk(const void* qI, const float* q_scale, const float* w, const void* kI, const float* k_scale,
+                   int dtype, const int32_t* n_valid, int B, int T, int64_t N, int k, int32_t* idx,
+                   int32_t* failed_rows, void* workspace, size_t ws_bytes, void* stream) {
+  if (B < 0 || T < 0 || N < 0 || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3 && dtype != CSA_MXFP4) return CSA_ERR_INVALID;
+  if (dtype != CSA_BF16 && dtype != CSA_E4M3) return CSA_ERR_UNSUPPORTED;
+  if (k > csa::kIndexTopkMaxK || N > csa::kRowSmemMax || B > 65535 ||
+      (int64_t)T * csa::kIdxHeads >= (int64_t(1) << 31))
+    return CSA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return CSA_OK;
+  if (!qI || !w || !kI || !n_valid || !idx) return CSA_ERR_INVALID;
+  if (dtype == CSA_E4M3 && (!q_scale || !k_scale)) return CSA_ERR_INVALID;
+  if (!aligned16(qI) || !aligned16(kI)) return CSA_ERR_INVALID;
+  cudaStream_t st = as_stream(stream);
+  const int64_t rows = (int64_t)B * T;
+  if (N == 0) {                                      // no keys: every row is -1
+    launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, 4, st, (const float*)nullptr, n_valid, N, k, idx,
+             (const int32_t*)nullptr, 0, (const int*)nullptr);
+    return launch_status();
+  }
+  const IndexTopkWs L = index_topk_layout(B, T, N, k, dtype);
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return CSA_ERR_INVALID;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* kI_s = ws + L.kI_s;
+  float* ks_s = dtype == CSA_E4M3 ? reinterpret_cast<float*>(ws + L.ks_s) : nullptr;
+  int32_t* nv_s = reinterpret_cast<int32_t*>(ws + L.nv_s);
+  float* s_scores = reinterpret_cast<float*>(ws + L.s_scores);
+  uint32_t* thr = reinterpret_cast<uint32_t*>(ws + L.thr);
+  int* cnt = reinterpret_cast<int*>(ws + L.cnt);
+  int* fail = reinterpret_cast<int*>(ws + L.fail);
+  auto* cand = reinterpret_cast<unsigned long long*>(ws + L.cand);
+  float* scores = reinterpret_cast<float*>(ws + L.scores);
+  const int mode = dtype == CSA_BF16 ? csa::kIdxBf16 : csa::kIdxE4m3;
+  const int row_bytes = dtype == CSA_BF16 ? 256 : 128;
+  // 1. the key sample and its n_valid
+  {
+    const int64_t work = std::max<int64_t>((int64_t)B * L.Ns * (row_bytes / 16), rows);
+    const unsigned blocks = (unsigned)std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 8);
+    launch_k(csa::sample_keys_kernel, blocks, 256, 0, st, static_cast<const uint8_t*>(kI), k_scale, B, N, L.Ns,
+             row_bytes, kI_s, ks_s, n_valid, rows, nv_s);
+    int rc = launch_status();
+    if (rc != CSA_OK) return rc;
+  }
+  // 2. the sample's scores
+  int rc = launch_index_tc(qI, kI_s, mode, index_params(mode, q_scale, w, ks_s, nv_s, s_scores, B, T, L.Ns), false,
+                           st);
+  if (rc != CSA_OK) return rc;
+  // 3. per-row thresholds (zeroes the candidate counts and the failure counts)
+  {
+    const int smem = (int)(L.Ns * 4);
+    if (!set_smem(csa::cand_threshold_kernel, std::max(smem, 4))) return CSA_ERR_CUDA;
+    launch_k(csa::cand_threshold_kernel, (unsigned)rows, 256, std::max(smem, 4), st, (const float*)s_scores, L.Ns,
+             n_valid, N, k, L.r0, thr, cnt, fail, failed_rows);
+    rc = launch_status();
+    if (rc != CSA_OK) return rc;
+  }
+  // 4. every key scored; the scores at or above their row's threshold become candidates
+  {
+    IndexParams p = index_params(mode, q_scale, w, k_scale, n_valid, nullptr, B, T, N);
+    p.thr = thr;
+    p.cand_cnt = cnt;
+    p.cand = cand;
+    p.cand_cap = L.cap;
+    rc = launch_index_tc(qI, kI, mode, p, true, st);
+    if (rc != CSA_OK) return rc;
+  }
+  // 5. the exact top-k of each row's candidates; rows that cannot be settled are counted
+  {
+    const int smem = L.cap * 8 + (int)((N + 31) / 32) * 4;
+    if (!set_smem(csa::cand_select_kernel, smem)) return CSA_ERR_CUDA;
+    launch_k(csa::cand_select_kernel, (unsigned)rows, 256, smem, st, (const unsigned long long*)cand,
+             (const int*)cnt, L.cap, n_valid, N, k, idx, fail, failed_rows);
+    rc = launch_status();
+    if (rc != CSA_OK) return rc;
+  }
+  // 6. the fallback, gated on the failure count: every row's scores, then the row top-k
+  {
+    IndexParams p = index_params(mode, q_scale, w, k_scale, n_valid, scores, B, T, N);
+    p.gate = fail;
+    rc = launch_index_tc(qI, kI, mode, p, false, st);
+    if (rc != CSA_OK) return rc;
+    const int smem = (int)(N * 4) + (N >= csa::kRowFastMin ? csa::kRowCand * 8 : 0);
+    if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
+    launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, smem, st, (const float*)scores, n_valid, N, k, idx,
+             (const int32_t*)nullptr, N >= csa::kRowFastMin ? 1 : 0, (const int*)fail);
+    return launch_status();
+  }
 }
 
 int csa_index_rerank(const void* qI, const float* w, const void* kI, int dtype, const int32_t* cand, int kc, int B,
@@ -779,7 +938,8 @@ int csa_index_rerank(const void* qI, const float* w, const void* kI, int dtype, 
   if (rc != CSA_OK) return rc;
   const int smem = kc * 4;
   if (!set_smem(csa::topk_row_kernel, std::max(smem, 4))) return CSA_ERR_CUDA;
-  launch_k(csa::topk_row_kernel, (unsigned)((int64_t)B * T), 1024, smem, st, cand_scores, nullptr, kc, k, idx, cand, 0);
+  launch_k(csa::topk_row_kernel, (unsigned)((int64_t)B * T), 1024, smem, st, cand_scores, nullptr, kc, k, idx, cand, 0,
+           (const int*)nullptr);
   return launch_status();
 }
 
@@ -821,7 +981,7 @@ int csa_topk(const float* scores, const int32_t* n_valid, int B, int T, int64_t 
                      (N >= csa::kRowFastMin ? csa::kRowCand * 8 : 0);
     if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
     launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, smem, st, scores, n_valid, N, k, idx, nullptr,
-             N >= csa::kRowFastMin ? 1 : 0);
+             N >= csa::kRowFastMin ? 1 : 0, (const int*)nullptr);
     return launch_status();
   }
   const size_t need = csa_topk_workspace_size(B, T, N, k);
@@ -870,7 +1030,8 @@ int csa_topk_select(const float* scores, const int32_t* n_valid, int B, int64_t 
   const size_t need = csa_select_workspace_size(B, N);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSA_ERR_INVALID;
   if (N == 0) {
-    launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr, 0);
+    launch_k(csa::topk_row_kernel, (unsigned)B, 1024, 4, as_stream(stream), scores, n_valid, N, k, idx, nullptr, 0,
+             (const int*)nullptr);
     if (idx_scores)
       launch_k(csa::fill_f32_kernel, (unsigned)std::min<int64_t>(((int64_t)B * k + 255) / 256, 1024), 256, 0,
                as_stream(stream), idx_scores, (int64_t)B * k, -INFINITY);
@@ -1070,7 +1231,7 @@ int csa_shard_select(const void* pairs, int G, int B, int k, int32_t* idx, void*
   const int smem = (int)std::max<int64_t>(4, n * 4);
   if (!set_smem(csa::topk_row_kernel, smem)) return CSA_ERR_CUDA;
   launch_k(csa::topk_row_kernel, (unsigned)B, 1024, smem, st, (const float*)row_scores, (const int32_t*)nullptr, n, k,
-           idx, (const int32_t*)row_idx, 0);
+           idx, (const int32_t*)row_idx, 0, (const int*)nullptr);
   return launch_status();
 }
 

@@ -45,14 +45,14 @@ constexpr int kKsAhead = 3;                     // key-scale prefetch distance (
 constexpr int kKsRing = kKsAhead + 1;
 constexpr int kHistBinsIdx = 4096;              // 12-bit histogram of order-preserving score keys
 
-// Top 12 bits of the order-preserving uint32 key of a score (-0.0 folded to +0.0):
-// bin order equals score order.
-__device__ __forceinline__ uint32_t score_bin(float x) {
+// Order-preserving uint32 key of a score (-0.0 folded to +0.0): key order equals score order.
+__device__ __forceinline__ uint32_t score_key(float x) {
   uint32_t u = __float_as_uint(x);
   if ((u << 1) == 0) u = 0;
-  const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return key >> 20;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// Its top 12 bits: bin order equals score order.
+__device__ __forceinline__ uint32_t score_bin(float x) { return score_key(x) >> 20; }
 
 struct IndexParams {
   const float* w;        // [B, T, 64]
@@ -68,6 +68,19 @@ struct IndexParams {
   int64_t N;
   int TQ;                // queries per group (1, 2 or 4)
   int stages;            // key pipeline depth
+  // candidate mode (index_tc_kernel<MODE, true>): no score is written; a valid score whose
+  // key is >= thr[row] is appended to row's list cand[row][..] as (key << 32) | ~i.
+  // cand_chunk 32: an epilogue warp reserves 32 slots of a row at a time (cand_cnt[row]
+  // += 32), fills them in order and zero-fills the unused tail of its last chunk (one
+  // atomic per 32 entries; for rows that span few CTAs, so few warps leave a tail).
+  // cand_chunk 1: each ballot reserves exactly its entries.  Slots at or past cand_cap
+  // are not written (cand_cnt still counts them).
+  const uint32_t* thr;          // [B*T]
+  int* cand_cnt;                // [B*T]
+  unsigned long long* cand;     // [B*T][cand_cap]
+  int cand_cap;
+  int cand_chunk;               // 32 or 1
+  const int* gate;              // null, or a device int written by an earlier launch: 0 -> no work
 };
 
 // Operand modes of index_tc_kernel.
@@ -114,7 +127,7 @@ __device__ __forceinline__ void index_next(IndexItem& it, int QG, int64_t KT) {
   }
 }
 
-template <int MODE>
+template <int MODE, bool EMIT = false>
 __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap qmap,
                                                           const IndexParams p) {
@@ -140,14 +153,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 2 + 2 * kMaxAcc);
   float* w_all = reinterpret_cast<float*>(qfull + 4 + 2 * kMaxAcc);  // [8 epilogue warps][TQ][64]
   float* ks_all = w_all + kIdxEpiWarps * TQ * kIdxHeads;             // [kKsRing][epilogue threads] key-scale ring
-  // score histograms of the first two rows this CTA touches (when p.hist is set)
+  // score histograms of the first two rows this CTA touches (when p.hist is set); in the
+  // candidate mode the same place holds each epilogue warp's row thresholds and open
+  // 32-slot chunks: [warp][thr 4 | chunk base 4 | slots used 4]
   int* hist_s = reinterpret_cast<int*>(ks_all + kKsRing * 32 * kIdxEpiWarps);   // [2][kHistBinsIdx]
 
   const int QG = (p.T + TQ - 1) / TQ;
   const int64_t KT = (p.N + kIdxTileKeys - 1) / kIdxTileKeys;
   const int64_t items = (int64_t)p.B * QG * KT;
   const int64_t w0 = items * blockIdx.x / gridDim.x;
-  const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
+  int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
   // TMEM accumulators in flight (2 or 4); mxfp4 keeps 32 columns for the block scales
   const int acc_fit = (FP4 ? 480 : 512) / NQ;
   const int NACC = acc_fit >= kMaxAcc ? kMaxAcc : (acc_fit >= 2 ? 2 : 1);
@@ -186,6 +201,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   griddep_sync();
+  if (p.gate && __ldcg(p.gate) == 0) w1 = w0;       // gated off: every role walks no items
   const int hist_row0 = index_item(w0, QG, KT).b;   // T == 1 whenever p.hist is set: row = sequence
 
   if (warp == 0) {
@@ -330,6 +346,32 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       for (int j = 0; j < kKsAhead; ++j) ks_fetch();
     int ring_get = 0;
     int prev_b = -1, prev_qg = -1;
+    // candidate mode: the group's row thresholds and this warp's open 32-slot chunk per
+    // query (base -1: none) live in shared memory (registers are at the cap); every lane
+    // reads them, lane 0 writes them
+    int* emit_s = hist_s + e * 12;
+    int64_t row0 = 0;                               // b * T + qg * TQ of the current group
+    auto close_chunks = [&]() {                     // zero-fill the unused tails
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int base = emit_s[4 + q], used = emit_s[8 + q];
+        if (base >= 0 && (int)lane_id() >= used && base + 32 <= p.cand_cap)
+          p.cand[(row0 + q) * p.cand_cap + base + lane_id()] = 0ull;
+      }
+      __syncwarp();
+      if (lane_id() < 4) {
+        emit_s[4 + lane_id()] = -1;
+        emit_s[8 + lane_id()] = 0;
+      }
+      __syncwarp();
+    };
+    if constexpr (EMIT) {
+      if (lane_id() < 4) {
+        emit_s[4 + lane_id()] = -1;
+        emit_s[8 + lane_id()] = 0;
+      }
+      __syncwarp();
+    }
     IndexItem it = index_item(w0, QG, KT);
     int64_t w = w0;
     int cnt = 0;
@@ -338,6 +380,15 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       if (cnt >= nsets)
         for (int j = 0; j < nsets; ++j) index_next(it, QG, KT);
       if (it.b != prev_b || it.qg != prev_qg) {
+        if constexpr (EMIT) {
+          close_chunks();
+          const int tq = it.qg * TQ + (int)lane_id();
+          if (lane_id() < 4)
+            emit_s[lane_id()] = (int)(((int)lane_id() < TQ && tq < p.T) ? __ldg(p.thr + (int64_t)it.b * p.T + tq)
+                                                                        : 0xffffffffu);
+          __syncwarp();
+          row0 = (int64_t)it.b * p.T + (int64_t)it.qg * TQ;
+        }
         // each epilogue warp keeps a private copy of the group's head weights; the
         // weights, query scales and n_valid are all requested before any is used
         // (one memory round trip, overlapping the wait for the first accumulator)
@@ -407,7 +458,38 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
         }
         const float2 s01 = f32x2_unpack(a01), s23 = f32x2_unpack(a23);
         const float sc = (s01.x + s01.y) + (s23.x + s23.y);
-        if (i < p.N) {
+        if constexpr (EMIT) {
+          const uint32_t key = score_key(sc * ks);
+          const bool pass = i < p.N && i < nv_q[q] && key >= (uint32_t)emit_s[q];
+          const uint32_t m = __ballot_sync(0xffffffffu, pass);
+          if (m) {                                    // uniform over the warp
+            const int n = __popc(m);
+            const int rank = __popc(m & ((1u << lane_id()) - 1u));
+            const bool chunked = p.cand_chunk != 1;
+            const int base = chunked ? emit_s[4 + q] : -1, used = chunked ? emit_s[8 + q] : 0;
+            const int room = base < 0 ? 0 : 32 - used;
+            int nb = base;
+            if (n > room) {                             // a new chunk (or exactly n slots) for the rest
+              int g = 0;
+              if (lane_id() == 0) g = atomicAdd(&p.cand_cnt[row0 + q], chunked ? 32 : n);
+              nb = __shfl_sync(0xffffffffu, g, 0);
+            }
+            if (pass) {
+              const int slot = rank < room ? base + used + rank : nb + (rank - room);
+              if (slot < p.cand_cap)                    // (past it the row fails: never read)
+                p.cand[(row0 + q) * p.cand_cap + slot] =
+                    ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)i);
+            }
+            if (chunked) {
+              __syncwarp();
+              if (lane_id() == 0) {
+                emit_s[4 + q] = n > room ? nb : base;
+                emit_s[8 + q] = n > room ? n - room : used + n;
+              }
+              __syncwarp();
+            }
+          }
+        } else if (i < p.N) {
           const bool valid = i < nv_q[q];
           const float val = valid ? sc * ks : -INFINITY;
           p.scores[((int64_t)it.b * p.T + t) * p.N + i] = val;
@@ -423,6 +505,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&tempty[acc]);
     }
+    if constexpr (EMIT) close_chunks();
     if (FP8) cp_async_wait_group<0>();              // no copy may land after the CTA has left
   }
 

@@ -214,12 +214,15 @@ __global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, in
 // original indices of a rescored candidate list; map rows must be ascending so
 // that the output stays ascending).  cand_smem: the dynamic shared memory also holds
 // kRowCand candidate keys and indices after the row's keys (rows of kRowFastMin or more
-// then try the sampled threshold first).
+// then try the sampled threshold first).  gate: null, or a device int written by an
+// earlier launch; 0 -> the launch does nothing.
 __global__ void __launch_bounds__(1024) topk_row_kernel(const float* __restrict__ scores,
                                                         const int32_t* __restrict__ n_valid, int64_t N, int k,
                                                         int32_t* __restrict__ idx,
-                                                        const int32_t* __restrict__ map, int cand_smem) {
+                                                        const int32_t* __restrict__ map, int cand_smem,
+                                                        const int* __restrict__ gate) {
   griddep_sync();
+  if (gate && __ldcg(gate) == 0) return;
   extern __shared__ __align__(16) uint32_t keys[];  // [min(N, kRowSmemMax)], then (long rows) the candidates
   __shared__ __align__(16) int rhist[kHistBins + kHistBins / 32];   // skewed
   __shared__ int scratch[33];

@@ -114,6 +114,33 @@ def test_index_and_attention_reject_bad_arguments(lib):
     assert g(p, p, p, p, 128, p, p, p, -1, 0.1, 1, 1, 16, 128, 100, 1, p, None, 0, None) == 1
 
 
+def test_index_topk_host_checks(lib):
+    """csa_index_topk: unsupported dtypes, k and N past the fused path's limits, a missing or
+    short workspace, and the workspace size of the prefill shape (it holds the fallback's
+    score matrix besides the candidate lists)."""
+    sz = lib.csa_index_topk_workspace_size
+    sz.restype = ctypes.c_size_t
+    sz.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+    need = sz(1, 4096, 32768, 512, 1)
+    assert need >= 4096 * 32768 * 4 + 4096 * 8192 * 8
+    assert sz(0, 4, 100, 8, 1) == 0
+    f = lib.csa_index_topk
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    p, ws = 16, 256
+    assert f(p, None, p, p, None, 0, p, 1, 4, 1000, 64, p, None, ws, 1 << 30, None) == 2   # fp32
+    assert f(p, None, p, p, None, 4, p, 1, 4, 1000, 64, p, None, ws, 1 << 30, None) == 2   # mxfp4
+    assert f(p, None, p, p, None, 1, p, 1, 4, 1000, 2048, p, None, ws, 1 << 30, None) == 2  # k > 1024
+    assert f(p, None, p, p, None, 1, p, 1, 4, 40000, 64, p, None, ws, 1 << 30, None) == 2  # N > 32768
+    assert f(p, None, p, p, None, 2, p, 1, 4, 1000, 64, p, None, ws, 1 << 30, None) == 1   # e4m3, no scales
+    assert f(p, None, p, p, None, 1, p, 1, 4, 1000, 0, p, None, ws, 1 << 30, None) == 1    # k = 0
+    assert f(p, None, p, p, None, 1, p, 1, 4, 1000, 64, p, None, None, 0, None) == 1       # no workspace
+    assert f(p, None, p, p, None, 1, p, 1, 4, 1000, 64, p, None, ws, 64, None) == 1        # too small
+    assert f(p, None, p, p, None, 1, p, 1, 4, 1000, 64, p, None, 16, 1 << 30, None) == 1   # misaligned
+
+
 def test_kv8_storage_host_checks(lib):
     """Mixed-precision entries: 608 bytes at D = 512, nothing else; bad arguments rejected."""
     eb = lib.csa_kv8_entry_bytes
