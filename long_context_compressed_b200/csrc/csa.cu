@@ -1255,21 +1255,15 @@ unsigned long long csa_launch_count(void) { return g_launches.load(); }
 static __device__ __align__(256) uint8_t g_topk_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-// Device address of the scratch array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once per
-// device with that device current (cudaGetSymbolAddress) and cached.
+// Device address of the scratch array in the current device's context.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up with the
+// device current (cudaGetSymbolAddress).  It is looked up on every call, not cached: after
+// a cudaDeviceReset the module is loaded again into a new context and the array may
+// move.
 void* noalloc_scratch_ptr() {
-  static std::mutex mu;
-  static void* ptrs[kMaxDev] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_topk_noalloc_scratch) != cudaSuccess) return nullptr;
-    ptrs[dev] = p;
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_topk_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 }  // namespace
 

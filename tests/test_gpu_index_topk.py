@@ -40,10 +40,13 @@ def _run(csa, op, w, nv, k):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
-@pytest.mark.parametrize("T,N,k", [(37, 5000, 256), (5, 1000, 64), (8, 32768, 512), (3, 20000, 1024)])
+@pytest.mark.parametrize("T,N,k", [(37, 5000, 256), (5, 1000, 64), (8, 32768, 512), (3, 20000, 1024),
+                                   (1023, 2048, 64)])
 def test_index_topk_matches_unfused(csa, dtype, T, N, k):
     """Ragged query groups and key tiles; rows with n_valid = 0, k - 1, k, k + 1, a short row
-    (every key a candidate) and full rows."""
+    (every key a candidate) and full rows.  The first four shapes spread a row's key tiles
+    over many CTAs (one reservation per ballot); the last gives each CTA whole rows (32-slot
+    chunks per warp, with zero-filled tails)."""
     B = 2
     wl = synth.Workload("idx_topk", "bf16", B=B, ctx=4 * N, T=T, q_pos0=4 * N - T, ratio=4, N=N, H=16, D=128,
                         index_dtype="bf16")
@@ -65,14 +68,16 @@ def test_index_topk_matches_unfused(csa, dtype, T, N, k):
 
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
 @pytest.mark.parametrize("case", ["sampled_keys_boosted", "all_keys_equal"])
-def test_index_topk_fallback(csa, dtype, case):
+@pytest.mark.parametrize("T,N,k", [(12, 6000, 256), (1024, 2048, 64)])
+def test_index_topk_fallback(csa, dtype, case, T, N, k):
     """Rows the sample misleads.  sampled_keys_boosted: every 16th key (the sampled ones)
     scaled by 6, so for most rows the sampled threshold lies above all but about r = 4k/16
     keys and the candidate list is short (a row whose scores are mostly negative can still
     get enough).  all_keys_equal: every score of a row ties, so the list overflows.  The
     call counts those rows, takes its fallback and still returns the oracle's top-k (the
-    lower index wins every tie)."""
-    B, T, N, k = 1, 12, 6000, 256
+    lower index wins every tie).  Both reservation modes: one per ballot (12 queries) and
+    32-slot chunks (1,024 queries, each CTA walking whole rows)."""
+    B = 1
     wl = synth.Workload("idx_topk_fb", "bf16", B=B, ctx=4 * N, T=T, q_pos0=4 * N - T, ratio=4, N=N, H=16, D=128,
                         index_dtype="bf16")
     ix = synth.draw_indexer(wl, seed=99)
