@@ -211,12 +211,12 @@ int csa_index_scores(const void *qI, const float *q_scale, const float *w, const
  * csa_index_scores followed by csa_topk on the same arguments (the same kernel computes
  * every score, so the values are bit-identical).  Steps, in stream order:
  *   1. every 16th key of each sequence (and its scale) is gathered and scored;
- *   2. per row, the r-th largest sampled score (r = ceil(4k / 16)) is the row's
- *      threshold: about 4k keys are expected at or above it, and at least r are (a
- *      row with r samples or fewer takes every valid key);
+ *   2. per row, the r-th largest sampled score (r = max(48, ceil(4k / 16))) is the
+ *      row's threshold: about 16r keys are expected at or above it, and at least r are
+ *      (a row with r samples or fewer takes every valid key);
  *   3. the indexer scores every key; each valid score at or above its row's threshold
  *      goes into the row's candidate list (score key, index); nothing else is written;
- *   4. per row with at least k and at most cap = min(8192, max(2048, 16k)) candidates, the exact
+ *   4. per row with at least k and at most cap = min(8192, max(4096, 16k)) candidates, the exact
  *      top-k of the list (ties toward the lower index), ascending; other rows are
  *      counted as failed;
  *   5. a fallback, launched every time and doing nothing unless a row failed: the

@@ -798,8 +798,11 @@ static IndexTopkWs index_topk_layout(int B, int T, int64_t N, int k, int dtype) 
   IndexTopkWs L;
   const int64_t rows = (int64_t)B * T;
   L.Ns = (N + csa::kSampleStride - 1) / csa::kSampleStride;
-  L.r0 = (4 * k + csa::kSampleStride - 1) / csa::kSampleStride;
-  L.cap = std::min(csa::kCandCapMax, std::max(2048, 16 * k));
+  // the sampled rank: about 4k candidates expected, and never fewer than 48 samples above
+  // the threshold, so that a row comes up short (fewer than k) only some 6 standard
+  // deviations from the mean for keys in random order
+  L.r0 = std::max(48, (4 * k + csa::kSampleStride - 1) / csa::kSampleStride);
+  L.cap = std::min(csa::kCandCapMax, std::max(4096, 16 * k));
   const size_t row_bytes = dtype == CSA_BF16 ? 256 : 128;
   size_t off = 0;
   auto take = [&](size_t bytes) {

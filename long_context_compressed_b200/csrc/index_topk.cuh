@@ -22,11 +22,11 @@ namespace csa {
 
 constexpr int kSampleStride = 16;     // keys per sampled key
 constexpr int kCandCapMax = 8192;     // candidate slots per row (shared memory of the select)
-constexpr int kIndexTopkMaxK = 1024;  // sample threshold at rank 4k/16: ~4k candidates expected
-// Candidate slots per row: min(kCandCapMax, max(2048, 16k)).  Reserved slots = candidates,
+constexpr int kIndexTopkMaxK = 1024;  // sample threshold at rank max(48, 4k/16): ~4k candidates
+// Candidate slots per row: min(kCandCapMax, max(4096, 16k)).  Reserved slots = candidates,
 // plus (32-slot chunks, when a row spans at most two CTAs) at most 31 unused per
-// contributing epilogue warp: 4k + 992 for a short row (every key a candidate), about
-// 4k + 992 otherwise.
+// contributing epilogue warp: at most 16r + 992 for a short row (every key a candidate),
+// about 16r + 992 otherwise, r = max(48, 4k/16).
 
 __global__ void __launch_bounds__(256) sample_keys_kernel(const uint8_t* __restrict__ kI,
                                                           const float* __restrict__ ks, int B, int64_t N,

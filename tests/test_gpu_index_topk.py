@@ -68,7 +68,7 @@ def test_index_topk_matches_unfused(csa, dtype, T, N, k):
 
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
 @pytest.mark.parametrize("case", ["sampled_keys_boosted", "all_keys_equal"])
-@pytest.mark.parametrize("T,N,k", [(12, 6000, 256), (1024, 2048, 64)])
+@pytest.mark.parametrize("T,N,k", [(12, 6000, 256), (1024, 8192, 64)])
 def test_index_topk_fallback(csa, dtype, case, T, N, k):
     """Rows the sample misleads.  sampled_keys_boosted: every 16th key (the sampled ones)
     scaled by 6, so for most rows the sampled threshold lies above all but about r = 4k/16
