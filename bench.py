@@ -427,8 +427,9 @@ class DecodeSet:
         if self.index == "e4m3":
             csa.csa_quantize_e4m3(x["qI"], codes=self.q8, scale=self.qs, hadamard=INDEX_ROTATION)
             mark("quantize_q")
+            # the launch before it is the query quantiser, which does not write the keys
             csa.csa_index_scores(self.q8, x["w"], self.k8, self.n_valid, q_scale=self.qs, k_scale=self.ks,
-                                 scores=self.scores, select_ws=self.select_ws)
+                                 scores=self.scores, select_ws=self.select_ws, keys_ready=True)
             mark("index")
             if SCHEDULE in ("streams", "serial"):
                 side_branch()
@@ -440,7 +441,7 @@ class DecodeSet:
             csa.csa_quantize_mxfp4_sf128(x["qI"], wl.B, codes=self.q4, sf=self.qsf)
             mark("quantize_q")
             csa.csa_index_scores(self.q4, x["w"], self.k4, self.n_valid, q_scale=self.qsf, k_scale=self.ksf,
-                                 scores=self.scores, select_ws=self.select_ws, mxfp4=True)
+                                 scores=self.scores, select_ws=self.select_ws, mxfp4=True, keys_ready=True)
             mark("index")
             if SCHEDULE in ("streams", "serial"):
                 side_branch()

@@ -205,6 +205,23 @@ int csa_index_scores(const void *qI, const float *q_scale, const float *w, const
                      void *stream);
 
 /*
+ * csa_index_scores_ex -- csa_index_scores with flags (0: the same call).
+ *   CSA_INDEX_KEYS_READY: the caller states that kI and k_scale were not written by the
+ *     launch just before this call on `stream` (they were written earlier, or on another
+ *     stream whose work this stream already waited for).  The library's kernels start
+ *     their successor on the stream before they finish (programmatic dependent launch);
+ *     with this flag the indexer streams its first key tiles into shared memory while
+ *     its predecessor (say, the query quantiser) still runs, and waits for that launch only
+ *     before it reads the queries.  Without the flag nothing is read before the wait.
+ *     Giving the flag when the predecessor does write the keys is a race (stale keys).
+ *   Other bits: CSA_ERR_INVALID.  T = 1 decode launches (B x 1 queries) are the intended use.
+ */
+#define CSA_INDEX_KEYS_READY 1u
+int csa_index_scores_ex(const void *qI, const float *q_scale, const float *w, const void *kI, const float *k_scale,
+                        int dtype, const int32_t *n_valid, int B, int T, int64_t N, float *scores, void *select_ws,
+                        unsigned flags, void *stream);
+
+/*
  * csa_index_topk -- the indexer and the top-k in one call, without writing the score
  * matrix ([HA] §4.2: a cheap scan of every compressed key, the expensive work only for
  * the top-k; the chunked-prefill shapes).  The result equals, index for index,

@@ -23,6 +23,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 CSA_OK, CSA_ERR_INVALID, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA, CSA_ERR_TIMEOUT = range(5)
 CSA_F32, CSA_BF16, CSA_E4M3, CSA_BF16_KV8, CSA_MXFP4 = 0, 1, 2, 3, 4
+CSA_INDEX_KEYS_READY = 1
 KV8_DIMS, KV8_BYTES = 512, 608   # mixed-precision compressed entry: 448 e4m3 dims, 64 bf16 RoPE dims, 7 scales
 INDEX_HEADS, INDEX_DIM, SWA_WINDOW, MAX_TOPK = 64, 128, 128, 2048
 
@@ -43,6 +44,8 @@ _SIGS = {
     "csa_kv8_entry_bytes": ([_i32], ctypes.c_longlong),
     "csa_quantize_kv8": ([_vp, _i64, _i32, _vp, _vp], _i32),
     "csa_index_scores": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, _vp], _i32),
+    "csa_index_scores_ex": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _vp, _vp, ctypes.c_uint, _vp],
+                            _i32),
     "csa_index_topk_workspace_size": ([_i32, _i32, _i64, _i32, _i32], _sz),
     "csa_index_topk": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "csa_select_workspace_size": ([_i32, _i64], _sz),
@@ -188,19 +191,22 @@ def csa_quantize_e4m3(x, codes=None, scale=None, stream=None, hadamard=False):
 
 
 def csa_index_scores(qI, w, kI, n_valid, *, q_scale=None, k_scale=None, scores=None, select_ws=None,
-                     mxfp4: bool = False, stream=None):
+                     mxfp4: bool = False, keys_ready: bool = False, stream=None):
     """Indexer scores.  qI [B, T, 64, 128] (fp32 | bf16 | uint8 e4m3 codes), w [B, T, 64] fp32,
     kI [B, N, 128] same dtype, n_valid [B, T] int32 -> scores [B, T, N] fp32.  With select_ws
     (T == 1) the per-row score histogram for csa_topk_select is accumulated there.
     mxfp4=True: qI [B, T, 64, 64] / kI [B, N, 64] packed E2M1 codes and q_scale / k_scale their
-    tensor-core-layout scales (csa_quantize_mxfp4_sf128)."""
+    tensor-core-layout scales (csa_quantize_mxfp4_sf128).  keys_ready=True: the caller states the
+    launch just before this call on the stream does not write kI / k_scale
+    (CSA_INDEX_KEYS_READY): the first key tiles then load while that launch finishes."""
     B, T = qI.shape[0], qI.shape[1]
     N = kI.shape[1]
     if scores is None:
         scores = torch.empty((B, T, N), dtype=torch.float32, device=qI.device)
     dt = CSA_MXFP4 if mxfp4 else _dtype_code(qI)
-    _check(_lib.csa_index_scores(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), dt,
-                                 _ptr(n_valid), B, T, N, _ptr(scores), _ptr(select_ws), _stream(stream)),
+    _check(_lib.csa_index_scores_ex(_ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI), _ptr(k_scale), dt,
+                                    _ptr(n_valid), B, T, N, _ptr(scores), _ptr(select_ws),
+                                    CSA_INDEX_KEYS_READY if keys_ready else 0, _stream(stream)),
            "csa_index_scores")
     return scores
 

@@ -754,6 +754,13 @@ static int launch_index_tc(const void* qI, const void* kI, int mode, IndexParams
 int csa_index_scores(const void* qI, const float* q_scale, const float* w, const void* kI, const float* k_scale,
                      int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* select_ws,
                      void* stream) {
+  return csa_index_scores_ex(qI, q_scale, w, kI, k_scale, dtype, n_valid, B, T, N, scores, select_ws, 0u, stream);
+}
+
+int csa_index_scores_ex(const void* qI, const float* q_scale, const float* w, const void* kI, const float* k_scale,
+                        int dtype, const int32_t* n_valid, int B, int T, int64_t N, float* scores, void* select_ws,
+                        unsigned flags, void* stream) {
+  if (flags & ~(unsigned)CSA_INDEX_KEYS_READY) return CSA_ERR_INVALID;
   if (B < 0 || T < 0 || N < 0) return CSA_ERR_INVALID;
   if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3 && dtype != CSA_MXFP4) return CSA_ERR_INVALID;
   if (B == 0 || T == 0 || N == 0) return CSA_OK;
@@ -779,6 +786,7 @@ int csa_index_scores(const void* qI, const float* q_scale, const float* w, const
     p.hist = reinterpret_cast<int*>(select_ws);
     p.hist_stride = csa::SelectWs::row_bytes(N) / 4;
   }
+  p.keys_ready = (flags & CSA_INDEX_KEYS_READY) ? 1 : 0;
   return launch_index_tc(qI, kI, mode, p, false, st);
 }
 

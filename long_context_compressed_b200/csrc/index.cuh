@@ -81,6 +81,10 @@ struct IndexParams {
   int cand_cap;
   int cand_chunk;               // 32 or 1
   const int* gate;              // null, or a device int written by an earlier launch: 0 -> no work
+  // keys_ready: the key operands (codes, scales) are not written by the launch before this
+  // one on the stream, so the producer issues the first `stages` key tiles before it waits
+  // for that launch (programmatic dependent launch); never together with gate
+  int keys_ready;
 };
 
 // Operand modes of index_tc_kernel.
@@ -200,6 +204,19 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // key tiles that do not depend on the previous launch stream in while it finishes
+  const int npre = p.keys_ready ? (int)(w1 - w0 < p.stages ? w1 - w0 : p.stages) : 0;
+  if (npre > 0 && warp == 0 && elect_one()) {
+    IndexItem it = index_item(w0, QG, KT);
+    for (int j = 0; j < npre; ++j, index_next(it, QG, KT)) {
+      mbar_arrive_expect_tx(&full[j], (uint32_t)(Cfg::kCodeBytes + Cfg::kSfBytes));
+      uint8_t* dst = k_smem + (size_t)j * Cfg::kKeyBytes;
+      for (int a = 0; a < Cfg::kAtoms; ++a)
+        tma_load_3d(dst + (size_t)a * kIdxTileKeys * 128, &kmap, &full[j], a * 64, (int)(it.kt * kIdxTileKeys),
+                    it.b);
+      if (FP4) bulk_load(dst + Cfg::kCodeBytes, p.k_sf + ((int64_t)it.b * KT + it.kt) * 512, 512, &full[j]);
+    }
+  }
   griddep_sync();
   if (p.gate && __ldcg(p.gate) == 0) w1 = w0;       // gated off: every role walks no items
   const int hist_row0 = index_item(w0, QG, KT).b;   // T == 1 whenever p.hist is set: row = sequence
@@ -232,6 +249,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_tc_kernel(const __grid_c
         const int s = st_i;
         const uint32_t ph = st_ph;
         if (++st_i == p.stages) { st_i = 0; st_ph ^= 1; }
+        if (cnt < npre) continue;                   // issued before the grid dependency wait
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(Cfg::kCodeBytes + Cfg::kSfBytes));
         uint8_t* dst = k_smem + (size_t)s * Cfg::kKeyBytes;

@@ -12,9 +12,10 @@ def test_traffic_records_follow_the_source_hash():
     """The committed summaries carry the hash of the source they were captured on: while it
     matches, every recorded workload is returned; once it differs, none is."""
     import re
-    for profile, source, names in (("attn_tc_kernel_decode_prefill_hca.md", "attn.cuh",
-                                    ("flash64k", "pro1m", "flash64k_kv8", "pro1m_kv8")),
-                                   ("index_tc_kernel_e4m3_decode.md", "index.cuh", ("flash64k", "pro1m"))):
+    for profile, source, names in (("attn_tc_kernel_decode_prefill_hca.md", "attn.cuh", ("flash64k_kv8", "pro1m_kv8")),
+                                   ("attn_t_kernel_decode.md", "attn_t.cuh", ("flash64k", "pro1m")),
+                                   ("index_tc_kernel_e4m3_decode.md", "index.cuh", ("flash64k", "pro1m")),
+                                   ("index_tc_kernel_mxfp4_decode.md", "index.cuh", ("flash64k", "pro1m"))):
         text = open(os.path.join(ROOT, "profiles", profile)).read()
         rec = re.search(r"source_sha256_prefix=([0-9a-f]+)", text).group(1)
         src = open(os.path.join(ROOT, "long_context_compressed_b200", "csrc", source), "rb").read()

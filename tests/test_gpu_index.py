@@ -179,3 +179,39 @@ def test_rerank_short_rows(csa):
                                k).cpu().numpy()
     assert got[0, 0].tolist() == list(range(0, 50, 2)) + [-1] * 15
     assert np.all(np.diff(got[0, 1]) > 0) and got[0, 1].min() >= 0
+
+
+@pytest.mark.parametrize("mode", ["e4m3", "mxfp4", "bf16"])
+@pytest.mark.parametrize("name", ["flash64k", "pro1m"])
+def test_keys_ready_prefetch(csa, mode, name):
+    """CSA_INDEX_KEYS_READY (first key tiles loaded before the wait for the previous launch)
+    gives the same scores and the same select histogram, bit for bit, as the plain call, with
+    the query quantiser as the launch just before the indexer (the decode step's order)."""
+    wl = synth.WORKLOADS[name]
+    ix, _, nv = _inputs(wl)
+    g_nv = torch.from_numpy(nv).cuda()
+    qI, kI, w = ix["qI"].cuda(), ix["kI"].cuda(), ix["w"].cuda()
+    if mode == "e4m3":
+        k, ks = csa.csa_quantize_e4m3(kI)
+        q, qs = csa.csa_quantize_e4m3(qI)
+        quant = lambda: csa.csa_quantize_e4m3(qI, codes=q, scale=qs)
+    elif mode == "mxfp4":
+        k, ks = csa.csa_quantize_mxfp4_sf128(kI, wl.B)
+        q, qs = csa.csa_quantize_mxfp4_sf128(qI, wl.B)
+        quant = lambda: csa.csa_quantize_mxfp4_sf128(qI, wl.B, codes=q, sf=qs)
+    else:
+        k, ks, q, qs = kI, None, qI, None
+        quant = lambda: csa.csa_n_valid(torch.zeros_like(g_nv, dtype=torch.int64), 4, 0, 1)
+    torch.cuda.synchronize()
+    out = {}
+    for ready in (False, True, True):
+        ws = csa.select_workspace(wl.B, wl.N)
+        quant()
+        s = csa.csa_index_scores(q, w, k, g_nv, q_scale=qs, k_scale=ks, select_ws=ws, mxfp4=mode == "mxfp4",
+                                 keys_ready=ready)
+        torch.cuda.synchronize()
+        out.setdefault(ready, []).append((s.clone(), ws.clone()))
+    base_s, base_ws = out[False][0]
+    for s, ws in out[True]:
+        assert torch.equal(s, base_s), f"{name} {mode}: scores differ with the key prefetch"
+        assert torch.equal(ws, base_ws), f"{name} {mode}: select histogram differs with the key prefetch"
