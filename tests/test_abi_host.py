@@ -100,6 +100,13 @@ def test_index_and_attention_reject_bad_arguments(lib):
     assert f(p, None, p, p, None, 2, p, 1, 1, 100, p, None) == 1   # e4m3 without scales
     assert f(p, None, p, p, None, 9, p, 1, 1, 100, p, None) == 1   # bad dtype
     assert f(p, None, None, p, None, 1, p, 1, 1, 100, p, None) == 1  # no head weights
+    fx = lib.csa_index_scores_ex
+    fx.restype = ctypes.c_int
+    fx.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint,
+                                           ctypes.c_void_p]
+    assert fx(p, None, p, p, None, 1, p, 1, 1, 100, p, None, 2, None) == 1   # unknown flag bit
+    assert fx(p, None, p, p, None, 2, p, 1, 1, 100, p, None, 1, None) == 1   # keys ready, e4m3 without scales
     g = lib.sparse_attn
     g.restype = ctypes.c_int
     g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
