@@ -843,19 +843,21 @@ int csa_index_topk(const void* qI, const float* q_scale, const float* w, const v
   if (dtype != CSA_F32 && dtype != CSA_BF16 && dtype != CSA_E4M3 && dtype != CSA_MXFP4) return CSA_ERR_INVALID;
   if (dtype != CSA_BF16 && dtype != CSA_E4M3) return CSA_ERR_UNSUPPORTED;
   if (k > csa::kIndexTopkMaxK || N > csa::kRowSmemMax || B > 65535 ||
-      (int64_t)T * csa::kIdxHeads >= (int64_t(1) << 31))
+      (int64_t)T * csa::kIdxHeads >= (int64_t(1) << 31) || (int64_t)B * T > INT32_MAX)
     return CSA_ERR_UNSUPPORTED;
   if (B == 0 || T == 0) return CSA_OK;
-  if (!qI || !w || !kI || !n_valid || !idx) return CSA_ERR_INVALID;
-  if (dtype == CSA_E4M3 && (!q_scale || !k_scale)) return CSA_ERR_INVALID;
-  if (!aligned16(qI) || !aligned16(kI)) return CSA_ERR_INVALID;
   cudaStream_t st = as_stream(stream);
   const int64_t rows = (int64_t)B * T;
   if (N == 0) {                                      // no keys: every row is -1
+    if (!n_valid || !idx) return CSA_ERR_INVALID;
+    if (failed_rows && cudaMemsetAsync(failed_rows, 0, sizeof(int32_t), st) != cudaSuccess) return CSA_ERR_CUDA;
     launch_k(csa::topk_row_kernel, (unsigned)rows, 1024, 4, st, (const float*)nullptr, n_valid, N, k, idx,
              (const int32_t*)nullptr, 0, (const int*)nullptr);
     return launch_status();
   }
+  if (!qI || !w || !kI || !n_valid || !idx) return CSA_ERR_INVALID;
+  if (dtype == CSA_E4M3 && (!q_scale || !k_scale)) return CSA_ERR_INVALID;
+  if (!aligned16(qI) || !aligned16(kI)) return CSA_ERR_INVALID;
   const IndexTopkWs L = index_topk_layout(B, T, N, k, dtype);
   if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return CSA_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

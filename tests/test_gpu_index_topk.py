@@ -116,3 +116,15 @@ def test_index_topk_prefill_shape(csa, dtype):
     ref = oracle.topk(s[:, rows].cpu().numpy(), nv[:, rows], wl.topk)
     assert np.array_equal(idx[:, rows].cpu().numpy(), ref)
     assert failed == 0, f"{failed} rows took the fallback"
+
+
+def test_index_topk_no_keys(csa):
+    """N = 0: every row is -1 and failed_rows is set to 0."""
+    B, T, k = 2, 5, 16
+    qI = torch.zeros((B, T, 64, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((B, T, 64), dtype=torch.float32, device="cuda")
+    kI = torch.zeros((B, 0, 128), dtype=torch.bfloat16, device="cuda")
+    nv = torch.zeros((B, T), dtype=torch.int32, device="cuda")
+    failed = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    idx = csa.csa_index_topk(qI, w, kI, nv, k, failed_rows=failed)
+    assert (idx.cpu() == -1).all() and int(failed.item()) == 0
