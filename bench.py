@@ -1242,8 +1242,8 @@ def main():
         extra = bench_workload("pro1m", args.index, False, args.steps, args.warmup, world, device)
     variants = {}
     if not args.no_extra and args.workload == "flash64k":
-        # the same configuration with the bf16 indexer (BASELINE's FP8 and BF16 variants),
-        # and the plain CSA layer without the HCA layer beside it
+        # the same configuration with the other index precision (the 64K decode is quoted with
+        # an FP8 and with a BF16 indexer), and the plain CSA layer without the HCA layer beside it
         other = "bf16" if args.index == "e4m3" else "e4m3"
         variants[f"flash64k_{other}_index"] = bench_workload("flash64k", other, True, args.steps, args.warmup, world,
                                                              device)
