@@ -286,12 +286,12 @@ int csa_topk(const float *scores, const int32_t *n_valid, int B, int T, int64_t 
  *   it returns CSA_ERR_UNSUPPORTED.  Every argument is checked before the array is
  *   touched: a rejected call enqueues nothing.  No cudaMalloc / cudaFree (or any
  *   allocating routine) is ever made; each call clears the part of the array it
- *   uses with cudaMemsetAsync on `stream`, since the array keeps whatever the
- *   previous call left in it.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current and keeps it for later calls;
- *   do not use this entry point after cudaDeviceReset (the kept address would be
- *   stale).  All calls share
+ *   uses with cudaMemsetAsync on `stream`: a completed call leaves that part zeroed,
+ *   but one cut short (an error) or one that overlapped another would not, and the
+ *   clear makes every call independent of the previous one.
+ *   Each call looks up the array's device address (cudaGetSymbolAddress) with the
+ *   call's device current, so the entry point stays valid after a cudaDeviceReset
+ *   (the array may then sit at another address).  All calls share
  *   the one array: calls that may overlap on the GPU (different streams, or work
  *   replayed concurrently) race on it and give wrong results -- order them on one
  *   stream.
