@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX helpers for sm_100a: mbarriers with bounded waits,
-// TMA tile loads (no multicast), cp.async, tcgen05 (TMEM alloc, MMA, commit,
+// TMA tile loads (each into the issuing CTA only), cp.async, tcgen05 (TMEM alloc, MMA, commit,
 // loads) and the shared-memory / instruction descriptors the MMA consumes.
 #pragma once
 #include <cstdint>
@@ -92,7 +92,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // 2-D / 3-D TMA tile load into this CTA's shared memory, completion counted on
-// the mbarrier in bytes.  Plain loads only: no cluster multicast anywhere.
+// the mbarrier in bytes.  Each load fills the issuing CTA's shared memory only.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z) {
   asm volatile(
@@ -114,7 +114,7 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
 
 // Bulk copy of `bytes` contiguous bytes from global memory into this CTA's shared
 // memory, completion counted on the mbarrier in bytes (addresses 16-byte aligned,
-// bytes a multiple of 16).  No multicast.
+// bytes a multiple of 16).  The issuing CTA's shared memory only.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
